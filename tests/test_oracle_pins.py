@@ -1,0 +1,389 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: numbers the
+pages print (tests/golden), closed forms, brute force on tiny inputs, an
+independent algorithm (Babai nearest plane, literal OBS re-inversion), or an
+invariant.  A plausible slip in the oracle (dropped compensation term, wrong
+sign, transposed factor, wrong group boundary, wrong rounding) fails at least
+one of them.
+"""
+
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import gptq_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def round_half_up(x, nd):
+    """Decimal rounding as printed on the pages (0.3125 -> 0.313)."""
+    f = 10 ** nd
+    return np.floor(x * f + 0.5) / f
+
+
+def _rand_problem(seed, d_out, d_in, n, hot=2):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((n, d_in))
+    if hot:
+        X[:, rng.choice(d_in, hot, replace=False)] *= 8.0
+    W = rng.standard_normal((d_out, d_in)) * 0.02
+    H = O.hessian(X)
+    Hd, lam = O.damp(H, 0.01)
+    U = O.hinv_upper_cholesky(Hd)
+    return X, W, H, Hd, U
+
+
+# ---------------------------------------------------------------- stage 1
+
+def test_hessian_is_sum_of_token_outer_products():
+    rng = np.random.default_rng(1)
+    X = rng.standard_normal((7, 5))
+    brute = np.zeros((5, 5))
+    for t in range(7):
+        for i in range(5):
+            for j in range(5):
+                brute[i, j] += 2.0 * X[t, i] * X[t, j]
+    np.testing.assert_allclose(O.hessian(X), brute, rtol=1e-13, atol=1e-13)
+
+
+def test_damping_closed_form():
+    H = np.diag([1.0, 2.0, 3.0, 4.0])
+    Hd, lam = O.damp(H, 0.01)
+    assert lam == pytest.approx(0.025, rel=1e-15)
+    np.testing.assert_allclose(np.diag(Hd), [1.025, 2.025, 3.025, 4.025], rtol=1e-15)
+    assert Hd[0, 1] == 0.0
+
+
+def test_U_is_the_upper_cholesky_factor_of_the_inverse():
+    _, _, _, Hd, U = _rand_problem(2, 3, 24, 40)
+    assert np.all(np.tril(U, -1) == 0.0)
+    assert np.all(np.diag(U) > 0)
+    np.testing.assert_allclose(U.T @ U @ Hd, np.eye(24), atol=1e-10)
+
+
+def test_U_rows_are_normalised_rows_of_trailing_inverses():
+    # OBS downdate form: row c of U is row 0 of inv(Hd[c:, c:]) / sqrt of its (0,0) entry
+    _, _, _, Hd, U = _rand_problem(3, 3, 12, 30)
+    for c in range(12):
+        Ri = np.linalg.inv(Hd[c:, c:])
+        np.testing.assert_allclose(U[c, c:], Ri[0, :] / np.sqrt(Ri[0, 0]), rtol=1e-9, atol=1e-12)
+
+
+def test_U_of_reversed_cholesky_route_agrees():
+    # Hd = R R^T with R upper (Cholesky of the index-reversed matrix) gives U = R^-1.
+    _, _, _, Hd, U = _rand_problem(4, 3, 16, 40)
+    J = np.arange(16)[::-1]
+    L = np.linalg.cholesky(Hd[np.ix_(J, J)])
+    R = L[np.ix_(J, J)]
+    assert np.allclose(np.tril(R, -1), 0.0)
+    np.testing.assert_allclose(np.linalg.inv(R), U, rtol=1e-8, atol=1e-12)
+
+
+# ---------------------------------------------------------------- quantizer
+
+def test_group_params_hand_values_asym():
+    v = np.array([[-0.02, 0.0, 0.01, 0.02]])
+    s, z, raw, lo, hi = O.group_params(v, 4, sym=False)
+    assert raw[0] == pytest.approx(0.04 / 15, rel=1e-15)
+    assert s[0] == float(np.float16(0.04 / 15))
+    # zero = rint(0.02 / s) with s slightly below 0.0026667 -> 7.5002 -> 8
+    assert z[0] == 8.0
+    q = O.quantize(v, s[:, None], z[:, None], 15)
+    assert list(q[0]) == [0.0, 8.0, 12.0, 15.0]
+
+
+def test_group_params_range_contains_zero():
+    v = np.array([[0.1, 0.2, 0.3]])
+    s, z, _, lo, hi = O.group_params(v, 4, sym=False)
+    assert lo[0] == 0.0 and z[0] == 0.0
+    assert s[0] == float(np.float16(0.3 / 15))
+
+
+def test_group_params_sym_and_degenerate():
+    v = np.array([[-0.5, 0.1, 0.25], [0.0, 0.0, 0.0]])
+    s, z, _, _, _ = O.group_params(v, 3, sym=True)
+    assert s[0] == float(np.float16(1.0 / 7)) and z[0] == 4.0
+    assert s[1] == 1.0 and z[1] == 4.0
+    q = O.quantize(np.zeros(3), 1.0, 4.0, 7)
+    assert np.all(O.dequantize(q, 1.0, 4.0) == 0.0)
+
+
+def test_tiny_range_scale_clamped_to_smallest_fp16():
+    v = np.array([[1e-12, -1e-12]])
+    s, z, _, _, _ = O.group_params(v, 4, sym=False)
+    assert s[0] == 2.0 ** -24
+
+
+def test_round_half_to_even_and_clamp():
+    s, z = 1.0, 0.0
+    assert list(O.quantize(np.array([0.5, 1.5, 2.5, -3.0, 99.0]), s, z, 15)) == [0.0, 2.0, 2.0, 0.0, 15.0]
+
+
+def test_grid_step_example_from_group_size_page():
+    g = json.load(open(os.path.join(GOLDEN, "grid_step_example.json")))
+    bits = g["bits"]
+    lo, hi = g["tight_group_range"]
+    tight = np.array([[lo, hi, 0.001]])
+    s1, _, raw1, _, _ = O.group_params(tight, bits, sym=True)
+    outl = np.array([[lo, hi, g["outlier_magnitude"]]])
+    s2, _, raw2, _, _ = O.group_params(outl, bits, sym=True)
+    assert raw1[0] == pytest.approx(g["tight_step_printed"], abs=0.5e-4)
+    assert raw2[0] == pytest.approx(g["outlier_step_printed"], abs=0.5e-3)
+    assert raw2[0] / raw1[0] == pytest.approx(g["coarser_factor_printed"], rel=1e-12)
+    assert (1 << bits) - 1 == g["levels_divisor"]
+    # the asymmetric grid on the tight range gives the same step
+    sa, _, rawa, _, _ = O.group_params(tight, bits, sym=False)
+    assert rawa[0] == pytest.approx(g["tight_step_printed"], abs=0.5e-4)
+
+
+# ---------------------------------------------------------------- metadata size
+
+def test_metadata_overhead_matches_group_size_page():
+    gd = json.load(open(os.path.join(GOLDEN, "group_size_overhead.json")))
+    d_out, d_in = 64, 1024
+    rng = np.random.default_rng(5)
+    for row in gd["overhead_bits_per_weight"]:
+        g = row["group_size"]
+        # measure from the arrays the packer actually writes
+        ng = O.n_groups(d_in, g)
+        zeros = rng.integers(0, 16, size=(ng, d_out))
+        scales = np.zeros((ng, d_out), dtype=np.float16)
+        qz = O.pack_qzeros(zeros, 4)
+        measured = (scales.nbytes + qz.nbytes) * 8 / (d_out * d_in)
+        assert measured == pytest.approx(O.metadata_bits_per_weight(d_out, d_in, 4, g, False), rel=1e-15)
+        if g == -1:
+            assert measured == pytest.approx(20.0 / d_in, rel=1e-15)
+            # "~0": one scale+zero per row of a real layer (d_in = 4096..11008) rounds to 0.00
+            for d_row in (4096, 11008):
+                big = O.metadata_bits_per_weight(8, d_row, 4, -1, False)
+                assert round_half_up(big, 2) == row["overhead"]
+                assert round_half_up(4 + big, 2) == row["total"]
+        else:
+            assert measured == 20.0 / g
+            assert round_half_up(measured, gd["printed_decimals"]) == pytest.approx(row["overhead"], abs=1e-12)
+            assert round_half_up(4 + measured, gd["printed_decimals"]) == pytest.approx(row["total"], abs=1e-12)
+    # symmetric drops the zero: numerator 16
+    assert O.metadata_bits_per_weight(d_out, d_in, 4, 128, True) * 128 == gd["symmetric_numerator_bits"]
+
+
+def test_model_size_lines_of_group_size_page():
+    gd = json.load(open(os.path.join(GOLDEN, "group_size_overhead.json")))
+    sizes = {}
+    for row in gd["model_7b_gb"]:
+        g = row["group_size"]
+        bpw = 4 + round_half_up(20.0 / g, 3)     # the page rounds the overhead before multiplying
+        gb = 7.0e9 * bpw / 8 / 1e9
+        sizes[g] = gb
+        assert round_half_up(gb, gd["gb_decimals"]) == pytest.approx(row["gb"], abs=1e-9)
+    span = sizes[32] - sizes[128]
+    assert round(span, 2) == pytest.approx(gd["span_128_to_32_gb"], abs=1e-9)
+    assert round(span / sizes[128], 2) == pytest.approx(gd["span_fraction_approx"], abs=1e-9)
+    extra = 20.0 / 32 - 20.0 / 128
+    assert round(extra, 3) == pytest.approx(gd["model_70b_extra_bits"], abs=1e-9)
+    assert round(70e9 * extra / 8 / 1e9, 1) == pytest.approx(gd["model_70b_extra_gb"], abs=1e-9)
+
+
+# ---------------------------------------------------------------- packing
+
+def test_pack_hand_example_4bit():
+    codes = np.array([[1, 2, 3, 4, 5, 6, 7, 8, 15, 0, 0, 0, 0, 0, 0, 9]])
+    w = O.pack_bitstream(codes, 4)
+    assert w.shape == (1, 2)
+    assert int(w[0, 0]) == 0x87654321
+    assert int(w[0, 1]) == 0x9000000F
+
+
+def test_pack_hand_example_3bit_straddle():
+    # 11 values of 3 bits: value 10 occupies bits 30..32, straddling words 0 and 1
+    codes = np.zeros((1, 11), dtype=np.int64)
+    codes[0, 0] = 5          # bits 0..2  -> 0b101
+    codes[0, 10] = 7         # bits 30..32 -> word0 bits 30,31 and word1 bit 0
+    w = O.pack_bitstream(codes, 3)
+    assert w.shape == (1, 2)
+    assert int(w[0, 0]) == (5 | (3 << 30))
+    assert int(w[0, 1]) == 1
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_pack_roundtrip(bits):
+    rng = np.random.default_rng(bits)
+    codes = rng.integers(0, 1 << bits, size=(5, 77))
+    w = O.pack_bitstream(codes, bits)
+    assert w.shape[1] == (77 * bits + 31) // 32
+    np.testing.assert_array_equal(O.unpack_bitstream(w, bits, 77), codes)
+
+
+def test_qweight_layout_and_dequant_hand_example():
+    # 2 output rows, 8 input columns, one group: W_hat = s * (q - z)
+    codes = np.array([[0, 1, 2, 3, 4, 5, 6, 7], [15, 14, 13, 12, 11, 10, 9, 8]])
+    qw = O.pack_qweight(codes, 4)
+    assert qw.shape == (1, 2)
+    assert int(qw.view(np.uint32)[0, 0]) == 0x76543210
+    assert int(qw.view(np.uint32)[0, 1]) == 0x89ABCDEF
+    scales = np.array([[0.5, 0.25]], dtype=np.float16)
+    qz = O.pack_qzeros(np.array([[3, 8]]), 4)
+    assert int(qz.view(np.uint32)[0, 0]) == 0x83
+    What = O.dequant_packed(qw, scales, qz, 2, 8, 4, -1, False)
+    np.testing.assert_array_equal(What[0], 0.5 * (np.arange(8) - 3))
+    np.testing.assert_array_equal(What[1], 0.25 * (np.arange(15, 7, -1) - 8))
+
+
+# ---------------------------------------------------------------- column loop
+
+@pytest.mark.parametrize("bits,g,sym", [(4, 128, False), (3, 64, True), (2, 32, False), (4, -1, False)])
+def test_identity_hessian_reduces_to_rtn(bits, g, sym):
+    rng = np.random.default_rng(7)
+    W = rng.standard_normal((9, 256)) * 0.02
+    U = O.hinv_upper_cholesky(np.eye(256))
+    r = O.gptq(W, U, bits, g, sym, block_size=128)
+    ref = O.rtn(W, bits, g, sym)
+    np.testing.assert_array_equal(r.codes, ref.codes)
+    np.testing.assert_array_equal(r.scales, ref.scales)
+    np.testing.assert_array_equal(r.zeros, ref.zeros)
+
+
+def test_diagonal_hessian_reduces_to_rtn():
+    rng = np.random.default_rng(8)
+    W = rng.standard_normal((6, 128)) * 0.02
+    Hd = np.diag(rng.uniform(0.5, 5.0, 128))
+    r = O.gptq(W, O.hinv_upper_cholesky(Hd), 4, 32, False, block_size=0)
+    np.testing.assert_array_equal(r.codes, O.rtn(W, 4, 32, False).codes)
+
+
+@pytest.mark.parametrize("bits,g,sym", [(4, 128, False), (3, 64, True), (2, 32, False), (4, -1, False), (8, 16, False)])
+def test_lazy_blocks_equal_eager(bits, g, sym):
+    _, W, _, _, U = _rand_problem(9, 17, 384, 300)
+    eager = O.gptq(W, U, bits, g, sym, block_size=0)
+    lazy = O.gptq(W, U, bits, g, sym, block_size=128)
+    np.testing.assert_array_equal(eager.codes, lazy.codes)
+    np.testing.assert_array_equal(eager.scales, lazy.scales)
+    np.testing.assert_allclose(eager.err, lazy.err, rtol=1e-9, atol=1e-12)
+
+
+def test_lazy_blocks_equal_eager_ragged():
+    _, W, _, _, U = _rand_problem(10, 5, 200, 150)
+    eager = O.gptq(W, U, 4, 32, False, block_size=0)
+    lazy = O.gptq(W, U, 4, 32, False, block_size=128)
+    np.testing.assert_array_equal(eager.codes, lazy.codes)
+    assert eager.scales.shape == (7, 5)      # 6 full groups + one of 8 columns
+
+
+@pytest.mark.parametrize("seed", [11, 12, 13])
+def test_U_form_equals_literal_obs_reinversion(seed):
+    _, W, _, Hd, U = _rand_problem(seed, 6, 8, 20, hot=1)
+    a = O.gptq(W, U, 3, 4, False, block_size=0)
+    b = O.gptq_naive_obs(W, Hd, 3, 4, False)
+    np.testing.assert_array_equal(a.codes, b.codes)
+    np.testing.assert_allclose(a.what, b.what, rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("seed", range(20, 30))
+def test_gptq_equals_babai_nearest_plane(seed):
+    X, W, H, Hd, U = _rand_problem(seed, 4, 7, 12, hot=1)
+    rng = np.random.default_rng(seed + 100)
+    s = np.full(4, 0.004)
+    z = rng.integers(0, 8, 4).astype(np.float64)
+    r = O.gptq(W, U, 4, -1, False, block_size=0, fixed_grid=(s, z))
+    # an independent basis with B^T B = Hd: symmetric square root
+    ev, V = np.linalg.eigh(Hd)
+    Bm = V @ np.diag(np.sqrt(ev)) @ V.T
+    for o in range(4):
+        c = O.babai_nearest_plane(W[o] / s[o] + z[o], Bm)
+        np.testing.assert_array_equal(r.codes[o], c.astype(np.int64))
+
+
+@pytest.mark.parametrize("seed", range(40, 46))
+def test_bruteforce_bracket_and_babai_bound(seed):
+    X, W, H, Hd, U = _rand_problem(seed, 1, 5, 9, hot=1)
+    s, z = np.array([0.01]), np.array([0.0])
+    r = O.gptq(W, U, 4, -1, False, block_size=0, fixed_grid=(s, z))
+    x = W[0] / s[0]
+    def loss(q):
+        d = s[0] * (x - q)
+        return d @ Hd @ d
+    l_gptq = loss(r.codes[0].astype(np.float64))
+    base = np.floor(x)
+    rad = int(np.max(np.abs(r.codes[0] - base))) + 2
+    offs = np.array(list(itertools.product(range(-rad, rad + 2), repeat=5)), dtype=np.float64)
+    D = s[0] * (x[None, :] - (base[None, :] + offs))
+    all_losses = np.einsum("ij,jk,ik->i", D, Hd, D)
+    best = all_losses.min()
+    assert best <= l_gptq * (1 + 1e-12)
+    assert l_gptq <= O.babai_bound(U, s[0]) * (1 + 1e-12)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_loss_identity_sum_of_squared_errors(bits):
+    # per row: (W0 - W_hat) Hd (W0 - W_hat)^T == sum_c e_c^2, for any codes (clamped ones too)
+    _, W, _, Hd, U = _rand_problem(50, 8, 96, 120)
+    r = O.gptq(W * 3.0, U, bits, 32, False, block_size=64)
+    D = W * 3.0 - r.what
+    lhs = np.einsum("ij,jk,ik->i", D, Hd, D)
+    np.testing.assert_allclose(lhs, np.sum(r.err ** 2, axis=1), rtol=1e-9)
+
+
+def test_layer_loss_is_half_the_quadratic_form_of_H():
+    X, W, H, Hd, U = _rand_problem(51, 5, 40, 60)
+    r = O.gptq(W, U, 4, 8, False, block_size=0)
+    D = W - r.what
+    np.testing.assert_allclose(O.layer_loss(W, r.what, X), 0.5 * np.einsum("ij,jk,ik->", D, H, D), rtol=1e-10)
+    np.testing.assert_allclose(O.row_losses(W, r.what, X).sum(), O.layer_loss(W, r.what, X), rtol=1e-12)
+
+
+def test_codes_invariant_under_hessian_scaling():
+    X, W, H, Hd, U = _rand_problem(52, 7, 128, 90)
+    U2 = O.hinv_upper_cholesky(7.3 * Hd)
+    a = O.gptq(W, U, 4, 32, False, 64)
+    b = O.gptq(W, U2, 4, 32, False, 64)
+    np.testing.assert_array_equal(a.codes, b.codes)
+
+
+def test_compensation_lowers_layer_loss_vs_rtn():
+    X, W, H, Hd, U = _rand_problem(53, 32, 128, 400, hot=4)
+    g = O.gptq(W, U, 3, 32, False, 64)
+    r = O.rtn(W, 3, 32, False)
+    assert O.layer_loss(W, g.what, X) < O.layer_loss(W, r.what, X)
+
+
+# ---------------------------------------------------------------- replay protocol
+
+def test_replay_accepts_own_outputs():
+    _, W, _, _, U = _rand_problem(60, 6, 128, 150)
+    a = O.gptq(W, U, 4, 32, False, 128)
+    rr = O.gptq_replay(W, U, a.codes, a.scales, a.zeros, 4, 32, False, 128)
+    assert rr.forced_codes == rr.hard_codes == rr.hard_params == rr.forced_params == 0
+
+
+def test_replay_flags_planted_far_mistake_and_forces_near_one():
+    _, W, _, _, U = _rand_problem(61, 6, 128, 150)
+    a = O.gptq(W, U, 4, 32, False, 128)
+    dist = O.boundary_distance(a.pre, np.repeat(a.scales.T, 32, axis=1), np.repeat(a.zeros.T, 32, axis=1), 15)
+    # planted far mistake: the entry farthest from any boundary gets a different code
+    far = np.unravel_index(np.argmax(dist), dist.shape)
+    bad = a.codes.copy()
+    bad[far] = bad[far] + 1 if bad[far] < 15 else bad[far] - 1
+    rr = O.gptq_replay(W, U, bad, a.scales, a.zeros, 4, 32, False, 128)
+    assert rr.hard_codes >= 1
+    # near-boundary disagreement: move one weight onto a boundary, flip it, replay with a loose tolerance
+    near = np.unravel_index(np.argmin(dist), dist.shape)
+    bad2 = a.codes.copy()
+    x = a.pre[near] / a.scales[near[1] // 32, near[0]] + a.zeros[near[1] // 32, near[0]]
+    bad2[near] = int(np.floor(x)) if a.codes[near] == int(np.floor(x)) + 1 else int(np.floor(x)) + 1
+    bad2[near] = min(max(bad2[near], 0), 15)
+    if bad2[near] != a.codes[near]:
+        tol = float(dist[near]) * 1.0001 + 1e-300
+        rr2 = O.gptq_replay(W, U, bad2, a.scales, a.zeros, 4, 32, False, 128, tol=tol)
+        assert rr2.forced_codes >= 1
+
+
+def test_boundary_distance_closed_form():
+    s, z = 0.1, 3.0
+    # w = 0.1*(1.5-3) + 0.004 -> grid coordinate 1.54, nearest boundary 1.5 -> distance 0.004
+    assert O.boundary_distance(np.array([0.1 * (1.5 - 3) + 0.004]), s, z, 15)[0] == pytest.approx(0.004, rel=1e-9)
+    # clamped low: x = -2 -> only boundary 0.5 matters -> 2.5 grid units
+    assert O.boundary_distance(np.array([0.1 * (-2 - 3)]), s, z, 15)[0] == pytest.approx(0.25, rel=1e-9)
