@@ -1,0 +1,344 @@
+#!/usr/bin/env python3
+"""GPTQ layer-quantization benchmark.
+
+One step = the whole hot path for one linear layer of 4096 x 4096 with n = 2048
+bf16 calibration tokens, 4-bit asymmetric, group 128, lambda = 0.01 * mean(diag H):
+  H = 2 X^T X (tensor cores) -> U = upper Cholesky factor of (H + lambda I)^-1 ->
+  GPTQ column loop with 128-column lazy blocks and 3xTF32 trailing updates,
+  writing packed int32 codes, fp16 scales and packed zeros.
+Inputs are seeded synthetic data (package ``inputs``: lognormal channel scales with
+0.5 % hot channels for X, N(0, 0.02^2) weights with 0.1 % outliers), resident in HBM
+when timing starts; W is restored from a pristine copy and the L2 is flushed (256 MB
+write) before every step, outside the per-step CUDA events.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+With N > 1 (torchrun, one rank per GPU) every rank quantizes its own independent
+layer (weak scaling, no collective on the data path); the reported time is the max
+over ranks.  Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms/layer & weights quantized/s at 4096×4096 n=2048 4b g128; % of roofline"
+UNIT = "weights/s"
+D_OUT, D_IN, N_TOK, BITS, GROUP, SYM = 4096, 4096, 2048, 4, 128, False
+WORKLOAD = "attn 4096x4096, n=2048 bf16 tokens, 4-bit asym g128"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------- clocks during the timed region
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+
+def oracle_layer_time(layer, rows_sample: int = 256) -> tuple[float, str, int]:
+    """Seconds per layer of the fp64 oracle: H and U in full, column loop on a row sample, extrapolated."""
+    import numpy as np
+
+    from oracle import gptq_oracle as O
+
+    X = layer.X.astype(np.float64)
+    t0 = time.perf_counter()
+    H = O.hessian(X)
+    t1 = time.perf_counter()
+    Hd, _ = O.damp(H, 0.01)
+    U = O.hinv_upper_cholesky(Hd)
+    t2 = time.perf_counter()
+    rows = min(rows_sample, layer.d_out)
+    O.gptq(layer.W[:rows], U, BITS, GROUP, SYM, 128)
+    t3 = time.perf_counter()
+    total = (t1 - t0) + (t2 - t1) + (t3 - t2) * (layer.d_out / rows)
+    sample = (f"H=2X^T X and U=chol(Hd^-1) in full (fp64 numpy/LAPACK), column loop on {rows} of "
+              f"{layer.d_out} rows extrapolated to the layer; H {t1 - t0:.2f}s U {t2 - t1:.2f}s rows {t3 - t2:.2f}s")
+    return total, sample, len(os.sched_getaffinity(0))
+
+
+def run_reference(args, rank: int, world: int) -> None:
+    if rank != 0:
+        return
+    from post_weight_quantization_14_b200 import inputs as I
+
+    layer = I.make_layer("attn", seed=0)
+    for _ in range(args.warmup):
+        oracle_layer_time(layer)
+    secs = []
+    for _ in range(args.steps):
+        s, sample, cores = oracle_layer_time(layer)
+        secs.append(s)
+    ms = 1e3 * sum(secs) / len(secs)
+    value = D_OUT * D_IN / (ms / 1e3)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "d_out": D_OUT, "d_in": D_IN, "n": N_TOK, "bits": BITS,
+                       "group_size": GROUP, "sym": SYM},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU leg
+
+def algorithmic_work(d_out: int, d_in: int, n: int) -> dict:
+    """Per-kernel-class algorithmic flops / bytes for one layer (roofline)."""
+    B = 128
+    nblk = (d_in + B - 1) // B
+    trailing_flops = sum(2.0 * d_out * (d_in - (b + 1) * B) * B for b in range(nblk) if (b + 1) * B < d_in)
+    col_bytes = 4.0 * d_out * d_in + BITS / 8 * d_out * d_in + (2 + BITS / 8) * d_out * (d_in // GROUP)
+    return {
+        "trailing_update": ("tensor_tf32x3", trailing_flops),
+        "hessian_syrk": ("tensor_bf16", 1.0 * n * d_in * (d_in + 1)),
+        "colloop": ("hbm", col_bytes),
+        "chol": ("tensor_tf32x3", 2.0 / 3.0 * d_in ** 3),
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import numpy as np
+    import torch
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    from post_weight_quantization_14_b200 import gptq as G
+    from post_weight_quantization_14_b200 import inputs as I
+
+    layer = I.make_layer("attn", seed=rank)
+    cfg = G.make_config(BITS, GROUP, SYM, 128, 0.01)
+    W0 = torch.from_numpy(layer.W).to(dev)
+    W = torch.empty_like(W0)
+    X = torch.from_numpy(layer.X_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    bufs = G.LayerBuffers(D_OUT, D_IN, N_TOK, torch.bfloat16, cfg, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        G.quantize_layer(W, X, buffers=bufs)
+
+    for _ in range(args.warmup):
+        W.copy_(W0)
+        step()
+    G.gptq_sync_status()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    for a, b in evs:
+        W.copy_(W0)
+        flush.fill_(1)
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    G.gptq_sync_status()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * D_OUT * D_IN * args.steps / (total_ms / 1e3)
+
+    # per-kernel times (instrumented steps; every launch bracketed by CUDA events on its stream)
+    G.gptq_timing_enable(True)
+    G.gptq_timing_report()
+    reps = 3
+    for _ in range(reps):
+        W.copy_(W0)
+        flush.fill_(1)
+        step()
+    kt = G.gptq_timing_report()
+    G.gptq_timing_enable(False)
+    launches_per_step = sum(c for c, _ in kt.values()) / reps
+    kernel_ms = {k: ms / reps for k, (c, ms) in kt.items()}
+    kernel_launches = {k: c // reps for k, (c, ms) in kt.items()}
+
+    hbm, bf16, bf16_sus, peak_kind = peaks()
+    tf32 = bf16 * (1.1 / 2.25)                      # nominal tf32 : bf16 dense ratio
+    work = algorithmic_work(D_OUT, D_IN, N_TOK)
+    chol_ms = sum(v for k, v in kernel_ms.items() if k in ("chol_leaf", "chol_panel", "chol_update", "inv_bu",
+                                                           "inv_ub", "split_panel", "damp_copy", "diag_mean",
+                                                           "zero_lower"))
+    stage_ms = {"hessian": kernel_ms.get("hessian_syrk", 0) + kernel_ms.get("transpose_x", 0),
+                "prepare_hinv": chol_ms,
+                "quantize": sum(kernel_ms.get(k, 0) for k in ("colloop", "trailing_update", "up_prep", "ut_split",
+                                                             "pack_zeros", "row_params"))}
+    dom = max(kernel_ms, key=kernel_ms.get)
+    def roof(name):
+        ms = kernel_ms.get(name, 0.0)
+        n = max(1, kernel_launches.get(name, 1))
+        if name == "trailing_update":
+            achieved = work[name][1] / (ms / 1e3) / 1e12
+            return {"bound": "tensor", "achieved": achieved, "peak": tf32 / 3, "unit": "TFLOP/s",
+                    "frac": achieved / (tf32 / 3), "traffic": None,
+                    "note": f"3xTF32: peak = measured bf16 x 1.1/2.25 / 3 ({peak_kind}); {n} launches"}
+        if name == "hessian_syrk":
+            achieved = work[name][1] / (ms / 1e3) / 1e12
+            return {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
+                    "frac": achieved / bf16, "traffic": None, "note": f"bf16 {peak_kind} burst peak"}
+        if name == "colloop":
+            achieved = work[name][1] / (ms / 1e3) / 1e9
+            return {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                    "traffic": None, "note": f"HBM {peak_kind}; {n} launches"}
+        if name in ("chol_leaf", "chol_update", "chol_panel", "inv_bu", "inv_ub"):
+            achieved = work["chol"][1] / (chol_ms / 1e3) / 1e12
+            return {"bound": "tensor", "achieved": achieved, "peak": tf32 / 3, "unit": "TFLOP/s",
+                    "frac": achieved / (tf32 / 3), "traffic": None,
+                    "note": f"whole factorization stage ({chol_ms:.3f} ms) vs 3xTF32 peak ({peak_kind})"}
+        return None
+    roofline = roof(dom) or roof("trailing_update")
+    roofline["kernel"] = dom
+
+    # end-to-end through the public API with host buffers (pinned), copies inside the timed region
+    W_host = torch.from_numpy(layer.W).pin_memory()
+    X_host = torch.from_numpy(layer.X_bits.view(np.int16)).pin_memory()
+    qw_host = torch.empty(bufs.qweight.shape, dtype=torch.int32).pin_memory()
+    sc_host = torch.empty(bufs.scales.shape, dtype=torch.float16).pin_memory()
+    qz_host = torch.empty(bufs.qzeros.shape, dtype=torch.int32).pin_memory()
+    Xd = torch.empty(X_host.shape, dtype=torch.int16, device=dev)
+    e2e_steps = max(3, min(args.steps, 30))
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(stream)
+    for _ in range(e2e_steps):
+        W.copy_(W_host, non_blocking=True)
+        Xd.copy_(X_host, non_blocking=True)
+        q = G.quantize_layer(W, Xd.view(torch.bfloat16), buffers=bufs)
+        qw_host.copy_(q.qweight, non_blocking=True)
+        sc_host.copy_(q.scales, non_blocking=True)
+        qz_host.copy_(q.qzeros, non_blocking=True)
+    eb.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ea.elapsed_time(eb)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * D_OUT * D_IN * e2e_steps / (e2e_ms / 1e3)
+    h2d = W_host.numel() * 4 + X_host.numel() * 2
+    d2h = qw_host.numel() * 4 + sc_host.numel() * 2 + qz_host.numel() * 4
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, sample, cores = oracle_layer_time(layer)
+        cpu = {"value": D_OUT * D_IN / secs, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "d_out": D_OUT, "d_in": D_IN, "n": N_TOK, "bits": BITS,
+                           "group_size": GROUP, "sym": SYM, "damp_rel": 0.01,
+                           "l2": "flushed (256 MB write) before every step, outside the step events",
+                           "parallelism": f"{world} independent layers, one per GPU"},
+                "roofline": roofline,
+                "stage_ms": stage_ms,
+                "kernel_ms_per_step": kernel_ms,
+                "kernel_launches_per_step": kernel_launches,
+                "cpu_baseline": cpu,
+                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                        "steps": e2e_steps},
+                "gpu_launches": int(round(launches_per_step * args.steps)),
+                "clocks": clocks,
+                "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms)}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

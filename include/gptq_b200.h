@@ -1,0 +1,181 @@
+/*
+ * gptq_b200.h — C ABI of the GPTQ layer-quantization library for NVIDIA B200 (sm_100a).
+ *
+ * The library quantizes one linear layer W (d_out x d_in, fp32, row-major) to a
+ * b-bit group-wise integer grid with the GPTQ method:
+ *
+ *   1. gptq_hessian_accumulate   H (+)= 2 X^T X over calibration tokens X (n x d_in).
+ *   2. gptq_prepare_hinv         lambda = damp_rel * mean(diag H), Hd = H + lambda I,
+ *                                U = upper Cholesky factor of Hd^-1 (U^T U = Hd^-1).
+ *   3. gptq_quantize_layer       greedy column-order rounding with OBS error compensation,
+ *                                lazy 128-column blocks and one trailing update per block;
+ *                                writes packed codes, fp16 scales and packed zero points.
+ *   4. gptq_pack_int / gptq_dequant   packing of b-bit codes; W_hat = s * (q - z).
+ *
+ * Sources (page titles as printed; sections in quotes):
+ *   - "GPTQ：基于近似二阶信息的大模型权重量化" (freeguideonline GPTQ tutorial):
+ *     "对称与仿射量化" (q = round(x/s) + z, group-wise scale/zero),
+ *     "阶段一：构建 Hessian 逆近似" (H = 2 X^T X + lambda I, upper Cholesky factor),
+ *     "阶段二：贪婪顺序量化与懒惰批更新" (fixed column order, lazy batch updates),
+ *     "阶段三：量化与反量化" (per-group scale found during the pass, INT x scale).
+ *   - "GPTQ/AWQ量化中Group Size的精确含义与计算" (feinterview group-size article):
+ *     codes 0..2^b-1, scale and zero per group along the input dimension,
+ *     group_size = -1 is one group per row, "存储代价" (16-bit scale, b-bit zero,
+ *     symmetric stores no zero).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named as device pointers must point to memory of the current CUDA
+ *     device; the caller owns all memory.  The library never allocates.
+ *   - ``stream`` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Work is enqueued asynchronously on it; argument errors are returned at once
+ *     and enqueue nothing.
+ *   - Errors detected on the device (non-finite values, a non-positive pivot, a
+ *     bounded wait that ran out) are recorded in a per-process device status word
+ *     and returned by the next call of gptq_sync_status() on that stream
+ *     (gptq_prepare_hinv synchronises by itself).
+ *   - gptq_last_error() returns a thread-local text for the last failing call.
+ *   - Nothing here is thread-safe against concurrent calls that share buffers.
+ */
+#ifndef GPTQ_B200_H
+#define GPTQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GPTQ_OK = 0,
+    GPTQ_ERR_INVALID_ARG = 1,   /* bad pointer, size, layout or config value            */
+    GPTQ_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement (desc_act) */
+    GPTQ_ERR_NOT_PD = 3,        /* damped Hessian not positive definite (bad_col set)    */
+    GPTQ_ERR_NONFINITE = 4,     /* NaN or Inf found in an input                          */
+    GPTQ_ERR_CUDA = 5,          /* a CUDA runtime or driver call failed                  */
+    GPTQ_ERR_TIMEOUT = 6,       /* a bounded device-side wait ran out                    */
+    GPTQ_ERR_WORKSPACE = 7      /* workspace missing or smaller than the query returned */
+} gptq_status;
+
+typedef enum { GPTQ_BF16 = 0, GPTQ_F32 = 1 } gptq_dtype;
+
+/* Quantization settings (tutorial "代码示例" BaseQuantizeConfig: bits, group_size,
+ * desc_act; group-size article: sym).
+ *   bits        2, 3, 4 or 8.
+ *   group_size  -1 (one group per row) or a divisor of block_size that is >= 16.
+ *   sym         0 = asymmetric (zero point stored), 1 = symmetric (implicit zero 2^(bits-1)).
+ *   block_size  lazy-batch width; 128 is the only value this build accepts.
+ *   damp_rel    lambda = damp_rel * mean(diag H); must be >= 0 and finite.
+ *   desc_act    activation ordering; must be 0 (GPTQ_ERR_UNSUPPORTED otherwise). */
+typedef struct {
+    int bits;
+    int group_size;
+    int sym;
+    int block_size;
+    float damp_rel;
+    int desc_act;
+} gptq_config;
+
+/* Fill *cfg with bits=4, group_size=128, sym=0, block_size=128, damp_rel=0.01, desc_act=0. */
+void gptq_default_config(gptq_config* cfg);
+
+/* Static text for a status code; never NULL. */
+const char* gptq_status_string(gptq_status s);
+
+/* Text describing the last non-OK return on the calling thread ("" if none). */
+const char* gptq_last_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int gptq_version(void);
+
+/* ------------------------------------------------------------------ stage 1
+ * H (+)= 2 X^T X          (tutorial "阶段一", H = 2 X^T X)
+ *   X        device, n x d_in row-major, bf16 (raw uint16 bit patterns) or fp32.
+ *   H        device, d_in x d_in row-major fp32, written in full (both triangles).
+ *   accumulate  0: H = 2 X^T X;  1: H += 2 X^T X (call once per calibration batch).
+ *   ws       device workspace of at least gptq_hessian_workspace_bytes(n, d_in, xt) bytes.
+ * Products are formed on the tensor cores (bf16 exact products, or fp32 split into
+ * two tf32 parts with three products), accumulated in fp32.
+ * Requires d_in % 8 == 0, 1 <= n, d_in <= 65536.  Non-finite X values propagate
+ * into H and are reported by gptq_prepare_hinv. */
+size_t gptq_hessian_workspace_bytes(int64_t n, int64_t d_in, gptq_dtype xt);
+gptq_status gptq_hessian_accumulate(const void* X, gptq_dtype xt, int64_t n, int64_t d_in,
+                                    float* H, int accumulate, void* ws, size_t ws_bytes,
+                                    void* stream);
+
+/* ------------------------------------------------------------------ stage 2
+ * U = upper Cholesky factor of (H + lambda I)^-1, lambda = damp_rel * mean(diag H)
+ * (tutorial "阶段一" steps 1-2 read as the upper factor of the inverse Hessian).
+ *   H        device, d_in x d_in fp32, symmetric; only the upper triangle is read. Not modified.
+ *   U        device, d_in x d_in fp32 row-major; written in full (strict lower triangle = 0).
+ *   bad_col  host pointer or NULL; on GPTQ_ERR_NOT_PD receives the first failing column.
+ *   lambda_out  host pointer or NULL; receives lambda.
+ * Computed as Hd = R R^T with R upper (Cholesky from the bottom-right), then U = R^-1,
+ * blocked by 128 with fp32 diagonal blocks and 3xTF32 tensor-core block updates.
+ * Synchronises ``stream`` once to report NOT_PD / NONFINITE.  Returns
+ * GPTQ_ERR_INVALID_ARG when mean(diag H) <= 0.  Requires d_in % 8 == 0. */
+size_t gptq_prepare_hinv_workspace_bytes(int64_t d_in);
+gptq_status gptq_prepare_hinv(const float* H, int64_t d_in, float damp_rel, float* U,
+                              void* ws, size_t ws_bytes, int64_t* bad_col, float* lambda_out,
+                              void* stream);
+
+/* ------------------------------------------------------------------ stage 3
+ * GPTQ column loop (tutorial "阶段二", "阶段三"; group-size article).
+ *   W        device, d_out x d_in fp32 row-major; consumed as scratch (holds the
+ *            compensated weights on return).
+ *   U        device, output of gptq_prepare_hinv.
+ *   qweight  device int32 [ceil(d_in*bits/32), d_out]: column o holds row o's codes as a
+ *            little-endian bits-wide stream along d_in (code j at bits j*bits..).
+ *   scales   device fp16 bit patterns [n_groups, d_out], n_groups = ceil(d_in/g) (1 for g=-1).
+ *   qzeros   device int32 [n_groups, ceil(d_out*bits/32)], zero points packed along d_out
+ *            the same way; must be NULL when cfg->sym != 0.
+ *   err_sq   device fp32 [d_out] or NULL: per row sum_c e_c^2 with e_c = (w_c - w_hat_c)/U_cc,
+ *            which equals (W0 - W_hat) Hd (W0 - W_hat)^T of that row.
+ *   ws       device workspace of at least gptq_quantize_workspace_bytes(d_out, d_in, cfg) bytes.
+ * Per group: scale = fp16(range/maxq) from the current compensated weights at the
+ * group's first column (asymmetric range includes 0); zero = clamp(rint(-xmin/s));
+ * code = clamp(rint(w/s) + zero, 0, maxq), ties to even.
+ * Requires d_in % 8 == 0, 1 <= d_out. */
+size_t gptq_quantize_workspace_bytes(int64_t d_out, int64_t d_in, const gptq_config* cfg);
+gptq_status gptq_quantize_layer(float* W, const float* U, int64_t d_out, int64_t d_in,
+                                const gptq_config* cfg, int32_t* qweight, uint16_t* scales,
+                                int32_t* qzeros, float* err_sq, void* ws, size_t ws_bytes,
+                                void* stream);
+
+/* ------------------------------------------------------------------ packing, dequantization
+ * gptq_pack_int: pack bits-wide codes (uint8, values < 2^bits) of each row into a
+ * little-endian bit stream of int32 words, nwords = ceil(cols*bits/32).
+ *   layout 0: packed[r * nwords + k]   (qzeros layout)
+ *   layout 1: packed[k * rows + r]     (qweight layout)
+ * Values >= 2^bits are masked to their low bits. */
+gptq_status gptq_pack_int(const uint8_t* codes, int64_t rows, int64_t cols, int bits,
+                          int layout, int32_t* packed, void* stream);
+
+/* W_hat[o, c] = scale[g(c), o] * (q[o, c] - zero[g(c), o])   (tutorial "阶段三";
+ * group-size article).  Same array layouts as gptq_quantize_layer; qzeros NULL iff sym. */
+gptq_status gptq_dequant(const int32_t* qweight, const uint16_t* scales, const int32_t* qzeros,
+                         int64_t d_out, int64_t d_in, const gptq_config* cfg, float* W_hat,
+                         void* stream);
+
+/* Synchronise ``stream`` and return (and clear) the device status word. */
+gptq_status gptq_sync_status(void* stream);
+
+/* ------------------------------------------------------------------ diagnostics
+ * gptq_timing_enable(1): every kernel launch of the library is bracketed by CUDA
+ * events on its stream.  gptq_timing_report() synchronises the device, writes a JSON
+ * object {"kernel_name": [launches, total_ms], ...} of everything recorded since the
+ * last report into buf (NUL-terminated, truncated to len) and returns the number of
+ * bytes needed.  Host-side bookkeeping only; not thread-safe.
+ *
+ * gptq_selftest_bounded_wait: launches one thread that waits on a barrier nobody
+ * arrives at, with a limit of limit_ns nanoseconds, the same bounded wait every
+ * pipeline in the library uses; the next gptq_sync_status() returns GPTQ_ERR_TIMEOUT.
+ * Used to test the timeout path without faulting or hanging the device. */
+void gptq_timing_enable(int on);
+size_t gptq_timing_report(char* buf, size_t len);
+gptq_status gptq_selftest_bounded_wait(uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPTQ_B200_H */

@@ -166,6 +166,7 @@ class GPTQResult:
     err: np.ndarray          # fp64 [d_out, d_in], e_c = (w_c - what_c) / U_cc
     pre: np.ndarray          # fp64 [d_out, d_in], value w_c that was rounded
     what: np.ndarray         # fp64 [d_out, d_in], dequantized weights
+    own_scales: np.ndarray | None = None   # replay only: this oracle's own fp16 scales
     forced_codes: int = 0
     forced_params: int = 0
     hard_codes: int = 0
@@ -198,9 +199,11 @@ class _Replay:
         self.tol = float(tol)
         self.forced_codes = self.forced_params = self.hard_codes = self.hard_params = 0
         self.worst = 0.0
+        self.own_scales = np.array(self.scales, copy=True)
 
     def params(self, gi, scale, zero, raw, lo, hi, bits, sym):
         maxq = (1 << bits) - 1
+        self.own_scales[gi] = scale
         other_s = self.scales[gi]
         diff = other_s != scale
         if np.any(diff):
@@ -307,6 +310,7 @@ def gptq(W0: np.ndarray, U: np.ndarray, bits: int = 4, group_size: int = 128,
         res.forced_codes, res.forced_params = replay.forced_codes, replay.forced_params
         res.hard_codes, res.hard_params = replay.hard_codes, replay.hard_params
         res.worst_forced_dist = replay.worst
+        res.own_scales = replay.own_scales
     return res
 
 

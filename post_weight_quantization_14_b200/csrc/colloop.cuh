@@ -1,0 +1,446 @@
+// GPTQ column loop for one 128-column lazy block (tutorial "阶段二" greedy order and
+// lazy batch updates, "阶段三" group-wise scale; group-size article for scale/zero).
+//
+// Rows are independent.  Four lanes share one row; lane k of the row holds the
+// block's columns k, k+4, ..., k+124 in registers (cyclic mapping keeps the per-step
+// update work balanced across the four lanes).  For column c of the block:
+//   owner lane (c % 4):  r = clamp(rint(w_c / s), -z, maxq - z);  d_c = w_c - s * r
+//   all four lanes:      w_j -= d_c * U[c, j] / U[c, c]   for the block columns j > c
+// which is e_c = d_c / U_cc pushed forward with row c of U.  The normalised rows of
+// the block's 128x128 diagonal part of U are prepared once per layer and staged into
+// shared memory by one bulk (TMA) copy per CTA.
+// At a group's first column the scale and zero come from the current values of the
+// group's columns (min/max by a 4-lane shuffle reduction).
+// At the end of the block the kernel writes the packed codes (qweight layout), the
+// errors e = d / U_cc as a tf32 split (operand of the trailing tensor-core update)
+// and the per-row sum of e^2.
+#pragma once
+#include "gemm_tc.cuh"
+#include "pack.cuh"
+
+namespace gq {
+
+constexpr int CB = 128;                  // lazy block width
+constexpr int CL_WARPS = 2;
+constexpr int CL_ROWS = CL_WARPS * 8;    // rows per CTA
+constexpr int UP_LD = 36;                // padded slot stride of one lane's row segment
+constexpr int UP_ROW = 4 * UP_LD;        // floats per normalised U row
+constexpr int UP_BLOCK = CB * UP_ROW;    // floats per block (73728 bytes)
+constexpr int CODE_LD = 132;
+constexpr int DV_LD = 129;
+constexpr float kF16MinPos = 5.9604644775390625e-08f;  // 2^-24, smallest positive fp16
+
+struct ColArgs {
+    float* W;
+    long long d_out, d_in;
+    int c0, nc;
+    const float* Up;      // normalised U rows of this block, [128][UP_ROW]
+    const float* inv_d;   // [d_in] 1 / U_cc
+    int g, sym;
+    const float* row_scale;
+    const float* row_zero;
+    int32_t* qweight;
+    __half* scales;
+    uint8_t* zeros_u8;
+    float* E_hi;
+    float* E_lo;
+    float* err_sq;
+    int first_block;
+};
+
+struct ColSmem {
+    float up[UP_BLOCK];
+    float dv[CL_ROWS][DV_LD];
+    float invd[CB];
+    uint8_t codes[CL_ROWS][CODE_LD];
+    uint64_t bar;
+};
+
+// Scale and zero of a group with grid range [lo, hi] (lo <= 0 <= hi, or -m..m).
+template <int BITS>
+__device__ __forceinline__ void group_grid(float lo, float hi, int sym, float& s, float& z) {
+    constexpr int MAXQ = (1 << BITS) - 1;
+    if (hi == lo) {
+        s = 1.f;
+    } else {
+        s = __half2float(__float2half_rn(__fdiv_rn(hi - lo, (float)MAXQ)));
+        if (s == 0.f) s = kF16MinPos;
+    }
+    if (sym)
+        z = (float)(1 << (BITS - 1));
+    else
+        z = fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.f), (float)MAXQ);
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p) {
+    extern __shared__ __align__(128) uint8_t cl_raw[];
+    ColSmem& S = *reinterpret_cast<ColSmem*>(cl_raw);
+    constexpr unsigned FULL = 0xffffffffu;
+    constexpr int MAXQ = (1 << BITS) - 1;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int k = lane & 3;
+    const int rloc = warp * 8 + (lane >> 2);
+    const long long row = (long long)blockIdx.x * CL_ROWS + rloc;
+    const bool row_ok = row < p.d_out;
+
+    if (tid == 0) {
+        mbar_init(&S.bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        constexpr uint32_t bytes = UP_BLOCK * 4;
+        constexpr uint32_t chunk = bytes / 4;
+        mbar_arrive_expect_tx(&S.bar, bytes);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            bulk_g2s(reinterpret_cast<uint8_t*>(S.up) + i * chunk,
+                     reinterpret_cast<const uint8_t*>(p.Up) + i * chunk, chunk, &S.bar);
+    }
+    for (int c = tid; c < CB; c += blockDim.x) S.invd[c] = (c < p.nc) ? p.inv_d[p.c0 + c] : 0.f;
+
+    float wv[32];
+    {
+        const float* wrow = p.W + row * p.d_in + p.c0;
+        bool finite = true;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            const int col = k + 4 * t;
+            float v = 0.f;
+            if (row_ok && col < p.nc) v = wrow[col];
+            finite = finite && isfinite(v);
+            wv[t] = v;
+        }
+        if (!finite) record_status(GPTQ_ERR_NONFINITE, row);
+    }
+
+    float s = 1.f, inv_s = 1.f, qlo = 0.f, qhi = (float)MAXQ;
+    if (p.g < 0 && row_ok) {
+        const float z = p.row_zero[row];
+        s = p.row_scale[row];
+        inv_s = __frcp_rn(s);
+        qlo = -z;
+        qhi = (float)MAXQ - z;
+    }
+    const bool ok = mbar_wait(&S.bar, 0, -1 - (long long)blockIdx.x);
+    __syncthreads();
+    if (!ok) return;
+
+    const int g = p.g;
+    const int gmask = g > 0 ? g - 1 : 0;
+#pragma unroll
+    for (int c = 0; c < CB; ++c) {
+        const int t = c >> 2, own = c & 3;
+        if (g > 0 && (c & gmask) == 0) {
+            const int tend = (c + g) >> 2;
+            float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+            for (int t2 = t; t2 < 32; ++t2) {
+                if (t2 < tend) {
+                    mn = fminf(mn, wv[t2]);
+                    mx = fmaxf(mx, wv[t2]);
+                }
+            }
+            mn = fminf(mn, __shfl_xor_sync(FULL, mn, 1));
+            mn = fminf(mn, __shfl_xor_sync(FULL, mn, 2));
+            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
+            float lo, hi;
+            if (p.sym) {
+                const float m = fmaxf(fabsf(mn), fabsf(mx));
+                lo = -m;
+                hi = m;
+            } else {
+                lo = fminf(mn, 0.f);
+                hi = fmaxf(mx, 0.f);
+            }
+            float z;
+            group_grid<BITS>(lo, hi, p.sym, s, z);
+            inv_s = __frcp_rn(s);
+            qlo = -z;
+            qhi = (float)MAXQ - z;
+            if (k == 0 && row_ok) {
+                const long long gi = (p.c0 + c) / g;
+                p.scales[gi * p.d_out + row] = __float2half_rn(s);
+                p.zeros_u8[gi * p.d_out + row] = (uint8_t)(int)z;
+            }
+        }
+        const float x = wv[t] * inv_s;
+        const float r = fminf(fmaxf(rintf(x), qlo), qhi);
+        const float dd = fmaf(-r, s, wv[t]);
+        const float db = __shfl_sync(FULL, dd, (lane & ~3) | own);
+        if (k == own) {
+            S.codes[rloc][c] = (uint8_t)(int)(r - qlo);
+            S.dv[rloc][c] = dd;
+        }
+        const float* urow = S.up + c * UP_ROW + k * UP_LD;
+#pragma unroll
+        for (int q4 = (t >> 2); q4 < 8; ++q4) {
+            const float4 u4 = *reinterpret_cast<const float4*>(urow + 4 * q4);
+            if (4 * q4 + 0 >= t) wv[4 * q4 + 0] = fmaf(-db, u4.x, wv[4 * q4 + 0]);
+            if (4 * q4 + 1 >= t) wv[4 * q4 + 1] = fmaf(-db, u4.y, wv[4 * q4 + 1]);
+            if (4 * q4 + 2 >= t) wv[4 * q4 + 2] = fmaf(-db, u4.z, wv[4 * q4 + 2]);
+            if (4 * q4 + 3 >= t) wv[4 * q4 + 3] = fmaf(-db, u4.w, wv[4 * q4 + 3]);
+        }
+    }
+    __syncwarp();
+
+    // errors of the block (operand of the trailing update) and per-row sum of e^2
+    const long long wrow0 = (long long)blockIdx.x * CL_ROWS + warp * 8;
+    for (int rr = 0; rr < 8; ++rr) {
+        const long long rw = wrow0 + rr;
+        const int rl = warp * 8 + rr;
+        float acc = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int col = lane + 32 * q;
+            const float e = S.dv[rl][col] * S.invd[col];
+            acc = fmaf(e, e, acc);
+            if (rw < p.d_out) {
+                float h, l;
+                split_tf32(e, h, l);
+                p.E_hi[rw * CB + col] = h;
+                p.E_lo[rw * CB + col] = l;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
+        if (lane == 0 && rw < p.d_out && p.err_sq)
+            p.err_sq[rw] = (p.first_block ? 0.f : p.err_sq[rw]) + acc;
+    }
+
+    // packed codes: word w of this block's stream for each of the warp's 8 rows
+    const int nwb = (p.nc * BITS + 31) / 32;
+    const long long wbase = (long long)p.c0 * BITS / 32;
+    for (int idx = lane; idx < 8 * nwb; idx += 32) {
+        const int rr = idx & 7, w = idx >> 3;
+        const long long rw = wrow0 + rr;
+        if (rw >= p.d_out) continue;
+        const int rl = warp * 8 + rr;
+        const int bit0 = w * 32;
+        const int j0 = bit0 / BITS, j1 = min(p.nc - 1, (bit0 + 31) / BITS);
+        unsigned long long acc = 0;
+        for (int j = j0; j <= j1; ++j)
+            acc |= (unsigned long long)(S.codes[rl][j] & MAXQ) << (j * BITS - bit0 + 8);
+        p.qweight[(wbase + w) * p.d_out + rw] = (int32_t)(uint32_t)(acc >> 8);
+    }
+}
+
+// Normalised, lane-permuted rows of each 128x128 diagonal block of U:
+// Up[b][c][k*UP_LD + t] = U[c0+c, c0+j] / U[c0+c, c0+c] for j = k + 4t > c (0 otherwise),
+// and inv_d[c] = 1 / U[c, c].
+__global__ void up_prep_kernel(const float* __restrict__ U, long long d, float* __restrict__ Up,
+                               float* __restrict__ inv_d) {
+    const int b = blockIdx.y, c = blockIdx.x;
+    const long long c0 = (long long)b * CB;
+    const int nc = (int)min((long long)CB, d - c0);
+    const float ucc = (c < nc) ? U[(c0 + c) * d + c0 + c] : 1.f;
+    float* dst = Up + ((long long)b * CB + c) * UP_ROW;
+    for (int e = threadIdx.x; e < UP_ROW; e += blockDim.x) {
+        const int kk = e / UP_LD, t = e % UP_LD;
+        const int j = kk + 4 * t;
+        float v = 0.f;
+        if (t < 32 && c < nc && j < nc && j > c) v = __fdiv_rn(U[(c0 + c) * d + c0 + j], ucc);
+        dst[e] = v;
+    }
+    if (threadIdx.x == 0 && c < nc) inv_d[c0 + c] = __frcp_rn(ucc);
+}
+
+// UT[j, i] = split(U[i, j]) for the 32x32 tiles on or above the diagonal of U.
+__global__ void ut_split_kernel(const float* __restrict__ U, long long d, float* __restrict__ UT_hi,
+                                float* __restrict__ UT_lo) {
+    __shared__ float tile[32][33];
+    const long long bi = blockIdx.y, bj = blockIdx.x;  // tile of U
+    if (bi > bj) return;
+    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+        const long long i = bi * 32 + r, j = bj * 32 + threadIdx.x;
+        tile[r][threadIdx.x] = (i < d && j < d) ? U[i * d + j] : 0.f;
+    }
+    __syncthreads();
+    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+        const long long j = bj * 32 + r, i = bi * 32 + threadIdx.x;
+        if (i < d && j < d) {
+            float h, l;
+            split_tf32(tile[threadIdx.x][r], h, l);
+            UT_hi[j * d + i] = h;
+            UT_lo[j * d + i] = l;
+        }
+    }
+}
+
+// group_size = -1: one scale/zero per row from the whole original row.
+template <int BITS>
+__global__ void row_params_kernel(const float* __restrict__ W, long long d_out, long long d_in, int sym,
+                                  float* __restrict__ row_scale, float* __restrict__ row_zero,
+                                  __half* __restrict__ scales, uint8_t* __restrict__ zeros_u8) {
+    const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= d_out) return;
+    float mn = INFINITY, mx = -INFINITY;
+    bool finite = true;
+    for (long long c = lane; c < d_in; c += 32) {
+        const float v = W[row * d_in + c];
+        finite = finite && isfinite(v);
+        mn = fminf(mn, v);
+        mx = fmaxf(mx, v);
+    }
+    for (int o = 16; o; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (!finite) record_status(GPTQ_ERR_NONFINITE, row);
+    if (lane == 0) {
+        float lo, hi;
+        if (sym) {
+            const float m = fmaxf(fabsf(mn), fabsf(mx));
+            lo = -m;
+            hi = m;
+        } else {
+            lo = fminf(mn, 0.f);
+            hi = fmaxf(mx, 0.f);
+        }
+        float s, z;
+        group_grid<BITS>(lo, hi, sym, s, z);
+        row_scale[row] = s;
+        row_zero[row] = z;
+        scales[row] = __float2half_rn(s);
+        zeros_u8[row] = (uint8_t)(int)z;
+    }
+}
+
+}  // namespace gq
+
+namespace gqh {
+
+struct QuantWs {
+    float *Up, *inv_d, *UT_hi, *UT_lo, *E_hi, *E_lo, *row_scale, *row_zero;
+    uint8_t* zeros_u8;
+};
+
+inline long long n_groups_of(long long d_in, int g) { return g < 0 ? 1 : (d_in + g - 1) / g; }
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline size_t quant_ws_bytes(long long d_out, long long d_in, int g) {
+    const long long nblk = (d_in + gq::CB - 1) / gq::CB;
+    size_t b = 0;
+    b += align256((size_t)nblk * gq::UP_BLOCK * 4);
+    b += align256((size_t)d_in * 4);
+    b += 2 * align256((size_t)d_in * d_in * 4);
+    b += 2 * align256((size_t)d_out * gq::CB * 4);
+    b += 2 * align256((size_t)d_out * 4);
+    b += align256((size_t)n_groups_of(d_in, g) * d_out);
+    return b;
+}
+
+inline QuantWs quant_ws_carve(void* ws, long long d_out, long long d_in, int g) {
+    const long long nblk = (d_in + gq::CB - 1) / gq::CB;
+    uint8_t* p = static_cast<uint8_t*>(ws);
+    QuantWs w;
+    auto take = [&](size_t bytes) {
+        uint8_t* q = p;
+        p += align256(bytes);
+        return q;
+    };
+    w.Up = reinterpret_cast<float*>(take((size_t)nblk * gq::UP_BLOCK * 4));
+    w.inv_d = reinterpret_cast<float*>(take((size_t)d_in * 4));
+    w.UT_hi = reinterpret_cast<float*>(take((size_t)d_in * d_in * 4));
+    w.UT_lo = reinterpret_cast<float*>(take((size_t)d_in * d_in * 4));
+    w.E_hi = reinterpret_cast<float*>(take((size_t)d_out * gq::CB * 4));
+    w.E_lo = reinterpret_cast<float*>(take((size_t)d_out * gq::CB * 4));
+    w.row_scale = reinterpret_cast<float*>(take((size_t)d_out * 4));
+    w.row_zero = reinterpret_cast<float*>(take((size_t)d_out * 4));
+    w.zeros_u8 = take((size_t)n_groups_of(d_in, g) * d_out);
+    return w;
+}
+
+template <int BITS>
+cudaError_t quant_run_bits(float* W, const float* U, long long d_out, long long d_in, const gptq_config& cfg,
+                           int32_t* qweight, __half* scales, int32_t* qzeros, float* err_sq, void* ws,
+                           cudaStream_t st) {
+    const int g = cfg.group_size;
+    QuantWs w = quant_ws_carve(ws, d_out, d_in, g);
+    const int nblk = (int)((d_in + gq::CB - 1) / gq::CB);
+    {
+        dim3 grid(gq::CB, nblk);
+        {
+            gqh::TimedScope ts__("up_prep", st);
+            gq::up_prep_kernel<<<grid, 160, 0, st>>>(U, d_in, w.Up, w.inv_d);
+        }
+        GQ_TRY(cudaGetLastError());
+        dim3 tb(32, 8), g2((unsigned)((d_in + 31) / 32), (unsigned)((d_in + 31) / 32));
+        {
+            gqh::TimedScope ts__("ut_split", st);
+            gq::ut_split_kernel<<<g2, tb, 0, st>>>(U, d_in, w.UT_hi, w.UT_lo);
+        }
+        GQ_TRY(cudaGetLastError());
+    }
+    if (g < 0) {
+        {
+            gqh::TimedScope ts__("row_params", st);
+            gq::row_params_kernel<BITS><<<(unsigned)((d_out + 7) / 8), 256, 0, st>>>(
+                W, d_out, d_in, cfg.sym, w.row_scale, w.row_zero, scales, w.zeros_u8);
+        }
+        GQ_TRY(cudaGetLastError());
+    }
+    const int smem = (int)sizeof(gq::ColSmem);
+    GQ_TRY(cudaFuncSetAttribute(gq::colloop_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    const unsigned grid = (unsigned)((d_out + gq::CL_ROWS - 1) / gq::CL_ROWS);
+    Mat eh{w.E_hi, (uint64_t)d_out, (uint64_t)gq::CB, (uint64_t)gq::CB};
+    Mat el{w.E_lo, (uint64_t)d_out, (uint64_t)gq::CB, (uint64_t)gq::CB};
+    Mat uh{w.UT_hi, (uint64_t)d_in, (uint64_t)d_in, (uint64_t)d_in};
+    Mat ul{w.UT_lo, (uint64_t)d_in, (uint64_t)d_in, (uint64_t)d_in};
+    for (int b = 0; b < nblk; ++b) {
+        gq::ColArgs a{};
+        a.W = W;
+        a.d_out = d_out;
+        a.d_in = d_in;
+        a.c0 = b * gq::CB;
+        a.nc = (int)std::min<long long>(gq::CB, d_in - a.c0);
+        a.Up = w.Up + (long long)b * gq::UP_BLOCK;
+        a.inv_d = w.inv_d;
+        a.g = g;
+        a.sym = cfg.sym;
+        a.row_scale = w.row_scale;
+        a.row_zero = w.row_zero;
+        a.qweight = qweight;
+        a.scales = scales;
+        a.zeros_u8 = w.zeros_u8;
+        a.E_hi = w.E_hi;
+        a.E_lo = w.E_lo;
+        a.err_sq = err_sq;
+        a.first_block = (b == 0);
+        {
+            gqh::TimedScope ts__("colloop", st);
+            gq::colloop_kernel<BITS><<<grid, gq::CL_WARPS * 32, smem, st>>>(a);
+        }
+        GQ_TRY(cudaGetLastError());
+        const long long e = (long long)a.c0 + gq::CB;
+        if (e < d_in) {  // trailing update W[:, e:] -= Err U[blk, e:]
+            gq::GemmArgs p = gemm_args((int)d_out, (int)(d_in - e), gq::CB);
+            p.b_row0 = (int)e;
+            p.b_col0 = a.c0;
+            p.alpha = -1.f;
+            p.beta = 1.f;
+            p.C = W;
+            p.ldc = d_in;
+            p.c_col0 = (int)e;
+            p.write_c = 1;
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 256, 2>(eh, el, uh, ul, p, 1, st, "trailing_update")));
+        }
+    }
+    if (!cfg.sym && qzeros) {
+        const long long ng = n_groups_of(d_in, g);
+        const long long words = ng * ((d_out * BITS + 31) / 32);
+        {
+            gqh::TimedScope ts__("pack_zeros", st);
+            gq::pack_int_kernel<<<(unsigned)std::min<long long>((words + 255) / 256, 4096), 256, 0, st>>>(
+                w.zeros_u8, ng, d_out, BITS, 0, qzeros);
+        }
+        GQ_TRY(cudaGetLastError());
+    }
+    return cudaSuccess;
+}
+
+}  // namespace gqh

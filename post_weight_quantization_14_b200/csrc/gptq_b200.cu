@@ -1,0 +1,353 @@
+// C ABI of the GPTQ layer-quantization library (declared in include/gptq_b200.h).
+// Argument validation, workspace carving, status handling; all arithmetic runs in
+// the kernels of the included headers.
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "hessian.cuh"
+#include "chol.cuh"
+#include "pack.cuh"
+#include "colloop.cuh"
+
+namespace gqh {
+
+static thread_local char g_last_error[512] = "";
+
+void set_last_error(const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+}
+
+// ---------------------------------------------------------------- per-launch timing
+struct PendingLaunch {
+    std::string name;
+    cudaEvent_t a, b;
+};
+static bool g_timing = false;
+static std::vector<PendingLaunch> g_pending;
+static std::vector<cudaEvent_t> g_event_pool;
+static std::map<std::string, std::pair<long long, double>> g_timing_acc;
+
+static cudaEvent_t pooled_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+bool timing_on() { return g_timing; }
+
+void timing_begin(const char* name, cudaStream_t st) {
+    PendingLaunch p{name, pooled_event(), pooled_event()};
+    cudaEventRecord(p.a, st);
+    g_pending.push_back(p);
+}
+
+void timing_end(cudaStream_t st) {
+    if (!g_pending.empty()) cudaEventRecord(g_pending.back().b, st);
+}
+
+static void timing_collect() {
+    cudaDeviceSynchronize();
+    for (auto& p : g_pending) {
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
+            auto& acc = g_timing_acc[p.name];
+            acc.first += 1;
+            acc.second += ms;
+        }
+        g_event_pool.push_back(p.a);
+        g_event_pool.push_back(p.b);
+    }
+    g_pending.clear();
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
+                  uint64_t ld, uint32_t box_rows, uint32_t box_cols) {
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return false;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    if (rows == 0 || cols == 0) return false;
+    const CUtensorMapDataType dt =
+        elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * (uint64_t)elem_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static gptq_status fail(gptq_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+static gptq_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(GPTQ_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static gptq_status check_config(const gptq_config* cfg) {
+    if (!cfg) return fail(GPTQ_ERR_INVALID_ARG, "cfg is NULL");
+    if (cfg->desc_act) return fail(GPTQ_ERR_UNSUPPORTED, "desc_act (activation ordering) is not implemented");
+    if (!(cfg->bits == 2 || cfg->bits == 3 || cfg->bits == 4 || cfg->bits == 8))
+        return fail(GPTQ_ERR_INVALID_ARG, "bits must be 2, 3, 4 or 8 (got %d)", cfg->bits);
+    if (cfg->block_size != 128) return fail(GPTQ_ERR_INVALID_ARG, "block_size must be 128 (got %d)", cfg->block_size);
+    const int g = cfg->group_size;
+    if (!(g == -1 || (g >= 16 && g <= cfg->block_size && cfg->block_size % g == 0 && (g & (g - 1)) == 0)))
+        return fail(GPTQ_ERR_INVALID_ARG, "group_size must be -1 or 16, 32, 64, 128 (got %d)", g);
+    if (cfg->sym != 0 && cfg->sym != 1) return fail(GPTQ_ERR_INVALID_ARG, "sym must be 0 or 1");
+    if (!(cfg->damp_rel >= 0.f) || cfg->damp_rel != cfg->damp_rel || cfg->damp_rel > 1e30f)
+        return fail(GPTQ_ERR_INVALID_ARG, "damp_rel must be finite and >= 0");
+    return GPTQ_OK;
+}
+
+static gptq_status read_status(cudaStream_t st, long long* index) {
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    unsigned long long v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, gq::g_status, sizeof(v));
+    if (e != cudaSuccess) return cuda_fail(e, "read status");
+    e = cudaMemcpyToSymbol(gq::g_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "clear status");
+    if (!v) return GPTQ_OK;
+    const int code = (int)(v >> 48);
+    long long idx = (long long)(v & 0xFFFFFFFFFFFFull);
+    if (idx & 0x800000000000ll) idx |= ~0xFFFFFFFFFFFFll;  // sign-extend 48-bit index
+    if (index) *index = idx;
+    return fail((gptq_status)code, "device reported %s at index %lld", gptq_status_string((gptq_status)code), idx);
+}
+
+}  // namespace gqh
+
+namespace gq {
+
+// One thread waits on an mbarrier that nobody arrives at; the bounded wait records
+// GPTQ_ERR_TIMEOUT and returns.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    (void)mbar_wait(&bar, 0, 0x7E57, limit_ns);
+}
+
+}  // namespace gq
+
+using namespace gqh;
+
+extern "C" {
+
+void gptq_default_config(gptq_config* cfg) {
+    if (!cfg) return;
+    cfg->bits = 4;
+    cfg->group_size = 128;
+    cfg->sym = 0;
+    cfg->block_size = 128;
+    cfg->damp_rel = 0.01f;
+    cfg->desc_act = 0;
+}
+
+const char* gptq_status_string(gptq_status s) {
+    switch (s) {
+        case GPTQ_OK: return "GPTQ_OK";
+        case GPTQ_ERR_INVALID_ARG: return "GPTQ_ERR_INVALID_ARG";
+        case GPTQ_ERR_UNSUPPORTED: return "GPTQ_ERR_UNSUPPORTED";
+        case GPTQ_ERR_NOT_PD: return "GPTQ_ERR_NOT_PD";
+        case GPTQ_ERR_NONFINITE: return "GPTQ_ERR_NONFINITE";
+        case GPTQ_ERR_CUDA: return "GPTQ_ERR_CUDA";
+        case GPTQ_ERR_TIMEOUT: return "GPTQ_ERR_TIMEOUT";
+        case GPTQ_ERR_WORKSPACE: return "GPTQ_ERR_WORKSPACE";
+    }
+    return "GPTQ_ERR_UNKNOWN";
+}
+
+const char* gptq_last_error(void) { return g_last_error; }
+
+int gptq_version(void) { return 100; }
+
+size_t gptq_hessian_workspace_bytes(int64_t n, int64_t d_in, gptq_dtype xt) {
+    if (n < 1 || d_in < 1) return 0;
+    return hessian_ws_bytes(n, d_in, xt);
+}
+
+gptq_status gptq_hessian_accumulate(const void* X, gptq_dtype xt, int64_t n, int64_t d_in, float* H,
+                                    int accumulate, void* ws, size_t ws_bytes, void* stream) {
+    if (!X || !H) return fail(GPTQ_ERR_INVALID_ARG, "X and H must be non-NULL");
+    if (xt != GPTQ_BF16 && xt != GPTQ_F32) return fail(GPTQ_ERR_INVALID_ARG, "unknown X dtype %d", (int)xt);
+    if (n < 1 || n > (1ll << 30)) return fail(GPTQ_ERR_INVALID_ARG, "n out of range (%lld)", (long long)n);
+    if (d_in < 8 || d_in > 65536 || d_in % 8) return fail(GPTQ_ERR_INVALID_ARG, "d_in must be a multiple of 8 in [8, 65536]");
+    if (!aligned16(X) || !aligned16(H)) return fail(GPTQ_ERR_INVALID_ARG, "X and H must be 16-byte aligned");
+    if (!ws || ws_bytes < hessian_ws_bytes(n, d_in, xt) || !aligned16(ws))
+        return fail(GPTQ_ERR_WORKSPACE, "workspace needs %zu bytes", hessian_ws_bytes(n, d_in, xt));
+    cudaError_t e = hessian_run(X, xt, n, d_in, H, accumulate ? 1 : 0, ws, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "hessian");
+    return GPTQ_OK;
+}
+
+size_t gptq_prepare_hinv_workspace_bytes(int64_t d_in) {
+    if (d_in < 1) return 0;
+    return hinv_ws_bytes(d_in);
+}
+
+gptq_status gptq_prepare_hinv(const float* H, int64_t d_in, float damp_rel, float* U, void* ws, size_t ws_bytes,
+                              int64_t* bad_col, float* lambda_out, void* stream) {
+    if (!H || !U) return fail(GPTQ_ERR_INVALID_ARG, "H and U must be non-NULL");
+    if (d_in < 8 || d_in > 65536 || d_in % 8) return fail(GPTQ_ERR_INVALID_ARG, "d_in must be a multiple of 8 in [8, 65536]");
+    if (!(damp_rel >= 0.f) || damp_rel > 1e30f) return fail(GPTQ_ERR_INVALID_ARG, "damp_rel must be finite and >= 0");
+    if (!aligned16(H) || !aligned16(U)) return fail(GPTQ_ERR_INVALID_ARG, "H and U must be 16-byte aligned");
+    if (!ws || ws_bytes < hinv_ws_bytes(d_in) || !aligned16(ws))
+        return fail(GPTQ_ERR_WORKSPACE, "workspace needs %zu bytes", hinv_ws_bytes(d_in));
+    cudaStream_t st = (cudaStream_t)stream;
+    long long idx = -1;
+    gptq_status pre = read_status(st, &idx);  // clears any stale device status
+    (void)pre;
+    cudaError_t e = hinv_run(H, d_in, damp_rel, U, ws, st);
+    if (e != cudaSuccess) return cuda_fail(e, "prepare_hinv");
+    idx = -1;
+    gptq_status s = read_status(st, &idx);
+    if (bad_col) *bad_col = (s == GPTQ_ERR_NOT_PD || s == GPTQ_ERR_NONFINITE) ? idx : -1;
+    if (lambda_out) {
+        HinvWs w = hinv_ws_carve(ws, d_in);
+        float lam = 0.f;
+        e = cudaMemcpy(&lam, w.scal, sizeof(float), cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail(e, "read lambda");
+        *lambda_out = lam;
+    }
+    return s;
+}
+
+size_t gptq_quantize_workspace_bytes(int64_t d_out, int64_t d_in, const gptq_config* cfg) {
+    if (d_out < 1 || d_in < 1 || !cfg) return 0;
+    return quant_ws_bytes(d_out, d_in, cfg->group_size);
+}
+
+gptq_status gptq_quantize_layer(float* W, const float* U, int64_t d_out, int64_t d_in, const gptq_config* cfg,
+                                int32_t* qweight, uint16_t* scales, int32_t* qzeros, float* err_sq, void* ws,
+                                size_t ws_bytes, void* stream) {
+    gptq_status cs = check_config(cfg);
+    if (cs != GPTQ_OK) return cs;
+    if (!W || !U || !qweight || !scales) return fail(GPTQ_ERR_INVALID_ARG, "W, U, qweight and scales must be non-NULL");
+    if (cfg->sym && qzeros) return fail(GPTQ_ERR_INVALID_ARG, "qzeros must be NULL for symmetric quantization");
+    if (!cfg->sym && !qzeros) return fail(GPTQ_ERR_INVALID_ARG, "qzeros is required for asymmetric quantization");
+    if (d_out < 1 || d_out > (1ll << 30)) return fail(GPTQ_ERR_INVALID_ARG, "d_out out of range");
+    if (d_in < 8 || d_in > 65536 || d_in % 8) return fail(GPTQ_ERR_INVALID_ARG, "d_in must be a multiple of 8 in [8, 65536]");
+    if (!aligned16(W) || !aligned16(U)) return fail(GPTQ_ERR_INVALID_ARG, "W and U must be 16-byte aligned");
+    const size_t need = quant_ws_bytes(d_out, d_in, cfg->group_size);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return fail(GPTQ_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+    cudaStream_t st = (cudaStream_t)stream;
+    __half* sc = reinterpret_cast<__half*>(scales);
+    cudaError_t e;
+    switch (cfg->bits) {
+        case 2: e = quant_run_bits<2>(W, U, d_out, d_in, *cfg, qweight, sc, qzeros, err_sq, ws, st); break;
+        case 3: e = quant_run_bits<3>(W, U, d_out, d_in, *cfg, qweight, sc, qzeros, err_sq, ws, st); break;
+        case 4: e = quant_run_bits<4>(W, U, d_out, d_in, *cfg, qweight, sc, qzeros, err_sq, ws, st); break;
+        default: e = quant_run_bits<8>(W, U, d_out, d_in, *cfg, qweight, sc, qzeros, err_sq, ws, st); break;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "quantize_layer");
+    return GPTQ_OK;
+}
+
+gptq_status gptq_pack_int(const uint8_t* codes, int64_t rows, int64_t cols, int bits, int layout, int32_t* packed,
+                          void* stream) {
+    if (!codes || !packed) return fail(GPTQ_ERR_INVALID_ARG, "codes and packed must be non-NULL");
+    if (rows < 1 || cols < 1) return fail(GPTQ_ERR_INVALID_ARG, "rows and cols must be >= 1");
+    if (!(bits == 2 || bits == 3 || bits == 4 || bits == 8)) return fail(GPTQ_ERR_INVALID_ARG, "bits must be 2, 3, 4 or 8");
+    if (layout != 0 && layout != 1) return fail(GPTQ_ERR_INVALID_ARG, "layout must be 0 or 1");
+    const long long words = rows * ((cols * bits + 31) / 32);
+    {
+        gqh::TimedScope ts__("pack_int", (cudaStream_t)stream);
+        gq::pack_int_kernel<<<(unsigned)std::min<long long>((words + 255) / 256, 8192), 256, 0, (cudaStream_t)stream>>>(
+            codes, rows, cols, bits, layout, packed);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "pack_int");
+    return GPTQ_OK;
+}
+
+gptq_status gptq_dequant(const int32_t* qweight, const uint16_t* scales, const int32_t* qzeros, int64_t d_out,
+                         int64_t d_in, const gptq_config* cfg, float* W_hat, void* stream) {
+    if (!cfg) return fail(GPTQ_ERR_INVALID_ARG, "cfg is NULL");
+    if (!(cfg->bits == 2 || cfg->bits == 3 || cfg->bits == 4 || cfg->bits == 8))
+        return fail(GPTQ_ERR_INVALID_ARG, "bits must be 2, 3, 4 or 8");
+    if (!qweight || !scales || !W_hat) return fail(GPTQ_ERR_INVALID_ARG, "qweight, scales and W_hat must be non-NULL");
+    if (cfg->sym ? (qzeros != nullptr) : (qzeros == nullptr))
+        return fail(GPTQ_ERR_INVALID_ARG, "qzeros must be given iff asymmetric");
+    if (d_out < 1 || d_in < 1) return fail(GPTQ_ERR_INVALID_ARG, "d_out and d_in must be >= 1");
+    const int g = cfg->group_size < 0 ? (int)d_in : cfg->group_size;
+    if (g < 1) return fail(GPTQ_ERR_INVALID_ARG, "group_size must be -1 or >= 1");
+    const long long total = d_out * d_in;
+    {
+        gqh::TimedScope ts__("dequant", (cudaStream_t)stream);
+        gq::dequant_kernel<<<(unsigned)std::min<long long>((total + 255) / 256, 16384), 256, 0, (cudaStream_t)stream>>>(
+            qweight, reinterpret_cast<const __half*>(scales), qzeros, d_out, d_in, cfg->bits, g, cfg->sym, W_hat);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "dequant");
+    return GPTQ_OK;
+}
+
+gptq_status gptq_sync_status(void* stream) { return read_status((cudaStream_t)stream, nullptr); }
+
+void gptq_timing_enable(int on) { g_timing = on != 0; }
+
+size_t gptq_timing_report(char* buf, size_t len) {
+    timing_collect();
+    std::string out = "{";
+    bool first = true;
+    for (auto& kv : g_timing_acc) {
+        char item[256];
+        snprintf(item, sizeof(item), "%s\"%s\": [%lld, %.6f]", first ? "" : ", ", kv.first.c_str(),
+                 kv.second.first, kv.second.second);
+        out += item;
+        first = false;
+    }
+    out += "}";
+    g_timing_acc.clear();
+    if (buf && len) {
+        const size_t n = std::min(len - 1, out.size());
+        memcpy(buf, out.data(), n);
+        buf[n] = 0;
+    }
+    return out.size() + 1;
+}
+
+gptq_status gptq_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
+    if (limit_ns > 10000000000ull) return fail(GPTQ_ERR_INVALID_ARG, "limit_ns must be <= 10 s");
+    {
+        TimedScope ts__("selftest_wait", (cudaStream_t)stream);
+        gq::selftest_wait_kernel<<<1, 1, 0, (cudaStream_t)stream>>>((unsigned long long)limit_ns);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "selftest_bounded_wait");
+    return GPTQ_OK;
+}
+
+}  // extern "C"

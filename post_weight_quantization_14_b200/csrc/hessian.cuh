@@ -1,0 +1,98 @@
+// H (+)= 2 X^T X on the tensor cores (tutorial "阶段一", H = 2 X^T X).
+// X (n x d_in, row-major) is first transposed to X^T (d_in x n_pad, zero padded) so
+// both GEMM operands are K-major; for fp32 X the transpose also splits each value
+// into two tf32 parts for the 3xTF32 product.  Only tiles on or above the diagonal
+// are computed; each off-diagonal tile is also written to its mirror position.
+#pragma once
+#include "gemm_tc.cuh"
+
+namespace gq {
+
+constexpr int kHessNPad = 64;
+
+// 32x32 tiled transpose: XT[c, t] = X[t, c] for t < n, 0 for n <= t < n_pad.
+__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ X, long long n, long long d_in,
+                                      long long n_pad, uint16_t* __restrict__ XT) {
+    __shared__ uint16_t tile[32][33];
+    const long long t0 = (long long)blockIdx.x * 32, c0 = (long long)blockIdx.y * 32;
+    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+        const long long t = t0 + r, c = c0 + threadIdx.x;
+        tile[r][threadIdx.x] = (t < n && c < d_in) ? X[t * d_in + c] : (uint16_t)0;
+    }
+    __syncthreads();
+    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+        const long long c = c0 + r, t = t0 + threadIdx.x;
+        if (c < d_in && t < n_pad) XT[c * n_pad + t] = tile[threadIdx.x][r];
+    }
+}
+
+__global__ void transpose_split_f32_kernel(const float* __restrict__ X, long long n, long long d_in,
+                                           long long n_pad, float* __restrict__ XT_hi,
+                                           float* __restrict__ XT_lo) {
+    __shared__ float tile[32][33];
+    const long long t0 = (long long)blockIdx.x * 32, c0 = (long long)blockIdx.y * 32;
+    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+        const long long t = t0 + r, c = c0 + threadIdx.x;
+        tile[r][threadIdx.x] = (t < n && c < d_in) ? X[t * d_in + c] : 0.f;
+    }
+    __syncthreads();
+    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+        const long long c = c0 + r, t = t0 + threadIdx.x;
+        if (c < d_in && t < n_pad) {
+            float hi, lo;
+            split_tf32(tile[threadIdx.x][r], hi, lo);
+            XT_hi[c * n_pad + t] = hi;
+            XT_lo[c * n_pad + t] = lo;
+        }
+    }
+}
+
+}  // namespace gq
+
+namespace gqh {
+
+inline long long hess_npad(long long n) { return (n + gq::kHessNPad - 1) / gq::kHessNPad * gq::kHessNPad; }
+
+inline size_t hessian_ws_bytes(long long n, long long d_in, gptq_dtype xt) {
+    const long long np = hess_npad(n);
+    return xt == GPTQ_BF16 ? (size_t)(d_in * np * 2) : (size_t)(2 * d_in * np * 4);
+}
+
+inline cudaError_t hessian_run(const void* X, gptq_dtype xt, long long n, long long d_in, float* H,
+                               int accumulate, void* ws, cudaStream_t st) {
+    const long long np = hess_npad(n);
+    dim3 tb(32, 8);
+    dim3 grid((unsigned)(np / 32), (unsigned)((d_in + 31) / 32));
+    gq::GemmArgs p = gemm_args((int)d_in, (int)d_in, (int)np);
+    p.triangular = 1;
+    p.mirror = 1;
+    p.alpha = 2.f;
+    p.beta = accumulate ? 1.f : 0.f;
+    p.C = H;
+    p.ldc = d_in;
+    p.write_c = 1;
+    if (xt == GPTQ_BF16) {
+        uint16_t* XT = static_cast<uint16_t*>(ws);
+        {
+            gqh::TimedScope ts__("transpose_x", st);
+            gq::transpose_bf16_kernel<<<grid, tb, 0, st>>>(static_cast<const uint16_t*>(X), n, d_in, np, XT);
+        }
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        Mat m{XT, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
+        return launch_gemm<gq::KIND_BF16, 128, 6>(m, m, m, m, p, 1, st, "hessian_syrk");
+    }
+    float* hi = static_cast<float*>(ws);
+    float* lo = hi + d_in * np;
+    {
+        gqh::TimedScope ts__("transpose_x", st);
+        gq::transpose_split_f32_kernel<<<grid, tb, 0, st>>>(static_cast<const float*>(X), n, d_in, np, hi, lo);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    Mat mh{hi, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
+    Mat ml{lo, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
+    return launch_gemm<gq::KIND_TF32X3, 128, 3>(mh, ml, mh, ml, p, 1, st, "hessian_syrk");
+}
+
+}  // namespace gqh

@@ -1,0 +1,252 @@
+"""Thin ctypes binding of the C ABI in include/gptq_b200.h.
+
+Argument marshalling only: every computation runs in the CUDA kernels of
+``libgptq_b200.so``.  PyTorch supplies device memory and the current stream.
+The functions keep the C names; ``quantize_layer`` chains the three stages for
+one linear layer (the call a user makes).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgptq_b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "gptq_b200.h")
+
+GPTQ_OK = 0
+GPTQ_ERR_INVALID_ARG = 1
+GPTQ_ERR_UNSUPPORTED = 2
+GPTQ_ERR_NOT_PD = 3
+GPTQ_ERR_NONFINITE = 4
+GPTQ_ERR_CUDA = 5
+GPTQ_ERR_TIMEOUT = 6
+GPTQ_ERR_WORKSPACE = 7
+
+GPTQ_BF16 = 0
+GPTQ_F32 = 1
+
+
+class GptqConfig(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int), ("group_size", ctypes.c_int), ("sym", ctypes.c_int),
+                ("block_size", ctypes.c_int), ("damp_rel", ctypes.c_float), ("desc_act", ctypes.c_int)]
+
+
+class GPTQError(RuntimeError):
+    def __init__(self, status: int, msg: str, index: int | None = None):
+        super().__init__(f"{msg} (status {status})")
+        self.status = status
+        self.index = index
+
+
+_lib = None
+_vp, _i64, _sz, _int, _f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
+
+_SIGS = {
+    "gptq_default_config": (None, [ctypes.POINTER(GptqConfig)]),
+    "gptq_status_string": (ctypes.c_char_p, [_int]),
+    "gptq_last_error": (ctypes.c_char_p, []),
+    "gptq_version": (_int, []),
+    "gptq_hessian_workspace_bytes": (_sz, [_i64, _i64, _int]),
+    "gptq_hessian_accumulate": (_int, [_vp, _int, _i64, _i64, _vp, _int, _vp, _sz, _vp]),
+    "gptq_prepare_hinv_workspace_bytes": (_sz, [_i64]),
+    "gptq_prepare_hinv": (_int, [_vp, _i64, _f32, _vp, _vp, _sz, ctypes.POINTER(_i64),
+                                 ctypes.POINTER(_f32), _vp]),
+    "gptq_quantize_workspace_bytes": (_sz, [_i64, _i64, ctypes.POINTER(GptqConfig)]),
+    "gptq_quantize_layer": (_int, [_vp, _vp, _i64, _i64, ctypes.POINTER(GptqConfig), _vp, _vp, _vp, _vp,
+                                   _vp, _sz, _vp]),
+    "gptq_pack_int": (_int, [_vp, _i64, _i64, _int, _int, _vp, _vp]),
+    "gptq_dequant": (_int, [_vp, _vp, _vp, _i64, _i64, ctypes.POINTER(GptqConfig), _vp, _vp]),
+    "gptq_sync_status": (_int, [_vp]),
+    "gptq_timing_enable": (None, [_int]),
+    "gptq_timing_report": (_sz, [ctypes.c_char_p, _sz]),
+    "gptq_selftest_bounded_wait": (_int, [ctypes.c_uint64, _vp]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgptq_b200.so (fails loudly when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with python -m post_weight_quantization_14_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions declared in include/gptq_b200.h."""
+    text = open(HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gptq_[a-z0-9_]+)\s*\(", text)))
+
+
+def make_config(bits=4, group_size=128, sym=False, block_size=128, damp_rel=0.01, desc_act=False) -> GptqConfig:
+    c = GptqConfig()
+    lib().gptq_default_config(ctypes.byref(c))
+    c.bits, c.group_size, c.sym, c.block_size = int(bits), int(group_size), int(bool(sym)), int(block_size)
+    c.damp_rel, c.desc_act = float(damp_rel), int(bool(desc_act))
+    return c
+
+
+def _check(status: int, index: int | None = None) -> None:
+    if status != GPTQ_OK:
+        msg = lib().gptq_last_error().decode()
+        raise GPTQError(status, msg or lib().gptq_status_string(status).decode(), index)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream or None
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------------------- stage wrappers
+
+def gptq_hessian_accumulate(X: torch.Tensor, H: torch.Tensor, accumulate: bool = False,
+                            workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """H (+)= 2 X^T X.  X: [n, d_in] bfloat16 or float32 on the device; H: [d_in, d_in] float32."""
+    n, d_in = X.shape
+    if X.dtype == torch.bfloat16:
+        xt = GPTQ_BF16
+    elif X.dtype == torch.float32:
+        xt = GPTQ_F32
+    else:
+        raise ValueError("X must be bfloat16 or float32")
+    if H.dtype != torch.float32 or tuple(H.shape) != (d_in, d_in):
+        raise ValueError("H must be float32 [d_in, d_in]")
+    need = lib().gptq_hessian_workspace_bytes(n, d_in, xt)
+    ws = workspace if workspace is not None else _workspace(need, X.device)
+    _check(lib().gptq_hessian_accumulate(_ptr(X), xt, n, d_in, _ptr(H), int(bool(accumulate)),
+                                         _ptr(ws), ws.numel(), _stream(stream)))
+    return H
+
+
+def gptq_prepare_hinv(H: torch.Tensor, U: torch.Tensor, damp_rel: float = 0.01,
+                      workspace: torch.Tensor | None = None, stream=None) -> float:
+    """U = upper Cholesky factor of (H + lambda I)^-1; returns lambda.  Synchronises the stream."""
+    d = H.shape[0]
+    need = lib().gptq_prepare_hinv_workspace_bytes(d)
+    ws = workspace if workspace is not None else _workspace(need, H.device)
+    bad = _i64(-1)
+    lam = _f32(0.0)
+    st = lib().gptq_prepare_hinv(_ptr(H), d, float(damp_rel), _ptr(U), _ptr(ws), ws.numel(),
+                                 ctypes.byref(bad), ctypes.byref(lam), _stream(stream))
+    _check(st, bad.value)
+    return float(lam.value)
+
+
+def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, cfg: GptqConfig, qweight: torch.Tensor,
+                        scales: torch.Tensor, qzeros: torch.Tensor | None, err_sq: torch.Tensor | None = None,
+                        workspace: torch.Tensor | None = None, stream=None) -> None:
+    """Column loop; W is consumed as scratch.  scales is a float16 tensor [n_groups, d_out]."""
+    d_out, d_in = W.shape
+    need = lib().gptq_quantize_workspace_bytes(d_out, d_in, ctypes.byref(cfg))
+    ws = workspace if workspace is not None else _workspace(need, W.device)
+    _check(lib().gptq_quantize_layer(_ptr(W), _ptr(U), d_out, d_in, ctypes.byref(cfg), _ptr(qweight),
+                                     _ptr(scales), _ptr(qzeros), _ptr(err_sq), _ptr(ws), ws.numel(),
+                                     _stream(stream)))
+
+
+def gptq_pack_int(codes: torch.Tensor, bits: int, layout: int, packed: torch.Tensor, stream=None) -> torch.Tensor:
+    rows, cols = codes.shape
+    _check(lib().gptq_pack_int(_ptr(codes), rows, cols, int(bits), int(layout), _ptr(packed), _stream(stream)))
+    return packed
+
+
+def gptq_dequant(qweight, scales, qzeros, d_out: int, d_in: int, cfg: GptqConfig, W_hat: torch.Tensor,
+                 stream=None) -> torch.Tensor:
+    _check(lib().gptq_dequant(_ptr(qweight), _ptr(scales), _ptr(qzeros), d_out, d_in, ctypes.byref(cfg),
+                              _ptr(W_hat), _stream(stream)))
+    return W_hat
+
+
+def gptq_sync_status(stream=None) -> None:
+    _check(lib().gptq_sync_status(_stream(stream)))
+
+
+def gptq_timing_enable(on: bool = True) -> None:
+    lib().gptq_timing_enable(int(bool(on)))
+
+
+def gptq_timing_report() -> dict:
+    """{kernel: (launches, total_ms)} since the last report (synchronises the device)."""
+    import json
+    n = lib().gptq_timing_report(None, 0)
+    buf = ctypes.create_string_buffer(n + 16)
+    lib().gptq_timing_report(buf, len(buf))
+    return {k: (int(v[0]), float(v[1])) for k, v in json.loads(buf.value.decode()).items()}
+
+
+def gptq_selftest_bounded_wait(limit_ns: int, stream=None) -> None:
+    _check(lib().gptq_selftest_bounded_wait(int(limit_ns), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------- whole layer
+
+def n_groups(d_in: int, group_size: int) -> int:
+    return 1 if group_size == -1 else (d_in + group_size - 1) // group_size
+
+
+@dataclass
+class QuantizedLayer:
+    qweight: torch.Tensor      # int32 [ceil(d_in*bits/32), d_out]
+    scales: torch.Tensor       # float16 [n_groups, d_out]
+    qzeros: torch.Tensor | None  # int32 [n_groups, ceil(d_out*bits/32)] (None if sym)
+    err_sq: torch.Tensor       # float32 [d_out]
+    lam: float
+
+
+class LayerBuffers:
+    """Device buffers for one layer shape, reusable across calls (no allocation per call)."""
+
+    def __init__(self, d_out: int, d_in: int, n: int, x_dtype: torch.dtype, cfg: GptqConfig, device):
+        xt = GPTQ_BF16 if x_dtype == torch.bfloat16 else GPTQ_F32
+        L = lib()
+        self.cfg = cfg
+        self.H = torch.empty((d_in, d_in), dtype=torch.float32, device=device)
+        self.U = torch.empty((d_in, d_in), dtype=torch.float32, device=device)
+        ws = max(L.gptq_hessian_workspace_bytes(n, d_in, xt), L.gptq_prepare_hinv_workspace_bytes(d_in),
+                 L.gptq_quantize_workspace_bytes(d_out, d_in, ctypes.byref(cfg)))
+        self.ws = _workspace(ws, device)
+        ng = n_groups(d_in, cfg.group_size)
+        self.qweight = torch.empty(((d_in * cfg.bits + 31) // 32, d_out), dtype=torch.int32, device=device)
+        self.scales = torch.empty((ng, d_out), dtype=torch.float16, device=device)
+        self.qzeros = None if cfg.sym else torch.empty((ng, (d_out * cfg.bits + 31) // 32), dtype=torch.int32,
+                                                      device=device)
+        self.err_sq = torch.empty((d_out,), dtype=torch.float32, device=device)
+
+
+def quantize_layer(W: torch.Tensor, X: torch.Tensor, bits=4, group_size=128, sym=False, damp_rel=0.01,
+                   buffers: LayerBuffers | None = None, stream=None) -> QuantizedLayer:
+    """GPTQ of one linear layer: H = 2 X^T X, U = chol(Hd^-1) upper, column loop.  W is overwritten."""
+    cfg = buffers.cfg if buffers is not None else make_config(bits, group_size, sym, 128, damp_rel)
+    d_out, d_in = W.shape
+    b = buffers or LayerBuffers(d_out, d_in, X.shape[0], X.dtype, cfg, W.device)
+    gptq_hessian_accumulate(X, b.H, accumulate=False, workspace=b.ws, stream=stream)
+    lam = gptq_prepare_hinv(b.H, b.U, cfg.damp_rel, workspace=b.ws, stream=stream)
+    gptq_quantize_layer(W, b.U, cfg, b.qweight, b.scales, b.qzeros, b.err_sq, workspace=b.ws, stream=stream)
+    return QuantizedLayer(b.qweight, b.scales, b.qzeros, b.err_sq, lam)

@@ -1,0 +1,119 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, every function
+declared in include/gptq_b200.h is exported, and argument validation rejects bad
+calls before anything is enqueued."""
+
+import ctypes
+
+import pytest
+
+from post_weight_quantization_14_b200 import gptq as G
+
+
+def test_library_exports_every_declared_function():
+    L = G.lib()
+    names = G.header_functions()
+    assert len(names) >= 16
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+    # every declared function has a ctypes signature in the binding
+    assert set(names) <= set(G._SIGS)
+
+
+def test_default_config_and_strings():
+    c = G.make_config()
+    assert (c.bits, c.group_size, c.sym, c.block_size, c.desc_act) == (4, 128, 0, 128, 0)
+    assert c.damp_rel == pytest.approx(0.01)
+    L = G.lib()
+    assert L.gptq_status_string(G.GPTQ_ERR_NOT_PD) == b"GPTQ_ERR_NOT_PD"
+    assert L.gptq_status_string(99) == b"GPTQ_ERR_UNKNOWN"
+    assert L.gptq_version() >= 100
+
+
+def test_workspace_queries_are_positive_and_grow():
+    L = G.lib()
+    c = G.make_config()
+    small = L.gptq_quantize_workspace_bytes(256, 256, ctypes.byref(c))
+    big = L.gptq_quantize_workspace_bytes(4096, 4096, ctypes.byref(c))
+    assert 0 < small < big
+    assert L.gptq_prepare_hinv_workspace_bytes(200) > 200 * 200 * 4
+    assert L.gptq_hessian_workspace_bytes(100, 64, G.GPTQ_BF16) >= 64 * 128 * 2
+    assert L.gptq_hessian_workspace_bytes(100, 64, G.GPTQ_F32) >= 2 * 64 * 128 * 4
+    assert L.gptq_hessian_workspace_bytes(0, 64, G.GPTQ_F32) == 0
+
+
+def _fake(n=1):
+    # host addresses are never dereferenced: validation fails before any CUDA call
+    return ctypes.c_void_p(0x1000 * n)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("bits", 5, G.GPTQ_ERR_INVALID_ARG),
+    ("bits", 1, G.GPTQ_ERR_INVALID_ARG),
+    ("group_size", 48, G.GPTQ_ERR_INVALID_ARG),
+    ("group_size", 8, G.GPTQ_ERR_INVALID_ARG),
+    ("group_size", 256, G.GPTQ_ERR_INVALID_ARG),
+    ("block_size", 64, G.GPTQ_ERR_INVALID_ARG),
+    ("sym", 2, G.GPTQ_ERR_INVALID_ARG),
+    ("desc_act", 1, G.GPTQ_ERR_UNSUPPORTED),
+    ("damp_rel", -1.0, G.GPTQ_ERR_INVALID_ARG),
+    ("damp_rel", float("nan"), G.GPTQ_ERR_INVALID_ARG),
+])
+def test_quantize_rejects_bad_config(field, value, status):
+    c = G.make_config()
+    setattr(c, field, value)
+    L = G.lib()
+    st = L.gptq_quantize_layer(_fake(1), _fake(2), 64, 64, ctypes.byref(c), _fake(3), _fake(4), _fake(5),
+                               None, _fake(6), 1 << 30, None)
+    assert st == status
+    assert L.gptq_last_error()
+
+
+def test_quantize_rejects_bad_shapes_and_pointers():
+    L = G.lib()
+    c = G.make_config()
+    args = lambda W, d_out, d_in, qz: L.gptq_quantize_layer(W, _fake(2), d_out, d_in, ctypes.byref(c), _fake(3),
+                                                            _fake(4), qz, None, _fake(6), 1 << 40, None)
+    assert args(None, 64, 64, _fake(5)) == G.GPTQ_ERR_INVALID_ARG
+    assert args(_fake(1), 64, 60, _fake(5)) == G.GPTQ_ERR_INVALID_ARG      # d_in % 8
+    assert args(_fake(1), 0, 64, _fake(5)) == G.GPTQ_ERR_INVALID_ARG
+    assert args(_fake(1), 64, 64, None) == G.GPTQ_ERR_INVALID_ARG          # asym needs qzeros
+    c.sym = 1
+    assert args(_fake(1), 64, 64, _fake(5)) == G.GPTQ_ERR_INVALID_ARG      # sym forbids qzeros
+    # workspace too small
+    c.sym = 0
+    st = L.gptq_quantize_layer(_fake(1), _fake(2), 64, 64, ctypes.byref(c), _fake(3), _fake(4), _fake(5), None,
+                               _fake(6), 16, None)
+    assert st == G.GPTQ_ERR_WORKSPACE
+
+
+def test_hessian_and_hinv_reject_bad_args():
+    L = G.lib()
+    assert L.gptq_hessian_accumulate(None, 0, 10, 64, _fake(2), 0, _fake(3), 1 << 30, None) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_hessian_accumulate(_fake(1), 7, 10, 64, _fake(2), 0, _fake(3), 1 << 30, None) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_hessian_accumulate(_fake(1), 0, 10, 66, _fake(2), 0, _fake(3), 1 << 30, None) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_hessian_accumulate(_fake(1), 0, 10, 64, _fake(2), 0, _fake(3), 8, None) == G.GPTQ_ERR_WORKSPACE
+    bad = ctypes.c_int64(0)
+    lam = ctypes.c_float(0)
+    assert L.gptq_prepare_hinv(None, 64, 0.01, _fake(2), _fake(3), 1 << 30, ctypes.byref(bad), ctypes.byref(lam),
+                               None) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_prepare_hinv(_fake(1), 64, -0.5, _fake(2), _fake(3), 1 << 30, None, None,
+                               None) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_prepare_hinv(_fake(1), 64, 0.01, _fake(2), _fake(3), 64, None, None, None) == G.GPTQ_ERR_WORKSPACE
+
+
+def test_pack_and_dequant_reject_bad_args():
+    L = G.lib()
+    assert L.gptq_pack_int(_fake(1), 4, 8, 5, 0, _fake(2), None) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_pack_int(_fake(1), 4, 8, 4, 2, _fake(2), None) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_pack_int(_fake(1), 0, 8, 4, 0, _fake(2), None) == G.GPTQ_ERR_INVALID_ARG
+    c = G.make_config(sym=True)
+    assert L.gptq_dequant(_fake(1), _fake(2), _fake(3), 4, 8, ctypes.byref(c), _fake(4), None) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_selftest_bounded_wait(10 ** 12, None) == G.GPTQ_ERR_INVALID_ARG
+
+
+def test_product_path_has_no_cpu_fallback():
+    # the binding refuses host tensors instead of computing on the CPU
+    import torch
+    W = torch.zeros(8, 8)
+    with pytest.raises(ValueError):
+        G._ptr(W)
