@@ -164,8 +164,8 @@ gptq_status gptq_sync_status(void* stream);
  * gptq_timing_enable(1): every kernel launch of the library is bracketed by CUDA
  * events on its stream.  gptq_timing_report() synchronises the device, writes a JSON
  * object {"kernel_name": [launches, total_ms], ...} of everything recorded since the
- * last report into buf (NUL-terminated, truncated to len) and returns the number of
- * bytes needed.  Host-side bookkeeping only; not thread-safe.
+ * last report into buf (NUL-terminated, truncated to len), clears the totals and
+ * returns the number of bytes needed; with buf == NULL it only returns that size.  Host-side bookkeeping only; not thread-safe.
  *
  * gptq_selftest_bounded_wait: launches one thread that waits on a barrier nobody
  * arrives at, with a limit of limit_ns nanoseconds, the same bounded wait every

@@ -92,14 +92,28 @@ __global__ void zero_lower_blocks_kernel(float* __restrict__ U, long long d) {
 }
 
 // Leaf: factor and invert one 128x128 diagonal block of A in shared memory.
-// Writes X = R_jj^-1 (upper, zeros below the diagonal) to the public U (clipped to
-// d), its row-major tf32 split (U_hi/U_lo) and its transposed split (UT_hi/UT_lo).
+// Works on the index-reversed block P = J A_jj J, for which the UL factor becomes an
+// ordinary lower Cholesky factor: A_jj = R R^T with R = J L J, and X_jj = R^-1 = J L^-1 J.
+// Blocked by 32.  For each diagonal 32-block one warp runs Gaussian elimination on
+// [P_kk | I] with unscaled pivot rows (lane = row): afterwards L_kk = L_u D^1/2 and
+// L_kk^-1 = D^-1/2 E, where E is the accumulated row-operation matrix.  All warps then
+// form the panel L_rk = P_rk L_kk^-T and the rank-32 update of the trailing lower
+// triangle, on 4x4 register micro-tiles fed from transposed copies of L and of the
+// diagonal inverses.  The inverse is assembled along block diagonals:
+// X_ij = -X_ii sum_{k=j}^{i-1} L_ik X_kj.
+// Writes X_jj (upper, zeros below the diagonal) to the public U (clipped to d), its
+// row-major tf32 split (U_hi/U_lo) and its transposed split (UT_hi/UT_lo).
+constexpr int LS = NB + 4;   // leaf smem row stride (16-byte aligned rows)
+
 struct LeafSmem {
-    float a[NB][NB + 1];
-    float u[NB][NB + 1];
-    float xinv[4][32][33];
-    float tmp[3][32][33];
+    float P[NB][LS];         // reversed block; lower triangle holds L after the factorization
+    float X[NB][LS];         // L^-1 (lower); upper blocks hold temporaries
+    float LT[NB][LS];        // L transposed: LT[m][r] = L[r][m]
+    float XDT[4][32][36];    // diagonal inverses transposed: XDT[kb][m][j] = X_kk[j][m]
+    float rowbuf[2][64];     // broadcast of the current pivot row (p part, x part)
 };
+
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
 __global__ void __launch_bounds__(512, 1)
     chol_leaf_kernel(const float* __restrict__ A, long long n, long long d, int jb, float* __restrict__ U,
@@ -110,133 +124,222 @@ __global__ void __launch_bounds__(512, 1)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr unsigned FULL = 0xffffffffu;
 
+    // P[127-r][127-c] = A[r][c]: coalesced reads of the whole diagonal tile (both
+    // triangles were updated); only P's lower triangle (A's upper) is used.
     for (int e = tid; e < NB * NB; e += blockDim.x) {
         const int r = e >> 7, c = e & 127;
-        S.a[r][c] = A[(long long)(jb + r) * n + jb + c];
-        S.u[r][c] = 0.f;
+        S.P[127 - r][127 - c] = A[(long long)(jb + r) * n + jb + c];
+        S.X[r][c] = 0.f;
     }
     __syncthreads();
 
-    for (int kb = 3; kb >= 0; --kb) {
-        const int rb = kb * 32;
+    for (int kb = 0; kb < 4; ++kb) {
+        const int k0 = kb * 32;
         if (warp == 0) {
-            // (a) UL-Cholesky of the 32x32 diagonal block, lane = row
-            float dv[32];
+            // (a) elimination of [P_kk | I] with unscaled pivot rows; lane = row
+            float pr[32], xr[32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) dv[c] = (c >= lane) ? S.a[rb + lane][rb + c] : 0.f;
+            for (int j = 0; j < 32; ++j) {
+                pr[j] = (j <= lane) ? S.P[k0 + lane][k0 + j] : S.P[k0 + j][k0 + lane];
+                xr[j] = (j == lane) ? 1.f : 0.f;
+            }
+            float my_rinv = 0.f;
 #pragma unroll
-            for (int k = 31; k >= 0; --k) {
-                const float piv = __shfl_sync(FULL, dv[k], k);
+            for (int k = 0; k < 32; ++k) {
+                const float piv = __shfl_sync(FULL, pr[k], k);
                 if (lane == 0 && !(piv > 0.f && isfinite(piv)))
-                    record_status(isfinite(piv) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE, jb + rb + k);
-                const float sq = sqrtf(piv);
-                const float rk = (lane < k) ? dv[k] / sq : ((lane == k) ? sq : 0.f);
-                dv[k] = rk;
+                    record_status(isfinite(piv) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE, jb + 127 - (k0 + k));
+                const float rinv = rsqrtf(piv);
+                float* rb = S.rowbuf[k & 1];
+                if (lane == k) {
+                    my_rinv = rinv;
 #pragma unroll
-                for (int c = 0; c < k; ++c) dv[c] -= rk * __shfl_sync(FULL, rk, c);
+                    for (int q = 0; q < 8; ++q) {
+                        if (4 * q + 3 > k)
+                            *reinterpret_cast<float4*>(rb + 4 * q) =
+                                make_float4(pr[4 * q], pr[4 * q + 1], pr[4 * q + 2], pr[4 * q + 3]);
+                        if (4 * q <= k)
+                            *reinterpret_cast<float4*>(rb + 32 + 4 * q) =
+                                make_float4(xr[4 * q], xr[4 * q + 1], xr[4 * q + 2], xr[4 * q + 3]);
+                    }
+                }
+                __syncwarp();
+                if (lane > k) {
+                    const float f = pr[k] * rinv * rinv;   // P_ik / P_kk
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        if (4 * q + 3 > k) {
+                            const float4 v = ld4(rb + 4 * q);
+                            if (4 * q + 0 > k) pr[4 * q + 0] = fmaf(-f, v.x, pr[4 * q + 0]);
+                            if (4 * q + 1 > k) pr[4 * q + 1] = fmaf(-f, v.y, pr[4 * q + 1]);
+                            if (4 * q + 2 > k) pr[4 * q + 2] = fmaf(-f, v.z, pr[4 * q + 2]);
+                            pr[4 * q + 3] = fmaf(-f, v.w, pr[4 * q + 3]);
+                        }
+                        if (4 * q <= k) {
+                            const float4 v = ld4(rb + 32 + 4 * q);
+                            xr[4 * q + 0] = fmaf(-f, v.x, xr[4 * q + 0]);
+                            if (4 * q + 1 <= k) xr[4 * q + 1] = fmaf(-f, v.y, xr[4 * q + 1]);
+                            if (4 * q + 2 <= k) xr[4 * q + 2] = fmaf(-f, v.z, xr[4 * q + 2]);
+                            if (4 * q + 3 <= k) xr[4 * q + 3] = fmaf(-f, v.w, xr[4 * q + 3]);
+                        }
+                    }
+                    pr[k] *= rinv;   // L[lane][k] = P_ik / sqrt(P_kk)
+                }
             }
+            // lane i: L[i][j] = pr[j] (j < i), L[i][i] = pivot * rinv, row i of L^-1 = rinv * xr
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-                if (c >= lane) S.a[rb + lane][rb + c] = dv[c];
+            for (int j = 0; j < 32; ++j) {
+                if (j <= lane) {
+                    const float lij = (j == lane) ? pr[j] * my_rinv : pr[j];
+                    const float xij = xr[j] * my_rinv;
+                    S.P[k0 + lane][k0 + j] = lij;
+                    S.LT[k0 + j][k0 + lane] = lij;
+                    S.X[k0 + lane][k0 + j] = xij;
+                    S.XDT[kb][j][lane] = xij;
+                } else {
+                    S.XDT[kb][j][lane] = 0.f;
+                }
+            }
+        }
+        __syncthreads();
+        if (kb == 3) break;
+        const int t0 = k0 + 32;
+        const int rows = NB - t0;
+        // (b) panel: L[r][k0+j] = sum_m P[r][k0+m] X_kk[j][m]; task = (row, 4 columns)
+        for (int base = 0; base < rows * 8; base += 512) {
+            const int task = base + tid;
+            const int r = t0 + (task >> 3), j4 = (task & 7) * 4;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (task < rows * 8) {
+#pragma unroll 8
+                for (int m = 0; m < 32; ++m) {
+                    const float pv = S.P[r][k0 + m];
+                    const float4 xv = ld4(&S.XDT[kb][m][j4]);
+                    acc.x = fmaf(pv, xv.x, acc.x);
+                    acc.y = fmaf(pv, xv.y, acc.y);
+                    acc.z = fmaf(pv, xv.z, acc.z);
+                    acc.w = fmaf(pv, xv.w, acc.w);
+                }
+            }
             __syncwarp();
-            // (b) X = R^-1 of the 32x32 block, lane = column, back substitution from the bottom
-            float xv[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) xv[i] = 0.f;
-#pragma unroll
-            for (int i = 31; i >= 0; --i) {
-                float s = 0.f;
-#pragma unroll
-                for (int m = i + 1; m < 32; ++m) s = fmaf(S.a[rb + i][rb + m], xv[m], s);
-                const float rii = S.a[rb + i][rb + i];
-                xv[i] = (i == lane) ? 1.f / rii : ((i < lane) ? -s / rii : 0.f);
-            }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) S.xinv[kb][i][lane] = xv[i];
-        }
-        __syncthreads();
-        if (kb == 0) break;
-        // (c) panel: R[0:rb, rb:rb+32] = A[0:rb, rb:rb+32] X^T
-        float pv[6];
-#pragma unroll
-        for (int it = 0; it < 6; ++it) {
-            const int e = tid + it * 512;
-            pv[it] = 0.f;
-            if (e < rb * 32) {
-                const int r = e >> 5, c = e & 31;
-                float s = 0.f;
-#pragma unroll
-                for (int k = 0; k < 32; ++k) s = fmaf(S.a[r][rb + k], S.xinv[kb][c][k], s);
-                pv[it] = s;
+            if (task < rows * 8) {
+                *reinterpret_cast<float4*>(&S.P[r][k0 + j4]) = acc;
+                S.LT[k0 + j4 + 0][r] = acc.x;
+                S.LT[k0 + j4 + 1][r] = acc.y;
+                S.LT[k0 + j4 + 2][r] = acc.z;
+                S.LT[k0 + j4 + 3][r] = acc.w;
             }
         }
         __syncthreads();
+        // (c) trailing update of the lower triangle on 4x4 micro-tiles
+        {
+            const int T = rows >> 2;
+            for (int task = tid; task < T * T; task += blockDim.x) {
+                const int tr = task / T, tc = task % T;
+                if (tc > tr) continue;
+                const int r0 = t0 + 4 * tr, c0 = t0 + 4 * tc;
+                float acc[4][4] = {};
+#pragma unroll 4
+                for (int m = 0; m < 32; ++m) {
+                    const float4 a = ld4(&S.LT[k0 + m][r0]);
+                    const float4 b = ld4(&S.LT[k0 + m][c0]);
+                    const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int it = 0; it < 6; ++it) {
-            const int e = tid + it * 512;
-            if (e < rb * 32) S.a[e >> 5][rb + (e & 31)] = pv[it];
-        }
-        __syncthreads();
-        // (d) A[0:rb, 0:rb] -= P P^T on the upper triangle
-        for (int e = tid; e < rb * rb; e += blockDim.x) {
-            const int r = e / rb, c = e % rb;
-            if (r > c) continue;
-            float s = 0.f;
+                    for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int k = 0; k < 32; ++k) s = fmaf(S.a[r][rb + k], S.a[c][rb + k], s);
-            S.a[r][c] -= s;
+                        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float4 pv = ld4(&S.P[r0 + i][c0]);
+                    pv.x -= acc[i][0];
+                    pv.y -= acc[i][1];
+                    pv.z -= acc[i][2];
+                    pv.w -= acc[i][3];
+                    *reinterpret_cast<float4*>(&S.P[r0 + i][c0]) = pv;
+                }
+            }
         }
         __syncthreads();
     }
 
-    // inverse of the 128x128 R from the four 32-block inverses
-    for (int e = tid; e < 4 * 1024; e += blockDim.x) {
-        const int kb = e >> 10, i = (e >> 5) & 31, j = e & 31;
-        S.u[kb * 32 + i][kb * 32 + j] = S.xinv[kb][i][j];
-    }
-    __syncthreads();
-    for (int ib = 2; ib >= 0; --ib) {
-        const int nj = 3 - ib;  // block columns ib+1 .. 3
-        for (int e = tid; e < nj * 1024; e += blockDim.x) {
-            const int jj = e >> 10, r = (e >> 5) & 31, c = e & 31;
-            const int jb2 = ib + 1 + jj;
-            float s = 0.f;
-            for (int kb2 = ib + 1; kb2 <= jb2; ++kb2) {
-#pragma unroll 8
-                for (int m = 0; m < 32; ++m)
-                    s = fmaf(S.a[ib * 32 + r][kb2 * 32 + m], S.u[kb2 * 32 + m][jb2 * 32 + c], s);
+    // inverse blocks below the diagonal, by block diagonals dd = i - j, 4x4 micro-tiles
+    for (int dd = 1; dd < 4; ++dd) {
+        const int nblk = 4 - dd;
+        for (int task = tid; task < nblk * 64; task += blockDim.x) {
+            // T_ij = sum_{m'=32j}^{32i-1} L[32i+r][m'] X[m'][32j+c] -> stored in X[32j+r][32i+c]
+            const int jbk = task >> 6, ib = jbk + dd, tr = (task >> 3) & 7, tc = task & 7;
+            const int r0 = 4 * tr, c0 = 4 * tc;
+            float acc[4][4] = {};
+            for (int m = 32 * jbk; m < 32 * ib; ++m) {
+                const float4 a = ld4(&S.LT[m][32 * ib + r0]);
+                const float4 b = ld4(&S.X[m][32 * jbk + c0]);
+                const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
             }
-            S.tmp[jj][r][c] = s;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<float4*>(&S.X[32 * jbk + r0 + i][32 * ib + c0]) =
+                    make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         }
         __syncthreads();
-        for (int e = tid; e < nj * 1024; e += blockDim.x) {
-            const int jj = e >> 10, r = (e >> 5) & 31, c = e & 31;
-            float s = 0.f;
-#pragma unroll 8
-            for (int m = 0; m < 32; ++m) s = fmaf(S.xinv[ib][r][m], S.tmp[jj][m][c], s);
-            S.u[ib * 32 + r][(ib + 1 + jj) * 32 + c] = -s;
+        for (int task = tid; task < nblk * 64; task += blockDim.x) {
+            // X_ij[r][c] = -sum_m X_ii[r][m] T[m][c]
+            const int jbk = task >> 6, ib = jbk + dd, tr = (task >> 3) & 7, tc = task & 7;
+            const int r0 = 4 * tr, c0 = 4 * tc;
+            float acc[4][4] = {};
+#pragma unroll 4
+            for (int m = 0; m < 32; ++m) {
+                const float4 a = ld4(&S.XDT[ib][m][r0]);
+                const float4 b = ld4(&S.X[32 * jbk + m][32 * ib + c0]);
+                const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<float4*>(&S.X[32 * ib + r0 + i][32 * jbk + c0]) =
+                    make_float4(-acc[i][0], -acc[i][1], -acc[i][2], -acc[i][3]);
         }
         __syncthreads();
     }
 
-    // outputs: row-major passes, then a transposed pass with consecutive threads on rows
-    for (int e = tid; e < NB * NB; e += blockDim.x) {
-        const int r = e >> 7, c = e & 127;
-        const float v = S.u[r][c];
+    // U block = J X J (upper): U[r][c] = X[127-r][127-c] for r <= c; 4 columns per thread
+    for (int task = tid; task < NB * 32; task += blockDim.x) {
+        const int r = task >> 5, c = (task & 31) * 4;
+        const float4 xv = ld4(&S.X[127 - r][124 - c]);   // columns 124-c .. 127-c, reversed below
+        float v[4] = {xv.w, xv.z, xv.y, xv.x};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (r > c + i) v[i] = 0.f;
+        float h[4], l[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) split_tf32(v[i], h[i], l[i]);
         const long long gr = jb + r, gc = jb + c;
-        float h, l;
-        split_tf32(v, h, l);
-        U_hi[gr * n + gc] = h;
-        U_lo[gr * n + gc] = l;
-        if (gr < d && gc < d) U[gr * d + gc] = v;
+        *reinterpret_cast<float4*>(U_hi + gr * n + gc) = make_float4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<float4*>(U_lo + gr * n + gc) = make_float4(l[0], l[1], l[2], l[3]);
+        if (gr < d) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (gc + i < d) U[gr * d + gc + i] = v[i];
+        }
     }
-    for (int e = tid; e < NB * NB; e += blockDim.x) {
-        const int c = e >> 7, r = e & 127;
-        const float v = S.u[r][c];
-        float h, l;
-        split_tf32(v, h, l);
-        UT_hi[(long long)(jb + c) * n + jb + r] = h;
-        UT_lo[(long long)(jb + c) * n + jb + r] = l;
+    // UT[c][r] = U[r][c] = X[127-r][127-c] = L^-1 read along a column of X
+    for (int task = tid; task < NB * 32; task += blockDim.x) {
+        const int c = task >> 5, r = (task & 31) * 4;
+        float v[4], h[4], l[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = (r + i <= c) ? S.X[127 - r - i][127 - c] : 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) split_tf32(v[i], h[i], l[i]);
+        const long long off = (long long)(jb + c) * n + jb + r;
+        *reinterpret_cast<float4*>(UT_hi + off) = make_float4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<float4*>(UT_lo + off) = make_float4(l[0], l[1], l[2], l[3]);
     }
 }
 
@@ -307,7 +410,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
         GQ_TRY(cudaGetLastError());
     }
     const int leaf_smem = (int)sizeof(gq::LeafSmem);
-    GQ_TRY(cudaFuncSetAttribute(gq::chol_leaf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, leaf_smem));
+    GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::chol_leaf_kernel), leaf_smem));
     const uint64_t N = (uint64_t)n;
     for (int j = T - 1; j >= 0; --j) {
         const int jb = j * gq::NB;
@@ -327,13 +430,13 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
             gq::GemmArgs p = gemm_args(jb, gq::NB, gq::NB);
             p.b_row0 = jb;
             p.b_col0 = jb;
-            p.S_hi = w.RS_hi;
-            p.S_lo = w.RS_lo;
-            p.lds = n;
             p.s_col0 = jb;
+            EpiMats o;
+            o.s_hi = Mat{w.RS_hi, N, N, N};
+            o.s_lo = Mat{w.RS_lo, N, N, N};
             Mat ah{w.AP_hi, (uint64_t)jb, 128, 128}, al{w.AP_lo, (uint64_t)jb, 128, 128};
             Mat bh{w.U_hi, N, N, N}, bl{w.U_lo, N, N, N};
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 3>(ah, al, bh, bl, p, 1, st, "chol_panel")));
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 3, false>(ah, al, bh, bl, o, p, 1, st, "chol_panel")));
         }
         {   // update: A[0:jb, 0:jb] -= RS_panel RS_panel^T (upper tiles)
             gq::GemmArgs p = gemm_args(jb, jb, gq::NB);
@@ -342,11 +445,11 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
             p.triangular = 1;
             p.alpha = -1.f;
             p.beta = 1.f;
-            p.C = w.A;
-            p.ldc = n;
             p.write_c = 1;
+            EpiMats o;
+            o.c = Mat{w.A, N, N, N};
             Mat rh{w.RS_hi, N, N, N}, rl{w.RS_lo, N, N, N};
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 3>(rh, rl, rh, rl, p, 1, st, "chol_update")));
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 2, true>(rh, rl, rh, rl, o, p, 1, st, "chol_update")));
         }
     }
     // U = R^-1 by doubling
@@ -380,13 +483,13 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
                 p.b_col0 = (int)(r0 + s);
                 p.b_zrow = p.b_zcol = zs;
                 p.k_to_n1 = 1;
-                p.T_hi = w.TT_hi;
-                p.T_lo = w.TT_lo;
-                p.ldt = n;
                 p.t_row0 = (int)(r0 + s);
                 p.t_col0 = (int)r0;
                 p.t_zrow = p.t_zcol = zs;
-                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 3>(rsh, rsl, uth, utl, p, (int)batch, st, "inv_bu")));
+                EpiMats o;
+                o.t_hi = Mat{w.TT_hi, N, N, N};
+                o.t_lo = Mat{w.TT_lo, N, N, N};
+                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 3, false>(rsh, rsl, uth, utl, o, p, (int)batch, st, "inv_bu")));
             }
             {   // U_b = -U_a T -> U (public, clipped), U split, UT split
                 gq::GemmArgs p = gemm_args((int)s, (int)cs, (int)s);
@@ -398,27 +501,25 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
                 p.b_zrow = p.b_zcol = zs;
                 p.k_from_m0 = 1;
                 p.alpha = -1.f;
-                p.C = U;
-                p.ldc = d;
                 p.c_row0 = (int)r0;
                 p.c_col0 = (int)(r0 + s);
                 p.c_zrow = p.c_zcol = zs;
                 p.c_lim_rows = (int)d;
                 p.c_lim_cols = (int)d;
                 p.write_c = 1;
-                p.S_hi = w.U_hi;
-                p.S_lo = w.U_lo;
-                p.lds = n;
                 p.s_row0 = (int)r0;
                 p.s_col0 = (int)(r0 + s);
                 p.s_zrow = p.s_zcol = zs;
-                p.T_hi = w.UT_hi;
-                p.T_lo = w.UT_lo;
-                p.ldt = n;
                 p.t_row0 = (int)(r0 + s);
                 p.t_col0 = (int)r0;
                 p.t_zrow = p.t_zcol = zs;
-                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 3>(uh, ul, tth, ttl, p, (int)batch, st, "inv_ub")));
+                EpiMats o;
+                o.c = Mat{U, (uint64_t)d, (uint64_t)d, (uint64_t)d};   // public U, clipped to d x d
+                o.s_hi = Mat{w.U_hi, N, N, N};
+                o.s_lo = Mat{w.U_lo, N, N, N};
+                o.t_hi = Mat{w.UT_hi, N, N, N};
+                o.t_lo = Mat{w.UT_lo, N, N, N};
+                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 3, false>(uh, ul, tth, ttl, o, p, (int)batch, st, "inv_ub")));
             }
         }
     }

@@ -1,16 +1,20 @@
 // GPTQ column loop for one 128-column lazy block (tutorial "阶段二" greedy order and
 // lazy batch updates, "阶段三" group-wise scale; group-size article for scale/zero).
 //
-// Rows are independent.  Four lanes share one row; lane k of the row holds the
-// block's columns k, k+4, ..., k+124 in registers (cyclic mapping keeps the per-step
-// update work balanced across the four lanes).  For column c of the block:
-//   owner lane (c % 4):  r = clamp(rint(w_c / s), -z, maxq - z);  d_c = w_c - s * r
-//   all four lanes:      w_j -= d_c * U[c, j] / U[c, c]   for the block columns j > c
+// Rows are independent.  Eight lanes share one row; lane k of the row holds the
+// block's columns k, k+8, ..., k+120 in registers (cyclic mapping keeps the per-step
+// update work balanced across the lanes).  The block is walked in 16 "octs" of eight
+// columns by a rolled loop: register slot 0 always holds the lane's column of the
+// current oct and the slots shift down by one after each oct, so the loop body stays
+// small (a fully unrolled 128-step loop thrashed the instruction cache).  Four phases
+// of four octs carry 16, 12, 8 and 4 live slots.  For column c:
+//   owner lane (c % 8):  r = clamp(rint(w_c / s), -z, maxq - z);  d_c = w_c - s * r
+//   all eight lanes:     w_j -= d_c * U[c, j] / U[c, c]   for the block columns j > c
 // which is e_c = d_c / U_cc pushed forward with row c of U.  The normalised rows of
 // the block's 128x128 diagonal part of U are prepared once per layer and staged into
 // shared memory by one bulk (TMA) copy per CTA.
 // At a group's first column the scale and zero come from the current values of the
-// group's columns (min/max by a 4-lane shuffle reduction).
+// group's columns (min/max by an 8-lane shuffle reduction).
 // At the end of the block the kernel writes the packed codes (qweight layout), the
 // errors e = d / U_cc as a tf32 split (operand of the trailing tensor-core update)
 // and the per-row sum of e^2.
@@ -21,11 +25,14 @@
 namespace gq {
 
 constexpr int CB = 128;                  // lazy block width
-constexpr int CL_WARPS = 2;
-constexpr int CL_ROWS = CL_WARPS * 8;    // rows per CTA
-constexpr int UP_LD = 36;                // padded slot stride of one lane's row segment
-constexpr int UP_ROW = 4 * UP_LD;        // floats per normalised U row
-constexpr int UP_BLOCK = CB * UP_ROW;    // floats per block (73728 bytes)
+constexpr int LPR = 8;                   // lanes per row
+constexpr int SLOTS = CB / LPR;          // register slots per lane
+constexpr int RPW = 32 / LPR;            // rows per warp
+constexpr int CL_WARPS = 4;
+constexpr int CL_ROWS = CL_WARPS * RPW;  // rows per CTA
+constexpr int UP_LD = 20;                // padded slot stride of one lane's row segment (16 used)
+constexpr int UP_ROW = LPR * UP_LD;      // floats per normalised U row
+constexpr int UP_BLOCK = CB * UP_ROW;    // floats per block (81920 bytes)
 constexpr int CODE_LD = 132;
 constexpr int DV_LD = 129;
 constexpr float kF16MinPos = 5.9604644775390625e-08f;  // 2^-24, smallest positive fp16
@@ -34,7 +41,7 @@ struct ColArgs {
     float* W;
     long long d_out, d_in;
     int c0, nc;
-    const float* Up;      // normalised U rows of this block, [128][UP_ROW]
+    const float* Up;      // normalised, quad-shifted U rows of this block, [128][UP_ROW]
     const float* inv_d;   // [d_in] 1 / U_cc
     int g, sym;
     const float* row_scale;
@@ -72,6 +79,87 @@ __device__ __forceinline__ void group_grid(float lo, float hi, int sym, float& s
         z = fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.f), (float)MAXQ);
 }
 
+struct QuadState {
+    float s, inv_s, qlo, qhi;  // current group: scale, 1/scale, -zero, maxq - zero
+};
+
+// Octs [t0, t1) of the block with LIVE register slots in use.  Slot i of lane k holds
+// column 8*(t + i) + k at oct t; the normalised U row of column c is stored shifted so
+// that its entry for slot i is at offset i (zeros for columns at or before c).
+template <int BITS, int LIVE>
+__device__ __forceinline__ void run_octs(float (&wv)[SLOTS], int t0, int t1, QuadState& st, const ColArgs& p,
+                                         ColSmem& S, int lane, int k, int rloc, long long row, bool row_ok) {
+    constexpr unsigned FULL = 0xffffffffu;
+    constexpr int MAXQ = (1 << BITS) - 1;
+    const int g = p.g;
+#pragma unroll 1
+    for (int t = t0; t < t1; ++t) {
+        const int c8 = LPR * t;
+        if (g > 0 && (c8 & (g - 1)) == 0) {
+            const int gslots = g / LPR;
+            float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < LIVE; ++i) {
+                if (i < gslots) {
+                    mn = fminf(mn, wv[i]);
+                    mx = fmaxf(mx, wv[i]);
+                }
+            }
+#pragma unroll
+            for (int o = 1; o < LPR; o <<= 1) {
+                mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
+                mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+            }
+            float lo, hi;
+            if (p.sym) {
+                const float m = fmaxf(fabsf(mn), fabsf(mx));
+                lo = -m;
+                hi = m;
+            } else {
+                lo = fminf(mn, 0.f);
+                hi = fmaxf(mx, 0.f);
+            }
+            float z;
+            group_grid<BITS>(lo, hi, p.sym, st.s, z);
+            st.inv_s = __frcp_rn(st.s);
+            st.qlo = -z;
+            st.qhi = (float)MAXQ - z;
+            if (k == 0 && row_ok) {
+                const long long gi = (p.c0 + c8) / g;
+                p.scales[gi * p.d_out + row] = __float2half_rn(st.s);
+                p.zeros_u8[gi * p.d_out + row] = (uint8_t)(int)z;
+            }
+        }
+        float my_r = 0.f, my_d = 0.f;
+#pragma unroll
+        for (int own = 0; own < LPR; ++own) {
+            const int c = c8 + own;
+            const float4* u = reinterpret_cast<const float4*>(S.up + c * UP_ROW + k * UP_LD);
+            float4 uu[LIVE / 4];
+#pragma unroll
+            for (int q = 0; q < LIVE / 4; ++q) uu[q] = u[q];
+            const float x = wv[0] * st.inv_s;
+            const float r = fminf(fmaxf(rintf(x), st.qlo), st.qhi);
+            const float dd = fmaf(-r, st.s, wv[0]);
+            const float db = __shfl_sync(FULL, dd, (lane & ~(LPR - 1)) | own);
+            my_r = (k == own) ? r : my_r;
+            my_d = (k == own) ? dd : my_d;
+#pragma unroll
+            for (int q = 0; q < LIVE / 4; ++q) {
+                wv[4 * q + 0] = fmaf(-db, uu[q].x, wv[4 * q + 0]);
+                wv[4 * q + 1] = fmaf(-db, uu[q].y, wv[4 * q + 1]);
+                wv[4 * q + 2] = fmaf(-db, uu[q].z, wv[4 * q + 2]);
+                wv[4 * q + 3] = fmaf(-db, uu[q].w, wv[4 * q + 3]);
+            }
+        }
+        S.codes[rloc][c8 + k] = (uint8_t)(int)(my_r - st.qlo);
+        S.dv[rloc][c8 + k] = my_d;
+#pragma unroll
+        for (int i = 0; i < LIVE - 1; ++i) wv[i] = wv[i + 1];
+        wv[LIVE - 1] = 0.f;
+    }
+}
+
 template <int BITS>
 __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p) {
     extern __shared__ __align__(128) uint8_t cl_raw[];
@@ -79,8 +167,8 @@ __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p)
     constexpr unsigned FULL = 0xffffffffu;
     constexpr int MAXQ = (1 << BITS) - 1;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int k = lane & 3;
-    const int rloc = warp * 8 + (lane >> 2);
+    const int k = lane & (LPR - 1);
+    const int rloc = warp * RPW + lane / LPR;
     const long long row = (long long)blockIdx.x * CL_ROWS + rloc;
     const bool row_ok = row < p.d_out;
 
@@ -100,13 +188,13 @@ __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p)
     }
     for (int c = tid; c < CB; c += blockDim.x) S.invd[c] = (c < p.nc) ? p.inv_d[p.c0 + c] : 0.f;
 
-    float wv[32];
+    float wv[SLOTS];
     {
         const float* wrow = p.W + row * p.d_in + p.c0;
         bool finite = true;
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            const int col = k + 4 * t;
+        for (int t = 0; t < SLOTS; ++t) {
+            const int col = k + LPR * t;
             float v = 0.f;
             if (row_ok && col < p.nc) v = wrow[col];
             finite = finite && isfinite(v);
@@ -127,70 +215,18 @@ __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p)
     __syncthreads();
     if (!ok) return;
 
-    const int g = p.g;
-    const int gmask = g > 0 ? g - 1 : 0;
-#pragma unroll
-    for (int c = 0; c < CB; ++c) {
-        const int t = c >> 2, own = c & 3;
-        if (g > 0 && (c & gmask) == 0) {
-            const int tend = (c + g) >> 2;
-            float mn = INFINITY, mx = -INFINITY;
-#pragma unroll
-            for (int t2 = t; t2 < 32; ++t2) {
-                if (t2 < tend) {
-                    mn = fminf(mn, wv[t2]);
-                    mx = fmaxf(mx, wv[t2]);
-                }
-            }
-            mn = fminf(mn, __shfl_xor_sync(FULL, mn, 1));
-            mn = fminf(mn, __shfl_xor_sync(FULL, mn, 2));
-            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
-            float lo, hi;
-            if (p.sym) {
-                const float m = fmaxf(fabsf(mn), fabsf(mx));
-                lo = -m;
-                hi = m;
-            } else {
-                lo = fminf(mn, 0.f);
-                hi = fmaxf(mx, 0.f);
-            }
-            float z;
-            group_grid<BITS>(lo, hi, p.sym, s, z);
-            inv_s = __frcp_rn(s);
-            qlo = -z;
-            qhi = (float)MAXQ - z;
-            if (k == 0 && row_ok) {
-                const long long gi = (p.c0 + c) / g;
-                p.scales[gi * p.d_out + row] = __float2half_rn(s);
-                p.zeros_u8[gi * p.d_out + row] = (uint8_t)(int)z;
-            }
-        }
-        const float x = wv[t] * inv_s;
-        const float r = fminf(fmaxf(rintf(x), qlo), qhi);
-        const float dd = fmaf(-r, s, wv[t]);
-        const float db = __shfl_sync(FULL, dd, (lane & ~3) | own);
-        if (k == own) {
-            S.codes[rloc][c] = (uint8_t)(int)(r - qlo);
-            S.dv[rloc][c] = dd;
-        }
-        const float* urow = S.up + c * UP_ROW + k * UP_LD;
-#pragma unroll
-        for (int q4 = (t >> 2); q4 < 8; ++q4) {
-            const float4 u4 = *reinterpret_cast<const float4*>(urow + 4 * q4);
-            if (4 * q4 + 0 >= t) wv[4 * q4 + 0] = fmaf(-db, u4.x, wv[4 * q4 + 0]);
-            if (4 * q4 + 1 >= t) wv[4 * q4 + 1] = fmaf(-db, u4.y, wv[4 * q4 + 1]);
-            if (4 * q4 + 2 >= t) wv[4 * q4 + 2] = fmaf(-db, u4.z, wv[4 * q4 + 2]);
-            if (4 * q4 + 3 >= t) wv[4 * q4 + 3] = fmaf(-db, u4.w, wv[4 * q4 + 3]);
-        }
-    }
+    QuadState st{s, inv_s, qlo, qhi};
+    run_octs<BITS, 16>(wv, 0, 4, st, p, S, lane, k, rloc, row, row_ok);
+    run_octs<BITS, 12>(wv, 4, 8, st, p, S, lane, k, rloc, row, row_ok);
+    run_octs<BITS, 8>(wv, 8, 12, st, p, S, lane, k, rloc, row, row_ok);
+    run_octs<BITS, 4>(wv, 12, 16, st, p, S, lane, k, rloc, row, row_ok);
     __syncwarp();
 
     // errors of the block (operand of the trailing update) and per-row sum of e^2
-    const long long wrow0 = (long long)blockIdx.x * CL_ROWS + warp * 8;
-    for (int rr = 0; rr < 8; ++rr) {
+    const long long wrow0 = (long long)blockIdx.x * CL_ROWS + warp * RPW;
+    for (int rr = 0; rr < RPW; ++rr) {
         const long long rw = wrow0 + rr;
-        const int rl = warp * 8 + rr;
+        const int rl = warp * RPW + rr;
         float acc = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -213,11 +249,11 @@ __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p)
     // packed codes: word w of this block's stream for each of the warp's 8 rows
     const int nwb = (p.nc * BITS + 31) / 32;
     const long long wbase = (long long)p.c0 * BITS / 32;
-    for (int idx = lane; idx < 8 * nwb; idx += 32) {
-        const int rr = idx & 7, w = idx >> 3;
+    for (int idx = lane; idx < RPW * nwb; idx += 32) {
+        const int rr = idx % RPW, w = idx / RPW;
         const long long rw = wrow0 + rr;
         if (rw >= p.d_out) continue;
-        const int rl = warp * 8 + rr;
+        const int rl = warp * RPW + rr;
         const int bit0 = w * 32;
         const int j0 = bit0 / BITS, j1 = min(p.nc - 1, (bit0 + 31) / BITS);
         unsigned long long acc = 0;
@@ -227,9 +263,9 @@ __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p)
     }
 }
 
-// Normalised, lane-permuted rows of each 128x128 diagonal block of U:
-// Up[b][c][k*UP_LD + t] = U[c0+c, c0+j] / U[c0+c, c0+c] for j = k + 4t > c (0 otherwise),
-// and inv_d[c] = 1 / U[c, c].
+// Normalised, lane-permuted, oct-shifted rows of each 128x128 diagonal block of U:
+// Up[b][c][k*UP_LD + i] = U[c0+c, c0+j] / U[c0+c, c0+c] with j = k + 8*(c/8 + i) for j > c
+// (0 otherwise), and inv_d[c] = 1 / U[c, c].
 __global__ void up_prep_kernel(const float* __restrict__ U, long long d, float* __restrict__ Up,
                                float* __restrict__ inv_d) {
     const int b = blockIdx.y, c = blockIdx.x;
@@ -238,10 +274,10 @@ __global__ void up_prep_kernel(const float* __restrict__ U, long long d, float* 
     const float ucc = (c < nc) ? U[(c0 + c) * d + c0 + c] : 1.f;
     float* dst = Up + ((long long)b * CB + c) * UP_ROW;
     for (int e = threadIdx.x; e < UP_ROW; e += blockDim.x) {
-        const int kk = e / UP_LD, t = e % UP_LD;
-        const int j = kk + 4 * t;
+        const int kk = e / UP_LD, i = e % UP_LD;
+        const int j = kk + LPR * ((c / LPR) + i);
         float v = 0.f;
-        if (t < 32 && c < nc && j < nc && j > c) v = __fdiv_rn(U[(c0 + c) * d + c0 + j], ucc);
+        if (i < SLOTS && c < nc && j < nc && j > c) v = __fdiv_rn(U[(c0 + c) * d + c0 + j], ucc);
         dst[e] = v;
     }
     if (threadIdx.x == 0 && c < nc) inv_d[c0 + c] = __frcp_rn(ucc);
@@ -385,7 +421,7 @@ cudaError_t quant_run_bits(float* W, const float* U, long long d_out, long long 
         GQ_TRY(cudaGetLastError());
     }
     const int smem = (int)sizeof(gq::ColSmem);
-    GQ_TRY(cudaFuncSetAttribute(gq::colloop_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::colloop_kernel<BITS>), smem));
     const unsigned grid = (unsigned)((d_out + gq::CL_ROWS - 1) / gq::CL_ROWS);
     Mat eh{w.E_hi, (uint64_t)d_out, (uint64_t)gq::CB, (uint64_t)gq::CB};
     Mat el{w.E_lo, (uint64_t)d_out, (uint64_t)gq::CB, (uint64_t)gq::CB};
@@ -423,11 +459,11 @@ cudaError_t quant_run_bits(float* W, const float* U, long long d_out, long long 
             p.b_col0 = a.c0;
             p.alpha = -1.f;
             p.beta = 1.f;
-            p.C = W;
-            p.ldc = d_in;
             p.c_col0 = (int)e;
             p.write_c = 1;
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 256, 2>(eh, el, uh, ul, p, 1, st, "trailing_update")));
+            EpiMats o;
+            o.c = Mat{W, (uint64_t)d_out, (uint64_t)d_in, (uint64_t)d_in};
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 2, true>(eh, el, uh, ul, o, p, 1, st, "trailing_update")));
         }
     }
     if (!cfg.sym && qzeros) {

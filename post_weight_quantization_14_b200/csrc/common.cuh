@@ -71,16 +71,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 // Bounded wait for the phase with the given parity.  Returns false (and records
-// GPTQ_ERR_TIMEOUT with ``where``) when the limit runs out.
+// GPTQ_ERR_TIMEOUT with ``where``) when the limit runs out.  The timer is read only
+// every 256 polls: waiting warps must not compete for issue slots with the warps they
+// wait for.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long where,
                                           unsigned long long limit_ns = kWaitLimitNs) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = globaltimer_ns();
-    while (true) {
+    unsigned long long t0 = 0;
+    for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > limit_ns) {
-            record_status(GPTQ_ERR_TIMEOUT, where);
-            return false;
+        if ((i & 255u) == 0u) {
+            const unsigned long long now = globaltimer_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > limit_ns) {
+                record_status(GPTQ_ERR_TIMEOUT, where);
+                return false;
+            }
         }
     }
 }
@@ -104,6 +110,20 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint3
             smem_u32(smem_dst)),
         "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+// TMA store of a shared-memory box (bulk-group completion) and its bookkeeping.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+                 "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most one committed bulk group still reads shared memory.
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Generic-proxy shared-memory writes become visible to the async (TMA) proxy.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
@@ -237,5 +257,8 @@ struct TimedScope {
 // box_rows x box_cols elements, 128-byte swizzle, out-of-bounds reads as zero.
 bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
                   uint64_t ld, uint32_t box_rows, uint32_t box_cols);
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device, size).
+cudaError_t ensure_smem_attr(const void* func, int bytes);
 
 }  // namespace gqh

@@ -12,8 +12,16 @@
 //               about fp32 accuracy on the tf32 tensor pipe.
 //
 // One 128 x BN output tile per CTA; warp 0 issues TMA, warp 1 issues MMAs, warps
-// 2..5 read the accumulator from tensor memory and run the epilogue.  Every wait is
-// bounded (GPTQ_ERR_TIMEOUT).  No TMA multicast.
+// 2..5 read the accumulator from tensor memory and run the epilogue.  The epilogue is
+// TMA-based: for C -= A B^T updates the C tile is fetched by TMA while the mainloop
+// runs (PREFETCH_C), and every output is written as 32x32 boxes staged in
+// 128-byte-swizzled shared memory and stored by TMA, double-buffered per warp, so the
+// HBM traffic of the epilogue runs asynchronously.  Tiles on the diagonal of a
+// mirrored (symmetric) output take a register path that writes j >= i and mirrors
+// it exactly.  Every wait is bounded (GPTQ_ERR_TIMEOUT).  No TMA multicast.
+//
+// Outputs are clipped by the extents of their tensor maps; every caller keeps M and
+// N either multiples of the tile or equal to the remaining extent of the output.
 #pragma once
 #include "common.cuh"
 
@@ -45,6 +53,9 @@ struct GemmArgs {
     long long ldt;
     int t_row0, t_col0, t_zrow, t_zcol;
 };
+
+constexpr int kEpiLd = 33;
+constexpr int kEpiBytes = 4 * 32 * kEpiLd * 4;
 
 template <int KIND>
 struct GemmCfg {
@@ -78,11 +89,32 @@ __device__ __forceinline__ void store_split(float* hi, float* lo, long long idx,
     lo[idx] = l;
 }
 
-template <int KIND, int BN, int STAGES>
+constexpr int kBoxBytes = 32 * 32 * 4;   // one 32x32 fp32 box, 128-byte rows
+
+// Byte offset of element (row, col) in a 128-byte-swizzled 32x32 fp32 box.
+__device__ __forceinline__ uint32_t box_off(int row, int col) {
+    return (uint32_t)(row * 128 + ((((col >> 2) ^ (row & 7))) << 4) + (col & 3) * 4);
+}
+// Thread `row` writes its 32 values as one row of the box.
+__device__ __forceinline__ void box_put_row(uint8_t* box, int row, const float (&v)[32]) {
+#pragma unroll
+    for (int c4 = 0; c4 < 8; ++c4)
+        *reinterpret_cast<float4*>(box + row * 128 + ((c4 ^ (row & 7)) << 4)) =
+            make_float4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
+}
+// Thread `col` writes its 32 values as one column of the box (transposed output).
+__device__ __forceinline__ void box_put_col(uint8_t* box, int col, const float (&v)[32]) {
+#pragma unroll
+    for (int t = 0; t < 32; ++t) *reinterpret_cast<float*>(box + box_off(t, col)) = v[t];
+}
+
+template <int KIND, int BN, int STAGES, bool PREFETCH_C>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
                    const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mB2,
-                   const GemmArgs p) {
+                   const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mS1,
+                   const __grid_constant__ CUtensorMap mS2, const __grid_constant__ CUtensorMap mT1,
+                   const __grid_constant__ CUtensorMap mT2, const GemmArgs p) {
     using Cfg = GemmCfg<KIND>;
     constexpr int BM = Cfg::BM, KT = Cfg::KT, NOPS = Cfg::NOPS;
     constexpr int A_BYTES = BM * 128;
@@ -94,10 +126,14 @@ __global__ void __launch_bounds__(192, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    constexpr int CIN_BYTES = PREFETCH_C ? BM * BN * 4 : 0;
+    uint8_t* cin = smem + STAGES * STAGE_BYTES;                       // prefetched C boxes
+    float* epi = reinterpret_cast<float*>(cin + CIN_BYTES);           // 4 warps x 32 x 33
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(epi) + kEpiBytes);
     uint64_t* empty_bar = full_bar + STAGES;
     uint64_t* acc_bar = empty_bar + STAGES;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_bar + 1);
+    uint64_t* cin_bar = acc_bar + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cin_bar + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int mt, nt;
@@ -115,6 +151,7 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(&empty_bar[s], 1);
         }
         mbar_init(acc_bar, 1);
+        mbar_init(cin_bar, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -136,6 +173,14 @@ __global__ void __launch_bounds__(192, 1)
         }
         const int ax = p.a_col0 + z * p.a_zcol, ay = p.a_row0 + z * p.a_zrow + m0;
         const int bx = p.b_col0 + z * p.b_zcol, by = p.b_row0 + z * p.b_zrow + n0;
+        if (PREFETCH_C && p.beta != 0.f) {   // the C tile, as 32x32 boxes, while the mainloop runs
+            prefetch_tmap(&mC);
+            mbar_arrive_expect_tx(cin_bar, CIN_BYTES);
+            const int cx = p.c_col0 + z * p.c_zcol + n0, cy = p.c_row0 + z * p.c_zrow + m0;
+            for (int q = 0; q < 4; ++q)
+                for (int c = 0; c < BN / 32; ++c)
+                    tma_load_2d(cin + (q * (BN / 32) + c) * kBoxBytes, &mC, cin_bar, cx + 32 * c, cy + 32 * q);
+        }
         for (int kt = 0; kt < nk; ++kt) {
             const int s = kt % STAGES;
             const uint32_t it = kt / STAGES;
@@ -184,93 +229,155 @@ __global__ void __launch_bounds__(192, 1)
     } else if (warp >= 2) {
         const bool ok = mbar_wait(acc_bar, 0, where);
         tc_fence_after();
-        const int q = warp & 3;
-        const int i = m0 + q * 32 + lane;
-        const bool row_ok = i < p.M;
-        const bool mirror = p.mirror && nt > mt;
+        const bool diag_mirror = p.mirror && nt == mt;
+        if (!diag_mirror) {
+            // TMA epilogue
+            const int q = warp & 3;
+            const bool mirror = p.mirror && nt > mt;
+            const bool has_c = p.write_c != 0, has_s = p.S_hi != nullptr, has_t = p.T_hi != nullptr;
+            const int nkinds = (has_c ? 1 : 0) + (has_s ? 2 : 0) + (has_t ? 2 : 0) + (mirror ? 1 : 0);
+            const int kc = 0, ks = kc + (has_c ? 1 : 0), kt = ks + (has_s ? 2 : 0), km = kt + (has_t ? 2 : 0);
+            const bool use_cin = PREFETCH_C && p.beta != 0.f;
+            bool cin_ok = true;
+            if (use_cin) cin_ok = mbar_wait(cin_bar, 0, where);
+            const int zc_x = p.c_col0 + z * p.c_zcol, zc_y = p.c_row0 + z * p.c_zrow;
+            const int zs_x = p.s_col0 + z * p.s_zcol, zs_y = p.s_row0 + z * p.s_zrow;
+            const int zt_x = p.t_col0 + z * p.t_zcol, zt_y = p.t_row0 + z * p.t_zrow;
+            const int iy = m0 + 32 * q;   // first accumulator row of this warp
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-            const int j0 = n0 + c * 32;
-            if (j0 >= p.N) break;
-            uint32_t r[32];
-            if (nk > 0 && ok) {
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), r);
-                tmem_ld_wait();
-            } else {
-#pragma unroll
-                for (int t = 0; t < 32; ++t) r[t] = 0u;
-            }
-            const int jn = min(32, p.N - j0);
-            float out[32];
-            if (row_ok) {
-                const long long ar = p.c_row0 + z * p.c_zrow + i;
-                const long long ac = p.c_col0 + z * p.c_zcol + j0;
-                const long long crow = ar * p.ldc + ac;
-                int jc = jn;
-                if (p.c_lim_rows > 0 && ar >= p.c_lim_rows) jc = 0;
-                if (p.c_lim_cols > 0) jc = (int)max(0LL, min((long long)jc, (long long)p.c_lim_cols - ac));
-                const bool vec = (jc == 32) && ((crow & 3) == 0);
-                if (p.beta != 0.f) {
-                    if (vec) {
-                        const float4* src = reinterpret_cast<const float4*>(p.C + crow);
-#pragma unroll
-                        for (int t = 0; t < 8; ++t) {
-                            float4 cv = src[t];
-                            out[4 * t + 0] = p.alpha * __uint_as_float(r[4 * t + 0]) + p.beta * cv.x;
-                            out[4 * t + 1] = p.alpha * __uint_as_float(r[4 * t + 1]) + p.beta * cv.y;
-                            out[4 * t + 2] = p.alpha * __uint_as_float(r[4 * t + 2]) + p.beta * cv.z;
-                            out[4 * t + 3] = p.alpha * __uint_as_float(r[4 * t + 3]) + p.beta * cv.w;
-                        }
-                    } else {
-#pragma unroll
-                        for (int t = 0; t < 32; ++t)
-                            out[t] = p.alpha * __uint_as_float(r[t]) +
-                                     (t < jc ? p.beta * p.C[crow + t] : 0.f);
-                    }
+            for (int c = 0; c < BN / 32; ++c) {
+                const int j0 = n0 + c * 32;
+                if (j0 >= p.N) break;
+                uint32_t r[32];
+                if (nk > 0 && ok) {
+                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), r);
+                    tmem_ld_wait();
                 } else {
 #pragma unroll
-                    for (int t = 0; t < 32; ++t) out[t] = p.alpha * __uint_as_float(r[t]);
+                    for (int t = 0; t < 32; ++t) r[t] = 0u;
                 }
-                if (p.write_c) {
-                    if (vec) {
-                        float4* dst = reinterpret_cast<float4*>(p.C + crow);
+                float out[32];
 #pragma unroll
-                        for (int t = 0; t < 8; ++t)
-                            dst[t] = make_float4(out[4 * t], out[4 * t + 1], out[4 * t + 2], out[4 * t + 3]);
+                for (int t = 0; t < 32; ++t) out[t] = p.alpha * __uint_as_float(r[t]);
+                if (use_cin && cin_ok) {
+                    const uint8_t* box = cin + (q * (BN / 32) + c) * kBoxBytes;
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 v = *reinterpret_cast<const float4*>(box + lane * 128 + ((c4 ^ (lane & 7)) << 4));
+                        out[4 * c4 + 0] = fmaf(p.beta, v.x, out[4 * c4 + 0]);
+                        out[4 * c4 + 1] = fmaf(p.beta, v.y, out[4 * c4 + 1]);
+                        out[4 * c4 + 2] = fmaf(p.beta, v.z, out[4 * c4 + 2]);
+                        out[4 * c4 + 3] = fmaf(p.beta, v.w, out[4 * c4 + 3]);
+                    }
+                }
+                // output boxes of this chunk live in the (now idle) stage buffers, two slots per warp
+                uint8_t* ob = smem + ((q * 2 + (c & 1)) * nkinds) * kBoxBytes;
+                if (c >= 2) {
+                    if (lane == 0) bulk_wait_read_1();
+                    __syncwarp();
+                }
+                if (has_c) box_put_row(ob + kc * kBoxBytes, lane, out);
+                if (has_s || has_t) {
+                    float hi[32], lo[32];
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) split_tf32(out[t], hi[t], lo[t]);
+                    if (has_s) {
+                        box_put_row(ob + ks * kBoxBytes, lane, hi);
+                        box_put_row(ob + (ks + 1) * kBoxBytes, lane, lo);
+                    }
+                    if (has_t) {
+                        box_put_col(ob + kt * kBoxBytes, lane, hi);
+                        box_put_col(ob + (kt + 1) * kBoxBytes, lane, lo);
+                    }
+                }
+                if (mirror) box_put_col(ob + km * kBoxBytes, lane, out);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    if (has_c) tma_store_2d(&mC, ob + kc * kBoxBytes, zc_x + j0, zc_y + iy);
+                    if (has_s) {
+                        tma_store_2d(&mS1, ob + ks * kBoxBytes, zs_x + j0, zs_y + iy);
+                        tma_store_2d(&mS2, ob + (ks + 1) * kBoxBytes, zs_x + j0, zs_y + iy);
+                    }
+                    if (has_t) {
+                        tma_store_2d(&mT1, ob + kt * kBoxBytes, zt_x + iy, zt_y + j0);
+                        tma_store_2d(&mT2, ob + (kt + 1) * kBoxBytes, zt_x + iy, zt_y + j0);
+                    }
+                    if (mirror) tma_store_2d(&mC, ob + km * kBoxBytes, zc_x + iy, zc_y + j0);
+                    bulk_commit();
+                }
+            }
+            if (lane == 0) bulk_wait_all();
+            __syncwarp();
+        } else {
+            // Register path for diagonal tiles of mirrored outputs: write j >= i and its exact mirror.
+            const int q = warp & 3;
+            float* tile = epi + q * 32 * kEpiLd;
+            const int rbase = m0 + q * 32;
+            const bool mirror = false;
+            const bool diag_tile = true;   // write j >= i only, mirrored below
+            const long long zc_row = p.c_row0 + (long long)z * p.c_zrow, zc_col = p.c_col0 + (long long)z * p.c_zcol;
+            const long long zs_row = p.s_row0 + (long long)z * p.s_zrow, zs_col = p.s_col0 + (long long)z * p.s_zcol;
+            const long long zt_row = p.t_row0 + (long long)z * p.t_zrow, zt_col = p.t_col0 + (long long)z * p.t_zcol;
+            const bool pass2 = (p.T_hi != nullptr) || mirror || diag_tile;
+    #pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                const int j0 = n0 + c * 32;
+                if (j0 >= p.N) break;
+                uint32_t r[32];
+                if (nk > 0 && ok) {
+                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), r);
+                    tmem_ld_wait();
+                } else {
+    #pragma unroll
+                    for (int t = 0; t < 32; ++t) r[t] = 0u;
+                }
+    #pragma unroll
+                for (int t = 0; t < 32; ++t) tile[lane * kEpiLd + t] = __uint_as_float(r[t]);
+                __syncwarp();
+                {   // pass 1: lane = column; all 32 row loads of C are issued before any use
+                    const int j = j0 + lane;
+                    const bool col_ok = j < p.N;
+                    const long long ac = zc_col + j;
+                    const bool c_col_ok = col_ok && (p.c_lim_cols <= 0 || ac < p.c_lim_cols);
+                    const int nrows = max(0, min(32, p.M - rbase));
+                    float cv[32];
+                    if (p.beta != 0.f) {
+    #pragma unroll
+                        for (int rr = 0; rr < 32; ++rr) {
+                            const long long ar = zc_row + rbase + rr;
+                            const bool c_ok = rr < nrows && c_col_ok && (p.c_lim_rows <= 0 || ar < p.c_lim_rows);
+                            cv[rr] = c_ok ? p.C[ar * p.ldc + ac] : 0.f;
+                        }
                     } else {
-#pragma unroll
-                        for (int t = 0; t < 32; ++t)
-                            if (t < jc) p.C[crow + t] = out[t];
+    #pragma unroll
+                        for (int rr = 0; rr < 32; ++rr) cv[rr] = 0.f;
+                    }
+    #pragma unroll
+                    for (int rr = 0; rr < 32; ++rr) {
+                        const int i = rbase + rr;
+                        const long long ar = zc_row + i;
+                        const bool c_ok = rr < nrows && c_col_ok && (p.c_lim_rows <= 0 || ar < p.c_lim_rows);
+                        const float out = fmaf(p.beta, cv[rr], p.alpha * tile[rr * kEpiLd + lane]);
+                        if (p.write_c && c_ok && (!diag_tile || j >= i)) p.C[ar * p.ldc + ac] = out;
+                        if (p.S_hi && col_ok && rr < nrows) store_split(p.S_hi, p.S_lo, (zs_row + i) * p.lds + zs_col + j, out);
+                        tile[rr * kEpiLd + lane] = out;
                     }
                 }
-                if (p.S_hi) {
-                    const long long srow = (long long)(p.s_row0 + z * p.s_zrow + i) * p.lds +
-                                           (p.s_col0 + z * p.s_zcol + j0);
-#pragma unroll
-                    for (int t = 0; t < 32; ++t)
-                        if (t < jn) store_split(p.S_hi, p.S_lo, srow + t, out[t]);
-                }
-            }
-            // transposed outputs: for fixed t the warp writes 32 consecutive rows i -> coalesced
-            if (p.T_hi) {
-#pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    if (t < jn && row_ok) {
-                        const long long idx = (long long)(p.t_row0 + z * p.t_zrow + j0 + t) * p.ldt +
-                                              (p.t_col0 + z * p.t_zcol + i);
-                        store_split(p.T_hi, p.T_lo, idx, out[t]);
+                __syncwarp();
+                if (pass2) {   // pass 2: lane = row
+                    const int i = rbase + lane;
+                    const bool row_ok = i < p.M;
+    #pragma unroll 4
+                    for (int t = 0; t < 32; ++t) {
+                        const int jj = j0 + t;
+                        if (jj >= p.N) break;
+                        const float out = tile[lane * kEpiLd + t];
+                        if (row_ok && p.T_hi) store_split(p.T_hi, p.T_lo, (zt_row + jj) * p.ldt + zt_col + i, out);
+                        if (row_ok && (mirror || (diag_tile && jj > i))) p.C[(zc_row + jj) * p.ldc + zc_col + i] = out;
                     }
                 }
-            }
-            if (mirror) {
-#pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    if (t < jn && row_ok) {
-                        const long long idx = (long long)(p.c_row0 + z * p.c_zrow + j0 + t) * p.ldc +
-                                              (p.c_col0 + z * p.c_zcol + i);
-                        p.C[idx] = out[t];
-                    }
-                }
+                __syncwarp();
             }
         }
     }
@@ -283,9 +390,10 @@ __global__ void __launch_bounds__(192, 1)
     }
 }
 
-template <int KIND, int BN, int STAGES>
+template <int KIND, int BN, int STAGES, bool PREFETCH_C>
 constexpr int gemm_smem_bytes() {
-    return STAGES * GemmCfg<KIND>::NOPS * (128 * 128 + BN * 128) + 1024 + 256;
+    return STAGES * GemmCfg<KIND>::NOPS * (128 * 128 + BN * 128) + (PREFETCH_C ? 128 * BN * 4 : 0) + kEpiBytes +
+           1024 + 256;
 }
 
 }  // namespace gq
@@ -298,37 +406,66 @@ struct Mat {
     uint64_t rows, cols, ld;  // elements
 };
 
+// Output matrices of the epilogue (ptr == nullptr: not written).  C is also the
+// matrix read when beta != 0 and the target of mirrored writes.
+struct EpiMats {
+    Mat c{nullptr, 0, 0, 0}, s_hi{nullptr, 0, 0, 0}, s_lo{nullptr, 0, 0, 0}, t_hi{nullptr, 0, 0, 0},
+        t_lo{nullptr, 0, 0, 0};
+};
+
+inline bool make_out_map(CUtensorMap* map, const Mat& m, const CUtensorMap& fallback) {
+    if (!m.ptr) {
+        *map = fallback;
+        return true;
+    }
+    return make_tmap_2d(map, m.ptr, 4, m.rows, m.cols, m.ld, 32, 32);
+}
+
 // Launch D = A B^T with the given epilogue.  For KIND_TF32X3 a2/b2 are the lo parts.
-template <int KIND, int BN, int STAGES>
-cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2, gq::GemmArgs p,
+// PREFETCH_C is required when p.beta != 0.
+template <int KIND, int BN, int STAGES, bool PREFETCH_C>
+cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2, const EpiMats& o, gq::GemmArgs p,
                         int batch, cudaStream_t stream, const char* name) {
     using Cfg = gq::GemmCfg<KIND>;
     const int eb = (KIND == gq::KIND_BF16) ? 2 : 4;
-    CUtensorMap ma, ma2, mb, mb2;
+    if (p.beta != 0.f && !PREFETCH_C) return cudaErrorInvalidValue;
+    CUtensorMap ma, ma2, mb, mb2, mc, ms1, ms2, mt1, mt2;
     if (!make_tmap_2d(&ma, a.ptr, eb, a.rows, a.cols, a.ld, 128, Cfg::KT)) return cudaErrorInvalidValue;
     if (!make_tmap_2d(&mb, b.ptr, eb, b.rows, b.cols, b.ld, BN, Cfg::KT)) return cudaErrorInvalidValue;
     if (KIND == gq::KIND_TF32X3) {
-        if (!make_tmap_2d(&ma2, a2.ptr, eb, a2.rows, a2.cols, a2.ld, 128, Cfg::KT))
-            return cudaErrorInvalidValue;
-        if (!make_tmap_2d(&mb2, b2.ptr, eb, b2.rows, b2.cols, b2.ld, BN, Cfg::KT))
-            return cudaErrorInvalidValue;
+        if (!make_tmap_2d(&ma2, a2.ptr, eb, a2.rows, a2.cols, a2.ld, 128, Cfg::KT)) return cudaErrorInvalidValue;
+        if (!make_tmap_2d(&mb2, b2.ptr, eb, b2.rows, b2.cols, b2.ld, BN, Cfg::KT)) return cudaErrorInvalidValue;
     } else {
         ma2 = ma;
         mb2 = mb;
     }
+    if (!make_out_map(&mc, o.c, ma) || !make_out_map(&ms1, o.s_hi, ma) || !make_out_map(&ms2, o.s_lo, ma) ||
+        !make_out_map(&mt1, o.t_hi, ma) || !make_out_map(&mt2, o.t_lo, ma))
+        return cudaErrorInvalidValue;
+    p.C = static_cast<float*>(const_cast<void*>(o.c.ptr));
+    p.ldc = (long long)o.c.ld;
+    p.S_hi = static_cast<float*>(const_cast<void*>(o.s_hi.ptr));
+    p.S_lo = static_cast<float*>(const_cast<void*>(o.s_lo.ptr));
+    p.lds = (long long)o.s_hi.ld;
+    p.T_hi = static_cast<float*>(const_cast<void*>(o.t_hi.ptr));
+    p.T_lo = static_cast<float*>(const_cast<void*>(o.t_lo.ptr));
+    p.ldt = (long long)o.t_hi.ld;
+    // output boxes (two slots per warp) must fit in the stage buffers they reuse
+    const int kinds = (p.write_c ? 1 : 0) + (p.S_hi ? 2 : 0) + (p.T_hi ? 2 : 0) + (p.mirror ? 1 : 0);
+    if (4 * 2 * kinds * gq::kBoxBytes > STAGES * Cfg::NOPS * (128 * 128 + BN * 128)) return cudaErrorInvalidValue;
     p.tiles_m = (p.M + 127) / 128;
     p.tiles_n = (p.N + BN - 1) / BN;
     long long tiles = p.triangular ? (long long)p.tiles_m * (p.tiles_m + 1) / 2
                                    : (long long)p.tiles_m * p.tiles_n;
     if (tiles <= 0 || batch <= 0) return cudaSuccess;
-    constexpr int smem = gq::gemm_smem_bytes<KIND, BN, STAGES>();
-    auto kern = gq::tc_gemm_kernel<KIND, BN, STAGES>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    constexpr int smem = gq::gemm_smem_bytes<KIND, BN, STAGES, PREFETCH_C>();
+    auto kern = gq::tc_gemm_kernel<KIND, BN, STAGES, PREFETCH_C>;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)tiles, 1, (unsigned)batch);
     {
         TimedScope ts__(name, stream);
-        kern<<<grid, 192, smem, stream>>>(ma, ma2, mb, mb2, p);
+        kern<<<grid, 192, smem, stream>>>(ma, ma2, mb, mb2, mc, ms1, ms2, mt1, mt2, p);
     }
     return cudaGetLastError();
 }

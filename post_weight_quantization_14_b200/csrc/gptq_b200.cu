@@ -7,7 +7,9 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <set>
 #include <string>
+#include <tuple>
 #include <vector>
 
 #include "common.cuh"
@@ -78,8 +80,42 @@ static void timing_collect() {
 
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+// Tensor maps depend only on (address, shape, box); the same buffers are reused by
+// every block and every call, so encoded maps are cached (host memory only).
+using TmapKey = std::tuple<uintptr_t, int, uint64_t, uint64_t, uint64_t, uint32_t, uint32_t>;
+static std::map<TmapKey, CUtensorMap> g_tmap_cache;
+
+static bool encode_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
+                           uint64_t ld, uint32_t box_rows, uint32_t box_cols);
+
 bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
                   uint64_t ld, uint32_t box_rows, uint32_t box_cols) {
+    const TmapKey key{reinterpret_cast<uintptr_t>(base), elem_bytes, rows, cols, ld, box_rows, box_cols};
+    auto it = g_tmap_cache.find(key);
+    if (it != g_tmap_cache.end()) {
+        *map = it->second;
+        return true;
+    }
+    if (!encode_tmap_2d(map, base, elem_bytes, rows, cols, ld, box_rows, box_cols)) return false;
+    if (g_tmap_cache.size() > 4096) g_tmap_cache.clear();
+    g_tmap_cache.emplace(key, *map);
+    return true;
+}
+
+cudaError_t ensure_smem_attr(const void* func, int bytes) {
+    static std::set<std::tuple<const void*, int, int>> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const auto key = std::make_tuple(func, dev, bytes);
+    if (done.count(key)) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.insert(key);
+    return e;
+}
+
+static bool encode_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
+                           uint64_t ld, uint32_t box_rows, uint32_t box_cols) {
     if (!g_encode) {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -330,11 +366,11 @@ size_t gptq_timing_report(char* buf, size_t len) {
         first = false;
     }
     out += "}";
-    g_timing_acc.clear();
-    if (buf && len) {
+    if (buf && len) {  // a size query (buf == NULL) keeps the totals
         const size_t n = std::min(len - 1, out.size());
         memcpy(buf, out.data(), n);
         buf[n] = 0;
+        g_timing_acc.clear();
     }
     return out.size() + 1;
 }

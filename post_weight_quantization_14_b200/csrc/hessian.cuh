@@ -68,9 +68,9 @@ inline cudaError_t hessian_run(const void* X, gptq_dtype xt, long long n, long l
     p.mirror = 1;
     p.alpha = 2.f;
     p.beta = accumulate ? 1.f : 0.f;
-    p.C = H;
-    p.ldc = d_in;
     p.write_c = 1;
+    EpiMats o;
+    o.c = Mat{H, (uint64_t)d_in, (uint64_t)d_in, (uint64_t)d_in};
     if (xt == GPTQ_BF16) {
         uint16_t* XT = static_cast<uint16_t*>(ws);
         {
@@ -80,7 +80,8 @@ inline cudaError_t hessian_run(const void* X, gptq_dtype xt, long long n, long l
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         Mat m{XT, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
-        return launch_gemm<gq::KIND_BF16, 128, 6>(m, m, m, m, p, 1, st, "hessian_syrk");
+        return accumulate ? launch_gemm<gq::KIND_BF16, 128, 4, true>(m, m, m, m, o, p, 1, st, "hessian_syrk")
+                          : launch_gemm<gq::KIND_BF16, 128, 6, false>(m, m, m, m, o, p, 1, st, "hessian_syrk");
     }
     float* hi = static_cast<float*>(ws);
     float* lo = hi + d_in * np;
@@ -92,7 +93,8 @@ inline cudaError_t hessian_run(const void* X, gptq_dtype xt, long long n, long l
     if (e != cudaSuccess) return e;
     Mat mh{hi, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
     Mat ml{lo, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
-    return launch_gemm<gq::KIND_TF32X3, 128, 3>(mh, ml, mh, ml, p, 1, st, "hessian_syrk");
+    return accumulate ? launch_gemm<gq::KIND_TF32X3, 128, 2, true>(mh, ml, mh, ml, o, p, 1, st, "hessian_syrk")
+                      : launch_gemm<gq::KIND_TF32X3, 128, 3, false>(mh, ml, mh, ml, o, p, 1, st, "hessian_syrk");
 }
 
 }  // namespace gqh
