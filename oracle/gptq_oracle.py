@@ -52,7 +52,6 @@ Readings of points the pages leave open (each is implemented below):
 
 from __future__ import annotations
 
-import math
 from dataclasses import dataclass
 
 import numpy as np
@@ -494,8 +493,3 @@ def quantize_layer(W0, X, bits=4, group_size=128, sym=False, block_size=128, dam
     U = hinv_upper_cholesky(Hd)
     res = gptq(W0, U, bits, group_size, sym, block_size)
     return res, H, U, lam
-
-
-def cond_estimate(Hd) -> float:
-    ev = np.linalg.eigvalsh(np.asarray(Hd, dtype=np.float64))
-    return float(ev[-1] / ev[0]) if ev[0] > 0 else math.inf
