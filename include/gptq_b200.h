@@ -175,6 +175,29 @@ void gptq_timing_enable(int on);
 size_t gptq_timing_report(char* buf, size_t len);
 gptq_status gptq_selftest_bounded_wait(uint64_t limit_ns, void* stream);
 
+/* ------------------------------------------------------------------ no-allocation variant
+ * gptq_hessian_accumulate_fixed_scratch: the same H (+)= 2 X^T X as
+ * gptq_hessian_accumulate, for callers that cannot hand the library a device
+ * workspace: a plain C program that links only this library and has no device
+ * allocator of its own, or a plug-in running inside a host application whose memory
+ * pool owns the whole device and forbids further cudaMalloc calls.  The pages have no
+ * counterpart to this entry point; it exists for those callers only.
+ *   - Scratch: a fixed 16 MiB array inside the library (16777216 bytes per GPU),
+ *     reserved on every GPU that loads the library until the process exits.  A batch
+ *     needs d_in * roundup(n, 64) * 2 bytes for bf16 X, or d_in * roundup(n, 64) * 8
+ *     bytes for fp32 X (two tf32 parts); a larger batch returns GPTQ_ERR_INVALID_ARG
+ *     with both sizes in gptq_last_error().  Split such a batch and call with
+ *     accumulate = 1.
+ *   - The first call on each device looks up the array's device address (a set-up the
+ *     library does once per device); make that first call before capturing any stream.
+ *   - All calls on one device share its array, which keeps the last call's contents.
+ *     Calls on one device that may overlap on the GPU (for example on two streams) race
+ *     and must be serialised by the caller.  Each call rewrites all of the scratch it
+ *     reads, so nothing needs clearing.
+ *   - Allocates no device or host memory; arguments as gptq_hessian_accumulate. */
+gptq_status gptq_hessian_accumulate_fixed_scratch(const void* X, gptq_dtype xt, int64_t n, int64_t d_in,
+                                                  float* H, int accumulate, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

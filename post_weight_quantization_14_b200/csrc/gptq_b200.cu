@@ -387,3 +387,104 @@ gptq_status gptq_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
 }
 
 }  // extern "C"
+
+// ============================================================================
+// Fixed-scratch Hessian accumulation (no device or host allocation).
+// The scratch for the transposed calibration batch lives in a file-scope device
+// array; host code must use its device address, taken with cudaGetSymbolAddress on
+// each device the first time this entry point runs there.
+// ============================================================================
+namespace gq {
+constexpr size_t kFixedHessScratchBytes = size_t(16) << 20;
+__device__ __align__(256) uint8_t g_fixed_hess_scratch[kFixedHessScratchBytes];
+}  // namespace gq
+
+namespace gqh {
+
+constexpr int kMaxDevices = 128;
+static void* g_fixed_hess_scratch_addr[kMaxDevices];  // zero-initialised; one slot per device ordinal
+
+// One GEMM launch with freshly encoded maps (no map cache, no timing bookkeeping).
+template <int KIND, int BN, int STAGES, bool PREFETCH_C>
+static cudaError_t fixed_gemm(const Mat& a, const Mat& a2, const Mat& c, gq::GemmArgs p, cudaStream_t st) {
+    using Cfg = gq::GemmCfg<KIND>;
+    const int eb = (KIND == gq::KIND_BF16) ? 2 : 4;
+    CUtensorMap ma, ma2, mc;
+    if (!encode_tmap_2d(&ma, a.ptr, eb, a.rows, a.cols, a.ld, 128, Cfg::KT)) return cudaErrorInvalidValue;
+    if (!encode_tmap_2d(&ma2, a2.ptr, eb, a2.rows, a2.cols, a2.ld, 128, Cfg::KT)) return cudaErrorInvalidValue;
+    if (!encode_tmap_2d(&mc, c.ptr, 4, c.rows, c.cols, c.ld, 32, 32)) return cudaErrorInvalidValue;
+    p.C = static_cast<float*>(const_cast<void*>(c.ptr));
+    p.ldc = (long long)c.ld;
+    p.tiles_m = (p.M + 127) / 128;
+    p.tiles_n = (p.N + BN - 1) / BN;
+    const long long tiles = (long long)p.tiles_m * (p.tiles_m + 1) / 2;
+    constexpr int smem = gq::gemm_smem_bytes<KIND, BN, STAGES, PREFETCH_C>();
+    auto kern = gq::tc_gemm_kernel<KIND, BN, STAGES, PREFETCH_C>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    // A and B are the same matrix (X^T); the epilogue writes C and its mirror
+    kern<<<dim3((unsigned)tiles, 1, 1), 192, smem, st>>>(ma, ma2, ma, ma2, mc, mc, mc, mc, mc, p);
+    return cudaGetLastError();
+}
+
+}  // namespace gqh
+
+extern "C" {
+
+gptq_status gptq_hessian_accumulate_fixed_scratch(const void* X, gptq_dtype xt, int64_t n, int64_t d_in, float* H,
+                                                  int accumulate, void* stream) {
+    if (!X || !H) return fail(GPTQ_ERR_INVALID_ARG, "X and H must be non-NULL");
+    if (xt != GPTQ_BF16 && xt != GPTQ_F32) return fail(GPTQ_ERR_INVALID_ARG, "unknown X dtype %d", (int)xt);
+    if (n < 1 || n > (1ll << 30)) return fail(GPTQ_ERR_INVALID_ARG, "n out of range (%lld)", (long long)n);
+    if (d_in < 8 || d_in > 65536 || d_in % 8) return fail(GPTQ_ERR_INVALID_ARG, "d_in must be a multiple of 8 in [8, 65536]");
+    if (!aligned16(X) || !aligned16(H)) return fail(GPTQ_ERR_INVALID_ARG, "X and H must be 16-byte aligned");
+    const size_t need = hessian_ws_bytes(n, d_in, xt);
+    if (need > gq::kFixedHessScratchBytes)
+        return fail(GPTQ_ERR_INVALID_ARG,
+                    "batch too large for the fixed scratch: needs %zu bytes, the library holds %zu; "
+                    "split the calibration batch or use gptq_hessian_accumulate with a workspace",
+                    need, gq::kFixedHessScratchBytes);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(GPTQ_ERR_INVALID_ARG, "device ordinal %d out of range", dev);
+    if (!g_fixed_hess_scratch_addr[dev]) {
+        void* addr = nullptr;
+        e = cudaGetSymbolAddress(&addr, gq::g_fixed_hess_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(fixed scratch)");
+        g_fixed_hess_scratch_addr[dev] = addr;
+    }
+    void* ws = g_fixed_hess_scratch_addr[dev];
+    cudaStream_t st = (cudaStream_t)stream;
+    const long long np = hess_npad(n);
+    dim3 tb(32, 8), grid((unsigned)(np / 32), (unsigned)((d_in + 31) / 32));
+    gq::GemmArgs p = gemm_args((int)d_in, (int)d_in, (int)np);
+    p.triangular = 1;
+    p.mirror = 1;
+    p.alpha = 2.f;
+    p.beta = accumulate ? 1.f : 0.f;
+    p.write_c = 1;
+    const Mat hm{H, (uint64_t)d_in, (uint64_t)d_in, (uint64_t)d_in};
+    if (xt == GPTQ_BF16) {
+        uint16_t* XT = static_cast<uint16_t*>(ws);
+        gq::transpose_bf16_kernel<<<grid, tb, 0, st>>>(static_cast<const uint16_t*>(X), n, d_in, np, XT);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "fixed-scratch transpose");
+        const Mat m{XT, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
+        e = accumulate ? fixed_gemm<gq::KIND_BF16, 128, 4, true>(m, m, hm, p, st)
+                       : fixed_gemm<gq::KIND_BF16, 128, 6, false>(m, m, hm, p, st);
+    } else {
+        float* hi = static_cast<float*>(ws);
+        float* lo = hi + d_in * np;
+        gq::transpose_split_f32_kernel<<<grid, tb, 0, st>>>(static_cast<const float*>(X), n, d_in, np, hi, lo);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "fixed-scratch transpose");
+        const Mat mh{hi, (uint64_t)d_in, (uint64_t)np, (uint64_t)np}, ml{lo, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
+        e = accumulate ? fixed_gemm<gq::KIND_TF32X3, 128, 2, true>(mh, ml, hm, p, st)
+                       : fixed_gemm<gq::KIND_TF32X3, 128, 3, false>(mh, ml, hm, p, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "fixed-scratch hessian");
+    return GPTQ_OK;
+}
+
+}  // extern "C"

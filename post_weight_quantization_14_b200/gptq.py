@@ -66,6 +66,7 @@ _SIGS = {
     "gptq_timing_enable": (None, [_int]),
     "gptq_timing_report": (_sz, [ctypes.c_char_p, _sz]),
     "gptq_selftest_bounded_wait": (_int, [ctypes.c_uint64, _vp]),
+    "gptq_hessian_accumulate_fixed_scratch": (_int, [_vp, _int, _i64, _i64, _vp, _int, _vp]),
 }
 
 
