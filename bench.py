@@ -141,18 +141,52 @@ def run_reference(args, rank: int, world: int) -> None:
 
 # ---------------------------------------------------------------- GPU leg
 
-def algorithmic_work(d_out: int, d_in: int, n: int) -> dict:
-    """Per-kernel-class algorithmic flops / bytes for one layer (roofline)."""
+CHOL_KERNELS = ("chol_leaf", "chol_panel", "chol_update", "inv_bu", "inv_ub", "split_panel", "damp_copy",
+                "diag_mean", "zero_lower")
+END_TO_END_BOUND_MS = 0.445   # sum of the stage bounds for this layer (roofline)
+
+
+def kernel_rooflines(kernel_ms: dict, launches: dict, hbm: float, bf16: float, peak_kind: str) -> dict:
+    """Achieved vs peak per kernel class, from algorithmic work and measured per-step time.
+
+    Algorithmic work (roofline table):
+      trailing_update  2 * d_out * (d_in - e) * 128 flops per launch, summed over the layer; 3xTF32
+      chol_panel/update, inv_*  2/3 d_in^3 flops for the whole factorization (shared); 3xTF32
+      hessian_syrk     n * d_in * (d_in + 1) flops; bf16
+      colloop          W read once + codes + scales/zeros written, bytes; HBM
+      chol_leaf        2/3 * 128^3 * 2 flops per 128x128 leaf (factor + inverse) on ONE SM; fp32 ALU
+    tf32 peak = measured bf16 x 1.1/2.25 (nominal ratio); 3xTF32 peak = a third of it.
+    """
     B = 128
-    nblk = (d_in + B - 1) // B
-    trailing_flops = sum(2.0 * d_out * (d_in - (b + 1) * B) * B for b in range(nblk) if (b + 1) * B < d_in)
+    d_out, d_in, n = D_OUT, D_IN, N_TOK
+    tf32x3 = bf16 * (1.1 / 2.25) / 3.0
+    sm_fp32 = 128 * 2 * 1.965e9 / 1e12            # one SM, TFLOP/s at max clock
+    out = {}
+    def add(name, bound, work, unit, peak, note):
+        ms = kernel_ms.get(name)
+        if not ms:
+            return
+        scale = 1e9 if unit == "GB/s" else 1e12
+        ach = work / (ms / 1e3) / scale
+        out[name] = {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+                     "traffic": None, "launches": launches.get(name), "note": note}
+    trailing = sum(2.0 * d_out * (d_in - (b + 1) * B) * B for b in range(d_in // B) if (b + 1) * B < d_in)
+    add("trailing_update", "tensor", trailing, "TFLOP/s", tf32x3, f"3xTF32 ({peak_kind} bf16 x 1.1/2.25 / 3)")
+    add("hessian_syrk", "tensor", 1.0 * n * d_in * (d_in + 1), "TFLOP/s", bf16, f"bf16 {peak_kind} burst")
     col_bytes = 4.0 * d_out * d_in + BITS / 8 * d_out * d_in + (2 + BITS / 8) * d_out * (d_in // GROUP)
-    return {
-        "trailing_update": ("tensor_tf32x3", trailing_flops),
-        "hessian_syrk": ("tensor_bf16", 1.0 * n * d_in * (d_in + 1)),
-        "colloop": ("hbm", col_bytes),
-        "chol": ("tensor_tf32x3", 2.0 / 3.0 * d_in ** 3),
-    }
+    add("colloop", "hbm", col_bytes, "GB/s", hbm, f"HBM {peak_kind}; latency chain of d_in rounding steps per row")
+    nleaf = d_in // B
+    add("chol_leaf", "alu", nleaf * 2.0 * (2.0 / 3.0) * B ** 3, "TFLOP/s", sm_fp32,
+        "one CTA per 128x128 leaf: peak = one SM's fp32 FMA rate at 1965 MHz")
+    gemm_ms = sum(kernel_ms.get(k, 0) for k in ("chol_panel", "chol_update", "inv_bu", "inv_ub"))
+    if gemm_ms:
+        ach = (2.0 / 3.0) * d_in ** 3 / (gemm_ms / 1e3) / 1e12
+        for k in ("chol_panel", "chol_update", "inv_bu", "inv_ub"):
+            if k in kernel_ms:
+                out[k] = {"bound": "tensor", "achieved": ach, "peak": tf32x3, "unit": "TFLOP/s", "frac": ach / tf32x3,
+                          "traffic": None, "launches": launches.get(k),
+                          "note": f"factorization GEMMs together ({gemm_ms:.3f} ms) vs 3xTF32"}
+    return out
 
 
 def main():
@@ -234,7 +268,7 @@ def main():
     G.gptq_timing_enable(True)
     G.gptq_timing_report()
     reps = 3
-    for _ in range(reps):
+    for _ in range(reps):  # instrumented steps (not part of the timed region)
         W.copy_(W0)
         flush.fill_(1)
         step()
@@ -245,40 +279,15 @@ def main():
     kernel_launches = {k: c // reps for k, (c, ms) in kt.items()}
 
     hbm, bf16, bf16_sus, peak_kind = peaks()
-    tf32 = bf16 * (1.1 / 2.25)                      # nominal tf32 : bf16 dense ratio
-    work = algorithmic_work(D_OUT, D_IN, N_TOK)
-    chol_ms = sum(v for k, v in kernel_ms.items() if k in ("chol_leaf", "chol_panel", "chol_update", "inv_bu",
-                                                           "inv_ub", "split_panel", "damp_copy", "diag_mean",
-                                                           "zero_lower"))
+    roof_all = kernel_rooflines(kernel_ms, kernel_launches, hbm, bf16, peak_kind)
     stage_ms = {"hessian": kernel_ms.get("hessian_syrk", 0) + kernel_ms.get("transpose_x", 0),
-                "prepare_hinv": chol_ms,
+                "prepare_hinv": sum(v for k, v in kernel_ms.items() if k in CHOL_KERNELS),
                 "quantize": sum(kernel_ms.get(k, 0) for k in ("colloop", "trailing_update", "up_prep", "ut_split",
                                                              "pack_zeros", "row_params"))}
-    dom = max(kernel_ms, key=kernel_ms.get)
-    def roof(name):
-        ms = kernel_ms.get(name, 0.0)
-        n = max(1, kernel_launches.get(name, 1))
-        if name == "trailing_update":
-            achieved = work[name][1] / (ms / 1e3) / 1e12
-            return {"bound": "tensor", "achieved": achieved, "peak": tf32 / 3, "unit": "TFLOP/s",
-                    "frac": achieved / (tf32 / 3), "traffic": None,
-                    "note": f"3xTF32: peak = measured bf16 x 1.1/2.25 / 3 ({peak_kind}); {n} launches"}
-        if name == "hessian_syrk":
-            achieved = work[name][1] / (ms / 1e3) / 1e12
-            return {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
-                    "frac": achieved / bf16, "traffic": None, "note": f"bf16 {peak_kind} burst peak"}
-        if name == "colloop":
-            achieved = work[name][1] / (ms / 1e3) / 1e9
-            return {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                    "traffic": None, "note": f"HBM {peak_kind}; {n} launches"}
-        if name in ("chol_leaf", "chol_update", "chol_panel", "inv_bu", "inv_ub"):
-            achieved = work["chol"][1] / (chol_ms / 1e3) / 1e12
-            return {"bound": "tensor", "achieved": achieved, "peak": tf32 / 3, "unit": "TFLOP/s",
-                    "frac": achieved / (tf32 / 3), "traffic": None,
-                    "note": f"whole factorization stage ({chol_ms:.3f} ms) vs 3xTF32 peak ({peak_kind})"}
-        return None
-    roofline = roof(dom) or roof("trailing_update")
+    dom = max((k for k in kernel_ms if k in roof_all), key=kernel_ms.get)
+    roofline = dict(roof_all[dom])
     roofline["kernel"] = dom
+    roofline["share_of_step"] = kernel_ms[dom] / max(1e-9, sum(kernel_ms.values()))
 
     # end-to-end through the public API with host buffers (pinned), copies inside the timed region
     W_host = torch.from_numpy(layer.W).pin_memory()
@@ -325,6 +334,8 @@ def main():
                            "l2": "flushed (256 MB write) before every step, outside the step events",
                            "parallelism": f"{world} independent layers, one per GPU"},
                 "roofline": roofline,
+                "roofline_by_kernel": roof_all,
+                "e2e_roofline": {"bound_ms": END_TO_END_BOUND_MS, "frac": END_TO_END_BOUND_MS / ms_per_step},
                 "stage_ms": stage_ms,
                 "kernel_ms_per_step": kernel_ms,
                 "kernel_launches_per_step": kernel_launches,

@@ -110,7 +110,6 @@ struct LeafSmem {
     float X[NB][LS];         // L^-1 (lower); upper blocks hold temporaries
     float LT[NB][LS];        // L transposed: LT[m][r] = L[r][m]
     float XDT[4][32][36];    // diagonal inverses transposed: XDT[kb][m][j] = X_kk[j][m]
-    float rowbuf[2][64];     // broadcast of the current pivot row (p part, x part)
 };
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
@@ -146,45 +145,19 @@ __global__ void __launch_bounds__(512, 1)
             float my_rinv = 0.f;
 #pragma unroll
             for (int k = 0; k < 32; ++k) {
+                // pivot row k (unscaled) is broadcast element by element with shuffles
                 const float piv = __shfl_sync(FULL, pr[k], k);
                 if (lane == 0 && !(piv > 0.f && isfinite(piv)))
                     record_status(isfinite(piv) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE, jb + 127 - (k0 + k));
                 const float rinv = rsqrtf(piv);
-                float* rb = S.rowbuf[k & 1];
-                if (lane == k) {
-                    my_rinv = rinv;
+                const bool below = lane > k;
+                const float f = below ? pr[k] * rinv * rinv : 0.f;   // P_ik / P_kk
+                my_rinv = (lane == k) ? rinv : my_rinv;
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        if (4 * q + 3 > k)
-                            *reinterpret_cast<float4*>(rb + 4 * q) =
-                                make_float4(pr[4 * q], pr[4 * q + 1], pr[4 * q + 2], pr[4 * q + 3]);
-                        if (4 * q <= k)
-                            *reinterpret_cast<float4*>(rb + 32 + 4 * q) =
-                                make_float4(xr[4 * q], xr[4 * q + 1], xr[4 * q + 2], xr[4 * q + 3]);
-                    }
-                }
-                __syncwarp();
-                if (lane > k) {
-                    const float f = pr[k] * rinv * rinv;   // P_ik / P_kk
+                for (int j = k + 1; j < 32; ++j) pr[j] = fmaf(-f, __shfl_sync(FULL, pr[j], k), pr[j]);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        if (4 * q + 3 > k) {
-                            const float4 v = ld4(rb + 4 * q);
-                            if (4 * q + 0 > k) pr[4 * q + 0] = fmaf(-f, v.x, pr[4 * q + 0]);
-                            if (4 * q + 1 > k) pr[4 * q + 1] = fmaf(-f, v.y, pr[4 * q + 1]);
-                            if (4 * q + 2 > k) pr[4 * q + 2] = fmaf(-f, v.z, pr[4 * q + 2]);
-                            pr[4 * q + 3] = fmaf(-f, v.w, pr[4 * q + 3]);
-                        }
-                        if (4 * q <= k) {
-                            const float4 v = ld4(rb + 32 + 4 * q);
-                            xr[4 * q + 0] = fmaf(-f, v.x, xr[4 * q + 0]);
-                            if (4 * q + 1 <= k) xr[4 * q + 1] = fmaf(-f, v.y, xr[4 * q + 1]);
-                            if (4 * q + 2 <= k) xr[4 * q + 2] = fmaf(-f, v.z, xr[4 * q + 2]);
-                            if (4 * q + 3 <= k) xr[4 * q + 3] = fmaf(-f, v.w, xr[4 * q + 3]);
-                        }
-                    }
-                    pr[k] *= rinv;   // L[lane][k] = P_ik / sqrt(P_kk)
-                }
+                for (int j = 0; j <= k; ++j) xr[j] = fmaf(-f, __shfl_sync(FULL, xr[j], k), xr[j]);
+                if (below) pr[k] *= rinv;   // L[lane][k] = P_ik / sqrt(P_kk)
             }
             // lane i: L[i][j] = pr[j] (j < i), L[i][i] = pivot * rinv, row i of L^-1 = rinv * xr
 #pragma unroll
@@ -329,9 +302,10 @@ __global__ void __launch_bounds__(512, 1)
                 if (gc + i < d) U[gr * d + gc + i] = v[i];
         }
     }
-    // UT[c][r] = U[r][c] = X[127-r][127-c] = L^-1 read along a column of X
+    // UT[c][r..r+3] = U[r..r+3][c] = X[127-r-i][127-c]; consecutive lanes take consecutive c
+    // so the shared-memory reads run along rows of X (conflict-free)
     for (int task = tid; task < NB * 32; task += blockDim.x) {
-        const int c = task >> 5, r = (task & 31) * 4;
+        const int r = (task >> 7) * 4, c = task & 127;
         float v[4], h[4], l[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) v[i] = (r + i <= c) ? S.X[127 - r - i][127 - c] : 0.f;
@@ -420,7 +394,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
         }
         GQ_TRY(cudaGetLastError());
         if (j == 0) break;
-        {
+        if (j == T - 1) {   // later panels are split by the previous update's epilogue
             gqh::TimedScope ts__("split_panel", st);
             gq::split_panel_kernel<<<(unsigned)std::min<long long>((jb * 128LL + 255) / 256, 4096), 256, 0, st>>>(
                 w.A, n, jb, jb, w.AP_hi, w.AP_lo);
@@ -448,6 +422,12 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
             p.write_c = 1;
             EpiMats o;
             o.c = Mat{w.A, N, N, N};
+            if (j >= 2) {   // tiles of block column j-1 above its diagonal also write the next panel's split
+                p.s_tile_n = j - 1;
+                p.s_col0 = -(j - 1) * gq::NB;
+                o.s_hi = Mat{w.AP_hi, (uint64_t)(jb - gq::NB), 128, 128};
+                o.s_lo = Mat{w.AP_lo, (uint64_t)(jb - gq::NB), 128, 128};
+            }
             Mat rh{w.RS_hi, N, N, N}, rl{w.RS_lo, N, N, N};
             GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 2, true>(rh, rl, rh, rl, o, p, 1, st, "chol_update")));
         }

@@ -48,6 +48,7 @@ struct GemmArgs {
     float* S_lo;
     long long lds;
     int s_row0, s_col0, s_zrow, s_zcol;
+    int s_tile_n;     // if > 0: S written only by tiles with nt == s_tile_n and mt < nt
     float* T_hi;
     float* T_lo;
     long long ldt;
@@ -234,7 +235,8 @@ __global__ void __launch_bounds__(192, 1)
             // TMA epilogue
             const int q = warp & 3;
             const bool mirror = p.mirror && nt > mt;
-            const bool has_c = p.write_c != 0, has_s = p.S_hi != nullptr, has_t = p.T_hi != nullptr;
+            const bool has_c = p.write_c != 0, has_t = p.T_hi != nullptr;
+            const bool has_s = p.S_hi != nullptr && (p.s_tile_n <= 0 || (nt == p.s_tile_n && mt < nt));
             const int nkinds = (has_c ? 1 : 0) + (has_s ? 2 : 0) + (has_t ? 2 : 0) + (mirror ? 1 : 0);
             const int kc = 0, ks = kc + (has_c ? 1 : 0), kt = ks + (has_s ? 2 : 0), km = kt + (has_t ? 2 : 0);
             const bool use_cin = PREFETCH_C && p.beta != 0.f;
