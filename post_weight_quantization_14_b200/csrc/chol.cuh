@@ -410,7 +410,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
             o.s_lo = Mat{w.RS_lo, N, N, N};
             Mat ah{w.AP_hi, (uint64_t)jb, 128, 128}, al{w.AP_lo, (uint64_t)jb, 128, 128};
             Mat bh{w.U_hi, N, N, N}, bl{w.U_lo, N, N, N};
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 3, false>(ah, al, bh, bl, o, p, 1, st, "chol_panel")));
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(ah, al, bh, bl, o, p, 1, st, "chol_panel")));
         }
         {   // update: A[0:jb, 0:jb] -= RS_panel RS_panel^T (upper tiles)
             gq::GemmArgs p = gemm_args(jb, jb, gq::NB);
@@ -429,7 +429,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
                 o.s_lo = Mat{w.AP_lo, (uint64_t)(jb - gq::NB), 128, 128};
             }
             Mat rh{w.RS_hi, N, N, N}, rl{w.RS_lo, N, N, N};
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 2, true>(rh, rl, rh, rl, o, p, 1, st, "chol_update")));
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(rh, rl, rh, rl, o, p, 1, st, "chol_update")));
         }
     }
     // U = R^-1 by doubling
@@ -469,7 +469,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
                 EpiMats o;
                 o.t_hi = Mat{w.TT_hi, N, N, N};
                 o.t_lo = Mat{w.TT_lo, N, N, N};
-                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 3, false>(rsh, rsl, uth, utl, o, p, (int)batch, st, "inv_bu")));
+                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(rsh, rsl, uth, utl, o, p, (int)batch, st, "inv_bu")));
             }
             {   // U_b = -U_a T -> U (public, clipped), U split, UT split
                 gq::GemmArgs p = gemm_args((int)s, (int)cs, (int)s);
@@ -484,8 +484,6 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
                 p.c_row0 = (int)r0;
                 p.c_col0 = (int)(r0 + s);
                 p.c_zrow = p.c_zcol = zs;
-                p.c_lim_rows = (int)d;
-                p.c_lim_cols = (int)d;
                 p.write_c = 1;
                 p.s_row0 = (int)r0;
                 p.s_col0 = (int)(r0 + s);
@@ -499,7 +497,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
                 o.s_lo = Mat{w.U_lo, N, N, N};
                 o.t_hi = Mat{w.UT_hi, N, N, N};
                 o.t_lo = Mat{w.UT_lo, N, N, N};
-                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 3, false>(uh, ul, tth, ttl, o, p, (int)batch, st, "inv_ub")));
+                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(uh, ul, tth, ttl, o, p, (int)batch, st, "inv_ub")));
             }
         }
     }

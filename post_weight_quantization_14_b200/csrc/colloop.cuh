@@ -463,7 +463,7 @@ cudaError_t quant_run_bits(float* W, const float* U, long long d_out, long long 
             p.write_c = 1;
             EpiMats o;
             o.c = Mat{W, (uint64_t)d_out, (uint64_t)d_in, (uint64_t)d_in};
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 128, 2, true>(eh, el, uh, ul, o, p, 1, st, "trailing_update")));
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(eh, el, uh, ul, o, p, 1, st, "trailing_update")));
         }
     }
     if (!cfg.sym && qzeros) {

@@ -102,6 +102,18 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t r
     return true;
 }
 
+int num_sms() {
+    static int cache[128];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+    if (!cache[dev]) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        cache[dev] = v;
+    }
+    return cache[dev];
+}
+
 cudaError_t ensure_smem_attr(const void* func, int bytes) {
     static std::set<std::tuple<const void*, int, int>> done;
     int dev = 0;
@@ -405,25 +417,31 @@ constexpr int kMaxDevices = 128;
 static void* g_fixed_hess_scratch_addr[kMaxDevices];  // zero-initialised; one slot per device ordinal
 
 // One GEMM launch with freshly encoded maps (no map cache, no timing bookkeeping).
-template <int KIND, int BN, int STAGES, bool PREFETCH_C>
+template <int KIND, int STAGES>
 static cudaError_t fixed_gemm(const Mat& a, const Mat& a2, const Mat& c, gq::GemmArgs p, cudaStream_t st) {
     using Cfg = gq::GemmCfg<KIND>;
     const int eb = (KIND == gq::KIND_BF16) ? 2 : 4;
     CUtensorMap ma, ma2, mc;
-    if (!encode_tmap_2d(&ma, a.ptr, eb, a.rows, a.cols, a.ld, 128, Cfg::KT)) return cudaErrorInvalidValue;
-    if (!encode_tmap_2d(&ma2, a2.ptr, eb, a2.rows, a2.cols, a2.ld, 128, Cfg::KT)) return cudaErrorInvalidValue;
+    if (!encode_tmap_2d(&ma, a.ptr, eb, a.rows, a.cols, a.ld, gq::BM, Cfg::KT)) return cudaErrorInvalidValue;
+    if (!encode_tmap_2d(&ma2, a2.ptr, eb, a2.rows, a2.cols, a2.ld, gq::BM, Cfg::KT)) return cudaErrorInvalidValue;
     if (!encode_tmap_2d(&mc, c.ptr, 4, c.rows, c.cols, c.ld, 32, 32)) return cudaErrorInvalidValue;
     p.C = static_cast<float*>(const_cast<void*>(c.ptr));
     p.ldc = (long long)c.ld;
-    p.tiles_m = (p.M + 127) / 128;
-    p.tiles_n = (p.N + BN - 1) / BN;
+    p.tiles_m = (p.M + gq::BM - 1) / gq::BM;
+    p.tiles_n = (p.N + gq::BN - 1) / gq::BN;
+    p.batch = 1;
     const long long tiles = (long long)p.tiles_m * (p.tiles_m + 1) / 2;
-    constexpr int smem = gq::gemm_smem_bytes<KIND, BN, STAGES, PREFETCH_C>();
-    auto kern = gq::tc_gemm_kernel<KIND, BN, STAGES, PREFETCH_C>;
+    constexpr int smem = gq::gemm_smem_bytes<KIND, STAGES>();
+    auto kern = gq::tc_gemm_kernel<KIND, STAGES>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    int sms = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
     // A and B are the same matrix (X^T); the epilogue writes C and its mirror
-    kern<<<dim3((unsigned)tiles, 1, 1), 192, smem, st>>>(ma, ma2, ma, ma2, mc, mc, mc, mc, mc, p);
+    kern<<<dim3((unsigned)std::min<long long>(tiles, sms), 1, 1), 192, smem, st>>>(ma, ma2, ma, ma2, mc, mc, mc, mc, mc,
+                                                                                     p);
     return cudaGetLastError();
 }
 
@@ -471,8 +489,7 @@ gptq_status gptq_hessian_accumulate_fixed_scratch(const void* X, gptq_dtype xt, 
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "fixed-scratch transpose");
         const Mat m{XT, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
-        e = accumulate ? fixed_gemm<gq::KIND_BF16, 128, 4, true>(m, m, hm, p, st)
-                       : fixed_gemm<gq::KIND_BF16, 128, 6, false>(m, m, hm, p, st);
+        e = fixed_gemm<gq::KIND_BF16, 4>(m, m, hm, p, st);
     } else {
         float* hi = static_cast<float*>(ws);
         float* lo = hi + d_in * np;
@@ -480,8 +497,7 @@ gptq_status gptq_hessian_accumulate_fixed_scratch(const void* X, gptq_dtype xt, 
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "fixed-scratch transpose");
         const Mat mh{hi, (uint64_t)d_in, (uint64_t)np, (uint64_t)np}, ml{lo, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
-        e = accumulate ? fixed_gemm<gq::KIND_TF32X3, 128, 2, true>(mh, ml, hm, p, st)
-                       : fixed_gemm<gq::KIND_TF32X3, 128, 3, false>(mh, ml, hm, p, st);
+        e = fixed_gemm<gq::KIND_TF32X3, 2>(mh, ml, hm, p, st);
     }
     if (e != cudaSuccess) return cuda_fail(e, "fixed-scratch hessian");
     return GPTQ_OK;
