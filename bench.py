@@ -141,8 +141,8 @@ def run_reference(args, rank: int, world: int) -> None:
 
 # ---------------------------------------------------------------- GPU leg
 
-CHOL_KERNELS = ("chol_leaf", "chol_panel", "chol_update", "inv_bu", "inv_ub", "split_panel", "damp_copy",
-                "diag_mean", "zero_lower")
+CHOL_KERNELS = ("chol_leaf", "chol_panel", "chol_update", "chol_update_next", "inv_bu", "inv_ub", "split_panel",
+                "damp_copy", "diag_mean", "zero_lower")
 END_TO_END_BOUND_MS = 0.445   # sum of the stage bounds for this layer (roofline)
 
 
@@ -178,10 +178,10 @@ def kernel_rooflines(kernel_ms: dict, launches: dict, hbm: float, bf16: float, p
     nleaf = d_in // B
     add("chol_leaf", "alu", nleaf * 2.0 * (2.0 / 3.0) * B ** 3, "TFLOP/s", sm_fp32,
         "one CTA per 128x128 leaf: peak = one SM's fp32 FMA rate at 1965 MHz")
-    gemm_ms = sum(kernel_ms.get(k, 0) for k in ("chol_panel", "chol_update", "inv_bu", "inv_ub"))
+    gemm_ms = sum(kernel_ms.get(k, 0) for k in ("chol_panel", "chol_update", "chol_update_next", "inv_bu", "inv_ub"))
     if gemm_ms:
         ach = (2.0 / 3.0) * d_in ** 3 / (gemm_ms / 1e3) / 1e12
-        for k in ("chol_panel", "chol_update", "inv_bu", "inv_ub"):
+        for k in ("chol_panel", "chol_update", "chol_update_next", "inv_bu", "inv_ub"):
             if k in kernel_ms:
                 out[k] = {"bound": "tensor", "achieved": ach, "peak": tf32x3, "unit": "TFLOP/s", "frac": ach / tf32x3,
                           "traffic": None, "launches": launches.get(k),

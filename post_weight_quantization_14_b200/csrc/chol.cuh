@@ -81,7 +81,7 @@ __global__ void split_panel_kernel(const float* __restrict__ A, long long n, int
 }
 
 // Zero the strictly-lower 128-blocks of the d x d output U (diagonal blocks are
-// written in full by the leaf kernel).
+// written in full by chol_diag_out_kernel).
 __global__ void zero_lower_blocks_kernel(float* __restrict__ U, long long d) {
     const long long total = d * d;
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
@@ -94,197 +94,235 @@ __global__ void zero_lower_blocks_kernel(float* __restrict__ U, long long d) {
 // Leaf: factor and invert one 128x128 diagonal block of A in shared memory.
 // Works on the index-reversed block P = J A_jj J, for which the UL factor becomes an
 // ordinary lower Cholesky factor: A_jj = R R^T with R = J L J, and X_jj = R^-1 = J L^-1 J.
-// Blocked by 32.  For each diagonal 32-block one warp runs Gaussian elimination on
-// [P_kk | I] with unscaled pivot rows (lane = row): afterwards L_kk = L_u D^1/2 and
-// L_kk^-1 = D^-1/2 E, where E is the accumulated row-operation matrix.  All warps then
-// form the panel L_rk = P_rk L_kk^-T and the rank-32 update of the trailing lower
-// triangle, on 4x4 register micro-tiles fed from transposed copies of L and of the
-// diagonal inverses.  The inverse is assembled along block diagonals:
-// X_ij = -X_ii sum_{k=j}^{i-1} L_ik X_kj.
-// Writes X_jj (upper, zeros below the diagonal) to the public U (clipped to d), its
-// row-major tf32 split (U_hi/U_lo) and its transposed split (UT_hi/UT_lo).
+//
+// Right-looking, blocked by 32 columns.  Panel kb (columns k0 = 32 kb .. k0 + 31, rows
+// k0 .. 127) is eliminated by the 4 - kb warps that own its rows (one row per lane, the
+// row's 32 panel entries in registers): at step k the warp holding the diagonal block
+// publishes the current column k of that block in shared memory, and every row r does
+// L_rk = P_rk / sqrt(P_kk) and P_rj -= P_rk P_jk / P_kk for j > k, with one named
+// barrier per step.  All warps then apply the rank-32 update of the trailing lower
+// triangle on 4x4 register micro-tiles.  Meanwhile the warps not in the elimination
+// build the inverse X = L^-1 block row by block row, one row behind:
+// X_ii = L_ii^-1 by forward substitution (lane = column), T_ij = sum_{k=j}^{i-1} L_ik X_kj,
+// X_ij = -X_ii T_ij.
+// Writes X_jj (upper, zeros below the diagonal) as U_hi = tf32(X_jj) and U_lo = X_jj - U_hi
+// (exact, not rounded: the tensor pipe reads only its tf32 part); U_hi + U_lo restores
+// X_jj exactly for chol_diag_out_kernel.
 constexpr int LS = NB + 4;   // leaf smem row stride (16-byte aligned rows)
+constexpr int LEAF_THREADS = 512;
+static_assert(NB * NB / 4 == 8 * LEAF_THREADS && NB * 32 == 8 * LEAF_THREADS, "leaf load and store loops");
 
 struct LeafSmem {
-    float P[NB][LS];         // reversed block; lower triangle holds L after the factorization
-    float X[NB][LS];         // L^-1 (lower); upper blocks hold temporaries
+    float P[NB][LS];         // reversed block; lower triangle holds the Schur complement
+    float X[NB][LS];         // L^-1 (lower); blocks above the diagonal hold T
     float LT[NB][LS];        // L transposed: LT[m][r] = L[r][m]
-    float XDT[4][32][36];    // diagonal inverses transposed: XDT[kb][m][j] = X_kk[j][m]
+    float XDT[4][32][36];    // diagonal inverses transposed: XDT[i][m][r] = X_ii[r][m]
+    float col[2][32];        // pivot column of the current step (double-buffered)
 };
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
-__global__ void __launch_bounds__(512, 1)
-    chol_leaf_kernel(const float* __restrict__ A, long long n, long long d, int jb, float* __restrict__ U,
-                     float* __restrict__ U_hi, float* __restrict__ U_lo, float* __restrict__ UT_hi,
-                     float* __restrict__ UT_lo) {
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Eliminate panel k0 .. k0+31 with nw warps (barrier 1); warp w owns rows k0 + 32 w + lane.
+__device__ __forceinline__ void leaf_eliminate(LeafSmem& S, int k0, int nw, int warp, int lane, int jb) {
+    const int r = k0 + 32 * warp + lane;
+    const bool dg = warp == 0;   // the warp holding the diagonal 32x32 block
+    float pr[32];
+#pragma unroll
+    for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 v = ld4(&S.P[r][k0 + 4 * j4]);
+        pr[4 * j4 + 0] = v.x;
+        pr[4 * j4 + 1] = v.y;
+        pr[4 * j4 + 2] = v.z;
+        pr[4 * j4 + 3] = v.w;
+    }
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        float* cb = S.col[k & 1];
+        if (dg) cb[lane] = pr[k];   // column k of the diagonal block (rows >= k are valid)
+        named_bar(1, nw * 32);
+        const float piv = cb[k];
+        if (dg && lane == 0 && !(piv > 0.f && isfinite(piv)))
+            record_status(isfinite(piv) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE, jb + 127 - (k0 + k));
+        const float rinv = rsqrtf(piv);
+        const float f = pr[k] * (rinv * rinv);   // P_rk / P_kk
+#pragma unroll
+        for (int j4 = (k + 1) >> 2; j4 < 8; ++j4) {
+            const float4 c4 = ld4(&cb[4 * j4]);
+            if (4 * j4 + 0 > k) pr[4 * j4 + 0] = fmaf(-f, c4.x, pr[4 * j4 + 0]);
+            if (4 * j4 + 1 > k) pr[4 * j4 + 1] = fmaf(-f, c4.y, pr[4 * j4 + 1]);
+            if (4 * j4 + 2 > k) pr[4 * j4 + 2] = fmaf(-f, c4.z, pr[4 * j4 + 2]);
+            if (4 * j4 + 3 > k) pr[4 * j4 + 3] = fmaf(-f, c4.w, pr[4 * j4 + 3]);
+        }
+        pr[k] *= rinv;   // L_rk (L_kk = sqrt(P_kk) on the diagonal)
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) S.LT[k0 + j][r] = (dg && j > lane) ? 0.f : pr[j];
+}
+
+// Rank-32 update of the trailing lower triangle (rows and columns >= k0 + 32) with the
+// panel just eliminated; 4x4 micro-tiles on the lower triangle of tiles only.
+__device__ __forceinline__ void leaf_trailing_update(LeafSmem& S, int k0, int tid) {
+    const int t0 = k0 + 32, tn = (NB - t0) >> 2;
+    const int ntask = tn * (tn + 1) / 2;
+    for (int task = tid; task < ntask; task += LEAF_THREADS) {
+        int tr = (int)((sqrtf(8.f * (float)task + 1.f) - 1.f) * 0.5f);
+        while (tr * (tr + 1) / 2 > task) --tr;
+        while ((tr + 1) * (tr + 2) / 2 <= task) ++tr;
+        const int tc = task - tr * (tr + 1) / 2;
+        const int r0 = t0 + 4 * tr, c0 = t0 + 4 * tc;
+        float acc[4][4] = {};
+#pragma unroll 8
+        for (int m = 0; m < 32; ++m) {
+            const float4 a = ld4(&S.LT[k0 + m][r0]);
+            const float4 b = ld4(&S.LT[k0 + m][c0]);
+            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float4 pv = ld4(&S.P[r0 + i][c0]);
+            pv.x -= acc[i][0];
+            pv.y -= acc[i][1];
+            pv.z -= acc[i][2];
+            pv.w -= acc[i][3];
+            *reinterpret_cast<float4*>(&S.P[r0 + i][c0]) = pv;
+        }
+    }
+}
+
+// X_ii = L_ii^-1 by forward substitution, one warp, lane = column j:
+// x_m = (delta_mj - sum_{m' < m} L_mm' x_m') / L_mm.
+__device__ __forceinline__ void leaf_diag_inverse(LeafSmem& S, int i, int lane) {
+    const int k0 = 32 * i;
+    float x[32], s[32];
+#pragma unroll
+    for (int m = 0; m < 32; ++m) s[m] = 0.f;
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
+        const float dinv = __frcp_rn(S.LT[k0 + m][k0 + m]);
+        x[m] = (((m == lane) ? 1.f : 0.f) - s[m]) * dinv;
+#pragma unroll
+        for (int q4 = (m + 1) >> 2; q4 < 8; ++q4) {
+            const float4 l4 = ld4(&S.LT[k0 + m][k0 + 4 * q4]);   // L_{q,m} for q = 4 q4 ..
+            if (4 * q4 + 0 > m) s[4 * q4 + 0] = fmaf(l4.x, x[m], s[4 * q4 + 0]);
+            if (4 * q4 + 1 > m) s[4 * q4 + 1] = fmaf(l4.y, x[m], s[4 * q4 + 1]);
+            if (4 * q4 + 2 > m) s[4 * q4 + 2] = fmaf(l4.z, x[m], s[4 * q4 + 2]);
+            if (4 * q4 + 3 > m) s[4 * q4 + 3] = fmaf(l4.w, x[m], s[4 * q4 + 3]);
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < 32; ++m) S.X[k0 + m][k0 + lane] = x[m];
+#pragma unroll
+    for (int m4 = 0; m4 < 8; ++m4)
+        *reinterpret_cast<float4*>(&S.XDT[i][lane][4 * m4]) =
+            make_float4(x[4 * m4], x[4 * m4 + 1], x[4 * m4 + 2], x[4 * m4 + 3]);
+}
+
+// Block row i of X = L^-1 by a group of g warps (group warp gw, barrier 2):
+// group warp 0 forms X_ii while the others form T_ij = sum_{k=j}^{i-1} L_ik X_kj (stored in
+// X's block (j, i)); then all form X_ij = -X_ii T_ij for j < i.
+__device__ __forceinline__ void leaf_x_block_row(LeafSmem& S, int i, int gw, int g, int lane) {
+    if (gw == 0) {
+        leaf_diag_inverse(S, i, lane);
+    } else if (i > 0) {
+        const int gt = (gw - 1) * 32 + lane, gn = (g - 1) * 32;
+        for (int task = gt; task < 64 * i; task += gn) {
+            const int jbk = task >> 6, tr = (task >> 3) & 7, tc = task & 7;
+            const int r0 = 4 * tr, c0 = 4 * tc;
+            float acc[4][4] = {};
+#pragma unroll 4
+            for (int m = 32 * jbk; m < 32 * i; ++m) {
+                const float4 a = ld4(&S.LT[m][32 * i + r0]);
+                const float4 b = ld4(&S.X[m][32 * jbk + c0]);
+                const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                *reinterpret_cast<float4*>(&S.X[32 * jbk + r0 + u][32 * i + c0]) =
+                    make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+        }
+    }
+    if (i == 0) return;
+    named_bar(2, g * 32);
+    const int gt = gw * 32 + lane, gn = g * 32;
+    for (int task = gt; task < 64 * i; task += gn) {
+        const int jbk = task >> 6, tr = (task >> 3) & 7, tc = task & 7;
+        const int r0 = 4 * tr, c0 = 4 * tc;
+        float acc[4][4] = {};
+#pragma unroll 8
+        for (int m = 0; m < 32; ++m) {
+            const float4 a = ld4(&S.XDT[i][m][r0]);
+            const float4 b = ld4(&S.X[32 * jbk + m][32 * i + c0]);
+            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<float4*>(&S.X[32 * i + r0 + u][32 * jbk + c0]) =
+                make_float4(-acc[u][0], -acc[u][1], -acc[u][2], -acc[u][3]);
+    }
+}
+
+__global__ void __launch_bounds__(LEAF_THREADS, 1)
+    chol_leaf_kernel(const float* __restrict__ A, long long n, int jb, float* __restrict__ U_hi,
+                     float* __restrict__ U_lo) {
     extern __shared__ __align__(16) uint8_t leaf_raw[];
     LeafSmem& S = *reinterpret_cast<LeafSmem*>(leaf_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    constexpr unsigned FULL = 0xffffffffu;
 
-    // P[127-r][127-c] = A[r][c]: coalesced reads of the whole diagonal tile (both
-    // triangles were updated); only P's lower triangle (A's upper) is used.
-    for (int e = tid; e < NB * NB; e += blockDim.x) {
-        const int r = e >> 7, c = e & 127;
-        S.P[127 - r][127 - c] = A[(long long)(jb + r) * n + jb + c];
-        S.X[r][c] = 0.f;
+    // P[127-r][127-c] = A[r][c]: the whole diagonal tile, in two halves whose loads are all
+    // issued before their stores
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        float4 v[4];
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int e = tid + (4 * half + it) * LEAF_THREADS, r = e >> 5, c = (e & 31) * 4;
+            v[it] = *reinterpret_cast<const float4*>(A + (long long)(jb + r) * n + jb + c);
+        }
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int e = tid + (4 * half + it) * LEAF_THREADS, r = e >> 5, c = (e & 31) * 4;
+            S.P[127 - r][127 - c] = v[it].x;
+            S.P[127 - r][126 - c] = v[it].y;
+            S.P[127 - r][125 - c] = v[it].z;
+            S.P[127 - r][124 - c] = v[it].w;
+        }
     }
     __syncthreads();
 
     for (int kb = 0; kb < 4; ++kb) {
-        const int k0 = kb * 32;
-        if (warp == 0) {
-            // (a) elimination of [P_kk | I] with unscaled pivot rows; lane = row
-            float pr[32], xr[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                pr[j] = (j <= lane) ? S.P[k0 + lane][k0 + j] : S.P[k0 + j][k0 + lane];
-                xr[j] = (j == lane) ? 1.f : 0.f;
-            }
-            float my_rinv = 0.f;
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                // pivot row k (unscaled) is broadcast element by element with shuffles
-                const float piv = __shfl_sync(FULL, pr[k], k);
-                if (lane == 0 && !(piv > 0.f && isfinite(piv)))
-                    record_status(isfinite(piv) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE, jb + 127 - (k0 + k));
-                const float rinv = rsqrtf(piv);
-                const bool below = lane > k;
-                const float f = below ? pr[k] * rinv * rinv : 0.f;   // P_ik / P_kk
-                my_rinv = (lane == k) ? rinv : my_rinv;
-#pragma unroll
-                for (int j = k + 1; j < 32; ++j) pr[j] = fmaf(-f, __shfl_sync(FULL, pr[j], k), pr[j]);
-#pragma unroll
-                for (int j = 0; j <= k; ++j) xr[j] = fmaf(-f, __shfl_sync(FULL, xr[j], k), xr[j]);
-                if (below) pr[k] *= rinv;   // L[lane][k] = P_ik / sqrt(P_kk)
-            }
-            // lane i: L[i][j] = pr[j] (j < i), L[i][i] = pivot * rinv, row i of L^-1 = rinv * xr
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                if (j <= lane) {
-                    const float lij = (j == lane) ? pr[j] * my_rinv : pr[j];
-                    const float xij = xr[j] * my_rinv;
-                    S.P[k0 + lane][k0 + j] = lij;
-                    S.LT[k0 + j][k0 + lane] = lij;
-                    S.X[k0 + lane][k0 + j] = xij;
-                    S.XDT[kb][j][lane] = xij;
-                } else {
-                    S.XDT[kb][j][lane] = 0.f;
-                }
-            }
-        }
+        const int nw = 4 - kb;
+        if (warp < nw)
+            leaf_eliminate(S, 32 * kb, nw, warp, lane, jb);
+        else if (kb > 0)
+            leaf_x_block_row(S, kb - 1, warp - nw, 16 - nw, lane);
         __syncthreads();
         if (kb == 3) break;
-        const int t0 = k0 + 32;
-        const int rows = NB - t0;
-        // (b) panel: L[r][k0+j] = sum_m P[r][k0+m] X_kk[j][m]; task = (row, 4 columns)
-        for (int base = 0; base < rows * 8; base += 512) {
-            const int task = base + tid;
-            const int r = t0 + (task >> 3), j4 = (task & 7) * 4;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (task < rows * 8) {
-#pragma unroll 8
-                for (int m = 0; m < 32; ++m) {
-                    const float pv = S.P[r][k0 + m];
-                    const float4 xv = ld4(&S.XDT[kb][m][j4]);
-                    acc.x = fmaf(pv, xv.x, acc.x);
-                    acc.y = fmaf(pv, xv.y, acc.y);
-                    acc.z = fmaf(pv, xv.z, acc.z);
-                    acc.w = fmaf(pv, xv.w, acc.w);
-                }
-            }
-            __syncwarp();
-            if (task < rows * 8) {
-                *reinterpret_cast<float4*>(&S.P[r][k0 + j4]) = acc;
-                S.LT[k0 + j4 + 0][r] = acc.x;
-                S.LT[k0 + j4 + 1][r] = acc.y;
-                S.LT[k0 + j4 + 2][r] = acc.z;
-                S.LT[k0 + j4 + 3][r] = acc.w;
-            }
-        }
-        __syncthreads();
-        // (c) trailing update of the lower triangle on 4x4 micro-tiles
-        {
-            const int T = rows >> 2;
-            for (int task = tid; task < T * T; task += blockDim.x) {
-                const int tr = task / T, tc = task % T;
-                if (tc > tr) continue;
-                const int r0 = t0 + 4 * tr, c0 = t0 + 4 * tc;
-                float acc[4][4] = {};
-#pragma unroll 4
-                for (int m = 0; m < 32; ++m) {
-                    const float4 a = ld4(&S.LT[k0 + m][r0]);
-                    const float4 b = ld4(&S.LT[k0 + m][c0]);
-                    const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float4 pv = ld4(&S.P[r0 + i][c0]);
-                    pv.x -= acc[i][0];
-                    pv.y -= acc[i][1];
-                    pv.z -= acc[i][2];
-                    pv.w -= acc[i][3];
-                    *reinterpret_cast<float4*>(&S.P[r0 + i][c0]) = pv;
-                }
-            }
-        }
+        leaf_trailing_update(S, 32 * kb, tid);
         __syncthreads();
     }
-
-    // inverse blocks below the diagonal, by block diagonals dd = i - j, 4x4 micro-tiles
-    for (int dd = 1; dd < 4; ++dd) {
-        const int nblk = 4 - dd;
-        for (int task = tid; task < nblk * 64; task += blockDim.x) {
-            // T_ij = sum_{m'=32j}^{32i-1} L[32i+r][m'] X[m'][32j+c] -> stored in X[32j+r][32i+c]
-            const int jbk = task >> 6, ib = jbk + dd, tr = (task >> 3) & 7, tc = task & 7;
-            const int r0 = 4 * tr, c0 = 4 * tc;
-            float acc[4][4] = {};
-            for (int m = 32 * jbk; m < 32 * ib; ++m) {
-                const float4 a = ld4(&S.LT[m][32 * ib + r0]);
-                const float4 b = ld4(&S.X[m][32 * jbk + c0]);
-                const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                *reinterpret_cast<float4*>(&S.X[32 * jbk + r0 + i][32 * ib + c0]) =
-                    make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-        }
-        __syncthreads();
-        for (int task = tid; task < nblk * 64; task += blockDim.x) {
-            // X_ij[r][c] = -sum_m X_ii[r][m] T[m][c]
-            const int jbk = task >> 6, ib = jbk + dd, tr = (task >> 3) & 7, tc = task & 7;
-            const int r0 = 4 * tr, c0 = 4 * tc;
-            float acc[4][4] = {};
-#pragma unroll 4
-            for (int m = 0; m < 32; ++m) {
-                const float4 a = ld4(&S.XDT[ib][m][r0]);
-                const float4 b = ld4(&S.X[32 * jbk + m][32 * ib + c0]);
-                const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                *reinterpret_cast<float4*>(&S.X[32 * ib + r0 + i][32 * jbk + c0]) =
-                    make_float4(-acc[i][0], -acc[i][1], -acc[i][2], -acc[i][3]);
-        }
-        __syncthreads();
-    }
+    leaf_x_block_row(S, 3, warp, 16, lane);
+    __syncthreads();
 
     // U block = J X J (upper): U[r][c] = X[127-r][127-c] for r <= c; 4 columns per thread
-    for (int task = tid; task < NB * 32; task += blockDim.x) {
-        const int r = task >> 5, c = (task & 31) * 4;
+#pragma unroll 2
+    for (int it = 0; it < NB * 32 / LEAF_THREADS; ++it) {
+        const int task = tid + it * LEAF_THREADS, r = task >> 5, c = (task & 31) * 4;
         const float4 xv = ld4(&S.X[127 - r][124 - c]);   // columns 124-c .. 127-c, reversed below
         float v[4] = {xv.w, xv.z, xv.y, xv.x};
 #pragma unroll
@@ -292,28 +330,39 @@ __global__ void __launch_bounds__(512, 1)
             if (r > c + i) v[i] = 0.f;
         float h[4], l[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) split_tf32(v[i], h[i], l[i]);
-        const long long gr = jb + r, gc = jb + c;
-        *reinterpret_cast<float4*>(U_hi + gr * n + gc) = make_float4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<float4*>(U_lo + gr * n + gc) = make_float4(l[0], l[1], l[2], l[3]);
-        if (gr < d) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                if (gc + i < d) U[gr * d + gc + i] = v[i];
+        for (int i = 0; i < 4; ++i) {
+            h[i] = to_tf32(v[i]);
+            l[i] = v[i] - h[i];
         }
+        const long long off = (long long)(jb + r) * n + jb + c;
+        *reinterpret_cast<float4*>(U_hi + off) = make_float4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<float4*>(U_lo + off) = make_float4(l[0], l[1], l[2], l[3]);
     }
-    // UT[c][r..r+3] = U[r..r+3][c] = X[127-r-i][127-c]; consecutive lanes take consecutive c
-    // so the shared-memory reads run along rows of X (conflict-free)
-    for (int task = tid; task < NB * 32; task += blockDim.x) {
-        const int r = (task >> 7) * 4, c = task & 127;
-        float v[4], h[4], l[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = (r + i <= c) ? S.X[127 - r - i][127 - c] : 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) split_tf32(v[i], h[i], l[i]);
-        const long long off = (long long)(jb + c) * n + jb + r;
-        *reinterpret_cast<float4*>(UT_hi + off) = make_float4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<float4*>(UT_lo + off) = make_float4(l[0], l[1], l[2], l[3]);
+}
+
+// One CTA per diagonal block jb = 128 * blockIdx.x: X_jj = U_hi + U_lo (exact, as the leaf
+// wrote them).  Writes X_jj to the public U (clipped to d) and its transposed tf32 split to
+// UT_hi/UT_lo.
+__global__ void __launch_bounds__(512)
+    chol_diag_out_kernel(const float* __restrict__ U_hi, const float* __restrict__ U_lo, float* __restrict__ UT_hi,
+                         float* __restrict__ UT_lo, float* __restrict__ U, long long n, long long d) {
+    extern __shared__ __align__(16) uint8_t dout_raw[];
+    float (*Vs)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dout_raw);
+    const long long jb = (long long)blockIdx.x * NB;
+    for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+        const int r = e >> 7, c = e & 127;
+        const long long off = (jb + r) * n + jb + c;
+        const float v = U_hi[off] + U_lo[off];
+        Vs[r][c] = v;
+        if (jb + r < d && jb + c < d) U[(jb + r) * d + jb + c] = v;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+        const int c = e >> 7, r = e & 127;   // UT[c][r] = U[r][c]
+        float h, l;
+        split_tf32(Vs[r][c], h, l);
+        UT_hi[(jb + c) * n + jb + r] = h;
+        UT_lo[(jb + c) * n + jb + r] = l;
     }
 }
 
@@ -386,11 +435,19 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
     const int leaf_smem = (int)sizeof(gq::LeafSmem);
     GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::chol_leaf_kernel), leaf_smem));
     const uint64_t N = (uint64_t)n;
+    // Look-ahead: the caller's stream carries the critical chain leaf -> panel -> update of
+    // the next block column; the rest of each Schur update runs on a helper stream next to
+    // the following leaf and panel, on at most SMs - 1 CTAs so the leaf finds an SM.
+    cudaStream_t st2;
+    cudaEvent_t ev_panel, ev_rest;
+    if (!aux_stream(&st2, &ev_panel, &ev_rest)) return cudaErrorUnknown;
+    bool rest_pending = false;
+    Mat rh{w.RS_hi, N, N, N}, rl{w.RS_lo, N, N, N};
     for (int j = T - 1; j >= 0; --j) {
         const int jb = j * gq::NB;
         {
             gqh::TimedScope ts__("chol_leaf", st);
-            gq::chol_leaf_kernel<<<1, 512, leaf_smem, st>>>(w.A, n, d, jb, U, w.U_hi, w.U_lo, w.UT_hi, w.UT_lo);
+            gq::chol_leaf_kernel<<<1, gq::LEAF_THREADS, leaf_smem, st>>>(w.A, n, jb, w.U_hi, w.U_lo);
         }
         GQ_TRY(cudaGetLastError());
         if (j == 0) break;
@@ -412,8 +469,30 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
             Mat bh{w.U_hi, N, N, N}, bl{w.U_lo, N, N, N};
             GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(ah, al, bh, bl, o, p, 1, st, "chol_panel")));
         }
-        {   // update: A[0:jb, 0:jb] -= RS_panel RS_panel^T (upper tiles)
-            gq::GemmArgs p = gemm_args(jb, jb, gq::NB);
+        const int jn = jb - gq::NB;   // first column of the next block column
+        if (j >= 2) GQ_TRY(cudaEventRecord(ev_panel, st));
+        if (rest_pending) GQ_TRY(cudaStreamWaitEvent(st, ev_rest, 0));   // it also wrote block column j-1
+        {   // next block column: A[0:jb, jn:jb] -= RS_panel RS_panel[jn:jb]^T, plus the next panel's split
+            gq::GemmArgs p = gemm_args(jb, gq::NB, gq::NB);
+            p.a_col0 = jb;
+            p.b_row0 = jn;
+            p.b_col0 = jb;
+            p.alpha = -1.f;
+            p.beta = 1.f;
+            p.write_c = 1;
+            p.c_col0 = jn;
+            EpiMats o;
+            o.c = Mat{w.A, N, N, N};
+            if (j >= 2) {   // tiles above the diagonal block write the next panel's tf32 split
+                p.s_mt_lim = j - 1;
+                o.s_hi = Mat{w.AP_hi, (uint64_t)jn, 128, 128};
+                o.s_lo = Mat{w.AP_lo, (uint64_t)jn, 128, 128};
+            }
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(rh, rl, rh, rl, o, p, 1, st, "chol_update_next")));
+        }
+        if (j >= 2) {   // the rest: A[0:jn, 0:jn] -= RS RS^T (upper tiles), on the helper stream
+            GQ_TRY(cudaStreamWaitEvent(st2, ev_panel, 0));
+            gq::GemmArgs p = gemm_args(jn, jn, gq::NB);
             p.a_col0 = jb;
             p.b_col0 = jb;
             p.triangular = 1;
@@ -422,16 +501,20 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
             p.write_c = 1;
             EpiMats o;
             o.c = Mat{w.A, N, N, N};
-            if (j >= 2) {   // tiles of block column j-1 above its diagonal also write the next panel's split
-                p.s_tile_n = j - 1;
-                p.s_col0 = -(j - 1) * gq::NB;
-                o.s_hi = Mat{w.AP_hi, (uint64_t)(jb - gq::NB), 128, 128};
-                o.s_lo = Mat{w.AP_lo, (uint64_t)(jb - gq::NB), 128, 128};
-            }
-            Mat rh{w.RS_hi, N, N, N}, rl{w.RS_lo, N, N, N};
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(rh, rl, rh, rl, o, p, 1, st, "chol_update")));
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(rh, rl, rh, rl, o, p, 1, st2, "chol_update",
+                                                   std::max(1, num_sms() - 1))));
+            GQ_TRY(cudaEventRecord(ev_rest, st2));
+            rest_pending = true;
         }
     }
+    if (rest_pending) GQ_TRY(cudaStreamWaitEvent(st, ev_rest, 0));
+    {
+        const int smem = (int)(gq::NB * (gq::NB + 1) * sizeof(float));
+        GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::chol_diag_out_kernel), smem));
+        gqh::TimedScope ts__("chol_diag_out", st);
+        gq::chol_diag_out_kernel<<<(unsigned)T, 512, smem, st>>>(w.U_hi, w.U_lo, w.UT_hi, w.UT_lo, U, n, d);
+    }
+    GQ_TRY(cudaGetLastError());
     // U = R^-1 by doubling
     Mat rsh{w.RS_hi, N, N, N}, rsl{w.RS_lo, N, N, N};
     Mat uth{w.UT_hi, N, N, N}, utl{w.UT_lo, N, N, N};

@@ -49,7 +49,7 @@ struct GemmArgs {
     float* S_lo;
     long long lds;
     int s_row0, s_col0, s_zrow, s_zcol;
-    int s_tile_n;     // if > 0: S written only by tiles with nt == s_tile_n and mt < nt
+    int s_mt_lim;     // if > 0: S written only by tiles with mt < s_mt_lim
     float* T_hi;
     float* T_lo;
     long long ldt;
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(192, 1)
             if (!diag_mirror) {
                 const bool mirror = p.mirror && nt > mt;
                 const bool has_c = p.write_c != 0, has_t = p.T_hi != nullptr;
-                const bool has_s = p.S_hi != nullptr && (p.s_tile_n <= 0 || (nt == p.s_tile_n && mt < nt));
+                const bool has_s = p.S_hi != nullptr && (p.s_mt_lim <= 0 || mt < p.s_mt_lim);
                 const bool single_slot = !use_c || has_s || has_t || mirror;
                 const int zs_x = p.s_col0 + z * p.s_zcol, zs_y = p.s_row0 + z * p.s_zrow;
                 const int zt_x = p.t_col0 + z * p.t_zcol, zt_y = p.t_row0 + z * p.t_zrow;
@@ -463,6 +463,9 @@ inline bool make_out_map(CUtensorMap* map, const Mat& m, const CUtensorMap& fall
 
 // Multiprocessor count of the current device (cached per device).
 int num_sms();
+// A non-blocking helper stream and two timing-free events of the current device,
+// created on first use and kept for the life of the process.
+bool aux_stream(cudaStream_t* st, cudaEvent_t* ev0, cudaEvent_t* ev1);
 
 // Output kinds the epilogue region can hold: with beta != 0 the C tile plus at most two
 // extra outputs; without, at most five outputs in total.
@@ -473,9 +476,10 @@ inline bool epilogue_fits(const gq::GemmArgs& p) {
 }
 
 // Launch D = A B^T with the given epilogue.  For KIND_TF32X3 a2/b2 are the lo parts.
+// max_ctas > 0 caps the persistent grid (to leave SMs to a concurrent kernel).
 template <int KIND, int STAGES>
 cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2, const EpiMats& o, gq::GemmArgs p,
-                        int batch, cudaStream_t stream, const char* name) {
+                        int batch, cudaStream_t stream, const char* name, int max_ctas = 0) {
     using Cfg = gq::GemmCfg<KIND>;
     const int eb = (KIND == gq::KIND_BF16) ? 2 : 4;
     CUtensorMap ma, ma2, mb, mb2, mc, ms1, ms2, mt1, mt2;
@@ -510,7 +514,7 @@ cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2
     auto kern = gq::tc_gemm_kernel<KIND, STAGES>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)std::min<long long>(tiles, num_sms());
+    const unsigned grid = (unsigned)std::min<long long>(tiles, max_ctas > 0 ? max_ctas : num_sms());
     {
         TimedScope ts__(name, stream);
         kern<<<grid, 192, smem, stream>>>(ma, ma2, mb, mb2, mc, ms1, ms2, mt1, mt2, p);

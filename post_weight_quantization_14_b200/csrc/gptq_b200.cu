@@ -114,6 +114,22 @@ int num_sms() {
     return cache[dev];
 }
 
+bool aux_stream(cudaStream_t* st, cudaEvent_t* ev0, cudaEvent_t* ev1) {
+    static cudaStream_t streams[128];
+    static cudaEvent_t events[128][2];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return false;
+    if (!streams[dev]) {
+        if (cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess) return false;
+        if (cudaEventCreateWithFlags(&events[dev][0], cudaEventDisableTiming) != cudaSuccess) return false;
+        if (cudaEventCreateWithFlags(&events[dev][1], cudaEventDisableTiming) != cudaSuccess) return false;
+    }
+    *st = streams[dev];
+    *ev0 = events[dev][0];
+    *ev1 = events[dev][1];
+    return true;
+}
+
 cudaError_t ensure_smem_attr(const void* func, int bytes) {
     static std::set<std::tuple<const void*, int, int>> done;
     int dev = 0;
