@@ -283,6 +283,8 @@ __global__ void __launch_bounds__(LEAF_THREADS, 1)
     extern __shared__ __align__(16) uint8_t leaf_raw[];
     LeafSmem& S = *reinterpret_cast<LeafSmem*>(leaf_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();
+    pdl_trigger();
 
     // P[127-r][127-c] = A[r][c]: the whole diagonal tile, in two halves whose loads are all
     // issued before their stores
@@ -447,9 +449,9 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
         const int jb = j * gq::NB;
         {
             gqh::TimedScope ts__("chol_leaf", st);
-            gq::chol_leaf_kernel<<<1, gq::LEAF_THREADS, leaf_smem, st>>>(w.A, n, jb, w.U_hi, w.U_lo);
+            GQ_TRY(launch_pdl(gq::chol_leaf_kernel, dim3(1), dim3(gq::LEAF_THREADS), (size_t)leaf_smem, st,
+                              (const float*)w.A, n, jb, w.U_hi, w.U_lo));
         }
-        GQ_TRY(cudaGetLastError());
         if (j == 0) break;
         if (j == T - 1) {   // later panels are split by the previous update's epilogue
             gqh::TimedScope ts__("split_panel", st);
@@ -488,7 +490,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
                 o.s_hi = Mat{w.AP_hi, (uint64_t)jn, 128, 128};
                 o.s_lo = Mat{w.AP_lo, (uint64_t)jn, 128, 128};
             }
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(rh, rl, rh, rl, o, p, 1, st, "chol_update_next")));
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(rh, rl, rh, rl, o, p, 1, st, "chol_update_next", 0, rest_pending)));
         }
         if (j >= 2) {   // the rest: A[0:jn, 0:jn] -= RS RS^T (upper tiles), on the helper stream
             GQ_TRY(cudaStreamWaitEvent(st2, ev_panel, 0));
@@ -502,7 +504,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
             EpiMats o;
             o.c = Mat{w.A, N, N, N};
             GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(rh, rl, rh, rl, o, p, 1, st2, "chol_update",
-                                                   std::max(1, num_sms() - 1))));
+                                                   std::max(1, num_sms() - 1), true)));
             GQ_TRY(cudaEventRecord(ev_rest, st2));
             rest_pending = true;
         }

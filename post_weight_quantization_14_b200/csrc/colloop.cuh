@@ -49,8 +49,9 @@ struct ColArgs {
     int32_t* qweight;
     __half* scales;
     uint8_t* zeros_u8;
-    float* E_hi;
+    float* E_hi;          // errors of this block: E[row * e_ld + col], tf32 split
     float* E_lo;
+    long long e_ld;
     float* err_sq;
     int first_block;
 };
@@ -177,6 +178,8 @@ __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p)
         fence_mbar_init();
     }
     __syncthreads();
+    pdl_wait();
+    pdl_trigger();
     if (tid == 0) {
         constexpr uint32_t bytes = UP_BLOCK * 4;
         constexpr uint32_t chunk = bytes / 4;
@@ -236,8 +239,8 @@ __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p)
             if (rw < p.d_out) {
                 float h, l;
                 split_tf32(e, h, l);
-                p.E_hi[rw * CB + col] = h;
-                p.E_lo[rw * CB + col] = l;
+                p.E_hi[rw * p.e_ld + col] = h;
+                p.E_lo[rw * p.e_ld + col] = l;
             }
         }
 #pragma unroll
@@ -356,6 +359,16 @@ struct QuantWs {
 
 inline long long n_groups_of(long long d_in, int g) { return g < 0 ? 1 : (d_in + g - 1) / g; }
 
+// Trailing updates are deferred within superblocks of SB_BLOCKS column blocks: after
+// each block only the rest of its superblock is updated (K = 128); the columns past the
+// superblock take one update with K = the superblock width when it ends.  The result is
+// the per-block lazy update regrouped by associativity.
+constexpr int SB_BLOCKS = 8;
+
+inline long long superblock_cols(long long d_in) {
+    return std::min<long long>((long long)SB_BLOCKS * gq::CB, ((d_in + gq::CB - 1) / gq::CB) * gq::CB);
+}
+
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 inline size_t quant_ws_bytes(long long d_out, long long d_in, int g) {
@@ -364,7 +377,7 @@ inline size_t quant_ws_bytes(long long d_out, long long d_in, int g) {
     b += align256((size_t)nblk * gq::UP_BLOCK * 4);
     b += align256((size_t)d_in * 4);
     b += 2 * align256((size_t)d_in * d_in * 4);
-    b += 2 * align256((size_t)d_out * gq::CB * 4);
+    b += 2 * align256((size_t)d_out * superblock_cols(d_in) * 4);
     b += 2 * align256((size_t)d_out * 4);
     b += align256((size_t)n_groups_of(d_in, g) * d_out);
     return b;
@@ -383,8 +396,8 @@ inline QuantWs quant_ws_carve(void* ws, long long d_out, long long d_in, int g) 
     w.inv_d = reinterpret_cast<float*>(take((size_t)d_in * 4));
     w.UT_hi = reinterpret_cast<float*>(take((size_t)d_in * d_in * 4));
     w.UT_lo = reinterpret_cast<float*>(take((size_t)d_in * d_in * 4));
-    w.E_hi = reinterpret_cast<float*>(take((size_t)d_out * gq::CB * 4));
-    w.E_lo = reinterpret_cast<float*>(take((size_t)d_out * gq::CB * 4));
+    w.E_hi = reinterpret_cast<float*>(take((size_t)d_out * superblock_cols(d_in) * 4));
+    w.E_lo = reinterpret_cast<float*>(take((size_t)d_out * superblock_cols(d_in) * 4));
     w.row_scale = reinterpret_cast<float*>(take((size_t)d_out * 4));
     w.row_zero = reinterpret_cast<float*>(take((size_t)d_out * 4));
     w.zeros_u8 = take((size_t)n_groups_of(d_in, g) * d_out);
@@ -423,11 +436,29 @@ cudaError_t quant_run_bits(float* W, const float* U, long long d_out, long long 
     const int smem = (int)sizeof(gq::ColSmem);
     GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::colloop_kernel<BITS>), smem));
     const unsigned grid = (unsigned)((d_out + gq::CL_ROWS - 1) / gq::CL_ROWS);
-    Mat eh{w.E_hi, (uint64_t)d_out, (uint64_t)gq::CB, (uint64_t)gq::CB};
-    Mat el{w.E_lo, (uint64_t)d_out, (uint64_t)gq::CB, (uint64_t)gq::CB};
+    const long long sbw = superblock_cols(d_in);
+    Mat eh{w.E_hi, (uint64_t)d_out, (uint64_t)sbw, (uint64_t)sbw};
+    Mat el{w.E_lo, (uint64_t)d_out, (uint64_t)sbw, (uint64_t)sbw};
     Mat uh{w.UT_hi, (uint64_t)d_in, (uint64_t)d_in, (uint64_t)d_in};
     Mat ul{w.UT_lo, (uint64_t)d_in, (uint64_t)d_in, (uint64_t)d_in};
+    // W[:, e:e+n] -= E[:, k0:k0+K] U[c0:c0+K, e:e+n]  (U^T split is the B operand)
+    auto trailing = [&](long long e, long long ncols, int k0, long long c0, int K, const char* name) {
+        gq::GemmArgs p = gemm_args((int)d_out, (int)ncols, K);
+        p.a_col0 = k0;
+        p.b_row0 = (int)e;
+        p.b_col0 = (int)c0;
+        p.alpha = -1.f;
+        p.beta = 1.f;
+        p.c_col0 = (int)e;
+        p.write_c = 1;
+        EpiMats o;
+        o.c = Mat{W, (uint64_t)d_out, (uint64_t)d_in, (uint64_t)d_in};
+        return launch_gemm<gq::KIND_TF32X3, 2>(eh, el, uh, ul, o, p, 1, st, name);
+    };
     for (int b = 0; b < nblk; ++b) {
+        const long long s0 = (long long)(b / SB_BLOCKS) * sbw;      // superblock columns
+        const long long s1 = std::min<long long>(s0 + sbw, d_in);
+        const int kin = (int)((long long)b * gq::CB - s0);                // block offset in it
         gq::ColArgs a{};
         a.W = W;
         a.d_out = d_out;
@@ -443,28 +474,21 @@ cudaError_t quant_run_bits(float* W, const float* U, long long d_out, long long 
         a.qweight = qweight;
         a.scales = scales;
         a.zeros_u8 = w.zeros_u8;
-        a.E_hi = w.E_hi;
-        a.E_lo = w.E_lo;
+        a.E_hi = w.E_hi + kin;
+        a.E_lo = w.E_lo + kin;
+        a.e_ld = sbw;
         a.err_sq = err_sq;
         a.first_block = (b == 0);
         {
             gqh::TimedScope ts__("colloop", st);
-            gq::colloop_kernel<BITS><<<grid, gq::CL_WARPS * 32, smem, st>>>(a);
+            GQ_TRY(launch_pdl(gq::colloop_kernel<BITS>, dim3(grid), dim3(gq::CL_WARPS * 32), (size_t)smem, st,
+                              (const gq::ColArgs)a));
         }
-        GQ_TRY(cudaGetLastError());
         const long long e = (long long)a.c0 + gq::CB;
-        if (e < d_in) {  // trailing update W[:, e:] -= Err U[blk, e:]
-            gq::GemmArgs p = gemm_args((int)d_out, (int)(d_in - e), gq::CB);
-            p.b_row0 = (int)e;
-            p.b_col0 = a.c0;
-            p.alpha = -1.f;
-            p.beta = 1.f;
-            p.c_col0 = (int)e;
-            p.write_c = 1;
-            EpiMats o;
-            o.c = Mat{W, (uint64_t)d_out, (uint64_t)d_in, (uint64_t)d_in};
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(eh, el, uh, ul, o, p, 1, st, "trailing_update")));
-        }
+        if (e < s1)   // the rest of this superblock
+            GQ_TRY(trailing(e, s1 - e, kin, a.c0, gq::CB, "trailing_update"));
+        if (e == s1 && s1 < d_in)   // superblock done: everything past it, K = its width
+            GQ_TRY(trailing(s1, d_in - s1, 0, s0, (int)(s1 - s0), "trailing_update_sb"));
     }
     if (!cfg.sym && qzeros) {
         const long long ng = n_groups_of(d_in, g);

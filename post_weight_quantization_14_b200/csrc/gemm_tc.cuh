@@ -15,14 +15,14 @@
 // Warp 0 issues TMA into a ring of STAGES operand buffers that runs across tiles;
 // warp 1 issues MMAs into one of two TMEM accumulators (tile parity), so the epilogue
 // of one tile overlaps the mainloop of the next; warps 2..5 run the epilogue: each
-// warp owns 32 accumulator rows, loads its C chunks by TMA when beta != 0 (hidden
-// behind the next tile's mainloop), and writes every output as 32x32 boxes staged in
-// 128-byte-swizzled shared memory and stored by TMA.  Tiles on the diagonal of a
-// mirrored (symmetric) output take a register path that writes j >= i and mirrors it
-// exactly.  Every wait is bounded (GPTQ_ERR_TIMEOUT).  No TMA multicast.
+// warp owns 32 accumulator rows, loads its C chunks by TMA when beta != 0, and writes
+// every output 32x32 block through a 128-byte-swizzled staging box in shared memory with
+// coalesced 16-byte stores (no store-completion waits inside a tile).  Tiles on the
+// diagonal of a mirrored (symmetric) output take a register path that writes j >= i and
+// mirrors it exactly.  Every wait is bounded (GPTQ_ERR_TIMEOUT).  No TMA multicast.
 //
-// Outputs are clipped by the extents of their tensor maps; every caller keeps M and
-// N either multiples of the tile or equal to the remaining extent of the output.
+// Outputs are clipped by their matrices' extents; every caller keeps M and N either
+// multiples of the tile or equal to the remaining extent of the output.
 #pragma once
 #include "common.cuh"
 
@@ -41,18 +41,18 @@ struct GemmArgs {
     int k_to_n1;      // K range of a tile ends at n0 + BN (B zero for k > j)
     float alpha, beta;
     float* C;
-    long long ldc;
+    long long ldc, c_rows, c_cols;   // extents clip the stores
     int c_row0, c_col0, c_zrow, c_zcol;
     int write_c;
     int mirror;       // also write C[j, i] for tiles above the diagonal
     float* S_hi;
     float* S_lo;
-    long long lds;
+    long long lds, s_rows, s_cols;
     int s_row0, s_col0, s_zrow, s_zcol;
     int s_mt_lim;     // if > 0: S written only by tiles with mt < s_mt_lim
     float* T_hi;
     float* T_lo;
-    long long ldt;
+    long long ldt, t_rows, t_cols;
     int t_row0, t_col0, t_zrow, t_zcol;
 };
 
@@ -130,13 +130,34 @@ __device__ __forceinline__ void box_put_col(uint8_t* box, int col, const float (
     for (int t = 0; t < 32; ++t) *reinterpret_cast<float*>(box + box_off(t, col)) = v[t];
 }
 
+// Warp-cooperative store of a 32x32 fp32 block, given one row per lane (or, transposed,
+// one column per lane), to rows y0.. and columns x0.. of a row-major matrix, clipped to
+// rows x cols.  The block passes through this warp's swizzled staging box so that every
+// global store instruction writes whole 128-byte row segments.  Columns come in groups of
+// four (x0 and cols are multiples of 4).
+__device__ __forceinline__ void emit_block(uint8_t* box, int lane, const float (&v)[32], bool transposed,
+                                           float* base, long long ld, long long rows, long long cols, long long y0,
+                                           long long x0) {
+    __syncwarp();   // earlier readers of the box are done
+    if (transposed)
+        box_put_col(box, lane, v);
+    else
+        box_put_row(box, lane, v);
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int row = 4 * i + (lane >> 3), c4 = lane & 7;
+        const float4 val = *reinterpret_cast<const float4*>(box + row * 128 + ((c4 ^ (row & 7)) << 4));
+        const long long gy = y0 + row, gx = x0 + 4 * c4;
+        if (gy < rows && gx < cols) *reinterpret_cast<float4*>(base + gy * ld + gx) = val;
+    }
+}
+
 template <int KIND, int STAGES>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
                    const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mB2,
-                   const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mS1,
-                   const __grid_constant__ CUtensorMap mS2, const __grid_constant__ CUtensorMap mT1,
-                   const __grid_constant__ CUtensorMap mT2, const GemmArgs p) {
+                   const __grid_constant__ CUtensorMap mC, const GemmArgs p) {
     using Cfg = GemmCfg<KIND>;
     constexpr int KT = Cfg::KT, NOPS = Cfg::NOPS, STAGE_BYTES = Cfg::STAGE_BYTES;
     constexpr int A_BYTES = BM * 128;
@@ -179,6 +200,8 @@ __global__ void __launch_bounds__(192, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0 && lane == 0) {
         // ---------------- TMA producer: one ring of stages across all tiles of this CTA
@@ -282,15 +305,13 @@ __global__ void __launch_bounds__(192, 1)
                 const bool mirror = p.mirror && nt > mt;
                 const bool has_c = p.write_c != 0, has_t = p.T_hi != nullptr;
                 const bool has_s = p.S_hi != nullptr && (p.s_mt_lim <= 0 || mt < p.s_mt_lim);
-                const bool single_slot = !use_c || has_s || has_t || mirror;
-                const int zs_x = p.s_col0 + z * p.s_zcol, zs_y = p.s_row0 + z * p.s_zrow;
-                const int zt_x = p.t_col0 + z * p.t_zcol, zt_y = p.t_row0 + z * p.t_zrow;
-                const int kc = 0, ks = use_c ? 0 : (has_c ? 1 : 0);
-                const int kt = ks + (has_s ? 2 : 0), km = kt + (has_t ? 2 : 0);
+                const long long zs_x = p.s_col0 + z * p.s_zcol, zs_y = p.s_row0 + z * p.s_zrow;
+                const long long zt_x = p.t_col0 + z * p.t_zcol, zt_y = p.t_row0 + z * p.t_zrow;
                 bool cin_ok = true;
                 if (use_c) {
+                    fence_proxy_async_smem();   // this warp's reads of cbox (previous tile) come first
+                    __syncwarp();
                     if (lane == 0) {
-                        bulk_wait_all();   // this warp's stores out of cbox have finished
                         mbar_arrive_expect_tx(&cin_bar[q], kCBoxPerWarp * kBoxBytes);
                         for (int c = 0; c < kCBoxPerWarp; ++c)
                             tma_load_2d(cbox + c * kBoxBytes, &mC, &cin_bar[q], zc_x + n0 + 32 * c, zc_y + iy);
@@ -319,8 +340,8 @@ __global__ void __launch_bounds__(192, 1)
                     float out[32];
 #pragma unroll
                     for (int t = 0; t < 32; ++t) out[t] = p.alpha * __uint_as_float(r[t]);
-                    uint8_t* cb = cbox + c * kBoxBytes;
                     if (use_c && cin_ok) {
+                        const uint8_t* cb = cbox + c * kBoxBytes;
 #pragma unroll
                         for (int c4 = 0; c4 < 8; ++c4) {
                             const float4 v =
@@ -331,40 +352,21 @@ __global__ void __launch_bounds__(192, 1)
                             out[4 * c4 + 3] = fmaf(p.beta, v.w, out[4 * c4 + 3]);
                         }
                     }
-                    if (single_slot) {   // the boxes written below were read by an earlier TMA store
-                        if (lane == 0) bulk_wait_read_0();
-                        __syncwarp();
-                    }
-                    if (has_c) box_put_row(use_c ? cb : kb + kc * kBoxBytes, lane, out);
+                    if (has_c) emit_block(kb, lane, out, false, p.C, p.ldc, p.c_rows, p.c_cols, zc_y + iy, zc_x + j0);
                     if (has_s || has_t) {
                         float hi[32], lo[32];
 #pragma unroll
                         for (int t = 0; t < 32; ++t) split_tf32(out[t], hi[t], lo[t]);
                         if (has_s) {
-                            box_put_row(kb + ks * kBoxBytes, lane, hi);
-                            box_put_row(kb + (ks + 1) * kBoxBytes, lane, lo);
+                            emit_block(kb, lane, hi, false, p.S_hi, p.lds, p.s_rows, p.s_cols, zs_y + iy, zs_x + j0);
+                            emit_block(kb, lane, lo, false, p.S_lo, p.lds, p.s_rows, p.s_cols, zs_y + iy, zs_x + j0);
                         }
                         if (has_t) {
-                            box_put_col(kb + kt * kBoxBytes, lane, hi);
-                            box_put_col(kb + (kt + 1) * kBoxBytes, lane, lo);
+                            emit_block(kb, lane, hi, true, p.T_hi, p.ldt, p.t_rows, p.t_cols, zt_y + j0, zt_x + iy);
+                            emit_block(kb, lane, lo, true, p.T_lo, p.ldt, p.t_rows, p.t_cols, zt_y + j0, zt_x + iy);
                         }
                     }
-                    if (mirror) box_put_col(kb + km * kBoxBytes, lane, out);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if (has_c) tma_store_2d(&mC, use_c ? cb : kb + kc * kBoxBytes, zc_x + j0, zc_y + iy);
-                        if (has_s) {
-                            tma_store_2d(&mS1, kb + ks * kBoxBytes, zs_x + j0, zs_y + iy);
-                            tma_store_2d(&mS2, kb + (ks + 1) * kBoxBytes, zs_x + j0, zs_y + iy);
-                        }
-                        if (has_t) {
-                            tma_store_2d(&mT1, kb + kt * kBoxBytes, zt_x + iy, zt_y + j0);
-                            tma_store_2d(&mT2, kb + (kt + 1) * kBoxBytes, zt_x + iy, zt_y + j0);
-                        }
-                        if (mirror) tma_store_2d(&mC, kb + km * kBoxBytes, zc_x + iy, zc_y + j0);
-                        bulk_commit();
-                    }
+                    if (mirror) emit_block(kb, lane, out, true, p.C, p.ldc, p.c_rows, p.c_cols, zc_y + j0, zc_x + iy);
                 }
             } else {
                 // Register path for diagonal tiles of mirrored outputs (C only): write j >= i
@@ -467,22 +469,19 @@ int num_sms();
 // created on first use and kept for the life of the process.
 bool aux_stream(cudaStream_t* st, cudaEvent_t* ev0, cudaEvent_t* ev1);
 
-// Output kinds the epilogue region can hold: with beta != 0 the C tile plus at most two
-// extra outputs; without, at most five outputs in total.
-inline bool epilogue_fits(const gq::GemmArgs& p) {
-    const int extra = (p.S_hi ? 2 : 0) + (p.T_hi ? 2 : 0) + (p.mirror ? 1 : 0);
-    if (p.beta != 0.f) return p.write_c && extra <= gq::kXBoxPerWarp;
-    return extra + (p.write_c ? 1 : 0) <= gq::kOBoxPerWarp;
-}
+// C is read (beta != 0) only where it is also written.
+inline bool epilogue_fits(const gq::GemmArgs& p) { return p.beta == 0.f || p.write_c; }
 
 // Launch D = A B^T with the given epilogue.  For KIND_TF32X3 a2/b2 are the lo parts.
-// max_ctas > 0 caps the persistent grid (to leave SMs to a concurrent kernel).
+// max_ctas > 0 caps the persistent grid (to leave SMs to a concurrent kernel).  after_event:
+// the launch follows a cross-stream event wait, so it is not a programmatic dependent.
 template <int KIND, int STAGES>
 cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2, const EpiMats& o, gq::GemmArgs p,
-                        int batch, cudaStream_t stream, const char* name, int max_ctas = 0) {
+                        int batch, cudaStream_t stream, const char* name, int max_ctas = 0,
+                        bool after_event = false) {
     using Cfg = gq::GemmCfg<KIND>;
     const int eb = (KIND == gq::KIND_BF16) ? 2 : 4;
-    CUtensorMap ma, ma2, mb, mb2, mc, ms1, ms2, mt1, mt2;
+    CUtensorMap ma, ma2, mb, mb2, mc;
     if (!make_tmap_2d(&ma, a.ptr, eb, a.rows, a.cols, a.ld, gq::BM, Cfg::KT)) return cudaErrorInvalidValue;
     if (!make_tmap_2d(&mb, b.ptr, eb, b.rows, b.cols, b.ld, gq::BN, Cfg::KT)) return cudaErrorInvalidValue;
     if (KIND == gq::KIND_TF32X3) {
@@ -492,11 +491,15 @@ cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2
         ma2 = ma;
         mb2 = mb;
     }
-    if (!make_out_map(&mc, o.c, ma) || !make_out_map(&ms1, o.s_hi, ma) || !make_out_map(&ms2, o.s_lo, ma) ||
-        !make_out_map(&mt1, o.t_hi, ma) || !make_out_map(&mt2, o.t_lo, ma))
-        return cudaErrorInvalidValue;
+    if (!make_out_map(&mc, o.c, ma)) return cudaErrorInvalidValue;
     p.C = static_cast<float*>(const_cast<void*>(o.c.ptr));
     p.ldc = (long long)o.c.ld;
+    p.c_rows = (long long)o.c.rows;
+    p.c_cols = (long long)o.c.cols;
+    p.s_rows = (long long)o.s_hi.rows;
+    p.s_cols = (long long)o.s_hi.cols;
+    p.t_rows = (long long)o.t_hi.rows;
+    p.t_cols = (long long)o.t_hi.cols;
     p.S_hi = static_cast<float*>(const_cast<void*>(o.s_hi.ptr));
     p.S_lo = static_cast<float*>(const_cast<void*>(o.s_lo.ptr));
     p.lds = (long long)o.s_hi.ld;
@@ -517,9 +520,10 @@ cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2
     const unsigned grid = (unsigned)std::min<long long>(tiles, max_ctas > 0 ? max_ctas : num_sms());
     {
         TimedScope ts__(name, stream);
-        kern<<<grid, 192, smem, stream>>>(ma, ma2, mb, mb2, mc, ms1, ms2, mt1, mt2, p);
+        e = after_event ? launch_plain(kern, dim3(grid), dim3(192), (size_t)smem, stream, ma, ma2, mb, mb2, mc, p)
+                        : launch_pdl(kern, dim3(grid), dim3(192), (size_t)smem, stream, ma, ma2, mb, mb2, mc, p);
     }
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 inline gq::GemmArgs gemm_args(int M, int N, int K) {

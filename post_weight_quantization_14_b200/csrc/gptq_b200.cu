@@ -443,6 +443,8 @@ static cudaError_t fixed_gemm(const Mat& a, const Mat& a2, const Mat& c, gq::Gem
     if (!encode_tmap_2d(&mc, c.ptr, 4, c.rows, c.cols, c.ld, 32, 32)) return cudaErrorInvalidValue;
     p.C = static_cast<float*>(const_cast<void*>(c.ptr));
     p.ldc = (long long)c.ld;
+    p.c_rows = (long long)c.rows;
+    p.c_cols = (long long)c.cols;
     p.tiles_m = (p.M + gq::BM - 1) / gq::BM;
     p.tiles_n = (p.N + gq::BN - 1) / gq::BN;
     p.batch = 1;
@@ -456,8 +458,7 @@ static cudaError_t fixed_gemm(const Mat& a, const Mat& a2, const Mat& c, gq::Gem
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (sms <= 0) sms = 148;
     // A and B are the same matrix (X^T); the epilogue writes C and its mirror
-    kern<<<dim3((unsigned)std::min<long long>(tiles, sms), 1, 1), 192, smem, st>>>(ma, ma2, ma, ma2, mc, mc, mc, mc, mc,
-                                                                                     p);
+    kern<<<dim3((unsigned)std::min<long long>(tiles, sms), 1, 1), 192, smem, st>>>(ma, ma2, ma, ma2, mc, p);
     return cudaGetLastError();
 }
 

@@ -114,6 +114,8 @@ CASES = [
     (33, 256, 8, 16, False),
     (64, 1024, 4, 128, True),
     (17, 136, 4, 32, False),
+    (96, 1152, 4, 128, False),   # a full superblock of deferred updates, then one more block
+    (40, 2200, 3, 64, True),     # three superblocks, the last one ragged
 ]
 
 
