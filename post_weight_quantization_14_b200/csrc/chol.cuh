@@ -97,14 +97,12 @@ __global__ void zero_lower_blocks_kernel(float* __restrict__ U, long long d) {
 //
 // Right-looking, blocked by 32 columns.  Panel kb (columns k0 = 32 kb .. k0 + 31, rows
 // k0 .. 127) is eliminated by the 4 - kb warps that own its rows (one row per lane, the
-// row's 32 panel entries in registers): at step k the warp holding the diagonal block
-// publishes the current column k of that block in shared memory, and every row r does
-// L_rk = P_rk / sqrt(P_kk) and P_rj -= P_rk P_jk / P_kk for j > k, with one named
-// barrier per step.  All warps then apply the rank-32 update of the trailing lower
+// row's 32 panel entries in registers), one named barrier per pivot (leaf_eliminate).
+// All warps then apply the rank-32 update of the trailing lower
 // triangle on 4x4 register micro-tiles.  Meanwhile the warps not in the elimination
 // build the inverse X = L^-1 block row by block row, one row behind:
-// X_ii = L_ii^-1 by forward substitution (lane = column), T_ij = sum_{k=j}^{i-1} L_ik X_kj,
-// X_ij = -X_ii T_ij.
+// X_ii = L_ii^-1 by forward substitution (lane = column), the partial products L_ik X_kj
+// (j <= k < i) one 32-block each, and X_ij = -X_ii sum_k L_ik X_kj.
 // Writes X_jj (upper, zeros below the diagonal) as U_hi = tf32(X_jj) and U_lo = X_jj - U_hi
 // (exact, not rounded: the tensor pipe reads only its tf32 part); U_hi + U_lo restores
 // X_jj exactly for chol_diag_out_kernel.
@@ -114,7 +112,7 @@ static_assert(NB * NB / 4 == 8 * LEAF_THREADS && NB * 32 == 8 * LEAF_THREADS, "l
 
 struct LeafSmem {
     float P[NB][LS];         // reversed block; lower triangle holds the Schur complement
-    float X[NB][LS];         // L^-1 (lower); blocks above the diagonal hold T
+    float X[NB][LS];         // L^-1 (lower); blocks above the diagonal hold partial products
     float LT[NB][LS];        // L transposed: LT[m][r] = L[r][m]
     float XDT[4][32][36];    // diagonal inverses transposed: XDT[i][m][r] = X_ii[r][m]
     float col[2][32];        // pivot column of the current step (double-buffered)
@@ -127,6 +125,9 @@ __device__ __forceinline__ void named_bar(int id, int nthreads) {
 }
 
 // Eliminate panel k0 .. k0+31 with nw warps (barrier 1); warp w owns rows k0 + 32 w + lane.
+// At step k the warp holding the diagonal block publishes the current column k of that
+// block in shared memory, and every row r does L_rk = P_rk / sqrt(P_kk) and
+// P_rj -= P_rk P_jk / P_kk for j > k.
 __device__ __forceinline__ void leaf_eliminate(LeafSmem& S, int k0, int nw, int warp, int lane, int jb) {
     const int r = k0 + 32 * warp + lane;
     const bool dg = warp == 0;   // the warp holding the diagonal 32x32 block
@@ -198,15 +199,18 @@ __device__ __forceinline__ void leaf_trailing_update(LeafSmem& S, int k0, int ti
 }
 
 // X_ii = L_ii^-1 by forward substitution, one warp, lane = column j:
-// x_m = (delta_mj - sum_{m' < m} L_mm' x_m') / L_mm.
+// x_m = (delta_mj - sum_{m' < m} L_mm' x_m') / L_mm.  The 32 reciprocals are formed up
+// front (lane m takes 1/L_mm) and broadcast by shuffle, off the substitution chain.
 __device__ __forceinline__ void leaf_diag_inverse(LeafSmem& S, int i, int lane) {
+    constexpr unsigned FULL = 0xffffffffu;
     const int k0 = 32 * i;
+    const float my_dinv = __frcp_rn(S.LT[k0 + lane][k0 + lane]);
     float x[32], s[32];
 #pragma unroll
     for (int m = 0; m < 32; ++m) s[m] = 0.f;
 #pragma unroll
     for (int m = 0; m < 32; ++m) {
-        const float dinv = __frcp_rn(S.LT[k0 + m][k0 + m]);
+        const float dinv = __shfl_sync(FULL, my_dinv, m);
         x[m] = (((m == lane) ? 1.f : 0.f) - s[m]) * dinv;
 #pragma unroll
         for (int q4 = (m + 1) >> 2; q4 < 8; ++q4) {
@@ -225,31 +229,47 @@ __device__ __forceinline__ void leaf_diag_inverse(LeafSmem& S, int i, int lane) 
             make_float4(x[4 * m4], x[4 * m4 + 1], x[4 * m4 + 2], x[4 * m4 + 3]);
 }
 
+// Slot of the partial product L_ik X_kj (j <= k < i) of block row i: one of the six
+// 32x32 blocks above X's block diagonal, all free while a block row is being formed.
+__device__ __forceinline__ float* leaf_partial_slot(LeafSmem& S, int j, int k) {
+    // pairs (j, k) in order (0,0), (0,1), (1,1), (0,2), (1,2), (2,2) -> blocks
+    // (0,1), (0,2), (0,3), (1,2), (1,3), (2,3)
+    const int idx = k * (k + 1) / 2 + j;
+    const int r = (idx >= 3) + (idx >= 5);
+    const int c = idx < 3 ? idx + 1 : (idx < 5 ? idx - 1 : 3);
+    return &S.X[32 * r][32 * c];
+}
+
 // Block row i of X = L^-1 by a group of g warps (group warp gw, barrier 2):
-// group warp 0 forms X_ii while the others form T_ij = sum_{k=j}^{i-1} L_ik X_kj (stored in
-// X's block (j, i)); then all form X_ij = -X_ii T_ij for j < i.
+// group warp 0 forms X_ii while the others form the partial products L_ik X_kj for
+// j <= k < i; then all form X_ij = -X_ii sum_{k=j}^{i-1} L_ik X_kj for j < i.
 __device__ __forceinline__ void leaf_x_block_row(LeafSmem& S, int i, int gw, int g, int lane) {
     if (gw == 0) {
         leaf_diag_inverse(S, i, lane);
     } else if (i > 0) {
         const int gt = (gw - 1) * 32 + lane, gn = (g - 1) * 32;
-        for (int task = gt; task < 64 * i; task += gn) {
-            const int jbk = task >> 6, tr = (task >> 3) & 7, tc = task & 7;
+        const int npairs = i * (i + 1) / 2;
+        for (int task = gt; task < 64 * npairs; task += gn) {
+            const int pr = task >> 6, tr = (task >> 3) & 7, tc = task & 7;
+            int k = 0;
+            while ((k + 1) * (k + 2) / 2 <= pr) ++k;
+            const int j = pr - k * (k + 1) / 2;
             const int r0 = 4 * tr, c0 = 4 * tc;
             float acc[4][4] = {};
-#pragma unroll 4
-            for (int m = 32 * jbk; m < 32 * i; ++m) {
-                const float4 a = ld4(&S.LT[m][32 * i + r0]);
-                const float4 b = ld4(&S.X[m][32 * jbk + c0]);
-                const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll 8
+            for (int m = 0; m < 32; ++m) {
+                const float4 a = ld4(&S.LT[32 * k + m][32 * i + r0]);   // L_ik[r][m]
+                const float4 bv4 = ld4(&S.X[32 * k + m][32 * j + c0]);   // X_kj[m][c]
+                const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bv4.x, bv4.y, bv4.z, bv4.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
 #pragma unroll
                     for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
             }
+            float* slot = leaf_partial_slot(S, j, k);
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                *reinterpret_cast<float4*>(&S.X[32 * jbk + r0 + u][32 * i + c0]) =
+                *reinterpret_cast<float4*>(slot + (r0 + u) * LS + c0) =
                     make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
         }
     }
@@ -259,12 +279,30 @@ __device__ __forceinline__ void leaf_x_block_row(LeafSmem& S, int i, int gw, int
     for (int task = gt; task < 64 * i; task += gn) {
         const int jbk = task >> 6, tr = (task >> 3) & 7, tc = task & 7;
         const int r0 = 4 * tr, c0 = 4 * tc;
+        const int np = i - jbk;   // partials k = jbk .. i-1 (1 to 3)
+        const float* p0 = leaf_partial_slot(S, jbk, jbk) + c0;
+        const float* p1 = leaf_partial_slot(S, jbk, min(jbk + 1, 2)) + c0;
+        const float* p2 = leaf_partial_slot(S, jbk, 2) + c0;
         float acc[4][4] = {};
-#pragma unroll 8
+#pragma unroll 4
         for (int m = 0; m < 32; ++m) {
             const float4 a = ld4(&S.XDT[i][m][r0]);
-            const float4 b = ld4(&S.X[32 * jbk + m][32 * i + c0]);
-            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+            float4 t4 = ld4(p0 + m * LS);
+            if (np > 1) {
+                const float4 q = ld4(p1 + m * LS);
+                t4.x += q.x;
+                t4.y += q.y;
+                t4.z += q.z;
+                t4.w += q.w;
+            }
+            if (np > 2) {
+                const float4 q = ld4(p2 + m * LS);
+                t4.x += q.x;
+                t4.y += q.y;
+                t4.z += q.z;
+                t4.w += q.w;
+            }
+            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
             for (int u = 0; u < 4; ++u)
 #pragma unroll
@@ -469,7 +507,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
             o.s_lo = Mat{w.RS_lo, N, N, N};
             Mat ah{w.AP_hi, (uint64_t)jb, 128, 128}, al{w.AP_lo, (uint64_t)jb, 128, 128};
             Mat bh{w.U_hi, N, N, N}, bl{w.U_lo, N, N, N};
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(ah, al, bh, bl, o, p, 1, st, "chol_panel")));
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32>(ah, al, bh, bl, o, p, 1, st, "chol_panel")));
         }
         const int jn = jb - gq::NB;   // first column of the next block column
         if (j >= 2) GQ_TRY(cudaEventRecord(ev_panel, st));
@@ -490,7 +528,8 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
                 o.s_hi = Mat{w.AP_hi, (uint64_t)jn, 128, 128};
                 o.s_lo = Mat{w.AP_lo, (uint64_t)jn, 128, 128};
             }
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(rh, rl, rh, rl, o, p, 1, st, "chol_update_next", 0, rest_pending)));
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32>(rh, rl, rh, rl, o, p, 1, st, "chol_update_next", 0,
+                                                        rest_pending)));
         }
         if (j >= 2) {   // the rest: A[0:jn, 0:jn] -= RS RS^T (upper tiles), on the helper stream
             GQ_TRY(cudaStreamWaitEvent(st2, ev_panel, 0));

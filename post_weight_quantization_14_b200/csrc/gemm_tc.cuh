@@ -38,7 +38,7 @@ struct GemmArgs {
     int batch;        // independent problems in the launch (offsets *_z* per problem)
     int triangular;   // enumerate only tiles with nt >= mt
     int k_from_m0;    // K range of a tile starts at its m0 (A upper triangular in (i,k))
-    int k_to_n1;      // K range of a tile ends at n0 + BN (B zero for k > j)
+    int k_to_n1;      // K range of a tile ends at n0 + tile N (B zero for k > j)
     float alpha, beta;
     float* C;
     long long ldc, c_rows, c_cols;   // extents clip the stores
@@ -60,22 +60,27 @@ constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int kEpiLd = 33;
 constexpr int kBoxBytes = 32 * 32 * 4;           // one 32x32 fp32 box, 128-byte rows
-constexpr int kCBoxPerWarp = BN / 32;            // C chunks of one warp (beta != 0)
-constexpr int kXBoxPerWarp = 2;                  // extra output boxes per warp when beta != 0
-constexpr int kOBoxPerWarp = 5;                  // output boxes per warp when beta == 0
-constexpr int kEpiBytes = 4 * (kCBoxPerWarp + kXBoxPerWarp) * kBoxBytes;   // 96 KB
-static_assert(4 * kOBoxPerWarp * kBoxBytes <= kEpiBytes, "epilogue region");
+// Tile N is a template parameter TBN (128, or 32 for launches with few tiles, whose
+// epilogue stores are then spread over four times as many SMs).  Each epilogue warp owns
+// a region of TBN / 32 C boxes (beta != 0) plus two boxes: the staging box and, for the
+// register path of mirrored diagonal tiles, room for a padded 32x33 tile.
+template <int TBN>
+__host__ __device__ constexpr int epi_boxes_per_warp() { return TBN / 32 + 2; }
+template <int TBN>
+__host__ __device__ constexpr int epi_bytes() { return 4 * epi_boxes_per_warp<TBN>() * kBoxBytes; }   // 96 KB at TBN = 128
+static_assert(32 * kEpiLd * 4 <= 2 * kBoxBytes, "register-path staging tile fits two boxes");
 
-template <int KIND>
+template <int KIND, int TBN = BN>
 struct GemmCfg {
+    static_assert(TBN == 32 || TBN == 64 || TBN == 128, "tile N");
     static constexpr int KT = (KIND == KIND_BF16) ? 64 : 32;  // K elements per stage (128 bytes)
     static constexpr int NOPS = (KIND == KIND_BF16) ? 1 : 2;
-    static constexpr int STAGE_BYTES = NOPS * (BM * 128 + BN * 128);
+    static constexpr int STAGE_BYTES = NOPS * (BM * 128 + TBN * 128);
 };
 
-template <int KIND, int STAGES>
-constexpr int gemm_smem_bytes() {
-    return STAGES * GemmCfg<KIND>::STAGE_BYTES + kEpiBytes + 1024 + 256;
+template <int KIND, int STAGES, int TBN = BN>
+__host__ __device__ constexpr int gemm_smem_bytes() {
+    return STAGES * GemmCfg<KIND, TBN>::STAGE_BYTES + epi_bytes<TBN>() + 1024 + 256;
 }
 
 __device__ __forceinline__ void tile_coords(const GemmArgs& p, int t, int& mt, int& nt) {
@@ -100,15 +105,15 @@ struct TileInfo {
     int z, mt, nt, m0, n0, kbeg, nk;
 };
 
-template <int KT>
+template <int KT, int TBN>
 __device__ __forceinline__ TileInfo tile_info(const GemmArgs& p, int w, int tiles_per_batch) {
     TileInfo ti;
     ti.z = w / tiles_per_batch;
     tile_coords(p, w % tiles_per_batch, ti.mt, ti.nt);
     ti.m0 = ti.mt * BM;
-    ti.n0 = ti.nt * BN;
+    ti.n0 = ti.nt * TBN;
     ti.kbeg = p.k_from_m0 ? ti.m0 : 0;
-    const int kend = p.k_to_n1 ? min(p.K, ti.n0 + BN) : p.K;
+    const int kend = p.k_to_n1 ? min(p.K, ti.n0 + TBN) : p.K;
     ti.nk = kend > ti.kbeg ? (kend - ti.kbeg + KT - 1) / KT : 0;
     return ti;
 }
@@ -153,22 +158,23 @@ __device__ __forceinline__ void emit_block(uint8_t* box, int lane, const float (
     }
 }
 
-template <int KIND, int STAGES>
+template <int KIND, int STAGES, int TBN>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
                    const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mB2,
                    const __grid_constant__ CUtensorMap mC, const GemmArgs p) {
-    using Cfg = GemmCfg<KIND>;
+    using Cfg = GemmCfg<KIND, TBN>;
     constexpr int KT = Cfg::KT, NOPS = Cfg::NOPS, STAGE_BYTES = Cfg::STAGE_BYTES;
     constexpr int A_BYTES = BM * 128;
-    constexpr int B_BYTES = BN * 128;
-    constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
+    constexpr int B_BYTES = TBN * 128;
+    constexpr uint32_t TMEM_COLS = 2 * TBN;  // two accumulators
+    constexpr int NCHUNK = TBN / 32;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* epi = smem + STAGES * STAGE_BYTES;
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(epi + kEpiBytes);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(epi + epi_bytes<TBN>());
     uint64_t* empty_bar = full_bar + STAGES;
     uint64_t* tfull_bar = empty_bar + STAGES;   // [2] accumulator ready
     uint64_t* tempty_bar = tfull_bar + 2;       // [2] accumulator drained (4 epilogue warps)
@@ -214,7 +220,7 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t kiter = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-            const TileInfo ti = tile_info<KT>(p, w, tiles_per_batch);
+            const TileInfo ti = tile_info<KT, TBN>(p, w, tiles_per_batch);
             const int ax = p.a_col0 + ti.z * p.a_zcol, ay = p.a_row0 + ti.z * p.a_zrow + ti.m0;
             const int bx = p.b_col0 + ti.z * p.b_zcol, by = p.b_row0 + ti.z * p.b_zrow + ti.n0;
             for (int kt = 0; kt < ti.nk; ++kt, ++kiter) {
@@ -235,12 +241,12 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer
-        constexpr uint32_t idesc = make_idesc(KIND == KIND_BF16 ? 1u : 2u, BM, BN);
+        constexpr uint32_t idesc = make_idesc(KIND == KIND_BF16 ? 1u : 2u, BM, TBN);
         uint32_t kiter = 0;
         bool ok = true;
         int local = 0;
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++local) {
-            const TileInfo ti = tile_info<KT>(p, w, tiles_per_batch);
+            const TileInfo ti = tile_info<KT, TBN>(p, w, tiles_per_batch);
             const int buf = local & 1;
             const uint32_t use = (uint32_t)(local >> 1);
             if (!mbar_wait(&tempty_bar[buf], (use & 1) ^ 1, w)) {
@@ -248,7 +254,7 @@ __global__ void __launch_bounds__(192, 1)
                 break;
             }
             tc_fence_after();
-            const uint32_t acc = tmem + (uint32_t)(buf * BN);
+            const uint32_t acc = tmem + (uint32_t)(buf * TBN);
             for (int kt = 0; kt < ti.nk; ++kt, ++kiter) {
                 const int s = kiter % STAGES;
                 const uint32_t it = kiter / STAGES;
@@ -281,22 +287,21 @@ __global__ void __launch_bounds__(192, 1)
         const int q = warp & 3;
         const bool use_c = p.beta != 0.f;
         // with beta: this warp's C chunks, then its extra boxes; without: its output boxes
-        uint8_t* cbox = epi + q * kCBoxPerWarp * kBoxBytes;
-        uint8_t* xbox = epi + 4 * kCBoxPerWarp * kBoxBytes + q * kXBoxPerWarp * kBoxBytes;
-        uint8_t* obox = epi + q * kOBoxPerWarp * kBoxBytes;
-        uint8_t* kb = use_c ? xbox : obox;
-        float* stage_t = reinterpret_cast<float*>(use_c ? cbox : obox);   // register-path staging (own region)
+        uint8_t* wreg = epi + q * epi_boxes_per_warp<TBN>() * kBoxBytes;   // this warp's region
+        uint8_t* cbox = wreg;
+        uint8_t* kb = use_c ? wreg + NCHUNK * kBoxBytes : wreg;             // staging box
+        float* stage_t = reinterpret_cast<float*>(wreg);   // register-path staging (own region)
         int local = 0;
         uint32_t cin_use = 0;
         bool alive = true;
         for (int w = blockIdx.x; w < total && alive; w += gridDim.x, ++local) {
-            const TileInfo ti = tile_info<KT>(p, w, tiles_per_batch);
+            const TileInfo ti = tile_info<KT, TBN>(p, w, tiles_per_batch);
             const int buf = local & 1;
             const uint32_t use = (uint32_t)(local >> 1);
             const bool ok = mbar_wait(&tfull_bar[buf], use & 1, w);
             alive = ok;
             tc_fence_after();
-            const uint32_t acc = tmem + (uint32_t)(buf * BN) + ((uint32_t)(q * 32) << 16);
+            const uint32_t acc = tmem + (uint32_t)(buf * TBN) + ((uint32_t)(q * 32) << 16);
             const int z = ti.z, n0 = ti.n0, mt = ti.mt, nt = ti.nt;
             const int zc_x = p.c_col0 + z * p.c_zcol, zc_y = p.c_row0 + z * p.c_zrow;
             const int iy = ti.m0 + 32 * q;
@@ -312,8 +317,8 @@ __global__ void __launch_bounds__(192, 1)
                     fence_proxy_async_smem();   // this warp's reads of cbox (previous tile) come first
                     __syncwarp();
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(&cin_bar[q], kCBoxPerWarp * kBoxBytes);
-                        for (int c = 0; c < kCBoxPerWarp; ++c)
+                        mbar_arrive_expect_tx(&cin_bar[q], NCHUNK * kBoxBytes);
+                        for (int c = 0; c < NCHUNK; ++c)
                             tma_load_2d(cbox + c * kBoxBytes, &mC, &cin_bar[q], zc_x + n0 + 32 * c, zc_y + iy);
                     }
                     __syncwarp();
@@ -321,7 +326,7 @@ __global__ void __launch_bounds__(192, 1)
                     ++cin_use;
                 }
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
+                for (int c = 0; c < NCHUNK; ++c) {
                     const int j0 = n0 + c * 32;
                     uint32_t r[32];
                     if (ti.nk > 0 && ok) {
@@ -331,7 +336,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                         for (int t = 0; t < 32; ++t) r[t] = 0u;
                     }
-                    if (c == BN / 32 - 1) {   // accumulator drained: the MMA warp may reuse it
+                    if (c == NCHUNK - 1) {   // accumulator drained: the MMA warp may reuse it
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&tempty_bar[buf]);
@@ -377,7 +382,7 @@ __global__ void __launch_bounds__(192, 1)
                 const int rbase = iy;
                 const long long zr = zc_y, zcc = zc_x;
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
+                for (int c = 0; c < NCHUNK; ++c) {
                     const int j0 = n0 + c * 32;
                     uint32_t r[32];
                     if (ti.nk > 0 && ok) {
@@ -387,7 +392,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                         for (int t = 0; t < 32; ++t) r[t] = 0u;
                     }
-                    if (c == BN / 32 - 1) {
+                    if (c == NCHUNK - 1) {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&tempty_bar[buf]);
@@ -475,18 +480,19 @@ inline bool epilogue_fits(const gq::GemmArgs& p) { return p.beta == 0.f || p.wri
 // Launch D = A B^T with the given epilogue.  For KIND_TF32X3 a2/b2 are the lo parts.
 // max_ctas > 0 caps the persistent grid (to leave SMs to a concurrent kernel).  after_event:
 // the launch follows a cross-stream event wait, so it is not a programmatic dependent.
-template <int KIND, int STAGES>
+template <int KIND, int STAGES, int TBN = gq::BN>
 cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2, const EpiMats& o, gq::GemmArgs p,
                         int batch, cudaStream_t stream, const char* name, int max_ctas = 0,
                         bool after_event = false) {
-    using Cfg = gq::GemmCfg<KIND>;
+    using Cfg = gq::GemmCfg<KIND, TBN>;
     const int eb = (KIND == gq::KIND_BF16) ? 2 : 4;
     CUtensorMap ma, ma2, mb, mb2, mc;
+    if ((p.triangular || p.mirror) && TBN != gq::BM) return cudaErrorInvalidValue;   // square tiles only
     if (!make_tmap_2d(&ma, a.ptr, eb, a.rows, a.cols, a.ld, gq::BM, Cfg::KT)) return cudaErrorInvalidValue;
-    if (!make_tmap_2d(&mb, b.ptr, eb, b.rows, b.cols, b.ld, gq::BN, Cfg::KT)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&mb, b.ptr, eb, b.rows, b.cols, b.ld, TBN, Cfg::KT)) return cudaErrorInvalidValue;
     if (KIND == gq::KIND_TF32X3) {
         if (!make_tmap_2d(&ma2, a2.ptr, eb, a2.rows, a2.cols, a2.ld, gq::BM, Cfg::KT)) return cudaErrorInvalidValue;
-        if (!make_tmap_2d(&mb2, b2.ptr, eb, b2.rows, b2.cols, b2.ld, gq::BN, Cfg::KT)) return cudaErrorInvalidValue;
+        if (!make_tmap_2d(&mb2, b2.ptr, eb, b2.rows, b2.cols, b2.ld, TBN, Cfg::KT)) return cudaErrorInvalidValue;
     } else {
         ma2 = ma;
         mb2 = mb;
@@ -508,13 +514,13 @@ cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2
     p.ldt = (long long)o.t_hi.ld;
     if (!epilogue_fits(p)) return cudaErrorInvalidValue;
     p.tiles_m = (p.M + gq::BM - 1) / gq::BM;
-    p.tiles_n = (p.N + gq::BN - 1) / gq::BN;
+    p.tiles_n = (p.N + TBN - 1) / TBN;
     p.batch = batch;
     const long long tiles = (p.triangular ? (long long)p.tiles_m * (p.tiles_m + 1) / 2
                                           : (long long)p.tiles_m * p.tiles_n) * batch;
     if (tiles <= 0) return cudaSuccess;
-    constexpr int smem = gq::gemm_smem_bytes<KIND, STAGES>();
-    auto kern = gq::tc_gemm_kernel<KIND, STAGES>;
+    constexpr int smem = gq::gemm_smem_bytes<KIND, STAGES, TBN>();
+    auto kern = gq::tc_gemm_kernel<KIND, STAGES, TBN>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)std::min<long long>(tiles, max_ctas > 0 ? max_ctas : num_sms());
