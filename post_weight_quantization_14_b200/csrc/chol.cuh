@@ -507,7 +507,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
             o.s_lo = Mat{w.RS_lo, N, N, N};
             Mat ah{w.AP_hi, (uint64_t)jb, 128, 128}, al{w.AP_lo, (uint64_t)jb, 128, 128};
             Mat bh{w.U_hi, N, N, N}, bl{w.U_lo, N, N, N};
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32>(ah, al, bh, bl, o, p, 1, st, "chol_panel")));
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(ah, al, bh, bl, o, p, 1, st, "chol_panel")));
         }
         const int jn = jb - gq::NB;   // first column of the next block column
         if (j >= 2) GQ_TRY(cudaEventRecord(ev_panel, st));
@@ -528,7 +528,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
                 o.s_hi = Mat{w.AP_hi, (uint64_t)jn, 128, 128};
                 o.s_lo = Mat{w.AP_lo, (uint64_t)jn, 128, 128};
             }
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32>(rh, rl, rh, rl, o, p, 1, st, "chol_update_next", 0,
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, rh, rl, o, p, 1, st, "chol_update_next", 0,
                                                         rest_pending)));
         }
         if (j >= 2) {   // the rest: A[0:jn, 0:jn] -= RS RS^T (upper tiles), on the helper stream
@@ -542,7 +542,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
             p.write_c = 1;
             EpiMats o;
             o.c = Mat{w.A, N, N, N};
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(rh, rl, rh, rl, o, p, 1, st2, "chol_update",
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rh, rl, rh, rl, o, p, 1, st2, "chol_update",
                                                    std::max(1, num_sms() - 1), true)));
             GQ_TRY(cudaEventRecord(ev_rest, st2));
             rest_pending = true;
@@ -593,7 +593,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
                 EpiMats o;
                 o.t_hi = Mat{w.TT_hi, N, N, N};
                 o.t_lo = Mat{w.TT_lo, N, N, N};
-                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(rsh, rsl, uth, utl, o, p, (int)batch, st, "inv_bu")));
+                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rsh, rsl, uth, utl, o, p, (int)batch, st, "inv_bu")));
             }
             {   // U_b = -U_a T -> U (public, clipped), U split, UT split
                 gq::GemmArgs p = gemm_args((int)s, (int)cs, (int)s);
@@ -621,7 +621,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
                 o.s_lo = Mat{w.U_lo, N, N, N};
                 o.t_hi = Mat{w.UT_hi, N, N, N};
                 o.t_lo = Mat{w.UT_lo, N, N, N};
-                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2>(uh, ul, tth, ttl, o, p, (int)batch, st, "inv_ub")));
+                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(uh, ul, tth, ttl, o, p, (int)batch, st, "inv_ub")));
             }
         }
     }

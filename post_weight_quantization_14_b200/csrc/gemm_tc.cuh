@@ -10,6 +10,13 @@
 // KIND_TF32X3 : A = A_hi + A_lo and B = B_hi + B_lo given as two tf32 arrays each;
 //               three MMAs per 8-element K step (hi*hi + hi*lo + lo*hi), which keeps
 //               about fp32 accuracy on the tf32 tensor pipe.
+// KIND_TF32X4 : the same operands with the lo*lo product added (four MMAs per K step).
+//
+// Segmented accumulation (SEG > 0): the tensor pipe's fp32 accumulation error grows with
+// the number of MMAs accumulated in place, so every SEG MMA k-steps the accumulator is
+// handed to the epilogue, which adds it into a running sum in tensor memory with
+// round-to-nearest fp32 adds; for the tf32 kinds the small cross products go to an
+// accumulator of their own, so segments hold hi*hi products only.
 //
 // Persistent and warp-specialised: each CTA walks tiles blockIdx.x, +gridDim.x, ...
 // Warp 0 issues TMA into a ring of STAGES operand buffers that runs across tiles;
@@ -28,7 +35,7 @@
 
 namespace gq {
 
-enum : int { KIND_BF16 = 0, KIND_TF32X3 = 1 };
+enum : int { KIND_BF16 = 0, KIND_TF32X3 = 1, KIND_TF32X4 = 2 };
 
 struct GemmArgs {
     int M, N, K;
@@ -36,7 +43,8 @@ struct GemmArgs {
     int b_row0, b_col0, b_zrow, b_zcol;   // B(j,k) at map (x = b_col0 + k, y = b_row0 + j)
     int tiles_m, tiles_n;
     int batch;        // independent problems in the launch (offsets *_z* per problem)
-    int triangular;   // enumerate only tiles with nt >= mt
+    int triangular;   // enumerate only tiles that reach the upper triangle (nt >= tri_r * mt)
+    int tri_r;        // tile M / tile N for triangular enumeration
     int k_from_m0;    // K range of a tile starts at its m0 (A upper triangular in (i,k))
     int k_to_n1;      // K range of a tile ends at n0 + tile N (B zero for k > j)
     float alpha, beta;
@@ -83,6 +91,14 @@ __host__ __device__ constexpr int gemm_smem_bytes() {
     return STAGES * GemmCfg<KIND, TBN>::STAGE_BYTES + epi_bytes<TBN>() + 1024 + 256;
 }
 
+// Tiles of one problem: all of them, or (triangular) in row mt those with nt >= r * mt.
+__host__ __device__ inline int tiles_of(int tiles_m, int tiles_n, int triangular, int r) {
+    if (!triangular) return tiles_m * tiles_n;
+    int t = 0;
+    for (int mt = 0; mt < tiles_m; ++mt) t += max(0, tiles_n - r * mt);
+    return t;
+}
+
 __device__ __forceinline__ void tile_coords(const GemmArgs& p, int t, int& mt, int& nt) {
     if (!p.triangular) {
         mt = t / p.tiles_n;
@@ -92,13 +108,13 @@ __device__ __forceinline__ void tile_coords(const GemmArgs& p, int t, int& mt, i
     int row = 0;
     int rem = t;
     while (row < p.tiles_m) {
-        int cnt = p.tiles_n - row;
+        const int cnt = max(0, p.tiles_n - p.tri_r * row);
         if (rem < cnt) break;
         rem -= cnt;
         ++row;
     }
     mt = row;
-    nt = row + rem;
+    nt = p.tri_r * row + rem;
 }
 
 struct TileInfo {
@@ -158,7 +174,58 @@ __device__ __forceinline__ void emit_block(uint8_t* box, int lane, const float (
     }
 }
 
-template <int KIND, int STAGES, int TBN>
+// Error-free sum: s + e == a + b exactly (Knuth's two-sum, round-to-nearest).
+__device__ __forceinline__ void two_sum(float a, float b, float& s, float& e) {
+    s = __fadd_rn(a, b);
+    const float bb = __fsub_rn(s, a);
+    e = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
+}
+
+// Chunk c (32 columns, this warp's 32 lanes) of a tile's final accumulator: the last
+// segment at acc, plus (multi) the running sum of the earlier segments, plus (XACC) the
+// cross-product accumulator.  Layout as in tc_gemm_kernel.
+template <int TBN, bool XACC, bool TSUM>
+__device__ __forceinline__ void fetch_chunk(uint32_t tmem, uint32_t acc, uint32_t lane_off, int c, bool multi,
+                                            uint32_t (&r)[32]) {
+    constexpr int SUM_HI = 2 * TBN, XOFF = 3 * TBN, SUM_LO = (XACC ? 4 : 3) * TBN;
+    tmem_ld_32x32b_x32(acc + (uint32_t)(c * 32), r);
+    float lo[32];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) lo[u] = 0.f;
+    if (XACC) {
+        uint32_t x[32];
+        tmem_ld_32x32b_x32(tmem + (uint32_t)(XOFF + c * 32) + lane_off, x);
+        tmem_ld_wait();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) lo[u] = __uint_as_float(x[u]);
+    }
+    if (multi) {
+        uint32_t h[32];
+        tmem_ld_32x32b_x32(tmem + (uint32_t)(SUM_HI + c * 32) + lane_off, h);
+        if (TSUM) {
+            uint32_t l[32];
+            tmem_ld_32x32b_x32(tmem + (uint32_t)(SUM_LO + c * 32) + lane_off, l);
+            tmem_ld_wait();
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+                float s, e;
+                two_sum(__uint_as_float(h[u]), __uint_as_float(r[u]), s, e);
+                lo[u] += __uint_as_float(l[u]) + e;
+                r[u] = __float_as_uint(s);
+            }
+        } else {
+            tmem_ld_wait();
+#pragma unroll
+            for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(__uint_as_float(h[u]) + __uint_as_float(r[u]));
+        }
+    } else {
+        tmem_ld_wait();
+    }
+#pragma unroll
+    for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) + lo[u]);
+}
+
+template <int KIND, int STAGES, int TBN, int SEG>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
                    const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mB2,
@@ -167,7 +234,18 @@ __global__ void __launch_bounds__(192, 1)
     constexpr int KT = Cfg::KT, NOPS = Cfg::NOPS, STAGE_BYTES = Cfg::STAGE_BYTES;
     constexpr int A_BYTES = BM * 128;
     constexpr int B_BYTES = TBN * 128;
-    constexpr uint32_t TMEM_COLS = 2 * TBN;  // two accumulators
+    // Two accumulators.  Segmented accumulation adds the running sum of a tile's segments
+    // and, for the tf32 kinds, an accumulator of the small cross products (hi*lo + lo*hi)
+    // that spans the whole tile, so each segment accumulates only hi*hi products.
+    constexpr bool XACC = SEG > 0 && KIND != KIND_BF16;
+    // Where it fits, the running sum is kept as an unevaluated pair hi + lo updated by
+    // two-sum, so adding the segments is exact up to the final rounding.
+    constexpr bool TSUM = SEG > 0 && ((XACC ? 5 : 4) * TBN <= 512);
+    constexpr int SUM_HI = 2 * TBN, XOFF = 3 * TBN, SUM_LO = (XACC ? 4 : 3) * TBN;
+    constexpr int TMEM_NEED = SEG > 0 ? (XACC ? 4 : 3) * TBN + (TSUM ? TBN : 0) : 2 * TBN;
+    constexpr uint32_t TMEM_COLS = TMEM_NEED <= 32 ? 32u : TMEM_NEED <= 64 ? 64u : TMEM_NEED <= 128 ? 128u
+                                 : TMEM_NEED <= 256 ? 256u : 512u;
+    static_assert(TMEM_NEED <= 512, "tensor memory columns");
     constexpr int NCHUNK = TBN / 32;
 
     extern __shared__ uint8_t smem_raw[];
@@ -182,7 +260,7 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cin_bar + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tiles_per_batch = p.triangular ? p.tiles_m * (p.tiles_m + 1) / 2 : p.tiles_m * p.tiles_n;
+    const int tiles_per_batch = tiles_of(p.tiles_m, p.tiles_n, p.triangular, p.tri_r);
     const int total = tiles_per_batch * p.batch;
 
     if (threadIdx.x == 0) {
@@ -244,18 +322,36 @@ __global__ void __launch_bounds__(192, 1)
         constexpr uint32_t idesc = make_idesc(KIND == KIND_BF16 ? 1u : 2u, BM, TBN);
         uint32_t kiter = 0;
         bool ok = true;
-        int local = 0;
-        for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++local) {
+        int seg = 0;   // accumulator segments issued by this CTA (buffer = seg & 1)
+        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             const TileInfo ti = tile_info<KT, TBN>(p, w, tiles_per_batch);
-            const int buf = local & 1;
-            const uint32_t use = (uint32_t)(local >> 1);
-            if (!mbar_wait(&tempty_bar[buf], (use & 1) ^ 1, w)) {
+            const int nkk = 4 * ti.nk;                        // MMA k-steps of the tile
+            const int segk = SEG > 0 ? SEG : max(nkk, 1);     // k-steps per segment
+            const uint32_t xacc = tmem + (uint32_t)(3 * TBN);
+            if (XACC && seg > 0) {   // the previous tile's cross accumulator has been read
+                const int pb = (seg - 1) & 1;
+                if (!mbar_wait(&tempty_bar[pb], (uint32_t)((seg - 1) >> 1) & 1, w)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+            }
+            // open segment: wait until its accumulator buffer has been drained
+            auto open_segment = [&](uint32_t& acc_out) -> bool {
+                const int buf = seg & 1;
+                if (!mbar_wait(&tempty_bar[buf], (uint32_t)((seg >> 1) & 1) ^ 1u, w)) return false;
+                tc_fence_after();
+                acc_out = tmem + (uint32_t)(buf * TBN);
+                return true;
+            };
+            uint32_t acc = 0;
+            if (!open_segment(acc)) {
                 ok = false;
                 break;
             }
-            tc_fence_after();
-            const uint32_t acc = tmem + (uint32_t)(buf * TBN);
-            for (int kt = 0; kt < ti.nk; ++kt, ++kiter) {
+            int kkc = 0;      // k-steps issued in this tile
+            int segpos = 0;   // k-steps issued in the open segment
+            for (int kt = 0; kt < ti.nk && ok; ++kt, ++kiter) {
                 const int s = kiter % STAGES;
                 const uint32_t it = kiter / STAGES;
                 if (!mbar_wait(&full_bar[s], it & 1, w)) {
@@ -267,20 +363,40 @@ __global__ void __launch_bounds__(192, 1)
                 const uint32_t a_hi = st, a_lo = st + A_BYTES;
                 const uint32_t b_hi = st + NOPS * A_BYTES, b_lo = b_hi + B_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
+                for (int kk = 0; kk < 4; ++kk, ++kkc, ++segpos) {
+                    if (SEG > 0 && segpos == segk) {   // close the segment, open the next
+                        umma_commit(&tfull_bar[seg & 1]);
+                        ++seg;
+                        segpos = 0;
+                        if (!open_segment(acc)) {
+                            ok = false;
+                            break;
+                        }
+                    }
                     const uint32_t off = kk * 32;
-                    const uint32_t acc0 = (kt > 0 || kk > 0) ? 1u : 0u;
+                    const uint32_t acc0 = segpos > 0 ? 1u : 0u;
                     if (KIND == KIND_BF16) {
                         umma_bf16(acc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_hi + off), idesc, acc0);
+                    } else if (XACC) {
+                        const uint32_t x0 = kkc > 0 ? 1u : 0u;
+                        umma_tf32(acc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_hi + off), idesc, acc0);
+                        umma_tf32(xacc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_lo + off), idesc, x0);
+                        umma_tf32(xacc, desc_sw128_kmajor(a_lo + off), desc_sw128_kmajor(b_hi + off), idesc, 1u);
+                        if (KIND == KIND_TF32X4)
+                            umma_tf32(xacc, desc_sw128_kmajor(a_lo + off), desc_sw128_kmajor(b_lo + off), idesc, 1u);
                     } else {
                         umma_tf32(acc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_hi + off), idesc, acc0);
                         umma_tf32(acc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_lo + off), idesc, 1u);
                         umma_tf32(acc, desc_sw128_kmajor(a_lo + off), desc_sw128_kmajor(b_hi + off), idesc, 1u);
+                        if (KIND == KIND_TF32X4)
+                            umma_tf32(acc, desc_sw128_kmajor(a_lo + off), desc_sw128_kmajor(b_lo + off), idesc, 1u);
                     }
                 }
                 umma_commit(&empty_bar[s]);
             }
-            umma_commit(&tfull_bar[buf]);
+            if (!ok) break;
+            umma_commit(&tfull_bar[seg & 1]);
+            ++seg;
         }
     } else if (warp >= 2) {
         // ---------------- epilogue: warp q owns accumulator rows 32q .. 32q+31 of every tile
@@ -291,17 +407,75 @@ __global__ void __launch_bounds__(192, 1)
         uint8_t* cbox = wreg;
         uint8_t* kb = use_c ? wreg + NCHUNK * kBoxBytes : wreg;             // staging box
         float* stage_t = reinterpret_cast<float*>(wreg);   // register-path staging (own region)
-        int local = 0;
+        int seg = 0;
         uint32_t cin_use = 0;
         bool alive = true;
-        for (int w = blockIdx.x; w < total && alive; w += gridDim.x, ++local) {
+        for (int w = blockIdx.x; w < total && alive; w += gridDim.x) {
             const TileInfo ti = tile_info<KT, TBN>(p, w, tiles_per_batch);
-            const int buf = local & 1;
-            const uint32_t use = (uint32_t)(local >> 1);
-            const bool ok = mbar_wait(&tfull_bar[buf], use & 1, w);
+            const int nkk = 4 * ti.nk;
+            const int segk = SEG > 0 ? SEG : max(nkk, 1);
+            const int nseg = max(1, (nkk + segk - 1) / segk);
+            const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+            bool ok = true;
+            // Segments before the last: add the accumulator into the running sum (TMEM
+            // columns SUM_HI .., and SUM_LO .. for two-sum) with round-to-nearest fp32
+            // arithmetic, then release the buffer.
+            for (int sg = 0; sg + 1 < nseg && ok; ++sg, ++seg) {
+                const int sb = seg & 1;
+                ok = mbar_wait(&tfull_bar[sb], (uint32_t)(seg >> 1) & 1, w);
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < NCHUNK; ++c) {
+                    const uint32_t src = tmem + (uint32_t)(sb * TBN + c * 32) + lane_off;
+                    const uint32_t dhi = tmem + (uint32_t)(SUM_HI + c * 32) + lane_off;
+                    const uint32_t dlo = tmem + (uint32_t)(SUM_LO + c * 32) + lane_off;
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(src, r);
+                    if (sg > 0) {
+                        uint32_t t[32];
+                        tmem_ld_32x32b_x32(dhi, t);
+                        if (TSUM) {
+                            uint32_t e[32];
+                            tmem_ld_32x32b_x32(dlo, e);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int u = 0; u < 32; ++u) {
+                                float s, er;
+                                two_sum(__uint_as_float(t[u]), __uint_as_float(r[u]), s, er);
+                                r[u] = __float_as_uint(s);
+                                e[u] = __float_as_uint(__uint_as_float(e[u]) + er);
+                            }
+                            tmem_st_32x32b_x32(dlo, e);
+                        } else {
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int u = 0; u < 32; ++u)
+                                r[u] = __float_as_uint(__uint_as_float(r[u]) + __uint_as_float(t[u]));
+                        }
+                    } else {
+                        tmem_ld_wait();
+                        if (TSUM) {
+                            uint32_t e[32];
+#pragma unroll
+                            for (int u = 0; u < 32; ++u) e[u] = 0u;
+                            tmem_st_32x32b_x32(dlo, e);
+                        }
+                    }
+                    tmem_st_32x32b_x32(dhi, r);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty_bar[sb]);
+            }
+            const int buf = seg & 1;
+            const uint32_t use = (uint32_t)(seg >> 1);
+            ++seg;
+            ok = ok && mbar_wait(&tfull_bar[buf], use & 1, w);
             alive = ok;
             tc_fence_after();
-            const uint32_t acc = tmem + (uint32_t)(buf * TBN) + ((uint32_t)(q * 32) << 16);
+            const uint32_t acc = tmem + (uint32_t)(buf * TBN) + lane_off;
+            const bool multi = nseg > 1;   // the last segment joins a running sum
             const int z = ti.z, n0 = ti.n0, mt = ti.mt, nt = ti.nt;
             const int zc_x = p.c_col0 + z * p.c_zcol, zc_y = p.c_row0 + z * p.c_zrow;
             const int iy = ti.m0 + 32 * q;
@@ -330,8 +504,7 @@ __global__ void __launch_bounds__(192, 1)
                     const int j0 = n0 + c * 32;
                     uint32_t r[32];
                     if (ti.nk > 0 && ok) {
-                        tmem_ld_32x32b_x32(acc + (uint32_t)(c * 32), r);
-                        tmem_ld_wait();
+                        fetch_chunk<TBN, XACC, TSUM>(tmem, acc, lane_off, c, multi, r);
                     } else {
 #pragma unroll
                         for (int t = 0; t < 32; ++t) r[t] = 0u;
@@ -386,8 +559,7 @@ __global__ void __launch_bounds__(192, 1)
                     const int j0 = n0 + c * 32;
                     uint32_t r[32];
                     if (ti.nk > 0 && ok) {
-                        tmem_ld_32x32b_x32(acc + (uint32_t)(c * 32), r);
-                        tmem_ld_wait();
+                        fetch_chunk<TBN, XACC, TSUM>(tmem, acc, lane_off, c, multi, r);
                     } else {
 #pragma unroll
                         for (int t = 0; t < 32; ++t) r[t] = 0u;
@@ -477,20 +649,20 @@ bool aux_stream(cudaStream_t* st, cudaEvent_t* ev0, cudaEvent_t* ev1);
 // C is read (beta != 0) only where it is also written.
 inline bool epilogue_fits(const gq::GemmArgs& p) { return p.beta == 0.f || p.write_c; }
 
-// Launch D = A B^T with the given epilogue.  For KIND_TF32X3 a2/b2 are the lo parts.
+// Launch D = A B^T with the given epilogue.  For the tf32 kinds a2/b2 are the lo parts.
 // max_ctas > 0 caps the persistent grid (to leave SMs to a concurrent kernel).  after_event:
 // the launch follows a cross-stream event wait, so it is not a programmatic dependent.
-template <int KIND, int STAGES, int TBN = gq::BN>
+template <int KIND, int STAGES, int TBN = gq::BN, int SEG = 0>
 cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2, const EpiMats& o, gq::GemmArgs p,
                         int batch, cudaStream_t stream, const char* name, int max_ctas = 0,
                         bool after_event = false) {
     using Cfg = gq::GemmCfg<KIND, TBN>;
     const int eb = (KIND == gq::KIND_BF16) ? 2 : 4;
     CUtensorMap ma, ma2, mb, mb2, mc;
-    if ((p.triangular || p.mirror) && TBN != gq::BM) return cudaErrorInvalidValue;   // square tiles only
+    if (p.mirror && TBN != gq::BM) return cudaErrorInvalidValue;   // mirrored outputs: square tiles only
     if (!make_tmap_2d(&ma, a.ptr, eb, a.rows, a.cols, a.ld, gq::BM, Cfg::KT)) return cudaErrorInvalidValue;
     if (!make_tmap_2d(&mb, b.ptr, eb, b.rows, b.cols, b.ld, TBN, Cfg::KT)) return cudaErrorInvalidValue;
-    if (KIND == gq::KIND_TF32X3) {
+    if (KIND != gq::KIND_BF16) {
         if (!make_tmap_2d(&ma2, a2.ptr, eb, a2.rows, a2.cols, a2.ld, gq::BM, Cfg::KT)) return cudaErrorInvalidValue;
         if (!make_tmap_2d(&mb2, b2.ptr, eb, b2.rows, b2.cols, b2.ld, TBN, Cfg::KT)) return cudaErrorInvalidValue;
     } else {
@@ -516,11 +688,11 @@ cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2
     p.tiles_m = (p.M + gq::BM - 1) / gq::BM;
     p.tiles_n = (p.N + TBN - 1) / TBN;
     p.batch = batch;
-    const long long tiles = (p.triangular ? (long long)p.tiles_m * (p.tiles_m + 1) / 2
-                                          : (long long)p.tiles_m * p.tiles_n) * batch;
+    p.tri_r = gq::BM / TBN;
+    const long long tiles = (long long)gq::tiles_of(p.tiles_m, p.tiles_n, p.triangular, p.tri_r) * batch;
     if (tiles <= 0) return cudaSuccess;
     constexpr int smem = gq::gemm_smem_bytes<KIND, STAGES, TBN>();
-    auto kern = gq::tc_gemm_kernel<KIND, STAGES, TBN>;
+    auto kern = gq::tc_gemm_kernel<KIND, STAGES, TBN, SEG>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)std::min<long long>(tiles, max_ctas > 0 ? max_ctas : num_sms());

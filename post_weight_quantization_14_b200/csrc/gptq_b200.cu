@@ -448,9 +448,10 @@ static cudaError_t fixed_gemm(const Mat& a, const Mat& a2, const Mat& c, gq::Gem
     p.tiles_m = (p.M + gq::BM - 1) / gq::BM;
     p.tiles_n = (p.N + gq::BN - 1) / gq::BN;
     p.batch = 1;
+    p.tri_r = 1;
     const long long tiles = (long long)p.tiles_m * (p.tiles_m + 1) / 2;
     constexpr int smem = gq::gemm_smem_bytes<KIND, STAGES, gq::BN>();
-    auto kern = gq::tc_gemm_kernel<KIND, STAGES, gq::BN>;
+    auto kern = gq::tc_gemm_kernel<KIND, STAGES, gq::BN, 0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int sms = 0;

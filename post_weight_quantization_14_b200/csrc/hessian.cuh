@@ -80,7 +80,7 @@ inline cudaError_t hessian_run(const void* X, gptq_dtype xt, long long n, long l
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         Mat m{XT, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
-        return launch_gemm<gq::KIND_BF16, 4>(m, m, m, m, o, p, 1, st, "hessian_syrk");
+        return launch_gemm<gq::KIND_BF16, 4, 128, 16>(m, m, m, m, o, p, 1, st, "hessian_syrk");
     }
     float* hi = static_cast<float*>(ws);
     float* lo = hi + d_in * np;
@@ -92,7 +92,7 @@ inline cudaError_t hessian_run(const void* X, gptq_dtype xt, long long n, long l
     if (e != cudaSuccess) return e;
     Mat mh{hi, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
     Mat ml{lo, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
-    return launch_gemm<gq::KIND_TF32X3, 2>(mh, ml, mh, ml, o, p, 1, st, "hessian_syrk");
+    return launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(mh, ml, mh, ml, o, p, 1, st, "hessian_syrk");
 }
 
 }  // namespace gqh

@@ -97,8 +97,6 @@ def test_ffn_up_11008x4096_3bit_sym():
 
 
 @pytest.mark.slow
-@pytest.mark.xfail(strict=False, reason="U of this all-nonnegative-activation layer misses the 1e-4 gate in fp32 "
-                                        "(fp32 LAPACK reaches 6.5e-4 on the same matrix); see DESIGN precision findings")
 def test_ffn_down_4096x11008_2bit_then_per_row_4bit():
     layer = I.make_layer("ffn_down", seed=0)
     gpu, bufs, Uo, _ = _full_check(layer, layer.spec, sample_rows=128, full_H=False)
