@@ -142,14 +142,20 @@ def run_reference(args, rank: int, world: int) -> None:
 # ---------------------------------------------------------------- GPU leg
 
 CHOL_KERNELS = ("chol_leaf", "chol_panel", "chol_update", "chol_update_next", "inv_bu", "inv_ub", "split_panel",
-                "damp_copy", "diag_mean", "zero_lower")
-END_TO_END_BOUND_MS = 0.445   # sum of the stage bounds for this layer (roofline)
+                "damp_copy", "diag_mean", "zero_lower", "chol_diag_out")
+QUANT_KERNELS = ("colloop", "trailing_update", "trailing_update_sb", "up_prep", "ut_split", "pack_zeros", "row_params")
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu --set full capture of this
+# workload, for kernels whose launches all do the same work (the kernel's ncu summary under profiles/).
+TRAFFIC_PER_LAUNCH = {"chol_leaf": 142336, "colloop": 2236416, "hessian_syrk": 16900608 + 10929408}
+# Sum of the stage bounds for this layer: Hessian 21.0 us (bf16), factor + invert 168.1 us and
+# trailing updates 244.3 us (3xTF32 at a third of bf16 x 1.1/2.25), column loop 11.6 us (HBM).
+END_TO_END_BOUND_MS = 0.445
 
 
 def kernel_rooflines(kernel_ms: dict, launches: dict, hbm: float, bf16: float, peak_kind: str) -> dict:
     """Achieved vs peak per kernel class, from algorithmic work and measured per-step time.
 
-    Algorithmic work (roofline table):
+    Algorithmic work:
       trailing_update  2 * d_out * (d_in - e) * 128 flops per launch, summed over the layer; 3xTF32
       chol_panel/update, inv_*  2/3 d_in^3 flops for the whole factorization (shared); 3xTF32
       hessian_syrk     n * d_in * (d_in + 1) flops; bf16
@@ -169,9 +175,16 @@ def kernel_rooflines(kernel_ms: dict, launches: dict, hbm: float, bf16: float, p
         scale = 1e9 if unit == "GB/s" else 1e12
         ach = work / (ms / 1e3) / scale
         out[name] = {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
-                     "traffic": None, "launches": launches.get(name), "note": note}
+                     "traffic": TRAFFIC_PER_LAUNCH.get(name), "launches": launches.get(name), "note": note}
     trailing = sum(2.0 * d_out * (d_in - (b + 1) * B) * B for b in range(d_in // B) if (b + 1) * B < d_in)
-    add("trailing_update", "tensor", trailing, "TFLOP/s", tf32x3, f"3xTF32 ({peak_kind} bf16 x 1.1/2.25 / 3)")
+    tr_ms = kernel_ms.get("trailing_update", 0) + kernel_ms.get("trailing_update_sb", 0)
+    if tr_ms:
+        ach = trailing / (tr_ms / 1e3) / 1e12
+        out["trailing_update"] = {"bound": "tensor", "achieved": ach, "peak": tf32x3, "unit": "TFLOP/s",
+                                  "frac": ach / tf32x3, "traffic": None,
+                                  "launches": launches.get("trailing_update", 0) + launches.get("trailing_update_sb", 0),
+                                  "note": f"all trailing updates (per block and per superblock, {tr_ms:.3f} ms); "
+                                          f"3xTF32 ({peak_kind} bf16 x 1.1/2.25 / 3)"}
     add("hessian_syrk", "tensor", 1.0 * n * d_in * (d_in + 1), "TFLOP/s", bf16, f"bf16 {peak_kind} burst")
     col_bytes = 4.0 * d_out * d_in + BITS / 8 * d_out * d_in + (2 + BITS / 8) * d_out * (d_in // GROUP)
     add("colloop", "hbm", col_bytes, "GB/s", hbm, f"HBM {peak_kind}; latency chain of d_in rounding steps per row")
@@ -282,9 +295,9 @@ def main():
     roof_all = kernel_rooflines(kernel_ms, kernel_launches, hbm, bf16, peak_kind)
     stage_ms = {"hessian": kernel_ms.get("hessian_syrk", 0) + kernel_ms.get("transpose_x", 0),
                 "prepare_hinv": sum(v for k, v in kernel_ms.items() if k in CHOL_KERNELS),
-                "quantize": sum(kernel_ms.get(k, 0) for k in ("colloop", "trailing_update", "up_prep", "ut_split",
-                                                             "pack_zeros", "row_params"))}
-    dom = max((k for k in kernel_ms if k in roof_all), key=kernel_ms.get)
+                "quantize": sum(kernel_ms.get(k, 0) for k in QUANT_KERNELS)}
+    dom = max((k for k in roof_all), key=lambda k: kernel_ms.get(k, 0) + (kernel_ms.get("trailing_update_sb", 0)
+                                                                         if k == "trailing_update" else 0))
     roofline = dict(roof_all[dom])
     roofline["kernel"] = dom
     roofline["share_of_step"] = kernel_ms[dom] / max(1e-9, sum(kernel_ms.values()))
