@@ -141,7 +141,8 @@ def run_reference(args, rank: int, world: int) -> None:
 
 # ---------------------------------------------------------------- GPU leg
 
-CHOL_KERNELS = ("chol_leaf", "chol_panel", "chol_update", "chol_update_next", "inv_bu", "inv_ub", "split_panel",
+CHOL_KERNELS = ("chol_leaf", "chol_panel", "chol_update", "chol_update_next", "chol_update_u2", "inv_bu", "inv_ub",
+                "split_panel",
                 "damp_copy", "diag_mean", "zero_lower", "chol_diag_out")
 QUANT_KERNELS = ("colloop", "trailing_update", "trailing_update_sb", "up_prep", "ut_split", "pack_zeros", "row_params")
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu --set full capture of this
@@ -191,10 +192,11 @@ def kernel_rooflines(kernel_ms: dict, launches: dict, hbm: float, bf16: float, p
     nleaf = d_in // B
     add("chol_leaf", "alu", nleaf * 2.0 * (2.0 / 3.0) * B ** 3, "TFLOP/s", sm_fp32,
         "one CTA per 128x128 leaf: peak = one SM's fp32 FMA rate at 1965 MHz")
-    gemm_ms = sum(kernel_ms.get(k, 0) for k in ("chol_panel", "chol_update", "chol_update_next", "inv_bu", "inv_ub"))
+    fact = ("chol_panel", "chol_update", "chol_update_next", "chol_update_u2", "inv_bu", "inv_ub")
+    gemm_ms = sum(kernel_ms.get(k, 0) for k in fact)
     if gemm_ms:
         ach = (2.0 / 3.0) * d_in ** 3 / (gemm_ms / 1e3) / 1e12
-        for k in ("chol_panel", "chol_update", "chol_update_next", "inv_bu", "inv_ub"):
+        for k in fact:
             if k in kernel_ms:
                 out[k] = {"bound": "tensor", "achieved": ach, "peak": tf32x3, "unit": "TFLOP/s", "frac": ach / tf32x3,
                           "traffic": None, "launches": launches.get(k),
@@ -242,8 +244,15 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step():
-        G.quantize_layer(W, X, buffers=bufs)
+    def step(marks=None):
+        # the three stages of G.quantize_layer, with optional events between them
+        G.gptq_hessian_accumulate(X, bufs.H, accumulate=False, workspace=bufs.ws)
+        if marks:
+            marks[0].record(stream)
+        G.gptq_prepare_hinv(bufs.H, bufs.U, cfg.damp_rel, workspace=bufs.ws)
+        if marks:
+            marks[1].record(stream)
+        G.gptq_quantize_layer(W, bufs.U, cfg, bufs.qweight, bufs.scales, bufs.qzeros, bufs.err_sq, workspace=bufs.ws)
 
     for _ in range(args.warmup):
         W.copy_(W0)
@@ -251,17 +260,18 @@ def main():
     G.gptq_sync_status()
 
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    marks = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     sampler = ClockSampler(local)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.3)
-    for a, b in evs:
+    for (a, b), m in zip(evs, marks):
         W.copy_(W0)
         flush.fill_(1)
         a.record(stream)
-        step()
+        step(m)
         b.record(stream)
     torch.cuda.synchronize()
     if dist:
@@ -269,6 +279,10 @@ def main():
     clocks = sampler.stop()
     G.gptq_sync_status()
     step_ms = [a.elapsed_time(b) for a, b in evs]
+    # stage times of the timed steps (events between the three C-ABI calls)
+    stage_timed = {"hessian": statistics.median(a.elapsed_time(m[0]) for (a, _), m in zip(evs, marks)),
+                   "prepare_hinv": statistics.median(m[0].elapsed_time(m[1]) for m in marks),
+                   "quantize": statistics.median(m[1].elapsed_time(b) for (_, b), m in zip(evs, marks))}
     total_ms = sum(step_ms)
     if dist:
         t = torch.tensor([total_ms], device=dev)
@@ -349,7 +363,8 @@ def main():
                 "roofline": roofline,
                 "roofline_by_kernel": roof_all,
                 "e2e_roofline": {"bound_ms": END_TO_END_BOUND_MS, "frac": END_TO_END_BOUND_MS / ms_per_step},
-                "stage_ms": stage_ms,
+                "stage_ms": stage_timed,
+                "stage_ms_instrumented": stage_ms,
                 "kernel_ms_per_step": kernel_ms,
                 "kernel_launches_per_step": kernel_launches,
                 "cpu_baseline": cpu,

@@ -40,27 +40,39 @@ __global__ void diag_mean_kernel(const float* __restrict__ H, long long d, float
 }
 
 // A (n x n) = Hd with only the upper triangle of H read; padding gets identity.
-__global__ void damp_copy_kernel(const float* __restrict__ H, long long d, long long n,
-                                 const float* __restrict__ lam, float* __restrict__ A) {
-    __shared__ float tile[32][33];
-    const long long bi = blockIdx.y, bj = blockIdx.x;
-    const bool lower = bi > bj;
-    const long long si = lower ? bj : bi, sj = lower ? bi : bj;  // source tile (upper)
+// A = H + lambda I on the upper 128-block triangle (bi <= bj, one CTA per block), from
+// H's upper triangle; diagonal blocks are symmetrised in full; indices >= d pad A with the
+// identity.  The strictly lower blocks of A are never read by the factorization and are
+// not written.
+__global__ void __launch_bounds__(256) damp_copy_kernel(const float* __restrict__ H, long long d, long long n,
+                                                        const float* __restrict__ lam, float* __restrict__ A) {
+    const int bi = blockIdx.y, bj = blockIdx.x;
+    if (bi > bj) return;
+    const long long r0 = (long long)bi * NB, c0 = (long long)bj * NB;
     const float l = lam[0];
-    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
-        const long long i = si * 32 + r, j = sj * 32 + threadIdx.x;
+    if (bi < bj) {
+        for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
+            const int r = e >> 5, c = (e & 31) * 4;
+            const long long i = r0 + r, j = c0 + c;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < d && j < d) {   // d % 4 == 0: a float4 is wholly inside or outside
+                v = *reinterpret_cast<const float4*>(H + i * d + j);
+                if (!(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w)))
+                    record_status(GPTQ_ERR_NONFINITE, i * d + j);
+            }
+            *reinterpret_cast<float4*>(A + i * n + j) = v;
+        }
+        return;
+    }
+    // diagonal block: A[i][j] = H[min(i,j)][max(i,j)] (the few transposed reads are strided)
+    for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+        const int r = e >> 7, c = e & 127;
+        const long long i = r0 + r, j = c0 + c;
         float v = 0.f;
         if (i < d && j < d) {
-            v = H[i * d + j];
-            if (i <= j && !isfinite(v)) record_status(GPTQ_ERR_NONFINITE, i * d + j);
+            v = (r <= c) ? H[i * d + j] : H[j * d + i];
+            if (r <= c && !isfinite(v)) record_status(GPTQ_ERR_NONFINITE, i * d + j);
         }
-        tile[r][threadIdx.x] = v;
-    }
-    __syncthreads();
-    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
-        const long long i = bi * 32 + r, j = bj * 32 + threadIdx.x;
-        if (i >= n || j >= n) continue;
-        float v = lower ? tile[threadIdx.x][r] : tile[r][threadIdx.x];
         if (i == j) v = (i < d) ? v + l : 1.f;
         A[i * n + j] = v;
     }
@@ -82,12 +94,14 @@ __global__ void split_panel_kernel(const float* __restrict__ A, long long n, int
 
 // Zero the strictly-lower 128-blocks of the d x d output U (diagonal blocks are
 // written in full by chol_diag_out_kernel).
-__global__ void zero_lower_blocks_kernel(float* __restrict__ U, long long d) {
-    const long long total = d * d;
-    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-         e += (long long)gridDim.x * blockDim.x) {
-        const long long r = e / d, c = e % d;
-        if ((r >> 7) > (c >> 7)) U[e] = 0.f;
+__global__ void __launch_bounds__(256) zero_lower_blocks_kernel(float* __restrict__ U, long long d) {
+    const int bi = blockIdx.y, bj = blockIdx.x;   // one CTA per 128-block, strictly lower only
+    if (bi <= bj) return;
+    const long long r0 = (long long)bi * NB, c0 = (long long)bj * NB;
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
+        const long long i = r0 + (e >> 5), j = c0 + (e & 31) * 4;
+        if (i < d && j < d) *reinterpret_cast<float4*>(U + i * d + j) = z;   // d % 4 == 0
     }
 }
 
@@ -465,23 +479,26 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
     }
     GQ_TRY(cudaGetLastError());
     {
-        dim3 tb(32, 8), grid((unsigned)(n / 32), (unsigned)(n / 32));
+        const dim3 grid((unsigned)(n / gq::NB), (unsigned)(n / gq::NB));
         {
             gqh::TimedScope ts__("damp_copy", st);
-            gq::damp_copy_kernel<<<grid, tb, 0, st>>>(H, d, n, w.scal, w.A);
+            gq::damp_copy_kernel<<<grid, 256, 0, st>>>(H, d, n, w.scal, w.A);
         }
         GQ_TRY(cudaGetLastError());
     }
     const int leaf_smem = (int)sizeof(gq::LeafSmem);
     GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::chol_leaf_kernel), leaf_smem));
     const uint64_t N = (uint64_t)n;
-    // Look-ahead: the caller's stream carries the critical chain leaf -> panel -> update of
-    // the next block column; the rest of each Schur update runs on a helper stream next to
-    // the following leaf and panel, on at most SMs - 1 CTAs so the leaf finds an SM.
+    // Look-ahead of depth two.  The caller's stream carries the critical chain
+    // leaf(j) -> panel(j) -> update of block column j-1 by panel j.  A helper stream takes
+    // the rest of panel j's Schur update: first block column j-2 (u2), then everything left
+    // of it (rest), on at most SMs - 1 CTAs so the next leaf finds an SM.  Block column j-1
+    // has received, before its update by panel j, u2(j+1) and rest(p) for p >= j+2, which
+    // the helper stream runs in that order; so the chain waits only for u2(j+1).
     cudaStream_t st2;
-    cudaEvent_t ev_panel, ev_rest;
-    if (!aux_stream(&st2, &ev_panel, &ev_rest)) return cudaErrorUnknown;
-    bool rest_pending = false;
+    cudaEvent_t ev_panel, ev_u2;
+    if (!aux_stream(&st2, &ev_panel, &ev_u2)) return cudaErrorUnknown;
+    bool u2_pending = false, st2_used = false;
     Mat rh{w.RS_hi, N, N, N}, rl{w.RS_lo, N, N, N};
     for (int j = T - 1; j >= 0; --j) {
         const int jb = j * gq::NB;
@@ -509,10 +526,12 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
             Mat bh{w.U_hi, N, N, N}, bl{w.U_lo, N, N, N};
             GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(ah, al, bh, bl, o, p, 1, st, "chol_panel")));
         }
-        const int jn = jb - gq::NB;   // first column of the next block column
+        const int jn = jb - gq::NB;    // first column of block column j-1
+        const int jn2 = jn - gq::NB;   // first column of block column j-2
         if (j >= 2) GQ_TRY(cudaEventRecord(ev_panel, st));
-        if (rest_pending) GQ_TRY(cudaStreamWaitEvent(st, ev_rest, 0));   // it also wrote block column j-1
-        {   // next block column: A[0:jb, jn:jb] -= RS_panel RS_panel[jn:jb]^T, plus the next panel's split
+        const bool waited = u2_pending;
+        if (u2_pending) GQ_TRY(cudaStreamWaitEvent(st, ev_u2, 0));
+        {   // block column j-1: A[0:jb, jn:jb] -= RS_panel RS_panel[jn:jb]^T, plus the next panel's split
             gq::GemmArgs p = gemm_args(jb, gq::NB, gq::NB);
             p.a_col0 = jb;
             p.b_row0 = jn;
@@ -529,26 +548,47 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
                 o.s_lo = Mat{w.AP_lo, (uint64_t)jn, 128, 128};
             }
             GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, rh, rl, o, p, 1, st, "chol_update_next", 0,
-                                                        rest_pending)));
+                                                        waited)));
         }
-        if (j >= 2) {   // the rest: A[0:jn, 0:jn] -= RS RS^T (upper tiles), on the helper stream
+        u2_pending = false;
+        if (j >= 2) {   // helper stream: block column j-2, then the rest
             GQ_TRY(cudaStreamWaitEvent(st2, ev_panel, 0));
-            gq::GemmArgs p = gemm_args(jn, jn, gq::NB);
-            p.a_col0 = jb;
-            p.b_col0 = jb;
-            p.triangular = 1;
-            p.alpha = -1.f;
-            p.beta = 1.f;
-            p.write_c = 1;
-            EpiMats o;
-            o.c = Mat{w.A, N, N, N};
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rh, rl, rh, rl, o, p, 1, st2, "chol_update",
-                                                   std::max(1, num_sms() - 1), true)));
-            GQ_TRY(cudaEventRecord(ev_rest, st2));
-            rest_pending = true;
+            st2_used = true;
+            {   // u2: A[0:jn, jn2:jn] -= RS_panel RS_panel[jn2:jn]^T
+                gq::GemmArgs p = gemm_args(jn, gq::NB, gq::NB);
+                p.a_col0 = jb;
+                p.b_row0 = jn2;
+                p.b_col0 = jb;
+                p.alpha = -1.f;
+                p.beta = 1.f;
+                p.write_c = 1;
+                p.c_col0 = jn2;
+                EpiMats o;
+                o.c = Mat{w.A, N, N, N};
+                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, rh, rl, o, p, 1, st2, "chol_update_u2",
+                                                            std::max(1, num_sms() - 1), true)));
+            }
+            GQ_TRY(cudaEventRecord(ev_u2, st2));
+            u2_pending = true;
+            if (j >= 3) {   // rest: A[0:jn2, 0:jn2] -= RS RS^T (upper tiles)
+                gq::GemmArgs p = gemm_args(jn2, jn2, gq::NB);
+                p.a_col0 = jb;
+                p.b_col0 = jb;
+                p.triangular = 1;
+                p.alpha = -1.f;
+                p.beta = 1.f;
+                p.write_c = 1;
+                EpiMats o;
+                o.c = Mat{w.A, N, N, N};
+                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rh, rl, rh, rl, o, p, 1, st2, "chol_update",
+                                                       std::max(1, num_sms() - 1), true)));
+            }
         }
     }
-    if (rest_pending) GQ_TRY(cudaStreamWaitEvent(st, ev_rest, 0));
+    if (st2_used) {   // everything on the helper stream is done before the inverse
+        GQ_TRY(cudaEventRecord(ev_u2, st2));
+        GQ_TRY(cudaStreamWaitEvent(st, ev_u2, 0));
+    }
     {
         const int smem = (int)(gq::NB * (gq::NB + 1) * sizeof(float));
         GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::chol_diag_out_kernel), smem));
@@ -626,10 +666,10 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
         }
     }
     {
-        const long long tot = d * d;
         {
             gqh::TimedScope ts__("zero_lower", st);
-            gq::zero_lower_blocks_kernel<<<(unsigned)std::min<long long>((tot + 255) / 256, 8192), 256, 0, st>>>(U, d);
+            const unsigned nb = (unsigned)((d + gq::NB - 1) / gq::NB);
+            gq::zero_lower_blocks_kernel<<<dim3(nb, nb), 256, 0, st>>>(U, d);
         }
         GQ_TRY(cudaGetLastError());
     }

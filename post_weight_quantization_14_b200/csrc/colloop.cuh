@@ -87,12 +87,18 @@ struct QuadState {
 // Octs [t0, t1) of the block with LIVE register slots in use.  Slot i of lane k holds
 // column 8*(t + i) + k at oct t; the normalised U row of column c is stored shifted so
 // that its entry for slot i is at offset i (zeros for columns at or before c).
+// Per oct, the 8 lanes of a row first gather the oct's 8 current column values (one
+// shuffle each, all independent), then every lane runs the oct's 8 rounding steps itself
+// in registers (the same operations in the same order in all 8 lanes, so the results
+// agree exactly), and finally applies the 8 errors to its remaining slots in column
+// order.  The dependent chain of one rounding step has no shuffle in it.
 template <int BITS, int LIVE>
 __device__ __forceinline__ void run_octs(float (&wv)[SLOTS], int t0, int t1, QuadState& st, const ColArgs& p,
                                          ColSmem& S, int lane, int k, int rloc, long long row, bool row_ok) {
     constexpr unsigned FULL = 0xffffffffu;
     constexpr int MAXQ = (1 << BITS) - 1;
     const int g = p.g;
+    const int base = lane & ~(LPR - 1);
 #pragma unroll 1
     for (int t = t0; t < t1; ++t) {
         const int c8 = LPR * t;
@@ -131,26 +137,35 @@ __device__ __forceinline__ void run_octs(float (&wv)[SLOTS], int t0, int t1, Qua
                 p.zeros_u8[gi * p.d_out + row] = (uint8_t)(int)z;
             }
         }
+        // the oct's columns c8 .. c8+7 as they stand (slot 0 of the row's 8 lanes)
+        float v[LPR];
+#pragma unroll
+        for (int j = 0; j < LPR; ++j) v[j] = __shfl_sync(FULL, wv[0], base | j);
+        // its 8 rounding steps, with the in-oct propagation v[m] -= d_j U[c8+j][c8+m]
+        float dd[LPR];
         float my_r = 0.f, my_d = 0.f;
 #pragma unroll
-        for (int own = 0; own < LPR; ++own) {
-            const int c = c8 + own;
-            const float4* u = reinterpret_cast<const float4*>(S.up + c * UP_ROW + k * UP_LD);
-            float4 uu[LIVE / 4];
+        for (int j = 0; j < LPR; ++j) {
+            const float r = fminf(fmaxf(rintf(v[j] * st.inv_s), st.qlo), st.qhi);
+            const float d = fmaf(-r, st.s, v[j]);
+            dd[j] = d;
+            my_r = (k == j) ? r : my_r;
+            my_d = (k == j) ? d : my_d;
+            const float* urow = S.up + (c8 + j) * UP_ROW;   // slot 0 of lane m at offset m * UP_LD
 #pragma unroll
-            for (int q = 0; q < LIVE / 4; ++q) uu[q] = u[q];
-            const float x = wv[0] * st.inv_s;
-            const float r = fminf(fmaxf(rintf(x), st.qlo), st.qhi);
-            const float dd = fmaf(-r, st.s, wv[0]);
-            const float db = __shfl_sync(FULL, dd, (lane & ~(LPR - 1)) | own);
-            my_r = (k == own) ? r : my_r;
-            my_d = (k == own) ? dd : my_d;
+            for (int m = j + 1; m < LPR; ++m) v[m] = fmaf(-d, urow[m * UP_LD], v[m]);
+        }
+        // the errors applied to this lane's later slots, in column order
+#pragma unroll
+        for (int j = 0; j < LPR; ++j) {
+            const float4* u = reinterpret_cast<const float4*>(S.up + (c8 + j) * UP_ROW + k * UP_LD);
 #pragma unroll
             for (int q = 0; q < LIVE / 4; ++q) {
-                wv[4 * q + 0] = fmaf(-db, uu[q].x, wv[4 * q + 0]);
-                wv[4 * q + 1] = fmaf(-db, uu[q].y, wv[4 * q + 1]);
-                wv[4 * q + 2] = fmaf(-db, uu[q].z, wv[4 * q + 2]);
-                wv[4 * q + 3] = fmaf(-db, uu[q].w, wv[4 * q + 3]);
+                const float4 uu = u[q];
+                if (4 * q + 0 > 0) wv[4 * q + 0] = fmaf(-dd[j], uu.x, wv[4 * q + 0]);
+                wv[4 * q + 1] = fmaf(-dd[j], uu.y, wv[4 * q + 1]);
+                wv[4 * q + 2] = fmaf(-dd[j], uu.z, wv[4 * q + 2]);
+                wv[4 * q + 3] = fmaf(-dd[j], uu.w, wv[4 * q + 3]);
             }
         }
         S.codes[rloc][c8 + k] = (uint8_t)(int)(my_r - st.qlo);

@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(192, 1)
     // Where it fits, the running sum is kept as an unevaluated pair hi + lo updated by
     // two-sum, so adding the segments is exact up to the final rounding.
     constexpr bool TSUM = SEG > 0 && ((XACC ? 5 : 4) * TBN <= 512);
-    constexpr int SUM_HI = 2 * TBN, XOFF = 3 * TBN, SUM_LO = (XACC ? 4 : 3) * TBN;
+    constexpr int SUM_HI = 2 * TBN, SUM_LO = (XACC ? 4 : 3) * TBN;
     constexpr int TMEM_NEED = SEG > 0 ? (XACC ? 4 : 3) * TBN + (TSUM ? TBN : 0) : 2 * TBN;
     constexpr uint32_t TMEM_COLS = TMEM_NEED <= 32 ? 32u : TMEM_NEED <= 64 ? 64u : TMEM_NEED <= 128 ? 128u
                                  : TMEM_NEED <= 256 ? 256u : 512u;
