@@ -115,6 +115,26 @@ def oracle_layer_time(layer, rows_sample: int = 256) -> tuple[float, str, int]:
     return total, sample, len(os.sched_getaffinity(0))
 
 
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The job's time: the slowest rank's (identity without a process group)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank_step: float, steps: int, total_ms: float) -> float:
+    """Units all ranks processed per second over the (max-over-ranks) timed region."""
+    return world * units_per_rank_step * steps / (total_ms / 1e3)
+
+
+def layer_seed(rank: int) -> int:
+    """Each rank quantizes its own independent layer (weak scaling)."""
+    return rank
+
+
 def run_reference(args, rank: int, world: int) -> None:
     if rank != 0:
         return
@@ -235,7 +255,7 @@ def main():
     from post_weight_quantization_14_b200 import gptq as G
     from post_weight_quantization_14_b200 import inputs as I
 
-    layer = I.make_layer("attn", seed=rank)
+    layer = I.make_layer("attn", seed=layer_seed(rank))
     cfg = G.make_config(BITS, GROUP, SYM, 128, 0.01)
     W0 = torch.from_numpy(layer.W).to(dev)
     W = torch.empty_like(W0)
@@ -283,13 +303,9 @@ def main():
     stage_timed = {"hessian": statistics.median(a.elapsed_time(m[0]) for (a, _), m in zip(evs, marks)),
                    "prepare_hinv": statistics.median(m[0].elapsed_time(m[1]) for m in marks),
                    "quantize": statistics.median(m[1].elapsed_time(b) for (_, b), m in zip(evs, marks))}
-    total_ms = sum(step_ms)
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, dev)
     ms_per_step = total_ms / args.steps
-    value = world * D_OUT * D_IN * args.steps / (total_ms / 1e3)
+    value = job_throughput(world, D_OUT * D_IN, args.steps, total_ms)
 
     # per-kernel times (instrumented steps; every launch bracketed by CUDA events on its stream)
     G.gptq_timing_enable(True)
@@ -338,12 +354,8 @@ def main():
         qz_host.copy_(q.qzeros, non_blocking=True)
     eb.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = ea.elapsed_time(eb)
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * D_OUT * D_IN * e2e_steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(ea.elapsed_time(eb), dist, dev)
+    e2e_value = job_throughput(world, D_OUT * D_IN, e2e_steps, e2e_ms)
     h2d = W_host.numel() * 4 + X_host.numel() * 2
     d2h = qw_host.numel() * 4 + sc_host.numel() * 2 + qz_host.numel() * 4
 

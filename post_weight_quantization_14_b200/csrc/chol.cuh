@@ -618,6 +618,8 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
             }
             if (batch <= 0) continue;
             const int zs = (int)(2 * s);
+            // levels with few 128x128 tiles take 128x32 tiles (more SMs share the epilogue stores)
+            const bool narrow = 4 * batch * (s / gq::NB) * ((cs + gq::NB - 1) / gq::NB) <= num_sms();
             {   // T = B U_c, stored transposed in TT at (r0+s+j, r0+i)
                 gq::GemmArgs p = gemm_args((int)s, (int)cs, (int)cs);
                 p.a_row0 = (int)r0;
@@ -633,7 +635,10 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
                 EpiMats o;
                 o.t_hi = Mat{w.TT_hi, N, N, N};
                 o.t_lo = Mat{w.TT_lo, N, N, N};
-                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rsh, rsl, uth, utl, o, p, (int)batch, st, "inv_bu")));
+                if (narrow)
+                    GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rsh, rsl, uth, utl, o, p, (int)batch, st, "inv_bu")));
+                else
+                    GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rsh, rsl, uth, utl, o, p, (int)batch, st, "inv_bu")));
             }
             {   // U_b = -U_a T -> U (public, clipped), U split, UT split
                 gq::GemmArgs p = gemm_args((int)s, (int)cs, (int)s);
@@ -661,7 +666,10 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
                 o.s_lo = Mat{w.U_lo, N, N, N};
                 o.t_hi = Mat{w.UT_hi, N, N, N};
                 o.t_lo = Mat{w.UT_lo, N, N, N};
-                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(uh, ul, tth, ttl, o, p, (int)batch, st, "inv_ub")));
+                if (narrow)
+                    GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(uh, ul, tth, ttl, o, p, (int)batch, st, "inv_ub")));
+                else
+                    GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(uh, ul, tth, ttl, o, p, (int)batch, st, "inv_ub")));
             }
         }
     }

@@ -468,6 +468,9 @@ cudaError_t quant_run_bits(float* W, const float* U, long long d_out, long long 
         p.write_c = 1;
         EpiMats o;
         o.c = Mat{W, (uint64_t)d_out, (uint64_t)d_in, (uint64_t)d_in};
+        // few 128-wide tiles: 128x32 tiles spread the work over more SMs, within one wave
+        if (4 * ((d_out + gq::BM - 1) / gq::BM) * ((ncols + gq::CB - 1) / gq::CB) <= num_sms())
+            return launch_gemm<gq::KIND_TF32X3, 4, 32, 0>(eh, el, uh, ul, o, p, 1, st, name);
         return launch_gemm<gq::KIND_TF32X3, 2>(eh, el, uh, ul, o, p, 1, st, name);
     };
     for (int b = 0; b < nblk; ++b) {

@@ -1,0 +1,43 @@
+"""The multi-rank (N > 1) host path of bench.py on CPU: two gloo ranks on 127.0.0.1.
+
+Each rank quantizes its own layer (weak scaling, no collective on the data path); the
+only collectives are the barrier and the max-over-ranks reduction of the timed region,
+and the reported value is the units all ranks processed over that time.  The ranks run
+in their own interpreters (torch.distributed.run), not inside the test process.
+"""
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_two_gloo_ranks_take_the_slowest_time_and_count_all_units():
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2", "--standalone",
+           "--local-addr", "127.0.0.1", os.path.join(ROOT, "tests", "multirank_worker.py")]
+    env = dict(os.environ, MASTER_ADDR="127.0.0.1", OMP_NUM_THREADS="1")
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=180, cwd=ROOT, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    res = {}
+    for line in r.stdout.splitlines():
+        if line.startswith("{"):
+            d = json.loads(line)
+            res[d["rank"]] = d
+    assert set(res) == {0, 1}
+    for d in res.values():
+        assert d["world"] == 2
+        assert d["job_ms"] == pytest.approx(15.0)                          # max over ranks, on every rank
+        assert d["value"] == pytest.approx(2 * 4096 * 4096 * 3 / 15e-3)    # all ranks' units / job time
+    assert res[0]["seed"] != res[1]["seed"]                                # independent layers per rank
+
+
+def test_single_process_path_needs_no_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert bench.max_over_ranks(7.5, None, None) == 7.5
+    assert bench.job_throughput(1, 100.0, 4, 2.0) == pytest.approx(100.0 * 4 / 2e-3)
