@@ -11,6 +11,8 @@
 //     leaf(j):   R_jj = UL-Cholesky(A_jj), X_jj = R_jj^-1           (one CTA, fp32)
 //     panel(j):  R_{0:j, j} = A_{0:j, j} X_jj^T                      (3xTF32 tcgen05)
 //     update(j): A_{0:j, 0:j} -= R_{0:j, j} R_{0:j, j}^T             (3xTF32 tcgen05)
+//   with the update split three ways: block column j-1 on the critical chain, then block
+//   column j-2 and the rest on a helper stream (look-ahead of depth two).
 //   then U = R^-1 by doubling: for s = 128, 256, ...: for each diagonal pair
 //     [[R_a, B], [0, R_c]] with known inverses U_a, U_c:  U_b = -U_a (B U_c).
 #pragma once

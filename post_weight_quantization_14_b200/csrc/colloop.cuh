@@ -7,9 +7,12 @@
 // columns by a rolled loop: register slot 0 always holds the lane's column of the
 // current oct and the slots shift down by one after each oct, so the loop body stays
 // small (a fully unrolled 128-step loop thrashed the instruction cache).  Four phases
-// of four octs carry 16, 12, 8 and 4 live slots.  For column c:
-//   owner lane (c % 8):  r = clamp(rint(w_c / s), -z, maxq - z);  d_c = w_c - s * r
-//   all eight lanes:     w_j -= d_c * U[c, j] / U[c, c]   for the block columns j > c
+// of four octs carry 16, 12, 8 and 4 live slots.  Per oct, the row's 8 lanes gather the
+// oct's 8 current values, and every lane then runs the oct's 8 rounding steps itself (the
+// same operations in the same order, so all lanes agree exactly): for column c,
+//   r = clamp(rint(w_c / s), -z, maxq - z);  d_c = w_c - s * r;
+//   w_j -= d_c * U[c, j] / U[c, c]   for the later columns j of the oct;
+// after the oct each lane applies the 8 errors d_c to its later slots in column order,
 // which is e_c = d_c / U_cc pushed forward with row c of U.  The normalised rows of
 // the block's 128x128 diagonal part of U are prepared once per layer and staged into
 // shared memory by one bulk (TMA) copy per CTA.

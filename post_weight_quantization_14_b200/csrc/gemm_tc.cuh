@@ -10,7 +10,6 @@
 // KIND_TF32X3 : A = A_hi + A_lo and B = B_hi + B_lo given as two tf32 arrays each;
 //               three MMAs per 8-element K step (hi*hi + hi*lo + lo*hi), which keeps
 //               about fp32 accuracy on the tf32 tensor pipe.
-// KIND_TF32X4 : the same operands with the lo*lo product added (four MMAs per K step).
 //
 // Segmented accumulation (SEG > 0): the tensor pipe's fp32 accumulation error grows with
 // the number of MMAs accumulated in place, so every SEG MMA k-steps the accumulator is
@@ -35,7 +34,7 @@
 
 namespace gq {
 
-enum : int { KIND_BF16 = 0, KIND_TF32X3 = 1, KIND_TF32X4 = 2 };
+enum : int { KIND_BF16 = 0, KIND_TF32X3 = 1 };
 
 struct GemmArgs {
     int M, N, K;
@@ -382,14 +381,10 @@ __global__ void __launch_bounds__(192, 1)
                         umma_tf32(acc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_hi + off), idesc, acc0);
                         umma_tf32(xacc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_lo + off), idesc, x0);
                         umma_tf32(xacc, desc_sw128_kmajor(a_lo + off), desc_sw128_kmajor(b_hi + off), idesc, 1u);
-                        if (KIND == KIND_TF32X4)
-                            umma_tf32(xacc, desc_sw128_kmajor(a_lo + off), desc_sw128_kmajor(b_lo + off), idesc, 1u);
                     } else {
                         umma_tf32(acc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_hi + off), idesc, acc0);
                         umma_tf32(acc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_lo + off), idesc, 1u);
                         umma_tf32(acc, desc_sw128_kmajor(a_lo + off), desc_sw128_kmajor(b_hi + off), idesc, 1u);
-                        if (KIND == KIND_TF32X4)
-                            umma_tf32(acc, desc_sw128_kmajor(a_lo + off), desc_sw128_kmajor(b_lo + off), idesc, 1u);
                     }
                 }
                 umma_commit(&empty_bar[s]);
@@ -549,8 +544,7 @@ __global__ void __launch_bounds__(192, 1)
             } else {
                 // Register path for diagonal tiles of mirrored outputs (C only): write j >= i
                 // and its exact mirror with plain stores.
-                if (lane == 0) bulk_wait_all();   // the staging area is this warp's own box region
-                __syncwarp();
+                __syncwarp();   // the staging area is this warp's own box region
                 float* tile = stage_t;
                 const int rbase = iy;
                 const long long zr = zc_y, zcc = zc_x;
@@ -603,7 +597,6 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
         }
-        if (lane == 0) bulk_wait_all();
         __syncwarp();
     }
     tc_fence_before();
