@@ -167,7 +167,7 @@ CHOL_KERNELS = ("chol_leaf", "chol_panel", "chol_update", "chol_update_next", "c
 QUANT_KERNELS = ("colloop", "trailing_update", "trailing_update_sb", "up_prep", "ut_split", "pack_zeros", "row_params")
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu --set full capture of this
 # workload, for kernels whose launches all do the same work (the kernel's ncu summary under profiles/).
-TRAFFIC_PER_LAUNCH = {"chol_leaf": 142336, "colloop": 2236416, "hessian_syrk": 16900608 + 10929408}
+TRAFFIC_PER_LAUNCH = {"chol_leaf": 142592, "colloop": 2239232, "hessian_syrk": 16879616 + 11550464}
 # Sum of the stage bounds for this layer: Hessian 21.0 us (bf16), factor + invert 168.1 us and
 # trailing updates 244.3 us (3xTF32 at a third of bf16 x 1.1/2.25), column loop 11.6 us (HBM).
 END_TO_END_BOUND_MS = 0.445
