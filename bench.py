@@ -12,6 +12,10 @@ when timing starts; W is restored from a pristine copy and the L2 is flushed (25
 write) before every step, outside the per-step CUDA events.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+       python bench.py --workload stack7b [--steps K] [--warmup W]
+The stack7b workload times one block of the 7B-shaped stack (q, k, v, o 4096 x 4096;
+gate, up 11008 x 4096; down 4096 x 11008; n = 2048 tokens each, 4-bit g128) per step;
+every block has the same shapes, so the 32-block stack time is 32 times that.
 With N > 1 (torchrun, one rank per GPU) every rank quantizes its own independent
 layer (weak scaling, no collective on the data path); the reported time is the max
 over ranks.  Rank 0 prints one JSON line.
@@ -224,6 +228,58 @@ def kernel_rooflines(kernel_ms: dict, launches: dict, hbm: float, bf16: float, p
     return out
 
 
+def run_stack(args) -> None:
+    """One step = the seven layers of block 0 of the 7B-shaped stack, end to end on the device."""
+    import numpy as np
+    import torch
+
+    from post_weight_quantization_14_b200 import gptq as G
+    from post_weight_quantization_14_b200 import inputs as I
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    layers = []
+    for index in range(7):
+        ly = I.make_stack_layer(0, index)
+        cfg = G.make_config(ly.spec.bits, ly.spec.group_size, ly.spec.sym, 128, ly.spec.damp_rel)
+        W0 = torch.from_numpy(ly.W).to(dev)
+        X = torch.from_numpy(ly.X_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+        bufs = G.LayerBuffers(ly.d_out, ly.d_in, ly.n, torch.bfloat16, cfg, dev)
+        layers.append((ly, W0, torch.empty_like(W0), X, bufs))
+    stream = torch.cuda.current_stream()
+
+    def step(marks=None):
+        for i, (ly, W0, W, X, bufs) in enumerate(layers):
+            W.copy_(W0)
+            if marks:
+                marks[i][0].record(stream)
+            G.quantize_layer(W, X, buffers=bufs)
+            if marks:
+                marks[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    G.gptq_sync_status()
+    marks = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in layers]
+             for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for m in marks:
+        step(m)
+    torch.cuda.synchronize()
+    G.gptq_sync_status()
+    per_layer = {ly.name.split(".")[-1]: statistics.median(m[i][0].elapsed_time(m[i][1]) for m in marks)
+                 for i, (ly, *_rest) in enumerate(layers)}
+    block_ms = sum(per_layer.values())
+    weights = sum(ly.d_out * ly.d_in for ly, *_rest in layers)
+    print(json.dumps({"metric": "7B-shaped stack end-to-end quantize time (32 blocks x 7 layers)",
+                      "value": 32 * block_ms / 1e3, "unit": "s", "higher_is_better": False, "n_gpus": 1,
+                      "steps": args.steps, "warmup": args.warmup, "dtype": "f32", "data": "synthetic",
+                      "config": {"workload": "stack7b: one block per step (block 0 seeds), x32 blocks",
+                                 "n": 2048, "bits": 4, "group_size": 128, "sym": False},
+                      "block_ms": block_ms, "layer_ms": per_layer,
+                      "weights_per_s": 32 * weights / (32 * block_ms / 1e3)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -231,7 +287,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="attn", choices=["attn", "stack7b"])
     args = ap.parse_args()
+    if args.workload == "stack7b":
+        run_stack(args)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -472,9 +472,12 @@ cudaError_t quant_run_bits(float* W, const float* U, long long d_out, long long 
         EpiMats o;
         o.c = Mat{W, (uint64_t)d_out, (uint64_t)d_in, (uint64_t)d_in};
         // few 128-wide tiles: 128x32 tiles spread the work over more SMs, within one wave
+        // Segmented accumulation (16 k-steps, cross products apart): the in-place fp32
+        // accumulation of a K = 1024 update drifts by ~1e-5 relative, enough to move
+        // near-tie rounding decisions of later columns.
         if (4 * ((d_out + gq::BM - 1) / gq::BM) * ((ncols + gq::CB - 1) / gq::CB) <= num_sms())
-            return launch_gemm<gq::KIND_TF32X3, 4, 32, 0>(eh, el, uh, ul, o, p, 1, st, name);
-        return launch_gemm<gq::KIND_TF32X3, 2>(eh, el, uh, ul, o, p, 1, st, name);
+            return launch_gemm<gq::KIND_TF32X3, 4, 32, 16>(eh, el, uh, ul, o, p, 1, st, name);
+        return launch_gemm<gq::KIND_TF32X3, 2, 128, 16>(eh, el, uh, ul, o, p, 1, st, name);
     };
     for (int b = 0; b < nblk; ++b) {
         const long long s0 = (long long)(b / SB_BLOCKS) * sbw;      // superblock columns

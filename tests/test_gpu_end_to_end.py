@@ -80,7 +80,7 @@ def _full_check(layer, spec, sample_rows=256, full_H=True, seed=1):
     own = O.gptq(layer.W[rows], Uo, spec.bits, spec.group_size, spec.sym, 128)
     l_gpu = O.row_losses(layer.W[rows], gpu["What"][rows], X).sum()
     l_ref = O.row_losses(layer.W[rows], own.what, X).sum()
-    assert abs(l_gpu - l_ref) <= U_.LOSS_TOL * l_ref
+    assert abs(l_gpu - l_ref) <= U_.LOSS_TOL * l_ref, (layer.name, l_gpu, l_ref, rr.forced_codes)
     return gpu, bufs, Uo, rr
 
 
@@ -113,3 +113,12 @@ def test_ffn_down_4096x11008_2bit_then_per_row_4bit():
     out = U_.unpack_outputs(qw, sc, qz, es, layer.d_out, layer.d_in, 4, -1, False)
     rows = np.sort(np.random.default_rng(7).choice(layer.d_out, 128, replace=False))
     U_.check_quant(layer.W, Uo, out, 4, -1, False, rows=rows)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("block", [0, 31])
+def test_7b_stack_blocks_first_and_last(block):
+    """The 7B-shaped stack: all seven linear layers of blocks 0 and 31 (4-bit asym g128)."""
+    for index in range(7):
+        layer = I.make_stack_layer(block, index)
+        _full_check(layer, layer.spec, sample_rows=512, full_H=layer.d_in <= 4096, seed=block * 7 + index)
