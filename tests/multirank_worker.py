@@ -1,7 +1,8 @@
 """One rank of the two-rank CPU check of bench.py's multi-rank host path (gloo).
 
-Run by tests/test_multirank_cpu.py through torch.distributed.run; prints one JSON line
-per rank with the job time, the job throughput and the rank's layer seed.
+Run by tests/test_multirank_cpu.py through torch.distributed.run; each rank writes one
+JSON file (rank<r>.json in the directory MULTIRANK_OUT) with the job time, the job
+throughput and the rank's layer seed.
 """
 
 import json
@@ -23,8 +24,9 @@ def main() -> None:
         job_ms = bench.max_over_ranks(my_ms, dist, torch.device("cpu"))
         value = bench.job_throughput(world, 4096 * 4096, 3, job_ms)
         dist.barrier()
-        print(json.dumps({"rank": rank, "world": world, "job_ms": job_ms, "value": value,
-                          "seed": bench.layer_seed(rank)}), flush=True)
+        with open(os.path.join(os.environ["MULTIRANK_OUT"], f"rank{rank}.json"), "w") as f:
+            json.dump({"rank": rank, "world": world, "job_ms": job_ms, "value": value,
+                       "seed": bench.layer_seed(rank)}, f)
     finally:
         dist.destroy_process_group()
 

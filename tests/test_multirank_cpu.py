@@ -16,17 +16,16 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def test_two_gloo_ranks_take_the_slowest_time_and_count_all_units():
+def test_two_gloo_ranks_take_the_slowest_time_and_count_all_units(tmp_path):
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2", "--standalone",
            "--local-addr", "127.0.0.1", os.path.join(ROOT, "tests", "multirank_worker.py")]
-    env = dict(os.environ, MASTER_ADDR="127.0.0.1", OMP_NUM_THREADS="1")
+    env = dict(os.environ, MASTER_ADDR="127.0.0.1", OMP_NUM_THREADS="1", MULTIRANK_OUT=str(tmp_path))
     r = subprocess.run(cmd, capture_output=True, text=True, timeout=180, cwd=ROOT, env=env)
     assert r.returncode == 0, r.stderr[-2000:]
     res = {}
-    for line in r.stdout.splitlines():
-        if line.startswith("{"):
-            d = json.loads(line)
-            res[d["rank"]] = d
+    for rank in range(2):
+        d = json.loads((tmp_path / f"rank{rank}.json").read_text())
+        res[d["rank"]] = d
     assert set(res) == {0, 1}
     for d in res.values():
         assert d["world"] == 2
