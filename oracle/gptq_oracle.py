@@ -18,6 +18,8 @@ What it follows (page titles as printed on the pages; section names in quotes):
     updates of the not-yet-quantized columns.
   - "阶段三：量化与反量化": group-wise scale (and zero) found during the pass;
     dequantization multiplies the integer by its scale.
+  - "激活排序（desc_act）": the columns may be visited in an order ranked by
+    the sum of absolute input activations instead of their natural order.
 * "GPTQ-2D: 三次时间复杂度的双侧自适应舍入" (ai-feeds summary), "问题背景" and
   "核心洞察": one-sided GPTQ equals Babai's nearest-plane algorithm.
 * "GPTQ/AWQ量化中Group Size的精确含义与计算" (feinterview group-size article),
@@ -48,6 +50,12 @@ Readings of points the pages leave open (each is implemented below):
   rounds to 0 in fp16 is raised to the smallest positive fp16 value 2^-24.
 * Rounding of codes: round half to even (IEEE rint), then clamp to [0, maxq].
 * Zero stored in b bits.
+* Activation ordering ("激活排序（desc_act）" on the tutorial page): the page
+  ranks columns by the sum of absolute input activations and quantizes the
+  least influential first, while the flag's name suggests descending order.
+  desc_act = 1 follows the text (ascending), desc_act = 2 the name
+  (descending); ties keep column order.  Groups are formed in quantization
+  order, and a per-column group index maps each column to its group.
 """
 
 from __future__ import annotations
@@ -341,17 +349,25 @@ def rtn(W0: np.ndarray, bits: int = 4, group_size: int = 128, sym: bool = False)
     return GPTQResult(codes, scales, zeros, np.zeros_like(what), W.copy(), what)
 
 
-def gptq_naive_obs(W0: np.ndarray, Hd: np.ndarray, bits=4, group_size=128, sym=False) -> GPTQResult:
+def gptq_naive_obs(W0: np.ndarray, Hd: np.ndarray, bits=4, group_size=128, sym=False,
+                   order: np.ndarray | None = None) -> GPTQResult:
     """Literal OBS form for tiny inputs: after each column, re-invert the remaining Hessian.
 
-    For column c the inverse of Hd[c:, c:] is formed explicitly; the error of
-    column c, divided by that inverse's (0, 0) entry, is pushed along its first
-    row (tutorial page, "阶段一" and the pseudocode's per-column downdate).
-    Uses no Cholesky factor, so it checks the U form independently.
+    For column c the inverse of Hd restricted to the not-yet-quantized columns
+    is formed explicitly; the error of column c, divided by that inverse's
+    diagonal entry for c, is pushed along its row (tutorial page, "阶段一" and
+    the pseudocode's per-column downdate).  Uses no Cholesky factor, so it
+    checks the U form independently.
+
+    ``order`` (a permutation of the columns) visits the columns in that order
+    and works in the original coordinates throughout: no permuted copy of W or
+    Hd is made, group k takes the columns order[k*g:(k+1)*g], and codes land in
+    their own columns.  It checks the permute/unpermute of the act-order form.
     """
     W = np.array(W0, dtype=np.float64, copy=True)
     Hd = np.asarray(Hd, dtype=np.float64)
     d_out, d_in = W.shape
+    order = np.arange(d_in) if order is None else np.asarray(order)
     maxq = (1 << bits) - 1
     g = _group_len(group_size, d_in)
     ng = n_groups(d_in, group_size)
@@ -359,16 +375,18 @@ def gptq_naive_obs(W0: np.ndarray, Hd: np.ndarray, bits=4, group_size=128, sym=F
     scales = np.zeros((ng, d_out))
     zeros = np.zeros((ng, d_out), dtype=np.int64)
     what = np.zeros((d_out, d_in))
-    for c in range(d_in):
-        if c % g == 0:
-            s, z, _, _, _ = group_params(W[:, c:min(c + g, d_in)], bits, sym)
-            scales[c // g], zeros[c // g] = s, z
-        Hinv_rem = np.linalg.inv(Hd[c:, c:])
+    for k in range(d_in):
+        c = order[k]
+        rest = order[k:]                 # c first, then the columns still to come
+        if k % g == 0:
+            s, z, _, _, _ = group_params(W[:, order[k:min(k + g, d_in)]], bits, sym)
+            scales[k // g], zeros[k // g] = s, z
+        Hinv_rem = np.linalg.inv(Hd[np.ix_(rest, rest)])
         w = W[:, c].copy()
         q = quantize(w, s, z, maxq)
         wh = dequantize(q, s, z)
         codes[:, c], what[:, c] = q.astype(np.int64), wh
-        W[:, c + 1:] -= np.outer((w - wh) / Hinv_rem[0, 0], Hinv_rem[0, 1:])
+        W[:, rest[1:]] -= np.outer((w - wh) / Hinv_rem[0, 0], Hinv_rem[0, 1:])
     return GPTQResult(codes, scales, zeros, np.zeros_like(what), np.zeros_like(what), what)
 
 
@@ -459,11 +477,14 @@ def pack_qzeros(zeros: np.ndarray, bits: int) -> np.ndarray:
     return np.ascontiguousarray(pack_bitstream(zeros, bits)).view(np.int32)
 
 
-def dequant_packed(qweight, scales, qzeros, d_out, d_in, bits, group_size, sym) -> np.ndarray:
-    """W_hat[o, c] = scale[g(c), o] * (q[o, c] - zero[g(c), o]) from the packed arrays."""
+def dequant_packed(qweight, scales, qzeros, d_out, d_in, bits, group_size, sym, g_idx=None) -> np.ndarray:
+    """W_hat[o, c] = scale[g(c), o] * (q[o, c] - zero[g(c), o]) from the packed arrays.
+
+    g(c) = c // group_size, or g_idx[c] when a per-column group index is given
+    (activation ordering)."""
     codes = unpack_bitstream(np.asarray(qweight).view(np.uint32).T, bits, d_in)
     g = _group_len(group_size, d_in)
-    gi = np.arange(d_in) // g
+    gi = np.arange(d_in) // g if g_idx is None else np.asarray(g_idx, dtype=np.int64)
     s = np.asarray(scales, dtype=np.float64)[gi, :].T
     if sym:
         z = float(1 << (bits - 1))
@@ -493,3 +514,77 @@ def quantize_layer(W0, X, bits=4, group_size=128, sym=False, block_size=128, dam
     U = hinv_upper_cholesky(Hd)
     res = gptq(W0, U, bits, group_size, sym, block_size)
     return res, H, U, lam
+
+
+# ----------------------------------------------------------------------------
+# Activation ordering (desc_act)
+# ----------------------------------------------------------------------------
+
+ACT_ASCENDING = 1    # the tutorial's procedure: least output impact first
+ACT_DESCENDING = 2   # the order the flag's name suggests
+
+
+def act_abs_sum(X: np.ndarray) -> np.ndarray:
+    """a_c = sum_t |X[t, c]| in fp64 (tutorial page, "激活排序（desc_act）": columns
+    are ranked by the sum of the absolute values of their input activations)."""
+    return np.sum(np.abs(np.asarray(X, dtype=np.float64)), axis=0)
+
+
+def act_order(a: np.ndarray, desc_act: int) -> np.ndarray:
+    """Quantization order perm: perm[k] is the column quantized at position k.
+
+    desc_act = 1 sorts a ascending: the columns whose activations move the output
+    least are quantized first and the sensitive ones, quantized last, absorb the
+    compensation (the tutorial's "激活排序（desc_act）" text).  desc_act = 2 sorts
+    descending.  Equal values keep increasing column index in both directions.
+    """
+    a = np.asarray(a, dtype=np.float64)
+    if desc_act == ACT_ASCENDING:
+        return np.argsort(a, kind="stable")
+    if desc_act == ACT_DESCENDING:
+        return np.argsort(-a, kind="stable")
+    raise ValueError("desc_act must be 1 (ascending) or 2 (descending)")
+
+
+def g_idx_of(perm: np.ndarray, group_size: int) -> np.ndarray:
+    """Per-column group index: column perm[k] belongs to group k // g."""
+    perm = np.asarray(perm)
+    g = _group_len(group_size, perm.size)
+    gi = np.empty(perm.size, dtype=np.int64)
+    gi[perm] = np.arange(perm.size) // g
+    return gi
+
+
+@dataclass
+class ActOrderResult:
+    codes: np.ndarray        # int64 [d_out, d_in], original column order
+    scales: np.ndarray       # fp64 [n_groups, d_out], groups in quantization order
+    zeros: np.ndarray        # int64 [n_groups, d_out]
+    g_idx: np.ndarray        # int64 [d_in]
+    what: np.ndarray         # fp64 [d_out, d_in], original column order
+    perm: np.ndarray         # quantization order
+    U: np.ndarray            # upper Cholesky factor of the permuted (P^T Hd P)^-1
+    lam: float
+    inner: GPTQResult        # the column loop's own result, in quantization order
+
+
+def gptq_act_order(W0: np.ndarray, H: np.ndarray, perm: np.ndarray, bits=4, group_size=128, sym=False,
+                   block_size=128, damp_rel=0.01) -> ActOrderResult:
+    """GPTQ with the columns visited in the order perm.
+
+    The column loop is the unchanged fixed-order one applied to the permuted
+    problem: Hp[i, j] = H[perm[i], perm[j]], Wp = W0[:, perm]; damping and U are
+    taken from Hp (lambda is unchanged: the diagonal is only reordered).  Codes
+    and dequantized weights are put back in the original columns; groups stay in
+    quantization order and g_idx maps each column to its group.
+    """
+    perm = np.asarray(perm)
+    Hp = np.asarray(H, dtype=np.float64)[np.ix_(perm, perm)]
+    Hd, lam = damp(Hp, damp_rel)
+    U = hinv_upper_cholesky(Hd)
+    res = gptq(np.asarray(W0, dtype=np.float64)[:, perm], U, bits, group_size, sym, block_size)
+    codes = np.empty_like(res.codes)
+    codes[:, perm] = res.codes
+    what = np.empty_like(res.what)
+    what[:, perm] = res.what
+    return ActOrderResult(codes, res.scales, res.zeros, g_idx_of(perm, group_size), what, perm, U, lam, res)

@@ -387,3 +387,84 @@ def test_boundary_distance_closed_form():
     assert O.boundary_distance(np.array([0.1 * (1.5 - 3) + 0.004]), s, z, 15)[0] == pytest.approx(0.004, rel=1e-9)
     # clamped low: x = -2 -> only boundary 0.5 matters -> 2.5 grid units
     assert O.boundary_distance(np.array([0.1 * (-2 - 3)]), s, z, 15)[0] == pytest.approx(0.25, rel=1e-9)
+
+
+# ---------------------------------------------------------------- activation ordering
+
+def test_act_abs_sum_closed_form():
+    # X[t, c] = (-1)^t (t + 1) (c + 1): sum_t |X[t, c]| = (c + 1) n (n + 1) / 2, exactly
+    n, d = 37, 9
+    t = np.arange(n)[:, None]
+    c = np.arange(d)[None, :]
+    X = np.where(t % 2 == 0, 1.0, -1.0) * (t + 1) * (c + 1)
+    np.testing.assert_array_equal(O.act_abs_sum(X), (np.arange(d) + 1) * n * (n + 1) / 2)
+
+
+def test_act_order_directions_and_ties():
+    a = np.array([3.0, 1.0, 2.0, 1.0, 5.0, 0.0])
+    np.testing.assert_array_equal(O.act_order(a, O.ACT_ASCENDING), [5, 1, 3, 2, 0, 4])
+    np.testing.assert_array_equal(O.act_order(a, O.ACT_DESCENDING), [4, 0, 2, 1, 3, 5])
+    # group index of column perm[k] is k // g
+    np.testing.assert_array_equal(O.g_idx_of(np.array([5, 1, 3, 2, 0, 4]), 2), [2, 0, 1, 1, 2, 0])
+    np.testing.assert_array_equal(O.g_idx_of(np.array([2, 0, 1]), -1), [0, 0, 0])
+
+
+@pytest.mark.parametrize("seed,desc", [(60, 1), (61, 2), (62, 1), (63, 2)])
+@pytest.mark.parametrize("g", [4, -1])
+def test_act_order_equals_literal_obs_in_that_order(seed, desc, g):
+    # an independent algorithm: OBS on the original coordinates, visiting columns in
+    # the order, re-inverting the remaining Hessian each step (no permuted copies)
+    X, W, H, Hd, U = _rand_problem(seed, 5, 12, 30, hot=2)
+    perm = O.act_order(O.act_abs_sum(X), desc)
+    a = O.gptq_act_order(W, H, perm, 3, g, False, block_size=0)
+    b = O.gptq_naive_obs(W, Hd, 3, g, False, order=perm)
+    np.testing.assert_array_equal(a.codes, b.codes)
+    np.testing.assert_allclose(a.scales, b.scales, rtol=0, atol=0)
+    np.testing.assert_array_equal(a.zeros, b.zeros)
+    np.testing.assert_allclose(a.what, b.what, rtol=0, atol=1e-15)
+
+
+def test_act_order_identity_order_is_plain_gptq():
+    # columns whose activation sums already increase: the ascending order is the identity
+    rng = np.random.default_rng(70)
+    d_in, n = 64, 96
+    X = rng.standard_normal((n, d_in))
+    X *= (1.0 + 0.1 * np.arange(d_in))[None, :] / np.sum(np.abs(X), axis=0)[None, :]
+    a = O.act_abs_sum(X)
+    assert np.all(np.diff(a) > 0)
+    perm = O.act_order(a, O.ACT_ASCENDING)
+    np.testing.assert_array_equal(perm, np.arange(d_in))
+    W = rng.standard_normal((8, d_in)) * 0.02
+    ao = O.gptq_act_order(W, O.hessian(X), perm, 4, 16, False)
+    plain, _, _, lam = O.quantize_layer(W, X, 4, 16, False)
+    np.testing.assert_array_equal(ao.codes, plain.codes)
+    np.testing.assert_array_equal(ao.g_idx, np.arange(d_in) // 16)
+    assert ao.lam == lam
+
+
+@pytest.mark.parametrize("seed", [71, 72])
+def test_act_order_equivariant_under_column_relabelling(seed):
+    # relabelling the input channels of W and X relabels the codes and g_idx the same way
+    rng = np.random.default_rng(seed)
+    X, W, H, _, _ = _rand_problem(seed, 6, 32, 64, hot=3)
+    Q = rng.permutation(32)
+    r1 = O.gptq_act_order(W, H, O.act_order(O.act_abs_sum(X), 1), 4, 8, False)
+    XQ, WQ = X[:, Q], W[:, Q]
+    r2 = O.gptq_act_order(WQ, O.hessian(XQ), O.act_order(O.act_abs_sum(XQ), 1), 4, 8, False)
+    np.testing.assert_array_equal(r2.codes, r1.codes[:, Q])
+    np.testing.assert_array_equal(r2.g_idx, r1.g_idx[Q])
+    np.testing.assert_array_equal(r2.scales, r1.scales)
+
+
+def test_act_order_error_identity_and_packed_roundtrip():
+    # sum_c e_c^2 of the permuted loop equals (W0 - W_hat) Hd (W0 - W_hat)^T in the
+    # original coordinates; packing + g_idx dequantization reproduces W_hat
+    X, W, H, Hd, _ = _rand_problem(73, 7, 48, 80, hot=2)
+    perm = O.act_order(O.act_abs_sum(X), 1)
+    r = O.gptq_act_order(W, H, perm, 4, 16, False, block_size=16)
+    D = W - r.what
+    np.testing.assert_allclose(np.sum(r.inner.err ** 2, axis=1), np.einsum("oi,ij,oj->o", D, Hd, D), rtol=1e-9)
+    qw = O.pack_qweight(r.codes, 4)
+    qz = O.pack_qzeros(r.zeros, 4)
+    Wh = O.dequant_packed(qw, r.scales, qz, 7, 48, 4, 16, False, g_idx=r.g_idx)
+    np.testing.assert_array_equal(Wh, r.what)
