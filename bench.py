@@ -167,8 +167,10 @@ def run_reference(args, rank: int, world: int) -> None:
 
 CHOL_KERNELS = ("chol_leaf", "chol_panel", "chol_update", "chol_update_next", "chol_update_u2", "inv_bu", "inv_ub",
                 "split_panel",
-                "damp_copy", "diag_mean", "zero_lower", "chol_diag_out")
-QUANT_KERNELS = ("colloop", "trailing_update", "trailing_update_sb", "up_prep", "ut_split", "pack_zeros", "row_params")
+                "damp_copy", "diag_mean", "zero_lower", "chol_diag_out", "perm_invert", "damp_copy_perm")
+QUANT_KERNELS = ("colloop", "trailing_update", "trailing_update_sb", "up_prep", "ut_split", "pack_zeros", "row_params",
+                 "gather_cols", "unpermute_codes")
+ACT_KERNELS = ("act_sum", "act_rank", "act_perm")   # activation ordering (--desc-act 1 or 2)
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu --set full capture of this
 # workload, for kernels whose launches all do the same work (the kernel's ncu summary under profiles/).
 TRAFFIC_PER_LAUNCH = {"chol_leaf": 142592, "colloop": 2239232, "hessian_syrk": 16879616 + 11550464}
@@ -288,6 +290,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="attn", choices=["attn", "stack7b"])
+    ap.add_argument("--desc-act", type=int, default=0, choices=[0, 1, 2],
+                    help="activation ordering: 0 natural column order, 1 ascending, 2 descending sum of |x|")
     args = ap.parse_args()
     if args.workload == "stack7b":
         run_stack(args)
@@ -316,7 +320,7 @@ def main():
     from post_weight_quantization_14_b200 import inputs as I
 
     layer = I.make_layer("attn", seed=layer_seed(rank))
-    cfg = G.make_config(BITS, GROUP, SYM, 128, 0.01)
+    cfg = G.make_config(BITS, GROUP, SYM, 128, 0.01, args.desc_act)
     W0 = torch.from_numpy(layer.W).to(dev)
     W = torch.empty_like(W0)
     X = torch.from_numpy(layer.X_bits.view(np.int16)).to(dev).view(torch.bfloat16)
@@ -327,12 +331,23 @@ def main():
     def step(marks=None):
         # the three stages of G.quantize_layer, with optional events between them
         G.gptq_hessian_accumulate(X, bufs.H, accumulate=False, workspace=bufs.ws)
+        if cfg.desc_act:
+            G.gptq_act_sum_accumulate(X, bufs.act)
+            G.gptq_act_order(bufs.act, cfg.desc_act, bufs.perm, bufs.rank)
         if marks:
             marks[0].record(stream)
-        G.gptq_prepare_hinv(bufs.H, bufs.U, cfg.damp_rel, workspace=bufs.ws)
+        if cfg.desc_act:
+            G.gptq_prepare_hinv_permuted(bufs.H, bufs.perm, bufs.U, cfg.damp_rel, workspace=bufs.ws)
+        else:
+            G.gptq_prepare_hinv(bufs.H, bufs.U, cfg.damp_rel, workspace=bufs.ws)
         if marks:
             marks[1].record(stream)
-        G.gptq_quantize_layer(W, bufs.U, cfg, bufs.qweight, bufs.scales, bufs.qzeros, bufs.err_sq, workspace=bufs.ws)
+        if cfg.desc_act:
+            G.gptq_quantize_layer_act_order(W, bufs.U, bufs.perm, cfg, bufs.qweight, bufs.scales, bufs.qzeros,
+                                            bufs.g_idx, bufs.err_sq, workspace=bufs.ws)
+        else:
+            G.gptq_quantize_layer(W, bufs.U, cfg, bufs.qweight, bufs.scales, bufs.qzeros, bufs.err_sq,
+                                  workspace=bufs.ws)
 
     for _ in range(args.warmup):
         W.copy_(W0)
@@ -383,7 +398,8 @@ def main():
 
     hbm, bf16, bf16_sus, peak_kind = peaks()
     roof_all = kernel_rooflines(kernel_ms, kernel_launches, hbm, bf16, peak_kind)
-    stage_ms = {"hessian": kernel_ms.get("hessian_syrk", 0) + kernel_ms.get("transpose_x", 0),
+    stage_ms = {"hessian": kernel_ms.get("hessian_syrk", 0) + kernel_ms.get("transpose_x", 0)
+                + sum(kernel_ms.get(k, 0) for k in ACT_KERNELS),
                 "prepare_hinv": sum(v for k, v in kernel_ms.items() if k in CHOL_KERNELS),
                 "quantize": sum(kernel_ms.get(k, 0) for k in QUANT_KERNELS)}
     dom = max((k for k in roof_all), key=lambda k: kernel_ms.get(k, 0) + (kernel_ms.get("trailing_update_sb", 0)
@@ -399,6 +415,7 @@ def main():
     sc_host = torch.empty(bufs.scales.shape, dtype=torch.float16).pin_memory()
     qz_host = torch.empty(bufs.qzeros.shape, dtype=torch.int32).pin_memory()
     Xd = torch.empty(X_host.shape, dtype=torch.int16, device=dev)
+    gi_host = torch.empty((D_IN,), dtype=torch.int32).pin_memory()
     e2e_steps = max(3, min(args.steps, 30))
     if dist:
         dist.barrier()
@@ -410,6 +427,8 @@ def main():
         Xd.copy_(X_host, non_blocking=True)
         q = G.quantize_layer(W, Xd.view(torch.bfloat16), buffers=bufs)
         qw_host.copy_(q.qweight, non_blocking=True)
+        if cfg.desc_act:
+            gi_host.copy_(q.g_idx, non_blocking=True)
         sc_host.copy_(q.scales, non_blocking=True)
         qz_host.copy_(q.qzeros, non_blocking=True)
     eb.record(stream)
@@ -417,7 +436,7 @@ def main():
     e2e_ms = max_over_ranks(ea.elapsed_time(eb), dist, dev)
     e2e_value = job_throughput(world, D_OUT * D_IN, e2e_steps, e2e_ms)
     h2d = W_host.numel() * 4 + X_host.numel() * 2
-    d2h = qw_host.numel() * 4 + sc_host.numel() * 2 + qz_host.numel() * 4
+    d2h = qw_host.numel() * 4 + sc_host.numel() * 2 + qz_host.numel() * 4 + (D_IN * 4 if cfg.desc_act else 0)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -429,7 +448,7 @@ def main():
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": {"workload": WORKLOAD, "d_out": D_OUT, "d_in": D_IN, "n": N_TOK, "bits": BITS,
-                           "group_size": GROUP, "sym": SYM, "damp_rel": 0.01,
+                           "group_size": GROUP, "sym": SYM, "damp_rel": 0.01, "desc_act": args.desc_act,
                            "l2": "flushed (256 MB write) before every step, outside the step events",
                            "parallelism": f"{world} independent layers, one per GPU"},
                 "roofline": roofline,

@@ -12,12 +12,19 @@
  *                                writes packed codes, fp16 scales and packed zero points.
  *   4. gptq_pack_int / gptq_dequant   packing of b-bit codes; W_hat = s * (q - z).
  *
+ * Activation ordering (desc_act) visits the columns in another order:
+ * gptq_act_sum_accumulate (beside stage 1) and gptq_act_order rank the columns,
+ * gptq_prepare_hinv_permuted replaces stage 2, gptq_quantize_layer_act_order stage 3,
+ * and gptq_dequant_g_idx reads the per-column group index the latter writes.
+ *
  * Sources (page titles as printed; sections in quotes):
  *   - "GPTQ：基于近似二阶信息的大模型权重量化" (freeguideonline GPTQ tutorial):
  *     "对称与仿射量化" (q = round(x/s) + z, group-wise scale/zero),
  *     "阶段一：构建 Hessian 逆近似" (H = 2 X^T X + lambda I, upper Cholesky factor),
  *     "阶段二：贪婪顺序量化与懒惰批更新" (fixed column order, lazy batch updates),
  *     "阶段三：量化与反量化" (per-group scale found during the pass, INT x scale).
+ *     "激活排序（desc_act）" (columns ranked by the sum of absolute input activations,
+ *     the least influential quantized first).
  *   - "GPTQ/AWQ量化中Group Size的精确含义与计算" (feinterview group-size article):
  *     codes 0..2^b-1, scale and zero per group along the input dimension,
  *     group_size = -1 is one group per row, "存储代价" (16-bit scale, b-bit zero,
@@ -49,7 +56,7 @@ extern "C" {
 typedef enum {
     GPTQ_OK = 0,
     GPTQ_ERR_INVALID_ARG = 1,   /* bad pointer, size, layout or config value            */
-    GPTQ_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement (desc_act) */
+    GPTQ_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement           */
     GPTQ_ERR_NOT_PD = 3,        /* damped Hessian not positive definite (bad_col set)    */
     GPTQ_ERR_NONFINITE = 4,     /* NaN or Inf found in an input                          */
     GPTQ_ERR_CUDA = 5,          /* a CUDA runtime or driver call failed                  */
@@ -66,7 +73,11 @@ typedef enum { GPTQ_BF16 = 0, GPTQ_F32 = 1 } gptq_dtype;
  *   sym         0 = asymmetric (zero point stored), 1 = symmetric (implicit zero 2^(bits-1)).
  *   block_size  lazy-batch width; 128 is the only value this build accepts.
  *   damp_rel    lambda = damp_rel * mean(diag H); must be >= 0 and finite.
- *   desc_act    activation ordering; must be 0 (GPTQ_ERR_UNSUPPORTED otherwise). */
+ *   desc_act    0 = natural column order (gptq_quantize_layer); 1 = activation ordering,
+ *               ascending sum of |x| (the tutorial's text: least influential columns first);
+ *               2 = descending (the reading the flag's name suggests).  1 and 2 are run by
+ *               gptq_quantize_layer_act_order, which rejects 0; gptq_quantize_layer rejects
+ *               1 and 2.  Any other value is GPTQ_ERR_INVALID_ARG. */
 typedef struct {
     int bits;
     int group_size;
@@ -156,6 +167,59 @@ gptq_status gptq_pack_int(const uint8_t* codes, int64_t rows, int64_t cols, int 
 gptq_status gptq_dequant(const int32_t* qweight, const uint16_t* scales, const int32_t* qzeros,
                          int64_t d_out, int64_t d_in, const gptq_config* cfg, float* W_hat,
                          void* stream);
+
+/* ------------------------------------------------------------------ activation ordering
+ * (tutorial "激活排序（desc_act）": columns ranked by the sum of absolute input
+ * activations; groups are formed in that order and a per-column group index maps each
+ * column back to its group).
+ *
+ * gptq_act_sum_accumulate: act[c] (+)= sum_t |X[t, c]|, accumulated in fp64 in a fixed
+ * order (the same bits on every run).  X as in gptq_hessian_accumulate (16-byte aligned,
+ * d_in % 8 == 0); act device fp64 [d_in], 8-byte aligned; accumulate 0 overwrites.  A
+ * non-finite sum is reported by the next gptq_sync_status() (GPTQ_ERR_NONFINITE). */
+gptq_status gptq_act_sum_accumulate(const void* X, gptq_dtype xt, int64_t n, int64_t d_in, double* act,
+                                    int accumulate, void* stream);
+
+/* gptq_act_order: the quantization order of the columns.
+ *   perm  device int32 [d_in]: perm[k] = the column quantized at position k.
+ *   rank  device int32 [d_in]: its inverse, rank[perm[k]] = k.
+ *   desc_act 1: act ascending; 2: act descending.  Equal values (+0 and -0 are equal) keep
+ *   increasing column index in both directions; NaN sorts by its bit pattern.
+ * Always writes a valid permutation.  1 <= d_in <= 65536. */
+gptq_status gptq_act_order(const double* act, int64_t d_in, int desc_act, int32_t* perm, int32_t* rank,
+                           void* stream);
+
+/* gptq_prepare_hinv_permuted: gptq_prepare_hinv of the permuted Hessian
+ * Hp[i][j] = H[perm[i]][perm[j]], i.e. U with U^T U = (Hp + lambda I)^-1.  lambda is that of
+ * H (the diagonal is only reordered).  H must hold both triangles (gptq_hessian_accumulate
+ * writes both); perm is a device int32 permutation of 0..d_in-1.  bad_col is a position
+ * in quantization order.  An entry of perm outside [0, d_in) or a repeated entry returns
+ * GPTQ_ERR_INVALID_ARG (index = its position) and U is then undefined.  Workspace as
+ * gptq_prepare_hinv_workspace_bytes(d_in). */
+gptq_status gptq_prepare_hinv_permuted(const float* H, const int32_t* perm, int64_t d_in, float damp_rel, float* U,
+                                       void* ws, size_t ws_bytes, int64_t* bad_col, float* lambda_out, void* stream);
+
+/* gptq_quantize_layer_act_order: the column loop of gptq_quantize_layer on the columns in
+ * the order perm; cfg->desc_act must be 1 or 2 (the order itself is the one in perm).
+ *   W        device fp32 [d_out, d_in] in the original column order; read only.
+ *   U        output of gptq_prepare_hinv_permuted with the same perm.
+ *   qweight  as gptq_quantize_layer, codes in the ORIGINAL column order.
+ *   scales, qzeros  as gptq_quantize_layer; group k holds the columns perm[k*g .. k*g+g-1].
+ *   g_idx    device int32 [d_in]: g_idx[c] = rank of c / g (0 for group_size -1).
+ *   err_sq   as gptq_quantize_layer (the row's quadratic form does not depend on the order).
+ *   ws       at least gptq_quantize_workspace_bytes(d_out, d_in, cfg) bytes with cfg->desc_act
+ *            set (the plain loop's workspace plus a permuted copy of W and of the codes).
+ * An invalid perm is reported by the next gptq_sync_status() (GPTQ_ERR_INVALID_ARG). */
+gptq_status gptq_quantize_layer_act_order(const float* W, const float* U, const int32_t* perm, int64_t d_out,
+                                          int64_t d_in, const gptq_config* cfg, int32_t* qweight, uint16_t* scales,
+                                          int32_t* qzeros, int32_t* g_idx, float* err_sq, void* ws, size_t ws_bytes,
+                                          void* stream);
+
+/* W_hat[o, c] = scale[g_idx[c], o] * (q[o, c] - zero[g_idx[c], o]); arrays as gptq_dequant.
+ * A g_idx entry outside [0, n_groups) is reported by the next gptq_sync_status(). */
+gptq_status gptq_dequant_g_idx(const int32_t* qweight, const uint16_t* scales, const int32_t* qzeros,
+                               const int32_t* g_idx, int64_t d_out, int64_t d_in, const gptq_config* cfg,
+                               float* W_hat, void* stream);
 
 /* Synchronise ``stream`` and return (and clear) the device status word. */
 gptq_status gptq_sync_status(void* stream);

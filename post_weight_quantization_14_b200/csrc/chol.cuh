@@ -17,6 +17,7 @@
 //     [[R_a, B], [0, R_c]] with known inverses U_a, U_c:  U_b = -U_a (B U_c).
 #pragma once
 #include "gemm_tc.cuh"
+#include "actorder.cuh"
 
 namespace gq {
 
@@ -77,6 +78,33 @@ __global__ void __launch_bounds__(256) damp_copy_kernel(const float* __restrict_
         }
         if (i == j) v = (i < d) ? v + l : 1.f;
         A[i * n + j] = v;
+    }
+}
+
+// The damped copy of damp_copy_kernel for the permuted Hessian: A[i][j] =
+// H[perm[i]][perm[j]] (+ lambda on the diagonal) for j >= the start of i's 128-block,
+// identity padding past d.  One CTA per row of A: it reads one row of H, so every
+// sector of H is fetched once.  H must hold both triangles.
+__global__ void __launch_bounds__(256) damp_copy_perm_kernel(const float* __restrict__ H,
+                                                             const int* __restrict__ perm, long long d, long long n,
+                                                             const float* __restrict__ lam, float* __restrict__ A) {
+    const long long i = blockIdx.x;
+    const long long j0 = (i / NB) * NB;
+    float* out = A + i * n;
+    if (i >= d) {
+        for (long long j = j0 + threadIdx.x; j < n; j += blockDim.x) out[j] = (i == j) ? 1.f : 0.f;
+        return;
+    }
+    const float l = lam[0];
+    const float* src = H + (long long)checked_index(perm, i, d) * d;
+    for (long long j = j0 + threadIdx.x; j < n; j += blockDim.x) {
+        float v = 0.f;
+        if (j < d) {
+            v = src[checked_index(perm, j, d)];
+            if (!isfinite(v)) record_status(GPTQ_ERR_NONFINITE, i * d + j);
+            if (i == j) v += l;
+        }
+        out[j] = v;
     }
 }
 
@@ -430,11 +458,12 @@ inline long long chol_n(long long d) { return (d + gq::NB - 1) / gq::NB * gq::NB
 
 struct HinvWs {
     float *A, *RS_hi, *RS_lo, *U_hi, *U_lo, *UT_hi, *UT_lo, *TT_hi, *TT_lo, *AP_hi, *AP_lo, *scal;
+    int* rank;   // inverse of a caller's permutation (permuted factorization only)
 };
 
 inline size_t hinv_ws_bytes(long long d) {
     const long long n = chol_n(d);
-    return (size_t)(9 * n * n + 2 * n * gq::NB + 64) * sizeof(float);
+    return (size_t)(9 * n * n + 2 * n * gq::NB + 64 + n) * sizeof(float);
 }
 
 inline HinvWs hinv_ws_carve(void* ws, long long d) {
@@ -464,6 +493,8 @@ inline HinvWs hinv_ws_carve(void* ws, long long d) {
     w.AP_lo = p;
     p += n * gq::NB;
     w.scal = p;
+    p += 64;
+    w.rank = reinterpret_cast<int*>(p);
     return w;
 }
 
@@ -471,7 +502,7 @@ inline HinvWs hinv_ws_carve(void* ws, long long d) {
 // Enqueue the whole factorization.  Leaves U (public, d x d) and the splits of U
 // (U_hi/U_lo row-major, UT_hi/UT_lo transposed; n x n) in the workspace.
 inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* U, void* ws,
-                            cudaStream_t st) {
+                            cudaStream_t st, const int* perm = nullptr) {
     const long long n = chol_n(d);
     const int T = (int)(n / gq::NB);
     HinvWs w = hinv_ws_carve(ws, d);
@@ -480,7 +511,19 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
         gq::diag_mean_kernel<<<1, 1024, 0, st>>>(H, d, damp_rel, w.scal);
     }
     GQ_TRY(cudaGetLastError());
-    {
+    if (perm) {   // factor P^T Hd P: validate the permutation, then a gathering damped copy
+        GQ_TRY(cudaMemsetAsync(w.rank, 0xFF, (size_t)d * sizeof(int), st));
+        {
+            gqh::TimedScope ts__("perm_invert", st);
+            gq::perm_invert_kernel<<<(unsigned)((d + 255) / 256), 256, 0, st>>>(perm, d, w.rank);
+        }
+        GQ_TRY(cudaGetLastError());
+        {
+            gqh::TimedScope ts__("damp_copy_perm", st);
+            gq::damp_copy_perm_kernel<<<(unsigned)n, 256, 0, st>>>(H, perm, d, n, w.scal, w.A);
+        }
+        GQ_TRY(cudaGetLastError());
+    } else {
         const dim3 grid((unsigned)(n / gq::NB), (unsigned)(n / gq::NB));
         {
             gqh::TimedScope ts__("damp_copy", st);

@@ -24,6 +24,7 @@
 #pragma once
 #include "gemm_tc.cuh"
 #include "pack.cuh"
+#include "actorder.cuh"
 
 namespace gq {
 
@@ -525,6 +526,50 @@ cudaError_t quant_run_bits(float* W, const float* U, long long d_out, long long 
         GQ_TRY(cudaGetLastError());
     }
     return cudaSuccess;
+}
+
+// Activation-ordered column loop: the workspace of the plain loop, then the gathered
+// weights Wp, the permuted codes and the inverse permutation.
+inline size_t act_quant_ws_bytes(long long d_out, long long d_in, int g, int bits) {
+    const long long words = (d_in * bits + 31) / 32;
+    return quant_ws_bytes(d_out, d_in, g) + align256((size_t)d_out * d_in * 4) +
+           align256((size_t)words * d_out * 4) + align256((size_t)d_in * 4);
+}
+
+// Validate perm (rank = its inverse), gather W's columns into quantization order, run
+// the unchanged column loop on them (scales, zeros and err_sq go straight to the
+// caller's buffers: groups are in quantization order), then repack the codes in the
+// original column order and write g_idx.
+template <int BITS>
+cudaError_t act_quant_run_bits(const float* W, const float* U, const int* perm, long long d_out, long long d_in,
+                               const gptq_config& cfg, int32_t* qweight, __half* scales, int32_t* qzeros,
+                               int32_t* g_idx, float* err_sq, void* ws, cudaStream_t st) {
+    const long long words = (d_in * BITS + 31) / 32;
+    uint8_t* p = static_cast<uint8_t*>(ws) + quant_ws_bytes(d_out, d_in, cfg.group_size);
+    float* Wp = reinterpret_cast<float*>(p);
+    p += align256((size_t)d_out * d_in * 4);
+    int32_t* qw_perm = reinterpret_cast<int32_t*>(p);
+    p += align256((size_t)words * d_out * 4);
+    int* rank = reinterpret_cast<int*>(p);
+    GQ_TRY(cudaMemsetAsync(rank, 0xFF, (size_t)d_in * sizeof(int), st));
+    {
+        gqh::TimedScope ts__("perm_invert", st);
+        gq::perm_invert_kernel<<<(unsigned)((d_in + 255) / 256), 256, 0, st>>>(perm, d_in, rank);
+    }
+    GQ_TRY(cudaGetLastError());
+    {
+        gqh::TimedScope ts__("gather_cols", st);
+        gq::gather_cols_kernel<<<(unsigned)std::min<long long>(d_out, 8192), 256, 0, st>>>(W, perm, d_out, d_in, Wp);
+    }
+    GQ_TRY(cudaGetLastError());
+    GQ_TRY(quant_run_bits<BITS>(Wp, U, d_out, d_in, cfg, qw_perm, scales, qzeros, err_sq, ws, st));
+    const long long items = std::max(words * d_out, d_in);
+    {
+        gqh::TimedScope ts__("unpermute_codes", st);
+        gq::unpermute_codes_kernel<<<(unsigned)std::min<long long>((items + 255) / 256, 8192), 256, 0, st>>>(
+            qw_perm, rank, d_out, d_in, BITS, cfg.group_size < 0 ? (int)d_in : cfg.group_size, qweight, g_idx);
+    }
+    return cudaGetLastError();
 }
 
 }  // namespace gqh

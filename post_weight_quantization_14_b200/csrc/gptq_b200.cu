@@ -181,7 +181,8 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 static gptq_status check_config(const gptq_config* cfg) {
     if (!cfg) return fail(GPTQ_ERR_INVALID_ARG, "cfg is NULL");
-    if (cfg->desc_act) return fail(GPTQ_ERR_UNSUPPORTED, "desc_act (activation ordering) is not implemented");
+    if (cfg->desc_act < 0 || cfg->desc_act > 2)
+        return fail(GPTQ_ERR_INVALID_ARG, "desc_act must be 0, 1 (ascending) or 2 (descending) (got %d)", cfg->desc_act);
     if (!(cfg->bits == 2 || cfg->bits == 3 || cfg->bits == 4 || cfg->bits == 8))
         return fail(GPTQ_ERR_INVALID_ARG, "bits must be 2, 3, 4 or 8 (got %d)", cfg->bits);
     if (cfg->block_size != 128) return fail(GPTQ_ERR_INVALID_ARG, "block_size must be 128 (got %d)", cfg->block_size);
@@ -281,8 +282,8 @@ size_t gptq_prepare_hinv_workspace_bytes(int64_t d_in) {
     return hinv_ws_bytes(d_in);
 }
 
-gptq_status gptq_prepare_hinv(const float* H, int64_t d_in, float damp_rel, float* U, void* ws, size_t ws_bytes,
-                              int64_t* bad_col, float* lambda_out, void* stream) {
+static gptq_status prepare_hinv_common(const float* H, const int32_t* perm, int64_t d_in, float damp_rel, float* U,
+                                       void* ws, size_t ws_bytes, int64_t* bad_col, float* lambda_out, void* stream) {
     if (!H || !U) return fail(GPTQ_ERR_INVALID_ARG, "H and U must be non-NULL");
     if (d_in < 8 || d_in > 65536 || d_in % 8) return fail(GPTQ_ERR_INVALID_ARG, "d_in must be a multiple of 8 in [8, 65536]");
     if (!(damp_rel >= 0.f) || damp_rel > 1e30f) return fail(GPTQ_ERR_INVALID_ARG, "damp_rel must be finite and >= 0");
@@ -293,7 +294,7 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d_in, float damp_rel, floa
     long long idx = -1;
     gptq_status pre = read_status(st, &idx);  // clears any stale device status
     (void)pre;
-    cudaError_t e = hinv_run(H, d_in, damp_rel, U, ws, st);
+    cudaError_t e = hinv_run(H, d_in, damp_rel, U, ws, st, perm);
     if (e != cudaSuccess) return cuda_fail(e, "prepare_hinv");
     idx = -1;
     gptq_status s = read_status(st, &idx);
@@ -308,8 +309,102 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d_in, float damp_rel, floa
     return s;
 }
 
+}  // extern "C"
+
+static gptq_status check_common(int64_t d_out, int64_t d_in, const float* W, const float* U) {
+    if (d_out < 1 || d_out > (1ll << 30)) return fail(GPTQ_ERR_INVALID_ARG, "d_out out of range");
+    if (d_in < 8 || d_in > 65536 || d_in % 8) return fail(GPTQ_ERR_INVALID_ARG, "d_in must be a multiple of 8 in [8, 65536]");
+    if (!aligned16(W) || !aligned16(U)) return fail(GPTQ_ERR_INVALID_ARG, "W and U must be 16-byte aligned");
+    return GPTQ_OK;
+}
+
+static gptq_status dequant_common(const int32_t* qweight, const uint16_t* scales, const int32_t* qzeros,
+                                  const int32_t* g_idx, int64_t d_out, int64_t d_in, const gptq_config* cfg,
+                                  float* W_hat, void* stream) {
+    if (!cfg) return fail(GPTQ_ERR_INVALID_ARG, "cfg is NULL");
+    if (!(cfg->bits == 2 || cfg->bits == 3 || cfg->bits == 4 || cfg->bits == 8))
+        return fail(GPTQ_ERR_INVALID_ARG, "bits must be 2, 3, 4 or 8");
+    if (!qweight || !scales || !W_hat) return fail(GPTQ_ERR_INVALID_ARG, "qweight, scales and W_hat must be non-NULL");
+    if (cfg->sym ? (qzeros != nullptr) : (qzeros == nullptr))
+        return fail(GPTQ_ERR_INVALID_ARG, "qzeros must be given iff asymmetric");
+    if (d_out < 1 || d_in < 1) return fail(GPTQ_ERR_INVALID_ARG, "d_out and d_in must be >= 1");
+    const int g = cfg->group_size < 0 ? (int)d_in : cfg->group_size;
+    if (g < 1) return fail(GPTQ_ERR_INVALID_ARG, "group_size must be -1 or >= 1");
+    const long long total = d_out * d_in;
+    {
+        gqh::TimedScope ts__("dequant", (cudaStream_t)stream);
+        gq::dequant_kernel<<<(unsigned)std::min<long long>((total + 255) / 256, 16384), 256, 0, (cudaStream_t)stream>>>(
+            qweight, reinterpret_cast<const __half*>(scales), qzeros, g_idx, d_out, d_in, cfg->bits, g, cfg->sym, W_hat);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "dequant");
+    return GPTQ_OK;
+}
+
+extern "C" {
+
+gptq_status gptq_prepare_hinv(const float* H, int64_t d_in, float damp_rel, float* U, void* ws, size_t ws_bytes,
+                              int64_t* bad_col, float* lambda_out, void* stream) {
+    return prepare_hinv_common(H, nullptr, d_in, damp_rel, U, ws, ws_bytes, bad_col, lambda_out, stream);
+}
+
+gptq_status gptq_prepare_hinv_permuted(const float* H, const int32_t* perm, int64_t d_in, float damp_rel, float* U,
+                                       void* ws, size_t ws_bytes, int64_t* bad_col, float* lambda_out, void* stream) {
+    if (!perm) return fail(GPTQ_ERR_INVALID_ARG, "perm must be non-NULL");
+    return prepare_hinv_common(H, perm, d_in, damp_rel, U, ws, ws_bytes, bad_col, lambda_out, stream);
+}
+
+gptq_status gptq_act_sum_accumulate(const void* X, gptq_dtype xt, int64_t n, int64_t d_in, double* act,
+                                    int accumulate, void* stream) {
+    if (!X || !act) return fail(GPTQ_ERR_INVALID_ARG, "X and act must be non-NULL");
+    if (xt != GPTQ_BF16 && xt != GPTQ_F32) return fail(GPTQ_ERR_INVALID_ARG, "unknown X dtype %d", (int)xt);
+    if (n < 1 || n > (1ll << 30)) return fail(GPTQ_ERR_INVALID_ARG, "n out of range (%lld)", (long long)n);
+    if (d_in < 8 || d_in > 65536 || d_in % 8) return fail(GPTQ_ERR_INVALID_ARG, "d_in must be a multiple of 8 in [8, 65536]");
+    if (!aligned16(X) || (reinterpret_cast<uintptr_t>(act) & 7u))
+        return fail(GPTQ_ERR_INVALID_ARG, "X must be 16-byte and act 8-byte aligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    const unsigned grid = (unsigned)((d_in + gq::AS_COLS - 1) / gq::AS_COLS);
+    {
+        gqh::TimedScope ts__("act_sum", st);
+        if (xt == GPTQ_BF16)
+            gq::act_sum_kernel<true><<<grid, 256, 0, st>>>(X, n, d_in, accumulate ? 1 : 0, act);
+        else
+            gq::act_sum_kernel<false><<<grid, 256, 0, st>>>(X, n, d_in, accumulate ? 1 : 0, act);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "act_sum_accumulate");
+    return GPTQ_OK;
+}
+
+gptq_status gptq_act_order(const double* act, int64_t d_in, int desc_act, int32_t* perm, int32_t* rank,
+                           void* stream) {
+    if (!act || !perm || !rank) return fail(GPTQ_ERR_INVALID_ARG, "act, perm and rank must be non-NULL");
+    if (d_in < 1 || d_in > 65536) return fail(GPTQ_ERR_INVALID_ARG, "d_in must be in [1, 65536]");
+    if (desc_act != 1 && desc_act != 2)
+        return fail(GPTQ_ERR_INVALID_ARG, "desc_act must be 1 (ascending) or 2 (descending) (got %d)", desc_act);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(rank, 0, (size_t)d_in * sizeof(int32_t), st);
+    if (e != cudaSuccess) return cuda_fail(e, "act_order");
+    {
+        gqh::TimedScope ts__("act_rank", st);
+        const dim3 grid((unsigned)((d_in + gq::RK_THREADS - 1) / gq::RK_THREADS),
+                        (unsigned)((d_in + gq::RK_CHUNK - 1) / gq::RK_CHUNK));
+        gq::act_rank_kernel<<<grid, gq::RK_THREADS, 0, st>>>(act, d_in, desc_act == 2 ? 1 : 0, rank);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "act_order");
+    {
+        gqh::TimedScope ts__("act_perm", st);
+        gq::act_perm_kernel<<<(unsigned)((d_in + 255) / 256), 256, 0, st>>>(rank, d_in, perm);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "act_order");
+    return GPTQ_OK;
+}
+
 size_t gptq_quantize_workspace_bytes(int64_t d_out, int64_t d_in, const gptq_config* cfg) {
     if (d_out < 1 || d_in < 1 || !cfg) return 0;
+    if (cfg->desc_act) return act_quant_ws_bytes(d_out, d_in, cfg->group_size, cfg->bits);
     return quant_ws_bytes(d_out, d_in, cfg->group_size);
 }
 
@@ -318,12 +413,13 @@ gptq_status gptq_quantize_layer(float* W, const float* U, int64_t d_out, int64_t
                                 size_t ws_bytes, void* stream) {
     gptq_status cs = check_config(cfg);
     if (cs != GPTQ_OK) return cs;
+    if (cfg->desc_act)
+        return fail(GPTQ_ERR_INVALID_ARG, "desc_act != 0: call gptq_quantize_layer_act_order with the permutation");
     if (!W || !U || !qweight || !scales) return fail(GPTQ_ERR_INVALID_ARG, "W, U, qweight and scales must be non-NULL");
     if (cfg->sym && qzeros) return fail(GPTQ_ERR_INVALID_ARG, "qzeros must be NULL for symmetric quantization");
     if (!cfg->sym && !qzeros) return fail(GPTQ_ERR_INVALID_ARG, "qzeros is required for asymmetric quantization");
-    if (d_out < 1 || d_out > (1ll << 30)) return fail(GPTQ_ERR_INVALID_ARG, "d_out out of range");
-    if (d_in < 8 || d_in > 65536 || d_in % 8) return fail(GPTQ_ERR_INVALID_ARG, "d_in must be a multiple of 8 in [8, 65536]");
-    if (!aligned16(W) || !aligned16(U)) return fail(GPTQ_ERR_INVALID_ARG, "W and U must be 16-byte aligned");
+    cs = check_common(d_out, d_in, W, U);
+    if (cs != GPTQ_OK) return cs;
     const size_t need = quant_ws_bytes(d_out, d_in, cfg->group_size);
     if (!ws || ws_bytes < need || !aligned16(ws)) return fail(GPTQ_ERR_WORKSPACE, "workspace needs %zu bytes", need);
     cudaStream_t st = (cudaStream_t)stream;
@@ -336,6 +432,34 @@ gptq_status gptq_quantize_layer(float* W, const float* U, int64_t d_out, int64_t
         default: e = quant_run_bits<8>(W, U, d_out, d_in, *cfg, qweight, sc, qzeros, err_sq, ws, st); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "quantize_layer");
+    return GPTQ_OK;
+}
+
+gptq_status gptq_quantize_layer_act_order(const float* W, const float* U, const int32_t* perm, int64_t d_out,
+                                          int64_t d_in, const gptq_config* cfg, int32_t* qweight, uint16_t* scales,
+                                          int32_t* qzeros, int32_t* g_idx, float* err_sq, void* ws, size_t ws_bytes,
+                                          void* stream) {
+    gptq_status cs = check_config(cfg);
+    if (cs != GPTQ_OK) return cs;
+    if (!cfg->desc_act) return fail(GPTQ_ERR_INVALID_ARG, "desc_act must be 1 or 2 for the activation-ordered loop");
+    if (!W || !U || !perm || !qweight || !scales || !g_idx)
+        return fail(GPTQ_ERR_INVALID_ARG, "W, U, perm, qweight, scales and g_idx must be non-NULL");
+    if (cfg->sym && qzeros) return fail(GPTQ_ERR_INVALID_ARG, "qzeros must be NULL for symmetric quantization");
+    if (!cfg->sym && !qzeros) return fail(GPTQ_ERR_INVALID_ARG, "qzeros is required for asymmetric quantization");
+    cs = check_common(d_out, d_in, W, U);
+    if (cs != GPTQ_OK) return cs;
+    const size_t need = act_quant_ws_bytes(d_out, d_in, cfg->group_size, cfg->bits);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return fail(GPTQ_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+    cudaStream_t st = (cudaStream_t)stream;
+    __half* sc = reinterpret_cast<__half*>(scales);
+    cudaError_t e;
+    switch (cfg->bits) {
+        case 2: e = act_quant_run_bits<2>(W, U, perm, d_out, d_in, *cfg, qweight, sc, qzeros, g_idx, err_sq, ws, st); break;
+        case 3: e = act_quant_run_bits<3>(W, U, perm, d_out, d_in, *cfg, qweight, sc, qzeros, g_idx, err_sq, ws, st); break;
+        case 4: e = act_quant_run_bits<4>(W, U, perm, d_out, d_in, *cfg, qweight, sc, qzeros, g_idx, err_sq, ws, st); break;
+        default: e = act_quant_run_bits<8>(W, U, perm, d_out, d_in, *cfg, qweight, sc, qzeros, g_idx, err_sq, ws, st); break;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "quantize_layer_act_order");
     return GPTQ_OK;
 }
 
@@ -358,24 +482,14 @@ gptq_status gptq_pack_int(const uint8_t* codes, int64_t rows, int64_t cols, int 
 
 gptq_status gptq_dequant(const int32_t* qweight, const uint16_t* scales, const int32_t* qzeros, int64_t d_out,
                          int64_t d_in, const gptq_config* cfg, float* W_hat, void* stream) {
-    if (!cfg) return fail(GPTQ_ERR_INVALID_ARG, "cfg is NULL");
-    if (!(cfg->bits == 2 || cfg->bits == 3 || cfg->bits == 4 || cfg->bits == 8))
-        return fail(GPTQ_ERR_INVALID_ARG, "bits must be 2, 3, 4 or 8");
-    if (!qweight || !scales || !W_hat) return fail(GPTQ_ERR_INVALID_ARG, "qweight, scales and W_hat must be non-NULL");
-    if (cfg->sym ? (qzeros != nullptr) : (qzeros == nullptr))
-        return fail(GPTQ_ERR_INVALID_ARG, "qzeros must be given iff asymmetric");
-    if (d_out < 1 || d_in < 1) return fail(GPTQ_ERR_INVALID_ARG, "d_out and d_in must be >= 1");
-    const int g = cfg->group_size < 0 ? (int)d_in : cfg->group_size;
-    if (g < 1) return fail(GPTQ_ERR_INVALID_ARG, "group_size must be -1 or >= 1");
-    const long long total = d_out * d_in;
-    {
-        gqh::TimedScope ts__("dequant", (cudaStream_t)stream);
-        gq::dequant_kernel<<<(unsigned)std::min<long long>((total + 255) / 256, 16384), 256, 0, (cudaStream_t)stream>>>(
-            qweight, reinterpret_cast<const __half*>(scales), qzeros, d_out, d_in, cfg->bits, g, cfg->sym, W_hat);
-    }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "dequant");
-    return GPTQ_OK;
+    return dequant_common(qweight, scales, qzeros, nullptr, d_out, d_in, cfg, W_hat, stream);
+}
+
+gptq_status gptq_dequant_g_idx(const int32_t* qweight, const uint16_t* scales, const int32_t* qzeros,
+                               const int32_t* g_idx, int64_t d_out, int64_t d_in, const gptq_config* cfg,
+                               float* W_hat, void* stream) {
+    if (!g_idx) return fail(GPTQ_ERR_INVALID_ARG, "g_idx must be non-NULL");
+    return dequant_common(qweight, scales, qzeros, g_idx, d_out, d_in, cfg, W_hat, stream);
 }
 
 gptq_status gptq_sync_status(void* stream) { return read_status((cudaStream_t)stream, nullptr); }

@@ -51,15 +51,26 @@ __device__ __forceinline__ uint32_t stream_code(const int32_t* words, long long 
 }
 
 // W_hat[o, c] = scale[g(c), o] * (q[o, c] - zero[g(c), o]); one thread per weight, row-major.
+// g(c) = c / g, or g_idx[c] when a per-column group index is given (activation ordering);
+// an index outside [0, n_groups) is recorded as GPTQ_ERR_INVALID_ARG and group 0 is used.
 __global__ void dequant_kernel(const int32_t* __restrict__ qweight, const __half* __restrict__ scales,
-                               const int32_t* __restrict__ qzeros, long long d_out, long long d_in,
-                               int bits, int g, int sym, float* __restrict__ W_hat) {
+                               const int32_t* __restrict__ qzeros, const int32_t* __restrict__ g_idx,
+                               long long d_out, long long d_in, int bits, int g, int sym,
+                               float* __restrict__ W_hat) {
     const long long total = d_out * d_in;
     const long long zwords = (d_out * bits + 31) / 32;
+    const long long ng = (d_in + g - 1) / g;
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
          idx += (long long)gridDim.x * blockDim.x) {
         const long long o = idx / d_in, c = idx % d_in;
-        const long long gi = c / g;
+        long long gi = c / g;
+        if (g_idx) {
+            gi = g_idx[c];
+            if (gi < 0 || gi >= ng) {
+                record_status(GPTQ_ERR_INVALID_ARG, c);
+                gi = 0;
+            }
+        }
         const uint32_t q = stream_code(qweight + o, d_out, c, bits);
         const float s = __half2float(scales[gi * d_out + o]);
         float z;

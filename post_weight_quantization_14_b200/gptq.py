@@ -67,6 +67,13 @@ _SIGS = {
     "gptq_timing_report": (_sz, [ctypes.c_char_p, _sz]),
     "gptq_selftest_bounded_wait": (_int, [ctypes.c_uint64, _vp]),
     "gptq_hessian_accumulate_fixed_scratch": (_int, [_vp, _int, _i64, _i64, _vp, _int, _vp]),
+    "gptq_act_sum_accumulate": (_int, [_vp, _int, _i64, _i64, _vp, _int, _vp]),
+    "gptq_act_order": (_int, [_vp, _i64, _int, _vp, _vp, _vp]),
+    "gptq_prepare_hinv_permuted": (_int, [_vp, _vp, _i64, _f32, _vp, _vp, _sz, ctypes.POINTER(_i64),
+                                          ctypes.POINTER(_f32), _vp]),
+    "gptq_quantize_layer_act_order": (_int, [_vp, _vp, _vp, _i64, _i64, ctypes.POINTER(GptqConfig), _vp, _vp, _vp,
+                                             _vp, _vp, _vp, _sz, _vp]),
+    "gptq_dequant_g_idx": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, ctypes.POINTER(GptqConfig), _vp, _vp]),
 }
 
 
@@ -92,11 +99,16 @@ def header_functions() -> list[str]:
     return sorted(set(re.findall(r"\b(gptq_[a-z0-9_]+)\s*\(", text)))
 
 
-def make_config(bits=4, group_size=128, sym=False, block_size=128, damp_rel=0.01, desc_act=False) -> GptqConfig:
+ACT_ASCENDING = 1    # desc_act = 1: ascending sum of |x|, least influential columns first
+ACT_DESCENDING = 2   # desc_act = 2: descending
+
+
+def make_config(bits=4, group_size=128, sym=False, block_size=128, damp_rel=0.01, desc_act=0) -> GptqConfig:
+    """desc_act: 0 natural order, 1 ascending and 2 descending activation order (True means 1)."""
     c = GptqConfig()
     lib().gptq_default_config(ctypes.byref(c))
     c.bits, c.group_size, c.sym, c.block_size = int(bits), int(group_size), int(bool(sym)), int(block_size)
-    c.damp_rel, c.desc_act = float(damp_rel), int(bool(desc_act))
+    c.damp_rel, c.desc_act = float(damp_rel), int(desc_act)
     return c
 
 
@@ -172,6 +184,57 @@ def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, cfg: GptqConfig, qweig
                                      _stream(stream)))
 
 
+def gptq_act_sum_accumulate(X: torch.Tensor, act: torch.Tensor, accumulate: bool = False, stream=None) -> torch.Tensor:
+    """act[c] (+)= sum_t |X[t, c]| (fp64).  X: [n, d_in] bfloat16 or float32; act: float64 [d_in]."""
+    n, d_in = X.shape
+    xt = GPTQ_BF16 if X.dtype == torch.bfloat16 else GPTQ_F32 if X.dtype == torch.float32 else None
+    if xt is None:
+        raise ValueError("X must be bfloat16 or float32")
+    if act.dtype != torch.float64 or tuple(act.shape) != (d_in,):
+        raise ValueError("act must be float64 [d_in]")
+    _check(lib().gptq_act_sum_accumulate(_ptr(X), xt, n, d_in, _ptr(act), int(bool(accumulate)), _stream(stream)))
+    return act
+
+
+def gptq_act_order(act: torch.Tensor, desc_act: int, perm: torch.Tensor, rank: torch.Tensor, stream=None) -> None:
+    """perm[k] = column quantized at position k, rank = its inverse (int32 [d_in] each)."""
+    _check(lib().gptq_act_order(_ptr(act), act.numel(), int(desc_act), _ptr(perm), _ptr(rank), _stream(stream)))
+
+
+def gptq_prepare_hinv_permuted(H: torch.Tensor, perm: torch.Tensor, U: torch.Tensor, damp_rel: float = 0.01,
+                               workspace: torch.Tensor | None = None, stream=None) -> float:
+    """U of the permuted Hessian H[perm][:, perm]; returns lambda.  Synchronises the stream."""
+    d = H.shape[0]
+    need = lib().gptq_prepare_hinv_workspace_bytes(d)
+    ws = workspace if workspace is not None else _workspace(need, H.device)
+    bad = _i64(-1)
+    lam = _f32(0.0)
+    st = lib().gptq_prepare_hinv_permuted(_ptr(H), _ptr(perm), d, float(damp_rel), _ptr(U), _ptr(ws), ws.numel(),
+                                          ctypes.byref(bad), ctypes.byref(lam), _stream(stream))
+    _check(st, bad.value)
+    return float(lam.value)
+
+
+def gptq_quantize_layer_act_order(W: torch.Tensor, U: torch.Tensor, perm: torch.Tensor, cfg: GptqConfig,
+                                  qweight: torch.Tensor, scales: torch.Tensor, qzeros: torch.Tensor | None,
+                                  g_idx: torch.Tensor, err_sq: torch.Tensor | None = None,
+                                  workspace: torch.Tensor | None = None, stream=None) -> None:
+    """Column loop in the order perm (cfg.desc_act 1 or 2); W is read only; codes in original order."""
+    d_out, d_in = W.shape
+    need = lib().gptq_quantize_workspace_bytes(d_out, d_in, ctypes.byref(cfg))
+    ws = workspace if workspace is not None else _workspace(need, W.device)
+    _check(lib().gptq_quantize_layer_act_order(_ptr(W), _ptr(U), _ptr(perm), d_out, d_in, ctypes.byref(cfg),
+                                               _ptr(qweight), _ptr(scales), _ptr(qzeros), _ptr(g_idx), _ptr(err_sq),
+                                               _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def gptq_dequant_g_idx(qweight, scales, qzeros, g_idx, d_out: int, d_in: int, cfg: GptqConfig, W_hat: torch.Tensor,
+                       stream=None) -> torch.Tensor:
+    _check(lib().gptq_dequant_g_idx(_ptr(qweight), _ptr(scales), _ptr(qzeros), _ptr(g_idx), d_out, d_in,
+                                    ctypes.byref(cfg), _ptr(W_hat), _stream(stream)))
+    return W_hat
+
+
 def gptq_pack_int(codes: torch.Tensor, bits: int, layout: int, packed: torch.Tensor, stream=None) -> torch.Tensor:
     rows, cols = codes.shape
     _check(lib().gptq_pack_int(_ptr(codes), rows, cols, int(bits), int(layout), _ptr(packed), _stream(stream)))
@@ -219,6 +282,8 @@ class QuantizedLayer:
     qzeros: torch.Tensor | None  # int32 [n_groups, ceil(d_out*bits/32)] (None if sym)
     err_sq: torch.Tensor       # float32 [d_out]
     lam: float
+    g_idx: torch.Tensor | None = None   # int32 [d_in] with activation ordering
+    perm: torch.Tensor | None = None    # int32 [d_in] quantization order
 
 
 class LayerBuffers:
@@ -239,15 +304,31 @@ class LayerBuffers:
         self.qzeros = None if cfg.sym else torch.empty((ng, (d_out * cfg.bits + 31) // 32), dtype=torch.int32,
                                                       device=device)
         self.err_sq = torch.empty((d_out,), dtype=torch.float32, device=device)
+        if cfg.desc_act:
+            self.act = torch.empty((d_in,), dtype=torch.float64, device=device)
+            self.perm = torch.empty((d_in,), dtype=torch.int32, device=device)
+            self.rank = torch.empty((d_in,), dtype=torch.int32, device=device)
+            self.g_idx = torch.empty((d_in,), dtype=torch.int32, device=device)
 
 
 def quantize_layer(W: torch.Tensor, X: torch.Tensor, bits=4, group_size=128, sym=False, damp_rel=0.01,
-                   buffers: LayerBuffers | None = None, stream=None) -> QuantizedLayer:
-    """GPTQ of one linear layer: H = 2 X^T X, U = chol(Hd^-1) upper, column loop.  W is overwritten."""
-    cfg = buffers.cfg if buffers is not None else make_config(bits, group_size, sym, 128, damp_rel)
+                   desc_act=0, buffers: LayerBuffers | None = None, stream=None) -> QuantizedLayer:
+    """GPTQ of one linear layer: H = 2 X^T X, U = chol(Hd^-1) upper, column loop.
+
+    desc_act 0: natural column order, W is overwritten.  desc_act 1 / 2: columns in
+    ascending / descending order of sum_t |X[t, c]|; W is left unchanged and the result
+    carries g_idx and perm."""
+    cfg = buffers.cfg if buffers is not None else make_config(bits, group_size, sym, 128, damp_rel, desc_act)
     d_out, d_in = W.shape
     b = buffers or LayerBuffers(d_out, d_in, X.shape[0], X.dtype, cfg, W.device)
     gptq_hessian_accumulate(X, b.H, accumulate=False, workspace=b.ws, stream=stream)
-    lam = gptq_prepare_hinv(b.H, b.U, cfg.damp_rel, workspace=b.ws, stream=stream)
-    gptq_quantize_layer(W, b.U, cfg, b.qweight, b.scales, b.qzeros, b.err_sq, workspace=b.ws, stream=stream)
-    return QuantizedLayer(b.qweight, b.scales, b.qzeros, b.err_sq, lam)
+    if not cfg.desc_act:
+        lam = gptq_prepare_hinv(b.H, b.U, cfg.damp_rel, workspace=b.ws, stream=stream)
+        gptq_quantize_layer(W, b.U, cfg, b.qweight, b.scales, b.qzeros, b.err_sq, workspace=b.ws, stream=stream)
+        return QuantizedLayer(b.qweight, b.scales, b.qzeros, b.err_sq, lam)
+    gptq_act_sum_accumulate(X, b.act, accumulate=False, stream=stream)
+    gptq_act_order(b.act, cfg.desc_act, b.perm, b.rank, stream=stream)
+    lam = gptq_prepare_hinv_permuted(b.H, b.perm, b.U, cfg.damp_rel, workspace=b.ws, stream=stream)
+    gptq_quantize_layer_act_order(W, b.U, b.perm, cfg, b.qweight, b.scales, b.qzeros, b.g_idx, b.err_sq,
+                                  workspace=b.ws, stream=stream)
+    return QuantizedLayer(b.qweight, b.scales, b.qzeros, b.err_sq, lam, b.g_idx, b.perm)

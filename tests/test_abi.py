@@ -54,7 +54,8 @@ def _fake(n=1):
     ("group_size", 256, G.GPTQ_ERR_INVALID_ARG),
     ("block_size", 64, G.GPTQ_ERR_INVALID_ARG),
     ("sym", 2, G.GPTQ_ERR_INVALID_ARG),
-    ("desc_act", 1, G.GPTQ_ERR_UNSUPPORTED),
+    ("desc_act", 1, G.GPTQ_ERR_INVALID_ARG),     # the natural-order loop; act order has its own call
+    ("desc_act", 3, G.GPTQ_ERR_INVALID_ARG),
     ("damp_rel", -1.0, G.GPTQ_ERR_INVALID_ARG),
     ("damp_rel", float("nan"), G.GPTQ_ERR_INVALID_ARG),
 ])
@@ -117,3 +118,35 @@ def test_product_path_has_no_cpu_fallback():
     W = torch.zeros(8, 8)
     with pytest.raises(ValueError):
         G._ptr(W)
+
+
+def test_act_order_entry_points_validate_arguments():
+    L = G.lib()
+    c = G.make_config(desc_act=0)
+    q = lambda cfg, perm=_fake(7), g_idx=_fake(8), ws=1 << 40: L.gptq_quantize_layer_act_order(
+        _fake(1), _fake(2), perm, 64, 64, ctypes.byref(cfg), _fake(3), _fake(4), _fake(5), g_idx, None, _fake(6),
+        ws, None)
+    assert q(c) == G.GPTQ_ERR_INVALID_ARG                      # desc_act 0 belongs to gptq_quantize_layer
+    c.desc_act = 1
+    assert q(c, perm=None) == G.GPTQ_ERR_INVALID_ARG
+    assert q(c, g_idx=None) == G.GPTQ_ERR_INVALID_ARG
+    assert q(c, ws=16) == G.GPTQ_ERR_WORKSPACE
+    c.desc_act = 5
+    assert q(c) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_act_order(_fake(1), 64, 0, _fake(2), _fake(3), None) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_act_order(_fake(1), 64, 3, _fake(2), _fake(3), None) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_act_order(_fake(1), 0, 1, _fake(2), _fake(3), None) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_act_sum_accumulate(_fake(1), G.GPTQ_F32, 10, 60, _fake(2), 0, None) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_act_sum_accumulate(_fake(1), 7, 10, 64, _fake(2), 0, None) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_prepare_hinv_permuted(_fake(1), None, 64, 0.01, _fake(2), _fake(3), 1 << 40, None, None,
+                                        None) == G.GPTQ_ERR_INVALID_ARG
+    assert L.gptq_dequant_g_idx(_fake(1), _fake(2), _fake(3), None, 8, 64, ctypes.byref(G.make_config()), _fake(4),
+                                None) == G.GPTQ_ERR_INVALID_ARG
+
+
+def test_act_order_workspace_covers_permuted_copies():
+    L = G.lib()
+    plain = L.gptq_quantize_workspace_bytes(4096, 4096, ctypes.byref(G.make_config()))
+    act = L.gptq_quantize_workspace_bytes(4096, 4096, ctypes.byref(G.make_config(desc_act=1)))
+    # a permuted copy of W (fp32) and of the packed 4-bit codes, plus the inverse permutation
+    assert act - plain >= 4096 * 4096 * 4 + 4096 * 4096 // 2 + 4096 * 4
