@@ -16,7 +16,7 @@ namespace gq {
 constexpr int AS_COLS = 64;        // columns per CTA of act_sum_kernel (8 lanes x 8 columns)
 constexpr int AS_ROWS = 32;        // rows in flight per pass (256 threads / 8 lanes)
 constexpr int RK_THREADS = 256;    // columns ranked per CTA
-constexpr int RK_CHUNK = 1024;     // keys compared per CTA (one shared-memory tile)
+constexpr int RK_CHUNK = 256;      // keys compared per CTA (one shared-memory tile)
 
 // a[c] (+)= sum_t |X[t, c]| in fp64.  Thread (ty, tx) owns columns c0 + 8 tx .. + 7 of
 // rows ty, ty + 32, ...; the 32 partial sums per column are added in a fixed order, so
@@ -75,7 +75,7 @@ __device__ __forceinline__ unsigned long long order_key(double x, int descending
 }
 
 // rank[c] += #{j in this CTA's key chunk : key_j < key_c, or key_j == key_c and j < c}.
-// Grid (ceil(d / 256), ceil(d / 1024)); rank must be zero before the launch.  Integer
+// Grid (ceil(d / 256), ceil(d / 256)); rank must be zero before the launch.  Integer
 // atomics make the sum order-independent.
 __global__ void __launch_bounds__(RK_THREADS) act_rank_kernel(const double* __restrict__ a, long long d,
                                                               int descending, int* __restrict__ rank) {
@@ -123,7 +123,34 @@ __device__ __forceinline__ int checked_index(const int* __restrict__ perm, long 
     return c;
 }
 
-// Wp[o][k] = W[o][perm[k]], one CTA per row (the row's sectors are fetched once).
+// Wp[o][k] = W[o][perm[k]] with the row staged in shared memory: 16-byte loads of the
+// row, gathers from shared memory, 16-byte stores (d_in % 8 == 0; d_in * 4 bytes of
+// dynamic shared memory).  One CTA per row, rows strided over the grid.
+__global__ void __launch_bounds__(256) gather_cols_smem_kernel(const float* __restrict__ W,
+                                                               const int* __restrict__ perm, long long d_out,
+                                                               long long d_in, float* __restrict__ Wp) {
+    extern __shared__ float4 row4[];
+    const float* row = reinterpret_cast<const float*>(row4);
+    const long long q4 = d_in / 4;
+    for (long long o = blockIdx.x; o < d_out; o += gridDim.x) {
+        const float4* src = reinterpret_cast<const float4*>(W + o * d_in);
+        for (long long k = threadIdx.x; k < q4; k += blockDim.x) row4[k] = src[k];
+        __syncthreads();
+        float4* dst = reinterpret_cast<float4*>(Wp + o * d_in);
+        for (long long k = threadIdx.x; k < q4; k += blockDim.x) {
+            float4 v;
+            v.x = row[checked_index(perm, 4 * k, d_in)];
+            v.y = row[checked_index(perm, 4 * k + 1, d_in)];
+            v.z = row[checked_index(perm, 4 * k + 2, d_in)];
+            v.w = row[checked_index(perm, 4 * k + 3, d_in)];
+            dst[k] = v;
+        }
+        __syncthreads();
+    }
+}
+
+// Wp[o][k] = W[o][perm[k]] for rows too wide for shared memory: one CTA per row, the
+// gathered reads go through L1.
 __global__ void __launch_bounds__(256) gather_cols_kernel(const float* __restrict__ W, const int* __restrict__ perm,
                                                           long long d_out, long long d_in, float* __restrict__ Wp) {
     for (long long o = blockIdx.x; o < d_out; o += gridDim.x) {

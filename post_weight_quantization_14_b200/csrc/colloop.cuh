@@ -559,7 +559,17 @@ cudaError_t act_quant_run_bits(const float* W, const float* U, const int* perm, 
     GQ_TRY(cudaGetLastError());
     {
         gqh::TimedScope ts__("gather_cols", st);
-        gq::gather_cols_kernel<<<(unsigned)std::min<long long>(d_out, 8192), 256, 0, st>>>(W, perm, d_out, d_in, Wp);
+        const size_t row_bytes = (size_t)d_in * sizeof(float);
+        constexpr int kMaxRowBytes = 96 * 1024;   // two or more CTAs per SM
+        if (row_bytes <= (size_t)kMaxRowBytes) {   // the attribute is a fixed upper bound for every width
+            GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::gather_cols_smem_kernel), kMaxRowBytes));
+            const long long per_sm = std::min<long long>(8, (200 * 1024) / row_bytes);
+            gq::gather_cols_smem_kernel<<<(unsigned)std::min<long long>(d_out, per_sm * num_sms()), 256, row_bytes,
+                                          st>>>(W, perm, d_out, d_in, Wp);
+        } else {
+            gq::gather_cols_kernel<<<(unsigned)std::min<long long>(d_out, 8192), 256, 0, st>>>(W, perm, d_out, d_in,
+                                                                                          Wp);
+        }
     }
     GQ_TRY(cudaGetLastError());
     GQ_TRY(quant_run_bits<BITS>(Wp, U, d_out, d_in, cfg, qw_perm, scales, qzeros, err_sq, ws, st));

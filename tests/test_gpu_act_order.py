@@ -84,7 +84,7 @@ def test_act_sum_reports_nonfinite():
     with pytest.raises(G.GPTQError) as ei:
         G.gptq_sync_status()
     assert ei.value.status == G.GPTQ_ERR_NONFINITE
-    assert ei.value.index == 17
+    assert "index 17" in str(ei.value)
 
 
 # ---------------------------------------------------------------- ranking
