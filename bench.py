@@ -13,6 +13,7 @@ write) before every step, outside the per-step CUDA events.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
        python bench.py --workload stack7b [--steps K] [--warmup W]
+       python bench.py --workload dqgemm [--steps K] [--warmup W]   (dequantizing GEMM on the output)
 The stack7b workload times one block of the 7B-shaped stack (q, k, v, o 4096 x 4096;
 gate, up 11008 x 4096; down 4096 x 11008; n = 2048 tokens each, 4-bit g128) per step;
 every block has the same shapes, so the 32-block stack time is 32 times that.
@@ -282,6 +283,104 @@ def run_stack(args) -> None:
                       "weights_per_s": 32 * weights / (32 * block_ms / 1e3)}), flush=True)
 
 
+def run_dqgemm(args) -> None:
+    """Dequantizing GEMM Y = X W_hat^T on the packed output of the quantizer (4096 x 4096
+    attention layer, 4-bit asym g128, quantized once by this library): prefill with the
+    layer's 2048 bf16 tokens (timed, tensor roofline) and a 16-token decode batch (HBM
+    roofline over the packed weights).  X is larger than nothing in L2 can hide for the
+    prefill; the L2 is flushed before every timed step anyway."""
+    import numpy as np
+    import torch
+
+    from post_weight_quantization_14_b200 import gptq as G
+    from post_weight_quantization_14_b200 import inputs as I
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    layer = I.make_layer("attn", seed=0)
+    cfg = G.make_config(BITS, GROUP, SYM, 128, 0.01)
+    W = torch.from_numpy(layer.W).to(dev)
+    X = torch.from_numpy(layer.X_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    q = G.quantize_layer(W, X, buffers=G.LayerBuffers(D_OUT, D_IN, N_TOK, torch.bfloat16, cfg, dev))
+    G.gptq_sync_status()
+    Y = torch.empty((N_TOK, D_OUT), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(Xm, Ym, steps):
+        for _ in range(args.warmup):
+            G.gptq_dequant_gemm(Xm, q.qweight, q.scales, q.qzeros, D_OUT, D_IN, cfg, Ym)
+        G.gptq_sync_status()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for a, b in evs:
+            flush.fill_(1)
+            a.record(stream)
+            G.gptq_dequant_gemm(Xm, q.qweight, q.scales, q.qzeros, D_OUT, D_IN, cfg, Ym)
+            b.record(stream)
+        torch.cuda.synchronize()
+        G.gptq_sync_status()
+        return [a.elapsed_time(b) for a, b in evs]
+
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.3)
+    ms = timed(X, Y, args.steps)
+    X16 = X[:16].contiguous()
+    Y16 = torch.empty((16, D_OUT), dtype=torch.float32, device=dev)
+    ms16 = timed(X16, Y16, args.steps)
+    clocks = sampler.stop()
+    t = sum(ms) / len(ms)
+    t16 = statistics.median(ms16)
+    flops = 2.0 * N_TOK * D_OUT * D_IN
+    hbm, bf16, _, peak_kind = peaks()
+    packed_bytes = q.qweight.numel() * 4 + q.scales.numel() * 2 + q.qzeros.numel() * 4
+    bytes16 = packed_bytes + 16 * D_IN * 2 + 16 * D_OUT * 4
+
+    # end to end through the C ABI: X from pinned host memory in, Y back to pinned host memory
+    X_host = torch.from_numpy(layer.X_bits.view(np.int16)).pin_memory()
+    Y_host = torch.empty((N_TOK, D_OUT), dtype=torch.float32).pin_memory()
+    Xd = torch.empty(X_host.shape, dtype=torch.int16, device=dev)
+    e2e_steps = max(3, min(args.steps, 20))
+    torch.cuda.synchronize()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(stream)
+    for _ in range(e2e_steps):
+        Xd.copy_(X_host, non_blocking=True)
+        G.gptq_dequant_gemm(Xd.view(torch.bfloat16), q.qweight, q.scales, q.qzeros, D_OUT, D_IN, cfg, Y)
+        Y_host.copy_(Y, non_blocking=True)
+    eb.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ea.elapsed_time(eb) / e2e_steps
+
+    cpu = None
+    if not args.no_cpu_baseline:
+        from oracle import gptq_oracle as O
+        Xs = layer.X[:64].astype(np.float64)
+        qw, sc, qz = q.qweight.cpu().numpy(), q.scales.cpu().numpy(), q.qzeros.cpu().numpy()
+        t0 = time.perf_counter()
+        O.dequant_gemm(Xs, qw, sc, qz, D_OUT, D_IN, BITS, GROUP, SYM)
+        secs = time.perf_counter() - t0
+        cpu = {"value": 2.0 * 64 * D_OUT * D_IN / secs / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
+               "kind": "oracle", "sample": "64 of the 2048 tokens (fp64 dequantization + matmul)"}
+
+    print(json.dumps({
+        "metric": "dequant-GEMM Y = X W_hat^T on the packed 4-bit g128 format, 2048 x 4096 x 4096",
+        "value": flops / (t / 1e3) / 1e12, "unit": "TFLOP/s", "higher_is_better": True, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 x int4 -> f32", "data": "synthetic",
+        "config": {"workload": "dqgemm: attn 4096x4096 quantized 4-bit asym g128, X = its 2048 bf16 tokens",
+                   "M": N_TOK, "N": D_OUT, "K": D_IN, "l2": "flushed (256 MB write) before every step"},
+        "roofline": {"bound": "tensor", "achieved": flops / (t / 1e3) / 1e12, "peak": bf16, "unit": "TFLOP/s",
+                     "frac": flops / (t / 1e3) / 1e12 / bf16, "traffic": None, "peak_kind": peak_kind},
+        "decode16": {"ms": t16, "bytes": bytes16, "achieved_gbs": bytes16 / (t16 / 1e3) / 1e9, "peak_gbs": hbm,
+                     "frac": bytes16 / (t16 / 1e3) / 1e9 / hbm},
+        "e2e": {"value": flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": X_host.numel() * 2, "d2h_bytes_per_step": Y_host.numel() * 4,
+                "steps": e2e_steps},
+        "cpu_baseline": cpu, "gpu_launches": 2 * args.steps, "clocks": clocks,
+        "step_ms_min": min(ms), "step_ms_median": statistics.median(ms)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -289,12 +388,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="attn", choices=["attn", "stack7b"])
+    ap.add_argument("--workload", default="attn", choices=["attn", "stack7b", "dqgemm"])
     ap.add_argument("--desc-act", type=int, default=0, choices=[0, 1, 2],
                     help="activation ordering: 0 natural column order, 1 ascending, 2 descending sum of |x|")
     args = ap.parse_args()
     if args.workload == "stack7b":
         run_stack(args)
+        return
+    if args.workload == "dqgemm":
+        run_dqgemm(args)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

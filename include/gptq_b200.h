@@ -11,6 +11,7 @@
  *                                lazy 128-column blocks and one trailing update per block;
  *                                writes packed codes, fp16 scales and packed zero points.
  *   4. gptq_pack_int / gptq_dequant   packing of b-bit codes; W_hat = s * (q - z).
+ *   5. gptq_dequant_gemm         Y = X W_hat^T straight from the packed arrays.
  *
  * Activation ordering (desc_act) visits the columns in another order:
  * gptq_act_sum_accumulate (beside stage 1) and gptq_act_order rank the columns,
@@ -220,6 +221,23 @@ gptq_status gptq_quantize_layer_act_order(const float* W, const float* U, const 
 gptq_status gptq_dequant_g_idx(const int32_t* qweight, const uint16_t* scales, const int32_t* qzeros,
                                const int32_t* g_idx, int64_t d_out, int64_t d_in, const gptq_config* cfg,
                                float* W_hat, void* stream);
+
+/* ------------------------------------------------------------------ dequantizing GEMM
+ * Y[m, n] = sum_k X[m, k] * W_hat[n, k] with W_hat[n, k] = scale[g(k), n] * (q[n, k] - zero[g(k), n])
+ * (tutorial "阶段三": the integer times its scale; group-size article: groups along d_in),
+ * straight from the packed arrays of gptq_quantize_layer: the consumer of its output.
+ *   X        device bf16 (raw uint16 bit patterns) [M, d_in] row-major.
+ *   qweight, scales, qzeros  as written by gptq_quantize_layer (qzeros NULL iff sym).
+ *   Y        device fp32 [M, d_out] row-major, written in full.
+ * Each group's partial product X (q - z)^T is formed on the tensor cores from exact
+ * products (q - z is exact in bf16) with fp32 accumulation, then scaled by the group's
+ * fp16 scales once per tile and summed in fp32; no rounded copy of W_hat is made.
+ * Requires bits 2, 4 or 8 and group_size -1 or a multiple of 64 dividing d_in
+ * (GPTQ_ERR_UNSUPPORTED otherwise, also for desc_act != 0), d_in % 64 == 0,
+ * d_out % 8 == 0, all pointers 16-byte aligned. */
+gptq_status gptq_dequant_gemm(const void* X, int64_t M, const int32_t* qweight, const uint16_t* scales,
+                              const int32_t* qzeros, int64_t d_out, int64_t d_in, const gptq_config* cfg, float* Y,
+                              void* stream);
 
 /* Synchronise ``stream`` and return (and clear) the device status word. */
 gptq_status gptq_sync_status(void* stream);

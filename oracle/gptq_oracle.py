@@ -494,6 +494,13 @@ def dequant_packed(qweight, scales, qzeros, d_out, d_in, bits, group_size, sym, 
     return s * (codes - z)
 
 
+def dequant_gemm(X, qweight, scales, qzeros, d_out, d_in, bits, group_size, sym, g_idx=None) -> np.ndarray:
+    """Y = X W_hat^T in fp64, W_hat dequantized from the packed arrays (tutorial page,
+    "阶段三": the weights a layer computes with are the integers times their scales)."""
+    What = dequant_packed(qweight, scales, qzeros, d_out, d_in, bits, group_size, sym, g_idx)
+    return np.asarray(X, dtype=np.float64) @ What.T
+
+
 def metadata_bits_per_weight(d_out, d_in, bits, group_size, sym, scale_bits=16) -> float:
     """Bits of stored scale + zero per weight (group-size article, "存储代价")."""
     ng = n_groups(d_in, group_size)

@@ -302,6 +302,11 @@ struct TimedScope {
 bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
                   uint64_t ld, uint32_t box_rows, uint32_t box_cols);
 
+// The same over 4-byte elements without swizzle (box rows of up to 256 elements), for
+// operands that threads read element by element rather than the tensor cores.
+bool make_tmap_2d_plain(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                        uint32_t box_rows, uint32_t box_cols);
+
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device, size).
 cudaError_t ensure_smem_attr(const void* func, int bytes);
 

@@ -18,6 +18,7 @@
 #include "chol.cuh"
 #include "pack.cuh"
 #include "colloop.cuh"
+#include "dqgemm.cuh"
 
 namespace gqh {
 
@@ -86,7 +87,12 @@ using TmapKey = std::tuple<uintptr_t, int, uint64_t, uint64_t, uint64_t, uint32_
 static std::map<TmapKey, CUtensorMap> g_tmap_cache;
 
 static bool encode_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
-                           uint64_t ld, uint32_t box_rows, uint32_t box_cols);
+                           uint64_t ld, uint32_t box_rows, uint32_t box_cols, bool swizzle = true);
+
+bool make_tmap_2d_plain(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                        uint32_t box_rows, uint32_t box_cols) {
+    return encode_tmap_2d(map, base, 4, rows, cols, ld, box_rows, box_cols, false);
+}
 
 bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
                   uint64_t ld, uint32_t box_rows, uint32_t box_cols) {
@@ -143,7 +149,7 @@ cudaError_t ensure_smem_attr(const void* func, int bytes) {
 }
 
 static bool encode_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
-                           uint64_t ld, uint32_t box_rows, uint32_t box_cols) {
+                           uint64_t ld, uint32_t box_rows, uint32_t box_cols, bool swizzle) {
     if (!g_encode) {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -160,7 +166,8 @@ static bool encode_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, u
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -490,6 +497,36 @@ gptq_status gptq_dequant_g_idx(const int32_t* qweight, const uint16_t* scales, c
                                float* W_hat, void* stream) {
     if (!g_idx) return fail(GPTQ_ERR_INVALID_ARG, "g_idx must be non-NULL");
     return dequant_common(qweight, scales, qzeros, g_idx, d_out, d_in, cfg, W_hat, stream);
+}
+
+gptq_status gptq_dequant_gemm(const void* X, int64_t M, const int32_t* qweight, const uint16_t* scales,
+                              const int32_t* qzeros, int64_t d_out, int64_t d_in, const gptq_config* cfg, float* Y,
+                              void* stream) {
+    if (!cfg) return fail(GPTQ_ERR_INVALID_ARG, "cfg is NULL");
+    if (!X || !qweight || !scales || !Y) return fail(GPTQ_ERR_INVALID_ARG, "X, qweight, scales and Y must be non-NULL");
+    if (cfg->sym ? (qzeros != nullptr) : (qzeros == nullptr))
+        return fail(GPTQ_ERR_INVALID_ARG, "qzeros must be given iff asymmetric");
+    if (M < 1 || M > (1ll << 30)) return fail(GPTQ_ERR_INVALID_ARG, "M out of range (%lld)", (long long)M);
+    if (d_in < 64 || d_in > 65536 || d_in % 64) return fail(GPTQ_ERR_INVALID_ARG, "d_in must be a multiple of 64 in [64, 65536]");
+    if (d_out < 8 || d_out > (1ll << 30) || d_out % 8) return fail(GPTQ_ERR_INVALID_ARG, "d_out must be a positive multiple of 8");
+    if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(Y) || (qzeros && !aligned16(qzeros)))
+        return fail(GPTQ_ERR_INVALID_ARG, "X, qweight, scales, qzeros and Y must be 16-byte aligned");
+    if (!(cfg->bits == 2 || cfg->bits == 4 || cfg->bits == 8))
+        return fail(GPTQ_ERR_UNSUPPORTED, "dequant_gemm: bits must be 2, 4 or 8 (3-bit codes straddle words)");
+    const int g = cfg->group_size;
+    if (!(g == -1 || (g >= 64 && g % 64 == 0 && d_in % g == 0)))
+        return fail(GPTQ_ERR_UNSUPPORTED, "dequant_gemm: group_size must be -1 or a multiple of 64 dividing d_in");
+    if (cfg->desc_act) return fail(GPTQ_ERR_UNSUPPORTED, "dequant_gemm: no per-column group index (desc_act)");
+    cudaStream_t st = (cudaStream_t)stream;
+    const __half* sc = reinterpret_cast<const __half*>(scales);
+    cudaError_t e;
+    switch (cfg->bits) {
+        case 2: e = dq_gemm_run<2>(X, M, qweight, sc, qzeros, d_out, d_in, g, Y, st); break;
+        case 4: e = dq_gemm_run<4>(X, M, qweight, sc, qzeros, d_out, d_in, g, Y, st); break;
+        default: e = dq_gemm_run<8>(X, M, qweight, sc, qzeros, d_out, d_in, g, Y, st); break;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "dequant_gemm");
+    return GPTQ_OK;
 }
 
 gptq_status gptq_sync_status(void* stream) { return read_status((cudaStream_t)stream, nullptr); }

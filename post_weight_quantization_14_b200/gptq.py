@@ -74,6 +74,7 @@ _SIGS = {
     "gptq_quantize_layer_act_order": (_int, [_vp, _vp, _vp, _i64, _i64, ctypes.POINTER(GptqConfig), _vp, _vp, _vp,
                                              _vp, _vp, _vp, _sz, _vp]),
     "gptq_dequant_g_idx": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, ctypes.POINTER(GptqConfig), _vp, _vp]),
+    "gptq_dequant_gemm": (_int, [_vp, _i64, _vp, _vp, _vp, _i64, _i64, ctypes.POINTER(GptqConfig), _vp, _vp]),
 }
 
 
@@ -233,6 +234,18 @@ def gptq_dequant_g_idx(qweight, scales, qzeros, g_idx, d_out: int, d_in: int, cf
     _check(lib().gptq_dequant_g_idx(_ptr(qweight), _ptr(scales), _ptr(qzeros), _ptr(g_idx), d_out, d_in,
                                     ctypes.byref(cfg), _ptr(W_hat), _stream(stream)))
     return W_hat
+
+
+def gptq_dequant_gemm(X: torch.Tensor, qweight, scales, qzeros, d_out: int, d_in: int, cfg: GptqConfig,
+                      Y: torch.Tensor, stream=None) -> torch.Tensor:
+    """Y = X W_hat^T from the packed arrays.  X: bfloat16 [M, d_in]; Y: float32 [M, d_out]."""
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.shape[1] != d_in:
+        raise ValueError("X must be bfloat16 [M, d_in]")
+    if Y.dtype != torch.float32 or tuple(Y.shape) != (X.shape[0], d_out):
+        raise ValueError("Y must be float32 [M, d_out]")
+    _check(lib().gptq_dequant_gemm(_ptr(X), X.shape[0], _ptr(qweight), _ptr(scales), _ptr(qzeros), d_out, d_in,
+                                   ctypes.byref(cfg), _ptr(Y), _stream(stream)))
+    return Y
 
 
 def gptq_pack_int(codes: torch.Tensor, bits: int, layout: int, packed: torch.Tensor, stream=None) -> torch.Tensor:

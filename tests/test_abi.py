@@ -150,3 +150,17 @@ def test_act_order_workspace_covers_permuted_copies():
     act = L.gptq_quantize_workspace_bytes(4096, 4096, ctypes.byref(G.make_config(desc_act=1)))
     # a permuted copy of W (fp32) and of the packed 4-bit codes, plus the inverse permutation
     assert act - plain >= 4096 * 4096 * 4 + 4096 * 4096 // 2 + 4096 * 4
+
+
+def test_dequant_gemm_validates_arguments():
+    L = G.lib()
+    call = lambda cfg, M=16, d_out=64, d_in=128, qz=_fake(4): L.gptq_dequant_gemm(
+        _fake(1), M, _fake(2), _fake(3), qz, d_out, d_in, ctypes.byref(cfg), _fake(5), None)
+    c = G.make_config(4, 128, False)
+    assert call(c, d_in=96) == G.GPTQ_ERR_INVALID_ARG            # d_in % 64
+    assert call(c, d_out=60) == G.GPTQ_ERR_INVALID_ARG           # d_out % 8
+    assert call(c, M=0) == G.GPTQ_ERR_INVALID_ARG
+    assert call(c, qz=None) == G.GPTQ_ERR_INVALID_ARG            # asymmetric needs qzeros
+    assert call(G.make_config(3, 128, False)) == G.GPTQ_ERR_UNSUPPORTED   # 3-bit codes straddle words
+    assert call(G.make_config(4, 32, False)) == G.GPTQ_ERR_UNSUPPORTED    # groups narrower than a K tile
+    assert call(G.make_config(4, 128, False, desc_act=1)) == G.GPTQ_ERR_UNSUPPORTED

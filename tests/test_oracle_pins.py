@@ -468,3 +468,25 @@ def test_act_order_error_identity_and_packed_roundtrip():
     qz = O.pack_qzeros(r.zeros, 4)
     Wh = O.dequant_packed(qw, r.scales, qz, 7, 48, 4, 16, False, g_idx=r.g_idx)
     np.testing.assert_array_equal(Wh, r.what)
+
+
+# ---------------------------------------------------------------- dequantizing GEMM
+
+def test_dequant_gemm_hand_example():
+    # 2 x 4 weights, 4-bit, groups of 2 along d_in; W_hat by hand:
+    #   row 0: 0.5 (1-1), 0.5 (2-1), 2 (3-0), 2 (4-0)   = [0, 0.5, 6, 8]
+    #   row 1: 0.25 (15-8), 0.25 (0-8), 1 (7-7), 1 (8-7) = [1.75, -2, 0, 1]
+    codes = np.array([[1, 2, 3, 4], [15, 0, 7, 8]])
+    scales = np.array([[0.5, 0.25], [2.0, 1.0]])
+    zeros = np.array([[1, 8], [0, 7]])
+    X = np.array([[1.0, 1.0, 1.0, 1.0], [1.0, -1.0, 0.0, 2.0]])
+    Y = O.dequant_gemm(X, O.pack_qweight(codes, 4), scales, O.pack_qzeros(zeros, 4), 2, 4, 4, 2, False)
+    np.testing.assert_array_equal(Y, [[14.5, 0.75], [15.5, 5.75]])
+
+
+def test_dequant_gemm_matches_the_column_loops_own_weights():
+    # packed arrays -> Y equals X times the dequantized weights the column loop produced
+    X, W, H, Hd, U = _rand_problem(80, 12, 64, 40, hot=2)
+    r = O.gptq(W, U, 4, 16, False, 16)
+    Y = O.dequant_gemm(X, O.pack_qweight(r.codes, 4), r.scales, O.pack_qzeros(r.zeros, 4), 12, 64, 4, 16, False)
+    np.testing.assert_allclose(Y, X @ r.what.T, rtol=1e-13, atol=1e-15)
