@@ -265,7 +265,9 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    if (e != cudaSuccess) (void)cudaGetLastError();   // a failed launch must not leak into later checks
+    return e;
 }
 
 template <typename... KArgs, typename... Args>
@@ -276,7 +278,9 @@ inline cudaError_t launch_plain(void (*kern)(KArgs...), dim3 grid, dim3 block, s
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    if (e != cudaSuccess) (void)cudaGetLastError();   // a failed launch must not leak into later checks
+    return e;
 }
 
 void set_last_error(const char* fmt, ...);

@@ -23,9 +23,11 @@
 //                as row t of the stage's B tile in the 128-byte-swizzled K-major layout
 //                (the layout TMA would produce), then fences it for the async proxy;
 //   warps 6-13   epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 and one half of
-//                the tile's columns, scales each segment by its group's fp16 scales into
-//                64 fp32 running sums per thread, and at the end of the tile writes Y
-//                through a swizzled staging box with 16-byte stores.
+//                the tile's columns, scales each segment by its group's fp16 scales and
+//                adds it into fp32 running sums kept in TMEM, and after the tile's last
+//                segment writes Y through swizzled staging boxes with 16-byte stores.
+// 448 threads: the register file of each of the SM's four partitions holds four warps
+// of at most 128 registers, which is what the launch bound gives.
 // Every wait is bounded (GPTQ_ERR_TIMEOUT).  No TMA multicast.
 #pragma once
 #include <cuda_bf16.h>
@@ -95,11 +97,12 @@ __device__ __forceinline__ uint4 dq_chunk(const uint32_t* col, int c, int z, __n
 }
 
 template <int BITS>
-__global__ void __maxnreg__(144)   // 448 threads x 144 registers fit one CTA per SM
+__global__ void __launch_bounds__(DQ_THREADS, 1)
     dq_gemm_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mP, const DqArgs p) {
     using Cfg = DqCfg<BITS>;
     constexpr int A_BYTES = Cfg::A_BYTES, B_BYTES = Cfg::B_BYTES, STAGE_BYTES = Cfg::STAGE_BYTES;
-    constexpr uint32_t TMEM_COLS = 2 * DQ_BN;
+    constexpr uint32_t SUM_COL = 2 * DQ_BN;    // running sums after the two segment buffers
+    constexpr uint32_t TMEM_COLS = 512;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -241,19 +244,19 @@ __global__ void __maxnreg__(144)   // 448 threads x 144 registers fit one CTA pe
         for (int w = blockIdx.x; w < total && alive; w += gridDim.x) {
             const int m0 = (w % p.tiles_m) * DQ_BM, n0 = (w / p.tiles_m) * DQ_BN;
             const int nc = n0 + 64 * h;        // first column of this warp
-            float sum[64];
-#pragma unroll
-            for (int j = 0; j < 64; ++j) sum[j] = 0.f;
             for (int sg = 0; sg < nseg; ++sg, ++seg) {
                 const int buf = seg & 1;
                 const bool ok = mbar_wait(&tfull_bar[buf], (uint32_t)(seg >> 1) & 1, w);
                 tc_fence_after();
                 if (ok) {
                     const __half* srow = p.scales + (long long)sg * p.N;
-#pragma unroll
+                    const bool last = sg + 1 == nseg;
+#pragma unroll 1
                     for (int c = 0; c < 2; ++c) {
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(tmem + (uint32_t)(buf * DQ_BN + 64 * h + 32 * c) + lane_off, r);
+                        const uint32_t col = (uint32_t)(64 * h + 32 * c);
+                        uint32_t r[32], t[32];
+                        tmem_ld_32x32b_x32(tmem + (uint32_t)(buf * DQ_BN) + col + lane_off, r);
+                        if (sg > 0) tmem_ld_32x32b_x32(tmem + SUM_COL + col + lane_off, t);
                         tmem_ld_wait();
 #pragma unroll
                         for (int j8 = 0; j8 < 4; ++j8) {
@@ -264,12 +267,24 @@ __global__ void __maxnreg__(144)   // 448 threads x 144 registers fit one CTA pe
 #pragma unroll
                             for (int u = 0; u < 4; ++u) {
                                 const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&sw[u]));
-                                const int j = 32 * c + 8 * j8 + 2 * u;
-                                sum[j] = fmaf(f.x, __uint_as_float(r[j - 32 * c]), sum[j]);
-                                sum[j + 1] = fmaf(f.y, __uint_as_float(r[j + 1 - 32 * c]), sum[j + 1]);
+                                const int j = 8 * j8 + 2 * u;
+                                const float a0 = sg > 0 ? __uint_as_float(t[j]) : 0.f;
+                                const float a1 = sg > 0 ? __uint_as_float(t[j + 1]) : 0.f;
+                                r[j] = __float_as_uint(fmaf(f.x, __uint_as_float(r[j]), a0));
+                                r[j + 1] = __float_as_uint(fmaf(f.y, __uint_as_float(r[j + 1]), a1));
                             }
                         }
+                        if (last) {   // final values straight into this chunk's staging box
+                            uint8_t* b = box + c * kBoxBytes;
+#pragma unroll
+                            for (int c4 = 0; c4 < 8; ++c4)
+                                *reinterpret_cast<uint4*>(b + lane * 128 + ((c4 ^ (lane & 7)) << 4)) =
+                                    make_uint4(r[4 * c4], r[4 * c4 + 1], r[4 * c4 + 2], r[4 * c4 + 3]);
+                        } else {
+                            tmem_st_32x32b_x32(tmem + SUM_COL + col + lane_off, r);
+                        }
                     }
+                    tmem_st_wait();
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -280,16 +295,7 @@ __global__ void __maxnreg__(144)   // 448 threads x 144 registers fit one CTA pe
                 }
             }
             if (!alive) break;
-            // both 32x32 blocks into the staging boxes first (the running sums die here),
-            // then coalesced 16-byte stores clipped to M x N
-            __syncwarp();
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-#pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4)
-                    *reinterpret_cast<float4*>(box + c * kBoxBytes + lane * 128 + ((c4 ^ (lane & 7)) << 4)) =
-                        make_float4(sum[32 * c + 4 * c4], sum[32 * c + 4 * c4 + 1], sum[32 * c + 4 * c4 + 2],
-                                    sum[32 * c + 4 * c4 + 3]);
+            // coalesced 16-byte stores of the two staged 32x32 blocks, clipped to M x N
             __syncwarp();
 #pragma unroll 1
             for (int c = 0; c < 2; ++c) {
@@ -302,6 +308,7 @@ __global__ void __maxnreg__(144)   // 448 threads x 144 registers fit one CTA pe
                     if (gy < p.M && gx < p.N) *reinterpret_cast<float4*>(p.Y + gy * p.N + gx) = val;
                 }
             }
+            __syncwarp();   // the boxes are rewritten by the next tile's last segment
         }
         __syncwarp();
     }
