@@ -37,7 +37,7 @@
 
 namespace gq {
 
-constexpr int DQ_BM = 128, DQ_BN = 128, DQ_BK = 64, DQ_STAGES = 4;
+constexpr int DQ_BM = 128, DQ_BN = 128, DQ_BK = 64;
 constexpr int DQ_THREADS = 448;
 constexpr int DQ_CONV_WARP0 = 2, DQ_EPI_WARP0 = 6;
 
@@ -48,12 +48,13 @@ struct DqCfg {
     static constexpr int B_BYTES = DQ_BN * 128;
     static constexpr int P_BYTES = KWT * DQ_BN * 4;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
+    static constexpr int STAGES = BITS == 8 ? 3 : 4;   // within 227 KB of shared memory
     static_assert(STAGE_BYTES % 1024 == 0, "each stage's tiles stay 1024-byte aligned");
 };
 
 template <int BITS>
 __host__ __device__ constexpr int dq_smem_bytes() {
-    return 1024 + DQ_STAGES * DqCfg<BITS>::STAGE_BYTES + 16 * kBoxBytes + 256;
+    return 1024 + DqCfg<BITS>::STAGES * DqCfg<BITS>::STAGE_BYTES + 16 * kBoxBytes + 8 * 256 + 256;
 }
 
 struct DqArgs {
@@ -101,17 +102,19 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
     dq_gemm_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mP, const DqArgs p) {
     using Cfg = DqCfg<BITS>;
     constexpr int A_BYTES = Cfg::A_BYTES, B_BYTES = Cfg::B_BYTES, STAGE_BYTES = Cfg::STAGE_BYTES;
+    constexpr int STAGES = Cfg::STAGES;
     constexpr uint32_t SUM_COL = 2 * DQ_BN;    // running sums after the two segment buffers
     constexpr uint32_t TMEM_COLS = 512;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    uint8_t* epi = smem + DQ_STAGES * STAGE_BYTES;
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(epi + 16 * kBoxBytes);  // TMA landed
-    uint64_t* conv_bar = full_bar + DQ_STAGES;                                 // B tile written
-    uint64_t* empty_bar = conv_bar + DQ_STAGES;                                // MMAs done
-    uint64_t* tfull_bar = empty_bar + DQ_STAGES;                               // [2] segment ready
+    uint8_t* epi = smem + STAGES * STAGE_BYTES;
+    uint8_t* scale_buf = epi + 16 * kBoxBytes;                                 // [8 warps][2][64] fp16
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(scale_buf + 8 * 256);    // TMA landed
+    uint64_t* conv_bar = full_bar + STAGES;                                 // B tile written
+    uint64_t* empty_bar = conv_bar + STAGES;                                // MMAs done
+    uint64_t* tfull_bar = empty_bar + STAGES;                               // [2] segment ready
     uint64_t* tempty_bar = tfull_bar + 2;                                      // [2] segment drained
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
 
@@ -121,7 +124,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
     const int nseg = nkt / p.kpg;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < DQ_STAGES; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full_bar[s], 1);
             mbar_init(&conv_bar[s], 4);
             mbar_init(&empty_bar[s], 1);
@@ -152,8 +155,8 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             const int m0 = (w % p.tiles_m) * DQ_BM, n0 = (w / p.tiles_m) * DQ_BN;
             for (int kt = 0; kt < nkt; ++kt, ++kiter) {
-                const int s = kiter % DQ_STAGES;
-                const uint32_t it = kiter / DQ_STAGES;
+                const int s = kiter % STAGES;
+                const uint32_t it = kiter / STAGES;
                 if (!mbar_wait(&empty_bar[s], (it & 1) ^ 1, w)) {
                     ok = false;
                     break;
@@ -180,8 +183,8 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
                 tc_fence_after();
                 const uint32_t acc = tmem + (uint32_t)(buf * DQ_BN);
                 for (int kt = 0; kt < p.kpg; ++kt, ++kiter) {
-                    const int s = kiter % DQ_STAGES;
-                    const uint32_t it = kiter / DQ_STAGES;
+                    const int s = kiter % STAGES;
+                    const uint32_t it = kiter / STAGES;
                     if (!mbar_wait(&full_bar[s], it & 1, w) || !mbar_wait(&conv_bar[s], it & 1, w)) {
                         ok = false;
                         break;
@@ -210,8 +213,8 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
             int z = 1 << (BITS - 1);
             __nv_bfloat162 zz = __floats2bfloat162_rn(0.f, 0.f);
             for (int kt = 0; kt < nkt; ++kt, ++kiter) {
-                const int s = kiter % DQ_STAGES;
-                const uint32_t it = kiter / DQ_STAGES;
+                const int s = kiter % STAGES;
+                const uint32_t it = kiter / STAGES;
                 if (kt % p.kpg == 0) {   // a new group: this row's zero point
                     if (p.qzeros != nullptr)
                         z = n < p.N ? (int)stream_code(p.qzeros + (long long)(kt / p.kpg) * zwords, 1, n, BITS) : 0;
@@ -244,12 +247,36 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
         for (int w = blockIdx.x; w < total && alive; w += gridDim.x) {
             const int m0 = (w % p.tiles_m) * DQ_BM, n0 = (w / p.tiles_m) * DQ_BN;
             const int nc = n0 + 64 * h;        // first column of this warp
+            // This warp's 64 scales of a group are fetched into shared memory one segment
+            // ahead (cp.async, eight lanes x 16 bytes), so their L2 latency overlaps the
+            // wait for the segment's accumulator.
+            uint8_t* sbuf = scale_buf + ew * 256;
+            auto prefetch_scales = [&](int sg, int slot) {
+                if (lane < 8) {
+                    const int n = nc + 8 * lane;
+                    const __half* src = p.scales + (long long)sg * p.N + (n < p.N ? n : 0);
+                    const uint32_t bytes = n < p.N ? 16u : 0u;   // zero fill past N
+                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                                     smem_u32(sbuf + slot * 128 + 16 * lane)),
+                                 "l"(src), "r"(bytes)
+                                 : "memory");
+                }
+                asm volatile("cp.async.commit_group;" ::: "memory");
+            };
+            prefetch_scales(0, 0);
             for (int sg = 0; sg < nseg; ++sg, ++seg) {
                 const int buf = seg & 1;
+                if (sg + 1 < nseg) {
+                    prefetch_scales(sg + 1, (sg + 1) & 1);
+                    asm volatile("cp.async.wait_group 1;" ::: "memory");
+                } else {
+                    asm volatile("cp.async.wait_group 0;" ::: "memory");
+                }
+                __syncwarp();
                 const bool ok = mbar_wait(&tfull_bar[buf], (uint32_t)(seg >> 1) & 1, w);
                 tc_fence_after();
                 if (ok) {
-                    const __half* srow = p.scales + (long long)sg * p.N;
+                    const uint8_t* srow = sbuf + (sg & 1) * 128;   // this group's 64 scales
                     const bool last = sg + 1 == nseg;
 #pragma unroll 1
                     for (int c = 0; c < 2; ++c) {
@@ -260,9 +287,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
                         tmem_ld_wait();
 #pragma unroll
                         for (int j8 = 0; j8 < 4; ++j8) {
-                            const int n = nc + 32 * c + 8 * j8;   // N % 8 == 0: eight columns in or out
-                            uint4 sv = make_uint4(0u, 0u, 0u, 0u);
-                            if (n < p.N) sv = __ldg(reinterpret_cast<const uint4*>(srow + n));
+                            const uint4 sv = *reinterpret_cast<const uint4*>(srow + 64 * c + 16 * j8);
                             const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
                             for (int u = 0; u < 4; ++u) {
