@@ -13,21 +13,22 @@
 // sums.  The scale is applied once per group and output, as in the definition, and no
 // rounded copy of W_hat is ever formed.
 //
-// Persistent kernel, one CTA per SM over 128 x 128 output tiles, 448 threads:
+// Persistent kernel, one CTA per SM over 128 x 128 output tiles, 576 threads:
 //   warp 0       TMA: the X tile (128 rows x 64 bf16, 128-byte swizzle) and the packed
 //                words of the weight tile (KWT words x 128 rows, no swizzle) into a ring
 //                of stages;
 //   warp 1       MMA issuer (kind::f16, bf16, M = N = 128, four K = 16 steps per stage);
 //                one accumulator segment per quantization group, two TMEM buffers;
-//   warps 2-5    converters: thread t unpacks weight row n0 + t and writes bf16 (q - z)
-//                as row t of the stage's B tile in the 128-byte-swizzled K-major layout
-//                (the layout TMA would produce), then fences it for the async proxy;
-//   warps 6-13   epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 and one half of
+//   warps 2-9    converters: two threads per weight row n0 + t, each unpacking half of
+//                the row's 64 weights into bf16 (q - z), written as row t of the stage's
+//                B tile in the 128-byte-swizzled K-major layout (the layout TMA would
+//                produce), then fenced for the async proxy;
+//   warps 10-17  epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 and one half of
 //                the tile's columns, scales each segment by its group's fp16 scales and
 //                adds it into fp32 running sums kept in TMEM, and after the tile's last
 //                segment writes Y through swizzled staging boxes with 16-byte stores.
-// 448 threads: the register file of each of the SM's four partitions holds four warps
-// of at most 128 registers, which is what the launch bound gives.
+// 576 threads: each of the SM's four partitions holds up to five warps, so the launch
+// bound caps the registers at 96 per thread (the epilogue keeps its sums in TMEM).
 // Every wait is bounded (GPTQ_ERR_TIMEOUT).  No TMA multicast.
 #pragma once
 #include <cuda_bf16.h>
@@ -38,8 +39,8 @@
 namespace gq {
 
 constexpr int DQ_BM = 128, DQ_BN = 128, DQ_BK = 64;
-constexpr int DQ_THREADS = 448;
-constexpr int DQ_CONV_WARP0 = 2, DQ_EPI_WARP0 = 6;
+constexpr int DQ_THREADS = 576;
+constexpr int DQ_CONV_WARP0 = 2, DQ_EPI_WARP0 = 10;   // eight converter warps, eight epilogue warps
 
 template <int BITS>
 struct DqCfg {
@@ -82,9 +83,22 @@ __device__ __forceinline__ uint4 dq_chunk(const uint32_t* col, int c, int z, __n
             out[i] = *reinterpret_cast<const uint32_t*>(&pa);
             out[2 + i] = *reinterpret_cast<const uint32_t*>(&pb);
         }
+    } else if constexpr (BITS == 4) {
+        // 0x4300 | q is the bf16 of 128 + q (q < 128); subtracting 128 + z is exact.  Byte
+        // permutes put the even and odd nibbles of the word side by side in 16-bit lanes.
+        const uint32_t w = col[c * DQ_BN];
+        const uint32_t even = w & 0x0F0F0F0Fu, odd = (w >> 4) & 0x0F0F0F0Fu;
+        const uint32_t q03 = __byte_perm(even, odd, 0x5140), q47 = __byte_perm(even, odd, 0x7362);
+        const uint32_t v[4] = {__byte_perm(q03, 0x43434343u, 0x4140), __byte_perm(q03, 0x43434343u, 0x4342),
+                               __byte_perm(q47, 0x43434343u, 0x4140), __byte_perm(q47, 0x43434343u, 0x4342)};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 d = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&v[i]), zz);
+            out[i] = *reinterpret_cast<const uint32_t*>(&d);
+        }
     } else {
         // 0x4300 | q is the bf16 of 128 + q (q < 128); subtracting 128 + z is exact.
-        const uint32_t w = (BITS == 4) ? col[c * DQ_BN] : (col[(c >> 1) * DQ_BN] >> ((c & 1) * 16));
+        const uint32_t w = col[(c >> 1) * DQ_BN] >> ((c & 1) * 16);
         constexpr uint32_t M = (1u << BITS) - 1u;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -126,7 +140,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&conv_bar[s], 4);
+            mbar_init(&conv_bar[s], 8);
             mbar_init(&empty_bar[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -203,8 +217,9 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
             }
         }
     } else if (warp >= DQ_CONV_WARP0 && warp < DQ_EPI_WARP0) {
-        // ---------------- converters: thread t owns row t of every B tile
-        const int t = threadIdx.x - 32 * DQ_CONV_WARP0;
+        // ---------------- converters: thread tc owns half (four 16-byte chunks) of row t
+        const int tc = threadIdx.x - 32 * DQ_CONV_WARP0;
+        const int t = tc & (DQ_BN - 1), c0 = 4 * (tc >> 7);
         const long long zwords = ((long long)p.N * BITS + 31) / 32;
         uint32_t kiter = 0;
         bool ok = true;
@@ -228,7 +243,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
                 const uint32_t* col = reinterpret_cast<const uint32_t*>(st + A_BYTES + B_BYTES) + t;
                 uint8_t* row = st + A_BYTES + (t >> 3) * 1024 + (t & 7) * 128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
+                for (int c = c0; c < c0 + 4; ++c)
                     *reinterpret_cast<uint4*>(row + ((c ^ (t & 7)) << 4)) = dq_chunk<BITS>(col, c, z, zz);
                 fence_proxy_async_smem();
                 __syncwarp();
