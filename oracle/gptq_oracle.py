@@ -21,7 +21,8 @@ What it follows (page titles as printed on the pages; section names in quotes):
   - "激活排序（desc_act）": the columns may be visited in an order ranked by
     the sum of absolute input activations instead of their natural order.
 * "GPTQ-2D: 三次时间复杂度的双侧自适应舍入" (ai-feeds summary), "问题背景" and
-  "核心洞察": one-sided GPTQ equals Babai's nearest-plane algorithm.
+  "核心洞察": one-sided GPTQ equals Babai's nearest-plane algorithm; "方法": the
+  two-sided problem and its vectorized (Kronecker Gram) form.
 * "GPTQ/AWQ量化中Group Size的精确含义与计算" (feinterview group-size article),
   opening paragraphs and "存储代价": 4-bit codes 0..15, one scale and one zero per
   group of consecutive weights along the input (reduction) dimension,
@@ -56,6 +57,11 @@ Readings of points the pages leave open (each is implemented below):
   desc_act = 1 follows the text (ascending), desc_act = 2 the name
   (descending); ties keep column order.  Groups are formed in quantization
   order, and a per-column group index maps each column to its group.
+* GPTQ-2D: the objective is ||A (X - Z) B||_F^2 with Gram matrices G_left = A^T A
+  and G_right = B B^T given, Z an integer matrix on the unbounded lattice (no scales,
+  no clamp); the vectorization is column-major, and the one-dimensional GPTQ over it
+  visits coordinates in increasing index, the GPTQ orientation of the rest of this
+  module (first coordinate first).
 """
 
 from __future__ import annotations
@@ -595,3 +601,38 @@ def gptq_act_order(W0: np.ndarray, H: np.ndarray, perm: np.ndarray, bits=4, grou
     what = np.empty_like(res.what)
     what[:, perm] = res.what
     return ActOrderResult(codes, res.scales, res.zeros, g_idx_of(perm, group_size), what, perm, U, lam, res)
+
+
+# ----------------------------------------------------------------------------
+# GPTQ-2D: two-sided adaptive rounding
+# ----------------------------------------------------------------------------
+
+def gptq2d_loss(X: np.ndarray, Z: np.ndarray, G_left: np.ndarray, G_right: np.ndarray) -> float:
+    """tr((X - Z)^T G_left (X - Z) G_right) = ||A (X - Z) B||_F^2 for G_left = A^T A and
+    G_right = B B^T (GPTQ-2D summary, "方法": a real matrix rounded to an integer one under a
+    quadratic metric with fixed nonsingular bases on both sides)."""
+    D = np.asarray(X, dtype=np.float64) - np.asarray(Z, dtype=np.float64)
+    return float(np.trace(D.T @ np.asarray(G_left, dtype=np.float64) @ D @ np.asarray(G_right, dtype=np.float64)))
+
+
+def gptq2d_vectorized(X: np.ndarray, G_left: np.ndarray, G_right: np.ndarray) -> np.ndarray:
+    """Two-sided adaptive rounding by the vectorized route (GPTQ-2D summary, "问题背景",
+    "方法"): the one-dimensional GPTQ run over vec(X).  Tiny sizes only.
+
+    Column-major vectorization (p = i + m j) turns the objective into the quadratic form of
+    the Kronecker Gram G = G_right (x) G_left.  GPTQ visits p = 0, 1, ... with U the upper
+    Cholesky factor of G^-1, formed explicitly as an mn x mn matrix; each coordinate is
+    rounded to the nearest integer (ties to even, no clamp: the unbounded lattice) and
+    its error e_p = (x_p - z_p) / U_pp is pushed forward along row p of U.  This is
+    Babai's nearest plane on that lattice; O((mn)^2) work in the loop, quartic in n.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    m, n = X.shape
+    U = hinv_upper_cholesky(np.kron(np.asarray(G_right, dtype=np.float64), np.asarray(G_left, dtype=np.float64)))
+    x = X.reshape(-1, order="F").copy()
+    z = np.zeros(m * n)
+    for p in range(m * n):
+        z[p] = np.rint(x[p])
+        e = (x[p] - z[p]) / U[p, p]
+        x[p + 1:] -= e * U[p, p + 1:]
+    return z.reshape((m, n), order="F")

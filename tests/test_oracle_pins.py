@@ -490,3 +490,87 @@ def test_dequant_gemm_matches_the_column_loops_own_weights():
     r = O.gptq(W, U, 4, 16, False, 16)
     Y = O.dequant_gemm(X, O.pack_qweight(r.codes, 4), r.scales, O.pack_qzeros(r.zeros, 4), 12, 64, 4, 16, False)
     np.testing.assert_allclose(Y, X @ r.what.T, rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------- GPTQ-2D (two-sided rounding)
+
+def _spd(rng, k, spread=1.0):
+    A = rng.standard_normal((k, k)) * np.exp(spread * rng.standard_normal(k))[None, :]
+    return A.T @ A + 0.1 * np.eye(k), A
+
+
+def _problem2d(seed, m, n):
+    rng = np.random.default_rng(seed)
+    G_left, A = _spd(rng, m)
+    G_right, B = _spd(rng, n)
+    X = rng.standard_normal((m, n)) * 3.0
+    return X, G_left, G_right, A, B
+
+
+@pytest.mark.parametrize("seed", range(90, 94))
+def test_gptq2d_one_sided_case_is_columnwise_gptq(seed):
+    # G_right = I: every column is an independent one-sided GPTQ problem with metric G_left
+    X, G_left, _, _, _ = _problem2d(seed, 6, 5)
+    Z = O.gptq2d_vectorized(X, G_left, np.eye(5))
+    U_left = O.hinv_upper_cholesky(G_left)
+    r = O.gptq(X.T, U_left, 4, -1, False, block_size=0, fixed_grid=(np.ones(5), np.zeros(5)))
+    np.testing.assert_array_equal(Z, r.codes.T)
+
+
+@pytest.mark.parametrize("seed", range(94, 98))
+def test_gptq2d_is_babai_on_the_kronecker_lattice(seed):
+    X, G_left, G_right, _, _ = _problem2d(seed, 4, 3)
+    Z = O.gptq2d_vectorized(X, G_left, G_right)
+    G = np.kron(G_right, G_left)
+    ev, V = np.linalg.eigh(G)
+    basis = V @ np.diag(np.sqrt(ev)) @ V.T          # independent basis with basis^T basis = G
+    z = O.babai_nearest_plane(X.reshape(-1, order="F"), basis)
+    np.testing.assert_array_equal(Z.reshape(-1, order="F"), z)
+
+
+def test_gptq2d_kronecker_factor_structure():
+    # the upper Cholesky factor of (G_right (x) G_left)^-1 is U_right (x) U_left
+    X, G_left, G_right, _, _ = _problem2d(98, 5, 4)
+    U = O.hinv_upper_cholesky(np.kron(G_right, G_left))
+    K = np.kron(O.hinv_upper_cholesky(G_right), O.hinv_upper_cholesky(G_left))
+    np.testing.assert_allclose(U, K, rtol=0, atol=1e-10 * np.abs(K).max())
+
+
+@pytest.mark.parametrize("seed", range(100, 106))
+def test_gptq2d_bruteforce_bracket(seed):
+    # best integer matrix <= two-sided GPTQ <= Babai's bound on the Kronecker lattice
+    X, G_left, G_right, _, _ = _problem2d(seed, 2, 2)
+    Z = O.gptq2d_vectorized(X, G_left, G_right)
+    best = min(O.gptq2d_loss(X, np.array(c, dtype=float).reshape(2, 2), G_left, G_right)
+               for c in itertools.product(*[range(int(np.floor(v)) - 2, int(np.floor(v)) + 4) for v in X.reshape(-1)]))
+    got = O.gptq2d_loss(X, Z, G_left, G_right)
+    bound = O.babai_bound(O.hinv_upper_cholesky(np.kron(G_right, G_left)), 1.0)
+    assert best <= got + 1e-12
+    assert got <= bound + 1e-12
+
+
+def _antidiagonal_rounding(X, U_left, U_right):
+    """The summary's cubic route ("方法" steps 1-3): anti-diagonals i + j = k in increasing k,
+    all entries of one anti-diagonal rounded together from corrections of the entries
+    before it, then their errors pushed forward through the two Cholesky factors.
+    T = E U_right accumulates the errors, so a correction is a length-m dot product."""
+    m, n = X.shape
+    Z = np.zeros((m, n))
+    T = np.zeros((m, n))
+    for k in range(m + n - 1):
+        diag = [(i, k - i) for i in range(max(0, k - n + 1), min(m, k + 1))]
+        vals = [X[i, j] - U_left[:, i] @ T[:, j] for i, j in diag]      # all before any update
+        for (i, j), v in zip(diag, vals):
+            Z[i, j] = np.rint(v)
+            e = (v - Z[i, j]) / (U_left[i, i] * U_right[j, j])
+            T[i, :] += e * U_right[j, :]
+    return Z
+
+
+@pytest.mark.parametrize("seed,m,n", [(110, 5, 7), (111, 8, 3), (112, 6, 6), (113, 1, 9), (114, 9, 1)])
+def test_gptq2d_antidiagonal_route_gives_the_same_integers(seed, m, n):
+    # the summary's claim the cubic route relies on: identical output to the quartic one
+    X, G_left, G_right, _, _ = _problem2d(seed, m, n)
+    Z = O.gptq2d_vectorized(X, G_left, G_right)
+    Zad = _antidiagonal_rounding(X, O.hinv_upper_cholesky(G_left), O.hinv_upper_cholesky(G_right))
+    np.testing.assert_array_equal(Z, Zad)
