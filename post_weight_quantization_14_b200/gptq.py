@@ -197,8 +197,17 @@ def gptq_act_sum_accumulate(X: torch.Tensor, act: torch.Tensor, accumulate: bool
     return act
 
 
+def _need(t: torch.Tensor, dtype: torch.dtype, shape: tuple, name: str) -> None:
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be {dtype} {list(shape)} (got {t.dtype} {list(t.shape)})")
+
+
 def gptq_act_order(act: torch.Tensor, desc_act: int, perm: torch.Tensor, rank: torch.Tensor, stream=None) -> None:
     """perm[k] = column quantized at position k, rank = its inverse (int32 [d_in] each)."""
+    d = act.numel()
+    _need(act, torch.float64, (d,), "act")
+    _need(perm, torch.int32, (d,), "perm")
+    _need(rank, torch.int32, (d,), "rank")
     _check(lib().gptq_act_order(_ptr(act), act.numel(), int(desc_act), _ptr(perm), _ptr(rank), _stream(stream)))
 
 
@@ -206,6 +215,9 @@ def gptq_prepare_hinv_permuted(H: torch.Tensor, perm: torch.Tensor, U: torch.Ten
                                workspace: torch.Tensor | None = None, stream=None) -> float:
     """U of the permuted Hessian H[perm][:, perm]; returns lambda.  Synchronises the stream."""
     d = H.shape[0]
+    _need(H, torch.float32, (d, d), "H")
+    _need(perm, torch.int32, (d,), "perm")
+    _need(U, torch.float32, (d, d), "U")
     need = lib().gptq_prepare_hinv_workspace_bytes(d)
     ws = workspace if workspace is not None else _workspace(need, H.device)
     bad = _i64(-1)
@@ -222,6 +234,9 @@ def gptq_quantize_layer_act_order(W: torch.Tensor, U: torch.Tensor, perm: torch.
                                   workspace: torch.Tensor | None = None, stream=None) -> None:
     """Column loop in the order perm (cfg.desc_act 1 or 2); W is read only; codes in original order."""
     d_out, d_in = W.shape
+    _need(W, torch.float32, (d_out, d_in), "W")
+    _need(perm, torch.int32, (d_in,), "perm")
+    _need(g_idx, torch.int32, (d_in,), "g_idx")
     need = lib().gptq_quantize_workspace_bytes(d_out, d_in, ctypes.byref(cfg))
     ws = workspace if workspace is not None else _workspace(need, W.device)
     _check(lib().gptq_quantize_layer_act_order(_ptr(W), _ptr(U), _ptr(perm), d_out, d_in, ctypes.byref(cfg),
@@ -231,6 +246,8 @@ def gptq_quantize_layer_act_order(W: torch.Tensor, U: torch.Tensor, perm: torch.
 
 def gptq_dequant_g_idx(qweight, scales, qzeros, g_idx, d_out: int, d_in: int, cfg: GptqConfig, W_hat: torch.Tensor,
                        stream=None) -> torch.Tensor:
+    _need(g_idx, torch.int32, (d_in,), "g_idx")
+    _need(W_hat, torch.float32, (d_out, d_in), "W_hat")
     _check(lib().gptq_dequant_g_idx(_ptr(qweight), _ptr(scales), _ptr(qzeros), _ptr(g_idx), d_out, d_in,
                                     ctypes.byref(cfg), _ptr(W_hat), _stream(stream)))
     return W_hat

@@ -164,3 +164,19 @@ def test_dequant_gemm_validates_arguments():
     assert call(G.make_config(3, 128, False)) == G.GPTQ_ERR_UNSUPPORTED   # 3-bit codes straddle words
     assert call(G.make_config(4, 32, False)) == G.GPTQ_ERR_UNSUPPORTED    # groups narrower than a K tile
     assert call(G.make_config(4, 128, False, desc_act=1)) == G.GPTQ_ERR_UNSUPPORTED
+
+
+def test_binding_checks_act_order_tensor_types_before_any_call():
+    import torch
+    d = 64
+    with pytest.raises(ValueError):
+        G.gptq_act_order(torch.zeros(d, dtype=torch.float32), 1, torch.zeros(d, dtype=torch.int32),
+                         torch.zeros(d, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        G.gptq_act_order(torch.zeros(d, dtype=torch.float64), 1, torch.zeros(d, dtype=torch.int64),
+                         torch.zeros(d, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        G.gptq_prepare_hinv_permuted(torch.zeros((d, d)), torch.zeros(d, dtype=torch.int64), torch.zeros((d, d)))
+    with pytest.raises(ValueError):
+        G.gptq_dequant_g_idx(None, None, None, torch.zeros(d, dtype=torch.int64), 8, d, G.make_config(),
+                             torch.zeros((8, d)))
