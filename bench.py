@@ -250,35 +250,53 @@ def run_stack(args) -> None:
         bufs = G.LayerBuffers(ly.d_out, ly.d_in, ly.n, torch.bfloat16, cfg, dev)
         layers.append((ly, W0, torch.empty_like(W0), X, bufs))
     stream = torch.cuda.current_stream()
+    # --shared-input: q, k, v read one input and gate, up another (as in a transformer
+    # block), so each group takes one H and one U; the group's first layer's X is used.
+    groups = [[0, 1, 2], [3], [4, 5], [6]] if args.shared_input else [[i] for i in range(7)]
+    shared = {}
+    if args.shared_input:
+        for grp in groups:
+            if len(grp) > 1:
+                ly0 = layers[grp[0]][0]
+                cfg = G.make_config(ly0.spec.bits, ly0.spec.group_size, ly0.spec.sym, 128, ly0.spec.damp_rel)
+                shared[grp[0]] = G.SharedInputBuffers([layers[i][0].d_out for i in grp], ly0.d_in, ly0.n,
+                                                      torch.bfloat16, cfg, dev)
 
     def step(marks=None):
-        for i, (ly, W0, W, X, bufs) in enumerate(layers):
-            W.copy_(W0)
+        for gi, grp in enumerate(groups):
+            for i in grp:
+                layers[i][2].copy_(layers[i][1])
             if marks:
-                marks[i][0].record(stream)
-            G.quantize_layer(W, X, buffers=bufs)
+                marks[gi][0].record(stream)
+            if len(grp) == 1:
+                ly, W0, W, X, bufs = layers[grp[0]]
+                G.quantize_layer(W, X, buffers=bufs)
+            else:
+                G.quantize_layers_shared_input([layers[i][2] for i in grp], layers[grp[0]][3],
+                                               buffers=shared[grp[0]])
             if marks:
-                marks[i][1].record(stream)
+                marks[gi][1].record(stream)
 
     for _ in range(args.warmup):
         step()
     G.gptq_sync_status()
-    marks = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in layers]
+    marks = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in groups]
              for _ in range(args.steps)]
     torch.cuda.synchronize()
     for m in marks:
         step(m)
     torch.cuda.synchronize()
     G.gptq_sync_status()
-    per_layer = {ly.name.split(".")[-1]: statistics.median(m[i][0].elapsed_time(m[i][1]) for m in marks)
-                 for i, (ly, *_rest) in enumerate(layers)}
+    per_layer = {"+".join(layers[i][0].name.split(".")[-1] for i in grp):
+                 statistics.median(m[gi][0].elapsed_time(m[gi][1]) for m in marks) for gi, grp in enumerate(groups)}
     block_ms = sum(per_layer.values())
     weights = sum(ly.d_out * ly.d_in for ly, *_rest in layers)
     print(json.dumps({"metric": "7B-shaped stack end-to-end quantize time (32 blocks x 7 layers)",
                       "value": 32 * block_ms / 1e3, "unit": "s", "higher_is_better": False, "n_gpus": 1,
                       "steps": args.steps, "warmup": args.warmup, "dtype": "f32", "data": "synthetic",
                       "config": {"workload": "stack7b: one block per step (block 0 seeds), x32 blocks",
-                                 "n": 2048, "bits": 4, "group_size": 128, "sym": False},
+                                 "n": 2048, "bits": 4, "group_size": 128, "sym": False,
+                                 "shared_input": bool(args.shared_input)},
                       "block_ms": block_ms, "layer_ms": per_layer,
                       "weights_per_s": 32 * weights / (32 * block_ms / 1e3)}), flush=True)
 
@@ -389,6 +407,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="attn", choices=["attn", "stack7b", "dqgemm"])
+    ap.add_argument("--shared-input", action="store_true",
+                    help="stack7b: q/k/v and gate/up share one H and U per group (one input each)")
     ap.add_argument("--desc-act", type=int, default=0, choices=[0, 1, 2],
                     help="activation ordering: 0 natural column order, 1 ascending, 2 descending sum of |x|")
     args = ap.parse_args()

@@ -362,3 +362,71 @@ def quantize_layer(W: torch.Tensor, X: torch.Tensor, bits=4, group_size=128, sym
     gptq_quantize_layer_act_order(W, b.U, b.perm, cfg, b.qweight, b.scales, b.qzeros, b.g_idx, b.err_sq,
                                   workspace=b.ws, stream=stream)
     return QuantizedLayer(b.qweight, b.scales, b.qzeros, b.err_sq, lam, b.g_idx, b.perm)
+
+
+class SharedInputBuffers:
+    """Device buffers for several layers that read the same calibration input X (for
+    example the q, k and v projections, or gate and up): one H, one U, one workspace
+    large enough for the widest layer, and per-layer outputs."""
+
+    def __init__(self, d_outs: list[int], d_in: int, n: int, x_dtype: torch.dtype, cfg: GptqConfig, device):
+        xt = GPTQ_BF16 if x_dtype == torch.bfloat16 else GPTQ_F32
+        L = lib()
+        self.cfg = cfg
+        self.d_in = d_in
+        self.H = torch.empty((d_in, d_in), dtype=torch.float32, device=device)
+        self.U = torch.empty((d_in, d_in), dtype=torch.float32, device=device)
+        ws = max([L.gptq_hessian_workspace_bytes(n, d_in, xt), L.gptq_prepare_hinv_workspace_bytes(d_in)] +
+                 [L.gptq_quantize_workspace_bytes(d, d_in, ctypes.byref(cfg)) for d in d_outs])
+        self.ws = _workspace(ws, device)
+        ng = n_groups(d_in, cfg.group_size)
+        self.outs = []
+        for d in d_outs:
+            self.outs.append(dict(
+                qweight=torch.empty(((d_in * cfg.bits + 31) // 32, d), dtype=torch.int32, device=device),
+                scales=torch.empty((ng, d), dtype=torch.float16, device=device),
+                qzeros=None if cfg.sym else torch.empty((ng, (d * cfg.bits + 31) // 32), dtype=torch.int32,
+                                                        device=device),
+                err_sq=torch.empty((d,), dtype=torch.float32, device=device),
+                g_idx=torch.empty((d_in,), dtype=torch.int32, device=device) if cfg.desc_act else None))
+        if cfg.desc_act:
+            self.act = torch.empty((d_in,), dtype=torch.float64, device=device)
+            self.perm = torch.empty((d_in,), dtype=torch.int32, device=device)
+            self.rank = torch.empty((d_in,), dtype=torch.int32, device=device)
+
+
+def quantize_layers_shared_input(Ws: list[torch.Tensor], X: torch.Tensor, bits=4, group_size=128, sym=False,
+                                 damp_rel=0.01, desc_act=0, buffers: SharedInputBuffers | None = None,
+                                 stream=None) -> list[QuantizedLayer]:
+    """GPTQ of several linear layers that share one input: H = 2 X^T X, the activation order
+    (desc_act 1 / 2) and U = chol(Hd^-1) upper are computed once, then one column loop runs
+    per weight.  Each result equals quantize_layer of that weight with the same X.  With
+    desc_act 0 every W is overwritten; with activation ordering they are left unchanged."""
+    if not Ws:
+        return []
+    d_in = Ws[0].shape[1]
+    if any(W.shape[1] != d_in for W in Ws) or X.shape[1] != d_in:
+        raise ValueError("all weights must have d_in columns, X must be [n, d_in]")
+    cfg = buffers.cfg if buffers is not None else make_config(bits, group_size, sym, 128, damp_rel, desc_act)
+    b = buffers or SharedInputBuffers([W.shape[0] for W in Ws], d_in, X.shape[0], X.dtype, cfg, Ws[0].device)
+    if len(b.outs) != len(Ws) or any(o["err_sq"].shape[0] != W.shape[0] for o, W in zip(b.outs, Ws)):
+        raise ValueError("buffers were made for other layer shapes")
+    gptq_hessian_accumulate(X, b.H, accumulate=False, workspace=b.ws, stream=stream)
+    if cfg.desc_act:
+        gptq_act_sum_accumulate(X, b.act, accumulate=False, stream=stream)
+        gptq_act_order(b.act, cfg.desc_act, b.perm, b.rank, stream=stream)
+        lam = gptq_prepare_hinv_permuted(b.H, b.perm, b.U, cfg.damp_rel, workspace=b.ws, stream=stream)
+    else:
+        lam = gptq_prepare_hinv(b.H, b.U, cfg.damp_rel, workspace=b.ws, stream=stream)
+    results = []
+    for W, o in zip(Ws, b.outs):
+        if cfg.desc_act:
+            gptq_quantize_layer_act_order(W, b.U, b.perm, cfg, o["qweight"], o["scales"], o["qzeros"], o["g_idx"],
+                                          o["err_sq"], workspace=b.ws, stream=stream)
+            results.append(QuantizedLayer(o["qweight"], o["scales"], o["qzeros"], o["err_sq"], lam, o["g_idx"],
+                                          b.perm))
+        else:
+            gptq_quantize_layer(W, b.U, cfg, o["qweight"], o["scales"], o["qzeros"], o["err_sq"], workspace=b.ws,
+                                stream=stream)
+            results.append(QuantizedLayer(o["qweight"], o["scales"], o["qzeros"], o["err_sq"], lam))
+    return results
