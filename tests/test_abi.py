@@ -180,3 +180,13 @@ def test_binding_checks_act_order_tensor_types_before_any_call():
     with pytest.raises(ValueError):
         G.gptq_dequant_g_idx(None, None, None, torch.zeros(d, dtype=torch.int64), 8, d, G.make_config(),
                              torch.zeros((8, d)))
+
+
+def test_shared_input_checks_shapes_before_any_call():
+    import torch
+    X = torch.zeros((16, 64))
+    with pytest.raises(ValueError):
+        G.quantize_layers_shared_input([torch.zeros((8, 64)), torch.zeros((8, 32))], X)
+    with pytest.raises(ValueError):
+        G.quantize_layers_shared_input([torch.zeros((8, 64))], torch.zeros((16, 48)))
+    assert G.quantize_layers_shared_input([], X) == []
