@@ -259,7 +259,8 @@ gptq_status gptq_selftest_bounded_wait(uint64_t limit_ns, void* stream);
 
 /* ------------------------------------------------------------------ no-allocation variant
  * gptq_hessian_accumulate_fixed_scratch: the same H (+)= 2 X^T X as
- * gptq_hessian_accumulate, for callers that cannot hand the library a device
+ * gptq_hessian_accumulate (the same kernels and the same segmented accumulation, so the
+ * same bits for the same X), for callers that cannot hand the library a device
  * workspace: a plain C program that links only this library and has no device
  * allocator of its own, or a plug-in running inside a host application whose memory
  * pool owns the whole device and forbids further cudaMalloc calls.  The pages have no
@@ -271,7 +272,8 @@ gptq_status gptq_selftest_bounded_wait(uint64_t limit_ns, void* stream);
  *     with both sizes in gptq_last_error().  Split such a batch and call with
  *     accumulate = 1.
  *   - The first call on each device looks up the array's device address (a set-up the
- *     library does once per device); make that first call before capturing any stream.
+ *     library does once per device, and again if the device's context was destroyed and
+ *     created anew); make that first call before capturing any stream.
  *   - All calls on one device share its array, which keeps the last call's contents.
  *     Calls on one device that may overlap on the GPU (for example on two streams) race
  *     and must be serialised by the caller.  Each call rewrites all of the scratch it

@@ -292,7 +292,8 @@ void timing_end(cudaStream_t st);
 struct TimedScope {
     cudaStream_t st;
     bool on;
-    TimedScope(const char* name, cudaStream_t s) : st(s), on(timing_on()) {
+    // name == nullptr: not timed (callers that must not allocate host memory)
+    TimedScope(const char* name, cudaStream_t s) : st(s), on(name != nullptr && timing_on()) {
         if (on) timing_begin(name, st);
     }
     ~TimedScope() {
@@ -313,5 +314,9 @@ bool make_tmap_2d_plain(CUtensorMap* map, const void* base, uint64_t rows, uint6
 
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device, size).
 cudaError_t ensure_smem_attr(const void* func, int bytes);
+
+// make_tmap_2d without the host-side map cache (allocates no host memory).
+bool make_tmap_2d_uncached(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
+                           uint64_t ld, uint32_t box_rows, uint32_t box_cols);
 
 }  // namespace gqh

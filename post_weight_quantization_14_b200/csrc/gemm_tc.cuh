@@ -625,12 +625,13 @@ struct EpiMats {
         t_lo{nullptr, 0, 0, 0};
 };
 
-inline bool make_out_map(CUtensorMap* map, const Mat& m, const CUtensorMap& fallback) {
+inline bool make_out_map(CUtensorMap* map, const Mat& m, const CUtensorMap& fallback, bool no_alloc = false) {
     if (!m.ptr) {
         *map = fallback;
         return true;
     }
-    return make_tmap_2d(map, m.ptr, 4, m.rows, m.cols, m.ld, 32, 32);
+    return no_alloc ? make_tmap_2d_uncached(map, m.ptr, 4, m.rows, m.cols, m.ld, 32, 32)
+                    : make_tmap_2d(map, m.ptr, 4, m.rows, m.cols, m.ld, 32, 32);
 }
 
 // Multiprocessor count of the current device (cached per device).
@@ -645,24 +646,30 @@ inline bool epilogue_fits(const gq::GemmArgs& p) { return p.beta == 0.f || p.wri
 // Launch D = A B^T with the given epilogue.  For the tf32 kinds a2/b2 are the lo parts.
 // max_ctas > 0 caps the persistent grid (to leave SMs to a concurrent kernel).  after_event:
 // the launch follows a cross-stream event wait, so it is not a programmatic dependent.
+// no_alloc: no host-side bookkeeping that allocates (tensor maps encoded afresh, the
+// shared-memory attribute set directly, no per-launch timing).
 template <int KIND, int STAGES, int TBN = gq::BN, int SEG = 0>
 cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2, const EpiMats& o, gq::GemmArgs p,
                         int batch, cudaStream_t stream, const char* name, int max_ctas = 0,
-                        bool after_event = false) {
+                        bool after_event = false, bool no_alloc = false) {
     using Cfg = gq::GemmCfg<KIND, TBN>;
     const int eb = (KIND == gq::KIND_BF16) ? 2 : 4;
     CUtensorMap ma, ma2, mb, mb2, mc;
+    auto tmap = [no_alloc](CUtensorMap* m, const Mat& x, int elb, uint32_t br, uint32_t bc) {
+        return no_alloc ? make_tmap_2d_uncached(m, x.ptr, elb, x.rows, x.cols, x.ld, br, bc)
+                        : make_tmap_2d(m, x.ptr, elb, x.rows, x.cols, x.ld, br, bc);
+    };
     if (p.mirror && TBN != gq::BM) return cudaErrorInvalidValue;   // mirrored outputs: square tiles only
-    if (!make_tmap_2d(&ma, a.ptr, eb, a.rows, a.cols, a.ld, gq::BM, Cfg::KT)) return cudaErrorInvalidValue;
-    if (!make_tmap_2d(&mb, b.ptr, eb, b.rows, b.cols, b.ld, TBN, Cfg::KT)) return cudaErrorInvalidValue;
+    if (!tmap(&ma, a, eb, gq::BM, Cfg::KT)) return cudaErrorInvalidValue;
+    if (!tmap(&mb, b, eb, TBN, Cfg::KT)) return cudaErrorInvalidValue;
     if (KIND != gq::KIND_BF16) {
-        if (!make_tmap_2d(&ma2, a2.ptr, eb, a2.rows, a2.cols, a2.ld, gq::BM, Cfg::KT)) return cudaErrorInvalidValue;
-        if (!make_tmap_2d(&mb2, b2.ptr, eb, b2.rows, b2.cols, b2.ld, TBN, Cfg::KT)) return cudaErrorInvalidValue;
+        if (!tmap(&ma2, a2, eb, gq::BM, Cfg::KT)) return cudaErrorInvalidValue;
+        if (!tmap(&mb2, b2, eb, TBN, Cfg::KT)) return cudaErrorInvalidValue;
     } else {
         ma2 = ma;
         mb2 = mb;
     }
-    if (!make_out_map(&mc, o.c, ma)) return cudaErrorInvalidValue;
+    if (!make_out_map(&mc, o.c, ma, no_alloc)) return cudaErrorInvalidValue;
     p.C = static_cast<float*>(const_cast<void*>(o.c.ptr));
     p.ldc = (long long)o.c.ld;
     p.c_rows = (long long)o.c.rows;
@@ -686,11 +693,12 @@ cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2
     if (tiles <= 0) return cudaSuccess;
     constexpr int smem = gq::gemm_smem_bytes<KIND, STAGES, TBN>();
     auto kern = gq::tc_gemm_kernel<KIND, STAGES, TBN, SEG>;
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem);
+    cudaError_t e = no_alloc ? cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+                             : ensure_smem_attr(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)std::min<long long>(tiles, max_ctas > 0 ? max_ctas : num_sms());
     {
-        TimedScope ts__(name, stream);
+        TimedScope ts__(no_alloc ? nullptr : name, stream);
         e = after_event ? launch_plain(kern, dim3(grid), dim3(192), (size_t)smem, stream, ma, ma2, mb, mb2, mc, p)
                         : launch_pdl(kern, dim3(grid), dim3(192), (size_t)smem, stream, ma, ma2, mb, mb2, mc, p);
     }

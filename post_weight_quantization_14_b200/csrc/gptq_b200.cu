@@ -94,6 +94,11 @@ bool make_tmap_2d_plain(CUtensorMap* map, const void* base, uint64_t rows, uint6
     return encode_tmap_2d(map, base, 4, rows, cols, ld, box_rows, box_cols, false);
 }
 
+bool make_tmap_2d_uncached(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
+                           uint64_t ld, uint32_t box_rows, uint32_t box_cols) {
+    return encode_tmap_2d(map, base, elem_bytes, rows, cols, ld, box_rows, box_cols);
+}
+
 bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows, uint64_t cols,
                   uint64_t ld, uint32_t box_rows, uint32_t box_cols) {
     const TmapKey key{reinterpret_cast<uintptr_t>(base), elem_bytes, rows, cols, ld, box_rows, box_cols};
@@ -581,37 +586,39 @@ __device__ __align__(256) uint8_t g_fixed_hess_scratch[kFixedHessScratchBytes];
 namespace gqh {
 
 constexpr int kMaxDevices = 128;
-static void* g_fixed_hess_scratch_addr[kMaxDevices];  // zero-initialised; one slot per device ordinal
+// Device address of the fixed scratch, looked up once per (device, context): a context that
+// was torn down and created again (cudaDeviceReset) may load the module elsewhere.
+struct FixedScratchSlot {
+    void* ctx;
+    void* addr;
+};
+static FixedScratchSlot g_fixed_scratch_slots[kMaxDevices];   // zero-initialised; one slot per device ordinal
 
-// One GEMM launch with freshly encoded maps (no map cache, no timing bookkeeping).
-template <int KIND, int STAGES>
-static cudaError_t fixed_gemm(const Mat& a, const Mat& a2, const Mat& c, gq::GemmArgs p, cudaStream_t st) {
-    using Cfg = gq::GemmCfg<KIND>;
-    const int eb = (KIND == gq::KIND_BF16) ? 2 : 4;
-    CUtensorMap ma, ma2, mc;
-    if (!encode_tmap_2d(&ma, a.ptr, eb, a.rows, a.cols, a.ld, gq::BM, Cfg::KT)) return cudaErrorInvalidValue;
-    if (!encode_tmap_2d(&ma2, a2.ptr, eb, a2.rows, a2.cols, a2.ld, gq::BM, Cfg::KT)) return cudaErrorInvalidValue;
-    if (!encode_tmap_2d(&mc, c.ptr, 4, c.rows, c.cols, c.ld, 32, 32)) return cudaErrorInvalidValue;
-    p.C = static_cast<float*>(const_cast<void*>(c.ptr));
-    p.ldc = (long long)c.ld;
-    p.c_rows = (long long)c.rows;
-    p.c_cols = (long long)c.cols;
-    p.tiles_m = (p.M + gq::BM - 1) / gq::BM;
-    p.tiles_n = (p.N + gq::BN - 1) / gq::BN;
-    p.batch = 1;
-    p.tri_r = 1;
-    const long long tiles = (long long)p.tiles_m * (p.tiles_m + 1) / 2;
-    constexpr int smem = gq::gemm_smem_bytes<KIND, STAGES, gq::BN>();
-    auto kern = gq::tc_gemm_kernel<KIND, STAGES, gq::BN, 0>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    int sms = 0;
-    int dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-    // A and B are the same matrix (X^T); the epilogue writes C and its mirror
-    kern<<<dim3((unsigned)std::min<long long>(tiles, sms), 1, 1), 192, smem, st>>>(ma, ma2, ma, ma2, mc, p);
-    return cudaGetLastError();
+using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
+static PfnCtxGetCurrent g_ctx_get_current = nullptr;
+
+static cudaError_t fixed_scratch_address(int dev, void** out) {
+    if (!g_ctx_get_current) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return cudaErrorUnknown;
+        g_ctx_get_current = reinterpret_cast<PfnCtxGetCurrent>(fn);
+    }
+    CUcontext ctx = nullptr;   // stays NULL before the runtime has used this device
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
+    FixedScratchSlot& slot = g_fixed_scratch_slots[dev];
+    if (slot.addr == nullptr || ctx == nullptr || slot.ctx != (void*)ctx) {
+        void* addr = nullptr;   // the lookup also initialises the device's primary context
+        const cudaError_t e = cudaGetSymbolAddress(&addr, gq::g_fixed_hess_scratch);
+        if (e != cudaSuccess) return e;
+        if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorUnknown;
+        slot.ctx = (void*)ctx;
+        slot.addr = addr;
+    }
+    *out = slot.addr;
+    return cudaSuccess;
 }
 
 }  // namespace gqh
@@ -635,39 +642,10 @@ gptq_status gptq_hessian_accumulate_fixed_scratch(const void* X, gptq_dtype xt, 
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices) return fail(GPTQ_ERR_INVALID_ARG, "device ordinal %d out of range", dev);
-    if (!g_fixed_hess_scratch_addr[dev]) {
-        void* addr = nullptr;
-        e = cudaGetSymbolAddress(&addr, gq::g_fixed_hess_scratch);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(fixed scratch)");
-        g_fixed_hess_scratch_addr[dev] = addr;
-    }
-    void* ws = g_fixed_hess_scratch_addr[dev];
-    cudaStream_t st = (cudaStream_t)stream;
-    const long long np = hess_npad(n);
-    dim3 tb(32, 8), grid((unsigned)(np / 32), (unsigned)((d_in + 31) / 32));
-    gq::GemmArgs p = gemm_args((int)d_in, (int)d_in, (int)np);
-    p.triangular = 1;
-    p.mirror = 1;
-    p.alpha = 2.f;
-    p.beta = accumulate ? 1.f : 0.f;
-    p.write_c = 1;
-    const Mat hm{H, (uint64_t)d_in, (uint64_t)d_in, (uint64_t)d_in};
-    if (xt == GPTQ_BF16) {
-        uint16_t* XT = static_cast<uint16_t*>(ws);
-        gq::transpose_bf16_kernel<<<grid, tb, 0, st>>>(static_cast<const uint16_t*>(X), n, d_in, np, XT);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "fixed-scratch transpose");
-        const Mat m{XT, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
-        e = fixed_gemm<gq::KIND_BF16, 4>(m, m, hm, p, st);
-    } else {
-        float* hi = static_cast<float*>(ws);
-        float* lo = hi + d_in * np;
-        gq::transpose_split_f32_kernel<<<grid, tb, 0, st>>>(static_cast<const float*>(X), n, d_in, np, hi, lo);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "fixed-scratch transpose");
-        const Mat mh{hi, (uint64_t)d_in, (uint64_t)np, (uint64_t)np}, ml{lo, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
-        e = fixed_gemm<gq::KIND_TF32X3, 2>(mh, ml, hm, p, st);
-    }
+    void* ws = nullptr;
+    e = fixed_scratch_address(dev, &ws);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(fixed scratch)");
+    e = hessian_run(X, xt, n, d_in, H, accumulate ? 1 : 0, ws, (cudaStream_t)stream, true);
     if (e != cudaSuccess) return cuda_fail(e, "fixed-scratch hessian");
     return GPTQ_OK;
 }

@@ -58,8 +58,13 @@ inline size_t hessian_ws_bytes(long long n, long long d_in, gptq_dtype xt) {
     return xt == GPTQ_BF16 ? (size_t)(d_in * np * 2) : (size_t)(2 * d_in * np * 4);
 }
 
+// Both Hessian entry points run this: the workspace one (no_alloc = false) and the
+// fixed-scratch one (no_alloc = true: ws is the library's static scratch array, and no
+// host-side bookkeeping that allocates is used), so they launch the same kernels with the
+// same segmented accumulation.
 inline cudaError_t hessian_run(const void* X, gptq_dtype xt, long long n, long long d_in, float* H,
-                               int accumulate, void* ws, cudaStream_t st) {
+                               int accumulate, void* ws, cudaStream_t st, bool no_alloc = false) {
+    const char* tname = no_alloc ? nullptr : "transpose_x";
     const long long np = hess_npad(n);
     dim3 tb(32, 8);
     dim3 grid((unsigned)(np / 32), (unsigned)((d_in + 31) / 32));
@@ -74,25 +79,26 @@ inline cudaError_t hessian_run(const void* X, gptq_dtype xt, long long n, long l
     if (xt == GPTQ_BF16) {
         uint16_t* XT = static_cast<uint16_t*>(ws);
         {
-            gqh::TimedScope ts__("transpose_x", st);
+            gqh::TimedScope ts__(tname, st);
             gq::transpose_bf16_kernel<<<grid, tb, 0, st>>>(static_cast<const uint16_t*>(X), n, d_in, np, XT);
         }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         Mat m{XT, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
-        return launch_gemm<gq::KIND_BF16, 4, 128, 16>(m, m, m, m, o, p, 1, st, "hessian_syrk");
+        return launch_gemm<gq::KIND_BF16, 4, 128, 16>(m, m, m, m, o, p, 1, st, "hessian_syrk", 0, false, no_alloc);
     }
     float* hi = static_cast<float*>(ws);
     float* lo = hi + d_in * np;
     {
-        gqh::TimedScope ts__("transpose_x", st);
+        gqh::TimedScope ts__(tname, st);
         gq::transpose_split_f32_kernel<<<grid, tb, 0, st>>>(static_cast<const float*>(X), n, d_in, np, hi, lo);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     Mat mh{hi, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
     Mat ml{lo, (uint64_t)d_in, (uint64_t)np, (uint64_t)np};
-    return launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(mh, ml, mh, ml, o, p, 1, st, "hessian_syrk");
+    return launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(mh, ml, mh, ml, o, p, 1, st, "hessian_syrk", 0, false,
+                                                   no_alloc);
 }
 
 }  // namespace gqh

@@ -140,9 +140,46 @@ def _workspace(nbytes: int, device) -> torch.Tensor:
 
 # ---------------------------------------------------------------------------- stage wrappers
 
+_WORD = (torch.int32, torch.uint32)   # packed 32-bit words: either signedness
+
+
+def _need(t: torch.Tensor, dtype, shape: tuple, name: str, flat_ok: bool = False) -> None:
+    """Shape and dtype check before any pointer reaches the library (the C side sees only
+    addresses and sizes, so a mismatch here would be an out-of-range access on the device).
+    dtype may be a tuple of accepted dtypes; flat_ok also accepts a 1-D tensor of the
+    same number of elements."""
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a torch.Tensor")
+    dtypes = dtype if isinstance(dtype, tuple) else (dtype,)
+    numel = 1
+    for x in shape:
+        numel *= int(x)
+    shape_ok = tuple(t.shape) == tuple(shape) or (flat_ok and t.dim() == 1 and t.numel() == numel)
+    if t.dtype not in dtypes or not shape_ok:
+        raise ValueError(f"{name} must be {dtypes[0]} {list(shape)} (got {t.dtype} {list(t.shape)})")
+
+
+def _quant_outputs(cfg: GptqConfig, d_out: int, d_in: int, qweight, scales, qzeros, err_sq) -> None:
+    """Shapes and dtypes of the column loop's output arrays (layouts of include/gptq_b200.h)."""
+    ng = n_groups(d_in, cfg.group_size)
+    _need(qweight, _WORD, ((d_in * cfg.bits + 31) // 32, d_out), "qweight")
+    _need(scales, torch.float16, (ng, d_out), "scales")
+    if cfg.sym:
+        if qzeros is not None:
+            raise ValueError("qzeros must be None for symmetric quantization")
+    else:
+        if qzeros is None:
+            raise ValueError("qzeros is required for asymmetric quantization")
+        _need(qzeros, _WORD, (ng, (d_out * cfg.bits + 31) // 32), "qzeros")
+    if err_sq is not None:
+        _need(err_sq, torch.float32, (d_out,), "err_sq")
+
+
 def gptq_hessian_accumulate(X: torch.Tensor, H: torch.Tensor, accumulate: bool = False,
                             workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """H (+)= 2 X^T X.  X: [n, d_in] bfloat16 or float32 on the device; H: [d_in, d_in] float32."""
+    if X.dim() != 2:
+        raise ValueError("X must be a [n, d_in] matrix")
     n, d_in = X.shape
     if X.dtype == torch.bfloat16:
         xt = GPTQ_BF16
@@ -162,7 +199,11 @@ def gptq_hessian_accumulate(X: torch.Tensor, H: torch.Tensor, accumulate: bool =
 def gptq_prepare_hinv(H: torch.Tensor, U: torch.Tensor, damp_rel: float = 0.01,
                       workspace: torch.Tensor | None = None, stream=None) -> float:
     """U = upper Cholesky factor of (H + lambda I)^-1; returns lambda.  Synchronises the stream."""
+    if H.dim() != 2:
+        raise ValueError("H must be a square float32 matrix")
     d = H.shape[0]
+    _need(H, torch.float32, (d, d), "H")
+    _need(U, torch.float32, (d, d), "U")
     need = lib().gptq_prepare_hinv_workspace_bytes(d)
     ws = workspace if workspace is not None else _workspace(need, H.device)
     bad = _i64(-1)
@@ -177,7 +218,12 @@ def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, cfg: GptqConfig, qweig
                         scales: torch.Tensor, qzeros: torch.Tensor | None, err_sq: torch.Tensor | None = None,
                         workspace: torch.Tensor | None = None, stream=None) -> None:
     """Column loop; W is consumed as scratch.  scales is a float16 tensor [n_groups, d_out]."""
+    if W.dim() != 2:
+        raise ValueError("W must be a float32 [d_out, d_in] matrix")
     d_out, d_in = W.shape
+    _need(W, torch.float32, (d_out, d_in), "W")
+    _need(U, torch.float32, (d_in, d_in), "U")
+    _quant_outputs(cfg, d_out, d_in, qweight, scales, qzeros, err_sq)
     need = lib().gptq_quantize_workspace_bytes(d_out, d_in, ctypes.byref(cfg))
     ws = workspace if workspace is not None else _workspace(need, W.device)
     _check(lib().gptq_quantize_layer(_ptr(W), _ptr(U), d_out, d_in, ctypes.byref(cfg), _ptr(qweight),
@@ -195,11 +241,6 @@ def gptq_act_sum_accumulate(X: torch.Tensor, act: torch.Tensor, accumulate: bool
         raise ValueError("act must be float64 [d_in]")
     _check(lib().gptq_act_sum_accumulate(_ptr(X), xt, n, d_in, _ptr(act), int(bool(accumulate)), _stream(stream)))
     return act
-
-
-def _need(t: torch.Tensor, dtype: torch.dtype, shape: tuple, name: str) -> None:
-    if t.dtype != dtype or tuple(t.shape) != tuple(shape):
-        raise ValueError(f"{name} must be {dtype} {list(shape)} (got {t.dtype} {list(t.shape)})")
 
 
 def gptq_act_order(act: torch.Tensor, desc_act: int, perm: torch.Tensor, rank: torch.Tensor, stream=None) -> None:
@@ -233,10 +274,14 @@ def gptq_quantize_layer_act_order(W: torch.Tensor, U: torch.Tensor, perm: torch.
                                   g_idx: torch.Tensor, err_sq: torch.Tensor | None = None,
                                   workspace: torch.Tensor | None = None, stream=None) -> None:
     """Column loop in the order perm (cfg.desc_act 1 or 2); W is read only; codes in original order."""
+    if W.dim() != 2:
+        raise ValueError("W must be a float32 [d_out, d_in] matrix")
     d_out, d_in = W.shape
     _need(W, torch.float32, (d_out, d_in), "W")
+    _need(U, torch.float32, (d_in, d_in), "U")
     _need(perm, torch.int32, (d_in,), "perm")
     _need(g_idx, torch.int32, (d_in,), "g_idx")
+    _quant_outputs(cfg, d_out, d_in, qweight, scales, qzeros, err_sq)
     need = lib().gptq_quantize_workspace_bytes(d_out, d_in, ctypes.byref(cfg))
     ws = workspace if workspace is not None else _workspace(need, W.device)
     _check(lib().gptq_quantize_layer_act_order(_ptr(W), _ptr(U), _ptr(perm), d_out, d_in, ctypes.byref(cfg),
@@ -246,6 +291,7 @@ def gptq_quantize_layer_act_order(W: torch.Tensor, U: torch.Tensor, perm: torch.
 
 def gptq_dequant_g_idx(qweight, scales, qzeros, g_idx, d_out: int, d_in: int, cfg: GptqConfig, W_hat: torch.Tensor,
                        stream=None) -> torch.Tensor:
+    _quant_outputs(cfg, d_out, d_in, qweight, scales, qzeros, None)
     _need(g_idx, torch.int32, (d_in,), "g_idx")
     _need(W_hat, torch.float32, (d_out, d_in), "W_hat")
     _check(lib().gptq_dequant_g_idx(_ptr(qweight), _ptr(scales), _ptr(qzeros), _ptr(g_idx), d_out, d_in,
@@ -260,19 +306,28 @@ def gptq_dequant_gemm(X: torch.Tensor, qweight, scales, qzeros, d_out: int, d_in
         raise ValueError("X must be bfloat16 [M, d_in]")
     if Y.dtype != torch.float32 or tuple(Y.shape) != (X.shape[0], d_out):
         raise ValueError("Y must be float32 [M, d_out]")
+    _quant_outputs(cfg, d_out, d_in, qweight, scales, qzeros, None)
     _check(lib().gptq_dequant_gemm(_ptr(X), X.shape[0], _ptr(qweight), _ptr(scales), _ptr(qzeros), d_out, d_in,
                                    ctypes.byref(cfg), _ptr(Y), _stream(stream)))
     return Y
 
 
 def gptq_pack_int(codes: torch.Tensor, bits: int, layout: int, packed: torch.Tensor, stream=None) -> torch.Tensor:
+    """codes uint8 [rows, cols] -> packed int32 ([rows, nwords] for layout 0, [nwords, rows] for 1)."""
+    if codes.dim() != 2:
+        raise ValueError("codes must be a uint8 [rows, cols] matrix")
     rows, cols = codes.shape
+    nw = (cols * int(bits) + 31) // 32
+    _need(codes, torch.uint8, (rows, cols), "codes")
+    _need(packed, _WORD, (rows, nw) if layout == 0 else (nw, rows), "packed", flat_ok=True)
     _check(lib().gptq_pack_int(_ptr(codes), rows, cols, int(bits), int(layout), _ptr(packed), _stream(stream)))
     return packed
 
 
 def gptq_dequant(qweight, scales, qzeros, d_out: int, d_in: int, cfg: GptqConfig, W_hat: torch.Tensor,
                  stream=None) -> torch.Tensor:
+    _quant_outputs(cfg, d_out, d_in, qweight, scales, qzeros, None)
+    _need(W_hat, torch.float32, (d_out, d_in), "W_hat")
     _check(lib().gptq_dequant(_ptr(qweight), _ptr(scales), _ptr(qzeros), d_out, d_in, ctypes.byref(cfg),
                               _ptr(W_hat), _stream(stream)))
     return W_hat
@@ -303,6 +358,29 @@ def gptq_selftest_bounded_wait(limit_ns: int, stream=None) -> None:
 
 def n_groups(d_in: int, group_size: int) -> int:
     return 1 if group_size == -1 else (d_in + group_size - 1) // group_size
+
+
+def _resolve_config(buffers, bits, group_size, sym, damp_rel, desc_act) -> GptqConfig:
+    """The configuration of a whole-layer call.  Without buffers the arguments give it (None
+    means the default: 4 bits, group 128, asymmetric, damp 0.01, natural order).  With
+    buffers the buffers' configuration is used, and an argument given explicitly that
+    disagrees with it is an error rather than silently ignored."""
+    given = dict(bits=bits, group_size=group_size, sym=sym, damp_rel=damp_rel, desc_act=desc_act)
+    if buffers is None:
+        d = dict(bits=4, group_size=128, sym=False, damp_rel=0.01, desc_act=0)
+        d.update({k: v for k, v in given.items() if v is not None})
+        return make_config(d["bits"], d["group_size"], d["sym"], 128, d["damp_rel"], d["desc_act"])
+    cfg = buffers.cfg
+    have = dict(bits=cfg.bits, group_size=cfg.group_size, sym=bool(cfg.sym), damp_rel=cfg.damp_rel,
+                desc_act=cfg.desc_act)
+    for k, v in given.items():
+        if v is None:
+            continue
+        same = abs(float(v) - have[k]) <= 1e-7 * max(1.0, abs(have[k])) if k == "damp_rel" else \
+            (bool(v) == have[k] if k == "sym" else int(v) == have[k])
+        if not same:
+            raise ValueError(f"{k}={v!r} conflicts with the buffers' configuration ({k}={have[k]!r})")
+    return cfg
 
 
 @dataclass
@@ -341,14 +419,18 @@ class LayerBuffers:
             self.g_idx = torch.empty((d_in,), dtype=torch.int32, device=device)
 
 
-def quantize_layer(W: torch.Tensor, X: torch.Tensor, bits=4, group_size=128, sym=False, damp_rel=0.01,
-                   desc_act=0, buffers: LayerBuffers | None = None, stream=None) -> QuantizedLayer:
+def quantize_layer(W: torch.Tensor, X: torch.Tensor, bits=None, group_size=None, sym=None, damp_rel=None,
+                   desc_act=None, buffers: LayerBuffers | None = None, stream=None) -> QuantizedLayer:
     """GPTQ of one linear layer: H = 2 X^T X, U = chol(Hd^-1) upper, column loop.
 
     desc_act 0: natural column order, W is overwritten.  desc_act 1 / 2: columns in
     ascending / descending order of sum_t |X[t, c]|; W is left unchanged and the result
-    carries g_idx and perm."""
-    cfg = buffers.cfg if buffers is not None else make_config(bits, group_size, sym, 128, damp_rel, desc_act)
+    carries g_idx and perm.
+
+    With ``buffers`` the configuration is the buffers' own (an explicit argument that
+    disagrees raises ValueError), and the returned tensors ARE the buffers' arrays: they
+    stay valid only until the next call with the same buffers, which overwrites them."""
+    cfg = _resolve_config(buffers, bits, group_size, sym, damp_rel, desc_act)
     d_out, d_in = W.shape
     b = buffers or LayerBuffers(d_out, d_in, X.shape[0], X.dtype, cfg, W.device)
     gptq_hessian_accumulate(X, b.H, accumulate=False, workspace=b.ws, stream=stream)
@@ -395,19 +477,24 @@ class SharedInputBuffers:
             self.rank = torch.empty((d_in,), dtype=torch.int32, device=device)
 
 
-def quantize_layers_shared_input(Ws: list[torch.Tensor], X: torch.Tensor, bits=4, group_size=128, sym=False,
-                                 damp_rel=0.01, desc_act=0, buffers: SharedInputBuffers | None = None,
+def quantize_layers_shared_input(Ws: list[torch.Tensor], X: torch.Tensor, bits=None, group_size=None, sym=None,
+                                 damp_rel=None, desc_act=None, buffers: SharedInputBuffers | None = None,
                                  stream=None) -> list[QuantizedLayer]:
     """GPTQ of several linear layers that share one input: H = 2 X^T X, the activation order
     (desc_act 1 / 2) and U = chol(Hd^-1) upper are computed once, then one column loop runs
     per weight.  Each result equals quantize_layer of that weight with the same X.  With
-    desc_act 0 every W is overwritten; with activation ordering they are left unchanged."""
+    desc_act 0 every W is overwritten; with activation ordering they are left unchanged.
+
+    With ``buffers`` the configuration is the buffers' own (an explicit argument that
+    disagrees raises ValueError), and the returned tensors ARE the buffers' arrays
+    (buffers.outs, buffers.perm): they stay valid only until the next call with the same
+    buffers, which overwrites them."""
     if not Ws:
         return []
     d_in = Ws[0].shape[1]
     if any(W.shape[1] != d_in for W in Ws) or X.shape[1] != d_in:
         raise ValueError("all weights must have d_in columns, X must be [n, d_in]")
-    cfg = buffers.cfg if buffers is not None else make_config(bits, group_size, sym, 128, damp_rel, desc_act)
+    cfg = _resolve_config(buffers, bits, group_size, sym, damp_rel, desc_act)
     b = buffers or SharedInputBuffers([W.shape[0] for W in Ws], d_in, X.shape[0], X.dtype, cfg, Ws[0].device)
     if len(b.outs) != len(Ws) or any(o["err_sq"].shape[0] != W.shape[0] for o, W in zip(b.outs, Ws)):
         raise ValueError("buffers were made for other layer shapes")

@@ -190,3 +190,57 @@ def test_shared_input_checks_shapes_before_any_call():
     with pytest.raises(ValueError):
         G.quantize_layers_shared_input([torch.zeros((8, 64))], torch.zeros((16, 48)))
     assert G.quantize_layers_shared_input([], X) == []
+
+
+def test_stage_wrappers_check_dtypes_and_shapes_before_any_call():
+    """A wrong dtype or size must be refused in the binding: the C side sees only pointers
+    and sizes, so it would read or write out of range on the device."""
+    import torch
+    d_out, d_in = 64, 128
+    cfg = G.make_config(4, 128, False)
+    qw = torch.zeros(((d_in * 4 + 31) // 32, d_out), dtype=torch.int32)
+    sc = torch.zeros((1, d_out), dtype=torch.float16)
+    qz = torch.zeros((1, (d_out * 4 + 31) // 32), dtype=torch.int32)
+    es = torch.zeros((d_out,), dtype=torch.float32)
+    W = torch.zeros((d_out, d_in), dtype=torch.float32)
+    U = torch.zeros((d_in, d_in), dtype=torch.float32)
+    bad = [
+        (W.to(torch.bfloat16), U, qw, sc, qz, es),                      # bf16 W
+        (W.half(), U, qw, sc, qz, es),                                  # fp16 W
+        (W, torch.zeros((d_in - 8, d_in - 8)), qw, sc, qz, es),         # U of the wrong size
+        (W, U.double(), qw, sc, qz, es),                                # fp64 U
+        (W, U, qw[:-1], sc, qz, es),                                    # qweight too short
+        (W, U, qw, sc.float(), qz, es),                                 # fp32 scales
+        (W, U, qw, sc, None, es),                                       # asymmetric without qzeros
+        (W, U, qw, sc, qz, torch.zeros((d_out - 1,))),                  # err_sq too short
+    ]
+    for args in bad:
+        with pytest.raises(ValueError):
+            G.gptq_quantize_layer(args[0], args[1], cfg, *args[2:])
+    with pytest.raises(ValueError):
+        G.gptq_prepare_hinv(torch.zeros((d_in, d_in)), torch.zeros((d_in, d_in - 8)))
+    with pytest.raises(ValueError):
+        G.gptq_prepare_hinv(torch.zeros((d_in, d_in), dtype=torch.float64), torch.zeros((d_in, d_in)))
+    with pytest.raises(ValueError):
+        G.gptq_dequant(qw, sc, qz, d_out, d_in, cfg, torch.zeros((d_out, d_in), dtype=torch.float16))
+    with pytest.raises(ValueError):
+        G.gptq_pack_int(torch.zeros((4, 8), dtype=torch.int32), 4, 0, torch.zeros((4, 1), dtype=torch.int32))
+    with pytest.raises(ValueError):
+        G.gptq_pack_int(torch.zeros((4, 8), dtype=torch.uint8), 4, 0, torch.zeros((4, 2), dtype=torch.int32))
+
+
+def test_whole_layer_calls_refuse_arguments_that_conflict_with_the_buffers():
+    from types import SimpleNamespace
+    cfg = G.make_config(3, 64, True, 128, 0.02)
+    bufs = SimpleNamespace(cfg=cfg)
+    assert G._resolve_config(bufs, None, None, None, None, None) is cfg
+    assert G._resolve_config(bufs, 3, 64, True, 0.02, 0) is cfg
+    for kw in (dict(bits=4), dict(group_size=128), dict(sym=False), dict(damp_rel=0.01), dict(desc_act=1)):
+        args = dict(bits=None, group_size=None, sym=None, damp_rel=None, desc_act=None)
+        args.update(kw)
+        with pytest.raises(ValueError):
+            G._resolve_config(bufs, **args)
+    d = G._resolve_config(None, None, None, None, None, None)
+    assert (d.bits, d.group_size, d.sym, d.desc_act) == (4, 128, 0, 0)
+    e = G._resolve_config(None, 2, 32, None, None, 2)
+    assert (e.bits, e.group_size, e.sym, e.desc_act) == (2, 32, 0, 2)

@@ -574,3 +574,105 @@ def test_gptq2d_antidiagonal_route_gives_the_same_integers(seed, m, n):
     Z = O.gptq2d_vectorized(X, G_left, G_right)
     Zad = _antidiagonal_rounding(X, O.hinv_upper_cholesky(G_left), O.hinv_upper_cholesky(G_right))
     np.testing.assert_array_equal(Z, Zad)
+
+
+# ---------------------------------------------------------------- replay protocol: scale and zero decisions
+#
+# The group-size article fixes the metadata of a group: a 16-bit scale and a b-bit zero
+# point ("存储代价").  The replay adopts the other side's scale or zero only when the
+# oracle's own unrounded quantity lies within tol (weight units) of that decision's
+# rounding tie.  These pins build groups whose distance to the tie is known exactly, so a
+# distance measured in the wrong units (grid units, raw-scale units) or against the wrong
+# point (the other value instead of the tie) fails one of them.
+
+def _f16_neighbours(s0: float) -> tuple[float, float]:
+    a = np.float16(s0)
+    return float(a), float(np.nextafter(a, np.float16(np.inf)))
+
+
+def _one_group_replay(v, other_scale, other_zero, bits, tol):
+    """Replay a single row holding one group (no compensation: U = I)."""
+    W = np.asarray(v, dtype=np.float64)[None, :]
+    g = W.shape[1]
+    maxq = (1 << bits) - 1
+    codes = np.clip(np.rint(W / other_scale) + other_zero, 0, maxq).astype(np.int64)
+    scales = np.array([[other_scale]])
+    zeros = np.array([[other_zero]], dtype=np.int64)
+    return O.gptq_replay(W, np.eye(g), codes, scales, zeros, bits, g, False, g, tol=tol)
+
+
+@pytest.mark.parametrize("delta", [1e-6, -1e-6, 3e-7])
+def test_replay_scale_tie_distance_is_the_range_distance_in_weight_units(delta):
+    bits, maxq = 4, 15
+    s0, s1 = _f16_neighbours(0.0068359375)          # two adjacent fp16 scales
+    mid = 0.5 * (s0 + s1)                            # the fp16 rounding tie of raw = range / maxq
+    hi = maxq * mid + delta                          # asymmetric, all values >= 0: lo = 0, range = hi
+    rng = np.random.default_rng(7)
+    v = np.concatenate([[hi], rng.uniform(0.0, hi, 31)])
+    own = s1 if delta > 0 else s0                    # what the oracle rounds to
+    other = s0 if delta > 0 else s1                  # the other side's neighbouring fp16 scale
+    assert float(O.fp16_round(hi / maxq)) == own
+    loose = _one_group_replay(v, other, 0, bits, tol=2.0 * abs(delta))
+    assert loose.forced_params == 1 and loose.hard_params == 0
+    strict = _one_group_replay(v, other, 0, bits, tol=0.5 * abs(delta))
+    assert strict.hard_params == 1 and strict.forced_params == 0
+
+
+@pytest.mark.parametrize("k,eps", [(7, 1e-6), (3, -1e-6), (12, 4e-7)])
+def test_replay_zero_tie_distance_is_in_weight_units(k, eps):
+    bits, maxq = 4, 15
+    s = float(np.float16(0.0068359375))
+    lo = -(k + 0.5) * s - eps                        # -lo / s = k + 1/2 + eps / s
+    hi = lo + maxq * s                               # range = maxq * s exactly: raw rounds to s
+    rng = np.random.default_rng(k)
+    v = np.concatenate([[lo, hi], rng.uniform(lo, hi, 30)])
+    _, z, _, _, _ = O.group_params(v[None, :], bits, False)
+    own = k + 1 if eps > 0 else k
+    assert int(z[0]) == own
+    other = k if eps > 0 else k + 1
+    loose = _one_group_replay(v, s, other, bits, tol=2.0 * abs(eps))
+    assert loose.forced_params == 1 and loose.hard_params == 0
+    strict = _one_group_replay(v, s, other, bits, tol=0.5 * abs(eps))
+    assert strict.hard_params == 1 and strict.forced_params == 0
+
+
+def _far_from_tie_problem():
+    _, W, _, _, U = _rand_problem(62, 8, 128, 150)
+    a = O.gptq(W, U, 4, 32, False, 128)
+    return W, U, a
+
+
+def test_replay_flags_a_scale_one_fp16_ulp_off_far_from_its_tie():
+    W, U, a = _far_from_tie_problem()
+    # the group (of row 0) whose range lies farthest from both neighbouring fp16 ties
+    best, best_d = None, -1.0
+    for gi in range(a.scales.shape[0]):
+        v = a.pre[0:1, 32 * gi:32 * gi + 32]
+        s, _, raw, lo, hi = O.group_params(v, 4, False)
+        lo_n = float(np.nextafter(np.float16(s[0]), np.float16(0)))
+        hi_n = float(np.nextafter(np.float16(s[0]), np.float16(np.inf)))
+        d = min(abs(raw[0] - 0.5 * (s[0] + lo_n)), abs(raw[0] - 0.5 * (s[0] + hi_n))) * 15
+        if d > best_d:
+            best, best_d = gi, d
+    assert best_d > 1e-5
+    sc = a.scales.copy()
+    sc[best, 0] = float(np.nextafter(np.float16(sc[best, 0]), np.float16(np.inf)))
+    rr = O.gptq_replay(W, U, a.codes, sc, a.zeros, 4, 32, False, 128)
+    assert rr.hard_params >= 1
+
+
+def test_replay_flags_a_zero_point_off_by_one_far_from_its_tie():
+    W, U, a = _far_from_tie_problem()
+    best, best_d = None, -1.0
+    for gi in range(a.scales.shape[0]):
+        v = a.pre[0:1, 32 * gi:32 * gi + 32]
+        s, z, _, lo, _ = O.group_params(v, 4, False)
+        x = -lo[0] / s[0]
+        d = abs(x - (np.floor(x) + 0.5)) * s[0]      # weight-unit distance to the nearest tie
+        if 0 < z[0] < 15 and d > best_d:
+            best, best_d = gi, d
+    assert best is not None and best_d > 1e-5
+    zz = a.zeros.copy()
+    zz[best, 0] += 1
+    rr = O.gptq_replay(W, U, a.codes, a.scales, zz, 4, 32, False, 128)
+    assert rr.hard_params >= 1
