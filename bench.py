@@ -98,8 +98,10 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- CPU oracle leg
 
-def oracle_layer_time(layer, rows_sample: int = 256) -> tuple[float, str, int]:
-    """Seconds per layer of the fp64 oracle: H and U in full, column loop on a row sample, extrapolated."""
+def oracle_layer_time(layer) -> tuple[float, str, int]:
+    """Seconds for the fp64 oracle to quantize the whole layer: H = 2 X^T X, U = chol(Hd^-1)
+    (explicit inverse, then Cholesky) and the lazy-block column loop over every row.
+    Measured, not extrapolated."""
     import numpy as np
 
     from oracle import gptq_oracle as O
@@ -111,13 +113,20 @@ def oracle_layer_time(layer, rows_sample: int = 256) -> tuple[float, str, int]:
     Hd, _ = O.damp(H, 0.01)
     U = O.hinv_upper_cholesky(Hd)
     t2 = time.perf_counter()
-    rows = min(rows_sample, layer.d_out)
-    O.gptq(layer.W[:rows], U, BITS, GROUP, SYM, 128)
+    O.gptq(layer.W, U, BITS, GROUP, SYM, 128)
     t3 = time.perf_counter()
-    total = (t1 - t0) + (t2 - t1) + (t3 - t2) * (layer.d_out / rows)
-    sample = (f"H=2X^T X and U=chol(Hd^-1) in full (fp64 numpy/LAPACK), column loop on {rows} of "
-              f"{layer.d_out} rows extrapolated to the layer; H {t1 - t0:.2f}s U {t2 - t1:.2f}s rows {t3 - t2:.2f}s")
-    return total, sample, len(os.sched_getaffinity(0))
+    sample = (f"the whole {layer.d_out}x{layer.d_in} layer, measured: H=2X^T X, U=chol(Hd^-1) and the column loop "
+              f"over all {layer.d_out} rows (fp64 numpy/LAPACK); H {t1 - t0:.2f}s U {t2 - t1:.2f}s "
+              f"column loop {t3 - t2:.2f}s")
+    return t3 - t0, sample, len(os.sched_getaffinity(0))
+
+
+def bench_config(world: int, desc_act: int) -> dict:
+    """The workload description both arms print (the same dict in each)."""
+    return {"workload": WORKLOAD, "d_out": D_OUT, "d_in": D_IN, "n": N_TOK, "bits": BITS, "group_size": GROUP,
+            "sym": SYM, "damp_rel": 0.01, "desc_act": desc_act,
+            "l2": "flushed (256 MB write) before every step, outside the step events",
+            "parallelism": f"{world} independent layers, one per GPU"}
 
 
 def max_over_ranks(ms: float, dist, device) -> float:
@@ -141,6 +150,8 @@ def layer_seed(rank: int) -> int:
 
 
 def run_reference(args, rank: int, world: int) -> None:
+    """The reference arm: the fp64 CPU oracle, as it stands, on the machine's host cores; every
+    step quantizes the whole layer.  Under torchrun only rank 0 runs it."""
     if rank != 0:
         return
     from post_weight_quantization_14_b200 import inputs as I
@@ -149,19 +160,50 @@ def run_reference(args, rank: int, world: int) -> None:
     for _ in range(args.warmup):
         oracle_layer_time(layer)
     secs = []
+    sample, cores = "", 0
     for _ in range(args.steps):
-        s, sample, cores = oracle_layer_time(layer)
-        secs.append(s)
+        s_, sample, cores = oracle_layer_time(layer)
+        secs.append(s_)
     ms = 1e3 * sum(secs) / len(secs)
     value = D_OUT * D_IN / (ms / 1e3)
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "d_out": D_OUT, "d_in": D_IN, "n": N_TOK, "bits": BITS,
-                       "group_size": GROUP, "sym": SYM},
+            "config": bench_config(world, args.desc_act),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
-            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "step_s": secs}
     print(json.dumps(line), flush=True)
+
+
+def relaunch_command(argv: list[str], n: int, port: int) -> list[str]:
+    """bench.py --gpus N started without torchrun: the same command as N ranks, one per GPU."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + list(argv)
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s_:
+        s_.bind(("127.0.0.1", 0))
+        return s_.getsockname()[1]
+
+
+def rank_probe(world: int, rank: int) -> None:
+    """--rank-probe: every rank joins a gloo group and reports its rank (a check of the
+    launch plumbing that needs no GPU)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    t = torch.tensor([float(rank)])
+    dist.all_reduce(t)
+    if rank == 0:
+        print(json.dumps({"rank_probe": True, "world": dist.get_world_size(), "rank_sum": float(t.item())}),
+              flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
 
 
 # ---------------------------------------------------------------- GPU leg
@@ -180,7 +222,37 @@ TRAFFIC_PER_LAUNCH = {"chol_leaf": 142592, "colloop": 2239232, "hessian_syrk": 1
 END_TO_END_BOUND_MS = 0.445
 
 
-def kernel_rooflines(kernel_ms: dict, launches: dict, hbm: float, bf16: float, peak_kind: str) -> dict:
+def measure_tf32_tflops(dev) -> float | None:
+    """Dense TF32 tensor-core throughput of this GPU, measured the way the bf16 peak is: a
+    cuBLAS fp32 GEMM with TF32 allowed, 8192^3 (2 N^3 flops), best of 5, CUDA events."""
+    import torch
+    prev = torch.backends.cuda.matmul.allow_tf32
+    try:
+        torch.backends.cuda.matmul.allow_tf32 = True
+        n = 8192
+        a = torch.randn((n, n), device=dev, dtype=torch.float32)
+        b = torch.randn((n, n), device=dev, dtype=torch.float32)
+        for _ in range(2):
+            torch.matmul(a, b)
+        best = None
+        for _ in range(5):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch.matmul(a, b)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        del a, b
+        return 2.0 * n ** 3 / (best / 1e3) / 1e12
+    except Exception:
+        return None
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
+
+
+def kernel_rooflines(kernel_ms: dict, launches: dict, hbm: float, bf16: float, peak_kind: str,
+                     tf32: float | None = None) -> dict:
     """Achieved vs peak per kernel class, from algorithmic work and measured per-step time.
 
     Algorithmic work:
@@ -193,7 +265,8 @@ def kernel_rooflines(kernel_ms: dict, launches: dict, hbm: float, bf16: float, p
     """
     B = 128
     d_out, d_in, n = D_OUT, D_IN, N_TOK
-    tf32x3 = bf16 * (1.1 / 2.25) / 3.0
+    tf32x3 = (tf32 if tf32 else bf16 * (1.1 / 2.25)) / 3.0
+    tf32_kind = "cuBLAS TF32 measured in this run" if tf32 else f"{peak_kind} bf16 x 1.1/2.25"
     sm_fp32 = 128 * 2 * 1.965e9 / 1e12            # one SM, TFLOP/s at max clock
     out = {}
     def add(name, bound, work, unit, peak, note):
@@ -212,7 +285,7 @@ def kernel_rooflines(kernel_ms: dict, launches: dict, hbm: float, bf16: float, p
                                   "frac": ach / tf32x3, "traffic": None,
                                   "launches": launches.get("trailing_update", 0) + launches.get("trailing_update_sb", 0),
                                   "note": f"all trailing updates (per block and per superblock, {tr_ms:.3f} ms); "
-                                          f"3xTF32 ({peak_kind} bf16 x 1.1/2.25 / 3)"}
+                                          f"3xTF32 ({tf32_kind} / 3)"}
     add("hessian_syrk", "tensor", 1.0 * n * d_in * (d_in + 1), "TFLOP/s", bf16, f"bf16 {peak_kind} burst")
     col_bytes = 4.0 * d_out * d_in + BITS / 8 * d_out * d_in + (2 + BITS / 8) * d_out * (d_in // GROUP)
     add("colloop", "hbm", col_bytes, "GB/s", hbm, f"HBM {peak_kind}; latency chain of d_in rounding steps per row")
@@ -227,7 +300,7 @@ def kernel_rooflines(kernel_ms: dict, launches: dict, hbm: float, bf16: float, p
             if k in kernel_ms:
                 out[k] = {"bound": "tensor", "achieved": ach, "peak": tf32x3, "unit": "TFLOP/s", "frac": ach / tf32x3,
                           "traffic": None, "launches": launches.get(k),
-                          "note": f"factorization GEMMs together ({gemm_ms:.3f} ms) vs 3xTF32"}
+                          "note": f"factorization GEMMs together ({gemm_ms:.3f} ms) vs 3xTF32 ({tf32_kind} / 3)"}
     return out
 
 
@@ -411,21 +484,38 @@ def main():
                     help="stack7b: q/k/v and gate/up share one H and U per group (one input each)")
     ap.add_argument("--desc-act", type=int, default=0, choices=[0, 1, 2],
                     help="activation ordering: 0 natural column order, 1 ascending, 2 descending sum of |x|")
+    ap.add_argument("--rank-probe", action="store_true",
+                    help="launch check only: the ranks join a gloo group and rank 0 reports the world size")
     args = ap.parse_args()
+
+    world_env = os.environ.get("WORLD_SIZE")
+    if args.gpus > 1 and world_env is None:
+        # started without torchrun: become N ranks, one per GPU, and return their status
+        cmd = relaunch_command(sys.argv[1:], args.gpus, free_port())
+        env = dict(os.environ, MASTER_ADDR="127.0.0.1")
+        sys.exit(subprocess.call(cmd, env=env))
+    world = int(world_env or "1")
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        sys.stderr.write(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}\n")
+        sys.exit(2)
+    if args.rank_probe:
+        rank_probe(world, rank)
+        return
     if args.workload == "stack7b":
         run_stack(args)
         return
     if args.workload == "dqgemm":
         run_dqgemm(args)
         return
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
+    run_gpu(args, world, rank, local)
 
+
+def run_gpu(args, world: int, rank: int, local: int) -> None:
     import numpy as np
     import torch
 
@@ -519,7 +609,8 @@ def main():
     kernel_launches = {k: c // reps for k, (c, ms) in kt.items()}
 
     hbm, bf16, bf16_sus, peak_kind = peaks()
-    roof_all = kernel_rooflines(kernel_ms, kernel_launches, hbm, bf16, peak_kind)
+    tf32 = measure_tf32_tflops(dev)
+    roof_all = kernel_rooflines(kernel_ms, kernel_launches, hbm, bf16, peak_kind, tf32)
     stage_ms = {"hessian": kernel_ms.get("hessian_syrk", 0) + kernel_ms.get("transpose_x", 0)
                 + sum(kernel_ms.get(k, 0) for k in ACT_KERNELS),
                 "prepare_hinv": sum(v for k, v in kernel_ms.items() if k in CHOL_KERNELS),
@@ -530,35 +621,80 @@ def main():
     roofline["kernel"] = dom
     roofline["share_of_step"] = kernel_ms[dom] / max(1e-9, sum(kernel_ms.values()))
 
-    # end-to-end through the public API with host buffers (pinned), copies inside the timed region
+    # end-to-end through the public API with host buffers (pinned), copies inside the timed region.
+    # Layers are pipelined: layer i+1's inputs go up on one copy stream and layer i-1's outputs
+    # come down on another while layer i computes; two sets of device buffers alternate, and
+    # events order every reuse (inputs after the compute that read them, outputs after the
+    # copy that read them).
     W_host = torch.from_numpy(layer.W).pin_memory()
     X_host = torch.from_numpy(layer.X_bits.view(np.int16)).pin_memory()
-    qw_host = torch.empty(bufs.qweight.shape, dtype=torch.int32).pin_memory()
-    sc_host = torch.empty(bufs.scales.shape, dtype=torch.float16).pin_memory()
-    qz_host = torch.empty(bufs.qzeros.shape, dtype=torch.int32).pin_memory()
-    Xd = torch.empty(X_host.shape, dtype=torch.int16, device=dev)
-    gi_host = torch.empty((D_IN,), dtype=torch.int32).pin_memory()
+    slots = []
+    for _ in range(2):
+        b_ = G.LayerBuffers(D_OUT, D_IN, N_TOK, torch.bfloat16, cfg, dev)
+        slots.append(dict(
+            bufs=b_, W=torch.empty_like(W0), X=torch.empty(X_host.shape, dtype=torch.int16, device=dev),
+            qw=torch.empty(b_.qweight.shape, dtype=torch.int32).pin_memory(),
+            sc=torch.empty(b_.scales.shape, dtype=torch.float16).pin_memory(),
+            qz=torch.empty(b_.qzeros.shape, dtype=torch.int32).pin_memory(),
+            gi=torch.empty((D_IN,), dtype=torch.int32).pin_memory(),
+            ev_in=torch.cuda.Event(), ev_done=torch.cuda.Event(), ev_out=torch.cuda.Event()))
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     e2e_steps = max(3, min(args.steps, 30))
+
+    def h2d(sl, after=None):
+        with torch.cuda.stream(up):
+            if after is not None:
+                up.wait_event(after)
+            sl["W"].copy_(W_host, non_blocking=True)
+            sl["X"].copy_(X_host, non_blocking=True)
+            sl["ev_in"].record(up)
+
+    def e2e_run(nsteps):
+        h2d(slots[0])
+        pending_out = [False, False]
+        for i_ in range(nsteps):
+            sl = slots[i_ % 2]
+            if i_ + 1 < nsteps:   # next layer's inputs, once the layer that last read that slot is done
+                nxt = slots[(i_ + 1) % 2]
+                h2d(nxt, nxt["ev_done"] if i_ >= 1 else None)
+            stream.wait_event(sl["ev_in"])
+            if pending_out[i_ % 2]:
+                stream.wait_event(sl["ev_out"])   # that slot's previous outputs have been copied out
+            q = G.quantize_layer(sl["W"], sl["X"].view(torch.bfloat16), buffers=sl["bufs"])
+            sl["ev_done"].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(sl["ev_done"])
+                sl["qw"].copy_(q.qweight, non_blocking=True)
+                sl["sc"].copy_(q.scales, non_blocking=True)
+                sl["qz"].copy_(q.qzeros, non_blocking=True)
+                if cfg.desc_act:
+                    sl["gi"].copy_(q.g_idx, non_blocking=True)
+                sl["ev_out"].record(down)
+            pending_out[i_ % 2] = True
+        for sl in slots:
+            stream.wait_event(sl["ev_out"])
+
+    e2e_run(2)   # warm the second set of buffers and the copy streams
+    torch.cuda.synchronize()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ea.record(stream)
-    for _ in range(e2e_steps):
-        W.copy_(W_host, non_blocking=True)
-        Xd.copy_(X_host, non_blocking=True)
-        q = G.quantize_layer(W, Xd.view(torch.bfloat16), buffers=bufs)
-        qw_host.copy_(q.qweight, non_blocking=True)
-        if cfg.desc_act:
-            gi_host.copy_(q.g_idx, non_blocking=True)
-        sc_host.copy_(q.scales, non_blocking=True)
-        qz_host.copy_(q.qzeros, non_blocking=True)
+    up.wait_event(ea)
+    e2e_run(e2e_steps)
     eb.record(stream)
     torch.cuda.synchronize()
+    G.gptq_sync_status()
     e2e_ms = max_over_ranks(ea.elapsed_time(eb), dist, dev)
     e2e_value = job_throughput(world, D_OUT * D_IN, e2e_steps, e2e_ms)
-    h2d = W_host.numel() * 4 + X_host.numel() * 2
-    d2h = qw_host.numel() * 4 + sc_host.numel() * 2 + qz_host.numel() * 4 + (D_IN * 4 if cfg.desc_act else 0)
+    h2d_bytes = W_host.numel() * 4 + X_host.numel() * 2
+    d2h_bytes = (slots[0]["qw"].numel() * 4 + slots[0]["sc"].numel() * 2 + slots[0]["qz"].numel() * 4
+                 + (D_IN * 4 if cfg.desc_act else 0))
+    # the last layer's outputs as they reached the host equal the device-timed path's
+    last = slots[(e2e_steps - 1) % 2]
+    e2e_outputs_match = bool(torch.equal(last["qw"], bufs.qweight.cpu()) and torch.equal(last["sc"], bufs.scales.cpu())
+                             and torch.equal(last["qz"], bufs.qzeros.cpu()))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -569,20 +705,21 @@ def main():
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                "config": {"workload": WORKLOAD, "d_out": D_OUT, "d_in": D_IN, "n": N_TOK, "bits": BITS,
-                           "group_size": GROUP, "sym": SYM, "damp_rel": 0.01, "desc_act": args.desc_act,
-                           "l2": "flushed (256 MB write) before every step, outside the step events",
-                           "parallelism": f"{world} independent layers, one per GPU"},
+                "config": bench_config(world, args.desc_act),
                 "roofline": roofline,
                 "roofline_by_kernel": roof_all,
+                "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16, "kind": peak_kind, "tf32_tflops_measured": tf32,
+                          "tf32x3_tflops": (tf32 / 3.0) if tf32 else None},
                 "e2e_roofline": {"bound_ms": END_TO_END_BOUND_MS, "frac": END_TO_END_BOUND_MS / ms_per_step},
                 "stage_ms": stage_timed,
                 "stage_ms_instrumented": stage_ms,
                 "kernel_ms_per_step": kernel_ms,
                 "kernel_launches_per_step": kernel_launches,
                 "cpu_baseline": cpu,
-                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                        "steps": e2e_steps},
+                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
+                        "d2h_bytes_per_step": d2h_bytes, "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
+                        "pipelined": "layer i+1 H2D and layer i-1 D2H on two copy streams beside layer i",
+                        "outputs_match_device_path": e2e_outputs_match},
                 "gpu_launches": int(round(launches_per_step * args.steps)),
                 "clocks": clocks,
                 "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms)}
