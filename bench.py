@@ -208,7 +208,8 @@ def rank_probe(world: int, rank: int) -> None:
 
 # ---------------------------------------------------------------- GPU leg
 
-CHOL_KERNELS = ("chol_leaf", "chol_panel", "chol_update", "chol_update_next", "chol_update_u2", "inv_bu", "inv_ub",
+CHOL_KERNELS = ("chol_leaf", "chol_panel", "chol_chain_r", "chol_chain_d", "chol_update", "chol_update_next",
+                "chol_update_u2", "inv_bu", "inv_ub",
                 "split_panel",
                 "damp_copy", "diag_mean", "zero_lower", "chol_diag_out", "perm_invert", "damp_copy_perm")
 QUANT_KERNELS = ("colloop", "trailing_update", "trailing_update_sb", "up_prep", "ut_split", "pack_zeros", "row_params",
@@ -292,7 +293,8 @@ def kernel_rooflines(kernel_ms: dict, launches: dict, hbm: float, bf16: float, p
     nleaf = d_in // B
     add("chol_leaf", "alu", nleaf * 2.0 * (2.0 / 3.0) * B ** 3, "TFLOP/s", sm_fp32,
         "one CTA per 128x128 leaf: peak = one SM's fp32 FMA rate at 1965 MHz")
-    fact = ("chol_panel", "chol_update", "chol_update_next", "chol_update_u2", "inv_bu", "inv_ub")
+    fact = ("chol_panel", "chol_chain_r", "chol_chain_d", "chol_update", "chol_update_next", "chol_update_u2",
+            "inv_bu", "inv_ub")
     gemm_ms = sum(kernel_ms.get(k, 0) for k in fact)
     if gemm_ms:
         ach = (2.0 / 3.0) * d_in ** 3 / (gemm_ms / 1e3) / 1e12

@@ -239,6 +239,26 @@ gptq_status gptq_dequant_gemm(const void* X, int64_t M, const int32_t* qweight, 
                               const int32_t* qzeros, int64_t d_out, int64_t d_in, const gptq_config* cfg, float* Y,
                               void* stream);
 
+/* ------------------------------------------------------------------ two-sided rounding
+ * GPTQ-2D (GPTQ-2D summary, "方法" steps 1-3 and "核心洞察"): round a real matrix X
+ * (m x n) to an integer matrix Z minimising tr((X - Z)^T G_left (X - Z) G_right), given the
+ * upper Cholesky factors U_left of G_left^-1 (m x m) and U_right of G_right^-1 (n x n)
+ * (for example from gptq_prepare_hinv with damp_rel = 0, or any other source).  The
+ * entries are taken anti-diagonal by anti-diagonal (i + j = 0, 1, ...); the entries of one
+ * anti-diagonal depend only on earlier ones and are rounded in parallel; each error is
+ * pushed forward through both factors.  The integers equal those of one-sided GPTQ run
+ * over the column-major vectorisation with the Kronecker Gram G_right (x) G_left.
+ *   X        device fp64, batch problems of m x n row-major, problem b at X + b m n.
+ *   U_left, U_right  device fp64 row-major, upper triangular, shared by the batch.
+ *   Z        device int32, same layout as X; round half to even, no clamp.
+ *   ws       device workspace of at least gptq_2d_workspace_bytes(m, n, batch) bytes.
+ * All arithmetic in fp64.  A non-finite value or |Z| >= 2^31 is reported by the next
+ * gptq_sync_status() (GPTQ_ERR_NONFINITE) and that entry is written as 0.
+ * Requires 1 <= m, n <= 16384; 8-byte aligned X, U_left, U_right, ws; 4-byte aligned Z. */
+size_t gptq_2d_workspace_bytes(int64_t m, int64_t n, int64_t batch);
+gptq_status gptq_2d_round(const double* X, int64_t m, int64_t n, int64_t batch, const double* U_left,
+                          const double* U_right, int32_t* Z, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronise ``stream`` and return (and clear) the device status word. */
 gptq_status gptq_sync_status(void* stream);
 

@@ -636,3 +636,35 @@ def gptq2d_vectorized(X: np.ndarray, G_left: np.ndarray, G_right: np.ndarray) ->
         e = (x[p] - z[p]) / U[p, p]
         x[p + 1:] -= e * U[p, p + 1:]
     return z.reshape((m, n), order="F")
+
+
+def gptq2d_antidiagonal(X: np.ndarray, U_left: np.ndarray, U_right: np.ndarray) -> np.ndarray:
+    """Two-sided adaptive rounding by the anti-diagonal route (GPTQ-2D summary, "方法",
+    steps 1-3): the entries of X are taken anti-diagonal by anti-diagonal, i + j = k for
+    k = 0, 1, ..., m + n - 2; every entry of one anti-diagonal is rounded from the errors of
+    the entries before that anti-diagonal (they do not depend on one another), and its error
+    is then pushed forward through the Cholesky factors of both sides.
+
+    U_left (m x m) and U_right (n x n) are the upper Cholesky factors of G_left^-1 and
+    G_right^-1.  Kept for row i: T[i, :] = sum of e_ij U_right[j, :] over the entries (i, j)
+    rounded so far, so the correction of entry (i, j) is the dot product of column i of
+    U_left with column j of T.  Rounding is to the nearest integer, ties to even, no clamp.
+    O(m n (m + n)) work; equal in exact arithmetic to gptq2d_vectorized (the errors of
+    entry (i', j') reach (i, j) only when i' <= i and j' <= j, and both routes visit such
+    entries first).
+    """
+    X = np.asarray(X, dtype=np.float64)
+    UL = np.asarray(U_left, dtype=np.float64)
+    UR = np.asarray(U_right, dtype=np.float64)
+    m, n = X.shape
+    Z = np.zeros((m, n))
+    T = np.zeros((m, n))
+    for k in range(m + n - 1):
+        cells = [(i, k - i) for i in range(max(0, k - n + 1), min(m, k + 1))]
+        vals = [X[i, j] - UL[:i + 1, i] @ T[:i + 1, j] for i, j in cells]   # all before any update
+        for (i, j), v in zip(cells, vals):
+            Z[i, j] = np.rint(v)
+            e = (v - Z[i, j]) / (UL[i, i] * UR[j, j])
+            T[i, j:] += e * UR[j, j:]
+    return Z
+

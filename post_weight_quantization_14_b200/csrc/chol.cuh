@@ -11,10 +11,13 @@
 //     leaf(j):   R_jj = UL-Cholesky(A_jj), X_jj = R_jj^-1           (one CTA, fp32)
 //     panel(j):  R_{0:j, j} = A_{0:j, j} X_jj^T                      (3xTF32 tcgen05)
 //     update(j): A_{0:j, 0:j} -= R_{0:j, j} R_{0:j, j}^T             (3xTF32 tcgen05)
-//   with the update split three ways: block column j-1 on the critical chain, then block
-//   column j-2 and the rest on a helper stream (look-ahead of depth two).
-//   then U = R^-1 by doubling: for s = 128, 256, ...: for each diagonal pair
-//     [[R_a, B], [0, R_c]] with known inverses U_a, U_c:  U_b = -U_a (B U_c).
+//   scheduled on three streams: the chain carries leaf(j) and, for the next leaf, only the
+//   128x128 products R_{j-1,j} and A_{j-1,j-1} -= R_{j-1,j} R_{j-1,j}^T; a high-priority
+//   stream the rest of the panel and block columns j-1 and j-2; a low-priority stream the
+//   Schur update of the block columns left of them (look-ahead of depth two).
+//   and U = R^-1 by doubling on a fourth stream, each product as soon as its inputs exist:
+//   for each diagonal pair [[R_a, B], [0, R_c]] of 128, 256, ... columns with known
+//   inverses U_a, U_c:  U_b = -U_a (B U_c).
 #pragma once
 #include "gemm_tc.cuh"
 #include "actorder.cuh"
@@ -139,14 +142,18 @@ __global__ void __launch_bounds__(256) zero_lower_blocks_kernel(float* __restric
 // Works on the index-reversed block P = J A_jj J, for which the UL factor becomes an
 // ordinary lower Cholesky factor: A_jj = R R^T with R = J L J, and X_jj = R^-1 = J L^-1 J.
 //
-// Right-looking, blocked by 32 columns.  Panel kb (columns k0 = 32 kb .. k0 + 31, rows
-// k0 .. 127) is eliminated by the 4 - kb warps that own its rows (one row per lane, the
-// row's 32 panel entries in registers), one named barrier per pivot (leaf_eliminate).
-// All warps then apply the rank-32 update of the trailing lower
-// triangle on 4x4 register micro-tiles.  Meanwhile the warps not in the elimination
-// build the inverse X = L^-1 block row by block row, one row behind:
-// X_ii = L_ii^-1 by forward substitution (lane = column), the partial products L_ik X_kj
-// (j <= k < i) one 32-block each, and X_ij = -X_ii sum_k L_ik X_kj.
+// Right-looking, blocked by 32 columns.  For panel kb (columns k0 = 32 kb .. k0 + 31):
+//   A. one warp factors the 32x32 diagonal block in registers, lane = row.  The only
+//      dependency from one pivot to the next is one shuffle of the next pivot, which each
+//      lane keeps up to date from its own multipliers (the broadcasts of the multipliers to
+//      the other rows are off that chain); 1/L_kk = rsqrt with one Newton step.
+//   B. the rows below the block (one thread per row, 32 - 96 rows) solve against L_kk by
+//      substitution with the reciprocals of step A; meanwhile one otherwise idle warp forms
+//      X_kk = L_kk^-1 by forward substitution (lane = column).
+//   C. all threads apply the rank-32 update of the trailing lower triangle on 4x4
+//      register micro-tiles.
+// Then the off-diagonal blocks of X = L^-1, block row by block row:
+// X_ij = -X_ii sum_{k=j}^{i-1} L_ik X_kj, the sums first (kept in X's free upper blocks).
 // Writes X_jj (upper, zeros below the diagonal) as U_hi = tf32(X_jj) and U_lo = X_jj - U_hi
 // (exact, not rounded: the tensor pipe reads only its tf32 part); U_hi + U_lo restores
 // X_jj exactly for chol_diag_out_kernel.
@@ -156,60 +163,86 @@ static_assert(NB * NB / 4 == 8 * LEAF_THREADS && NB * 32 == 8 * LEAF_THREADS, "l
 
 struct LeafSmem {
     float P[NB][LS];         // reversed block; lower triangle holds the Schur complement
-    float X[NB][LS];         // L^-1 (lower); blocks above the diagonal hold partial products
+    float X[NB][LS];         // L^-1 (lower); blocks above the diagonal hold the block-row sums
     float LT[NB][LS];        // L transposed: LT[m][r] = L[r][m]
     float XDT[4][32][36];    // diagonal inverses transposed: XDT[i][m][r] = X_ii[r][m]
-    float col[2][32];        // pivot column of the current step (double-buffered)
+    float rinv[NB];          // 1 / L_kk
 };
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
-__device__ __forceinline__ void named_bar(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// Eliminate panel k0 .. k0+31 with nw warps (barrier 1); warp w owns rows k0 + 32 w + lane.
-// At step k the warp holding the diagonal block publishes the current column k of that
-// block in shared memory, and every row r does L_rk = P_rk / sqrt(P_kk) and
-// P_rj -= P_rk P_jk / P_kk for j > k.
-__device__ __forceinline__ void leaf_eliminate(LeafSmem& S, int k0, int nw, int warp, int lane, int jb) {
-    const int r = k0 + 32 * warp + lane;
-    const bool dg = warp == 0;   // the warp holding the diagonal 32x32 block
-    float pr[32];
+// A. Factor the 32x32 diagonal block at (k0, k0) with one warp; lane i holds row k0 + i.
+// Writes L_kk (lower, zeros above) to P and LT, and 1/L_kk to rinv.
+__device__ __forceinline__ void leaf_diag_factor(LeafSmem& S, int k0, int lane, int jb) {
+    constexpr unsigned FULL = 0xffffffffu;
+    float a[32];
 #pragma unroll
     for (int j4 = 0; j4 < 8; ++j4) {
-        const float4 v = ld4(&S.P[r][k0 + 4 * j4]);
-        pr[4 * j4 + 0] = v.x;
-        pr[4 * j4 + 1] = v.y;
-        pr[4 * j4 + 2] = v.z;
-        pr[4 * j4 + 3] = v.w;
+        const float4 v = ld4(&S.P[k0 + lane][k0 + 4 * j4]);
+        a[4 * j4 + 0] = v.x;
+        a[4 * j4 + 1] = v.y;
+        a[4 * j4 + 2] = v.z;
+        a[4 * j4 + 3] = v.w;
+    }
+    // this lane's diagonal entry, kept current with the lane's own multipliers
+    float dg = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) dg = (lane == j) ? a[j] : dg;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        const float p = __shfl_sync(FULL, dg, k);   // pivot: P_kk after pivots 0..k-1
+        if (lane == 0 && !(p > 0.f && isfinite(p)))
+            record_status(isfinite(p) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE, jb + 127 - (k0 + k));
+        float r = rsqrtf(p);
+        r = r * fmaf(-0.5f * p * r, r, 1.5f);       // one Newton step for 1/sqrt(p)
+        const float l = (lane == k) ? p * r : a[k] * r;   // L_kk = sqrt(p); L_ik = P_ik / L_kk
+        a[k] = l;
+        if (lane > k) dg = fmaf(-l, l, dg);
+        if (lane == k) S.rinv[k0 + k] = r;
+#pragma unroll
+        for (int j = k + 1; j < 32; ++j) {
+            const float lj = __shfl_sync(FULL, l, j);
+            a[j] = fmaf(-l, lj, a[j]);              // P_ij -= L_ik L_jk (meaningful for lanes >= j)
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const float v = (j <= lane) ? a[j] : 0.f;
+        S.P[k0 + lane][k0 + j] = v;
+        S.LT[k0 + j][k0 + lane] = v;
+    }
+}
+
+// B. Rows k0+32 .. 127 (one thread each): L_i,kb = P_i,kb L_kk^-T by substitution.
+__device__ __forceinline__ void leaf_panel_solve(LeafSmem& S, int k0, int i) {
+    float a[32];
+#pragma unroll
+    for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 v = ld4(&S.P[i][k0 + 4 * j4]);
+        a[4 * j4 + 0] = v.x;
+        a[4 * j4 + 1] = v.y;
+        a[4 * j4 + 2] = v.z;
+        a[4 * j4 + 3] = v.w;
     }
 #pragma unroll
     for (int k = 0; k < 32; ++k) {
-        float* cb = S.col[k & 1];
-        if (dg) cb[lane] = pr[k];   // column k of the diagonal block (rows >= k are valid)
-        named_bar(1, nw * 32);
-        const float piv = cb[k];
-        if (dg && lane == 0 && !(piv > 0.f && isfinite(piv)))
-            record_status(isfinite(piv) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE, jb + 127 - (k0 + k));
-        const float rinv = rsqrtf(piv);
-        const float f = pr[k] * (rinv * rinv);   // P_rk / P_kk
+        const float l = a[k] * S.rinv[k0 + k];
+        a[k] = l;
 #pragma unroll
         for (int j4 = (k + 1) >> 2; j4 < 8; ++j4) {
-            const float4 c4 = ld4(&cb[4 * j4]);
-            if (4 * j4 + 0 > k) pr[4 * j4 + 0] = fmaf(-f, c4.x, pr[4 * j4 + 0]);
-            if (4 * j4 + 1 > k) pr[4 * j4 + 1] = fmaf(-f, c4.y, pr[4 * j4 + 1]);
-            if (4 * j4 + 2 > k) pr[4 * j4 + 2] = fmaf(-f, c4.z, pr[4 * j4 + 2]);
-            if (4 * j4 + 3 > k) pr[4 * j4 + 3] = fmaf(-f, c4.w, pr[4 * j4 + 3]);
+            const float4 c4 = ld4(&S.LT[k0 + k][k0 + 4 * j4]);   // L_jk for j = 4 j4 ..
+            if (4 * j4 + 0 > k) a[4 * j4 + 0] = fmaf(-l, c4.x, a[4 * j4 + 0]);
+            if (4 * j4 + 1 > k) a[4 * j4 + 1] = fmaf(-l, c4.y, a[4 * j4 + 1]);
+            if (4 * j4 + 2 > k) a[4 * j4 + 2] = fmaf(-l, c4.z, a[4 * j4 + 2]);
+            if (4 * j4 + 3 > k) a[4 * j4 + 3] = fmaf(-l, c4.w, a[4 * j4 + 3]);
         }
-        pr[k] *= rinv;   // L_rk (L_kk = sqrt(P_kk) on the diagonal)
     }
 #pragma unroll
-    for (int j = 0; j < 32; ++j) S.LT[k0 + j][r] = (dg && j > lane) ? 0.f : pr[j];
+    for (int j = 0; j < 32; ++j) S.LT[k0 + j][i] = a[j];
 }
 
-// Rank-32 update of the trailing lower triangle (rows and columns >= k0 + 32) with the
-// panel just eliminated; 4x4 micro-tiles on the lower triangle of tiles only.
+// C. Rank-32 update of the trailing lower triangle (rows and columns >= k0 + 32) with the
+// panel just factored; 4x4 micro-tiles on the lower triangle of tiles only.
 __device__ __forceinline__ void leaf_trailing_update(LeafSmem& S, int k0, int tid) {
     const int t0 = k0 + 32, tn = (NB - t0) >> 2;
     const int ntask = tn * (tn + 1) / 2;
@@ -243,19 +276,15 @@ __device__ __forceinline__ void leaf_trailing_update(LeafSmem& S, int k0, int ti
 }
 
 // X_ii = L_ii^-1 by forward substitution, one warp, lane = column j:
-// x_m = (delta_mj - sum_{m' < m} L_mm' x_m') / L_mm.  The 32 reciprocals are formed up
-// front (lane m takes 1/L_mm) and broadcast by shuffle, off the substitution chain.
+// x_m = (delta_mj - sum_{m' < m} L_mm' x_m') / L_mm, with 1/L_mm from step A.
 __device__ __forceinline__ void leaf_diag_inverse(LeafSmem& S, int i, int lane) {
-    constexpr unsigned FULL = 0xffffffffu;
     const int k0 = 32 * i;
-    const float my_dinv = __frcp_rn(S.LT[k0 + lane][k0 + lane]);
     float x[32], s[32];
 #pragma unroll
     for (int m = 0; m < 32; ++m) s[m] = 0.f;
 #pragma unroll
     for (int m = 0; m < 32; ++m) {
-        const float dinv = __shfl_sync(FULL, my_dinv, m);
-        x[m] = (((m == lane) ? 1.f : 0.f) - s[m]) * dinv;
+        x[m] = (((m == lane) ? 1.f : 0.f) - s[m]) * S.rinv[k0 + m];
 #pragma unroll
         for (int q4 = (m + 1) >> 2; q4 < 8; ++q4) {
             const float4 l4 = ld4(&S.LT[k0 + m][k0 + 4 * q4]);   // L_{q,m} for q = 4 q4 ..
@@ -273,80 +302,38 @@ __device__ __forceinline__ void leaf_diag_inverse(LeafSmem& S, int i, int lane) 
             make_float4(x[4 * m4], x[4 * m4 + 1], x[4 * m4 + 2], x[4 * m4 + 3]);
 }
 
-// Slot of the partial product L_ik X_kj (j <= k < i) of block row i: one of the six
-// 32x32 blocks above X's block diagonal, all free while a block row is being formed.
-__device__ __forceinline__ float* leaf_partial_slot(LeafSmem& S, int j, int k) {
-    // pairs (j, k) in order (0,0), (0,1), (1,1), (0,2), (1,2), (2,2) -> blocks
-    // (0,1), (0,2), (0,3), (1,2), (1,3), (2,3)
-    const int idx = k * (k + 1) / 2 + j;
-    const int r = (idx >= 3) + (idx >= 5);
-    const int c = idx < 3 ? idx + 1 : (idx < 5 ? idx - 1 : 3);
-    return &S.X[32 * r][32 * c];
-}
-
-// Block row i of X = L^-1 by a group of g warps (group warp gw, barrier 2):
-// group warp 0 forms X_ii while the others form the partial products L_ik X_kj for
-// j <= k < i; then all form X_ij = -X_ii sum_{k=j}^{i-1} L_ik X_kj for j < i.
-__device__ __forceinline__ void leaf_x_block_row(LeafSmem& S, int i, int gw, int g, int lane) {
-    if (gw == 0) {
-        leaf_diag_inverse(S, i, lane);
-    } else if (i > 0) {
-        const int gt = (gw - 1) * 32 + lane, gn = (g - 1) * 32;
-        const int npairs = i * (i + 1) / 2;
-        for (int task = gt; task < 64 * npairs; task += gn) {
-            const int pr = task >> 6, tr = (task >> 3) & 7, tc = task & 7;
-            int k = 0;
-            while ((k + 1) * (k + 2) / 2 <= pr) ++k;
-            const int j = pr - k * (k + 1) / 2;
-            const int r0 = 4 * tr, c0 = 4 * tc;
-            float acc[4][4] = {};
+// Block row i of X = L^-1 with all threads: T_ij = sum_{k=j}^{i-1} L_ik X_kj into X's free
+// upper block (j, i), then X_ij = -X_ii T_ij.  Block rows < i must be complete.
+__device__ __forceinline__ void leaf_x_block_row(LeafSmem& S, int i, int tid) {
+    for (int task = tid; task < 64 * i; task += LEAF_THREADS) {
+        const int j = task >> 6, r0 = 4 * ((task >> 3) & 7), c0 = 4 * (task & 7);
+        float acc[4][4] = {};
+        for (int k = j; k < i; ++k) {
 #pragma unroll 8
             for (int m = 0; m < 32; ++m) {
                 const float4 a = ld4(&S.LT[32 * k + m][32 * i + r0]);   // L_ik[r][m]
-                const float4 bv4 = ld4(&S.X[32 * k + m][32 * j + c0]);   // X_kj[m][c]
-                const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bv4.x, bv4.y, bv4.z, bv4.w};
+                const float4 b = ld4(&S.X[32 * k + m][32 * j + c0]);    // X_kj[m][c]
+                const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
 #pragma unroll
                     for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
             }
-            float* slot = leaf_partial_slot(S, j, k);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                *reinterpret_cast<float4*>(slot + (r0 + u) * LS + c0) =
-                    make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
         }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<float4*>(&S.X[32 * j + r0 + u][32 * i + c0]) =
+                make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
     }
-    if (i == 0) return;
-    named_bar(2, g * 32);
-    const int gt = gw * 32 + lane, gn = g * 32;
-    for (int task = gt; task < 64 * i; task += gn) {
-        const int jbk = task >> 6, tr = (task >> 3) & 7, tc = task & 7;
-        const int r0 = 4 * tr, c0 = 4 * tc;
-        const int np = i - jbk;   // partials k = jbk .. i-1 (1 to 3)
-        const float* p0 = leaf_partial_slot(S, jbk, jbk) + c0;
-        const float* p1 = leaf_partial_slot(S, jbk, min(jbk + 1, 2)) + c0;
-        const float* p2 = leaf_partial_slot(S, jbk, 2) + c0;
+    __syncthreads();
+    for (int task = tid; task < 64 * i; task += LEAF_THREADS) {
+        const int j = task >> 6, r0 = 4 * ((task >> 3) & 7), c0 = 4 * (task & 7);
         float acc[4][4] = {};
-#pragma unroll 4
+#pragma unroll 8
         for (int m = 0; m < 32; ++m) {
-            const float4 a = ld4(&S.XDT[i][m][r0]);
-            float4 t4 = ld4(p0 + m * LS);
-            if (np > 1) {
-                const float4 q = ld4(p1 + m * LS);
-                t4.x += q.x;
-                t4.y += q.y;
-                t4.z += q.z;
-                t4.w += q.w;
-            }
-            if (np > 2) {
-                const float4 q = ld4(p2 + m * LS);
-                t4.x += q.x;
-                t4.y += q.y;
-                t4.z += q.z;
-                t4.w += q.w;
-            }
-            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {t4.x, t4.y, t4.z, t4.w};
+            const float4 a = ld4(&S.XDT[i][m][r0]);                   // X_ii[r][m]
+            const float4 b = ld4(&S.X[32 * j + m][32 * i + c0]);      // T_ij[m][c]
+            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
             for (int u = 0; u < 4; ++u)
 #pragma unroll
@@ -354,9 +341,10 @@ __device__ __forceinline__ void leaf_x_block_row(LeafSmem& S, int i, int gw, int
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-            *reinterpret_cast<float4*>(&S.X[32 * i + r0 + u][32 * jbk + c0]) =
+            *reinterpret_cast<float4*>(&S.X[32 * i + r0 + u][32 * j + c0]) =
                 make_float4(-acc[u][0], -acc[u][1], -acc[u][2], -acc[u][3]);
     }
+    __syncthreads();
 }
 
 __global__ void __launch_bounds__(LEAF_THREADS, 1)
@@ -390,18 +378,18 @@ __global__ void __launch_bounds__(LEAF_THREADS, 1)
     __syncthreads();
 
     for (int kb = 0; kb < 4; ++kb) {
-        const int nw = 4 - kb;
-        if (warp < nw)
-            leaf_eliminate(S, 32 * kb, nw, warp, lane, jb);
-        else if (kb > 0)
-            leaf_x_block_row(S, kb - 1, warp - nw, 16 - nw, lane);
+        const int k0 = 32 * kb;
+        if (warp == 0) leaf_diag_factor(S, k0, lane, jb);
         __syncthreads();
-        if (kb == 3) break;
-        leaf_trailing_update(S, 32 * kb, tid);
+        if (tid >= 32 && tid < 32 + (NB - k0 - 32)) leaf_panel_solve(S, k0, k0 + tid);   // rows k0+32 ..
+        else if (warp == 15) leaf_diag_inverse(S, kb, lane);
         __syncthreads();
+        if (kb < 3) {
+            leaf_trailing_update(S, k0, tid);
+            __syncthreads();
+        }
     }
-    leaf_x_block_row(S, 3, warp, 16, lane);
-    __syncthreads();
+    for (int i = 1; i < 4; ++i) leaf_x_block_row(S, i, tid);
 
     // U block = J X J (upper): U[r][c] = X[127-r][127-c] for r <= c; 4 columns per thread
 #pragma unroll 2
@@ -424,15 +412,15 @@ __global__ void __launch_bounds__(LEAF_THREADS, 1)
     }
 }
 
-// One CTA per diagonal block jb = 128 * blockIdx.x: X_jj = U_hi + U_lo (exact, as the leaf
+// One CTA per diagonal block jb = 128 * (blk0 + blockIdx.x): X_jj = U_hi + U_lo (exact, as the leaf
 // wrote them).  Writes X_jj to the public U (clipped to d) and its transposed tf32 split to
 // UT_hi/UT_lo.
 __global__ void __launch_bounds__(512)
     chol_diag_out_kernel(const float* __restrict__ U_hi, const float* __restrict__ U_lo, float* __restrict__ UT_hi,
-                         float* __restrict__ UT_lo, float* __restrict__ U, long long n, long long d) {
+                         float* __restrict__ UT_lo, float* __restrict__ U, long long n, long long d, int blk0) {
     extern __shared__ __align__(16) uint8_t dout_raw[];
     float (*Vs)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dout_raw);
-    const long long jb = (long long)blockIdx.x * NB;
+    const long long jb = (long long)(blk0 + blockIdx.x) * NB;
     for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
         const int r = e >> 7, c = e & 127;
         const long long off = (jb + r) * n + jb + c;
@@ -463,7 +451,7 @@ struct HinvWs {
 
 inline size_t hinv_ws_bytes(long long d) {
     const long long n = chol_n(d);
-    return (size_t)(9 * n * n + 2 * n * gq::NB + 64 + n) * sizeof(float);
+    return (size_t)(9 * n * n + 4 * n * gq::NB + 64 + n) * sizeof(float);
 }
 
 inline HinvWs hinv_ws_carve(void* ws, long long d) {
@@ -488,10 +476,10 @@ inline HinvWs hinv_ws_carve(void* ws, long long d) {
     p += n * n;
     w.TT_lo = p;
     p += n * n;
-    w.AP_hi = p;
-    p += n * gq::NB;
+    w.AP_hi = p;   // two panel splits (block columns of either parity), n x 128 each
+    p += 2 * n * gq::NB;
     w.AP_lo = p;
-    p += n * gq::NB;
+    p += 2 * n * gq::NB;
     w.scal = p;
     p += 64;
     w.rank = reinterpret_cast<int*>(p);
@@ -534,198 +522,208 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
     const int leaf_smem = (int)sizeof(gq::LeafSmem);
     GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::chol_leaf_kernel), leaf_smem));
     const uint64_t N = (uint64_t)n;
-    // Look-ahead of depth two.  The caller's stream carries the critical chain
-    // leaf(j) -> panel(j) -> update of block column j-1 by panel j.  A helper stream takes
-    // the rest of panel j's Schur update: first block column j-2 (u2), then everything left
-    // of it (rest), on at most SMs - 1 CTAs so the next leaf finds an SM.  Block column j-1
-    // has received, before its update by panel j, u2(j+1) and rest(p) for p >= j+2, which
-    // the helper stream runs in that order; so the chain waits only for u2(j+1).
-    cudaStream_t st2;
-    cudaEvent_t ev_panel, ev_u2;
-    if (!aux_stream(&st2, &ev_panel, &ev_u2)) return cudaErrorUnknown;
-    bool u2_pending = false, st2_used = false;
-    Mat rh{w.RS_hi, N, N, N}, rl{w.RS_lo, N, N, N};
-    for (int j = T - 1; j >= 0; --j) {
-        const int jb = j * gq::NB;
-        {
-            gqh::TimedScope ts__("chol_leaf", st);
-            GQ_TRY(launch_pdl(gq::chol_leaf_kernel, dim3(1), dim3(gq::LEAF_THREADS), (size_t)leaf_smem, st,
-                              (const float*)w.A, n, jb, w.U_hi, w.U_lo));
-        }
-        if (j == 0) break;
-        if (j == T - 1) {   // later panels are split by the previous update's epilogue
-            gqh::TimedScope ts__("split_panel", st);
-            gq::split_panel_kernel<<<(unsigned)std::min<long long>((jb * 128LL + 255) / 256, 4096), 256, 0, st>>>(
-                w.A, n, jb, jb, w.AP_hi, w.AP_lo);
-        }
-        GQ_TRY(cudaGetLastError());
-        {   // panel: RS[0:jb, jb:jb+128] = AP * X^T, X = U block (row-major split)
-            gq::GemmArgs p = gemm_args(jb, gq::NB, gq::NB);
-            p.b_row0 = jb;
-            p.b_col0 = jb;
-            p.s_col0 = jb;
-            EpiMats o;
-            o.s_hi = Mat{w.RS_hi, N, N, N};
-            o.s_lo = Mat{w.RS_lo, N, N, N};
-            Mat ah{w.AP_hi, (uint64_t)jb, 128, 128}, al{w.AP_lo, (uint64_t)jb, 128, 128};
-            Mat bh{w.U_hi, N, N, N}, bl{w.U_lo, N, N, N};
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(ah, al, bh, bl, o, p, 1, st, "chol_panel")));
-        }
-        const int jn = jb - gq::NB;    // first column of block column j-1
-        const int jn2 = jn - gq::NB;   // first column of block column j-2
-        if (j >= 2) GQ_TRY(cudaEventRecord(ev_panel, st));
-        const bool waited = u2_pending;
-        if (u2_pending) GQ_TRY(cudaStreamWaitEvent(st, ev_u2, 0));
-        {   // block column j-1: A[0:jb, jn:jb] -= RS_panel RS_panel[jn:jb]^T, plus the next panel's split
-            gq::GemmArgs p = gemm_args(jb, gq::NB, gq::NB);
-            p.a_col0 = jb;
-            p.b_row0 = jn;
-            p.b_col0 = jb;
-            p.alpha = -1.f;
-            p.beta = 1.f;
-            p.write_c = 1;
-            p.c_col0 = jn;
-            EpiMats o;
-            o.c = Mat{w.A, N, N, N};
-            if (j >= 2) {   // tiles above the diagonal block write the next panel's tf32 split
-                p.s_mt_lim = j - 1;
-                o.s_hi = Mat{w.AP_hi, (uint64_t)jn, 128, 128};
-                o.s_lo = Mat{w.AP_lo, (uint64_t)jn, 128, 128};
-            }
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, rh, rl, o, p, 1, st, "chol_update_next", 0,
-                                                        waited)));
-        }
-        u2_pending = false;
-        if (j >= 2) {   // helper stream: block column j-2, then the rest
-            GQ_TRY(cudaStreamWaitEvent(st2, ev_panel, 0));
-            st2_used = true;
-            {   // u2: A[0:jn, jn2:jn] -= RS_panel RS_panel[jn2:jn]^T
-                gq::GemmArgs p = gemm_args(jn, gq::NB, gq::NB);
-                p.a_col0 = jb;
-                p.b_row0 = jn2;
-                p.b_col0 = jb;
-                p.alpha = -1.f;
-                p.beta = 1.f;
-                p.write_c = 1;
-                p.c_col0 = jn2;
-                EpiMats o;
-                o.c = Mat{w.A, N, N, N};
-                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, rh, rl, o, p, 1, st2, "chol_update_u2",
-                                                            std::max(1, num_sms() - 1), true)));
-            }
-            GQ_TRY(cudaEventRecord(ev_u2, st2));
-            u2_pending = true;
-            if (j >= 3) {   // rest: A[0:jn2, 0:jn2] -= RS RS^T (upper tiles)
-                gq::GemmArgs p = gemm_args(jn2, jn2, gq::NB);
-                p.a_col0 = jb;
-                p.b_col0 = jb;
-                p.triangular = 1;
-                p.alpha = -1.f;
-                p.beta = 1.f;
-                p.write_c = 1;
-                EpiMats o;
-                o.c = Mat{w.A, N, N, N};
-                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rh, rl, rh, rl, o, p, 1, st2, "chol_update",
-                                                       std::max(1, num_sms() - 1), true)));
-            }
-        }
-    }
-    if (st2_used) {   // everything on the helper stream is done before the inverse
-        GQ_TRY(cudaEventRecord(ev_u2, st2));
-        GQ_TRY(cudaStreamWaitEvent(st, ev_u2, 0));
-    }
+    // Streams.  The chain stream carries, per block column j, only what the next leaf needs:
+    //   leaf(j) -> C1: R_{j-1,j} = A_{j-1,j} X_jj^T (one 128x128 block of the panel)
+    //           -> C2: A_{j-1,j-1} -= R_{j-1,j} R_{j-1,j}^T        -> leaf(j-1).
+    // The near stream: P, the rest of the panel (rows 0 .. j-2); N, block column j-1 above its
+    // diagonal block (and the tf32 split of the next panel); U2, block column j-2 with its
+    // diagonal block.  The far stream: R, the Schur update of block columns 0 .. j-3.
+    // Every block is updated in step order: C1(j) reads the panel split N(j+1) wrote; C2(j)
+    // follows U2(j+1) on block (j-1, j-1); U2(j) follows R(j+1) on block column j-2.
+    FactStreams fs;
+    if (!fact_streams(&fs)) return cudaErrorUnknown;
+    cudaEvent_t ev_start = fs.ev[0], ev_leaf = fs.ev[1], ev_P = fs.ev[2], ev_C1 = fs.ev[3], ev_N = fs.ev[4],
+                ev_U2 = fs.ev[5], ev_R = fs.ev[6], ev_near = fs.ev[7], ev_far = fs.ev[8], ev_chain = fs.ev[9],
+                ev_inv = fs.ev[10];
+    cudaStream_t sc = fs.chain, sn = fs.near, sf = fs.far, si = fs.inv;
     {
-        const int smem = (int)(gq::NB * (gq::NB + 1) * sizeof(float));
-        GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::chol_diag_out_kernel), smem));
-        gqh::TimedScope ts__("chol_diag_out", st);
-        gq::chol_diag_out_kernel<<<(unsigned)T, 512, smem, st>>>(w.U_hi, w.U_lo, w.UT_hi, w.UT_lo, U, n, d);
+        gqh::TimedScope ts__("zero_lower", st);   // the public U's strictly lower blocks
+        const unsigned nb = (unsigned)((d + gq::NB - 1) / gq::NB);
+        gq::zero_lower_blocks_kernel<<<dim3(nb, nb), 256, 0, st>>>(U, d);
     }
     GQ_TRY(cudaGetLastError());
-    // U = R^-1 by doubling
-    Mat rsh{w.RS_hi, N, N, N}, rsl{w.RS_lo, N, N, N};
+    GQ_TRY(cudaEventRecord(ev_start, st));
+    GQ_TRY(cudaStreamWaitEvent(sc, ev_start, 0));
+    GQ_TRY(cudaStreamWaitEvent(sn, ev_start, 0));
+    GQ_TRY(cudaStreamWaitEvent(sf, ev_start, 0));
+    GQ_TRY(cudaStreamWaitEvent(si, ev_start, 0));
+    const int side = std::max(1, num_sms() - 8);   // helper grids leave SMs to the chain
+    Mat rh{w.RS_hi, N, N, N}, rl{w.RS_lo, N, N, N};
+    Mat xh{w.U_hi, N, N, N}, xl{w.U_lo, N, N, N};
+    float* ap_hi[2] = {w.AP_hi, w.AP_hi + n * gq::NB};
+    float* ap_lo[2] = {w.AP_lo, w.AP_lo + n * gq::NB};
+    // C -= RS(rows a_row0 ..) RS(rows b_row0 ..)^T over the panel of block column j
+    auto schur = [&](int jb, int M, int Ncols, int b_row0, int c_row0, int c_col0, bool tri, cudaStream_t s_,
+                     const char* name, int max_ctas, const EpiMats* extra_s, bool after) -> cudaError_t {
+        gq::GemmArgs p = gemm_args(M, Ncols, gq::NB);
+        p.a_row0 = c_row0;
+        p.a_col0 = jb;
+        p.b_row0 = b_row0;
+        p.b_col0 = jb;
+        p.alpha = -1.f;
+        p.beta = 1.f;
+        p.write_c = 1;
+        p.c_row0 = c_row0;
+        p.c_col0 = c_col0;
+        p.triangular = tri ? 1 : 0;
+        EpiMats o;
+        if (extra_s) o = *extra_s;
+        o.c = Mat{w.A, N, N, N};
+        if (tri) return launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rh, rl, rh, rl, o, p, 1, s_, name, max_ctas, after);
+        return launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, rh, rl, o, p, 1, s_, name, max_ctas, after);
+    };
+    // RS(rows r0 .. r0+M, block column j) = AP(rows r0 ..) X_jj^T
+    auto panel = [&](int jb, int r0, int M, cudaStream_t s_, const char* name, int max_ctas, bool after) {
+        const int par = (jb / gq::NB) & 1;
+        gq::GemmArgs p = gemm_args(M, gq::NB, gq::NB);
+        p.a_row0 = r0;
+        p.b_row0 = jb;
+        p.b_col0 = jb;
+        p.s_row0 = r0;
+        p.s_col0 = jb;
+        EpiMats o;
+        o.s_hi = Mat{w.RS_hi, N, N, N};
+        o.s_lo = Mat{w.RS_lo, N, N, N};
+        Mat ah{ap_hi[par], (uint64_t)jb, 128, 128}, al{ap_lo[par], (uint64_t)jb, 128, 128};
+        return launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(ah, al, xh, xl, o, p, 1, s_, name, max_ctas, after);
+    };
+    // U = R^-1 by doubling, each product issued on the inverse stream as soon as its inputs
+    // exist: for the diagonal pair [[R_a, B], [0, R_c]] of level s (a-half rows r0 .. r0+s,
+    // c-half r0+s .. r0+s+cs) with inverses U_a and U_c known, T = B U_c (stored transposed) as
+    // soon as the c-half is inverted and the panels of its block columns are formed, and
+    // U_b = -U_a T once the a-half is inverted.  Only the products of the pairs that contain
+    // block 0 wait for the last leaf.
     Mat uth{w.UT_hi, N, N, N}, utl{w.UT_lo, N, N, N};
-    Mat uh{w.U_hi, N, N, N}, ul{w.U_lo, N, N, N};
     Mat tth{w.TT_hi, N, N, N}, ttl{w.TT_lo, N, N, N};
-    for (long long s = gq::NB; s < n; s *= 2) {
-        const long long full = n / (2 * s);
-        const long long rem = n - full * 2 * s;
-        for (int part = 0; part < 2; ++part) {
-            long long r0, cs, batch;
-            if (part == 0) {
-                r0 = 0;
-                cs = s;
-                batch = full;
-            } else {
-                if (rem <= s) break;
-                r0 = full * 2 * s;
-                cs = rem - s;
-                batch = 1;
-            }
-            if (batch <= 0) continue;
-            const int zs = (int)(2 * s);
-            // levels with few 128x128 tiles take 128x32 tiles (more SMs share the epilogue stores)
-            const bool narrow = 4 * batch * (s / gq::NB) * ((cs + gq::NB - 1) / gq::NB) <= num_sms();
-            {   // T = B U_c, stored transposed in TT at (r0+s+j, r0+i)
-                gq::GemmArgs p = gemm_args((int)s, (int)cs, (int)cs);
-                p.a_row0 = (int)r0;
-                p.a_col0 = (int)(r0 + s);
-                p.a_zrow = p.a_zcol = zs;
-                p.b_row0 = (int)(r0 + s);
-                p.b_col0 = (int)(r0 + s);
-                p.b_zrow = p.b_zcol = zs;
-                p.k_to_n1 = 1;
-                p.t_row0 = (int)(r0 + s);
-                p.t_col0 = (int)r0;
-                p.t_zrow = p.t_zcol = zs;
-                EpiMats o;
-                o.t_hi = Mat{w.TT_hi, N, N, N};
-                o.t_lo = Mat{w.TT_lo, N, N, N};
-                if (narrow)
-                    GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rsh, rsl, uth, utl, o, p, (int)batch, st, "inv_bu")));
-                else
-                    GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rsh, rsl, uth, utl, o, p, (int)batch, st, "inv_bu")));
-            }
-            {   // U_b = -U_a T -> U (public, clipped), U split, UT split
-                gq::GemmArgs p = gemm_args((int)s, (int)cs, (int)s);
-                p.a_row0 = (int)r0;
-                p.a_col0 = (int)r0;
-                p.a_zrow = p.a_zcol = zs;
-                p.b_row0 = (int)(r0 + s);
-                p.b_col0 = (int)r0;
-                p.b_zrow = p.b_zcol = zs;
-                p.k_from_m0 = 1;
-                p.alpha = -1.f;
-                p.c_row0 = (int)r0;
-                p.c_col0 = (int)(r0 + s);
-                p.c_zrow = p.c_zcol = zs;
-                p.write_c = 1;
-                p.s_row0 = (int)r0;
-                p.s_col0 = (int)(r0 + s);
-                p.s_zrow = p.s_zcol = zs;
-                p.t_row0 = (int)(r0 + s);
-                p.t_col0 = (int)r0;
-                p.t_zrow = p.t_zcol = zs;
-                EpiMats o;
-                o.c = Mat{U, (uint64_t)d, (uint64_t)d, (uint64_t)d};   // public U, clipped to d x d
-                o.s_hi = Mat{w.U_hi, N, N, N};
-                o.s_lo = Mat{w.U_lo, N, N, N};
-                o.t_hi = Mat{w.UT_hi, N, N, N};
-                o.t_lo = Mat{w.UT_lo, N, N, N};
-                if (narrow)
-                    GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(uh, ul, tth, ttl, o, p, (int)batch, st, "inv_ub")));
-                else
-                    GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(uh, ul, tth, ttl, o, p, (int)batch, st, "inv_ub")));
-            }
-        }
-    }
-    {
+    const int dout_smem = (int)(gq::NB * (gq::NB + 1) * sizeof(float));
+    GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::chol_diag_out_kernel), dout_smem));
+    auto inv_bu = [&](long long s_, long long r0, long long cs) -> cudaError_t {   // T = B U_c -> TT
+        gq::GemmArgs p = gemm_args((int)s_, (int)cs, (int)cs);
+        p.a_row0 = (int)r0;
+        p.a_col0 = (int)(r0 + s_);
+        p.b_row0 = (int)(r0 + s_);
+        p.b_col0 = (int)(r0 + s_);
+        p.k_to_n1 = 1;
+        p.t_row0 = (int)(r0 + s_);
+        p.t_col0 = (int)r0;
+        EpiMats o;
+        o.t_hi = Mat{w.TT_hi, N, N, N};
+        o.t_lo = Mat{w.TT_lo, N, N, N};
+        const bool narrow = 4 * (s_ / gq::NB) * ((cs + gq::NB - 1) / gq::NB) <= num_sms();
+        if (narrow) return launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, uth, utl, o, p, 1, si, "inv_bu", side, true);
+        return launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rh, rl, uth, utl, o, p, 1, si, "inv_bu", side, true);
+    };
+    auto inv_ub = [&](long long s_, long long r0, long long cs) -> cudaError_t {   // U_b = -U_a T
+        gq::GemmArgs p = gemm_args((int)s_, (int)cs, (int)s_);
+        p.a_row0 = (int)r0;
+        p.a_col0 = (int)r0;
+        p.b_row0 = (int)(r0 + s_);
+        p.b_col0 = (int)r0;
+        p.k_from_m0 = 1;
+        p.alpha = -1.f;
+        p.c_row0 = (int)r0;
+        p.c_col0 = (int)(r0 + s_);
+        p.write_c = 1;
+        p.s_row0 = (int)r0;
+        p.s_col0 = (int)(r0 + s_);
+        p.t_row0 = (int)(r0 + s_);
+        p.t_col0 = (int)r0;
+        EpiMats o;
+        o.c = Mat{U, (uint64_t)d, (uint64_t)d, (uint64_t)d};   // public U, clipped to d x d
+        o.s_hi = Mat{w.U_hi, N, N, N};
+        o.s_lo = Mat{w.U_lo, N, N, N};
+        o.t_hi = Mat{w.UT_hi, N, N, N};
+        o.t_lo = Mat{w.UT_lo, N, N, N};
+        const bool narrow = 4 * (s_ / gq::NB) * ((cs + gq::NB - 1) / gq::NB) <= num_sms();
+        if (narrow) return launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(xh, xl, tth, ttl, o, p, 1, si, "inv_ub", side, true);
+        return launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(xh, xl, tth, ttl, o, p, 1, si, "inv_ub", side, true);
+    };
+    // the inverse work that becomes possible once leaf(j) and the panels of block column j exist
+    auto inverse_step = [&](int j) -> cudaError_t {
+        const long long jb = (long long)j * gq::NB;
+        GQ_TRY(cudaStreamWaitEvent(si, ev_leaf, 0));
         {
-            gqh::TimedScope ts__("zero_lower", st);
-            const unsigned nb = (unsigned)((d + gq::NB - 1) / gq::NB);
-            gq::zero_lower_blocks_kernel<<<dim3(nb, nb), 256, 0, st>>>(U, d);
+            gqh::TimedScope ts__("chol_diag_out", si);
+            gq::chol_diag_out_kernel<<<1, 512, dout_smem, si>>>(w.U_hi, w.U_lo, w.UT_hi, w.UT_lo, U, n, d, j);
         }
         GQ_TRY(cudaGetLastError());
+        for (long long s_ = gq::NB; s_ < n; s_ *= 2)   // pairs whose a-half starts at block j
+            if (jb % (2 * s_) == 0 && jb + s_ < n) GQ_TRY(inv_ub(s_, jb, std::min(s_, n - jb - s_)));
+        if (j > 0) {
+            GQ_TRY(cudaStreamWaitEvent(si, ev_P, 0));
+            GQ_TRY(cudaStreamWaitEvent(si, ev_C1, 0));
+        }
+        for (long long s_ = gq::NB; s_ < n; s_ *= 2)   // pairs whose c-half starts at block j
+            if (jb >= s_ && (jb - s_) % (2 * s_) == 0) GQ_TRY(inv_bu(s_, jb - s_, std::min(s_, n - jb)));
+        return cudaSuccess;
+    };
+    for (int j = T - 1; j >= 0; --j) {
+        const int jb = j * gq::NB;
+        const int jn = jb - gq::NB;    // first column of block column j-1
+        const int jn2 = jn - gq::NB;   // first column of block column j-2
+        {
+            gqh::TimedScope ts__("chol_leaf", sc);
+            if (j == T - 1)   // follows the wait for the damped copy on the caller's stream
+                GQ_TRY(launch_plain(gq::chol_leaf_kernel, dim3(1), dim3(gq::LEAF_THREADS), (size_t)leaf_smem, sc,
+                                    (const float*)w.A, n, jb, w.U_hi, w.U_lo));
+            else
+                GQ_TRY(launch_pdl(gq::chol_leaf_kernel, dim3(1), dim3(gq::LEAF_THREADS), (size_t)leaf_smem, sc,
+                                  (const float*)w.A, n, jb, w.U_hi, w.U_lo));
+        }
+        if (j == 0) {
+            GQ_TRY(cudaEventRecord(ev_leaf, sc));
+            GQ_TRY(inverse_step(0));
+            break;
+        }
+        if (j == T - 1) {   // the first panel's tf32 split; later ones come from N
+            gqh::TimedScope ts__("split_panel", sc);
+            gq::split_panel_kernel<<<(unsigned)std::min<long long>((jb * 128LL + 255) / 256, 4096), 256, 0, sc>>>(
+                w.A, n, jb, jb, ap_hi[j & 1], ap_lo[j & 1]);
+            GQ_TRY(cudaGetLastError());
+        }
+        GQ_TRY(cudaEventRecord(ev_leaf, sc));
+        // near stream: the panel's rows 0 .. j-2
+        GQ_TRY(cudaStreamWaitEvent(sn, ev_leaf, 0));
+        if (jn > 0) GQ_TRY(panel(jb, 0, jn, sn, "chol_panel", side, true));
+        GQ_TRY(cudaEventRecord(ev_P, sn));
+        // chain: C1, C2
+        GQ_TRY(cudaStreamWaitEvent(sc, ev_N, 0));
+        GQ_TRY(panel(jb, jn, gq::NB, sc, "chol_chain_r", 0, true));
+        GQ_TRY(cudaEventRecord(ev_C1, sc));
+        GQ_TRY(cudaStreamWaitEvent(sc, ev_U2, 0));
+        GQ_TRY(schur(jb, gq::NB, gq::NB, jn, jn, jn, false, sc, "chol_chain_d", 0, nullptr, true));
+        if (jn > 0) {
+            // near stream: N(j) = block column j-1 above its diagonal block + the next panel's split
+            GQ_TRY(cudaStreamWaitEvent(sn, ev_C1, 0));
+            EpiMats so;
+            so.s_hi = Mat{ap_hi[(j - 1) & 1], (uint64_t)jn, 128, 128};
+            so.s_lo = Mat{ap_lo[(j - 1) & 1], (uint64_t)jn, 128, 128};
+            GQ_TRY(schur(jb, jn, gq::NB, jn, 0, jn, false, sn, "chol_update_next", side, &so, true));
+            GQ_TRY(cudaEventRecord(ev_N, sn));
+            // U2(j) = block column j-2, rows 0 .. j-2 (with its diagonal block), after R(j+1)
+            if (jn2 >= 0) {
+                GQ_TRY(cudaStreamWaitEvent(sn, ev_R, 0));
+                GQ_TRY(schur(jb, jn, gq::NB, jn2, 0, jn2, false, sn, "chol_update_u2", side, nullptr, true));
+            }
+            GQ_TRY(cudaEventRecord(ev_U2, sn));
+            // far stream: R(j) = block columns 0 .. j-3
+            if (jn2 > 0) {
+                GQ_TRY(cudaStreamWaitEvent(sf, ev_P, 0));
+                GQ_TRY(schur(jb, jn2, jn2, 0, 0, 0, true, sf, "chol_update", side, nullptr, true));
+                GQ_TRY(cudaEventRecord(ev_R, sf));
+            }
+        }
+        GQ_TRY(inverse_step(j));
     }
+    // all streams are done before the caller's stream continues
+    GQ_TRY(cudaEventRecord(ev_near, sn));
+    GQ_TRY(cudaEventRecord(ev_far, sf));
+    GQ_TRY(cudaEventRecord(ev_chain, sc));
+    GQ_TRY(cudaEventRecord(ev_inv, si));
+    GQ_TRY(cudaStreamWaitEvent(st, ev_near, 0));
+    GQ_TRY(cudaStreamWaitEvent(st, ev_far, 0));
+    GQ_TRY(cudaStreamWaitEvent(st, ev_chain, 0));
+    GQ_TRY(cudaStreamWaitEvent(st, ev_inv, 0));
     return cudaSuccess;
 }
 

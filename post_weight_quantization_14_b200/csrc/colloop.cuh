@@ -19,7 +19,7 @@
 // At a group's first column the scale and zero come from the current values of the
 // group's columns (min/max by an 8-lane shuffle reduction).
 // At the end of the block the kernel writes the packed codes (qweight layout), the
-// errors e = d / U_cc as a tf32 split (operand of the trailing tensor-core update)
+// errors e = d / U_cc as a bf16 split (operand of the bf16x3 trailing tensor-core update)
 // and the per-row sum of e^2.
 #pragma once
 #include "gemm_tc.cuh"
@@ -53,8 +53,8 @@ struct ColArgs {
     int32_t* qweight;
     __half* scales;
     uint8_t* zeros_u8;
-    float* E_hi;          // errors of this block: E[row * e_ld + col], tf32 split
-    float* E_lo;
+    uint16_t* E_hi;       // errors of this block: E[row * e_ld + col], bf16 split (bit patterns)
+    uint16_t* E_lo;
     long long e_ld;
     float* err_sq;
     int first_block;
@@ -256,8 +256,8 @@ __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p)
             const float e = S.dv[rl][col] * S.invd[col];
             acc = fmaf(e, e, acc);
             if (rw < p.d_out) {
-                float h, l;
-                split_tf32(e, h, l);
+                uint16_t h, l;
+                split_bf16(e, h, l);
                 p.E_hi[rw * p.e_ld + col] = h;
                 p.E_lo[rw * p.e_ld + col] = l;
             }
@@ -305,9 +305,9 @@ __global__ void up_prep_kernel(const float* __restrict__ U, long long d, float* 
     if (threadIdx.x == 0 && c < nc) inv_d[c0 + c] = __frcp_rn(ucc);
 }
 
-// UT[j, i] = split(U[i, j]) for the 32x32 tiles on or above the diagonal of U.
-__global__ void ut_split_kernel(const float* __restrict__ U, long long d, float* __restrict__ UT_hi,
-                                float* __restrict__ UT_lo) {
+// UT[j, i] = bf16 split of U[i, j] for the 32x32 tiles on or above the diagonal of U.
+__global__ void ut_split_kernel(const float* __restrict__ U, long long d, uint16_t* __restrict__ UT_hi,
+                                uint16_t* __restrict__ UT_lo) {
     __shared__ float tile[32][33];
     const long long bi = blockIdx.y, bj = blockIdx.x;  // tile of U
     if (bi > bj) return;
@@ -319,8 +319,8 @@ __global__ void ut_split_kernel(const float* __restrict__ U, long long d, float*
     for (int r = threadIdx.y; r < 32; r += blockDim.y) {
         const long long j = bj * 32 + r, i = bi * 32 + threadIdx.x;
         if (i < d && j < d) {
-            float h, l;
-            split_tf32(tile[threadIdx.x][r], h, l);
+            uint16_t h, l;
+            split_bf16(tile[threadIdx.x][r], h, l);
             UT_hi[j * d + i] = h;
             UT_lo[j * d + i] = l;
         }
@@ -372,7 +372,8 @@ __global__ void row_params_kernel(const float* __restrict__ W, long long d_out, 
 namespace gqh {
 
 struct QuantWs {
-    float *Up, *inv_d, *UT_hi, *UT_lo, *E_hi, *E_lo, *row_scale, *row_zero;
+    float *Up, *inv_d, *row_scale, *row_zero;
+    uint16_t *UT_hi, *UT_lo, *E_hi, *E_lo;   // bf16 splits (operands of the trailing updates)
     uint8_t* zeros_u8;
 };
 
@@ -395,8 +396,8 @@ inline size_t quant_ws_bytes(long long d_out, long long d_in, int g) {
     size_t b = 0;
     b += align256((size_t)nblk * gq::UP_BLOCK * 4);
     b += align256((size_t)d_in * 4);
-    b += 2 * align256((size_t)d_in * d_in * 4);
-    b += 2 * align256((size_t)d_out * superblock_cols(d_in) * 4);
+    b += 2 * align256((size_t)d_in * d_in * 2);
+    b += 2 * align256((size_t)d_out * superblock_cols(d_in) * 2);
     b += 2 * align256((size_t)d_out * 4);
     b += align256((size_t)n_groups_of(d_in, g) * d_out);
     return b;
@@ -413,10 +414,10 @@ inline QuantWs quant_ws_carve(void* ws, long long d_out, long long d_in, int g) 
     };
     w.Up = reinterpret_cast<float*>(take((size_t)nblk * gq::UP_BLOCK * 4));
     w.inv_d = reinterpret_cast<float*>(take((size_t)d_in * 4));
-    w.UT_hi = reinterpret_cast<float*>(take((size_t)d_in * d_in * 4));
-    w.UT_lo = reinterpret_cast<float*>(take((size_t)d_in * d_in * 4));
-    w.E_hi = reinterpret_cast<float*>(take((size_t)d_out * superblock_cols(d_in) * 4));
-    w.E_lo = reinterpret_cast<float*>(take((size_t)d_out * superblock_cols(d_in) * 4));
+    w.UT_hi = reinterpret_cast<uint16_t*>(take((size_t)d_in * d_in * 2));
+    w.UT_lo = reinterpret_cast<uint16_t*>(take((size_t)d_in * d_in * 2));
+    w.E_hi = reinterpret_cast<uint16_t*>(take((size_t)d_out * superblock_cols(d_in) * 2));
+    w.E_lo = reinterpret_cast<uint16_t*>(take((size_t)d_out * superblock_cols(d_in) * 2));
     w.row_scale = reinterpret_cast<float*>(take((size_t)d_out * 4));
     w.row_zero = reinterpret_cast<float*>(take((size_t)d_out * 4));
     w.zeros_u8 = take((size_t)n_groups_of(d_in, g) * d_out);
@@ -472,13 +473,14 @@ cudaError_t quant_run_bits(float* W, const float* U, long long d_out, long long 
         p.write_c = 1;
         EpiMats o;
         o.c = Mat{W, (uint64_t)d_out, (uint64_t)d_in, (uint64_t)d_in};
-        // few 128-wide tiles: 128x32 tiles spread the work over more SMs, within one wave
-        // Segmented accumulation (16 k-steps, cross products apart): the in-place fp32
+        // few 128-wide tiles: 128x32 tiles spread the work over more SMs, within one wave.
+        // bf16x3 products (16-bit operand splits) at the bf16 rate; segmented accumulation
+        // (8 k-steps = 128 K per segment, cross products apart): the in-place fp32
         // accumulation of a K = 1024 update drifts by ~1e-5 relative, enough to move
         // near-tie rounding decisions of later columns.
         if (4 * ((d_out + gq::BM - 1) / gq::BM) * ((ncols + gq::CB - 1) / gq::CB) <= num_sms())
-            return launch_gemm<gq::KIND_TF32X3, 4, 32, 16>(eh, el, uh, ul, o, p, 1, st, name);
-        return launch_gemm<gq::KIND_TF32X3, 2, 128, 16>(eh, el, uh, ul, o, p, 1, st, name);
+            return launch_gemm<gq::KIND_BF16X3, 4, 32, 8>(eh, el, uh, ul, o, p, 1, st, name);
+        return launch_gemm<gq::KIND_BF16X3, 2, 128, 8>(eh, el, uh, ul, o, p, 1, st, name);
     };
     for (int b = 0; b < nblk; ++b) {
         const long long s0 = (long long)(b / SB_BLOCKS) * sbw;      // superblock columns

@@ -235,6 +235,18 @@ __device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
     hi = to_tf32(x);
     lo = to_tf32(x - hi);
 }
+// bf16 split: x ~ hi + lo with hi = bf16(x), lo = bf16(x - hi) (round to nearest even; x - hi
+// is exact in fp32), returned as bf16 bit patterns.
+__device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
+    uint16_t r;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+__device__ __forceinline__ void split_bf16(float x, uint16_t& hi, uint16_t& lo) {
+    hi = bf16_bits_rn(x);
+    lo = bf16_bits_rn(x - bf16_bits_to_f32(hi));
+}
 
 }  // namespace gq
 

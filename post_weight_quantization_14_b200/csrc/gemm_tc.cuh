@@ -10,6 +10,9 @@
 // KIND_TF32X3 : A = A_hi + A_lo and B = B_hi + B_lo given as two tf32 arrays each;
 //               three MMAs per 8-element K step (hi*hi + hi*lo + lo*hi), which keeps
 //               about fp32 accuracy on the tf32 tensor pipe.
+// KIND_BF16X3 : the same three-product split with bf16 parts (hi = bf16(x),
+//               lo = bf16(x - hi): 16 significant bits), one 16-element K step per MMA
+//               triple, at the bf16 rate and half the operand bytes of KIND_TF32X3.
 //
 // Segmented accumulation (SEG > 0): the tensor pipe's fp32 accumulation error grows with
 // the number of MMAs accumulated in place, so every SEG MMA k-steps the accumulator is
@@ -34,7 +37,10 @@
 
 namespace gq {
 
-enum : int { KIND_BF16 = 0, KIND_TF32X3 = 1 };
+enum : int { KIND_BF16 = 0, KIND_TF32X3 = 1, KIND_BF16X3 = 2 };
+
+// Bytes per operand element of a kind.
+__host__ __device__ constexpr int kind_elem_bytes(int kind) { return kind == KIND_TF32X3 ? 4 : 2; }
 
 struct GemmArgs {
     int M, N, K;
@@ -80,7 +86,7 @@ static_assert(32 * kEpiLd * 4 <= 2 * kBoxBytes, "register-path staging tile fits
 template <int KIND, int TBN = BN>
 struct GemmCfg {
     static_assert(TBN == 32 || TBN == 64 || TBN == 128, "tile N");
-    static constexpr int KT = (KIND == KIND_BF16) ? 64 : 32;  // K elements per stage (128 bytes)
+    static constexpr int KT = 128 / kind_elem_bytes(KIND);      // K elements per stage (128 bytes)
     static constexpr int NOPS = (KIND == KIND_BF16) ? 1 : 2;
     static constexpr int STAGE_BYTES = NOPS * (BM * 128 + TBN * 128);
 };
@@ -318,7 +324,7 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer
-        constexpr uint32_t idesc = make_idesc(KIND == KIND_BF16 ? 1u : 2u, BM, TBN);
+        constexpr uint32_t idesc = make_idesc(KIND == KIND_TF32X3 ? 2u : 1u, BM, TBN);
         uint32_t kiter = 0;
         bool ok = true;
         int seg = 0;   // accumulator segments issued by this CTA (buffer = seg & 1)
@@ -376,6 +382,15 @@ __global__ void __launch_bounds__(192, 1)
                     const uint32_t acc0 = segpos > 0 ? 1u : 0u;
                     if (KIND == KIND_BF16) {
                         umma_bf16(acc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_hi + off), idesc, acc0);
+                    } else if (KIND == KIND_BF16X3 && XACC) {
+                        const uint32_t x0 = kkc > 0 ? 1u : 0u;
+                        umma_bf16(acc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_hi + off), idesc, acc0);
+                        umma_bf16(xacc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_lo + off), idesc, x0);
+                        umma_bf16(xacc, desc_sw128_kmajor(a_lo + off), desc_sw128_kmajor(b_hi + off), idesc, 1u);
+                    } else if (KIND == KIND_BF16X3) {
+                        umma_bf16(acc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_hi + off), idesc, acc0);
+                        umma_bf16(acc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_lo + off), idesc, 1u);
+                        umma_bf16(acc, desc_sw128_kmajor(a_lo + off), desc_sw128_kmajor(b_hi + off), idesc, 1u);
                     } else if (XACC) {
                         const uint32_t x0 = kkc > 0 ? 1u : 0u;
                         umma_tf32(acc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_hi + off), idesc, acc0);
@@ -639,6 +654,15 @@ int num_sms();
 // A non-blocking helper stream and two timing-free events of the current device,
 // created on first use and kept for the life of the process.
 bool aux_stream(cudaStream_t* st, cudaEvent_t* ev0, cudaEvent_t* ev1);
+// Streams of the blocked factorization, created once per device: the critical chain and
+// the near updates at the highest stream priority, the far updates and the inverse at the
+// lowest; events
+// for the cross-stream dependencies (timing disabled).
+struct FactStreams {
+    cudaStream_t chain, near, far, inv;
+    cudaEvent_t ev[12];
+};
+bool fact_streams(FactStreams* fs);
 
 // C is read (beta != 0) only where it is also written.
 inline bool epilogue_fits(const gq::GemmArgs& p) { return p.beta == 0.f || p.write_c; }
@@ -653,7 +677,7 @@ cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2
                         int batch, cudaStream_t stream, const char* name, int max_ctas = 0,
                         bool after_event = false, bool no_alloc = false) {
     using Cfg = gq::GemmCfg<KIND, TBN>;
-    const int eb = (KIND == gq::KIND_BF16) ? 2 : 4;
+    const int eb = gq::kind_elem_bytes(KIND);
     CUtensorMap ma, ma2, mb, mb2, mc;
     auto tmap = [no_alloc](CUtensorMap* m, const Mat& x, int elb, uint32_t br, uint32_t bc) {
         return no_alloc ? make_tmap_2d_uncached(m, x.ptr, elb, x.rows, x.cols, x.ld, br, bc)

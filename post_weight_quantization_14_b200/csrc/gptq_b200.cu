@@ -19,6 +19,7 @@
 #include "pack.cuh"
 #include "colloop.cuh"
 #include "dqgemm.cuh"
+#include "gptq2d.cuh"
 
 namespace gqh {
 
@@ -138,6 +139,28 @@ bool aux_stream(cudaStream_t* st, cudaEvent_t* ev0, cudaEvent_t* ev1) {
     *st = streams[dev];
     *ev0 = events[dev][0];
     *ev1 = events[dev][1];
+    return true;
+}
+
+bool fact_streams(FactStreams* fs) {
+    static FactStreams cache[128];
+    static bool made[128];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return false;
+    if (!made[dev]) {
+        int least = 0, greatest = 0;
+        if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return false;
+        FactStreams f{};
+        if (cudaStreamCreateWithPriority(&f.chain, cudaStreamNonBlocking, greatest) != cudaSuccess) return false;
+        if (cudaStreamCreateWithPriority(&f.near, cudaStreamNonBlocking, greatest) != cudaSuccess) return false;
+        if (cudaStreamCreateWithPriority(&f.far, cudaStreamNonBlocking, least) != cudaSuccess) return false;
+        if (cudaStreamCreateWithPriority(&f.inv, cudaStreamNonBlocking, least) != cudaSuccess) return false;
+        for (auto& e : f.ev)
+            if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
+        cache[dev] = f;
+        made[dev] = true;
+    }
+    *fs = cache[dev];
     return true;
 }
 
@@ -531,6 +554,28 @@ gptq_status gptq_dequant_gemm(const void* X, int64_t M, const int32_t* qweight, 
         default: e = dq_gemm_run<8>(X, M, qweight, sc, qzeros, d_out, d_in, g, Y, st); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "dequant_gemm");
+    return GPTQ_OK;
+}
+
+size_t gptq_2d_workspace_bytes(int64_t m, int64_t n, int64_t batch) {
+    if (m < 1 || n < 1 || batch < 1) return 0;
+    return g2_ws_bytes(m, n, batch);
+}
+
+gptq_status gptq_2d_round(const double* X, int64_t m, int64_t n, int64_t batch, const double* U_left,
+                          const double* U_right, int32_t* Z, void* ws, size_t ws_bytes, void* stream) {
+    if (!X || !U_left || !U_right || !Z) return fail(GPTQ_ERR_INVALID_ARG, "X, U_left, U_right and Z must be non-NULL");
+    if (m < 1 || n < 1 || m > 16384 || n > 16384) return fail(GPTQ_ERR_INVALID_ARG, "m and n must be in [1, 16384]");
+    if (batch < 1 || batch > (1ll << 20) || batch * m * n > (1ll << 40))
+        return fail(GPTQ_ERR_INVALID_ARG, "batch out of range (%lld)", (long long)batch);
+    const uintptr_t mis = reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(U_left) |
+                          reinterpret_cast<uintptr_t>(U_right) | reinterpret_cast<uintptr_t>(ws);
+    if ((mis & 7u) || (reinterpret_cast<uintptr_t>(Z) & 3u))
+        return fail(GPTQ_ERR_INVALID_ARG, "X, U_left, U_right and ws must be 8-byte, Z 4-byte aligned");
+    const size_t need = g2_ws_bytes(m, n, batch);
+    if (!ws || ws_bytes < need) return fail(GPTQ_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+    cudaError_t e = g2_run(X, m, n, batch, U_left, U_right, Z, ws, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "gptq_2d_round");
     return GPTQ_OK;
 }
 

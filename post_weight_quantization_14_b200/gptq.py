@@ -75,6 +75,8 @@ _SIGS = {
                                              _vp, _vp, _vp, _sz, _vp]),
     "gptq_dequant_g_idx": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, ctypes.POINTER(GptqConfig), _vp, _vp]),
     "gptq_dequant_gemm": (_int, [_vp, _i64, _vp, _vp, _vp, _i64, _i64, ctypes.POINTER(GptqConfig), _vp, _vp]),
+    "gptq_2d_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "gptq_2d_round": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _sz, _vp]),
 }
 
 
@@ -310,6 +312,28 @@ def gptq_dequant_gemm(X: torch.Tensor, qweight, scales, qzeros, d_out: int, d_in
     _check(lib().gptq_dequant_gemm(_ptr(X), X.shape[0], _ptr(qweight), _ptr(scales), _ptr(qzeros), d_out, d_in,
                                    ctypes.byref(cfg), _ptr(Y), _stream(stream)))
     return Y
+
+
+def gptq_2d_round(X: torch.Tensor, U_left: torch.Tensor, U_right: torch.Tensor, Z: torch.Tensor | None = None,
+                  workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """GPTQ-2D two-sided rounding.  X: float64 [m, n] or [batch, m, n]; U_left float64 [m, m],
+    U_right float64 [n, n] (upper Cholesky factors of the inverse Grams); returns Z int32 of
+    X's shape."""
+    if X.dim() not in (2, 3):
+        raise ValueError("X must be [m, n] or [batch, m, n]")
+    batch = 1 if X.dim() == 2 else X.shape[0]
+    m, n = X.shape[-2], X.shape[-1]
+    _need(X, torch.float64, tuple(X.shape), "X")
+    _need(U_left, torch.float64, (m, m), "U_left")
+    _need(U_right, torch.float64, (n, n), "U_right")
+    if Z is None:
+        Z = torch.empty(X.shape, dtype=torch.int32, device=X.device)
+    _need(Z, torch.int32, tuple(X.shape), "Z")
+    need = lib().gptq_2d_workspace_bytes(m, n, batch)
+    ws = workspace if workspace is not None else _workspace(need, X.device)
+    _check(lib().gptq_2d_round(_ptr(X), m, n, batch, _ptr(U_left), _ptr(U_right), _ptr(Z), _ptr(ws), ws.numel(),
+                               _stream(stream)))
+    return Z
 
 
 def gptq_pack_int(codes: torch.Tensor, bits: int, layout: int, packed: torch.Tensor, stream=None) -> torch.Tensor:

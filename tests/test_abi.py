@@ -244,3 +244,19 @@ def test_whole_layer_calls_refuse_arguments_that_conflict_with_the_buffers():
     assert (d.bits, d.group_size, d.sym, d.desc_act) == (4, 128, 0, 0)
     e = G._resolve_config(None, 2, 32, None, None, 2)
     assert (e.bits, e.group_size, e.sym, e.desc_act) == (2, 32, 0, 2)
+
+
+def test_gptq2d_entry_validates_before_any_call():
+    L = G.lib()
+    ws = L.gptq_2d_workspace_bytes(64, 64, 1)
+    assert ws >= 64 * 64 * 8
+    assert L.gptq_2d_workspace_bytes(200, 150, 3) >= 200 * 200 * 8 + 3 * 200 * 150 * 8
+    assert L.gptq_2d_workspace_bytes(0, 5, 1) == 0
+    ok = lambda m=8, n=8, b=1, X=_fake(1), Z=_fake(4), wsb=1 << 30: L.gptq_2d_round(X, m, n, b, _fake(2), _fake(3), Z,
+                                                                                     _fake(5), wsb, None)
+    assert ok(m=0) == G.GPTQ_ERR_INVALID_ARG
+    assert ok(n=20000) == G.GPTQ_ERR_INVALID_ARG
+    assert ok(b=0) == G.GPTQ_ERR_INVALID_ARG
+    assert ok(X=None) == G.GPTQ_ERR_INVALID_ARG
+    assert ok(X=ctypes.c_void_p(0x1004)) == G.GPTQ_ERR_INVALID_ARG      # misaligned fp64
+    assert ok(wsb=16) == G.GPTQ_ERR_WORKSPACE

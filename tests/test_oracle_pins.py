@@ -549,30 +549,14 @@ def test_gptq2d_bruteforce_bracket(seed):
     assert got <= bound + 1e-12
 
 
-def _antidiagonal_rounding(X, U_left, U_right):
-    """The summary's cubic route ("方法" steps 1-3): anti-diagonals i + j = k in increasing k,
-    all entries of one anti-diagonal rounded together from corrections of the entries
-    before it, then their errors pushed forward through the two Cholesky factors.
-    T = E U_right accumulates the errors, so a correction is a length-m dot product."""
-    m, n = X.shape
-    Z = np.zeros((m, n))
-    T = np.zeros((m, n))
-    for k in range(m + n - 1):
-        diag = [(i, k - i) for i in range(max(0, k - n + 1), min(m, k + 1))]
-        vals = [X[i, j] - U_left[:, i] @ T[:, j] for i, j in diag]      # all before any update
-        for (i, j), v in zip(diag, vals):
-            Z[i, j] = np.rint(v)
-            e = (v - Z[i, j]) / (U_left[i, i] * U_right[j, j])
-            T[i, :] += e * U_right[j, :]
-    return Z
-
-
-@pytest.mark.parametrize("seed,m,n", [(110, 5, 7), (111, 8, 3), (112, 6, 6), (113, 1, 9), (114, 9, 1)])
+@pytest.mark.parametrize("seed,m,n", [(110, 5, 7), (111, 8, 3), (112, 6, 6), (113, 1, 9), (114, 9, 1),
+                                      (115, 12, 10), (116, 16, 3)])
 def test_gptq2d_antidiagonal_route_gives_the_same_integers(seed, m, n):
-    # the summary's claim the cubic route relies on: identical output to the quartic one
+    # the summary's claim ("方法", "核心洞察"): the anti-diagonal route gives exactly the
+    # integers of the quartic vectorized route
     X, G_left, G_right, _, _ = _problem2d(seed, m, n)
     Z = O.gptq2d_vectorized(X, G_left, G_right)
-    Zad = _antidiagonal_rounding(X, O.hinv_upper_cholesky(G_left), O.hinv_upper_cholesky(G_right))
+    Zad = O.gptq2d_antidiagonal(X, O.hinv_upper_cholesky(G_left), O.hinv_upper_cholesky(G_right))
     np.testing.assert_array_equal(Z, Zad)
 
 
