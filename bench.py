@@ -212,7 +212,8 @@ CHOL_KERNELS = ("chol_leaf", "chol_panel", "chol_chain_r", "chol_chain_d", "chol
                 "chol_update_u2", "inv_bu", "inv_ub",
                 "split_panel",
                 "damp_copy", "diag_mean", "zero_lower", "chol_diag_out", "perm_invert", "damp_copy_perm")
-QUANT_KERNELS = ("colloop", "trailing_update", "trailing_update_sb", "up_prep", "ut_split", "pack_zeros", "row_params",
+QUANT_KERNELS = ("colloop", "trailing_update", "trailing_update_wide", "trailing_update_sb", "up_prep", "ut_split",
+                 "tc_un_prep", "tc_ut_prep", "pack_zeros", "row_params",
                  "gather_cols", "unpermute_codes")
 ACT_KERNELS = ("act_sum", "act_rank", "act_perm")   # activation ordering (--desc-act 1 or 2)
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu --set full capture of this
@@ -486,6 +487,8 @@ def main():
                     help="stack7b: q/k/v and gate/up share one H and U per group (one input each)")
     ap.add_argument("--desc-act", type=int, default=0, choices=[0, 1, 2],
                     help="activation ordering: 0 natural column order, 1 ascending, 2 descending sum of |x|")
+    ap.add_argument("--timeline", default="",
+                    help="write the per-launch timeline of the instrumented steps (JSON) to this file")
     ap.add_argument("--rank-probe", action="store_true",
                     help="launch check only: the ranks join a gloo group and rank 0 reports the world size")
     args = ap.parse_args()
@@ -550,10 +553,9 @@ def run_gpu(args, world: int, rank: int, local: int) -> None:
             G.gptq_act_order(bufs.act, cfg.desc_act, bufs.perm, bufs.rank)
         if marks:
             marks[0].record(stream)
-        if cfg.desc_act:
-            G.gptq_prepare_hinv_permuted(bufs.H, bufs.perm, bufs.U, cfg.damp_rel, workspace=bufs.ws)
-        else:
-            G.gptq_prepare_hinv(bufs.H, bufs.U, cfg.damp_rel, workspace=bufs.ws)
+        # enqueued without host synchronisation (errors are read once after the timed steps)
+        G.gptq_prepare_hinv_async(bufs.H, bufs.U, cfg.damp_rel, workspace=bufs.ws, lam=bufs.lam,
+                                  perm=bufs.perm if cfg.desc_act else None)
         if marks:
             marks[1].record(stream)
         if cfg.desc_act:
@@ -605,7 +607,11 @@ def run_gpu(args, world: int, rank: int, local: int) -> None:
         flush.fill_(1)
         step()
     kt = G.gptq_timing_report()
+    timeline = G.gptq_timing_timeline()
     G.gptq_timing_enable(False)
+    if args.timeline:
+        with open(args.timeline, "w") as f:
+            json.dump(timeline, f)
     launches_per_step = sum(c for c, _ in kt.values()) / reps
     kernel_ms = {k: ms / reps for k, (c, ms) in kt.items()}
     kernel_launches = {k: c // reps for k, (c, ms) in kt.items()}

@@ -131,6 +131,15 @@ gptq_status gptq_prepare_hinv(const float* H, int64_t d_in, float damp_rel, floa
                               void* ws, size_t ws_bytes, int64_t* bad_col, float* lambda_out,
                               void* stream);
 
+/* gptq_prepare_hinv without any host synchronisation: the same U, enqueued on ``stream``
+ * and returned at once, so that a whole layer (stages 1-3) can be enqueued without a
+ * round trip to the host.  lambda_dev (device float, or NULL) receives lambda on the
+ * stream.  A non-positive pivot, a non-finite value or a zero Hessian is reported by the
+ * next gptq_sync_status() (GPTQ_ERR_NOT_PD / NONFINITE / INVALID_ARG, with the column
+ * in gptq_last_error()); until then U is undefined.  Arguments as gptq_prepare_hinv. */
+gptq_status gptq_prepare_hinv_async(const float* H, int64_t d_in, float damp_rel, float* U,
+                                    void* ws, size_t ws_bytes, float* lambda_dev, void* stream);
+
 /* ------------------------------------------------------------------ stage 3
  * GPTQ column loop (tutorial "阶段二", "阶段三"; group-size article).
  *   W        device, d_out x d_in fp32 row-major; consumed as scratch (holds the
@@ -199,6 +208,10 @@ gptq_status gptq_act_order(const double* act, int64_t d_in, int desc_act, int32_
  * gptq_prepare_hinv_workspace_bytes(d_in). */
 gptq_status gptq_prepare_hinv_permuted(const float* H, const int32_t* perm, int64_t d_in, float damp_rel, float* U,
                                        void* ws, size_t ws_bytes, int64_t* bad_col, float* lambda_out, void* stream);
+/* The same without host synchronisation (see gptq_prepare_hinv_async); an invalid perm is
+ * reported by the next gptq_sync_status(). */
+gptq_status gptq_prepare_hinv_permuted_async(const float* H, const int32_t* perm, int64_t d_in, float damp_rel,
+                                             float* U, void* ws, size_t ws_bytes, float* lambda_dev, void* stream);
 
 /* gptq_quantize_layer_act_order: the column loop of gptq_quantize_layer on the columns in
  * the order perm; cfg->desc_act must be 1 or 2 (the order itself is the one in perm).
@@ -272,9 +285,16 @@ gptq_status gptq_sync_status(void* stream);
  * gptq_selftest_bounded_wait: launches one thread that waits on a barrier nobody
  * arrives at, with a limit of limit_ns nanoseconds, the same bounded wait every
  * pipeline in the library uses; the next gptq_sync_status() returns GPTQ_ERR_TIMEOUT.
- * Used to test the timeout path without faulting or hanging the device. */
+ * Used to test the timeout path without faulting or hanging the device.
+ *
+ * gptq_timing_timeline: the same recorded launches as a JSON list
+ * [["kernel_name", stream_index, start_ms, end_ms], ...] in launch order, times from the
+ * first recorded launch; start is when the launch's stream reached it (the previous work
+ * in that stream done), end when it finished.  Collects, clears and sizes like
+ * gptq_timing_report. */
 void gptq_timing_enable(int on);
 size_t gptq_timing_report(char* buf, size_t len);
+size_t gptq_timing_timeline(char* buf, size_t len);
 gptq_status gptq_selftest_bounded_wait(uint64_t limit_ns, void* stream);
 
 /* ------------------------------------------------------------------ no-allocation variant

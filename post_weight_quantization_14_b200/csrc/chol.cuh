@@ -11,10 +11,9 @@
 //     leaf(j):   R_jj = UL-Cholesky(A_jj), X_jj = R_jj^-1           (one CTA, fp32)
 //     panel(j):  R_{0:j, j} = A_{0:j, j} X_jj^T                      (3xTF32 tcgen05)
 //     update(j): A_{0:j, 0:j} -= R_{0:j, j} R_{0:j, j}^T             (3xTF32 tcgen05)
-//   scheduled on three streams: the chain carries leaf(j) and, for the next leaf, only the
-//   128x128 products R_{j-1,j} and A_{j-1,j-1} -= R_{j-1,j} R_{j-1,j}^T; a high-priority
-//   stream the rest of the panel and block columns j-1 and j-2; a low-priority stream the
-//   Schur update of the block columns left of them (look-ahead of depth two).
+//   with the update split three ways: block column j-1 on the critical chain (a stream of
+//   the highest priority), then block column j-2 and the rest on a low-priority stream
+//   (look-ahead of depth two).
 //   and U = R^-1 by doubling on a fourth stream, each product as soon as its inputs exist:
 //   for each diagonal pair [[R_a, B], [0, R_c]] of 128, 256, ... columns with known
 //   inverses U_a, U_c:  U_b = -U_a (B U_c).
@@ -145,8 +144,8 @@ __global__ void __launch_bounds__(256) zero_lower_blocks_kernel(float* __restric
 // Right-looking, blocked by 32 columns.  For panel kb (columns k0 = 32 kb .. k0 + 31):
 //   A. one warp factors the 32x32 diagonal block in registers, lane = row.  The only
 //      dependency from one pivot to the next is one shuffle of the next pivot, which each
-//      lane keeps up to date from its own multipliers (the broadcasts of the multipliers to
-//      the other rows are off that chain); 1/L_kk = rsqrt with one Newton step.
+//      lane keeps up to date from its own multipliers; the multiplier column reaches the
+//      other rows through shared memory, off that chain; 1/L_kk = rsqrt with one Newton step.
 //   B. the rows below the block (one thread per row, 32 - 96 rows) solve against L_kk by
 //      substitution with the reciprocals of step A; meanwhile one otherwise idle warp forms
 //      X_kk = L_kk^-1 by forward substitution (lane = column).
@@ -167,11 +166,15 @@ struct LeafSmem {
     float LT[NB][LS];        // L transposed: LT[m][r] = L[r][m]
     float XDT[4][32][36];    // diagonal inverses transposed: XDT[i][m][r] = X_ii[r][m]
     float rinv[NB];          // 1 / L_kk
+    float col[2][32];        // multiplier column of the current pivot (double-buffered)
 };
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
 // A. Factor the 32x32 diagonal block at (k0, k0) with one warp; lane i holds row k0 + i.
+// Per pivot k the pivot value is the only shuffle on the dependency chain (each lane keeps
+// its own diagonal entry current); the multipliers L_jk reach the other rows through a
+// double-buffered column in shared memory (one store, a warp barrier and vector loads).
 // Writes L_kk (lower, zeros above) to P and LT, and 1/L_kk to rinv.
 __device__ __forceinline__ void leaf_diag_factor(LeafSmem& S, int k0, int lane, int jb) {
     constexpr unsigned FULL = 0xffffffffu;
@@ -184,27 +187,40 @@ __device__ __forceinline__ void leaf_diag_factor(LeafSmem& S, int k0, int lane, 
         a[4 * j4 + 2] = v.z;
         a[4 * j4 + 3] = v.w;
     }
-    // this lane's diagonal entry, kept current with the lane's own multipliers
-    float dg = 0.f;
+    float dg = 0.f;   // this lane's diagonal entry, kept current with its own multipliers
 #pragma unroll
     for (int j = 0; j < 32; ++j) dg = (lane == j) ? a[j] : dg;
+    int bad = -1;     // first pivot that is not positive and finite
+    float bad_p = 0.f, rr = 0.f;
 #pragma unroll
     for (int k = 0; k < 32; ++k) {
         const float p = __shfl_sync(FULL, dg, k);   // pivot: P_kk after pivots 0..k-1
-        if (lane == 0 && !(p > 0.f && isfinite(p)))
-            record_status(isfinite(p) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE, jb + 127 - (k0 + k));
+        const bool pk = p > 0.f && isfinite(p);
+        bad_p = (bad < 0 && !pk) ? p : bad_p;
+        bad = (bad < 0 && !pk) ? k : bad;
         float r = rsqrtf(p);
         r = r * fmaf(-0.5f * p * r, r, 1.5f);       // one Newton step for 1/sqrt(p)
         const float l = (lane == k) ? p * r : a[k] * r;   // L_kk = sqrt(p); L_ik = P_ik / L_kk
         a[k] = l;
         if (lane > k) dg = fmaf(-l, l, dg);
-        if (lane == k) S.rinv[k0 + k] = r;
+        rr = (lane == k) ? r : rr;
+        if (k < 31) {
+            float* cb = S.col[k & 1];
+            cb[lane] = l;
+            __syncwarp();
 #pragma unroll
-        for (int j = k + 1; j < 32; ++j) {
-            const float lj = __shfl_sync(FULL, l, j);
-            a[j] = fmaf(-l, lj, a[j]);              // P_ij -= L_ik L_jk (meaningful for lanes >= j)
+            for (int j4 = (k + 1) >> 2; j4 < 8; ++j4) {
+                const float4 c4 = ld4(&cb[4 * j4]);    // L_jk for j = 4 j4 ..
+                if (4 * j4 + 0 > k) a[4 * j4 + 0] = fmaf(-l, c4.x, a[4 * j4 + 0]);
+                if (4 * j4 + 1 > k) a[4 * j4 + 1] = fmaf(-l, c4.y, a[4 * j4 + 1]);
+                if (4 * j4 + 2 > k) a[4 * j4 + 2] = fmaf(-l, c4.z, a[4 * j4 + 2]);
+                if (4 * j4 + 3 > k) a[4 * j4 + 3] = fmaf(-l, c4.w, a[4 * j4 + 3]);
+            }
         }
     }
+    if (lane == 0 && bad >= 0)
+        record_status(isfinite(bad_p) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE, jb + 127 - (k0 + bad));
+    S.rinv[k0 + lane] = rr;
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         const float v = (j <= lane) ? a[j] : 0.f;
@@ -451,7 +467,7 @@ struct HinvWs {
 
 inline size_t hinv_ws_bytes(long long d) {
     const long long n = chol_n(d);
-    return (size_t)(9 * n * n + 4 * n * gq::NB + 64 + n) * sizeof(float);
+    return (size_t)(9 * n * n + 2 * n * gq::NB + 64 + n) * sizeof(float);
 }
 
 inline HinvWs hinv_ws_carve(void* ws, long long d) {
@@ -476,10 +492,10 @@ inline HinvWs hinv_ws_carve(void* ws, long long d) {
     p += n * n;
     w.TT_lo = p;
     p += n * n;
-    w.AP_hi = p;   // two panel splits (block columns of either parity), n x 128 each
-    p += 2 * n * gq::NB;
+    w.AP_hi = p;   // tf32 split of the next panel, n x 128
+    p += n * gq::NB;
     w.AP_lo = p;
-    p += 2 * n * gq::NB;
+    p += n * gq::NB;
     w.scal = p;
     p += 64;
     w.rank = reinterpret_cast<int*>(p);
@@ -522,20 +538,18 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
     const int leaf_smem = (int)sizeof(gq::LeafSmem);
     GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::chol_leaf_kernel), leaf_smem));
     const uint64_t N = (uint64_t)n;
-    // Streams.  The chain stream carries, per block column j, only what the next leaf needs:
-    //   leaf(j) -> C1: R_{j-1,j} = A_{j-1,j} X_jj^T (one 128x128 block of the panel)
-    //           -> C2: A_{j-1,j-1} -= R_{j-1,j} R_{j-1,j}^T        -> leaf(j-1).
-    // The near stream: P, the rest of the panel (rows 0 .. j-2); N, block column j-1 above its
-    // diagonal block (and the tf32 split of the next panel); U2, block column j-2 with its
-    // diagonal block.  The far stream: R, the Schur update of block columns 0 .. j-3.
-    // Every block is updated in step order: C1(j) reads the panel split N(j+1) wrote; C2(j)
-    // follows U2(j+1) on block (j-1, j-1); U2(j) follows R(j+1) on block column j-2.
+    // Streams.  The chain stream (highest priority) carries, per block column j,
+    //   leaf(j) -> panel(j): R_{0:j,j} = A_{0:j,j} X_jj^T
+    //           -> block column j-1 updated by panel j (and the next panel's tf32 split).
+    // The far stream takes the rest of panel j's Schur update: first block column j-2 (u2),
+    // then everything left of it (rest).  Block column j-1 has received, before its update by
+    // panel j, u2(j+1) and rest(p) for p >= j+2, which the far stream runs in that order, so
+    // the chain waits only for u2(j+1).  The inverse stream runs the doubling products.
     FactStreams fs;
     if (!fact_streams(&fs)) return cudaErrorUnknown;
-    cudaEvent_t ev_start = fs.ev[0], ev_leaf = fs.ev[1], ev_P = fs.ev[2], ev_C1 = fs.ev[3], ev_N = fs.ev[4],
-                ev_U2 = fs.ev[5], ev_R = fs.ev[6], ev_near = fs.ev[7], ev_far = fs.ev[8], ev_chain = fs.ev[9],
-                ev_inv = fs.ev[10];
-    cudaStream_t sc = fs.chain, sn = fs.near, sf = fs.far, si = fs.inv;
+    cudaEvent_t ev_start = fs.ev[0], ev_leaf = fs.ev[1], ev_panel = fs.ev[2], ev_u2 = fs.ev[5],
+                ev_far = fs.ev[8], ev_chain = fs.ev[9], ev_inv = fs.ev[10];
+    cudaStream_t sc = fs.chain, sf = fs.far, si = fs.inv;
     {
         gqh::TimedScope ts__("zero_lower", st);   // the public U's strictly lower blocks
         const unsigned nb = (unsigned)((d + gq::NB - 1) / gq::NB);
@@ -544,49 +558,12 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
     GQ_TRY(cudaGetLastError());
     GQ_TRY(cudaEventRecord(ev_start, st));
     GQ_TRY(cudaStreamWaitEvent(sc, ev_start, 0));
-    GQ_TRY(cudaStreamWaitEvent(sn, ev_start, 0));
     GQ_TRY(cudaStreamWaitEvent(sf, ev_start, 0));
     GQ_TRY(cudaStreamWaitEvent(si, ev_start, 0));
-    const int side = std::max(1, num_sms() - 8);   // helper grids leave SMs to the chain
+    const int far_ctas = std::max(1, num_sms() - 1);            // leave an SM for the next leaf
+    const int inv_ctas = std::max(1, num_sms() / 4);            // the inverse fills in around the chain
     Mat rh{w.RS_hi, N, N, N}, rl{w.RS_lo, N, N, N};
     Mat xh{w.U_hi, N, N, N}, xl{w.U_lo, N, N, N};
-    float* ap_hi[2] = {w.AP_hi, w.AP_hi + n * gq::NB};
-    float* ap_lo[2] = {w.AP_lo, w.AP_lo + n * gq::NB};
-    // C -= RS(rows a_row0 ..) RS(rows b_row0 ..)^T over the panel of block column j
-    auto schur = [&](int jb, int M, int Ncols, int b_row0, int c_row0, int c_col0, bool tri, cudaStream_t s_,
-                     const char* name, int max_ctas, const EpiMats* extra_s, bool after) -> cudaError_t {
-        gq::GemmArgs p = gemm_args(M, Ncols, gq::NB);
-        p.a_row0 = c_row0;
-        p.a_col0 = jb;
-        p.b_row0 = b_row0;
-        p.b_col0 = jb;
-        p.alpha = -1.f;
-        p.beta = 1.f;
-        p.write_c = 1;
-        p.c_row0 = c_row0;
-        p.c_col0 = c_col0;
-        p.triangular = tri ? 1 : 0;
-        EpiMats o;
-        if (extra_s) o = *extra_s;
-        o.c = Mat{w.A, N, N, N};
-        if (tri) return launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rh, rl, rh, rl, o, p, 1, s_, name, max_ctas, after);
-        return launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, rh, rl, o, p, 1, s_, name, max_ctas, after);
-    };
-    // RS(rows r0 .. r0+M, block column j) = AP(rows r0 ..) X_jj^T
-    auto panel = [&](int jb, int r0, int M, cudaStream_t s_, const char* name, int max_ctas, bool after) {
-        const int par = (jb / gq::NB) & 1;
-        gq::GemmArgs p = gemm_args(M, gq::NB, gq::NB);
-        p.a_row0 = r0;
-        p.b_row0 = jb;
-        p.b_col0 = jb;
-        p.s_row0 = r0;
-        p.s_col0 = jb;
-        EpiMats o;
-        o.s_hi = Mat{w.RS_hi, N, N, N};
-        o.s_lo = Mat{w.RS_lo, N, N, N};
-        Mat ah{ap_hi[par], (uint64_t)jb, 128, 128}, al{ap_lo[par], (uint64_t)jb, 128, 128};
-        return launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(ah, al, xh, xl, o, p, 1, s_, name, max_ctas, after);
-    };
     // U = R^-1 by doubling, each product issued on the inverse stream as soon as its inputs
     // exist: for the diagonal pair [[R_a, B], [0, R_c]] of level s (a-half rows r0 .. r0+s,
     // c-half r0+s .. r0+s+cs) with inverses U_a and U_c known, T = B U_c (stored transposed) as
@@ -610,8 +587,8 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
         o.t_hi = Mat{w.TT_hi, N, N, N};
         o.t_lo = Mat{w.TT_lo, N, N, N};
         const bool narrow = 4 * (s_ / gq::NB) * ((cs + gq::NB - 1) / gq::NB) <= num_sms();
-        if (narrow) return launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, uth, utl, o, p, 1, si, "inv_bu", side, true);
-        return launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rh, rl, uth, utl, o, p, 1, si, "inv_bu", side, true);
+        if (narrow) return launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, uth, utl, o, p, 1, si, "inv_bu", inv_ctas, true);
+        return launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rh, rl, uth, utl, o, p, 1, si, "inv_bu", inv_ctas, true);
     };
     auto inv_ub = [&](long long s_, long long r0, long long cs) -> cudaError_t {   // U_b = -U_a T
         gq::GemmArgs p = gemm_args((int)s_, (int)cs, (int)s_);
@@ -634,14 +611,16 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
         o.s_lo = Mat{w.U_lo, N, N, N};
         o.t_hi = Mat{w.UT_hi, N, N, N};
         o.t_lo = Mat{w.UT_lo, N, N, N};
+        // the pairs that contain block 0 are the tail after the last leaf: all SMs
+        const int cap = r0 == 0 ? 0 : inv_ctas;
         const bool narrow = 4 * (s_ / gq::NB) * ((cs + gq::NB - 1) / gq::NB) <= num_sms();
-        if (narrow) return launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(xh, xl, tth, ttl, o, p, 1, si, "inv_ub", side, true);
-        return launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(xh, xl, tth, ttl, o, p, 1, si, "inv_ub", side, true);
+        if (narrow) return launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(xh, xl, tth, ttl, o, p, 1, si, "inv_ub", cap, true);
+        return launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(xh, xl, tth, ttl, o, p, 1, si, "inv_ub", cap, true);
     };
-    // the inverse work that becomes possible once leaf(j) and the panels of block column j exist
-    auto inverse_step = [&](int j) -> cudaError_t {
+    // the inverse work that becomes possible once leaf(j) and panel(j) are done (event ev)
+    auto inverse_step = [&](int j, cudaEvent_t ev) -> cudaError_t {
         const long long jb = (long long)j * gq::NB;
-        GQ_TRY(cudaStreamWaitEvent(si, ev_leaf, 0));
+        GQ_TRY(cudaStreamWaitEvent(si, ev, 0));
         {
             gqh::TimedScope ts__("chol_diag_out", si);
             gq::chol_diag_out_kernel<<<1, 512, dout_smem, si>>>(w.U_hi, w.U_lo, w.UT_hi, w.UT_lo, U, n, d, j);
@@ -649,18 +628,13 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
         GQ_TRY(cudaGetLastError());
         for (long long s_ = gq::NB; s_ < n; s_ *= 2)   // pairs whose a-half starts at block j
             if (jb % (2 * s_) == 0 && jb + s_ < n) GQ_TRY(inv_ub(s_, jb, std::min(s_, n - jb - s_)));
-        if (j > 0) {
-            GQ_TRY(cudaStreamWaitEvent(si, ev_P, 0));
-            GQ_TRY(cudaStreamWaitEvent(si, ev_C1, 0));
-        }
         for (long long s_ = gq::NB; s_ < n; s_ *= 2)   // pairs whose c-half starts at block j
             if (jb >= s_ && (jb - s_) % (2 * s_) == 0) GQ_TRY(inv_bu(s_, jb - s_, std::min(s_, n - jb)));
         return cudaSuccess;
     };
+    bool u2_pending = false;
     for (int j = T - 1; j >= 0; --j) {
         const int jb = j * gq::NB;
-        const int jn = jb - gq::NB;    // first column of block column j-1
-        const int jn2 = jn - gq::NB;   // first column of block column j-2
         {
             gqh::TimedScope ts__("chol_leaf", sc);
             if (j == T - 1)   // follows the wait for the damped copy on the caller's stream
@@ -672,55 +646,90 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
         }
         if (j == 0) {
             GQ_TRY(cudaEventRecord(ev_leaf, sc));
-            GQ_TRY(inverse_step(0));
+            GQ_TRY(inverse_step(0, ev_leaf));
             break;
         }
-        if (j == T - 1) {   // the first panel's tf32 split; later ones come from N
+        if (j == T - 1) {   // later panels are split by the previous update's epilogue
             gqh::TimedScope ts__("split_panel", sc);
             gq::split_panel_kernel<<<(unsigned)std::min<long long>((jb * 128LL + 255) / 256, 4096), 256, 0, sc>>>(
-                w.A, n, jb, jb, ap_hi[j & 1], ap_lo[j & 1]);
+                w.A, n, jb, jb, w.AP_hi, w.AP_lo);
             GQ_TRY(cudaGetLastError());
         }
-        GQ_TRY(cudaEventRecord(ev_leaf, sc));
-        // near stream: the panel's rows 0 .. j-2
-        GQ_TRY(cudaStreamWaitEvent(sn, ev_leaf, 0));
-        if (jn > 0) GQ_TRY(panel(jb, 0, jn, sn, "chol_panel", side, true));
-        GQ_TRY(cudaEventRecord(ev_P, sn));
-        // chain: C1, C2
-        GQ_TRY(cudaStreamWaitEvent(sc, ev_N, 0));
-        GQ_TRY(panel(jb, jn, gq::NB, sc, "chol_chain_r", 0, true));
-        GQ_TRY(cudaEventRecord(ev_C1, sc));
-        GQ_TRY(cudaStreamWaitEvent(sc, ev_U2, 0));
-        GQ_TRY(schur(jb, gq::NB, gq::NB, jn, jn, jn, false, sc, "chol_chain_d", 0, nullptr, true));
-        if (jn > 0) {
-            // near stream: N(j) = block column j-1 above its diagonal block + the next panel's split
-            GQ_TRY(cudaStreamWaitEvent(sn, ev_C1, 0));
-            EpiMats so;
-            so.s_hi = Mat{ap_hi[(j - 1) & 1], (uint64_t)jn, 128, 128};
-            so.s_lo = Mat{ap_lo[(j - 1) & 1], (uint64_t)jn, 128, 128};
-            GQ_TRY(schur(jb, jn, gq::NB, jn, 0, jn, false, sn, "chol_update_next", side, &so, true));
-            GQ_TRY(cudaEventRecord(ev_N, sn));
-            // U2(j) = block column j-2, rows 0 .. j-2 (with its diagonal block), after R(j+1)
-            if (jn2 >= 0) {
-                GQ_TRY(cudaStreamWaitEvent(sn, ev_R, 0));
-                GQ_TRY(schur(jb, jn, gq::NB, jn2, 0, jn2, false, sn, "chol_update_u2", side, nullptr, true));
+        {   // panel: RS[0:jb, jb:jb+128] = AP * X^T, X = U block (row-major split)
+            gq::GemmArgs p = gemm_args(jb, gq::NB, gq::NB);
+            p.b_row0 = jb;
+            p.b_col0 = jb;
+            p.s_col0 = jb;
+            EpiMats o;
+            o.s_hi = Mat{w.RS_hi, N, N, N};
+            o.s_lo = Mat{w.RS_lo, N, N, N};
+            Mat ah{w.AP_hi, (uint64_t)jb, 128, 128}, al{w.AP_lo, (uint64_t)jb, 128, 128};
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(ah, al, xh, xl, o, p, 1, sc, "chol_panel", 0,
+                                                        j == T - 1)));
+        }
+        const int jn = jb - gq::NB;    // first column of block column j-1
+        const int jn2 = jn - gq::NB;   // first column of block column j-2
+        GQ_TRY(cudaEventRecord(ev_panel, sc));
+        const bool waited = u2_pending;
+        if (u2_pending) GQ_TRY(cudaStreamWaitEvent(sc, ev_u2, 0));
+        {   // block column j-1: A[0:jb, jn:jb] -= RS_panel RS_panel[jn:jb]^T, plus the next panel's split
+            gq::GemmArgs p = gemm_args(jb, gq::NB, gq::NB);
+            p.a_col0 = jb;
+            p.b_row0 = jn;
+            p.b_col0 = jb;
+            p.alpha = -1.f;
+            p.beta = 1.f;
+            p.write_c = 1;
+            p.c_col0 = jn;
+            EpiMats o;
+            o.c = Mat{w.A, N, N, N};
+            if (j >= 2) {   // tiles above the diagonal block write the next panel's tf32 split
+                p.s_mt_lim = j - 1;
+                o.s_hi = Mat{w.AP_hi, (uint64_t)jn, 128, 128};
+                o.s_lo = Mat{w.AP_lo, (uint64_t)jn, 128, 128};
             }
-            GQ_TRY(cudaEventRecord(ev_U2, sn));
-            // far stream: R(j) = block columns 0 .. j-3
-            if (jn2 > 0) {
-                GQ_TRY(cudaStreamWaitEvent(sf, ev_P, 0));
-                GQ_TRY(schur(jb, jn2, jn2, 0, 0, 0, true, sf, "chol_update", side, nullptr, true));
-                GQ_TRY(cudaEventRecord(ev_R, sf));
+            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, rh, rl, o, p, 1, sc, "chol_update_next", 0,
+                                                        waited)));
+        }
+        u2_pending = false;
+        if (j >= 2) {   // far stream: block column j-2, then the rest
+            GQ_TRY(cudaStreamWaitEvent(sf, ev_panel, 0));
+            {   // u2: A[0:jn, jn2:jn] -= RS_panel RS_panel[jn2:jn]^T
+                gq::GemmArgs p = gemm_args(jn, gq::NB, gq::NB);
+                p.a_col0 = jb;
+                p.b_row0 = jn2;
+                p.b_col0 = jb;
+                p.alpha = -1.f;
+                p.beta = 1.f;
+                p.write_c = 1;
+                p.c_col0 = jn2;
+                EpiMats o;
+                o.c = Mat{w.A, N, N, N};
+                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, rh, rl, o, p, 1, sf, "chol_update_u2",
+                                                            far_ctas, true)));
+            }
+            GQ_TRY(cudaEventRecord(ev_u2, sf));
+            u2_pending = true;
+            if (j >= 3) {   // rest: A[0:jn2, 0:jn2] -= RS RS^T (upper tiles)
+                gq::GemmArgs p = gemm_args(jn2, jn2, gq::NB);
+                p.a_col0 = jb;
+                p.b_col0 = jb;
+                p.triangular = 1;
+                p.alpha = -1.f;
+                p.beta = 1.f;
+                p.write_c = 1;
+                EpiMats o;
+                o.c = Mat{w.A, N, N, N};
+                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rh, rl, rh, rl, o, p, 1, sf, "chol_update",
+                                                       far_ctas, true)));
             }
         }
-        GQ_TRY(inverse_step(j));
+        GQ_TRY(inverse_step(j, ev_panel));
     }
     // all streams are done before the caller's stream continues
-    GQ_TRY(cudaEventRecord(ev_near, sn));
     GQ_TRY(cudaEventRecord(ev_far, sf));
     GQ_TRY(cudaEventRecord(ev_chain, sc));
     GQ_TRY(cudaEventRecord(ev_inv, si));
-    GQ_TRY(cudaStreamWaitEvent(st, ev_near, 0));
     GQ_TRY(cudaStreamWaitEvent(st, ev_far, 0));
     GQ_TRY(cudaStreamWaitEvent(st, ev_chain, 0));
     GQ_TRY(cudaStreamWaitEvent(st, ev_inv, 0));

@@ -17,7 +17,7 @@
 #include "hessian.cuh"
 #include "chol.cuh"
 #include "pack.cuh"
-#include "colloop.cuh"
+#include "colloop_host.cuh"
 #include "dqgemm.cuh"
 #include "gptq2d.cuh"
 
@@ -36,9 +36,17 @@ void set_last_error(const char* fmt, ...) {
 struct PendingLaunch {
     std::string name;
     cudaEvent_t a, b;
+    cudaStream_t st;
+};
+struct TimelineEntry {
+    std::string name;
+    int stream;
+    float t0, t1;   // ms from the first launch of the collected batch
 };
 static bool g_timing = false;
 static std::vector<PendingLaunch> g_pending;
+static std::vector<TimelineEntry> g_timeline;
+static std::vector<cudaStream_t> g_timeline_streams;
 static std::vector<cudaEvent_t> g_event_pool;
 static std::map<std::string, std::pair<long long, double>> g_timing_acc;
 
@@ -56,7 +64,7 @@ static cudaEvent_t pooled_event() {
 bool timing_on() { return g_timing; }
 
 void timing_begin(const char* name, cudaStream_t st) {
-    PendingLaunch p{name, pooled_event(), pooled_event()};
+    PendingLaunch p{name, pooled_event(), pooled_event(), st};
     cudaEventRecord(p.a, st);
     g_pending.push_back(p);
 }
@@ -67,12 +75,25 @@ void timing_end(cudaStream_t st) {
 
 static void timing_collect() {
     cudaDeviceSynchronize();
+    const cudaEvent_t ref = g_pending.empty() ? nullptr : g_pending.front().a;
     for (auto& p : g_pending) {
         float ms = 0.f;
         if (cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
             auto& acc = g_timing_acc[p.name];
             acc.first += 1;
             acc.second += ms;
+        }
+        float t0 = 0.f, t1 = 0.f;
+        if (g_timeline.size() < 100000 && cudaEventElapsedTime(&t0, ref, p.a) == cudaSuccess &&
+            cudaEventElapsedTime(&t1, ref, p.b) == cudaSuccess) {
+            int si = -1;
+            for (size_t k = 0; k < g_timeline_streams.size(); ++k)
+                if (g_timeline_streams[k] == p.st) si = (int)k;
+            if (si < 0) {
+                si = (int)g_timeline_streams.size();
+                g_timeline_streams.push_back(p.st);
+            }
+            g_timeline.push_back(TimelineEntry{p.name, si, t0, t1});
         }
         g_event_pool.push_back(p.a);
         g_event_pool.push_back(p.b);
@@ -152,7 +173,6 @@ bool fact_streams(FactStreams* fs) {
         if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return false;
         FactStreams f{};
         if (cudaStreamCreateWithPriority(&f.chain, cudaStreamNonBlocking, greatest) != cudaSuccess) return false;
-        if (cudaStreamCreateWithPriority(&f.near, cudaStreamNonBlocking, greatest) != cudaSuccess) return false;
         if (cudaStreamCreateWithPriority(&f.far, cudaStreamNonBlocking, least) != cudaSuccess) return false;
         if (cudaStreamCreateWithPriority(&f.inv, cudaStreamNonBlocking, least) != cudaSuccess) return false;
         for (auto& e : f.ev)
@@ -376,7 +396,39 @@ static gptq_status dequant_common(const int32_t* qweight, const uint16_t* scales
     return GPTQ_OK;
 }
 
+static gptq_status prepare_hinv_async_common(const float* H, const int32_t* perm, int64_t d_in, float damp_rel,
+                                             float* U, void* ws, size_t ws_bytes, float* lambda_dev, void* stream) {
+    if (!H || !U) return fail(GPTQ_ERR_INVALID_ARG, "H and U must be non-NULL");
+    if (d_in < 8 || d_in > 65536 || d_in % 8) return fail(GPTQ_ERR_INVALID_ARG, "d_in must be a multiple of 8 in [8, 65536]");
+    if (!(damp_rel >= 0.f) || damp_rel > 1e30f) return fail(GPTQ_ERR_INVALID_ARG, "damp_rel must be finite and >= 0");
+    if (!aligned16(H) || !aligned16(U)) return fail(GPTQ_ERR_INVALID_ARG, "H and U must be 16-byte aligned");
+    if (lambda_dev && (reinterpret_cast<uintptr_t>(lambda_dev) & 3u))
+        return fail(GPTQ_ERR_INVALID_ARG, "lambda_dev must be 4-byte aligned");
+    if (!ws || ws_bytes < hinv_ws_bytes(d_in) || !aligned16(ws))
+        return fail(GPTQ_ERR_WORKSPACE, "workspace needs %zu bytes", hinv_ws_bytes(d_in));
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = hinv_run(H, d_in, damp_rel, U, ws, st, perm);
+    if (e != cudaSuccess) return cuda_fail(e, "prepare_hinv");
+    if (lambda_dev) {
+        HinvWs w = hinv_ws_carve(ws, d_in);
+        e = cudaMemcpyAsync(lambda_dev, w.scal, sizeof(float), cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return cuda_fail(e, "lambda copy");
+    }
+    return GPTQ_OK;
+}
+
 extern "C" {
+
+gptq_status gptq_prepare_hinv_async(const float* H, int64_t d_in, float damp_rel, float* U, void* ws,
+                                    size_t ws_bytes, float* lambda_dev, void* stream) {
+    return prepare_hinv_async_common(H, nullptr, d_in, damp_rel, U, ws, ws_bytes, lambda_dev, stream);
+}
+
+gptq_status gptq_prepare_hinv_permuted_async(const float* H, const int32_t* perm, int64_t d_in, float damp_rel,
+                                             float* U, void* ws, size_t ws_bytes, float* lambda_dev, void* stream) {
+    if (!perm) return fail(GPTQ_ERR_INVALID_ARG, "perm must be non-NULL");
+    return prepare_hinv_async_common(H, perm, d_in, damp_rel, U, ws, ws_bytes, lambda_dev, stream);
+}
 
 gptq_status gptq_prepare_hinv(const float* H, int64_t d_in, float damp_rel, float* U, void* ws, size_t ws_bytes,
                               int64_t* bad_col, float* lambda_out, void* stream) {
@@ -600,6 +652,27 @@ size_t gptq_timing_report(char* buf, size_t len) {
         memcpy(buf, out.data(), n);
         buf[n] = 0;
         g_timing_acc.clear();
+    }
+    return out.size() + 1;
+}
+
+size_t gptq_timing_timeline(char* buf, size_t len) {
+    timing_collect();
+    std::string out = "[";
+    for (size_t k = 0; k < g_timeline.size(); ++k) {
+        char item[256];
+        const TimelineEntry& t = g_timeline[k];
+        snprintf(item, sizeof(item), "%s[\"%s\", %d, %.4f, %.4f]", k ? ", " : "", t.name.c_str(), t.stream,
+                 (double)t.t0, (double)t.t1);
+        out += item;
+    }
+    out += "]";
+    if (buf && len) {
+        const size_t n = std::min(len - 1, out.size());
+        memcpy(buf, out.data(), n);
+        buf[n] = 0;
+        g_timeline.clear();
+        g_timeline_streams.clear();
     }
     return out.size() + 1;
 }

@@ -10,19 +10,36 @@ namespace gq {
 
 constexpr int kHessNPad = 64;
 
-// 32x32 tiled transpose: XT[c, t] = X[t, c] for t < n, 0 for n <= t < n_pad.
-__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ X, long long n, long long d_in,
-                                      long long n_pad, uint16_t* __restrict__ XT) {
-    __shared__ uint16_t tile[32][33];
-    const long long t0 = (long long)blockIdx.x * 32, c0 = (long long)blockIdx.y * 32;
-    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
-        const long long t = t0 + r, c = c0 + threadIdx.x;
-        tile[r][threadIdx.x] = (t < n && c < d_in) ? X[t * d_in + c] : (uint16_t)0;
+// 64x64 tiled transpose: XT[c, t] = X[t, c] for t < n, 0 for n <= t < n_pad.  Both global
+// sides move 16-byte vectors (8 bf16) with a warp covering four whole 128-byte rows; the
+// shared tile [t][c] has 33-word rows, so the row-wise writes are conflict-free and the
+// column-wise reads at most 2-way.  d_in % 8 == 0 and n_pad % 64 == 0.
+constexpr int TR_T = 64, TR_C = 64, TR_LD = TR_C + 2;
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t* __restrict__ X, long long n,
+                                                             long long d_in, long long n_pad,
+                                                             uint16_t* __restrict__ XT) {
+    __shared__ __align__(16) uint16_t tile[TR_T][TR_LD];   // tile[t][c]
+    const long long t0 = (long long)blockIdx.x * TR_T, c0 = (long long)blockIdx.y * TR_C;
+    for (int e = threadIdx.x; e < TR_T * (TR_C / 8); e += blockDim.x) {
+        const int r = e >> 3, v8 = e & 7;
+        const long long t = t0 + r, c = c0 + 8 * v8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (t < n && c < d_in) v = *reinterpret_cast<const uint4*>(X + t * d_in + c);
+        uint32_t* dst = reinterpret_cast<uint32_t*>(&tile[r][8 * v8]);
+        dst[0] = v.x;
+        dst[1] = v.y;
+        dst[2] = v.z;
+        dst[3] = v.w;
     }
     __syncthreads();
-    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
-        const long long c = c0 + r, t = t0 + threadIdx.x;
-        if (c < d_in && t < n_pad) XT[c * n_pad + t] = tile[threadIdx.x][r];
+    for (int e = threadIdx.x; e < TR_C * (TR_T / 8); e += blockDim.x) {
+        const int cr = e >> 3, v8 = e & 7;
+        const long long c = c0 + cr, t = t0 + 8 * v8;
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            w[q] = (uint32_t)tile[8 * v8 + 2 * q][cr] | ((uint32_t)tile[8 * v8 + 2 * q + 1][cr] << 16);
+        if (c < d_in && t < n_pad) *reinterpret_cast<uint4*>(XT + c * n_pad + t) = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
@@ -68,6 +85,7 @@ inline cudaError_t hessian_run(const void* X, gptq_dtype xt, long long n, long l
     const long long np = hess_npad(n);
     dim3 tb(32, 8);
     dim3 grid((unsigned)(np / 32), (unsigned)((d_in + 31) / 32));
+    const dim3 grid64((unsigned)(np / gq::TR_T), (unsigned)((d_in + gq::TR_C - 1) / gq::TR_C));
     gq::GemmArgs p = gemm_args((int)d_in, (int)d_in, (int)np);
     p.triangular = 1;
     p.mirror = 1;
@@ -80,7 +98,7 @@ inline cudaError_t hessian_run(const void* X, gptq_dtype xt, long long n, long l
         uint16_t* XT = static_cast<uint16_t*>(ws);
         {
             gqh::TimedScope ts__(tname, st);
-            gq::transpose_bf16_kernel<<<grid, tb, 0, st>>>(static_cast<const uint16_t*>(X), n, d_in, np, XT);
+            gq::transpose_bf16_kernel<<<grid64, 256, 0, st>>>(static_cast<const uint16_t*>(X), n, d_in, np, XT);
         }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;

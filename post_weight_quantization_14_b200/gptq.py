@@ -57,6 +57,8 @@ _SIGS = {
     "gptq_prepare_hinv_workspace_bytes": (_sz, [_i64]),
     "gptq_prepare_hinv": (_int, [_vp, _i64, _f32, _vp, _vp, _sz, ctypes.POINTER(_i64),
                                  ctypes.POINTER(_f32), _vp]),
+    "gptq_prepare_hinv_async": (_int, [_vp, _i64, _f32, _vp, _vp, _sz, _vp, _vp]),
+    "gptq_prepare_hinv_permuted_async": (_int, [_vp, _vp, _i64, _f32, _vp, _vp, _sz, _vp, _vp]),
     "gptq_quantize_workspace_bytes": (_sz, [_i64, _i64, ctypes.POINTER(GptqConfig)]),
     "gptq_quantize_layer": (_int, [_vp, _vp, _i64, _i64, ctypes.POINTER(GptqConfig), _vp, _vp, _vp, _vp,
                                    _vp, _sz, _vp]),
@@ -65,6 +67,7 @@ _SIGS = {
     "gptq_sync_status": (_int, [_vp]),
     "gptq_timing_enable": (None, [_int]),
     "gptq_timing_report": (_sz, [ctypes.c_char_p, _sz]),
+    "gptq_timing_timeline": (_sz, [ctypes.c_char_p, _sz]),
     "gptq_selftest_bounded_wait": (_int, [ctypes.c_uint64, _vp]),
     "gptq_hessian_accumulate_fixed_scratch": (_int, [_vp, _int, _i64, _i64, _vp, _int, _vp]),
     "gptq_act_sum_accumulate": (_int, [_vp, _int, _i64, _i64, _vp, _int, _vp]),
@@ -214,6 +217,30 @@ def gptq_prepare_hinv(H: torch.Tensor, U: torch.Tensor, damp_rel: float = 0.01,
                                  ctypes.byref(bad), ctypes.byref(lam), _stream(stream))
     _check(st, bad.value)
     return float(lam.value)
+
+
+def gptq_prepare_hinv_async(H: torch.Tensor, U: torch.Tensor, damp_rel: float = 0.01,
+                            workspace: torch.Tensor | None = None, lam: torch.Tensor | None = None,
+                            perm: torch.Tensor | None = None, stream=None) -> None:
+    """U as gptq_prepare_hinv (of H[perm][:, perm] when perm is given) with no host
+    synchronisation; lam (float32 [1] on the device, optional) receives lambda.  Errors
+    surface at the next gptq_sync_status()."""
+    if H.dim() != 2:
+        raise ValueError("H must be a square float32 matrix")
+    d = H.shape[0]
+    _need(H, torch.float32, (d, d), "H")
+    _need(U, torch.float32, (d, d), "U")
+    if lam is not None:
+        _need(lam, torch.float32, (1,), "lam")
+    need = lib().gptq_prepare_hinv_workspace_bytes(d)
+    ws = workspace if workspace is not None else _workspace(need, H.device)
+    if perm is None:
+        _check(lib().gptq_prepare_hinv_async(_ptr(H), d, float(damp_rel), _ptr(U), _ptr(ws), ws.numel(), _ptr(lam),
+                                             _stream(stream)))
+    else:
+        _need(perm, torch.int32, (d,), "perm")
+        _check(lib().gptq_prepare_hinv_permuted_async(_ptr(H), _ptr(perm), d, float(damp_rel), _ptr(U), _ptr(ws),
+                                                      ws.numel(), _ptr(lam), _stream(stream)))
 
 
 def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, cfg: GptqConfig, qweight: torch.Tensor,
@@ -374,6 +401,16 @@ def gptq_timing_report() -> dict:
     return {k: (int(v[0]), float(v[1])) for k, v in json.loads(buf.value.decode()).items()}
 
 
+def gptq_timing_timeline() -> list:
+    """[(kernel, stream_index, start_ms, end_ms), ...] of the launches recorded since the last
+    collection (synchronises the device)."""
+    import json
+    n = lib().gptq_timing_timeline(None, 0)
+    buf = ctypes.create_string_buffer(n + 16)
+    lib().gptq_timing_timeline(buf, len(buf))
+    return [tuple(x) for x in json.loads(buf.value.decode())]
+
+
 def gptq_selftest_bounded_wait(limit_ns: int, stream=None) -> None:
     _check(lib().gptq_selftest_bounded_wait(int(limit_ns), _stream(stream)))
 
@@ -427,6 +464,7 @@ class LayerBuffers:
         self.cfg = cfg
         self.H = torch.empty((d_in, d_in), dtype=torch.float32, device=device)
         self.U = torch.empty((d_in, d_in), dtype=torch.float32, device=device)
+        self.lam = torch.zeros((1,), dtype=torch.float32, device=device)
         ws = max(L.gptq_hessian_workspace_bytes(n, d_in, xt), L.gptq_prepare_hinv_workspace_bytes(d_in),
                  L.gptq_quantize_workspace_bytes(d_out, d_in, ctypes.byref(cfg)))
         self.ws = _workspace(ws, device)
@@ -457,17 +495,21 @@ def quantize_layer(W: torch.Tensor, X: torch.Tensor, bits=None, group_size=None,
     cfg = _resolve_config(buffers, bits, group_size, sym, damp_rel, desc_act)
     d_out, d_in = W.shape
     b = buffers or LayerBuffers(d_out, d_in, X.shape[0], X.dtype, cfg, W.device)
+    # the three stages are enqueued without a host round trip; one synchronisation at the end
+    # reports any device-detected error (a non-positive pivot, non-finite values)
     gptq_hessian_accumulate(X, b.H, accumulate=False, workspace=b.ws, stream=stream)
     if not cfg.desc_act:
-        lam = gptq_prepare_hinv(b.H, b.U, cfg.damp_rel, workspace=b.ws, stream=stream)
+        gptq_prepare_hinv_async(b.H, b.U, cfg.damp_rel, workspace=b.ws, lam=b.lam, stream=stream)
         gptq_quantize_layer(W, b.U, cfg, b.qweight, b.scales, b.qzeros, b.err_sq, workspace=b.ws, stream=stream)
-        return QuantizedLayer(b.qweight, b.scales, b.qzeros, b.err_sq, lam)
+        gptq_sync_status(stream)
+        return QuantizedLayer(b.qweight, b.scales, b.qzeros, b.err_sq, float(b.lam.item()))
     gptq_act_sum_accumulate(X, b.act, accumulate=False, stream=stream)
     gptq_act_order(b.act, cfg.desc_act, b.perm, b.rank, stream=stream)
-    lam = gptq_prepare_hinv_permuted(b.H, b.perm, b.U, cfg.damp_rel, workspace=b.ws, stream=stream)
+    gptq_prepare_hinv_async(b.H, b.U, cfg.damp_rel, workspace=b.ws, lam=b.lam, perm=b.perm, stream=stream)
     gptq_quantize_layer_act_order(W, b.U, b.perm, cfg, b.qweight, b.scales, b.qzeros, b.g_idx, b.err_sq,
                                   workspace=b.ws, stream=stream)
-    return QuantizedLayer(b.qweight, b.scales, b.qzeros, b.err_sq, lam, b.g_idx, b.perm)
+    gptq_sync_status(stream)
+    return QuantizedLayer(b.qweight, b.scales, b.qzeros, b.err_sq, float(b.lam.item()), b.g_idx, b.perm)
 
 
 class SharedInputBuffers:
