@@ -208,17 +208,13 @@ def rank_probe(world: int, rank: int) -> None:
 
 # ---------------------------------------------------------------- GPU leg
 
-CHOL_KERNELS = ("chol_leaf", "chol_panel", "chol_chain_r", "chol_chain_d", "chol_update", "chol_update_next",
-                "chol_update_u2", "inv_bu", "inv_ub",
-                "split_panel",
-                "damp_copy", "diag_mean", "zero_lower", "chol_diag_out", "perm_invert", "damp_copy_perm")
-QUANT_KERNELS = ("colloop", "trailing_update", "trailing_update_wide", "trailing_update_sb", "up_prep", "ut_split",
-                 "tc_un_prep", "tc_ut_prep", "pack_zeros", "row_params",
+CHOL_KERNELS = ("chol_dag", "damp_copy", "diag_mean", "zero_lower", "perm_invert", "damp_copy_perm")
+QUANT_KERNELS = ("colloop", "trailing_update", "trailing_update_sb", "up_prep", "ut_split", "pack_zeros", "row_params",
                  "gather_cols", "unpermute_codes")
 ACT_KERNELS = ("act_sum", "act_rank", "act_perm")   # activation ordering (--desc-act 1 or 2)
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu --set full capture of this
 # workload, for kernels whose launches all do the same work (the kernel's ncu summary under profiles/).
-TRAFFIC_PER_LAUNCH = {"chol_leaf": 142592, "colloop": 2239232, "hessian_syrk": 16879616 + 11550464}
+TRAFFIC_PER_LAUNCH = {"colloop": 2239232, "hessian_syrk": 16879616 + 11550464}
 # Sum of the stage bounds for this layer: Hessian 21.0 us (bf16), factor + invert 168.1 us and
 # trailing updates 244.3 us (3xTF32 at a third of bf16 x 1.1/2.25), column loop 11.6 us (HBM).
 END_TO_END_BOUND_MS = 0.445
@@ -259,10 +255,9 @@ def kernel_rooflines(kernel_ms: dict, launches: dict, hbm: float, bf16: float, p
 
     Algorithmic work:
       trailing_update  2 * d_out * (d_in - e) * 128 flops per launch, summed over the layer; 3xTF32
-      chol_panel/update, inv_*  2/3 d_in^3 flops for the whole factorization (shared); 3xTF32
+      chol_dag         2/3 d_in^3 flops (factor + triangular inverse) per launch; 3xTF32
       hessian_syrk     n * d_in * (d_in + 1) flops; bf16
       colloop          W read once + codes + scales/zeros written, bytes; HBM
-      chol_leaf        2/3 * 128^3 * 2 flops per 128x128 leaf (factor + inverse) on ONE SM; fp32 ALU
     tf32 peak = measured bf16 x 1.1/2.25 (nominal ratio); 3xTF32 peak = a third of it.
     """
     B = 128
@@ -291,19 +286,9 @@ def kernel_rooflines(kernel_ms: dict, launches: dict, hbm: float, bf16: float, p
     add("hessian_syrk", "tensor", 1.0 * n * d_in * (d_in + 1), "TFLOP/s", bf16, f"bf16 {peak_kind} burst")
     col_bytes = 4.0 * d_out * d_in + BITS / 8 * d_out * d_in + (2 + BITS / 8) * d_out * (d_in // GROUP)
     add("colloop", "hbm", col_bytes, "GB/s", hbm, f"HBM {peak_kind}; latency chain of d_in rounding steps per row")
-    nleaf = d_in // B
-    add("chol_leaf", "alu", nleaf * 2.0 * (2.0 / 3.0) * B ** 3, "TFLOP/s", sm_fp32,
-        "one CTA per 128x128 leaf: peak = one SM's fp32 FMA rate at 1965 MHz")
-    fact = ("chol_panel", "chol_chain_r", "chol_chain_d", "chol_update", "chol_update_next", "chol_update_u2",
-            "inv_bu", "inv_ub")
-    gemm_ms = sum(kernel_ms.get(k, 0) for k in fact)
-    if gemm_ms:
-        ach = (2.0 / 3.0) * d_in ** 3 / (gemm_ms / 1e3) / 1e12
-        for k in fact:
-            if k in kernel_ms:
-                out[k] = {"bound": "tensor", "achieved": ach, "peak": tf32x3, "unit": "TFLOP/s", "frac": ach / tf32x3,
-                          "traffic": None, "launches": launches.get(k),
-                          "note": f"factorization GEMMs together ({gemm_ms:.3f} ms) vs 3xTF32 ({tf32_kind} / 3)"}
+    add("chol_dag", "tensor", (2.0 / 3.0) * d_in ** 3, "TFLOP/s", tf32x3,
+        f"Cholesky d^3/3 + triangular inverse d^3/3 flops in one persistent launch; 3xTF32 ({tf32_kind} / 3); "
+        "its time is bounded below by the chain of 128x128 diagonal blocks")
     return out
 
 

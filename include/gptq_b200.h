@@ -295,6 +295,19 @@ gptq_status gptq_sync_status(void* stream);
 void gptq_timing_enable(int on);
 size_t gptq_timing_report(char* buf, size_t len);
 size_t gptq_timing_timeline(char* buf, size_t len);
+/* gptq_chol_schedule: the order in which the factorization kernel behind
+ * gptq_prepare_hinv hands out its 128 x 128 tile products, for a d_in with T = ceil(d_in / 128)
+ * tiles per side (host-side; no device work).  Writes up to max_tasks entries of four int32
+ * (type, a, b, c) to tasks (may be NULL) and returns the total number of products:
+ *   type 0  PANEL(j = b, i = a):     R_ij = A_ij R_jj^-T
+ *   type 1  UPDATE(j = c, i = a, k = b): A_ik -= R_ij R_kj^T
+ *   type 2  FIN(i = a, m = b):       U_im = -R_ii^-1 S_im
+ *   type 3  SUPD(i = a, k = c, m = b):  S_im += R_ik U_km
+ * with Hd = R R^T (R upper), U = R^-1.  The diagonal blocks (R_jj and R_jj^-1 from A_jj) are
+ * formed in the order j = T-1 .. 0 by one CTA, LEAF(j) needing the updates of A_jj.  Every
+ * product's inputs come from products earlier in the list or from a leaf before its step;
+ * returns -1 for T < 1. */
+int64_t gptq_chol_schedule(int64_t T, int32_t* tasks, int64_t max_tasks);
 gptq_status gptq_selftest_bounded_wait(uint64_t limit_ns, void* stream);
 
 /* ------------------------------------------------------------------ no-allocation variant

@@ -50,12 +50,14 @@ __global__ void diag_mean_kernel(const float* __restrict__ H, long long d, float
 // identity.  The strictly lower blocks of A are never read by the factorization and are
 // not written.
 __global__ void __launch_bounds__(256) damp_copy_kernel(const float* __restrict__ H, long long d, long long n,
-                                                        const float* __restrict__ lam, float* __restrict__ A) {
+                                                        const float* __restrict__ lam, float* __restrict__ A,
+                                                        float* __restrict__ RS_hi, float* __restrict__ RS_lo) {
     const int bi = blockIdx.y, bj = blockIdx.x;
     if (bi > bj) return;
     const long long r0 = (long long)bi * NB, c0 = (long long)bj * NB;
     const float l = lam[0];
     if (bi < bj) {
+        const bool last = c0 + NB == n;   // the first panel: also its tf32 split
         for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
             const int r = e >> 5, c = (e & 31) * 4;
             const long long i = r0 + r, j = c0 + c;
@@ -66,6 +68,15 @@ __global__ void __launch_bounds__(256) damp_copy_kernel(const float* __restrict_
                     record_status(GPTQ_ERR_NONFINITE, i * d + j);
             }
             *reinterpret_cast<float4*>(A + i * n + j) = v;
+            if (last) {
+                float4 h, q;
+                split_tf32(v.x, h.x, q.x);
+                split_tf32(v.y, h.y, q.y);
+                split_tf32(v.z, h.z, q.z);
+                split_tf32(v.w, h.w, q.w);
+                *reinterpret_cast<float4*>(RS_hi + i * n + j) = h;
+                *reinterpret_cast<float4*>(RS_lo + i * n + j) = q;
+            }
         }
         return;
     }
@@ -89,12 +100,21 @@ __global__ void __launch_bounds__(256) damp_copy_kernel(const float* __restrict_
 // sector of H is fetched once.  H must hold both triangles.
 __global__ void __launch_bounds__(256) damp_copy_perm_kernel(const float* __restrict__ H,
                                                              const int* __restrict__ perm, long long d, long long n,
-                                                             const float* __restrict__ lam, float* __restrict__ A) {
+                                                             const float* __restrict__ lam, float* __restrict__ A,
+                                                             float* __restrict__ RS_hi, float* __restrict__ RS_lo) {
     const long long i = blockIdx.x;
     const long long j0 = (i / NB) * NB;
+    const long long jl = n - NB;   // the first panel (block column T-1, rows above its block): also split
     float* out = A + i * n;
     if (i >= d) {
-        for (long long j = j0 + threadIdx.x; j < n; j += blockDim.x) out[j] = (i == j) ? 1.f : 0.f;
+        for (long long j = j0 + threadIdx.x; j < n; j += blockDim.x) {
+            const float v = (i == j) ? 1.f : 0.f;
+            out[j] = v;
+            if (i < jl && j >= jl) {
+                RS_hi[i * n + j] = v;
+                RS_lo[i * n + j] = 0.f;
+            }
+        }
         return;
     }
     const float l = lam[0];
@@ -107,20 +127,12 @@ __global__ void __launch_bounds__(256) damp_copy_perm_kernel(const float* __rest
             if (i == j) v += l;
         }
         out[j] = v;
-    }
-}
-
-// Split A[0:rows, col0:col0+128] into tf32 hi/lo arrays with leading dimension 128.
-__global__ void split_panel_kernel(const float* __restrict__ A, long long n, int rows, int col0,
-                                   float* __restrict__ hi, float* __restrict__ lo) {
-    const long long total = (long long)rows * NB;
-    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-         e += (long long)gridDim.x * blockDim.x) {
-        const long long r = e >> 7, c = e & 127;
-        float h, l;
-        split_tf32(A[r * n + col0 + c], h, l);
-        hi[e] = h;
-        lo[e] = l;
+        if (i < jl && j >= jl) {
+            float h, q;
+            split_tf32(v, h, q);
+            RS_hi[i * n + j] = h;
+            RS_lo[i * n + j] = q;
+        }
     }
 }
 
@@ -157,8 +169,7 @@ __global__ void __launch_bounds__(256) zero_lower_blocks_kernel(float* __restric
 // (exact, not rounded: the tensor pipe reads only its tf32 part); U_hi + U_lo restores
 // X_jj exactly for chol_diag_out_kernel.
 constexpr int LS = NB + 4;   // leaf smem row stride (16-byte aligned rows)
-constexpr int LEAF_THREADS = 512;
-static_assert(NB * NB / 4 == 8 * LEAF_THREADS && NB * 32 == 8 * LEAF_THREADS, "leaf load and store loops");
+constexpr int LEAF_THREADS = 256;
 
 struct LeafSmem {
     float P[NB][LS];         // reversed block; lower triangle holds the Schur complement
@@ -259,10 +270,11 @@ __device__ __forceinline__ void leaf_panel_solve(LeafSmem& S, int k0, int i) {
 
 // C. Rank-32 update of the trailing lower triangle (rows and columns >= k0 + 32) with the
 // panel just factored; 4x4 micro-tiles on the lower triangle of tiles only.
+template <int NT = LEAF_THREADS>
 __device__ __forceinline__ void leaf_trailing_update(LeafSmem& S, int k0, int tid) {
     const int t0 = k0 + 32, tn = (NB - t0) >> 2;
     const int ntask = tn * (tn + 1) / 2;
-    for (int task = tid; task < ntask; task += LEAF_THREADS) {
+    for (int task = tid; task < ntask; task += NT) {
         int tr = (int)((sqrtf(8.f * (float)task + 1.f) - 1.f) * 0.5f);
         while (tr * (tr + 1) / 2 > task) --tr;
         while ((tr + 1) * (tr + 2) / 2 <= task) ++tr;
@@ -320,8 +332,9 @@ __device__ __forceinline__ void leaf_diag_inverse(LeafSmem& S, int i, int lane) 
 
 // Block row i of X = L^-1 with all threads: T_ij = sum_{k=j}^{i-1} L_ik X_kj into X's free
 // upper block (j, i), then X_ij = -X_ii T_ij.  Block rows < i must be complete.
+template <int NT = LEAF_THREADS>
 __device__ __forceinline__ void leaf_x_block_row(LeafSmem& S, int i, int tid) {
-    for (int task = tid; task < 64 * i; task += LEAF_THREADS) {
+    for (int task = tid; task < 64 * i; task += NT) {
         const int j = task >> 6, r0 = 4 * ((task >> 3) & 7), c0 = 4 * (task & 7);
         float acc[4][4] = {};
         for (int k = j; k < i; ++k) {
@@ -342,7 +355,7 @@ __device__ __forceinline__ void leaf_x_block_row(LeafSmem& S, int i, int tid) {
                 make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
     }
     __syncthreads();
-    for (int task = tid; task < 64 * i; task += LEAF_THREADS) {
+    for (int task = tid; task < 64 * i; task += NT) {
         const int j = task >> 6, r0 = 4 * ((task >> 3) & 7), c0 = 4 * (task & 7);
         float acc[4][4] = {};
 #pragma unroll 8
@@ -363,377 +376,4 @@ __device__ __forceinline__ void leaf_x_block_row(LeafSmem& S, int i, int tid) {
     __syncthreads();
 }
 
-__global__ void __launch_bounds__(LEAF_THREADS, 1)
-    chol_leaf_kernel(const float* __restrict__ A, long long n, int jb, float* __restrict__ U_hi,
-                     float* __restrict__ U_lo) {
-    extern __shared__ __align__(16) uint8_t leaf_raw[];
-    LeafSmem& S = *reinterpret_cast<LeafSmem*>(leaf_raw);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    pdl_wait();
-    pdl_trigger();
-
-    // P[127-r][127-c] = A[r][c]: the whole diagonal tile, in two halves whose loads are all
-    // issued before their stores
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        float4 v[4];
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int e = tid + (4 * half + it) * LEAF_THREADS, r = e >> 5, c = (e & 31) * 4;
-            v[it] = *reinterpret_cast<const float4*>(A + (long long)(jb + r) * n + jb + c);
-        }
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int e = tid + (4 * half + it) * LEAF_THREADS, r = e >> 5, c = (e & 31) * 4;
-            S.P[127 - r][127 - c] = v[it].x;
-            S.P[127 - r][126 - c] = v[it].y;
-            S.P[127 - r][125 - c] = v[it].z;
-            S.P[127 - r][124 - c] = v[it].w;
-        }
-    }
-    __syncthreads();
-
-    for (int kb = 0; kb < 4; ++kb) {
-        const int k0 = 32 * kb;
-        if (warp == 0) leaf_diag_factor(S, k0, lane, jb);
-        __syncthreads();
-        if (tid >= 32 && tid < 32 + (NB - k0 - 32)) leaf_panel_solve(S, k0, k0 + tid);   // rows k0+32 ..
-        else if (warp == 15) leaf_diag_inverse(S, kb, lane);
-        __syncthreads();
-        if (kb < 3) {
-            leaf_trailing_update(S, k0, tid);
-            __syncthreads();
-        }
-    }
-    for (int i = 1; i < 4; ++i) leaf_x_block_row(S, i, tid);
-
-    // U block = J X J (upper): U[r][c] = X[127-r][127-c] for r <= c; 4 columns per thread
-#pragma unroll 2
-    for (int it = 0; it < NB * 32 / LEAF_THREADS; ++it) {
-        const int task = tid + it * LEAF_THREADS, r = task >> 5, c = (task & 31) * 4;
-        const float4 xv = ld4(&S.X[127 - r][124 - c]);   // columns 124-c .. 127-c, reversed below
-        float v[4] = {xv.w, xv.z, xv.y, xv.x};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            if (r > c + i) v[i] = 0.f;
-        float h[4], l[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            h[i] = to_tf32(v[i]);
-            l[i] = v[i] - h[i];
-        }
-        const long long off = (long long)(jb + r) * n + jb + c;
-        *reinterpret_cast<float4*>(U_hi + off) = make_float4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<float4*>(U_lo + off) = make_float4(l[0], l[1], l[2], l[3]);
-    }
-}
-
-// One CTA per diagonal block jb = 128 * (blk0 + blockIdx.x): X_jj = U_hi + U_lo (exact, as the leaf
-// wrote them).  Writes X_jj to the public U (clipped to d) and its transposed tf32 split to
-// UT_hi/UT_lo.
-__global__ void __launch_bounds__(512)
-    chol_diag_out_kernel(const float* __restrict__ U_hi, const float* __restrict__ U_lo, float* __restrict__ UT_hi,
-                         float* __restrict__ UT_lo, float* __restrict__ U, long long n, long long d, int blk0) {
-    extern __shared__ __align__(16) uint8_t dout_raw[];
-    float (*Vs)[NB + 1] = reinterpret_cast<float (*)[NB + 1]>(dout_raw);
-    const long long jb = (long long)(blk0 + blockIdx.x) * NB;
-    for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-        const int r = e >> 7, c = e & 127;
-        const long long off = (jb + r) * n + jb + c;
-        const float v = U_hi[off] + U_lo[off];
-        Vs[r][c] = v;
-        if (jb + r < d && jb + c < d) U[(jb + r) * d + jb + c] = v;
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-        const int c = e >> 7, r = e & 127;   // UT[c][r] = U[r][c]
-        float h, l;
-        split_tf32(Vs[r][c], h, l);
-        UT_hi[(jb + c) * n + jb + r] = h;
-        UT_lo[(jb + c) * n + jb + r] = l;
-    }
-}
-
 }  // namespace gq
-
-namespace gqh {
-
-inline long long chol_n(long long d) { return (d + gq::NB - 1) / gq::NB * gq::NB; }
-
-struct HinvWs {
-    float *A, *RS_hi, *RS_lo, *U_hi, *U_lo, *UT_hi, *UT_lo, *TT_hi, *TT_lo, *AP_hi, *AP_lo, *scal;
-    int* rank;   // inverse of a caller's permutation (permuted factorization only)
-};
-
-inline size_t hinv_ws_bytes(long long d) {
-    const long long n = chol_n(d);
-    return (size_t)(9 * n * n + 2 * n * gq::NB + 64 + n) * sizeof(float);
-}
-
-inline HinvWs hinv_ws_carve(void* ws, long long d) {
-    const long long n = chol_n(d);
-    float* p = static_cast<float*>(ws);
-    HinvWs w;
-    w.A = p;
-    p += n * n;
-    w.RS_hi = p;
-    p += n * n;
-    w.RS_lo = p;
-    p += n * n;
-    w.U_hi = p;
-    p += n * n;
-    w.U_lo = p;
-    p += n * n;
-    w.UT_hi = p;
-    p += n * n;
-    w.UT_lo = p;
-    p += n * n;
-    w.TT_hi = p;
-    p += n * n;
-    w.TT_lo = p;
-    p += n * n;
-    w.AP_hi = p;   // tf32 split of the next panel, n x 128
-    p += n * gq::NB;
-    w.AP_lo = p;
-    p += n * gq::NB;
-    w.scal = p;
-    p += 64;
-    w.rank = reinterpret_cast<int*>(p);
-    return w;
-}
-
-
-// Enqueue the whole factorization.  Leaves U (public, d x d) and the splits of U
-// (U_hi/U_lo row-major, UT_hi/UT_lo transposed; n x n) in the workspace.
-inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* U, void* ws,
-                            cudaStream_t st, const int* perm = nullptr) {
-    const long long n = chol_n(d);
-    const int T = (int)(n / gq::NB);
-    HinvWs w = hinv_ws_carve(ws, d);
-    {
-        gqh::TimedScope ts__("diag_mean", st);
-        gq::diag_mean_kernel<<<1, 1024, 0, st>>>(H, d, damp_rel, w.scal);
-    }
-    GQ_TRY(cudaGetLastError());
-    if (perm) {   // factor P^T Hd P: validate the permutation, then a gathering damped copy
-        GQ_TRY(cudaMemsetAsync(w.rank, 0xFF, (size_t)d * sizeof(int), st));
-        {
-            gqh::TimedScope ts__("perm_invert", st);
-            gq::perm_invert_kernel<<<(unsigned)((d + 255) / 256), 256, 0, st>>>(perm, d, w.rank);
-        }
-        GQ_TRY(cudaGetLastError());
-        {
-            gqh::TimedScope ts__("damp_copy_perm", st);
-            gq::damp_copy_perm_kernel<<<(unsigned)n, 256, 0, st>>>(H, perm, d, n, w.scal, w.A);
-        }
-        GQ_TRY(cudaGetLastError());
-    } else {
-        const dim3 grid((unsigned)(n / gq::NB), (unsigned)(n / gq::NB));
-        {
-            gqh::TimedScope ts__("damp_copy", st);
-            gq::damp_copy_kernel<<<grid, 256, 0, st>>>(H, d, n, w.scal, w.A);
-        }
-        GQ_TRY(cudaGetLastError());
-    }
-    const int leaf_smem = (int)sizeof(gq::LeafSmem);
-    GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::chol_leaf_kernel), leaf_smem));
-    const uint64_t N = (uint64_t)n;
-    // Streams.  The chain stream (highest priority) carries, per block column j,
-    //   leaf(j) -> panel(j): R_{0:j,j} = A_{0:j,j} X_jj^T
-    //           -> block column j-1 updated by panel j (and the next panel's tf32 split).
-    // The far stream takes the rest of panel j's Schur update: first block column j-2 (u2),
-    // then everything left of it (rest).  Block column j-1 has received, before its update by
-    // panel j, u2(j+1) and rest(p) for p >= j+2, which the far stream runs in that order, so
-    // the chain waits only for u2(j+1).  The inverse stream runs the doubling products.
-    FactStreams fs;
-    if (!fact_streams(&fs)) return cudaErrorUnknown;
-    cudaEvent_t ev_start = fs.ev[0], ev_leaf = fs.ev[1], ev_panel = fs.ev[2], ev_u2 = fs.ev[5],
-                ev_far = fs.ev[8], ev_chain = fs.ev[9], ev_inv = fs.ev[10];
-    cudaStream_t sc = fs.chain, sf = fs.far, si = fs.inv;
-    {
-        gqh::TimedScope ts__("zero_lower", st);   // the public U's strictly lower blocks
-        const unsigned nb = (unsigned)((d + gq::NB - 1) / gq::NB);
-        gq::zero_lower_blocks_kernel<<<dim3(nb, nb), 256, 0, st>>>(U, d);
-    }
-    GQ_TRY(cudaGetLastError());
-    GQ_TRY(cudaEventRecord(ev_start, st));
-    GQ_TRY(cudaStreamWaitEvent(sc, ev_start, 0));
-    GQ_TRY(cudaStreamWaitEvent(sf, ev_start, 0));
-    GQ_TRY(cudaStreamWaitEvent(si, ev_start, 0));
-    const int far_ctas = std::max(1, num_sms() - 1);            // leave an SM for the next leaf
-    const int inv_ctas = std::max(1, num_sms() / 4);            // the inverse fills in around the chain
-    Mat rh{w.RS_hi, N, N, N}, rl{w.RS_lo, N, N, N};
-    Mat xh{w.U_hi, N, N, N}, xl{w.U_lo, N, N, N};
-    // U = R^-1 by doubling, each product issued on the inverse stream as soon as its inputs
-    // exist: for the diagonal pair [[R_a, B], [0, R_c]] of level s (a-half rows r0 .. r0+s,
-    // c-half r0+s .. r0+s+cs) with inverses U_a and U_c known, T = B U_c (stored transposed) as
-    // soon as the c-half is inverted and the panels of its block columns are formed, and
-    // U_b = -U_a T once the a-half is inverted.  Only the products of the pairs that contain
-    // block 0 wait for the last leaf.
-    Mat uth{w.UT_hi, N, N, N}, utl{w.UT_lo, N, N, N};
-    Mat tth{w.TT_hi, N, N, N}, ttl{w.TT_lo, N, N, N};
-    const int dout_smem = (int)(gq::NB * (gq::NB + 1) * sizeof(float));
-    GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::chol_diag_out_kernel), dout_smem));
-    auto inv_bu = [&](long long s_, long long r0, long long cs) -> cudaError_t {   // T = B U_c -> TT
-        gq::GemmArgs p = gemm_args((int)s_, (int)cs, (int)cs);
-        p.a_row0 = (int)r0;
-        p.a_col0 = (int)(r0 + s_);
-        p.b_row0 = (int)(r0 + s_);
-        p.b_col0 = (int)(r0 + s_);
-        p.k_to_n1 = 1;
-        p.t_row0 = (int)(r0 + s_);
-        p.t_col0 = (int)r0;
-        EpiMats o;
-        o.t_hi = Mat{w.TT_hi, N, N, N};
-        o.t_lo = Mat{w.TT_lo, N, N, N};
-        const bool narrow = 4 * (s_ / gq::NB) * ((cs + gq::NB - 1) / gq::NB) <= num_sms();
-        if (narrow) return launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, uth, utl, o, p, 1, si, "inv_bu", inv_ctas, true);
-        return launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rh, rl, uth, utl, o, p, 1, si, "inv_bu", inv_ctas, true);
-    };
-    auto inv_ub = [&](long long s_, long long r0, long long cs) -> cudaError_t {   // U_b = -U_a T
-        gq::GemmArgs p = gemm_args((int)s_, (int)cs, (int)s_);
-        p.a_row0 = (int)r0;
-        p.a_col0 = (int)r0;
-        p.b_row0 = (int)(r0 + s_);
-        p.b_col0 = (int)r0;
-        p.k_from_m0 = 1;
-        p.alpha = -1.f;
-        p.c_row0 = (int)r0;
-        p.c_col0 = (int)(r0 + s_);
-        p.write_c = 1;
-        p.s_row0 = (int)r0;
-        p.s_col0 = (int)(r0 + s_);
-        p.t_row0 = (int)(r0 + s_);
-        p.t_col0 = (int)r0;
-        EpiMats o;
-        o.c = Mat{U, (uint64_t)d, (uint64_t)d, (uint64_t)d};   // public U, clipped to d x d
-        o.s_hi = Mat{w.U_hi, N, N, N};
-        o.s_lo = Mat{w.U_lo, N, N, N};
-        o.t_hi = Mat{w.UT_hi, N, N, N};
-        o.t_lo = Mat{w.UT_lo, N, N, N};
-        // the pairs that contain block 0 are the tail after the last leaf: all SMs
-        const int cap = r0 == 0 ? 0 : inv_ctas;
-        const bool narrow = 4 * (s_ / gq::NB) * ((cs + gq::NB - 1) / gq::NB) <= num_sms();
-        if (narrow) return launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(xh, xl, tth, ttl, o, p, 1, si, "inv_ub", cap, true);
-        return launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(xh, xl, tth, ttl, o, p, 1, si, "inv_ub", cap, true);
-    };
-    // the inverse work that becomes possible once leaf(j) and panel(j) are done (event ev)
-    auto inverse_step = [&](int j, cudaEvent_t ev) -> cudaError_t {
-        const long long jb = (long long)j * gq::NB;
-        GQ_TRY(cudaStreamWaitEvent(si, ev, 0));
-        {
-            gqh::TimedScope ts__("chol_diag_out", si);
-            gq::chol_diag_out_kernel<<<1, 512, dout_smem, si>>>(w.U_hi, w.U_lo, w.UT_hi, w.UT_lo, U, n, d, j);
-        }
-        GQ_TRY(cudaGetLastError());
-        for (long long s_ = gq::NB; s_ < n; s_ *= 2)   // pairs whose a-half starts at block j
-            if (jb % (2 * s_) == 0 && jb + s_ < n) GQ_TRY(inv_ub(s_, jb, std::min(s_, n - jb - s_)));
-        for (long long s_ = gq::NB; s_ < n; s_ *= 2)   // pairs whose c-half starts at block j
-            if (jb >= s_ && (jb - s_) % (2 * s_) == 0) GQ_TRY(inv_bu(s_, jb - s_, std::min(s_, n - jb)));
-        return cudaSuccess;
-    };
-    bool u2_pending = false;
-    for (int j = T - 1; j >= 0; --j) {
-        const int jb = j * gq::NB;
-        {
-            gqh::TimedScope ts__("chol_leaf", sc);
-            if (j == T - 1)   // follows the wait for the damped copy on the caller's stream
-                GQ_TRY(launch_plain(gq::chol_leaf_kernel, dim3(1), dim3(gq::LEAF_THREADS), (size_t)leaf_smem, sc,
-                                    (const float*)w.A, n, jb, w.U_hi, w.U_lo));
-            else
-                GQ_TRY(launch_pdl(gq::chol_leaf_kernel, dim3(1), dim3(gq::LEAF_THREADS), (size_t)leaf_smem, sc,
-                                  (const float*)w.A, n, jb, w.U_hi, w.U_lo));
-        }
-        if (j == 0) {
-            GQ_TRY(cudaEventRecord(ev_leaf, sc));
-            GQ_TRY(inverse_step(0, ev_leaf));
-            break;
-        }
-        if (j == T - 1) {   // later panels are split by the previous update's epilogue
-            gqh::TimedScope ts__("split_panel", sc);
-            gq::split_panel_kernel<<<(unsigned)std::min<long long>((jb * 128LL + 255) / 256, 4096), 256, 0, sc>>>(
-                w.A, n, jb, jb, w.AP_hi, w.AP_lo);
-            GQ_TRY(cudaGetLastError());
-        }
-        {   // panel: RS[0:jb, jb:jb+128] = AP * X^T, X = U block (row-major split)
-            gq::GemmArgs p = gemm_args(jb, gq::NB, gq::NB);
-            p.b_row0 = jb;
-            p.b_col0 = jb;
-            p.s_col0 = jb;
-            EpiMats o;
-            o.s_hi = Mat{w.RS_hi, N, N, N};
-            o.s_lo = Mat{w.RS_lo, N, N, N};
-            Mat ah{w.AP_hi, (uint64_t)jb, 128, 128}, al{w.AP_lo, (uint64_t)jb, 128, 128};
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(ah, al, xh, xl, o, p, 1, sc, "chol_panel", 0,
-                                                        j == T - 1)));
-        }
-        const int jn = jb - gq::NB;    // first column of block column j-1
-        const int jn2 = jn - gq::NB;   // first column of block column j-2
-        GQ_TRY(cudaEventRecord(ev_panel, sc));
-        const bool waited = u2_pending;
-        if (u2_pending) GQ_TRY(cudaStreamWaitEvent(sc, ev_u2, 0));
-        {   // block column j-1: A[0:jb, jn:jb] -= RS_panel RS_panel[jn:jb]^T, plus the next panel's split
-            gq::GemmArgs p = gemm_args(jb, gq::NB, gq::NB);
-            p.a_col0 = jb;
-            p.b_row0 = jn;
-            p.b_col0 = jb;
-            p.alpha = -1.f;
-            p.beta = 1.f;
-            p.write_c = 1;
-            p.c_col0 = jn;
-            EpiMats o;
-            o.c = Mat{w.A, N, N, N};
-            if (j >= 2) {   // tiles above the diagonal block write the next panel's tf32 split
-                p.s_mt_lim = j - 1;
-                o.s_hi = Mat{w.AP_hi, (uint64_t)jn, 128, 128};
-                o.s_lo = Mat{w.AP_lo, (uint64_t)jn, 128, 128};
-            }
-            GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, rh, rl, o, p, 1, sc, "chol_update_next", 0,
-                                                        waited)));
-        }
-        u2_pending = false;
-        if (j >= 2) {   // far stream: block column j-2, then the rest
-            GQ_TRY(cudaStreamWaitEvent(sf, ev_panel, 0));
-            {   // u2: A[0:jn, jn2:jn] -= RS_panel RS_panel[jn2:jn]^T
-                gq::GemmArgs p = gemm_args(jn, gq::NB, gq::NB);
-                p.a_col0 = jb;
-                p.b_row0 = jn2;
-                p.b_col0 = jb;
-                p.alpha = -1.f;
-                p.beta = 1.f;
-                p.write_c = 1;
-                p.c_col0 = jn2;
-                EpiMats o;
-                o.c = Mat{w.A, N, N, N};
-                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 4, 32, 2>(rh, rl, rh, rl, o, p, 1, sf, "chol_update_u2",
-                                                            far_ctas, true)));
-            }
-            GQ_TRY(cudaEventRecord(ev_u2, sf));
-            u2_pending = true;
-            if (j >= 3) {   // rest: A[0:jn2, 0:jn2] -= RS RS^T (upper tiles)
-                gq::GemmArgs p = gemm_args(jn2, jn2, gq::NB);
-                p.a_col0 = jb;
-                p.b_col0 = jb;
-                p.triangular = 1;
-                p.alpha = -1.f;
-                p.beta = 1.f;
-                p.write_c = 1;
-                EpiMats o;
-                o.c = Mat{w.A, N, N, N};
-                GQ_TRY((launch_gemm<gq::KIND_TF32X3, 2, 128, 4>(rh, rl, rh, rl, o, p, 1, sf, "chol_update",
-                                                       far_ctas, true)));
-            }
-        }
-        GQ_TRY(inverse_step(j, ev_panel));
-    }
-    // all streams are done before the caller's stream continues
-    GQ_TRY(cudaEventRecord(ev_far, sf));
-    GQ_TRY(cudaEventRecord(ev_chain, sc));
-    GQ_TRY(cudaEventRecord(ev_inv, si));
-    GQ_TRY(cudaStreamWaitEvent(st, ev_far, 0));
-    GQ_TRY(cudaStreamWaitEvent(st, ev_chain, 0));
-    GQ_TRY(cudaStreamWaitEvent(st, ev_inv, 0));
-    return cudaSuccess;
-}
-
-}  // namespace gqh

@@ -1,0 +1,796 @@
+// The blocked factorization of chol.cuh as one persistent dataflow kernel.
+//
+// With T = n / 128 tiles per side, tile indices i, j, k, m < T, and Hd = R R^T (R upper,
+// factored from the bottom-right corner), U = R^-1:
+//   LEAF(j)         R_jj from A_jj, X_jj = R_jj^-1                       (one CTA, fp32)
+//   PANEL(j, i)     R_ij  = A_ij X_jj^T                      i < j
+//   UPDATE(j, i, k) A_ik -= R_ij R_kj^T                       i <= k < j
+//   SUPD(i, k, m)   S_im += R_ik U_km                         i < k <= m    (U_mm = X_mm)
+//   FIN(i, m)       U_im  = -X_ii S_im                        i < m
+// (block back-substitution for U = R^-1: U_im = -X_ii sum_{k=i+1}^{m} R_ik U_km).  Every
+// product is one 128 x 128 x 128 tile in 3xTF32 on the tensor cores (tcgen05, operands by
+// TMA, accumulators in tensor memory; K split into four segments added in fp32 round-to-
+// nearest, cross products apart), with fp32 read-modify-write of A and S in global memory.
+//
+// One CTA (the first to start) runs the leaves in order j = T-1 .. 0.  Every other CTA
+// takes the product tasks from a global ticket counter in a fixed order (dag_step_task):
+// per step j the two tiles the next leaf needs, the rest of panel j, block column j-1, row j
+// of U, the S contributions of panel j, then the far updates.  Each task waits (bounded) for
+// the counters of the tasks it reads from, all of which come earlier in that order; so the
+// lowest unfinished task can always run, whatever subset of CTAs is resident.  Within a CTA
+// the task fetch and TMA loads (warp 0), the MMAs (warp 1) and the epilogue (warps 2-5) are
+// pipelined across tasks as in tc_gemm_kernel.  Counters are released with a gpu-scope fence
+// after the producing stores and acquired before the consuming loads (with a proxy fence in
+// front of TMA reads).
+#pragma once
+#include "chol.cuh"
+
+namespace gq {
+
+enum : int { DT_PANEL = 0, DT_UPDATE = 1, DT_FIN = 2, DT_SUPD = 3, DT_STOP = 15 };
+
+// PANEL(j, i): a = i, b = j.  UPDATE(j, i, k): a = i, b = k, c = j.
+// FIN(i, m): a = i, b = m.    SUPD(i, k, m): a = i, b = m, c = k.
+struct DagTask {
+    int type, a, b, c;
+};
+
+__host__ __device__ inline long long dag_step_tasks(int T, int j) {
+    const long long jj = j;
+    long long c = (T - 1 - jj) + jj * (T - jj);
+    if (j >= 1) c += 2;
+    if (j >= 2) c += 2 * (jj - 1) + (jj - 1) * jj / 2;
+    return c;
+}
+
+__host__ __device__ inline long long dag_total_tasks(int T) {
+    long long c = 0;
+    for (int j = 0; j < T; ++j) c += dag_step_tasks(T, j);
+    return c;
+}
+
+// Task idx of step j.
+__host__ __device__ inline DagTask dag_step_task(int T, int j, long long idx) {
+    if (j >= 1) {
+        if (idx == 0) return DagTask{DT_PANEL, j - 1, j, 0};
+        if (idx == 1) return DagTask{DT_UPDATE, j - 1, j - 1, j};
+        idx -= 2;
+    }
+    if (j >= 2) {
+        if (idx < j - 1) return DagTask{DT_PANEL, j - 2 - (int)idx, j, 0};
+        idx -= j - 1;
+        if (idx < j - 1) return DagTask{DT_UPDATE, j - 2 - (int)idx, j - 1, j};
+        idx -= j - 1;
+    }
+    if (idx < T - 1 - j) return DagTask{DT_FIN, j, j + 1 + (int)idx, 0};
+    idx -= T - 1 - j;
+    if (idx < (long long)j * (T - j)) return DagTask{DT_SUPD, (int)(idx % j), j + (int)(idx / j), j};
+    idx -= (long long)j * (T - j);
+    for (int k = j - 2; k >= 0; --k) {   // far updates, nearest block column first
+        if (idx < k + 1) return DagTask{DT_UPDATE, (int)idx, k, j};
+        idx -= k + 1;
+    }
+    return DagTask{DT_STOP, 0, 0, 0};
+}
+
+// Tickets arrive in increasing order per CTA: the cursor walks the steps forward.
+struct DagCursor {
+    int j;
+    long long base;
+};
+__host__ __device__ inline DagTask dag_decode(int T, DagCursor& cur, long long t) {
+    while (cur.j >= 0 && t >= cur.base + dag_step_tasks(T, cur.j)) {
+        cur.base += dag_step_tasks(T, cur.j);
+        --cur.j;
+    }
+    if (cur.j < 0) return DagTask{DT_STOP, 0, 0, 0};
+    return dag_step_task(T, cur.j, t - cur.base);
+}
+
+// Counter block (ints): [0] ticket, [1] role, [2] abort, [3] spare, then T x T arrays
+// a_cnt (updates applied to A_ik), rs_done (R_ij final), s_cnt (contributions applied to
+// S_im), u_done (U_im final), then leaf_done[T] (X_jj split written) and diag_done[T]
+// (U_jj written to U and to the transposed split).
+__host__ __device__ inline long long dag_ctr_ints(int T) { return 4 + 4LL * T * T + 2LL * T; }
+
+struct DagArgs {
+    int T;
+    long long n, d;
+    float* A;                    // n x n, damped copy of H (upper tiles), updated in place
+    float* S;                    // n x n, S_im accumulators
+    float* RS_hi, *RS_lo;        // n x n tf32 split of R (and of the panel inputs)
+    float* Xd_hi, *Xd_lo;        // T x 128 x 128 tf32 split of X_jj (row-major)
+    float* UT_hi, *UT_lo;        // n x n tf32 split of U^T
+    float* TT_hi, *TT_lo;        // n x n tf32 split of S^T
+    float* U;                    // d x d public output (strictly lower blocks zeroed beforehand)
+    int* ctr;
+};
+
+__device__ __forceinline__ int ld_acquire_s32(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ int ld_volatile_s32(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// Wait until *p >= target.  Bounded: after kWaitLimitNs records GPTQ_ERR_TIMEOUT (with
+// `where`) and raises the abort flag; returns false also when another CTA has aborted.
+__device__ __noinline__ bool dag_wait_ge(const int* p, int target, int* abort, long long where) {
+    if (ld_acquire_s32(p) >= target) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    unsigned ns = 32;
+    for (;;) {
+        __nanosleep(ns);
+        if (ns < 256) ns <<= 1;
+        if (ld_acquire_s32(p) >= target) return true;
+        if (ld_volatile_s32(abort)) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            record_status(GPTQ_ERR_TIMEOUT, where);
+            atomicExch(abort, 1);
+            return false;
+        }
+    }
+}
+
+// Counters a task waits for (the values it needs are reached exactly when the tasks it
+// reads from have completed).
+__device__ __forceinline__ bool dag_deps(const DagArgs& g, const DagTask& t) {
+    const int T = g.T;
+    int* c = g.ctr;
+    int* abort = c + 2;
+    const int* a_cnt = c + 4;
+    const int* rs_done = a_cnt + T * T;
+    const int* s_cnt = rs_done + T * T;
+    const int* u_done = s_cnt + T * T;
+    const int* leaf_done = u_done + T * T;
+    const int* diag_done = leaf_done + T;
+    const long long where = -(1000000LL + t.type * 100000LL + t.a * 1000LL + t.b);
+    switch (t.type) {
+        case DT_PANEL:
+            return dag_wait_ge(&leaf_done[t.b], 1, abort, where) &&
+                   dag_wait_ge(&a_cnt[t.a * T + t.b], T - 1 - t.b, abort, where);
+        case DT_UPDATE:
+            return dag_wait_ge(&rs_done[t.a * T + t.c], 1, abort, where) &&
+                   dag_wait_ge(&rs_done[t.b * T + t.c], 1, abort, where) &&
+                   dag_wait_ge(&a_cnt[t.a * T + t.b], T - 1 - t.c, abort, where);
+        case DT_FIN:
+            return dag_wait_ge(&leaf_done[t.a], 1, abort, where) &&
+                   dag_wait_ge(&s_cnt[t.a * T + t.b], t.b - t.a, abort, where);
+        case DT_SUPD:
+            return dag_wait_ge(&rs_done[t.a * T + t.c], 1, abort, where) &&
+                   dag_wait_ge(t.c == t.b ? &diag_done[t.b] : &u_done[t.c * T + t.b], 1, abort, where) &&
+                   dag_wait_ge(&s_cnt[t.a * T + t.b], t.b - t.c, abort, where);
+    }
+    return false;
+}
+
+// The counter a completed task advances.
+__device__ __forceinline__ int* dag_done_ctr(const DagArgs& g, const DagTask& t) {
+    const int T = g.T;
+    int* a_cnt = g.ctr + 4;
+    int* rs_done = a_cnt + T * T;
+    int* s_cnt = rs_done + T * T;
+    int* u_done = s_cnt + T * T;
+    switch (t.type) {
+        case DT_PANEL: return &rs_done[t.a * T + t.b];
+        case DT_UPDATE: return &a_cnt[t.a * T + t.b];
+        case DT_FIN: return &u_done[t.a * T + t.b];
+        default: return &s_cnt[t.a * T + t.b];
+    }
+}
+
+constexpr int DAG_THREADS = 256;
+constexpr int DAG_STAGES = 2;
+constexpr int DAG_SLOTS = 4;
+constexpr int DAG_NK = NB / GemmCfg<KIND_TF32X3, 128>::KT;   // 4 TMA stages of K = 32 per task
+constexpr int DAG_SEG = 4;                                   // MMA k-steps per accumulator segment
+constexpr int DAG_GEMM_BYTES = DAG_STAGES * GemmCfg<KIND_TF32X3, 128>::STAGE_BYTES + epi_bytes<128>();
+
+struct DagCtl {
+    uint64_t full[DAG_STAGES], empty[DAG_STAGES], tfull[2], tempty[2], cin[4];
+    uint64_t task_full[DAG_SLOTS], task_empty[DAG_SLOTS];
+    DagTask slot[DAG_SLOTS];
+    uint32_t tmem_slot;
+    int flag;
+    int epi_ok[4];
+};
+constexpr int DAG_SMEM_BODY = (DAG_GEMM_BYTES > (int)sizeof(LeafSmem) ? DAG_GEMM_BYTES : (int)sizeof(LeafSmem));
+constexpr int DAG_SMEM = 1024 + DAG_SMEM_BODY + (int)sizeof(DagCtl);
+static_assert(DAG_SMEM <= 232448, "persistent factorization: shared memory per CTA");
+static_assert(NB * NB / 4 == 16 * DAG_THREADS, "leaf load and store loops");
+
+__device__ __forceinline__ void named_bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------------------
+// The leaf CTA: LEAF(j) for j = T-1 .. 0 (256 threads; the pieces are chol.cuh's).
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, DagCtl& ctl) {
+    const int T = g.T;
+    const long long n = g.n, d = g.d;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int* c = g.ctr;
+    int* abort = c + 2;
+    int* a_cnt = c + 4;
+    int* leaf_done = a_cnt + 4 * T * T;
+    int* diag_done = leaf_done + T;
+    for (int j = T - 1; j >= 0; --j) {
+        const long long jb = (long long)j * NB;
+        if (tid == 0) ctl.flag = dag_wait_ge(&a_cnt[j * T + j], T - 1 - j, abort, -(2000000LL + j)) ? 1 : 0;
+        __syncthreads();
+        if (!ctl.flag) return;
+        // P[127-r][127-c] = A[r][c]
+#pragma unroll
+        for (int quarter = 0; quarter < 4; ++quarter) {
+            float4 v[4];
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+                const int e = tid + (4 * quarter + it) * DAG_THREADS, r = e >> 5, cc = (e & 31) * 4;
+                v[it] = __ldcg(reinterpret_cast<const float4*>(g.A + (jb + r) * n + jb + cc));
+            }
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+                const int e = tid + (4 * quarter + it) * DAG_THREADS, r = e >> 5, cc = (e & 31) * 4;
+                S.P[127 - r][127 - cc] = v[it].x;
+                S.P[127 - r][126 - cc] = v[it].y;
+                S.P[127 - r][125 - cc] = v[it].z;
+                S.P[127 - r][124 - cc] = v[it].w;
+            }
+        }
+        __syncthreads();
+        for (int kb = 0; kb < 4; ++kb) {
+            const int k0 = 32 * kb;
+            if (warp == 0) leaf_diag_factor(S, k0, lane, (int)jb);
+            __syncthreads();
+            if (tid >= 32 && tid < 32 + (NB - k0 - 32)) leaf_panel_solve(S, k0, k0 + tid);   // rows k0+32 ..
+            else if (warp == 7) leaf_diag_inverse(S, kb, lane);
+            __syncthreads();
+            if (kb < 3) {
+                leaf_trailing_update<DAG_THREADS>(S, k0, tid);
+                __syncthreads();
+            }
+        }
+        for (int i = 1; i < 4; ++i) leaf_x_block_row<DAG_THREADS>(S, i, tid);
+
+        // X_jj (block of U = J X J, upper) as its tf32 split, row-major: the operand of the
+        // panels of step j and of row j of U
+        float* xh = g.Xd_hi + (long long)j * NB * NB;
+        float* xl = g.Xd_lo + (long long)j * NB * NB;
+#pragma unroll 4
+        for (int it = 0; it < 16; ++it) {
+            const int task = tid + it * DAG_THREADS, r = task >> 5, cc = (task & 31) * 4;
+            const float4 xv = ld4(&S.X[127 - r][124 - cc]);
+            float v[4] = {xv.w, xv.z, xv.y, xv.x};
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (r > cc + q) v[q] = 0.f;
+            float h[4], l[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) split_tf32(v[q], h[q], l[q]);
+            *reinterpret_cast<float4*>(xh + r * NB + cc) = make_float4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<float4*>(xl + r * NB + cc) = make_float4(l[0], l[1], l[2], l[3]);
+        }
+        fence_proxy_async_global();
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            atomicAdd(&leaf_done[j], 1);
+        }
+        // U_jj to the public output (clipped to d; d % 4 == 0) and its transposed split
+#pragma unroll 4
+        for (int it = 0; it < 16; ++it) {
+            const int task = tid + it * DAG_THREADS, r = task >> 5, cc = (task & 31) * 4;
+            if (jb + r < d && jb + cc < d) {
+                const float4 xv = ld4(&S.X[127 - r][124 - cc]);
+                float v[4] = {xv.w, xv.z, xv.y, xv.x};
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (r > cc + q) v[q] = 0.f;
+                *reinterpret_cast<float4*>(g.U + (jb + r) * d + jb + cc) = make_float4(v[0], v[1], v[2], v[3]);
+            }
+            // UT row cc' = r (column r of U_jj), columns 4 (task & 31) .. +3 (rows of U_jj)
+            const int col = r, r4 = cc;
+            float h[4], l[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int rr = r4 + q;   // U_jj[rr][col] = X[127-rr][127-col]
+                const float v = (rr <= col) ? S.X[127 - rr][127 - col] : 0.f;
+                split_tf32(v, h[q], l[q]);
+            }
+            *reinterpret_cast<float4*>(g.UT_hi + (jb + col) * n + jb + r4) = make_float4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<float4*>(g.UT_lo + (jb + col) * n + jb + r4) = make_float4(l[0], l[1], l[2], l[3]);
+        }
+        fence_proxy_async_global();
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            atomicAdd(&diag_done[j], 1);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Product CTAs.
+// ---------------------------------------------------------------------------------------
+struct DagMaps {
+    CUtensorMap rs_hi, rs_lo, xd_hi, xd_lo, tt_hi, tt_lo, ut_hi, ut_lo, ca, cs;
+};
+
+__global__ void __launch_bounds__(DAG_THREADS, 1)
+    chol_dag_kernel(const __grid_constant__ DagMaps maps, const DagArgs g) {
+    extern __shared__ uint8_t dag_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dag_raw) + 1023) & ~uintptr_t(1023));
+    DagCtl& ctl = *reinterpret_cast<DagCtl*>(smem + DAG_SMEM_BODY);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = g.T;
+    int* abort = g.ctr + 2;
+
+    if (threadIdx.x == 0) ctl.flag = atomicAdd(g.ctr + 1, 1);
+    __syncthreads();
+    if (ctl.flag == 0) {   // the first CTA to start runs the leaves
+        __syncthreads();
+        dag_leaf_role(g, *reinterpret_cast<LeafSmem*>(smem), ctl);
+        return;
+    }
+
+    using Cfg = GemmCfg<KIND_TF32X3, 128>;
+    constexpr int TBN = 128, KT = Cfg::KT, STAGE_BYTES = Cfg::STAGE_BYTES;
+    constexpr int A_BYTES = BM * 128, B_BYTES = TBN * 128;
+    constexpr int SUM_HI = 2 * TBN, XOFF = 3 * TBN;
+    constexpr uint32_t TMEM_COLS = 512;
+    constexpr int NCHUNK = TBN / 32;
+    uint8_t* epi = smem + DAG_STAGES * STAGE_BYTES;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < DAG_STAGES; ++s) {
+            mbar_init(&ctl.full[s], 1);
+            mbar_init(&ctl.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl.tfull[b], 1);
+            mbar_init(&ctl.tempty[b], 4);
+        }
+        for (int q = 0; q < 4; ++q) mbar_init(&ctl.cin[q], 1);
+        for (int s = 0; s < DAG_SLOTS; ++s) {
+            mbar_init(&ctl.task_full[s], 1);
+            mbar_init(&ctl.task_empty[s], 1);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        __syncwarp();
+        tmem_alloc(&ctl.tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl.tmem_slot;
+
+    if (warp == 0 && lane == 0) {
+        // ---------------- task fetch, dependency waits, TMA producer
+        prefetch_tmap(&maps.rs_hi);
+        prefetch_tmap(&maps.rs_lo);
+        prefetch_tmap(&maps.xd_hi);
+        prefetch_tmap(&maps.xd_lo);
+        prefetch_tmap(&maps.tt_hi);
+        prefetch_tmap(&maps.tt_lo);
+        prefetch_tmap(&maps.ut_hi);
+        prefetch_tmap(&maps.ut_lo);
+        DagCursor cur{T - 1, 0};
+        uint32_t kiter = 0;
+        for (int nt = 0;; ++nt) {
+            const int s = nt % DAG_SLOTS;
+            DagTask tk{DT_STOP, 0, 0, 0};
+            const bool slot_ok = mbar_wait(&ctl.task_empty[s], (uint32_t)((nt / DAG_SLOTS) & 1) ^ 1u, -3000000LL - blockIdx.x);
+            if (slot_ok && !ld_volatile_s32(abort)) {
+                const long long t = atomicAdd(g.ctr, 1);
+                tk = dag_decode(T, cur, t);
+                if (tk.type != DT_STOP && !dag_deps(g, tk)) tk.type = DT_STOP;
+            } else if (!slot_ok) {
+                atomicExch(abort, 1);
+            }
+            ctl.slot[s] = tk;
+            mbar_arrive(&ctl.task_full[s]);
+            if (tk.type == DT_STOP) break;
+            fence_proxy_async_global();   // the counters were acquired; TMA reads follow
+            const CUtensorMap *ma_h, *ma_l, *mb_h, *mb_l;
+            int ax, ay, bx, by;
+            switch (tk.type) {
+                case DT_PANEL:   // A = R-split(i, j) (the updated panel input), B = X_jj
+                    ma_h = &maps.rs_hi; ma_l = &maps.rs_lo; ax = tk.b * NB; ay = tk.a * NB;
+                    mb_h = &maps.xd_hi; mb_l = &maps.xd_lo; bx = 0; by = tk.b * NB;
+                    break;
+                case DT_UPDATE:  // A = R(i, j), B = R(k, j)
+                    ma_h = &maps.rs_hi; ma_l = &maps.rs_lo; ax = tk.c * NB; ay = tk.a * NB;
+                    mb_h = &maps.rs_hi; mb_l = &maps.rs_lo; bx = tk.c * NB; by = tk.b * NB;
+                    break;
+                case DT_FIN:     // A = X_ii, B = S_im^T
+                    ma_h = &maps.xd_hi; ma_l = &maps.xd_lo; ax = 0; ay = tk.a * NB;
+                    mb_h = &maps.tt_hi; mb_l = &maps.tt_lo; bx = tk.a * NB; by = tk.b * NB;
+                    break;
+                default:         // SUPD: A = R(i, k), B = U_km^T
+                    ma_h = &maps.rs_hi; ma_l = &maps.rs_lo; ax = tk.c * NB; ay = tk.a * NB;
+                    mb_h = &maps.ut_hi; mb_l = &maps.ut_lo; bx = tk.c * NB; by = tk.b * NB;
+                    break;
+            }
+            for (int kt = 0; kt < DAG_NK; ++kt, ++kiter) {
+                const int st = kiter % DAG_STAGES;
+                const uint32_t it = kiter / DAG_STAGES;
+                if (!mbar_wait(&ctl.empty[st], (it & 1) ^ 1, -4000000LL - blockIdx.x)) {
+                    atomicExch(abort, 1);
+                    break;
+                }
+                uint8_t* sb = smem + st * STAGE_BYTES;
+                mbar_arrive_expect_tx(&ctl.full[st], STAGE_BYTES);
+                const int k = kt * KT;
+                tma_load_2d(sb, ma_h, &ctl.full[st], ax + k, ay);
+                tma_load_2d(sb + A_BYTES, ma_l, &ctl.full[st], ax + k, ay);
+                tma_load_2d(sb + 2 * A_BYTES, mb_h, &ctl.full[st], bx + k, by);
+                tma_load_2d(sb + 2 * A_BYTES + B_BYTES, mb_l, &ctl.full[st], bx + k, by);
+            }
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---------------- MMA issuer (segmented accumulation as in tc_gemm_kernel)
+        constexpr uint32_t idesc = make_idesc(2u, BM, TBN);
+        const uint32_t xacc = tmem + (uint32_t)XOFF;
+        uint32_t kiter = 0;
+        int seg = 0;
+        bool ok = true;
+        for (int nt = 0; ok; ++nt) {
+            const int s = nt % DAG_SLOTS;
+            if (!mbar_wait(&ctl.task_full[s], (uint32_t)(nt / DAG_SLOTS) & 1, -5000000LL - blockIdx.x)) break;
+            const DagTask tk = ctl.slot[s];
+            if (tk.type == DT_STOP) break;
+            if (seg > 0) {   // the previous task's cross accumulator has been read
+                const int pb = (seg - 1) & 1;
+                if (!mbar_wait(&ctl.tempty[pb], (uint32_t)((seg - 1) >> 1) & 1, -5100000LL - blockIdx.x)) break;
+                tc_fence_after();
+            }
+            auto open_segment = [&](uint32_t& acc_out) -> bool {
+                const int buf = seg & 1;
+                if (!mbar_wait(&ctl.tempty[buf], (uint32_t)((seg >> 1) & 1) ^ 1u, -5200000LL - blockIdx.x))
+                    return false;
+                tc_fence_after();
+                acc_out = tmem + (uint32_t)(buf * TBN);
+                return true;
+            };
+            uint32_t acc = 0;
+            if (!open_segment(acc)) break;
+            int kkc = 0, segpos = 0;
+            for (int kt = 0; kt < DAG_NK && ok; ++kt, ++kiter) {
+                const int st = kiter % DAG_STAGES;
+                const uint32_t it = kiter / DAG_STAGES;
+                if (!mbar_wait(&ctl.full[st], it & 1, -5300000LL - blockIdx.x)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sb = smem_u32(smem + st * STAGE_BYTES);
+                const uint32_t a_hi = sb, a_lo = sb + A_BYTES;
+                const uint32_t b_hi = sb + 2 * A_BYTES, b_lo = b_hi + B_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk, ++kkc, ++segpos) {
+                    if (segpos == DAG_SEG) {
+                        umma_commit(&ctl.tfull[seg & 1]);
+                        ++seg;
+                        segpos = 0;
+                        if (!open_segment(acc)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    const uint32_t off = kk * 32;
+                    const uint32_t acc0 = segpos > 0 ? 1u : 0u;
+                    const uint32_t x0 = kkc > 0 ? 1u : 0u;
+                    umma_tf32(acc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_hi + off), idesc, acc0);
+                    umma_tf32(xacc, desc_sw128_kmajor(a_hi + off), desc_sw128_kmajor(b_lo + off), idesc, x0);
+                    umma_tf32(xacc, desc_sw128_kmajor(a_lo + off), desc_sw128_kmajor(b_hi + off), idesc, 1u);
+                }
+                umma_commit(&ctl.empty[st]);
+            }
+            if (!ok) break;
+            umma_commit(&ctl.tfull[seg & 1]);
+            ++seg;
+        }
+    } else if (warp >= 2 && warp < 6) {
+        // ---------------- epilogue: warp q owns accumulator rows 32q .. 32q+31
+        const int q = warp & 3;
+        uint8_t* wreg = epi + q * epi_boxes_per_warp<TBN>() * kBoxBytes;
+        uint8_t* cbox = wreg;
+        uint8_t* kb = wreg + NCHUNK * kBoxBytes;
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        constexpr int nseg = DAG_NK * 4 / DAG_SEG;
+        int seg = 0;
+        uint32_t cin_use = 0;
+        for (int nt = 0;; ++nt) {
+            const int s = nt % DAG_SLOTS;
+            // the four warps agree on whether a task came (each wait is bounded), so none of
+            // them can be left alone at the task's named barriers
+            const bool got = mbar_wait(&ctl.task_full[s], (uint32_t)(nt / DAG_SLOTS) & 1, -6000000LL - blockIdx.x);
+            if (lane == 0) ctl.epi_ok[q] = got ? 1 : 0;
+            named_bar_epi();
+            const bool all = ctl.epi_ok[0] && ctl.epi_ok[1] && ctl.epi_ok[2] && ctl.epi_ok[3];
+            const DagTask tk = ctl.slot[s];
+            named_bar_epi();
+            if (!all || tk.type == DT_STOP) break;
+            bool ok = true;
+            // segments before the last: add into the running sum (columns SUM_HI ..)
+            for (int sg = 0; sg + 1 < nseg && ok; ++sg, ++seg) {
+                const int sb = seg & 1;
+                ok = mbar_wait(&ctl.tfull[sb], (uint32_t)(seg >> 1) & 1, -6100000LL - blockIdx.x);
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < NCHUNK; ++c) {
+                    const uint32_t src = tmem + (uint32_t)(sb * TBN + c * 32) + lane_off;
+                    const uint32_t dhi = tmem + (uint32_t)(SUM_HI + c * 32) + lane_off;
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(src, r);
+                    if (sg > 0) {
+                        uint32_t t[32];
+                        tmem_ld_32x32b_x32(dhi, t);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int u = 0; u < 32; ++u)
+                            r[u] = __float_as_uint(__uint_as_float(r[u]) + __uint_as_float(t[u]));
+                    } else {
+                        tmem_ld_wait();
+                    }
+                    tmem_st_32x32b_x32(dhi, r);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl.tempty[sb]);
+            }
+            const int buf = seg & 1;
+            const uint32_t use = (uint32_t)(seg >> 1);
+            ++seg;
+            ok = ok && mbar_wait(&ctl.tfull[buf], use & 1, -6200000LL - blockIdx.x);
+            tc_fence_after();
+            const uint32_t acc = tmem + (uint32_t)(buf * TBN) + lane_off;
+
+            // the task's epilogue
+            const long long n = g.n;
+            const int i0 = tk.a * NB + 32 * q;   // first tile row of this warp (global row)
+            float alpha = 1.f, beta = 0.f;
+            float* C = nullptr;
+            long long ldc = n, c_rows = n, c_cols = n, c_col0 = 0;
+            const CUtensorMap* mc = nullptr;
+            bool s_split = false;
+            float *t_hi = nullptr, *t_lo = nullptr;
+            long long t_row0 = 0;
+            long long s_col0 = 0;
+            switch (tk.type) {
+                case DT_PANEL:
+                    s_split = true;
+                    s_col0 = (long long)tk.b * NB;
+                    break;
+                case DT_UPDATE:
+                    alpha = -1.f;
+                    beta = 1.f;
+                    C = g.A;
+                    mc = &maps.ca;
+                    c_col0 = (long long)tk.b * NB;
+                    s_split = (tk.b == tk.c - 1) && (tk.a < tk.b);   // the next panel's input
+                    s_col0 = c_col0;
+                    break;
+                case DT_FIN:
+                    alpha = -1.f;
+                    C = g.U;
+                    ldc = g.d;
+                    c_rows = g.d;
+                    c_cols = g.d;
+                    c_col0 = (long long)tk.b * NB;
+                    t_hi = g.UT_hi;
+                    t_lo = g.UT_lo;
+                    t_row0 = (long long)tk.b * NB;
+                    break;
+                default:   // SUPD
+                    beta = (tk.c == tk.b) ? 0.f : 1.f;
+                    C = g.S;
+                    mc = &maps.cs;
+                    c_col0 = (long long)tk.b * NB;
+                    if (tk.c == tk.a + 1) {
+                        t_hi = g.TT_hi;
+                        t_lo = g.TT_lo;
+                        t_row0 = (long long)tk.b * NB;
+                    }
+                    break;
+            }
+            bool cin_ok = true;
+            if (beta != 0.f) {
+                fence_proxy_async_smem();   // this warp's reads of cbox (previous task) come first
+                __syncwarp();
+                if (lane == 0) {
+                    fence_proxy_async_global();   // C was written by another task (acquired by warp 0)
+                    mbar_arrive_expect_tx(&ctl.cin[q], NCHUNK * kBoxBytes);
+                    for (int c = 0; c < NCHUNK; ++c)
+                        tma_load_2d(cbox + c * kBoxBytes, mc, &ctl.cin[q], (int)(c_col0 + 32 * c), i0);
+                }
+                __syncwarp();
+                cin_ok = mbar_wait(&ctl.cin[q], cin_use & 1, -6300000LL - blockIdx.x);
+                ++cin_use;
+            }
+#pragma unroll 1
+            for (int c = 0; c < NCHUNK; ++c) {
+                uint32_t r[32];
+                if (ok) {
+                    fetch_chunk<TBN, true, false>(tmem, acc, lane_off, c, true, r);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) r[u] = 0u;
+                }
+                if (c == NCHUNK - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ctl.tempty[buf]);
+                }
+                float out[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) out[u] = alpha * __uint_as_float(r[u]);
+                if (beta != 0.f && cin_ok) {
+                    const uint8_t* cb = cbox + c * kBoxBytes;
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 v = *reinterpret_cast<const float4*>(cb + lane * 128 + ((c4 ^ (lane & 7)) << 4));
+                        out[4 * c4 + 0] += v.x;
+                        out[4 * c4 + 1] += v.y;
+                        out[4 * c4 + 2] += v.z;
+                        out[4 * c4 + 3] += v.w;
+                    }
+                }
+                const long long j0 = c_col0 + 32 * c;
+                if (C) emit_block(kb, lane, out, false, C, ldc, c_rows, c_cols, i0, j0);
+                if (s_split || t_hi) {
+                    float hi[32], lo[32];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) split_tf32(out[u], hi[u], lo[u]);
+                    if (s_split) {
+                        emit_block(kb, lane, hi, false, g.RS_hi, n, n, n, i0, s_col0 + 32 * c);
+                        emit_block(kb, lane, lo, false, g.RS_lo, n, n, n, i0, s_col0 + 32 * c);
+                    }
+                    if (t_hi) {
+                        emit_block(kb, lane, hi, true, t_hi, n, n, n, t_row0 + 32 * c, i0);
+                        emit_block(kb, lane, lo, true, t_lo, n, n, n, t_row0 + 32 * c, i0);
+                    }
+                }
+            }
+            // completion: the stores of all four warps, then the counter
+            fence_proxy_async_global();
+            __threadfence();
+            named_bar_epi();
+            if (warp == 2 && lane == 0) {
+                __threadfence();
+                if (ok && cin_ok) atomicAdd(dag_done_ctr(g, tk), 1);
+                else atomicExch(abort, 1);
+                mbar_arrive(&ctl.task_empty[s]);
+            }
+        }
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+}  // namespace gq
+
+namespace gqh {
+
+inline long long chol_n(long long d) { return (d + gq::NB - 1) / gq::NB * gq::NB; }
+
+struct HinvWs {
+    float *A, *S, *RS_hi, *RS_lo, *UT_hi, *UT_lo, *TT_hi, *TT_lo, *Xd_hi, *Xd_lo, *scal;
+    int* ctr;
+    int* rank;   // inverse of a caller's permutation (permuted factorization only)
+};
+
+inline size_t hinv_ws_bytes(long long d) {
+    const long long n = chol_n(d), T = n / gq::NB;
+    return (size_t)(8 * n * n + 2 * n * gq::NB + 64) * sizeof(float) +
+           (size_t)(gq::dag_ctr_ints((int)T) + n) * sizeof(int);
+}
+
+inline HinvWs hinv_ws_carve(void* ws, long long d) {
+    const long long n = chol_n(d), T = n / gq::NB;
+    float* p = static_cast<float*>(ws);
+    HinvWs w;
+    float** big[] = {&w.A, &w.S, &w.RS_hi, &w.RS_lo, &w.UT_hi, &w.UT_lo, &w.TT_hi, &w.TT_lo};
+    for (float** b : big) {
+        *b = p;
+        p += n * n;
+    }
+    w.Xd_hi = p;
+    p += n * gq::NB;
+    w.Xd_lo = p;
+    p += n * gq::NB;
+    w.scal = p;
+    p += 64;
+    w.ctr = reinterpret_cast<int*>(p);
+    w.rank = w.ctr + gq::dag_ctr_ints((int)T);
+    return w;
+}
+
+// Enqueue the whole factorization on stream st: lambda, the damped copy (with the first
+// panel's split), the public U's strictly lower blocks zeroed, the counters cleared, then
+// the persistent kernel (one CTA per SM).
+inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* U, void* ws, cudaStream_t st,
+                            const int* perm = nullptr) {
+    const long long n = chol_n(d);
+    const int T = (int)(n / gq::NB);
+    HinvWs w = hinv_ws_carve(ws, d);
+    {
+        gqh::TimedScope ts__("diag_mean", st);
+        gq::diag_mean_kernel<<<1, 1024, 0, st>>>(H, d, damp_rel, w.scal);
+    }
+    GQ_TRY(cudaGetLastError());
+    if (perm) {   // factor P^T Hd P: validate the permutation, then a gathering damped copy
+        GQ_TRY(cudaMemsetAsync(w.rank, 0xFF, (size_t)d * sizeof(int), st));
+        {
+            gqh::TimedScope ts__("perm_invert", st);
+            gq::perm_invert_kernel<<<(unsigned)((d + 255) / 256), 256, 0, st>>>(perm, d, w.rank);
+        }
+        GQ_TRY(cudaGetLastError());
+        {
+            gqh::TimedScope ts__("damp_copy_perm", st);
+            gq::damp_copy_perm_kernel<<<(unsigned)n, 256, 0, st>>>(H, perm, d, n, w.scal, w.A, w.RS_hi, w.RS_lo);
+        }
+        GQ_TRY(cudaGetLastError());
+    } else {
+        const dim3 grid((unsigned)T, (unsigned)T);
+        {
+            gqh::TimedScope ts__("damp_copy", st);
+            gq::damp_copy_kernel<<<grid, 256, 0, st>>>(H, d, n, w.scal, w.A, w.RS_hi, w.RS_lo);
+        }
+        GQ_TRY(cudaGetLastError());
+    }
+    {
+        gqh::TimedScope ts__("zero_lower", st);
+        gq::zero_lower_blocks_kernel<<<dim3((unsigned)T, (unsigned)T), 256, 0, st>>>(U, d);
+    }
+    GQ_TRY(cudaGetLastError());
+    GQ_TRY(cudaMemsetAsync(w.ctr, 0, (size_t)gq::dag_ctr_ints(T) * sizeof(int), st));
+    const uint64_t N = (uint64_t)n;
+    gq::DagMaps m;
+    if (!make_tmap_2d(&m.rs_hi, w.RS_hi, 4, N, N, N, gq::BM, 32) || !make_tmap_2d(&m.rs_lo, w.RS_lo, 4, N, N, N, gq::BM, 32) ||
+        !make_tmap_2d(&m.xd_hi, w.Xd_hi, 4, N, gq::NB, gq::NB, gq::BM, 32) ||
+        !make_tmap_2d(&m.xd_lo, w.Xd_lo, 4, N, gq::NB, gq::NB, gq::BM, 32) ||
+        !make_tmap_2d(&m.tt_hi, w.TT_hi, 4, N, N, N, gq::BM, 32) || !make_tmap_2d(&m.tt_lo, w.TT_lo, 4, N, N, N, gq::BM, 32) ||
+        !make_tmap_2d(&m.ut_hi, w.UT_hi, 4, N, N, N, gq::BM, 32) || !make_tmap_2d(&m.ut_lo, w.UT_lo, 4, N, N, N, gq::BM, 32) ||
+        !make_tmap_2d(&m.ca, w.A, 4, N, N, N, 32, 32) || !make_tmap_2d(&m.cs, w.S, 4, N, N, N, 32, 32))
+        return cudaErrorInvalidValue;
+    gq::DagArgs a{};
+    a.T = T;
+    a.n = n;
+    a.d = d;
+    a.A = w.A;
+    a.S = w.S;
+    a.RS_hi = w.RS_hi;
+    a.RS_lo = w.RS_lo;
+    a.Xd_hi = w.Xd_hi;
+    a.Xd_lo = w.Xd_lo;
+    a.UT_hi = w.UT_hi;
+    a.UT_lo = w.UT_lo;
+    a.TT_hi = w.TT_hi;
+    a.TT_lo = w.TT_lo;
+    a.U = U;
+    a.ctr = w.ctr;
+    GQ_TRY(ensure_smem_attr(reinterpret_cast<const void*>(gq::chol_dag_kernel), gq::DAG_SMEM));
+    // one CTA per SM (the shared memory allows no second); a single tile needs only the leaf
+    const unsigned grid = T == 1 ? 1u : (unsigned)std::min<long long>(num_sms(), 1 + gq::dag_total_tasks(T));
+    {
+        gqh::TimedScope ts__("chol_dag", st);
+        GQ_TRY(launch_plain(gq::chol_dag_kernel, dim3(grid), dim3(gq::DAG_THREADS), (size_t)gq::DAG_SMEM, st, m,
+                            (const gq::DagArgs)a));
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace gqh

@@ -15,7 +15,7 @@
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "hessian.cuh"
-#include "chol.cuh"
+#include "chol_dag.cuh"
 #include "pack.cuh"
 #include "colloop_host.cuh"
 #include "dqgemm.cuh"
@@ -330,6 +330,22 @@ gptq_status gptq_hessian_accumulate(const void* X, gptq_dtype xt, int64_t n, int
     cudaError_t e = hessian_run(X, xt, n, d_in, H, accumulate ? 1 : 0, ws, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "hessian");
     return GPTQ_OK;
+}
+
+int64_t gptq_chol_schedule(int64_t T, int32_t* tasks, int64_t max_tasks) {
+    if (T < 1 || T > 65536 / gq::NB + 1) return -1;
+    const long long total = gq::dag_total_tasks((int)T);
+    if (tasks) {
+        gq::DagCursor cur{(int)T - 1, 0};
+        for (long long t = 0; t < total && t < max_tasks; ++t) {
+            const gq::DagTask k = gq::dag_decode((int)T, cur, t);
+            tasks[4 * t + 0] = k.type;
+            tasks[4 * t + 1] = k.a;
+            tasks[4 * t + 2] = k.b;
+            tasks[4 * t + 3] = k.c;
+        }
+    }
+    return total;
 }
 
 size_t gptq_prepare_hinv_workspace_bytes(int64_t d_in) {

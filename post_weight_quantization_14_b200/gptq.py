@@ -68,6 +68,7 @@ _SIGS = {
     "gptq_timing_enable": (None, [_int]),
     "gptq_timing_report": (_sz, [ctypes.c_char_p, _sz]),
     "gptq_timing_timeline": (_sz, [ctypes.c_char_p, _sz]),
+    "gptq_chol_schedule": (_i64, [_i64, ctypes.c_void_p, _i64]),
     "gptq_selftest_bounded_wait": (_int, [ctypes.c_uint64, _vp]),
     "gptq_hessian_accumulate_fixed_scratch": (_int, [_vp, _int, _i64, _i64, _vp, _int, _vp]),
     "gptq_act_sum_accumulate": (_int, [_vp, _int, _i64, _i64, _vp, _int, _vp]),
@@ -409,6 +410,17 @@ def gptq_timing_timeline() -> list:
     buf = ctypes.create_string_buffer(n + 16)
     lib().gptq_timing_timeline(buf, len(buf))
     return [tuple(x) for x in json.loads(buf.value.decode())]
+
+
+def gptq_chol_schedule(T: int) -> list:
+    """The factorization kernel's product order for T tiles per side: [(type, a, b, c), ...]
+    (host-side; the encoding is the one include/gptq_b200.h gives)."""
+    total = lib().gptq_chol_schedule(int(T), None, 0)
+    if total < 0:
+        raise GPTQError(int(GPTQ_ERR_INVALID_ARG), f"T out of range ({T})")
+    buf = (ctypes.c_int32 * (4 * total))()
+    lib().gptq_chol_schedule(int(T), buf, total)
+    return [tuple(buf[4 * t:4 * t + 4]) for t in range(total)]
 
 
 def gptq_selftest_bounded_wait(limit_ns: int, stream=None) -> None:
