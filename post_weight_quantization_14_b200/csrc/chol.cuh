@@ -153,23 +153,20 @@ __global__ void __launch_bounds__(256) zero_lower_blocks_kernel(float* __restric
 // Works on the index-reversed block P = J A_jj J, for which the UL factor becomes an
 // ordinary lower Cholesky factor: A_jj = R R^T with R = J L J, and X_jj = R^-1 = J L^-1 J.
 //
-// Right-looking, blocked by 32 columns.  For panel kb (columns k0 = 32 kb .. k0 + 31):
-//   A. one warp factors the 32x32 diagonal block in registers, lane = row.  The only
-//      dependency from one pivot to the next is one shuffle of the next pivot, which each
-//      lane keeps up to date from its own multipliers; the multiplier column reaches the
-//      other rows through shared memory, off that chain; 1/L_kk = rsqrt with one Newton step.
-//   B. the rows below the block (one thread per row, 32 - 96 rows) solve against L_kk by
-//      substitution with the reciprocals of step A; meanwhile one otherwise idle warp forms
-//      X_kk = L_kk^-1 by forward substitution (lane = column).
-//   C. all threads apply the rank-32 update of the trailing lower triangle on 4x4
-//      register micro-tiles.
-// Then the off-diagonal blocks of X = L^-1, block row by block row:
-// X_ij = -X_ii sum_{k=j}^{i-1} L_ik X_kj, the sums first (kept in X's free upper blocks).
-// Writes X_jj (upper, zeros below the diagonal) as U_hi = tf32(X_jj) and U_lo = X_jj - U_hi
-// (exact, not rounded: the tensor pipe reads only its tf32 part); U_hi + U_lo restores
-// X_jj exactly for chol_diag_out_kernel.
+// Right-looking, blocked by 32 columns, on 256 threads: warp 0 (F) factors the 32x32
+// diagonal blocks; warps 1-7 (W) do everything else, around F's chain.  For panel kb
+// (columns k0 = 32 kb .. k0 + 31):
+//   F: the diagonal block in registers, lane = row (leaf_diag_factor);
+//   W: the rows below by substitution (one thread per row), X_kk = L_kk^-1 (one warp), the
+//      rank-32 update of the next diagonal block, which releases F for panel kb+1; then,
+//      while F factors it, the rest of the trailing update and the inverse's block rows
+//      X_ij = -X_ii sum_{k=j}^{i-1} L_ik X_kj (the sums as soon as their inputs exist, the
+//      products by X_ii once it is known).
+// F and W meet on named barriers (3: F's block done, 4: the next block updated); W syncs
+// on barrier 2 among its 224 threads.
 constexpr int LS = NB + 4;   // leaf smem row stride (16-byte aligned rows)
 constexpr int LEAF_THREADS = 256;
+constexpr int LEAF_W = LEAF_THREADS - 32;   // threads of warps 1-7
 
 struct LeafSmem {
     float P[NB][LS];         // reversed block; lower triangle holds the Schur complement
@@ -177,15 +174,21 @@ struct LeafSmem {
     float LT[NB][LS];        // L transposed: LT[m][r] = L[r][m]
     float XDT[4][32][36];    // diagonal inverses transposed: XDT[i][m][r] = X_ii[r][m]
     float rinv[NB];          // 1 / L_kk
-    float col[2][32];        // multiplier column of the current pivot (double-buffered)
+    float lc[32][32];        // multiplier columns of the diagonal block being factored: lc[k][i] = L_ik
 };
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void nbar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+__device__ __forceinline__ void nbar_arrive(int id, int n) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void wsync() { nbar_sync(2, LEAF_W); }
 
-// A. Factor the 32x32 diagonal block at (k0, k0) with one warp; lane i holds row k0 + i.
-// Per pivot k the pivot value is the only shuffle on the dependency chain (each lane keeps
-// its own diagonal entry current); the multipliers L_jk reach the other rows through a
-// double-buffered column in shared memory (one store, a warp barrier and vector loads).
+// F: factor the 32x32 diagonal block at (k0, k0); lane i holds row k0 + i.  Per pivot k the
+// dependency chain is: the pivot (one shuffle of the diagonal entry that lane k keeps current
+// from its own multipliers), 1/sqrt (rsqrt and one Newton step), the multipliers, and the
+// next column's update with one more shuffle (L_{k+1,k}); the columns past it take the
+// multipliers through shared memory, one pivot behind, off that chain.
 // Writes L_kk (lower, zeros above) to P and LT, and 1/L_kk to rinv.
 __device__ __forceinline__ void leaf_diag_factor(LeafSmem& S, int k0, int lane, int jb) {
     constexpr unsigned FULL = 0xffffffffu;
@@ -211,21 +214,25 @@ __device__ __forceinline__ void leaf_diag_factor(LeafSmem& S, int k0, int lane, 
         bad = (bad < 0 && !pk) ? k : bad;
         float r = rsqrtf(p);
         r = r * fmaf(-0.5f * p * r, r, 1.5f);       // one Newton step for 1/sqrt(p)
-        const float l = (lane == k) ? p * r : a[k] * r;   // L_kk = sqrt(p); L_ik = P_ik / L_kk
-        a[k] = l;
+        float l = (lane == k) ? p * r : a[k] * r;   // L_kk = sqrt(p); L_ik = P_ik / L_kk
+        if (lane < k) l = 0.f;                      // rows above: finished, untouched
+        a[k] = (lane >= k) ? l : a[k];
         if (lane > k) dg = fmaf(-l, l, dg);
         rr = (lane == k) ? r : rr;
         if (k < 31) {
-            float* cb = S.col[k & 1];
-            cb[lane] = l;
-            __syncwarp();
+            const float c1 = __shfl_sync(FULL, l, k + 1);   // L_{k+1,k}: the next column first
+            a[k + 1] = fmaf(-l, c1, a[k + 1]);
+            if (k < 30) {
+                S.lc[k][lane] = l;
+                __syncwarp();
 #pragma unroll
-            for (int j4 = (k + 1) >> 2; j4 < 8; ++j4) {
-                const float4 c4 = ld4(&cb[4 * j4]);    // L_jk for j = 4 j4 ..
-                if (4 * j4 + 0 > k) a[4 * j4 + 0] = fmaf(-l, c4.x, a[4 * j4 + 0]);
-                if (4 * j4 + 1 > k) a[4 * j4 + 1] = fmaf(-l, c4.y, a[4 * j4 + 1]);
-                if (4 * j4 + 2 > k) a[4 * j4 + 2] = fmaf(-l, c4.z, a[4 * j4 + 2]);
-                if (4 * j4 + 3 > k) a[4 * j4 + 3] = fmaf(-l, c4.w, a[4 * j4 + 3]);
+                for (int j4 = (k + 2) >> 2; j4 < 8; ++j4) {
+                    const float4 c4 = ld4(&S.lc[k][4 * j4]);   // L_jk for j = 4 j4 ..
+                    if (4 * j4 + 0 >= k + 2) a[4 * j4 + 0] = fmaf(-l, c4.x, a[4 * j4 + 0]);
+                    if (4 * j4 + 1 >= k + 2) a[4 * j4 + 1] = fmaf(-l, c4.y, a[4 * j4 + 1]);
+                    if (4 * j4 + 2 >= k + 2) a[4 * j4 + 2] = fmaf(-l, c4.z, a[4 * j4 + 2]);
+                    if (4 * j4 + 3 >= k + 2) a[4 * j4 + 3] = fmaf(-l, c4.w, a[4 * j4 + 3]);
+                }
             }
         }
     }
@@ -240,7 +247,7 @@ __device__ __forceinline__ void leaf_diag_factor(LeafSmem& S, int k0, int lane, 
     }
 }
 
-// B. Rows k0+32 .. 127 (one thread each): L_i,kb = P_i,kb L_kk^-T by substitution.
+// W: row i (below the diagonal block): L_i,kb = P_i,kb L_kk^-T by substitution.
 __device__ __forceinline__ void leaf_panel_solve(LeafSmem& S, int k0, int i) {
     float a[32];
 #pragma unroll
@@ -268,17 +275,43 @@ __device__ __forceinline__ void leaf_panel_solve(LeafSmem& S, int k0, int i) {
     for (int j = 0; j < 32; ++j) S.LT[k0 + j][i] = a[j];
 }
 
-// C. Rank-32 update of the trailing lower triangle (rows and columns >= k0 + 32) with the
-// panel just factored; 4x4 micro-tiles on the lower triangle of tiles only.
-template <int NT = LEAF_THREADS>
-__device__ __forceinline__ void leaf_trailing_update(LeafSmem& S, int k0, int tid) {
+// W: rank-32 update of the next diagonal block (rows and columns k0+32 .. k0+63, lower
+// triangle) by panel kb, on 2x2 micro-tiles (136 threads).
+__device__ __forceinline__ void leaf_next_diag_update(LeafSmem& S, int k0, int wt) {
+    if (wt >= 136) return;
+    int tr = 0, rem = wt;
+    while (rem > tr) {
+        rem -= tr + 1;
+        ++tr;
+    }
+    const int r0 = k0 + 32 + 2 * tr, c0 = k0 + 32 + 2 * rem;
+    float acc[2][2] = {};
+#pragma unroll 8
+    for (int m = 0; m < 32; ++m) {
+        const float2 a = *reinterpret_cast<const float2*>(&S.LT[k0 + m][r0]);
+        const float2 b = *reinterpret_cast<const float2*>(&S.LT[k0 + m][c0]);
+        acc[0][0] = fmaf(a.x, b.x, acc[0][0]);
+        acc[0][1] = fmaf(a.x, b.y, acc[0][1]);
+        acc[1][0] = fmaf(a.y, b.x, acc[1][0]);
+        acc[1][1] = fmaf(a.y, b.y, acc[1][1]);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) S.P[r0 + i][c0 + j] -= acc[i][j];
+}
+
+// W: the rest of the rank-32 trailing update (rows and columns >= k0 + 32, lower
+// triangle, without the next diagonal block), 4x4 micro-tiles.
+__device__ __forceinline__ void leaf_rest_update(LeafSmem& S, int k0, int wt) {
     const int t0 = k0 + 32, tn = (NB - t0) >> 2;
     const int ntask = tn * (tn + 1) / 2;
-    for (int task = tid; task < ntask; task += NT) {
+    for (int task = wt; task < ntask; task += LEAF_W) {
         int tr = (int)((sqrtf(8.f * (float)task + 1.f) - 1.f) * 0.5f);
         while (tr * (tr + 1) / 2 > task) --tr;
         while ((tr + 1) * (tr + 2) / 2 <= task) ++tr;
         const int tc = task - tr * (tr + 1) / 2;
+        if (tr < 8) continue;   // rows of the next diagonal block: leaf_next_diag_update
         const int r0 = t0 + 4 * tr, c0 = t0 + 4 * tc;
         float acc[4][4] = {};
 #pragma unroll 8
@@ -304,7 +337,7 @@ __device__ __forceinline__ void leaf_trailing_update(LeafSmem& S, int k0, int ti
 }
 
 // X_ii = L_ii^-1 by forward substitution, one warp, lane = column j:
-// x_m = (delta_mj - sum_{m' < m} L_mm' x_m') / L_mm, with 1/L_mm from step A.
+// x_m = (delta_mj - sum_{m' < m} L_mm' x_m') / L_mm, with 1/L_mm from leaf_diag_factor.
 __device__ __forceinline__ void leaf_diag_inverse(LeafSmem& S, int i, int lane) {
     const int k0 = 32 * i;
     float x[32], s[32];
@@ -330,11 +363,10 @@ __device__ __forceinline__ void leaf_diag_inverse(LeafSmem& S, int i, int lane) 
             make_float4(x[4 * m4], x[4 * m4 + 1], x[4 * m4 + 2], x[4 * m4 + 3]);
 }
 
-// Block row i of X = L^-1 with all threads: T_ij = sum_{k=j}^{i-1} L_ik X_kj into X's free
-// upper block (j, i), then X_ij = -X_ii T_ij.  Block rows < i must be complete.
-template <int NT = LEAF_THREADS>
-__device__ __forceinline__ void leaf_x_block_row(LeafSmem& S, int i, int tid) {
-    for (int task = tid; task < 64 * i; task += NT) {
+// Block row i of X = L^-1, first part: T_ij = sum_{k=j}^{i-1} L_ik X_kj for j < i, kept in
+// X's free upper block (j, i).  Needs block rows < i of X and L's block row i.
+__device__ __forceinline__ void leaf_band_sums(LeafSmem& S, int i, int wt) {
+    for (int task = wt; task < 64 * i; task += LEAF_W) {
         const int j = task >> 6, r0 = 4 * ((task >> 3) & 7), c0 = 4 * (task & 7);
         float acc[4][4] = {};
         for (int k = j; k < i; ++k) {
@@ -354,8 +386,11 @@ __device__ __forceinline__ void leaf_x_block_row(LeafSmem& S, int i, int tid) {
             *reinterpret_cast<float4*>(&S.X[32 * j + r0 + u][32 * i + c0]) =
                 make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
     }
-    __syncthreads();
-    for (int task = tid; task < 64 * i; task += NT) {
+}
+
+// Second part: X_ij = -X_ii T_ij (X_ii from leaf_diag_inverse).
+__device__ __forceinline__ void leaf_band_mul(LeafSmem& S, int i, int wt, int nthreads) {
+    for (int task = wt; task < 64 * i; task += nthreads) {
         const int j = task >> 6, r0 = 4 * ((task >> 3) & 7), c0 = 4 * (task & 7);
         float acc[4][4] = {};
 #pragma unroll 8
@@ -372,6 +407,38 @@ __device__ __forceinline__ void leaf_x_block_row(LeafSmem& S, int i, int tid) {
         for (int u = 0; u < 4; ++u)
             *reinterpret_cast<float4*>(&S.X[32 * i + r0 + u][32 * j + c0]) =
                 make_float4(-acc[u][0], -acc[u][1], -acc[u][2], -acc[u][3]);
+    }
+}
+
+// The whole leaf on P (loaded, reversed, and visible to all 256 threads): L in P/LT and
+// X = L^-1 in S.X (lower) on return, visible to all threads.
+__device__ __forceinline__ void leaf_factor(LeafSmem& S, int jb) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (warp == 0) {
+        for (int kb = 0; kb < 4; ++kb) {
+            if (kb > 0) nbar_sync(4, LEAF_THREADS);   // W has updated diagonal block kb
+            leaf_diag_factor(S, 32 * kb, lane, jb);
+            nbar_arrive(3, LEAF_THREADS);             // diagonal block kb factored
+        }
+    } else {
+        const int wt = tid - 32;
+        for (int kb = 0; kb < 4; ++kb) {
+            const int k0 = 32 * kb;
+            nbar_sync(3, LEAF_THREADS);
+            if (wt < NB - k0 - 32) leaf_panel_solve(S, k0, k0 + 32 + wt);   // rows below, one each
+            else if (warp == 7) leaf_diag_inverse(S, kb, lane);
+            wsync();
+            if (kb < 3) {
+                leaf_next_diag_update(S, k0, wt);
+                nbar_arrive(4, LEAF_THREADS);
+                leaf_rest_update(S, k0, wt);
+            }
+            if (kb >= 1) {
+                leaf_band_mul(S, kb, wt, LEAF_W);
+                wsync();
+            }
+            if (kb < 3) leaf_band_sums(S, kb + 1, wt);
+        }
     }
     __syncthreads();
 }

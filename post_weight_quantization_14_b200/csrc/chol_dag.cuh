@@ -29,10 +29,26 @@ namespace gq {
 
 enum : int { DT_PANEL = 0, DT_UPDATE = 1, DT_FIN = 2, DT_SUPD = 3, DT_STOP = 15 };
 
+// Optional event trace for profiling builds (GQ_DAG_TRACE defined): %globaltimer stamps of
+// each leaf (4 per leaf) and each ticket (8 per ticket, after 4 T leaf slots): fetched,
+// inputs ready, first stage landed, accumulator ready, done, CTA.
+#ifdef GQ_DAG_TRACE
+__device__ unsigned long long* g_dag_trace = nullptr;
+#define DAG_TRACE(slot, val)                                   \
+    do {                                                       \
+        if (g_dag_trace) g_dag_trace[(slot)] = (val);          \
+    } while (0)
+#else
+#define DAG_TRACE(slot, val) \
+    do {                     \
+    } while (0)
+#endif
+
 // PANEL(j, i): a = i, b = j.  UPDATE(j, i, k): a = i, b = k, c = j.
 // FIN(i, m): a = i, b = m.    SUPD(i, k, m): a = i, b = m, c = k.
 struct DagTask {
     int type, a, b, c;
+    int t;   // ticket (set by the fetching CTA)
 };
 
 __host__ __device__ inline long long dag_step_tasks(int T, int j) {
@@ -52,25 +68,25 @@ __host__ __device__ inline long long dag_total_tasks(int T) {
 // Task idx of step j.
 __host__ __device__ inline DagTask dag_step_task(int T, int j, long long idx) {
     if (j >= 1) {
-        if (idx == 0) return DagTask{DT_PANEL, j - 1, j, 0};
-        if (idx == 1) return DagTask{DT_UPDATE, j - 1, j - 1, j};
+        if (idx == 0) return DagTask{DT_PANEL, j - 1, j, 0, 0};
+        if (idx == 1) return DagTask{DT_UPDATE, j - 1, j - 1, j, 0};
         idx -= 2;
     }
     if (j >= 2) {
-        if (idx < j - 1) return DagTask{DT_PANEL, j - 2 - (int)idx, j, 0};
+        if (idx < j - 1) return DagTask{DT_PANEL, j - 2 - (int)idx, j, 0, 0};
         idx -= j - 1;
-        if (idx < j - 1) return DagTask{DT_UPDATE, j - 2 - (int)idx, j - 1, j};
+        if (idx < j - 1) return DagTask{DT_UPDATE, j - 2 - (int)idx, j - 1, j, 0};
         idx -= j - 1;
     }
-    if (idx < T - 1 - j) return DagTask{DT_FIN, j, j + 1 + (int)idx, 0};
+    if (idx < T - 1 - j) return DagTask{DT_FIN, j, j + 1 + (int)idx, 0, 0};
     idx -= T - 1 - j;
-    if (idx < (long long)j * (T - j)) return DagTask{DT_SUPD, (int)(idx % j), j + (int)(idx / j), j};
+    if (idx < (long long)j * (T - j)) return DagTask{DT_SUPD, (int)(idx % j), j + (int)(idx / j), j, 0};
     idx -= (long long)j * (T - j);
     for (int k = j - 2; k >= 0; --k) {   // far updates, nearest block column first
-        if (idx < k + 1) return DagTask{DT_UPDATE, (int)idx, k, j};
+        if (idx < k + 1) return DagTask{DT_UPDATE, (int)idx, k, j, 0};
         idx -= k + 1;
     }
-    return DagTask{DT_STOP, 0, 0, 0};
+    return DagTask{DT_STOP, 0, 0, 0, 0};
 }
 
 // Tickets arrive in increasing order per CTA: the cursor walks the steps forward.
@@ -83,7 +99,7 @@ __host__ __device__ inline DagTask dag_decode(int T, DagCursor& cur, long long t
         cur.base += dag_step_tasks(T, cur.j);
         --cur.j;
     }
-    if (cur.j < 0) return DagTask{DT_STOP, 0, 0, 0};
+    if (cur.j < 0) return DagTask{DT_STOP, 0, 0, 0, 0};
     return dag_step_task(T, cur.j, t - cur.base);
 }
 
@@ -208,7 +224,7 @@ __device__ __forceinline__ void named_bar_epi() { asm volatile("bar.sync 1, 128;
 __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, DagCtl& ctl) {
     const int T = g.T;
     const long long n = g.n, d = g.d;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     int* c = g.ctr;
     int* abort = c + 2;
     int* a_cnt = c + 4;
@@ -216,7 +232,10 @@ __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, Dag
     int* diag_done = leaf_done + T;
     for (int j = T - 1; j >= 0; --j) {
         const long long jb = (long long)j * NB;
-        if (tid == 0) ctl.flag = dag_wait_ge(&a_cnt[j * T + j], T - 1 - j, abort, -(2000000LL + j)) ? 1 : 0;
+        if (tid == 0) {
+            ctl.flag = dag_wait_ge(&a_cnt[j * T + j], T - 1 - j, abort, -(2000000LL + j)) ? 1 : 0;
+            DAG_TRACE(4 * j, globaltimer_ns());
+        }
         __syncthreads();
         if (!ctl.flag) return;
         // P[127-r][127-c] = A[r][c]
@@ -238,19 +257,7 @@ __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, Dag
             }
         }
         __syncthreads();
-        for (int kb = 0; kb < 4; ++kb) {
-            const int k0 = 32 * kb;
-            if (warp == 0) leaf_diag_factor(S, k0, lane, (int)jb);
-            __syncthreads();
-            if (tid >= 32 && tid < 32 + (NB - k0 - 32)) leaf_panel_solve(S, k0, k0 + tid);   // rows k0+32 ..
-            else if (warp == 7) leaf_diag_inverse(S, kb, lane);
-            __syncthreads();
-            if (kb < 3) {
-                leaf_trailing_update<DAG_THREADS>(S, k0, tid);
-                __syncthreads();
-            }
-        }
-        for (int i = 1; i < 4; ++i) leaf_x_block_row<DAG_THREADS>(S, i, tid);
+        leaf_factor(S, (int)jb);
 
         // X_jj (block of U = J X J, upper) as its tf32 split, row-major: the operand of the
         // panels of step j and of row j of U
@@ -276,6 +283,7 @@ __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, Dag
         if (tid == 0) {
             __threadfence();
             atomicAdd(&leaf_done[j], 1);
+            DAG_TRACE(4 * j + 1, globaltimer_ns());
         }
         // U_jj to the public output (clipped to d; d % 4 == 0) and its transposed split
 #pragma unroll 4
@@ -307,6 +315,7 @@ __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, Dag
         if (tid == 0) {
             __threadfence();
             atomicAdd(&diag_done[j], 1);
+            DAG_TRACE(4 * j + 2, globaltimer_ns());
         }
     }
 }
@@ -387,8 +396,14 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
             const bool slot_ok = mbar_wait(&ctl.task_empty[s], (uint32_t)((nt / DAG_SLOTS) & 1) ^ 1u, -3000000LL - blockIdx.x);
             if (slot_ok && !ld_volatile_s32(abort)) {
                 const long long t = atomicAdd(g.ctr, 1);
+                DAG_TRACE(4 * T + 8 * t + 0, globaltimer_ns());
                 tk = dag_decode(T, cur, t);
                 if (tk.type != DT_STOP && !dag_deps(g, tk)) tk.type = DT_STOP;
+                if (tk.type != DT_STOP) {
+                    DAG_TRACE(4 * T + 8 * t + 1, globaltimer_ns());
+                    DAG_TRACE(4 * T + 8 * t + 5, blockIdx.x);
+                    tk.t = (int)t;
+                }
             } else if (!slot_ok) {
                 atomicExch(abort, 1);
             }
@@ -467,6 +482,7 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
                     ok = false;
                     break;
                 }
+                if (kt == 0) DAG_TRACE(4 * T + 8 * (long long)tk.t + 2, globaltimer_ns());
                 tc_fence_after();
                 const uint32_t sb = smem_u32(smem + st * STAGE_BYTES);
                 const uint32_t a_hi = sb, a_lo = sb + A_BYTES;
@@ -549,6 +565,7 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
             const uint32_t use = (uint32_t)(seg >> 1);
             ++seg;
             ok = ok && mbar_wait(&ctl.tfull[buf], use & 1, -6200000LL - blockIdx.x);
+            if (warp == 2 && lane == 0) DAG_TRACE(4 * T + 8 * (long long)tk.t + 3, globaltimer_ns());
             tc_fence_after();
             const uint32_t acc = tmem + (uint32_t)(buf * TBN) + lane_off;
 
@@ -613,6 +630,7 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
                 __syncwarp();
                 cin_ok = mbar_wait(&ctl.cin[q], cin_use & 1, -6300000LL - blockIdx.x);
                 ++cin_use;
+                if (warp == 2 && lane == 0) DAG_TRACE(4 * T + 8 * (long long)tk.t + 7, globaltimer_ns());
             }
 #pragma unroll 1
             for (int c = 0; c < NCHUNK; ++c) {
@@ -659,6 +677,7 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
                 }
             }
             // completion: the stores of all four warps, then the counter
+            if (warp == 2 && lane == 0) DAG_TRACE(4 * T + 8 * (long long)tk.t + 6, globaltimer_ns());
             fence_proxy_async_global();
             __threadfence();
             named_bar_epi();
@@ -666,6 +685,7 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
                 __threadfence();
                 if (ok && cin_ok) atomicAdd(dag_done_ctr(g, tk), 1);
                 else atomicExch(abort, 1);
+                DAG_TRACE(4 * T + 8 * (long long)tk.t + 4, globaltimer_ns());
                 mbar_arrive(&ctl.task_empty[s]);
             }
         }
