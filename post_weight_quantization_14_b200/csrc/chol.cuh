@@ -303,10 +303,10 @@ __device__ __forceinline__ void leaf_next_diag_update(LeafSmem& S, int k0, int w
 
 // W: the rest of the rank-32 trailing update (rows and columns >= k0 + 32, lower
 // triangle, without the next diagonal block), 4x4 micro-tiles.
-__device__ __forceinline__ void leaf_rest_update(LeafSmem& S, int k0, int wt) {
+__device__ __forceinline__ void leaf_rest_update(LeafSmem& S, int k0, int wt, int nthreads) {
     const int t0 = k0 + 32, tn = (NB - t0) >> 2;
     const int ntask = tn * (tn + 1) / 2;
-    for (int task = wt; task < ntask; task += LEAF_W) {
+    for (int task = wt; task < ntask; task += nthreads) {
         int tr = (int)((sqrtf(8.f * (float)task + 1.f) - 1.f) * 0.5f);
         while (tr * (tr + 1) / 2 > task) --tr;
         while ((tr + 1) * (tr + 2) / 2 <= task) ++tr;
@@ -365,8 +365,8 @@ __device__ __forceinline__ void leaf_diag_inverse(LeafSmem& S, int i, int lane) 
 
 // Block row i of X = L^-1, first part: T_ij = sum_{k=j}^{i-1} L_ik X_kj for j < i, kept in
 // X's free upper block (j, i).  Needs block rows < i of X and L's block row i.
-__device__ __forceinline__ void leaf_band_sums(LeafSmem& S, int i, int wt) {
-    for (int task = wt; task < 64 * i; task += LEAF_W) {
+__device__ __forceinline__ void leaf_band_sums(LeafSmem& S, int i, int wt, int nthreads) {
+    for (int task = wt; task < 64 * i; task += nthreads) {
         const int j = task >> 6, r0 = 4 * ((task >> 3) & 7), c0 = 4 * (task & 7);
         float acc[4][4] = {};
         for (int k = j; k < i; ++k) {
@@ -412,16 +412,34 @@ __device__ __forceinline__ void leaf_band_mul(LeafSmem& S, int i, int wt, int nt
 
 // The whole leaf on P (loaded, reversed, and visible to all 256 threads): L in P/LT and
 // X = L^-1 in S.X (lower) on return, visible to all threads.
+// Optional event trace for profiling builds (GQ_DAG_TRACE defined): %globaltimer stamps,
+// 16 slots per leaf (the factorization kernel adds 8 per product task after them).
+#ifdef GQ_DAG_TRACE
+__device__ unsigned long long* g_dag_trace = nullptr;
+#define GQ_LEAF_STAMP(slot)                                                              \
+    do {                                                                                 \
+        if (g_dag_trace) g_dag_trace[16 * (long long)(jb >> 7) + (slot)] = globaltimer_ns(); \
+    } while (0)
+#else
+#define GQ_LEAF_STAMP(slot) \
+    do {                    \
+    } while (0)
+#endif
 __device__ __forceinline__ void leaf_factor(LeafSmem& S, int jb) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (warp == 0) {
         for (int kb = 0; kb < 4; ++kb) {
             if (kb > 0) nbar_sync(4, LEAF_THREADS);   // W has updated diagonal block kb
             leaf_diag_factor(S, 32 * kb, lane, jb);
+            if (lane == 0) GQ_LEAF_STAMP(3 + kb);
             nbar_arrive(3, LEAF_THREADS);             // diagonal block kb factored
         }
     } else {
+        // while F factors, warp 4 (which shares F's scheduler) stays out of the way: the
+        // work that overlaps a diagonal factor runs on warps 1-3 and 5-7
         const int wt = tid - 32;
+        const int wo = warp < 4 ? wt : wt - 32;   // index among warps 1-3, 5-7
+        constexpr int NO = LEAF_W - 32;
         for (int kb = 0; kb < 4; ++kb) {
             const int k0 = 32 * kb;
             nbar_sync(3, LEAF_THREADS);
@@ -431,13 +449,16 @@ __device__ __forceinline__ void leaf_factor(LeafSmem& S, int jb) {
             if (kb < 3) {
                 leaf_next_diag_update(S, k0, wt);
                 nbar_arrive(4, LEAF_THREADS);
-                leaf_rest_update(S, k0, wt);
+                if (warp != 4) leaf_rest_update(S, k0, wo, NO);
             }
-            if (kb >= 1) {
+            if (kb == 3) {   // F is done: all of W
                 leaf_band_mul(S, kb, wt, LEAF_W);
                 wsync();
+            } else if (kb >= 1) {
+                if (warp != 4) leaf_band_mul(S, kb, wo, NO);
+                wsync();
             }
-            if (kb < 3) leaf_band_sums(S, kb + 1, wt);
+            if (kb < 3 && warp != 4) leaf_band_sums(S, kb + 1, wo, NO);
         }
     }
     __syncthreads();

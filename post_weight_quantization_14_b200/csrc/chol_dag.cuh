@@ -19,9 +19,9 @@
 // the counters of the tasks it reads from, all of which come earlier in that order; so the
 // lowest unfinished task can always run, whatever subset of CTAs is resident.  Within a CTA
 // the task fetch and TMA loads (warp 0), the MMAs (warp 1) and the epilogue (warps 2-5) are
-// pipelined across tasks as in tc_gemm_kernel.  Counters are released with a gpu-scope fence
-// after the producing stores and acquired before the consuming loads (with a proxy fence in
-// front of TMA reads).
+// pipelined across tasks as in tc_gemm_kernel.  Counters are released by one thread after a
+// barrier over the producing threads' stores (gpu-scope fence, then the atomic) and acquired
+// before the consuming loads (with a proxy fence in front of TMA reads).
 #pragma once
 #include "chol.cuh"
 
@@ -30,10 +30,9 @@ namespace gq {
 enum : int { DT_PANEL = 0, DT_UPDATE = 1, DT_FIN = 2, DT_SUPD = 3, DT_STOP = 15 };
 
 // Optional event trace for profiling builds (GQ_DAG_TRACE defined): %globaltimer stamps of
-// each leaf (4 per leaf) and each ticket (8 per ticket, after 4 T leaf slots): fetched,
+// each leaf (16 per leaf) and each ticket (8 per ticket, after 16 T leaf slots): fetched,
 // inputs ready, first stage landed, accumulator ready, done, CTA.
 #ifdef GQ_DAG_TRACE
-__device__ unsigned long long* g_dag_trace = nullptr;
 #define DAG_TRACE(slot, val)                                   \
     do {                                                       \
         if (g_dag_trace) g_dag_trace[(slot)] = (val);          \
@@ -218,6 +217,13 @@ static_assert(NB * NB / 4 == 16 * DAG_THREADS, "leaf load and store loops");
 
 __device__ __forceinline__ void named_bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+struct DagMaps {
+    // operands (128 x 32 boxes) and C in/out (32 x 32 boxes), all 128-byte swizzled
+    CUtensorMap rs_hi, rs_lo, xd_hi, xd_lo, tt_hi, tt_lo, ut_hi, ut_lo, ca, cs;
+    // stores of the epilogue (32 x 32 boxes): R's split, U^T's and S^T's splits, the public U
+    CUtensorMap rs_hi32, rs_lo32, ut_hi32, ut_lo32, tt_hi32, tt_lo32, u32;
+};
+
 // ---------------------------------------------------------------------------------------
 // The leaf CTA: LEAF(j) for j = T-1 .. 0 (256 threads; the pieces are chol.cuh's).
 // ---------------------------------------------------------------------------------------
@@ -234,7 +240,7 @@ __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, Dag
         const long long jb = (long long)j * NB;
         if (tid == 0) {
             ctl.flag = dag_wait_ge(&a_cnt[j * T + j], T - 1 - j, abort, -(2000000LL + j)) ? 1 : 0;
-            DAG_TRACE(4 * j, globaltimer_ns());
+            DAG_TRACE(16 * j, globaltimer_ns());
         }
         __syncthreads();
         if (!ctl.flag) return;
@@ -257,7 +263,9 @@ __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, Dag
             }
         }
         __syncthreads();
+        if (tid == 0) DAG_TRACE(16 * j + 12, globaltimer_ns());
         leaf_factor(S, (int)jb);
+        if (tid == 0) DAG_TRACE(16 * j + 11, globaltimer_ns());
 
         // X_jj (block of U = J X J, upper) as its tf32 split, row-major: the operand of the
         // panels of step j and of row j of U
@@ -277,13 +285,12 @@ __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, Dag
             *reinterpret_cast<float4*>(xh + r * NB + cc) = make_float4(h[0], h[1], h[2], h[3]);
             *reinterpret_cast<float4*>(xl + r * NB + cc) = make_float4(l[0], l[1], l[2], l[3]);
         }
-        fence_proxy_async_global();
-        __threadfence();
         __syncthreads();
-        if (tid == 0) {
+        if (tid == 0) {   // release: the CTA's stores (ordered by the barrier), then the counter
+            fence_proxy_async_global();
             __threadfence();
             atomicAdd(&leaf_done[j], 1);
-            DAG_TRACE(4 * j + 1, globaltimer_ns());
+            DAG_TRACE(16 * j + 1, globaltimer_ns());
         }
         // U_jj to the public output (clipped to d; d % 4 == 0) and its transposed split
 #pragma unroll 4
@@ -309,13 +316,12 @@ __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, Dag
             *reinterpret_cast<float4*>(g.UT_hi + (jb + col) * n + jb + r4) = make_float4(h[0], h[1], h[2], h[3]);
             *reinterpret_cast<float4*>(g.UT_lo + (jb + col) * n + jb + r4) = make_float4(l[0], l[1], l[2], l[3]);
         }
-        fence_proxy_async_global();
-        __threadfence();
         __syncthreads();
         if (tid == 0) {
+            fence_proxy_async_global();
             __threadfence();
             atomicAdd(&diag_done[j], 1);
-            DAG_TRACE(4 * j + 2, globaltimer_ns());
+            DAG_TRACE(16 * j + 2, globaltimer_ns());
         }
     }
 }
@@ -323,9 +329,6 @@ __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, Dag
 // ---------------------------------------------------------------------------------------
 // Product CTAs.
 // ---------------------------------------------------------------------------------------
-struct DagMaps {
-    CUtensorMap rs_hi, rs_lo, xd_hi, xd_lo, tt_hi, tt_lo, ut_hi, ut_lo, ca, cs;
-};
 
 __global__ void __launch_bounds__(DAG_THREADS, 1)
     chol_dag_kernel(const __grid_constant__ DagMaps maps, const DagArgs g) {
@@ -396,12 +399,12 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
             const bool slot_ok = mbar_wait(&ctl.task_empty[s], (uint32_t)((nt / DAG_SLOTS) & 1) ^ 1u, -3000000LL - blockIdx.x);
             if (slot_ok && !ld_volatile_s32(abort)) {
                 const long long t = atomicAdd(g.ctr, 1);
-                DAG_TRACE(4 * T + 8 * t + 0, globaltimer_ns());
+                DAG_TRACE(16 * T + 8 * t + 0, globaltimer_ns());
                 tk = dag_decode(T, cur, t);
                 if (tk.type != DT_STOP && !dag_deps(g, tk)) tk.type = DT_STOP;
                 if (tk.type != DT_STOP) {
-                    DAG_TRACE(4 * T + 8 * t + 1, globaltimer_ns());
-                    DAG_TRACE(4 * T + 8 * t + 5, blockIdx.x);
+                    DAG_TRACE(16 * T + 8 * t + 1, globaltimer_ns());
+                    DAG_TRACE(16 * T + 8 * t + 5, blockIdx.x);
                     tk.t = (int)t;
                 }
             } else if (!slot_ok) {
@@ -482,7 +485,7 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
                     ok = false;
                     break;
                 }
-                if (kt == 0) DAG_TRACE(4 * T + 8 * (long long)tk.t + 2, globaltimer_ns());
+                if (kt == 0) DAG_TRACE(16 * T + 8 * (long long)tk.t + 2, globaltimer_ns());
                 tc_fence_after();
                 const uint32_t sb = smem_u32(smem + st * STAGE_BYTES);
                 const uint32_t a_hi = sb, a_lo = sb + A_BYTES;
@@ -532,6 +535,67 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
             const DagTask tk = ctl.slot[s];
             named_bar_epi();
             if (!all || tk.type == DT_STOP) break;
+            // the task's epilogue: outputs
+            const long long n = g.n;
+            const int i0 = tk.a * NB + 32 * q;   // first tile row of this warp (global row)
+            float alpha = 1.f, beta = 0.f;
+            bool C = false;
+            long long c_rows = n, c_cols = n, c_col0 = 0;
+            const CUtensorMap* mc = nullptr;         // C load
+            const CUtensorMap* mc_store = nullptr;   // C store
+            bool s_split = false;
+            const CUtensorMap *t_hi = nullptr, *t_lo = nullptr;
+            long long t_row0 = 0;
+            long long s_col0 = 0;
+            switch (tk.type) {
+                case DT_PANEL:
+                    s_split = true;
+                    s_col0 = (long long)tk.b * NB;
+                    break;
+                case DT_UPDATE:
+                    alpha = -1.f;
+                    beta = 1.f;
+                    C = true;
+                    mc = mc_store = &maps.ca;
+                    c_col0 = (long long)tk.b * NB;
+                    s_split = (tk.b == tk.c - 1) && (tk.a < tk.b);   // the next panel's input
+                    s_col0 = c_col0;
+                    break;
+                case DT_FIN:
+                    alpha = -1.f;
+                    C = true;
+                    mc_store = &maps.u32;
+                    c_rows = g.d;
+                    c_cols = g.d;
+                    c_col0 = (long long)tk.b * NB;
+                    t_hi = &maps.ut_hi32;
+                    t_lo = &maps.ut_lo32;
+                    t_row0 = (long long)tk.b * NB;
+                    break;
+                default:   // SUPD
+                    beta = (tk.c == tk.b) ? 0.f : 1.f;
+                    C = true;
+                    mc = mc_store = &maps.cs;
+                    c_col0 = (long long)tk.b * NB;
+                    if (tk.c == tk.a + 1) {
+                        t_hi = &maps.tt_hi32;
+                        t_lo = &maps.tt_lo32;
+                        t_row0 = (long long)tk.b * NB;
+                    }
+                    break;
+            }
+            // C (beta != 0) is fetched now, while the MMAs run
+            if (beta != 0.f) {
+                fence_proxy_async_smem();   // this warp's reads of cbox (previous task) come first
+                __syncwarp();
+                if (lane == 0) {
+                    fence_proxy_async_global();   // C was written by another task (acquired by warp 0)
+                    mbar_arrive_expect_tx(&ctl.cin[q], NCHUNK * kBoxBytes);
+                    for (int c = 0; c < NCHUNK; ++c)
+                        tma_load_2d(cbox + c * kBoxBytes, mc, &ctl.cin[q], (int)(c_col0 + 32 * c), i0);
+                }
+                __syncwarp();
+            }
             bool ok = true;
             // segments before the last: add into the running sum (columns SUM_HI ..)
             for (int sg = 0; sg + 1 < nseg && ok; ++sg, ++seg) {
@@ -565,72 +629,15 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
             const uint32_t use = (uint32_t)(seg >> 1);
             ++seg;
             ok = ok && mbar_wait(&ctl.tfull[buf], use & 1, -6200000LL - blockIdx.x);
-            if (warp == 2 && lane == 0) DAG_TRACE(4 * T + 8 * (long long)tk.t + 3, globaltimer_ns());
+            if (warp == 2 && lane == 0) DAG_TRACE(16 * T + 8 * (long long)tk.t + 3, globaltimer_ns());
             tc_fence_after();
             const uint32_t acc = tmem + (uint32_t)(buf * TBN) + lane_off;
 
-            // the task's epilogue
-            const long long n = g.n;
-            const int i0 = tk.a * NB + 32 * q;   // first tile row of this warp (global row)
-            float alpha = 1.f, beta = 0.f;
-            float* C = nullptr;
-            long long ldc = n, c_rows = n, c_cols = n, c_col0 = 0;
-            const CUtensorMap* mc = nullptr;
-            bool s_split = false;
-            float *t_hi = nullptr, *t_lo = nullptr;
-            long long t_row0 = 0;
-            long long s_col0 = 0;
-            switch (tk.type) {
-                case DT_PANEL:
-                    s_split = true;
-                    s_col0 = (long long)tk.b * NB;
-                    break;
-                case DT_UPDATE:
-                    alpha = -1.f;
-                    beta = 1.f;
-                    C = g.A;
-                    mc = &maps.ca;
-                    c_col0 = (long long)tk.b * NB;
-                    s_split = (tk.b == tk.c - 1) && (tk.a < tk.b);   // the next panel's input
-                    s_col0 = c_col0;
-                    break;
-                case DT_FIN:
-                    alpha = -1.f;
-                    C = g.U;
-                    ldc = g.d;
-                    c_rows = g.d;
-                    c_cols = g.d;
-                    c_col0 = (long long)tk.b * NB;
-                    t_hi = g.UT_hi;
-                    t_lo = g.UT_lo;
-                    t_row0 = (long long)tk.b * NB;
-                    break;
-                default:   // SUPD
-                    beta = (tk.c == tk.b) ? 0.f : 1.f;
-                    C = g.S;
-                    mc = &maps.cs;
-                    c_col0 = (long long)tk.b * NB;
-                    if (tk.c == tk.a + 1) {
-                        t_hi = g.TT_hi;
-                        t_lo = g.TT_lo;
-                        t_row0 = (long long)tk.b * NB;
-                    }
-                    break;
-            }
             bool cin_ok = true;
             if (beta != 0.f) {
-                fence_proxy_async_smem();   // this warp's reads of cbox (previous task) come first
-                __syncwarp();
-                if (lane == 0) {
-                    fence_proxy_async_global();   // C was written by another task (acquired by warp 0)
-                    mbar_arrive_expect_tx(&ctl.cin[q], NCHUNK * kBoxBytes);
-                    for (int c = 0; c < NCHUNK; ++c)
-                        tma_load_2d(cbox + c * kBoxBytes, mc, &ctl.cin[q], (int)(c_col0 + 32 * c), i0);
-                }
-                __syncwarp();
                 cin_ok = mbar_wait(&ctl.cin[q], cin_use & 1, -6300000LL - blockIdx.x);
                 ++cin_use;
-                if (warp == 2 && lane == 0) DAG_TRACE(4 * T + 8 * (long long)tk.t + 7, globaltimer_ns());
+                if (warp == 2 && lane == 0) DAG_TRACE(16 * T + 8 * (long long)tk.t + 7, globaltimer_ns());
             }
 #pragma unroll 1
             for (int c = 0; c < NCHUNK; ++c) {
@@ -660,32 +667,57 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
                         out[4 * c4 + 3] += v.w;
                     }
                 }
-                const long long j0 = c_col0 + 32 * c;
-                if (C) emit_block(kb, lane, out, false, C, ldc, c_rows, c_cols, i0, j0);
+                // outputs: each 32x32 block through a swizzled box in shared memory and one TMA
+                // store; box 0 is this chunk's C box (read above), boxes 1 and 2 the staging pair
+                __syncwarp();   // every lane has read its C row before the boxes are rewritten
+                uint8_t* box[3] = {cbox + c * kBoxBytes, kb, kb + kBoxBytes};
+                const int j0 = (int)(c_col0 + 32 * c);
+                int nb = 0;
+                auto put = [&](const float (&v)[32], bool transposed, const CUtensorMap* map, int x, int y,
+                               bool in_range) {
+                    uint8_t* bx = box[nb++];
+                    if (transposed)
+                        box_put_col(bx, lane, v);
+                    else
+                        box_put_row(bx, lane, v);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && in_range) tma_store_2d(map, bx, x, y);
+                };
+                if (C) put(out, false, mc_store, j0, i0, i0 < c_rows && j0 < c_cols);
                 if (s_split || t_hi) {
                     float hi[32], lo[32];
 #pragma unroll
                     for (int u = 0; u < 32; ++u) split_tf32(out[u], hi[u], lo[u]);
                     if (s_split) {
-                        emit_block(kb, lane, hi, false, g.RS_hi, n, n, n, i0, s_col0 + 32 * c);
-                        emit_block(kb, lane, lo, false, g.RS_lo, n, n, n, i0, s_col0 + 32 * c);
+                        put(hi, false, &maps.rs_hi32, (int)(s_col0 + 32 * c), i0, true);
+                        put(lo, false, &maps.rs_lo32, (int)(s_col0 + 32 * c), i0, true);
                     }
                     if (t_hi) {
-                        emit_block(kb, lane, hi, true, t_hi, n, n, n, t_row0 + 32 * c, i0);
-                        emit_block(kb, lane, lo, true, t_lo, n, n, n, t_row0 + 32 * c, i0);
+                        put(hi, true, t_hi, i0, (int)(t_row0 + 32 * c), true);
+                        put(lo, true, t_lo, i0, (int)(t_row0 + 32 * c), true);
                     }
                 }
+                if (lane == 0) {
+                    bulk_commit();
+                    bulk_wait_read<0>();   // the boxes may be rewritten by the next chunk
+                }
+                __syncwarp();
             }
+            if (lane == 0) {
+                bulk_wait<0>();            // this warp's stores are complete
+                fence_proxy_async_global();
+            }
+            __syncwarp();
             // completion: the stores of all four warps, then the counter
-            if (warp == 2 && lane == 0) DAG_TRACE(4 * T + 8 * (long long)tk.t + 6, globaltimer_ns());
-            fence_proxy_async_global();
-            __threadfence();
+            if (warp == 2 && lane == 0) DAG_TRACE(16 * T + 8 * (long long)tk.t + 6, globaltimer_ns());
             named_bar_epi();
-            if (warp == 2 && lane == 0) {
+            if (warp == 2 && lane == 0) {   // release: the four warps' stores, then the counter
+                fence_proxy_async_global();
                 __threadfence();
                 if (ok && cin_ok) atomicAdd(dag_done_ctr(g, tk), 1);
                 else atomicExch(abort, 1);
-                DAG_TRACE(4 * T + 8 * (long long)tk.t + 4, globaltimer_ns());
+                DAG_TRACE(16 * T + 8 * (long long)tk.t + 4, globaltimer_ns());
                 mbar_arrive(&ctl.task_empty[s]);
             }
         }
@@ -784,7 +816,11 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
         !make_tmap_2d(&m.xd_lo, w.Xd_lo, 4, N, gq::NB, gq::NB, gq::BM, 32) ||
         !make_tmap_2d(&m.tt_hi, w.TT_hi, 4, N, N, N, gq::BM, 32) || !make_tmap_2d(&m.tt_lo, w.TT_lo, 4, N, N, N, gq::BM, 32) ||
         !make_tmap_2d(&m.ut_hi, w.UT_hi, 4, N, N, N, gq::BM, 32) || !make_tmap_2d(&m.ut_lo, w.UT_lo, 4, N, N, N, gq::BM, 32) ||
-        !make_tmap_2d(&m.ca, w.A, 4, N, N, N, 32, 32) || !make_tmap_2d(&m.cs, w.S, 4, N, N, N, 32, 32))
+        !make_tmap_2d(&m.ca, w.A, 4, N, N, N, 32, 32) || !make_tmap_2d(&m.cs, w.S, 4, N, N, N, 32, 32) ||
+        !make_tmap_2d(&m.rs_hi32, w.RS_hi, 4, N, N, N, 32, 32) || !make_tmap_2d(&m.rs_lo32, w.RS_lo, 4, N, N, N, 32, 32) ||
+        !make_tmap_2d(&m.ut_hi32, w.UT_hi, 4, N, N, N, 32, 32) || !make_tmap_2d(&m.ut_lo32, w.UT_lo, 4, N, N, N, 32, 32) ||
+        !make_tmap_2d(&m.tt_hi32, w.TT_hi, 4, N, N, N, 32, 32) || !make_tmap_2d(&m.tt_lo32, w.TT_lo, 4, N, N, N, 32, 32) ||
+        !make_tmap_2d(&m.u32, U, 4, (uint64_t)d, (uint64_t)d, (uint64_t)d, 32, 32))
         return cudaErrorInvalidValue;
     gq::DagArgs a{};
     a.T = T;
