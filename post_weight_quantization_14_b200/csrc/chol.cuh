@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(256) zero_lower_blocks_kernel(float* __restric
 //      X_ij = -X_ii sum_{k=j}^{i-1} L_ik X_kj (the sums as soon as their inputs exist, the
 //      products by X_ii once it is known).
 // F and W meet on named barriers (3: F's block done, 4: the next block updated); W syncs
-// on barrier 2 among its 224 threads.
+// on barrier 2 among its 224 threads, the whole leaf on barrier 5.
 constexpr int LS = NB + 4;   // leaf smem row stride (16-byte aligned rows)
 constexpr int LEAF_THREADS = 256;
 constexpr int LEAF_W = LEAF_THREADS - 32;   // threads of warps 1-7
@@ -183,6 +183,8 @@ __device__ __forceinline__ void nbar_arrive(int id, int n) {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 __device__ __forceinline__ void wsync() { nbar_sync(2, LEAF_W); }
+// All 256 threads of the leaf (the CTA may have more warps, which take no part).
+__device__ __forceinline__ void leaf_sync() { nbar_sync(5, LEAF_THREADS); }
 
 // F: factor the 32x32 diagonal block at (k0, k0); lane i holds row k0 + i.  Per pivot k the
 // dependency chain is: the pivot (one shuffle of the diagonal entry that lane k keeps current
@@ -411,7 +413,7 @@ __device__ __forceinline__ void leaf_band_mul(LeafSmem& S, int i, int wt, int nt
 }
 
 // The whole leaf on P (loaded, reversed, and visible to all 256 threads): L in P/LT and
-// X = L^-1 in S.X (lower) on return, visible to all threads.
+// X = L^-1 in S.X (lower) on return, visible to all 256 threads.
 // Optional event trace for profiling builds (GQ_DAG_TRACE defined): %globaltimer stamps,
 // 16 slots per leaf (the factorization kernel adds 8 per product task after them).
 #ifdef GQ_DAG_TRACE
@@ -461,7 +463,7 @@ __device__ __forceinline__ void leaf_factor(LeafSmem& S, int jb) {
             if (kb < 3 && warp != 4) leaf_band_sums(S, kb + 1, wo, NO);
         }
     }
-    __syncthreads();
+    leaf_sync();
 }
 
 }  // namespace gq

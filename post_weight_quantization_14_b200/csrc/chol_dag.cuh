@@ -195,27 +195,31 @@ __device__ __forceinline__ int* dag_done_ctr(const DagArgs& g, const DagTask& t)
     }
 }
 
-constexpr int DAG_THREADS = 256;
+constexpr int DAG_THREADS = 256;                 // the leaf's threads (warps 0-7)
+constexpr int DAG_BLOCK = 320;                   // product CTAs: TMA, MMA, 8 epilogue warps
+constexpr int DAG_EPI_WARPS = 8;                 // two per TMEM lane quadrant, two chunks each
+constexpr int DAG_EPI_BOXES = 3;                 // 32x32 fp32 boxes per epilogue warp: 2 C + 1 staging
 constexpr int DAG_STAGES = 2;
 constexpr int DAG_SLOTS = 4;
 constexpr int DAG_NK = NB / GemmCfg<KIND_TF32X3, 128>::KT;   // 4 TMA stages of K = 32 per task
 constexpr int DAG_SEG = 4;                                   // MMA k-steps per accumulator segment
-constexpr int DAG_GEMM_BYTES = DAG_STAGES * GemmCfg<KIND_TF32X3, 128>::STAGE_BYTES + epi_bytes<128>();
+constexpr int DAG_GEMM_BYTES =
+    DAG_STAGES * GemmCfg<KIND_TF32X3, 128>::STAGE_BYTES + DAG_EPI_WARPS * DAG_EPI_BOXES * kBoxBytes;
 
 struct DagCtl {
-    uint64_t full[DAG_STAGES], empty[DAG_STAGES], tfull[2], tempty[2], cin[4];
+    uint64_t full[DAG_STAGES], empty[DAG_STAGES], tfull[2], tempty[2], cin[DAG_EPI_WARPS];
     uint64_t task_full[DAG_SLOTS], task_empty[DAG_SLOTS];
     DagTask slot[DAG_SLOTS];
     uint32_t tmem_slot;
     int flag;
-    int epi_ok[4];
+    int epi_ok[DAG_EPI_WARPS];
 };
 constexpr int DAG_SMEM_BODY = (DAG_GEMM_BYTES > (int)sizeof(LeafSmem) ? DAG_GEMM_BYTES : (int)sizeof(LeafSmem));
 constexpr int DAG_SMEM = 1024 + DAG_SMEM_BODY + (int)sizeof(DagCtl);
 static_assert(DAG_SMEM <= 232448, "persistent factorization: shared memory per CTA");
 static_assert(NB * NB / 4 == 16 * DAG_THREADS, "leaf load and store loops");
 
-__device__ __forceinline__ void named_bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void named_bar_epi() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 struct DagMaps {
     // operands (128 x 32 boxes) and C in/out (32 x 32 boxes), all 128-byte swizzled
@@ -242,7 +246,7 @@ __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, Dag
             ctl.flag = dag_wait_ge(&a_cnt[j * T + j], T - 1 - j, abort, -(2000000LL + j)) ? 1 : 0;
             DAG_TRACE(16 * j, globaltimer_ns());
         }
-        __syncthreads();
+        leaf_sync();
         if (!ctl.flag) return;
         // P[127-r][127-c] = A[r][c]
 #pragma unroll
@@ -262,7 +266,7 @@ __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, Dag
                 S.P[127 - r][124 - cc] = v[it].w;
             }
         }
-        __syncthreads();
+        leaf_sync();
         if (tid == 0) DAG_TRACE(16 * j + 12, globaltimer_ns());
         leaf_factor(S, (int)jb);
         if (tid == 0) DAG_TRACE(16 * j + 11, globaltimer_ns());
@@ -285,7 +289,7 @@ __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, Dag
             *reinterpret_cast<float4*>(xh + r * NB + cc) = make_float4(h[0], h[1], h[2], h[3]);
             *reinterpret_cast<float4*>(xl + r * NB + cc) = make_float4(l[0], l[1], l[2], l[3]);
         }
-        __syncthreads();
+        leaf_sync();
         if (tid == 0) {   // release: the CTA's stores (ordered by the barrier), then the counter
             fence_proxy_async_global();
             __threadfence();
@@ -316,7 +320,7 @@ __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, Dag
             *reinterpret_cast<float4*>(g.UT_hi + (jb + col) * n + jb + r4) = make_float4(h[0], h[1], h[2], h[3]);
             *reinterpret_cast<float4*>(g.UT_lo + (jb + col) * n + jb + r4) = make_float4(l[0], l[1], l[2], l[3]);
         }
-        __syncthreads();
+        leaf_sync();
         if (tid == 0) {
             fence_proxy_async_global();
             __threadfence();
@@ -330,7 +334,7 @@ __device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, Dag
 // Product CTAs.
 // ---------------------------------------------------------------------------------------
 
-__global__ void __launch_bounds__(DAG_THREADS, 1)
+__global__ void __launch_bounds__(DAG_BLOCK, 1)
     chol_dag_kernel(const __grid_constant__ DagMaps maps, const DagArgs g) {
     extern __shared__ uint8_t dag_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dag_raw) + 1023) & ~uintptr_t(1023));
@@ -341,8 +345,9 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
 
     if (threadIdx.x == 0) ctl.flag = atomicAdd(g.ctr + 1, 1);
     __syncthreads();
-    if (ctl.flag == 0) {   // the first CTA to start runs the leaves
-        __syncthreads();
+    if (ctl.flag == 0) {   // the first CTA to start runs the leaves, on warps 0-7
+        if (warp >= DAG_THREADS / 32) return;
+        leaf_sync();
         dag_leaf_role(g, *reinterpret_cast<LeafSmem*>(smem), ctl);
         return;
     }
@@ -352,7 +357,6 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
     constexpr int A_BYTES = BM * 128, B_BYTES = TBN * 128;
     constexpr int SUM_HI = 2 * TBN, XOFF = 3 * TBN;
     constexpr uint32_t TMEM_COLS = 512;
-    constexpr int NCHUNK = TBN / 32;
     uint8_t* epi = smem + DAG_STAGES * STAGE_BYTES;
 
     if (threadIdx.x == 0) {
@@ -362,9 +366,9 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl.tfull[b], 1);
-            mbar_init(&ctl.tempty[b], 4);
+            mbar_init(&ctl.tempty[b], DAG_EPI_WARPS);
         }
-        for (int q = 0; q < 4; ++q) mbar_init(&ctl.cin[q], 1);
+        for (int q = 0; q < DAG_EPI_WARPS; ++q) mbar_init(&ctl.cin[q], 1);
         for (int s = 0; s < DAG_SLOTS; ++s) {
             mbar_init(&ctl.task_full[s], 1);
             mbar_init(&ctl.task_empty[s], 1);
@@ -514,12 +518,13 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
             umma_commit(&ctl.tfull[seg & 1]);
             ++seg;
         }
-    } else if (warp >= 2 && warp < 6) {
-        // ---------------- epilogue: warp q owns accumulator rows 32q .. 32q+31
-        const int q = warp & 3;
-        uint8_t* wreg = epi + q * epi_boxes_per_warp<TBN>() * kBoxBytes;
-        uint8_t* cbox = wreg;
-        uint8_t* kb = wreg + NCHUNK * kBoxBytes;
+    } else if (warp >= 2) {
+        // ---------------- epilogue: warp w (2..9) owns accumulator rows 32q .. 32q+31, q = w % 4,
+        // and the chunks (32 columns each) 2h, 2h+1 of them, h = (w - 2) / 4
+        const int q = warp & 3, ew = warp - 2, h = ew >> 2;
+        uint8_t* wreg = epi + ew * DAG_EPI_BOXES * kBoxBytes;
+        uint8_t* cbox = wreg;                      // this warp's two C chunks
+        uint8_t* kb = wreg + 2 * kBoxBytes;        // staging box
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         constexpr int nseg = DAG_NK * 4 / DAG_SEG;
         int seg = 0;
@@ -529,9 +534,11 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
             // the four warps agree on whether a task came (each wait is bounded), so none of
             // them can be left alone at the task's named barriers
             const bool got = mbar_wait(&ctl.task_full[s], (uint32_t)(nt / DAG_SLOTS) & 1, -6000000LL - blockIdx.x);
-            if (lane == 0) ctl.epi_ok[q] = got ? 1 : 0;
+            if (lane == 0) ctl.epi_ok[ew] = got ? 1 : 0;
             named_bar_epi();
-            const bool all = ctl.epi_ok[0] && ctl.epi_ok[1] && ctl.epi_ok[2] && ctl.epi_ok[3];
+            bool all = true;
+#pragma unroll
+            for (int e = 0; e < DAG_EPI_WARPS; ++e) all = all && ctl.epi_ok[e];
             const DagTask tk = ctl.slot[s];
             named_bar_epi();
             if (!all || tk.type == DT_STOP) break;
@@ -590,9 +597,9 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
                 __syncwarp();
                 if (lane == 0) {
                     fence_proxy_async_global();   // C was written by another task (acquired by warp 0)
-                    mbar_arrive_expect_tx(&ctl.cin[q], NCHUNK * kBoxBytes);
-                    for (int c = 0; c < NCHUNK; ++c)
-                        tma_load_2d(cbox + c * kBoxBytes, mc, &ctl.cin[q], (int)(c_col0 + 32 * c), i0);
+                    mbar_arrive_expect_tx(&ctl.cin[ew], 2 * kBoxBytes);
+                    for (int cl = 0; cl < 2; ++cl)
+                        tma_load_2d(cbox + cl * kBoxBytes, mc, &ctl.cin[ew], (int)(c_col0 + 32 * (2 * h + cl)), i0);
                 }
                 __syncwarp();
             }
@@ -603,7 +610,7 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
                 ok = mbar_wait(&ctl.tfull[sb], (uint32_t)(seg >> 1) & 1, -6100000LL - blockIdx.x);
                 tc_fence_after();
 #pragma unroll 1
-                for (int c = 0; c < NCHUNK; ++c) {
+                for (int c = 2 * h; c < 2 * h + 2; ++c) {
                     const uint32_t src = tmem + (uint32_t)(sb * TBN + c * 32) + lane_off;
                     const uint32_t dhi = tmem + (uint32_t)(SUM_HI + c * 32) + lane_off;
                     uint32_t r[32];
@@ -635,12 +642,13 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
 
             bool cin_ok = true;
             if (beta != 0.f) {
-                cin_ok = mbar_wait(&ctl.cin[q], cin_use & 1, -6300000LL - blockIdx.x);
+                cin_ok = mbar_wait(&ctl.cin[ew], cin_use & 1, -6300000LL - blockIdx.x);
                 ++cin_use;
                 if (warp == 2 && lane == 0) DAG_TRACE(16 * T + 8 * (long long)tk.t + 7, globaltimer_ns());
             }
 #pragma unroll 1
-            for (int c = 0; c < NCHUNK; ++c) {
+            for (int cl = 0; cl < 2; ++cl) {
+                const int c = 2 * h + cl;   // chunk: columns 32c .. 32c+31 of the tile
                 uint32_t r[32];
                 if (ok) {
                     fetch_chunk<TBN, true, false>(tmem, acc, lane_off, c, true, r);
@@ -648,7 +656,7 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
 #pragma unroll
                     for (int u = 0; u < 32; ++u) r[u] = 0u;
                 }
-                if (c == NCHUNK - 1) {
+                if (cl == 1) {   // this warp has read its part of the accumulator
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&ctl.tempty[buf]);
@@ -657,7 +665,7 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
 #pragma unroll
                 for (int u = 0; u < 32; ++u) out[u] = alpha * __uint_as_float(r[u]);
                 if (beta != 0.f && cin_ok) {
-                    const uint8_t* cb = cbox + c * kBoxBytes;
+                    const uint8_t* cb = cbox + cl * kBoxBytes;
 #pragma unroll
                     for (int c4 = 0; c4 < 8; ++c4) {
                         const float4 v = *reinterpret_cast<const float4*>(cb + lane * 128 + ((c4 ^ (lane & 7)) << 4));
@@ -668,13 +676,24 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
                     }
                 }
                 // outputs: each 32x32 block through a swizzled box in shared memory and one TMA
-                // store; box 0 is this chunk's C box (read above), boxes 1 and 2 the staging pair
+                // store.  Boxes: this chunk's C box (read above), the staging box, and for the
+                // second chunk also the first chunk's C box; a box is rewritten only after the
+                // TMA has read it.
                 __syncwarp();   // every lane has read its C row before the boxes are rewritten
-                uint8_t* box[3] = {cbox + c * kBoxBytes, kb, kb + kBoxBytes};
+                uint8_t* box[3] = {cbox + cl * kBoxBytes, kb, cbox};
+                const int nbox = cl == 0 ? 2 : 3;
                 const int j0 = (int)(c_col0 + 32 * c);
                 int nb = 0;
                 auto put = [&](const float (&v)[32], bool transposed, const CUtensorMap* map, int x, int y,
                                bool in_range) {
+                    if (nb == nbox) {   // out of boxes: wait until the TMA has read them
+                        if (lane == 0) {
+                            bulk_commit();
+                            bulk_wait_read<0>();
+                        }
+                        __syncwarp();
+                        nb = 0;
+                    }
                     uint8_t* bx = box[nb++];
                     if (transposed)
                         box_put_col(bx, lane, v);
@@ -700,7 +719,7 @@ __global__ void __launch_bounds__(DAG_THREADS, 1)
                 }
                 if (lane == 0) {
                     bulk_commit();
-                    bulk_wait_read<0>();   // the boxes may be rewritten by the next chunk
+                    if (cl == 0) bulk_wait_read<0>();   // the boxes are rewritten by the second chunk
                 }
                 __syncwarp();
             }
@@ -843,7 +862,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
     const unsigned grid = T == 1 ? 1u : (unsigned)std::min<long long>(num_sms(), 1 + gq::dag_total_tasks(T));
     {
         gqh::TimedScope ts__("chol_dag", st);
-        GQ_TRY(launch_plain(gq::chol_dag_kernel, dim3(grid), dim3(gq::DAG_THREADS), (size_t)gq::DAG_SMEM, st, m,
+        GQ_TRY(launch_plain(gq::chol_dag_kernel, dim3(grid), dim3(gq::DAG_BLOCK), (size_t)gq::DAG_SMEM, st, m,
                             (const gq::DagArgs)a));
     }
     return cudaGetLastError();

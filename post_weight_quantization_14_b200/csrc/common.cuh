@@ -252,11 +252,14 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_format, int M, int
            ((uint32_t)(M >> 4) << 24);
 }
 
-// tf32 split: x = hi + lo with hi = tf32(x) (round to nearest) and lo = tf32(x - hi).
+// tf32 split: x = hi + lo with hi = tf32(x) (round to nearest, ties away from zero) and
+// lo = tf32(x - hi).  The rounding works on the bit pattern: adding half a unit of the 13
+// dropped mantissa bits to the sign-magnitude encoding and clearing them rounds the
+// magnitude (carries move into the exponent as they should); two integer operations at the
+// full ALU rate.  Infinities stay infinite; a NaN may lose its payload in hi, but lo = x - hi
+// is then NaN, so the pair still carries it.
 __device__ __forceinline__ float to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
 __device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
     hi = to_tf32(x);
