@@ -123,7 +123,9 @@ gptq_status gptq_hessian_accumulate(const void* X, gptq_dtype xt, int64_t n, int
  *   bad_col  host pointer or NULL; on GPTQ_ERR_NOT_PD receives the first failing column.
  *   lambda_out  host pointer or NULL; receives lambda.
  * Computed as Hd = R R^T with R upper (Cholesky from the bottom-right), then U = R^-1,
- * blocked by 128 with fp32 diagonal blocks and 3xTF32 tensor-core block updates.
+ * blocked by 128: fp32 diagonal blocks, every off-diagonal block product a 3xTF32
+ * tensor-core tile, all in one persistent launch that takes the tiles in the dependency
+ * order gptq_chol_schedule returns (one CTA per SM; waits between tiles are bounded).
  * Synchronises ``stream`` once to report NOT_PD / NONFINITE.  Returns
  * GPTQ_ERR_INVALID_ARG when mean(diag H) <= 0.  Requires d_in % 8 == 0. */
 size_t gptq_prepare_hinv_workspace_bytes(int64_t d_in);
