@@ -305,10 +305,12 @@ size_t gptq_timing_timeline(char* buf, size_t len);
  *   type 1  UPDATE(j = c, i = a, k = b): A_ik -= R_ij R_kj^T
  *   type 2  FIN(i = a, m = b):       U_im = -R_ii^-1 S_im
  *   type 3  SUPD(i = a, k = c, m = b):  S_im += R_ik U_km
+ *   type 4  DIAG(j = a):             U_jj = R_jj^-1 to U and to the split of U^T (a copy)
  * with Hd = R R^T (R upper), U = R^-1.  The diagonal blocks (R_jj and R_jj^-1 from A_jj) are
- * formed in the order j = T-1 .. 0 by one CTA, LEAF(j) needing the updates of A_jj.  Every
- * product's inputs come from products earlier in the list or from a leaf before its step;
- * returns -1 for T < 1. */
+ * formed in the order j = T-1 .. 0 by one CTA, which also forms, right after LEAF(j), the two
+ * products the next leaf needs: PANEL(j, j-1) and UPDATE(j, j-1, j-1) (not in the list).
+ * Every product's inputs come from products earlier in the list or from a leaf step before
+ * its own step; returns -1 for T < 1. */
 int64_t gptq_chol_schedule(int64_t T, int32_t* tasks, int64_t max_tasks);
 gptq_status gptq_selftest_bounded_wait(uint64_t limit_ns, void* stream);
 

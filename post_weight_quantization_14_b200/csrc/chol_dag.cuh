@@ -27,7 +27,7 @@
 
 namespace gq {
 
-enum : int { DT_PANEL = 0, DT_UPDATE = 1, DT_FIN = 2, DT_SUPD = 3, DT_STOP = 15 };
+enum : int { DT_PANEL = 0, DT_UPDATE = 1, DT_FIN = 2, DT_SUPD = 3, DT_DIAG = 4, DT_STOP = 15 };
 
 // Optional event trace for profiling builds (GQ_DAG_TRACE defined): %globaltimer stamps of
 // each leaf (16 per leaf) and each ticket (8 per ticket, after 16 T leaf slots): fetched,
@@ -45,15 +45,18 @@ enum : int { DT_PANEL = 0, DT_UPDATE = 1, DT_FIN = 2, DT_SUPD = 3, DT_STOP = 15 
 
 // PANEL(j, i): a = i, b = j.  UPDATE(j, i, k): a = i, b = k, c = j.
 // FIN(i, m): a = i, b = m.    SUPD(i, k, m): a = i, b = m, c = k.
+// DIAG(j): a = j -- U_jj to the public U and to the U^T split (a copy of X_jj's split).
 struct DagTask {
     int type, a, b, c;
     int t;   // ticket (set by the fetching CTA)
 };
 
+// Products of step j handed out by ticket.  PANEL(j, j-1) and UPDATE(j, j-1, j-1), the two
+// tiles the next leaf needs, are not among them: the leaf CTA forms them itself right after
+// LEAF(j) (dag_leaf_role).
 __host__ __device__ inline long long dag_step_tasks(int T, int j) {
     const long long jj = j;
-    long long c = (T - 1 - jj) + jj * (T - jj);
-    if (j >= 1) c += 2;
+    long long c = 1 + (T - 1 - jj) + jj * (T - jj);
     if (j >= 2) c += 2 * (jj - 1) + (jj - 1) * jj / 2;
     return c;
 }
@@ -66,11 +69,8 @@ __host__ __device__ inline long long dag_total_tasks(int T) {
 
 // Task idx of step j.
 __host__ __device__ inline DagTask dag_step_task(int T, int j, long long idx) {
-    if (j >= 1) {
-        if (idx == 0) return DagTask{DT_PANEL, j - 1, j, 0, 0};
-        if (idx == 1) return DagTask{DT_UPDATE, j - 1, j - 1, j, 0};
-        idx -= 2;
-    }
+    if (idx == 0) return DagTask{DT_DIAG, j, 0, 0, 0};
+    idx -= 1;
     if (j >= 2) {
         if (idx < j - 1) return DagTask{DT_PANEL, j - 2 - (int)idx, j, 0, 0};
         idx -= j - 1;
@@ -172,6 +172,8 @@ __device__ __forceinline__ bool dag_deps(const DagArgs& g, const DagTask& t) {
         case DT_FIN:
             return dag_wait_ge(&leaf_done[t.a], 1, abort, where) &&
                    dag_wait_ge(&s_cnt[t.a * T + t.b], t.b - t.a, abort, where);
+        case DT_DIAG:
+            return dag_wait_ge(&leaf_done[t.a], 1, abort, where);
         case DT_SUPD:
             return dag_wait_ge(&rs_done[t.a * T + t.c], 1, abort, where) &&
                    dag_wait_ge(t.c == t.b ? &diag_done[t.b] : &u_done[t.c * T + t.b], 1, abort, where) &&
@@ -187,7 +189,9 @@ __device__ __forceinline__ int* dag_done_ctr(const DagArgs& g, const DagTask& t)
     int* rs_done = a_cnt + T * T;
     int* s_cnt = rs_done + T * T;
     int* u_done = s_cnt + T * T;
+    int* diag_done = u_done + T * T + T;
     switch (t.type) {
+        case DT_DIAG: return &diag_done[t.a];
         case DT_PANEL: return &rs_done[t.a * T + t.b];
         case DT_UPDATE: return &a_cnt[t.a * T + t.b];
         case DT_FIN: return &u_done[t.a * T + t.b];
@@ -229,104 +233,340 @@ struct DagMaps {
 };
 
 // ---------------------------------------------------------------------------------------
-// The leaf CTA: LEAF(j) for j = T-1 .. 0 (256 threads; the pieces are chol.cuh's).
+// The leaf CTA.  Warps 0-7 (256 threads) form LEAF(j) for j = T-1 .. 0 and, after each leaf
+// j >= 1, the two products the next leaf needs, on this CTA's own tensor cores:
+//   PANEL(j, j-1):       R_ij = A_ij X_jj^T        (i = j-1; X_jj taken from shared memory)
+//   UPDATE(j, j-1, j-1): A_ii - R_ij R_ij^T        (written straight into the next leaf's P)
+// R_ij also goes to R's split in global memory (TMA stores) for the other products; U_jj
+// goes to the public U and the U^T split by a product task (DIAG(j)).  Warps 8-9 idle.
+// Tensor memory (512 columns): three hi*hi segments of 6, 5 and 5 k-steps and the cross
+// products apart, summed in fp32 when read; each mbarrier completes once per chain step, so
+// its phase parity is the step count.
 // ---------------------------------------------------------------------------------------
-__device__ __forceinline__ void dag_leaf_role(const DagArgs& g, LeafSmem& S, DagCtl& ctl) {
+__device__ __forceinline__ int chain_seg(int kk) { return kk < 6 ? 0 : (kk < 11 ? 1 : 2); }
+__device__ __forceinline__ bool chain_seg_first(int kk) { return kk == 0 || kk == 6 || kk == 11; }
+
+// One product's 16 k-steps of 3xTF32 MMAs (A rows x K, B rows x K, both K-major, 128-byte
+// swizzled; K-slice s of 32 at a_hi(s) / a_lo(s) = a_hi(s) + 16 KB and likewise for B).
+template <typename FA, typename FB>
+__device__ __forceinline__ void chain_mma_slices(uint32_t tmem, int s0, int s1, FA a_hi, FB b_hi) {
+    constexpr uint32_t idesc = make_idesc(2u, BM, 128);
+    for (int s = s0; s < s1; ++s) {
+        const uint32_t ah = a_hi(s), al = ah + 16384, bh = b_hi(s), bl = bh + 16384;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const int kg = 4 * s + kk;
+            const uint32_t off = kk * 32;
+            const uint32_t acc = tmem + (uint32_t)(128 * chain_seg(kg));
+            umma_tf32(acc, desc_sw128_kmajor(ah + off), desc_sw128_kmajor(bh + off), idesc,
+                      chain_seg_first(kg) ? 0u : 1u);
+            umma_tf32(tmem + 384u, desc_sw128_kmajor(ah + off), desc_sw128_kmajor(bl + off), idesc, kg > 0 ? 1u : 0u);
+            umma_tf32(tmem + 384u, desc_sw128_kmajor(al + off), desc_sw128_kmajor(bh + off), idesc, 1u);
+        }
+    }
+}
+
+// Chunk c (32 columns) of a chain product for this warp's 32 rows: ((s0 + s1) + s2) + x.
+__device__ __forceinline__ void chain_fetch(uint32_t tmem, uint32_t lane_off, int c, float (&v)[32]) {
+    uint32_t a[32], b[32];
+    tmem_ld_32x32b_x32(tmem + (uint32_t)(c * 32) + lane_off, a);
+    tmem_ld_32x32b_x32(tmem + (uint32_t)(128 + c * 32) + lane_off, b);
+    tmem_ld_wait();
+#pragma unroll
+    for (int u = 0; u < 32; ++u) v[u] = __uint_as_float(a[u]) + __uint_as_float(b[u]);
+    tmem_ld_32x32b_x32(tmem + (uint32_t)(256 + c * 32) + lane_off, a);
+    tmem_ld_32x32b_x32(tmem + (uint32_t)(384 + c * 32) + lane_off, b);
+    tmem_ld_wait();
+#pragma unroll
+    for (int u = 0; u < 32; ++u) v[u] = (v[u] + __uint_as_float(a[u])) + __uint_as_float(b[u]);
+}
+
+__device__ __forceinline__ void dag_leaf_role(const DagMaps& maps, const DagArgs& g, LeafSmem& S, DagCtl& ctl) {
     const int T = g.T;
-    const long long n = g.n, d = g.d;
-    const int tid = threadIdx.x;
+    const long long n = g.n;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int* c = g.ctr;
     int* abort = c + 2;
     int* a_cnt = c + 4;
+    int* rs_done = a_cnt + T * T;
     int* leaf_done = a_cnt + 4 * T * T;
-    int* diag_done = leaf_done + T;
-    for (int j = T - 1; j >= 0; --j) {
-        const long long jb = (long long)j * NB;
-        if (tid == 0) {
-            ctl.flag = dag_wait_ge(&a_cnt[j * T + j], T - 1 - j, abort, -(2000000LL + j)) ? 1 : 0;
-            DAG_TRACE(16 * j, globaltimer_ns());
-        }
-        leaf_sync();
-        if (!ctl.flag) return;
-        // P[127-r][127-c] = A[r][c]
-#pragma unroll
-        for (int quarter = 0; quarter < 4; ++quarter) {
-            float4 v[4];
-#pragma unroll
-            for (int it = 0; it < 4; ++it) {
-                const int e = tid + (4 * quarter + it) * DAG_THREADS, r = e >> 5, cc = (e & 31) * 4;
-                v[it] = __ldcg(reinterpret_cast<const float4*>(g.A + (jb + r) * n + jb + cc));
-            }
-#pragma unroll
-            for (int it = 0; it < 4; ++it) {
-                const int e = tid + (4 * quarter + it) * DAG_THREADS, r = e >> 5, cc = (e & 31) * 4;
-                S.P[127 - r][127 - cc] = v[it].x;
-                S.P[127 - r][126 - cc] = v[it].y;
-                S.P[127 - r][125 - cc] = v[it].z;
-                S.P[127 - r][124 - cc] = v[it].w;
-            }
-        }
-        leaf_sync();
-        if (tid == 0) DAG_TRACE(16 * j + 12, globaltimer_ns());
-        leaf_factor(S, (int)jb);
-        if (tid == 0) DAG_TRACE(16 * j + 11, globaltimer_ns());
+    uint8_t* buf0 = reinterpret_cast<uint8_t*>(&S.P[0][0]);    // chain operand slices 0, 1
+    uint8_t* buf1 = reinterpret_cast<uint8_t*>(&S.LT[0][0]);   // chain operand slices 2, 3
+    uint8_t* cbuf = reinterpret_cast<uint8_t*>(&S.X[0][0]);    // A_ii, 16 boxes of 32 x 32
+    // barriers, one completion per chain step each: A slices 0-3 landed (full[0], full[1],
+    // empty[0], empty[1]), slices 0-1 consumed (tempty[0]), panel done (tfull[0]), update
+    // done (tfull[1]), A_ii landed (cin[0])
+    uint64_t* bar_a[4] = {&ctl.full[0], &ctl.full[1], &ctl.empty[0], &ctl.empty[1]};
+    if (tid == 0) {
+        for (int q = 0; q < 4; ++q) mbar_init(bar_a[q], 1);
+        mbar_init(&ctl.tempty[0], 1);
+        mbar_init(&ctl.tfull[0], 1);
+        mbar_init(&ctl.tfull[1], 1);
+        mbar_init(&ctl.cin[0], 1);
+        fence_mbar_init();
+        ctl.flag = 1;
+    }
+    if (warp == 0) {
+        __syncwarp();
+        tmem_alloc(&ctl.tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl.tmem_slot;
 
-        // X_jj (block of U = J X J, upper) as its tf32 split, row-major: the operand of the
-        // panels of step j and of row j of U
-        float* xh = g.Xd_hi + (long long)j * NB * NB;
-        float* xl = g.Xd_lo + (long long)j * NB * NB;
-#pragma unroll 4
-        for (int it = 0; it < 16; ++it) {
-            const int task = tid + it * DAG_THREADS, r = task >> 5, cc = (task & 31) * 4;
-            const float4 xv = ld4(&S.X[127 - r][124 - cc]);
-            float v[4] = {xv.w, xv.z, xv.y, xv.x};
+    if (warp < DAG_THREADS / 32) {   // warps 8-9 take no part
+        // ---- warps 0-7: the leaves and the chain products
+        const int q = warp & 3, h = warp >> 2;              // TMEM lane quadrant, chunk half
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        bool have_tile = false;   // P already holds the next leaf's tile (from the chain step)
+        for (int j = T - 1; j >= 0; --j) {
+            const long long jb = (long long)j * NB;
+            const uint32_t par = (uint32_t)((T - 1 - j) & 1);   // chain step count parity
+            // ctl.flag is written by thread 0 only between barriers; every branch that holds a
+            // barrier takes its condition from a value all threads read after the same barrier
+            const bool need_load = ctl.flag && !have_tile;
+            leaf_sync();
+            if (need_load) {
+                if (tid == 0) {
+                    if (!dag_wait_ge(&a_cnt[j * T + j], T - 1 - j, abort, -(2000000LL + j))) ctl.flag = 0;
+                    DAG_TRACE(16 * j, globaltimer_ns());
+                }
+                leaf_sync();
+                if (ctl.flag) {   // P[127-r][127-c] = A[r][c]
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                if (r > cc + q) v[q] = 0.f;
-            float h[4], l[4];
+                    for (int quarter = 0; quarter < 4; ++quarter) {
+                        float4 v[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) split_tf32(v[q], h[q], l[q]);
-            *reinterpret_cast<float4*>(xh + r * NB + cc) = make_float4(h[0], h[1], h[2], h[3]);
-            *reinterpret_cast<float4*>(xl + r * NB + cc) = make_float4(l[0], l[1], l[2], l[3]);
-        }
-        leaf_sync();
-        if (tid == 0) {   // release: the CTA's stores (ordered by the barrier), then the counter
-            fence_proxy_async_global();
-            __threadfence();
-            atomicAdd(&leaf_done[j], 1);
-            DAG_TRACE(16 * j + 1, globaltimer_ns());
-        }
-        // U_jj to the public output (clipped to d; d % 4 == 0) and its transposed split
-#pragma unroll 4
-        for (int it = 0; it < 16; ++it) {
-            const int task = tid + it * DAG_THREADS, r = task >> 5, cc = (task & 31) * 4;
-            if (jb + r < d && jb + cc < d) {
-                const float4 xv = ld4(&S.X[127 - r][124 - cc]);
-                float v[4] = {xv.w, xv.z, xv.y, xv.x};
+                        for (int it = 0; it < 4; ++it) {
+                            const int e = tid + (4 * quarter + it) * DAG_THREADS, r = e >> 5, cc = (e & 31) * 4;
+                            v[it] = __ldcg(reinterpret_cast<const float4*>(g.A + (jb + r) * n + jb + cc));
+                        }
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    if (r > cc + q) v[q] = 0.f;
-                *reinterpret_cast<float4*>(g.U + (jb + r) * d + jb + cc) = make_float4(v[0], v[1], v[2], v[3]);
+                        for (int it = 0; it < 4; ++it) {
+                            const int e = tid + (4 * quarter + it) * DAG_THREADS, r = e >> 5, cc = (e & 31) * 4;
+                            S.P[127 - r][127 - cc] = v[it].x;
+                            S.P[127 - r][126 - cc] = v[it].y;
+                            S.P[127 - r][125 - cc] = v[it].z;
+                            S.P[127 - r][124 - cc] = v[it].w;
+                        }
+                    }
+                }
+                leaf_sync();
+            } else if (tid == 0) {
+                DAG_TRACE(16 * j, globaltimer_ns());
             }
-            // UT row cc' = r (column r of U_jj), columns 4 (task & 31) .. +3 (rows of U_jj)
-            const int col = r, r4 = cc;
-            float h[4], l[4];
+            const bool alive = ctl.flag != 0;
+            if (alive) {
+                if (tid == 0) DAG_TRACE(16 * j + 12, globaltimer_ns());
+                leaf_factor(S, (int)jb);
+                // X_jj (block of U = J X J, upper) as its tf32 split, row-major: the operand of
+                // the other panels of step j and of row j of U
+                float* xh = g.Xd_hi + (long long)j * NB * NB;
+                float* xl = g.Xd_lo + (long long)j * NB * NB;
+#pragma unroll 4
+                for (int it = 0; it < 16; ++it) {
+                    const int task = tid + it * DAG_THREADS, r = task >> 5, cc = (task & 31) * 4;
+                    const float4 xv = ld4(&S.X[127 - r][124 - cc]);
+                    float v[4] = {xv.w, xv.z, xv.y, xv.x};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int rr = r4 + q;   // U_jj[rr][col] = X[127-rr][127-col]
-                const float v = (rr <= col) ? S.X[127 - rr][127 - col] : 0.f;
-                split_tf32(v, h[q], l[q]);
+                    for (int e = 0; e < 4; ++e)
+                        if (r > cc + e) v[e] = 0.f;
+                    float hh[4], ll[4];   // lo unrounded: hi + lo restores X_jj exactly
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        hh[e] = to_tf32(v[e]);
+                        ll[e] = v[e] - hh[e];
+                    }
+                    *reinterpret_cast<float4*>(xh + r * NB + cc) = make_float4(hh[0], hh[1], hh[2], hh[3]);
+                    *reinterpret_cast<float4*>(xl + r * NB + cc) = make_float4(ll[0], ll[1], ll[2], ll[3]);
+                }
+                leaf_sync();
+                if (tid == 0) {   // release: the stores (ordered by the barrier), then the counter
+                    fence_proxy_async_global();
+                    __threadfence();
+                    atomicAdd(&leaf_done[j], 1);
+                    DAG_TRACE(16 * j + 1, globaltimer_ns());
+                }
             }
-            *reinterpret_cast<float4*>(g.UT_hi + (jb + col) * n + jb + r4) = make_float4(h[0], h[1], h[2], h[3]);
-            *reinterpret_cast<float4*>(g.UT_lo + (jb + col) * n + jb + r4) = make_float4(l[0], l[1], l[2], l[3]);
+            have_tile = false;
+            if (!alive || j == 0) continue;
+
+            // ---------------- the chain products of step j (i = j - 1)
+            const int i = j - 1;
+            const int ib = i * NB;
+            // operand slice s (K = 32 s .. 32 s + 31): slices 0, 1 in buf0 / buf1, then 2, 3
+            // again; [A hi | A lo | B hi | B lo], 16 KB each
+            auto slice_buf = [&](int s) { return (s & 1) ? buf1 : buf0; };
+            // B slices of the panel: X_jj rows n, columns 32 s .. (U_jj[n][k] = S.X[127-n][127-k])
+            auto put_x_slices = [&](int s0) {
+                for (int sl = s0; sl < s0 + 2; ++sl) {
+                    uint8_t* bh = slice_buf(sl) + 32768;
+                    const int nrow = tid >> 1, c4b = (tid & 1) * 4;
+#pragma unroll
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const int c4 = c4b + e4, k = 32 * sl + 4 * c4;
+                        const float4 xv = ld4(&S.X[127 - nrow][124 - k]);
+                        float v[4] = {xv.w, xv.z, xv.y, xv.x};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            if (nrow > k + e) v[e] = 0.f;
+                        float hh[4], ll[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            hh[e] = to_tf32(v[e]);
+                            ll[e] = v[e] - hh[e];
+                        }
+                        const uint32_t off = (uint32_t)(nrow * 128 + ((c4 ^ (nrow & 7)) << 4));
+                        *reinterpret_cast<float4*>(bh + off) = make_float4(hh[0], hh[1], hh[2], hh[3]);
+                        *reinterpret_cast<float4*>(bh + 16384 + off) = make_float4(ll[0], ll[1], ll[2], ll[3]);
+                    }
+                }
+            };
+            auto load_a_slices = [&](int s0) {   // tid 0: A_ij's split, slices s0, s0 + 1
+                for (int sl = s0; sl < s0 + 2; ++sl) {
+                    uint8_t* ab = slice_buf(sl);
+                    mbar_arrive_expect_tx(bar_a[sl], 32768);
+                    tma_load_2d(ab, &maps.rs_hi, bar_a[sl], (int)jb + 32 * sl, ib);
+                    tma_load_2d(ab + 16384, &maps.rs_lo, bar_a[sl], (int)jb + 32 * sl, ib);
+                }
+            };
+            bool ok = true;
+            if (tid == 0) {
+                ok = dag_wait_ge(&a_cnt[i * T + j], T - 1 - j, abort, -(2200000LL + j));
+                if (ok) {
+                    fence_proxy_async_global();
+                    load_a_slices(0);
+                } else {
+                    ctl.flag = 0;
+                }
+            }
+            put_x_slices(0);
+            fence_proxy_async_smem();
+            leaf_sync();
+            if (tid == 0) DAG_TRACE(16 * j + 3, globaltimer_ns());
+            auto panel_a = [&](int s) { return smem_u32(slice_buf(s)); };
+            auto panel_b = [&](int s) { return smem_u32(slice_buf(s)) + 32768u; };
+            if (tid == 0 && ok) {
+                for (int sl = 0; sl < 2 && ok; ++sl) {
+                    ok = mbar_wait(bar_a[sl], par, -(2300000LL + j));
+                    tc_fence_after();
+                    if (ok) chain_mma_slices(tmem, sl, sl + 1, panel_a, panel_b);
+                }
+                umma_commit(&ctl.tempty[0]);
+                ok = ok && mbar_wait(&ctl.tempty[0], par, -(2400000LL + j));   // slices 0-1 consumed
+                if (ok) load_a_slices(2);
+                if (!ok) ctl.flag = 0;
+            }
+            leaf_sync();
+            if (tid == 0) DAG_TRACE(16 * j + 4, globaltimer_ns());
+            if (ctl.flag) put_x_slices(2);
+            fence_proxy_async_smem();
+            leaf_sync();
+            if (tid == 0 && ctl.flag) {
+                for (int sl = 2; sl < 4 && ok; ++sl) {
+                    ok = mbar_wait(bar_a[sl], par, -(2300000LL + j));
+                    tc_fence_after();
+                    if (ok) chain_mma_slices(tmem, sl, sl + 1, panel_a, panel_b);
+                }
+                umma_commit(&ctl.tfull[0]);
+                if (!ok) ctl.flag = 0;
+            }
+            // A_ii (its other updates done) into S.X's space (X_jj is no longer read)
+            if (tid == 0 && ctl.flag) {
+                if (dag_wait_ge(&a_cnt[i * T + i], T - 1 - j, abort, -(2500000LL + j))) {
+                    fence_proxy_async_global();
+                    mbar_arrive_expect_tx(&ctl.cin[0], NB * NB * 4);
+                    for (int b = 0; b < 16; ++b)
+                        tma_load_2d(cbuf + b * 4096, &maps.ca, &ctl.cin[0], ib + 32 * (b & 3), ib + 32 * (b >> 2));
+                } else {
+                    ctl.flag = 0;
+                }
+            }
+            // R_ij: from tensor memory to the update's operand slices (both A and B) and, by
+            // TMA, to R's split in global memory; warp (q, h) takes rows 32q.., chunks 2h, 2h+1
+            bool wok = mbar_wait(&ctl.tfull[0], par, -(2600000LL + j));
+            tc_fence_after();
+            if (tid == 0) DAG_TRACE(16 * j + 5, globaltimer_ns());
+            if (wok) {
+                for (int cl = 0; cl < 2; ++cl) {
+                    const int cc = 2 * h + cl;
+                    float v[32];
+                    chain_fetch(tmem, lane_off, cc, v);
+                    float hh[32], ll[32];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) split_tf32(v[u], hh[u], ll[u]);
+                    uint8_t* sh = ((cc >> 1) ? buf1 : buf0) + (cc & 1) * 32768 + q * 4096;   // rows 32q.. of slice cc
+                    box_put_row(sh, lane, hh);
+                    box_put_row(sh + 16384, lane, ll);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&maps.rs_hi32, sh, (int)jb + 32 * cc, ib + 32 * q);
+                        tma_store_2d(&maps.rs_lo32, sh + 16384, (int)jb + 32 * cc, ib + 32 * q);
+                        bulk_commit();
+                    }
+                }
+            } else if (lane == 0) {
+                ctl.flag = 0;
+            }
+            tc_fence_before();
+            leaf_sync();
+            if (tid == 0 && ctl.flag) {   // the update: A = B = R_ij's slices (cc: buffer cc >> 1, half cc & 1)
+                DAG_TRACE(16 * j + 6, globaltimer_ns());
+                tc_fence_after();
+                auto upd = [&](int cc) { return smem_u32((cc >> 1) ? buf1 : buf0) + (uint32_t)((cc & 1) * 32768); };
+                chain_mma_slices(tmem, 0, 4, upd, upd);
+                umma_commit(&ctl.tfull[1]);
+            }
+            // the next leaf's tile: P[127-r][127-c] = A_ii[r][c] - (R R^T)[r][c]
+            wok = ctl.flag && mbar_wait(&ctl.tfull[1], par, -(2700000LL + j)) &&
+                  mbar_wait(&ctl.cin[0], par, -(2800000LL + j));
+            tc_fence_after();
+            if (lane == 0) bulk_wait_read<0>();   // R_ij's TMA stores have read the slices P overlays
+            if (tid == 0) DAG_TRACE(16 * j + 7, globaltimer_ns());
+            leaf_sync();
+            if (wok) {
+                for (int cl = 0; cl < 2; ++cl) {
+                    const int cc = 2 * h + cl;
+                    float v[32];
+                    chain_fetch(tmem, lane_off, cc, v);
+                    const uint8_t* cb = cbuf + (q * 4 + cc) * 4096;   // box (rows 32q.., columns 32 cc..)
+                    const int r = 32 * q + lane;
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 a4 = *reinterpret_cast<const float4*>(cb + lane * 128 + ((c4 ^ (lane & 7)) << 4));
+                        const int col = 32 * cc + 4 * c4;
+                        S.P[127 - r][127 - col] = a4.x - v[4 * c4 + 0];
+                        S.P[127 - r][126 - col] = a4.y - v[4 * c4 + 1];
+                        S.P[127 - r][125 - col] = a4.z - v[4 * c4 + 2];
+                        S.P[127 - r][124 - col] = a4.w - v[4 * c4 + 3];
+                    }
+                }
+            } else if (lane == 0) {
+                ctl.flag = 0;
+            }
+            if (lane == 0) {   // this warp's stores of R_ij are complete
+                bulk_wait<0>();
+                fence_proxy_async_global();
+            }
+            tc_fence_before();
+            leaf_sync();
+            if (tid == 0 && ctl.flag) {
+                __threadfence();
+                atomicAdd(&rs_done[i * T + j], 1);
+                DAG_TRACE(16 * j + 8, globaltimer_ns());
+            }
+            have_tile = ctl.flag != 0;
         }
-        leaf_sync();
-        if (tid == 0) {
-            fence_proxy_async_global();
-            __threadfence();
-            atomicAdd(&diag_done[j], 1);
-            DAG_TRACE(16 * j + 2, globaltimer_ns());
-        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -345,10 +585,9 @@ __global__ void __launch_bounds__(DAG_BLOCK, 1)
 
     if (threadIdx.x == 0) ctl.flag = atomicAdd(g.ctr + 1, 1);
     __syncthreads();
-    if (ctl.flag == 0) {   // the first CTA to start runs the leaves, on warps 0-7
-        if (warp >= DAG_THREADS / 32) return;
-        leaf_sync();
-        dag_leaf_role(g, *reinterpret_cast<LeafSmem*>(smem), ctl);
+    if (ctl.flag == 0) {   // the first CTA to start runs the leaves
+        __syncthreads();
+        dag_leaf_role(maps, g, *reinterpret_cast<LeafSmem*>(smem), ctl);
         return;
     }
 
@@ -417,6 +656,7 @@ __global__ void __launch_bounds__(DAG_BLOCK, 1)
             ctl.slot[s] = tk;
             mbar_arrive(&ctl.task_full[s]);
             if (tk.type == DT_STOP) break;
+            if (tk.type == DT_DIAG) continue;   // no operands: the epilogue warps copy
             fence_proxy_async_global();   // the counters were acquired; TMA reads follow
             const CUtensorMap *ma_h, *ma_l, *mb_h, *mb_l;
             int ax, ay, bx, by;
@@ -466,6 +706,7 @@ __global__ void __launch_bounds__(DAG_BLOCK, 1)
             if (!mbar_wait(&ctl.task_full[s], (uint32_t)(nt / DAG_SLOTS) & 1, -5000000LL - blockIdx.x)) break;
             const DagTask tk = ctl.slot[s];
             if (tk.type == DT_STOP) break;
+            if (tk.type == DT_DIAG) continue;
             if (seg > 0) {   // the previous task's cross accumulator has been read
                 const int pb = (seg - 1) & 1;
                 if (!mbar_wait(&ctl.tempty[pb], (uint32_t)((seg - 1) >> 1) & 1, -5100000LL - blockIdx.x)) break;
@@ -542,6 +783,38 @@ __global__ void __launch_bounds__(DAG_BLOCK, 1)
             const DagTask tk = ctl.slot[s];
             named_bar_epi();
             if (!all || tk.type == DT_STOP) break;
+            if (tk.type == DT_DIAG) {
+                // U_jj = X_jj hi + lo (exact: lo is unrounded) to the public U (clipped), and
+                // the split transposed to U^T: 32 x 32 blocks through this warp's staging box
+                const long long jb = (long long)tk.a * NB, nn = g.n;
+                const float* xh = g.Xd_hi + (long long)tk.a * NB * NB;
+                const float* xl = g.Xd_lo + (long long)tk.a * NB * NB;
+                for (int bk = ew; bk < 16; bk += DAG_EPI_WARPS) {
+                    const int bi = bk >> 2, bj = bk & 3;
+                    float vh[32], vl[32], vu[32];
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 a4 = __ldcg(reinterpret_cast<const float4*>(xh + (32 * bi + lane) * NB + 32 * bj + 4 * c4));
+                        const float4 b4 = __ldcg(reinterpret_cast<const float4*>(xl + (32 * bi + lane) * NB + 32 * bj + 4 * c4));
+                        vh[4 * c4] = a4.x, vh[4 * c4 + 1] = a4.y, vh[4 * c4 + 2] = a4.z, vh[4 * c4 + 3] = a4.w;
+                        vl[4 * c4] = b4.x, vl[4 * c4 + 1] = b4.y, vl[4 * c4 + 2] = b4.z, vl[4 * c4 + 3] = b4.w;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) vu[u] = vh[u] + vl[u];
+                    emit_block(kb, lane, vu, false, g.U, g.d, g.d, g.d, jb + 32 * bi, jb + 32 * bj);
+                    emit_block(kb, lane, vh, true, g.UT_hi, nn, nn, nn, jb + 32 * bj, jb + 32 * bi);
+                    emit_block(kb, lane, vl, true, g.UT_lo, nn, nn, nn, jb + 32 * bj, jb + 32 * bi);
+                }
+                named_bar_epi();
+                if (warp == 2 && lane == 0) {
+                    fence_proxy_async_global();
+                    __threadfence();
+                    atomicAdd(dag_done_ctr(g, tk), 1);
+                    DAG_TRACE(16 * (long long)tk.a + 2, globaltimer_ns());
+                    mbar_arrive(&ctl.task_empty[s]);
+                }
+                continue;
+            }
             // the task's epilogue: outputs
             const long long n = g.n;
             const int i0 = tk.a * NB + 32 * q;   // first tile row of this warp (global row)

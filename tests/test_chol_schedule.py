@@ -2,7 +2,9 @@
 
 The factorization kernel behind gptq_prepare_hinv hands out 128 x 128 tile products in the
 order gptq_chol_schedule returns, one CTA forming the diagonal blocks (leaves) in the order
-j = T-1 .. 0.  These tests take that order from the library and check, on the host:
+j = T-1 .. 0 and, after each leaf j >= 1, the two products the next leaf needs (the panel
+tile PANEL(j, j-1) and the diagonal update UPDATE(j, j-1, j-1)).  These tests take that
+order from the library and check, on the host:
   * every product appears exactly once;
   * every product's inputs are produced earlier (the leaf of step j before step j's
     products), which makes the dynamic ticket order deadlock-free on any number of CTAs;
@@ -18,22 +20,26 @@ import pytest
 
 from post_weight_quantization_14_b200 import gptq
 
-PANEL, UPDATE, FIN, SUPD = 0, 1, 2, 3
+PANEL, UPDATE, FIN, SUPD, DIAG = 0, 1, 2, 3, 4
 
 
 def step_of(t):
     typ, a, b, c = t
-    return {PANEL: b, UPDATE: c, FIN: a, SUPD: c}[typ]
+    return {PANEL: b, UPDATE: c, FIN: a, SUPD: c, DIAG: a}[typ]
 
 
 def expected_tasks(T):
+    """Every product of the factorization except those the leaf CTA forms itself."""
     s = set()
     for j in range(T):
         for i in range(j):
-            s.add((PANEL, i, j, 0))
+            if i != j - 1:
+                s.add((PANEL, i, j, 0))
             for k in range(i, j):
-                s.add((UPDATE, i, k, j))
+                if not (i == k == j - 1):
+                    s.add((UPDATE, i, k, j))
     for i in range(T):
+        s.add((DIAG, i, 0, 0))
         for m in range(i + 1, T):
             s.add((FIN, i, m, 0))
             for k in range(i + 1, m + 1):
@@ -68,12 +74,16 @@ class Counters:
         self.s_cnt = np.zeros((T, T), int)
         self.u_done = np.zeros((T, T), int)
         self.leaf_done = np.zeros(T, int)
+        self.diag_done = np.zeros(T, int)
 
     def ready(self, t):
         T = self.T
-        if t[0] == "LEAF":
+        if t[0] == "LEAF":   # the leaf of j, then (j >= 1) the panel tile (j-1, j) and A_{j-1,j-1}'s update
             j = t[1]
-            return self.a_cnt[j, j] >= T - 1 - j
+            ok = self.a_cnt[j, j] >= T - 1 - j
+            if j >= 1:
+                ok = ok and self.a_cnt[j - 1, j] >= T - 1 - j and self.a_cnt[j - 1, j - 1] >= T - 1 - j
+            return ok
         typ, a, b, c = t
         if typ == PANEL:
             return self.leaf_done[b] >= 1 and self.a_cnt[a, b] >= T - 1 - b
@@ -81,14 +91,17 @@ class Counters:
             return self.rs_done[a, c] >= 1 and self.rs_done[b, c] >= 1 and self.a_cnt[a, b] >= T - 1 - c
         if typ == FIN:
             return self.leaf_done[a] >= 1 and self.s_cnt[a, b] >= b - a
-        up = self.leaf_done[b] >= 1 if c == b else self.u_done[c, b] >= 1
+        if typ == DIAG:
+            return self.leaf_done[a] >= 1
+        up = self.diag_done[b] >= 1 if c == b else self.u_done[c, b] >= 1
         return self.rs_done[a, c] >= 1 and up and self.s_cnt[a, b] >= b - c
 
     def exact(self, t):
         """A read-modify-write task must see exactly the earlier contributions."""
         T = self.T
         if t[0] == "LEAF":
-            return self.a_cnt[t[1], t[1]] == T - 1 - t[1]
+            j = t[1]
+            return self.a_cnt[j, j] == T - 1 - j and (j == 0 or self.a_cnt[j - 1, j - 1] == T - 1 - j)
         typ, a, b, c = t
         if typ == UPDATE:
             return self.a_cnt[a, b] == T - 1 - c
@@ -98,7 +111,11 @@ class Counters:
 
     def done(self, t):
         if t[0] == "LEAF":
-            self.leaf_done[t[1]] += 1
+            j = t[1]
+            self.leaf_done[j] += 1
+            if j >= 1:
+                self.rs_done[j - 1, j] += 1
+                self.a_cnt[j - 1, j - 1] += 1
             return
         typ, a, b, c = t
         if typ == PANEL:
@@ -107,6 +124,8 @@ class Counters:
             self.a_cnt[a, b] += 1
         elif typ == FIN:
             self.u_done[a, b] += 1
+        elif typ == DIAG:
+            self.diag_done[a] += 1
         else:
             self.s_cnt[a, b] += 1
 
@@ -161,6 +180,9 @@ def test_block_formulas_give_hinv_factor(T, b):
             R[blk(j), blk(j)] = Rjj
             X_inv[j] = np.linalg.inv(Rjj)
             U[blk(j), blk(j)] = X_inv[j]
+            if j >= 1:   # the leaf CTA's two products for the next leaf
+                R[blk(j - 1), blk(j)] = A[blk(j - 1), blk(j)] @ X_inv[j].T
+                A[blk(j - 1), blk(j - 1)] -= R[blk(j - 1), blk(j)] @ R[blk(j - 1), blk(j)].T
             continue
         typ, a, bb, c = t
         if typ == PANEL:
@@ -172,6 +194,8 @@ def test_block_formulas_give_hinv_factor(T, b):
         elif typ == FIN:
             i, m = a, bb
             U[blk(i), blk(m)] = -X_inv[i] @ S[blk(i), blk(m)]
+        elif typ == DIAG:
+            pass   # a copy of U_jj, already in place
         else:
             i, m, k = a, bb, c
             S[blk(i), blk(m)] += R[blk(i), blk(k)] @ U[blk(k), blk(m)]
