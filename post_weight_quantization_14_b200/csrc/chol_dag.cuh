@@ -316,7 +316,62 @@ __device__ __forceinline__ void dag_leaf_role(const DagMaps& maps, const DagArgs
     tc_fence_after();
     const uint32_t tmem = ctl.tmem_slot;
 
-    if (warp < DAG_THREADS / 32) {   // warps 8-9 take no part
+    if (warp == DAG_THREADS / 32) {
+        // ---- warp 8: per chain step j >= 1, X_jj's split (the panel tile's B slices) to global
+        // memory, then leaf_done; R_ij (the panel tile) to R's split, then rs_done; three
+        // handshakes with warps 0-7 (barrier 6: slices written, barrier 7: slices read by the TMA)
+        for (int j = T - 1; j >= 1; --j) {
+            const int i = j - 1, ib = i * NB;
+            int* leaf_done_ = a_cnt + 4 * T * T;
+            // X slices s0, s0 + 1: B hi at buffer + 32 KB, lo at + 48 KB, 128 rows x 32 columns each
+            auto store_x = [&](int s0) {
+                for (int sl = s0; sl < s0 + 2; ++sl) {
+                    uint8_t* bh = ((sl & 1) ? buf1 : buf0) + 32768;
+                    tma_store_2d(&maps.xd_hi, bh, 32 * sl, j * NB);
+                    tma_store_2d(&maps.xd_lo, bh + 16384, 32 * sl, j * NB);
+                }
+                bulk_commit();
+                bulk_wait_read<0>();
+            };
+            for (int hs = 0; hs < 2; ++hs) {   // X_jj's split, two slices at a time
+                nbar_sync(6, DAG_THREADS + 32);
+                const bool st = ctl.flag != 0;
+                if (lane == 0 && st) store_x(2 * hs);
+                __syncwarp();
+                nbar_arrive(7, DAG_THREADS + 32);
+            }
+            if (lane == 0 && ctl.flag) {
+                bulk_wait<0>();
+                fence_proxy_async_global();
+                __threadfence();
+                atomicAdd(&leaf_done_[j], 1);
+                DAG_TRACE(16 * j + 1, globaltimer_ns());
+            }
+            __syncwarp();
+            nbar_sync(6, DAG_THREADS + 32);   // R_ij's slices
+            const bool st = ctl.flag != 0;
+            if (lane == 0 && st) {
+                for (int cc = 0; cc < 4; ++cc)
+                    for (int qq = 0; qq < 4; ++qq) {
+                        uint8_t* sh = ((cc >> 1) ? buf1 : buf0) + (cc & 1) * 32768 + qq * 4096;
+                        tma_store_2d(&maps.rs_hi32, sh, j * NB + 32 * cc, ib + 32 * qq);
+                        tma_store_2d(&maps.rs_lo32, sh + 16384, j * NB + 32 * cc, ib + 32 * qq);
+                    }
+                bulk_commit();
+                bulk_wait_read<0>();
+            }
+            __syncwarp();
+            nbar_arrive(7, DAG_THREADS + 32);
+            if (lane == 0 && st) {
+                bulk_wait<0>();
+                fence_proxy_async_global();
+                __threadfence();
+                atomicAdd(&rs_done[i * T + j], 1);
+                DAG_TRACE(16 * j + 8, globaltimer_ns());
+            }
+            __syncwarp();
+        }
+    } else if (warp < DAG_THREADS / 32) {   // warp 9 takes no part
         // ---- warps 0-7: the leaves and the chain products
         const int q = warp & 3, h = warp >> 2;              // TMEM lane quadrant, chunk half
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
@@ -358,46 +413,11 @@ __device__ __forceinline__ void dag_leaf_role(const DagMaps& maps, const DagArgs
                 DAG_TRACE(16 * j, globaltimer_ns());
             }
             const bool alive = ctl.flag != 0;
-            if (alive) {
-                if (tid == 0) DAG_TRACE(16 * j + 12, globaltimer_ns());
-                leaf_factor(S, (int)jb);
-                // X_jj (block of U = J X J, upper) as its tf32 split, row-major: the operand of
-                // the other panels of step j and of row j of U
-                float* xh = g.Xd_hi + (long long)j * NB * NB;
-                float* xl = g.Xd_lo + (long long)j * NB * NB;
-#pragma unroll 4
-                for (int it = 0; it < 16; ++it) {
-                    const int task = tid + it * DAG_THREADS, r = task >> 5, cc = (task & 31) * 4;
-                    const float4 xv = ld4(&S.X[127 - r][124 - cc]);
-                    float v[4] = {xv.w, xv.z, xv.y, xv.x};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        if (r > cc + e) v[e] = 0.f;
-                    float hh[4], ll[4];   // lo unrounded: hi + lo restores X_jj exactly
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        hh[e] = to_tf32(v[e]);
-                        ll[e] = v[e] - hh[e];
-                    }
-                    *reinterpret_cast<float4*>(xh + r * NB + cc) = make_float4(hh[0], hh[1], hh[2], hh[3]);
-                    *reinterpret_cast<float4*>(xl + r * NB + cc) = make_float4(ll[0], ll[1], ll[2], ll[3]);
-                }
-                leaf_sync();
-                if (tid == 0) {   // release: the stores (ordered by the barrier), then the counter
-                    fence_proxy_async_global();
-                    __threadfence();
-                    atomicAdd(&leaf_done[j], 1);
-                    DAG_TRACE(16 * j + 1, globaltimer_ns());
-                }
-            }
-            have_tile = false;
-            if (!alive || j == 0) continue;
-
-            // ---------------- the chain products of step j (i = j - 1)
+            const bool chain = alive && j >= 1;
             const int i = j - 1;
             const int ib = i * NB;
-            // operand slice s (K = 32 s .. 32 s + 31): slices 0, 1 in buf0 / buf1, then 2, 3
-            // again; [A hi | A lo | B hi | B lo], 16 KB each
+            // chain operand slice s (K = 32 s .. 32 s + 31): slices 0, 1 in buf0 / buf1, then
+            // 2, 3 again; [A hi | A lo | B hi | B lo], 16 KB each
             auto slice_buf = [&](int s) { return (s & 1) ? buf1 : buf0; };
             // B slices of the panel: X_jj rows n, columns 32 s .. (U_jj[n][k] = S.X[127-n][127-k])
             auto put_x_slices = [&](int s0) {
@@ -432,7 +452,55 @@ __device__ __forceinline__ void dag_leaf_role(const DagMaps& maps, const DagArgs
                     tma_load_2d(ab + 16384, &maps.rs_lo, bar_a[sl], (int)jb + 32 * sl, ib);
                 }
             };
+            auto panel_a = [&](int s) { return smem_u32(slice_buf(s)); };
+            auto panel_b = [&](int s) { return smem_u32(slice_buf(s)) + 32768u; };
             bool ok = true;
+            if (alive) {
+                if (tid == 0) DAG_TRACE(16 * j + 12, globaltimer_ns());
+                leaf_factor(S, (int)jb);
+            }
+            have_tile = false;
+            if (!chain) {
+                if (alive) {   // the last leaf: X_jj's split stored by the leaf warps
+                    float* xh = g.Xd_hi + (long long)j * NB * NB;
+                    float* xl = g.Xd_lo + (long long)j * NB * NB;
+#pragma unroll 4
+                    for (int it = 0; it < 16; ++it) {
+                        const int task = tid + it * DAG_THREADS, r = task >> 5, cc = (task & 31) * 4;
+                        const float4 xv = ld4(&S.X[127 - r][124 - cc]);
+                        float v[4] = {xv.w, xv.z, xv.y, xv.x};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            if (r > cc + e) v[e] = 0.f;
+                        float hh[4], ll[4];   // lo unrounded: hi + lo restores X_jj exactly
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            hh[e] = to_tf32(v[e]);
+                            ll[e] = v[e] - hh[e];
+                        }
+                        *reinterpret_cast<float4*>(xh + r * NB + cc) = make_float4(hh[0], hh[1], hh[2], hh[3]);
+                        *reinterpret_cast<float4*>(xl + r * NB + cc) = make_float4(ll[0], ll[1], ll[2], ll[3]);
+                    }
+                    leaf_sync();
+                    if (tid == 0) {   // release: the stores (ordered by the barrier), then the counter
+                        fence_proxy_async_global();
+                        __threadfence();
+                        atomicAdd(&leaf_done[j], 1);
+                        DAG_TRACE(16 * j + 1, globaltimer_ns());
+                    }
+                }
+                if (j >= 1)   // keep the store warp's three handshakes (see below) in step
+                    for (int hs = 0; hs < 3; ++hs) {
+                        nbar_arrive(6, DAG_THREADS + 32);
+                        nbar_sync(7, DAG_THREADS + 32);
+                    }
+                continue;
+            }
+
+            // ---------------- the chain products of step j (i = j - 1).  X_jj's split is formed
+            // once, as the panel tile's B operand; warp 8 stores those slices to X_jj's split in
+            // global memory (then leaf_done) and, later, R_ij's slices (then rs_done), while
+            // these warps go on; each store is a handshake (barrier 6: written, 7: read).
             if (tid == 0) {
                 ok = dag_wait_ge(&a_cnt[i * T + j], T - 1 - j, abort, -(2200000LL + j));
                 if (ok) {
@@ -445,10 +513,9 @@ __device__ __forceinline__ void dag_leaf_role(const DagMaps& maps, const DagArgs
             put_x_slices(0);
             fence_proxy_async_smem();
             leaf_sync();
-            if (tid == 0) DAG_TRACE(16 * j + 3, globaltimer_ns());
-            auto panel_a = [&](int s) { return smem_u32(slice_buf(s)); };
-            auto panel_b = [&](int s) { return smem_u32(slice_buf(s)) + 32768u; };
+            nbar_arrive(6, DAG_THREADS + 32);   // X slices 0-1 written
             if (tid == 0 && ok) {
+                DAG_TRACE(16 * j + 3, globaltimer_ns());
                 for (int sl = 0; sl < 2 && ok; ++sl) {
                     ok = mbar_wait(bar_a[sl], par, -(2300000LL + j));
                     tc_fence_after();
@@ -459,11 +526,12 @@ __device__ __forceinline__ void dag_leaf_role(const DagMaps& maps, const DagArgs
                 if (ok) load_a_slices(2);
                 if (!ok) ctl.flag = 0;
             }
-            leaf_sync();
+            nbar_sync(7, DAG_THREADS + 32);     // ... and read by the TMA
             if (tid == 0) DAG_TRACE(16 * j + 4, globaltimer_ns());
             if (ctl.flag) put_x_slices(2);
             fence_proxy_async_smem();
             leaf_sync();
+            nbar_arrive(6, DAG_THREADS + 32);   // X slices 2-3 written
             if (tid == 0 && ctl.flag) {
                 for (int sl = 2; sl < 4 && ok; ++sl) {
                     ok = mbar_wait(bar_a[sl], par, -(2300000LL + j));
@@ -484,10 +552,12 @@ __device__ __forceinline__ void dag_leaf_role(const DagMaps& maps, const DagArgs
                     ctl.flag = 0;
                 }
             }
-            // R_ij: from tensor memory to the update's operand slices (both A and B) and, by
-            // TMA, to R's split in global memory; warp (q, h) takes rows 32q.., chunks 2h, 2h+1
+            // R_ij: from tensor memory to the update's operand slices (both A and B); warp
+            // (q, h) takes rows 32q.., chunks 2h, 2h+1.  Warp 8 stores the slices to R's split
+            // in global memory by TMA and releases rs_done, off this chain.
             bool wok = mbar_wait(&ctl.tfull[0], par, -(2600000LL + j));
             tc_fence_after();
+            nbar_sync(7, DAG_THREADS + 32);     // X slices 2-3 read by the TMA
             if (tid == 0) DAG_TRACE(16 * j + 5, globaltimer_ns());
             if (wok) {
                 for (int cl = 0; cl < 2; ++cl) {
@@ -500,18 +570,13 @@ __device__ __forceinline__ void dag_leaf_role(const DagMaps& maps, const DagArgs
                     uint8_t* sh = ((cc >> 1) ? buf1 : buf0) + (cc & 1) * 32768 + q * 4096;   // rows 32q.. of slice cc
                     box_put_row(sh, lane, hh);
                     box_put_row(sh + 16384, lane, ll);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&maps.rs_hi32, sh, (int)jb + 32 * cc, ib + 32 * q);
-                        tma_store_2d(&maps.rs_lo32, sh + 16384, (int)jb + 32 * cc, ib + 32 * q);
-                        bulk_commit();
-                    }
                 }
             } else if (lane == 0) {
                 ctl.flag = 0;
             }
+            fence_proxy_async_smem();
             tc_fence_before();
+            nbar_arrive(6, DAG_THREADS + 32);   // the slices are written: warp 8 may store them
             leaf_sync();
             if (tid == 0 && ctl.flag) {   // the update: A = B = R_ij's slices (cc: buffer cc >> 1, half cc & 1)
                 DAG_TRACE(16 * j + 6, globaltimer_ns());
@@ -524,9 +589,8 @@ __device__ __forceinline__ void dag_leaf_role(const DagMaps& maps, const DagArgs
             wok = ctl.flag && mbar_wait(&ctl.tfull[1], par, -(2700000LL + j)) &&
                   mbar_wait(&ctl.cin[0], par, -(2800000LL + j));
             tc_fence_after();
-            if (lane == 0) bulk_wait_read<0>();   // R_ij's TMA stores have read the slices P overlays
+            nbar_sync(7, DAG_THREADS + 32);   // warp 8's stores have read the slices P overlays
             if (tid == 0) DAG_TRACE(16 * j + 7, globaltimer_ns());
-            leaf_sync();
             if (wok) {
                 for (int cl = 0; cl < 2; ++cl) {
                     const int cc = 2 * h + cl;
@@ -547,17 +611,8 @@ __device__ __forceinline__ void dag_leaf_role(const DagMaps& maps, const DagArgs
             } else if (lane == 0) {
                 ctl.flag = 0;
             }
-            if (lane == 0) {   // this warp's stores of R_ij are complete
-                bulk_wait<0>();
-                fence_proxy_async_global();
-            }
             tc_fence_before();
             leaf_sync();
-            if (tid == 0 && ctl.flag) {
-                __threadfence();
-                atomicAdd(&rs_done[i * T + j], 1);
-                DAG_TRACE(16 * j + 8, globaltimer_ns());
-            }
             have_tile = ctl.flag != 0;
         }
     }
