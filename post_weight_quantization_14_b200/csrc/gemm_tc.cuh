@@ -427,6 +427,21 @@ __global__ void __launch_bounds__(192, 1)
             const int nseg = max(1, (nkk + segk - 1) / segk);
             const uint32_t lane_off = (uint32_t)(q * 32) << 16;
             bool ok = true;
+            // C (beta != 0) is fetched while the MMAs run
+            const int zc_x = p.c_col0 + ti.z * p.c_zcol, zc_y = p.c_row0 + ti.z * p.c_zrow;
+            const int iy = ti.m0 + 32 * q;
+            const bool diag_mirror = p.mirror && ti.nt == ti.mt;
+            const bool fetch_c = use_c && !diag_mirror;
+            if (fetch_c) {
+                fence_proxy_async_smem();   // this warp's reads of cbox (previous tile) come first
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&cin_bar[q], NCHUNK * kBoxBytes);
+                    for (int c = 0; c < NCHUNK; ++c)
+                        tma_load_2d(cbox + c * kBoxBytes, &mC, &cin_bar[q], zc_x + ti.n0 + 32 * c, zc_y + iy);
+                }
+                __syncwarp();
+            }
             // Segments before the last: add the accumulator into the running sum (TMEM
             // columns SUM_HI .., and SUM_LO .. for two-sum) with round-to-nearest fp32
             // arithmetic, then release the buffer.
@@ -487,9 +502,6 @@ __global__ void __launch_bounds__(192, 1)
             const uint32_t acc = tmem + (uint32_t)(buf * TBN) + lane_off;
             const bool multi = nseg > 1;   // the last segment joins a running sum
             const int z = ti.z, n0 = ti.n0, mt = ti.mt, nt = ti.nt;
-            const int zc_x = p.c_col0 + z * p.c_zcol, zc_y = p.c_row0 + z * p.c_zrow;
-            const int iy = ti.m0 + 32 * q;
-            const bool diag_mirror = p.mirror && nt == mt;
             if (!diag_mirror) {
                 const bool mirror = p.mirror && nt > mt;
                 const bool has_c = p.write_c != 0, has_t = p.T_hi != nullptr;
@@ -497,15 +509,7 @@ __global__ void __launch_bounds__(192, 1)
                 const long long zs_x = p.s_col0 + z * p.s_zcol, zs_y = p.s_row0 + z * p.s_zrow;
                 const long long zt_x = p.t_col0 + z * p.t_zcol, zt_y = p.t_row0 + z * p.t_zrow;
                 bool cin_ok = true;
-                if (use_c) {
-                    fence_proxy_async_smem();   // this warp's reads of cbox (previous tile) come first
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(&cin_bar[q], NCHUNK * kBoxBytes);
-                        for (int c = 0; c < NCHUNK; ++c)
-                            tma_load_2d(cbox + c * kBoxBytes, &mC, &cin_bar[q], zc_x + n0 + 32 * c, zc_y + iy);
-                    }
-                    __syncwarp();
+                if (fetch_c) {
                     cin_ok = mbar_wait(&cin_bar[q], cin_use & 1, w);
                     ++cin_use;
                 }
