@@ -136,8 +136,8 @@ __global__ void __launch_bounds__(256) damp_copy_perm_kernel(const float* __rest
     }
 }
 
-// Zero the strictly-lower 128-blocks of the d x d output U (diagonal blocks are
-// written in full by chol_diag_out_kernel).
+// Zero the strictly-lower 128-blocks of the d x d output U (the diagonal and upper
+// blocks are written by the factorization).
 __global__ void __launch_bounds__(256) zero_lower_blocks_kernel(float* __restrict__ U, long long d) {
     const int bi = blockIdx.y, bj = blockIdx.x;   // one CTA per 128-block, strictly lower only
     if (bi <= bj) return;

@@ -1151,7 +1151,7 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
         GQ_TRY(cudaGetLastError());
     }
     {
-        gqh::TimedScope ts__("zero_lower", st);
+        gqh::TimedScope ts__("zero_lower", st);   // the public U's strictly lower blocks
         gq::zero_lower_blocks_kernel<<<dim3((unsigned)T, (unsigned)T), 256, 0, st>>>(U, d);
     }
     GQ_TRY(cudaGetLastError());

@@ -2,9 +2,8 @@
 // operands and fp32 accumulators in tensor memory.
 //
 //   D[i, j] = sum_k A[i, k] * B[j, k]      (i < M, j < N, k in the tile's K range)
-//   out     = alpha * D + beta * C[i, j]   -> written to any of: C (row-major fp32),
-//             S_hi/S_lo (row-major tf32 split of out), T_hi/T_lo (transposed tf32 split),
-//             and, for symmetric updates, the mirrored C[j, i].
+//   out     = alpha * D + beta * C[i, j]   -> written to C (row-major fp32) and, for
+//             symmetric products, also to the mirrored C[j, i].
 //
 // KIND_BF16   : A, B bf16 (kind::f16), one MMA per 16-element K step.
 // KIND_TF32X3 : A = A_hi + A_lo and B = B_hi + B_lo given as two tf32 arrays each;
@@ -23,8 +22,10 @@
 // Persistent and warp-specialised: each CTA walks tiles blockIdx.x, +gridDim.x, ...
 // Warp 0 issues TMA into a ring of STAGES operand buffers that runs across tiles;
 // warp 1 issues MMAs into one of two TMEM accumulators (tile parity), so the epilogue
-// of one tile overlaps the mainloop of the next; warps 2..5 run the epilogue: each
-// warp owns 32 accumulator rows, loads its C chunks by TMA when beta != 0, and writes
+// of one tile overlaps the mainloop of the next; the epilogue warps (eight for 128-wide
+// tiles: two per TMEM lane quadrant, two 32-column chunks each; four otherwise) own 32
+// accumulator rows each, load their C chunks by TMA while the MMAs run when beta != 0,
+// and write
 // every output 32x32 block through a 128-byte-swizzled staging box in shared memory with
 // coalesced 16-byte stores (no store-completion waits inside a tile).  Tiles on the
 // diagonal of a mirrored (symmetric) output take a register path that writes j >= i and
@@ -58,15 +59,6 @@ struct GemmArgs {
     int c_row0, c_col0, c_zrow, c_zcol;
     int write_c;
     int mirror;       // also write C[j, i] for tiles above the diagonal
-    float* S_hi;
-    float* S_lo;
-    long long lds, s_rows, s_cols;
-    int s_row0, s_col0, s_zrow, s_zcol;
-    int s_mt_lim;     // if > 0: S written only by tiles with mt < s_mt_lim
-    float* T_hi;
-    float* T_lo;
-    long long ldt, t_rows, t_cols;
-    int t_row0, t_col0, t_zrow, t_zcol;
 };
 
 constexpr int BM = 128;
@@ -77,10 +69,20 @@ constexpr int kBoxBytes = 32 * 32 * 4;           // one 32x32 fp32 box, 128-byte
 // epilogue stores are then spread over four times as many SMs).  Each epilogue warp owns
 // a region of TBN / 32 C boxes (beta != 0) plus two boxes: the staging box and, for the
 // register path of mirrored diagonal tiles, room for a padded 32x33 tile.
+// Epilogue warps: eight for 128-wide tiles (two per TMEM lane quadrant, two 32-column chunks
+// each), four otherwise (one per quadrant, all chunks).  Each owns three boxes: its C chunks
+// (beta != 0) and a staging box for the coalesced stores.
 template <int TBN>
-__host__ __device__ constexpr int epi_boxes_per_warp() { return TBN / 32 + 2; }
+__host__ __device__ constexpr int epi_warps() { return TBN == 128 ? 8 : 4; }
 template <int TBN>
-__host__ __device__ constexpr int epi_bytes() { return 4 * epi_boxes_per_warp<TBN>() * kBoxBytes; }   // 96 KB at TBN = 128
+__host__ __device__ constexpr int epi_chunks_per_warp() { return (TBN / 32) / (epi_warps<TBN>() / 4); }
+template <int TBN>
+__host__ __device__ constexpr int epi_boxes_per_warp() { return 3; }
+template <int TBN>
+__host__ __device__ constexpr int epi_bytes() { return epi_warps<TBN>() * epi_boxes_per_warp<TBN>() * kBoxBytes; }   // 96 KB at TBN = 128
+template <int TBN>
+__host__ __device__ constexpr int gemm_threads() { return 64 + 32 * epi_warps<TBN>(); }
+static_assert(epi_chunks_per_warp<128>() + 1 <= 3 && epi_chunks_per_warp<32>() + 1 <= 3, "C chunks + staging box");
 static_assert(32 * kEpiLd * 4 <= 2 * kBoxBytes, "register-path staging tile fits two boxes");
 
 template <int KIND, int TBN = BN>
@@ -231,7 +233,7 @@ __device__ __forceinline__ void fetch_chunk(uint32_t tmem, uint32_t acc, uint32_
 }
 
 template <int KIND, int STAGES, int TBN, int SEG>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(gemm_threads<TBN>(), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
                    const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mB2,
                    const __grid_constant__ CUtensorMap mC, const GemmArgs p) {
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(192, 1)
     constexpr uint32_t TMEM_COLS = TMEM_NEED <= 32 ? 32u : TMEM_NEED <= 64 ? 64u : TMEM_NEED <= 128 ? 128u
                                  : TMEM_NEED <= 256 ? 256u : 512u;
     static_assert(TMEM_NEED <= 512, "tensor memory columns");
-    constexpr int NCHUNK = TBN / 32;
+
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -261,8 +263,9 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* empty_bar = full_bar + STAGES;
     uint64_t* tfull_bar = empty_bar + STAGES;   // [2] accumulator ready
     uint64_t* tempty_bar = tfull_bar + 2;       // [2] accumulator drained (4 epilogue warps)
-    uint64_t* cin_bar = tempty_bar + 2;         // [4] per-warp C chunk loads
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cin_bar + 4);
+    constexpr int EPIW = epi_warps<TBN>(), CPW = epi_chunks_per_warp<TBN>();
+    uint64_t* cin_bar = tempty_bar + 2;         // [EPIW] per-warp C chunk loads
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cin_bar + EPIW);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tiles_per_batch = tiles_of(p.tiles_m, p.tiles_n, p.triangular, p.tri_r);
@@ -275,9 +278,9 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull_bar[b], 1);
-            mbar_init(&tempty_bar[b], 4);
+            mbar_init(&tempty_bar[b], EPIW);
         }
-        for (int q = 0; q < 4; ++q) mbar_init(&cin_bar[q], 1);
+        for (int q = 0; q < EPIW; ++q) mbar_init(&cin_bar[q], 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -409,13 +412,14 @@ __global__ void __launch_bounds__(192, 1)
             ++seg;
         }
     } else if (warp >= 2) {
-        // ---------------- epilogue: warp q owns accumulator rows 32q .. 32q+31 of every tile
-        const int q = warp & 3;
+        // ---------------- epilogue: warp w (2 ..) owns accumulator rows 32q .. 32q+31 of every
+        // tile, q = w % 4, and the chunks c0e .. c0e + CPW - 1 of them
+        const int q = warp & 3, ew = warp - 2, c0e = (ew >> 2) * CPW;
         const bool use_c = p.beta != 0.f;
-        // with beta: this warp's C chunks, then its extra boxes; without: its output boxes
-        uint8_t* wreg = epi + q * epi_boxes_per_warp<TBN>() * kBoxBytes;   // this warp's region
+        // this warp's C chunks (beta != 0), then its staging box
+        uint8_t* wreg = epi + ew * epi_boxes_per_warp<TBN>() * kBoxBytes;   // this warp's region
         uint8_t* cbox = wreg;
-        uint8_t* kb = use_c ? wreg + NCHUNK * kBoxBytes : wreg;             // staging box
+        uint8_t* kb = wreg + CPW * kBoxBytes;                               // staging box
         float* stage_t = reinterpret_cast<float*>(wreg);   // register-path staging (own region)
         int seg = 0;
         uint32_t cin_use = 0;
@@ -436,9 +440,9 @@ __global__ void __launch_bounds__(192, 1)
                 fence_proxy_async_smem();   // this warp's reads of cbox (previous tile) come first
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&cin_bar[q], NCHUNK * kBoxBytes);
-                    for (int c = 0; c < NCHUNK; ++c)
-                        tma_load_2d(cbox + c * kBoxBytes, &mC, &cin_bar[q], zc_x + ti.n0 + 32 * c, zc_y + iy);
+                    mbar_arrive_expect_tx(&cin_bar[ew], CPW * kBoxBytes);
+                    for (int c = 0; c < CPW; ++c)
+                        tma_load_2d(cbox + c * kBoxBytes, &mC, &cin_bar[ew], zc_x + ti.n0 + 32 * (c0e + c), zc_y + iy);
                 }
                 __syncwarp();
             }
@@ -450,7 +454,7 @@ __global__ void __launch_bounds__(192, 1)
                 ok = mbar_wait(&tfull_bar[sb], (uint32_t)(seg >> 1) & 1, w);
                 tc_fence_after();
 #pragma unroll 1
-                for (int c = 0; c < NCHUNK; ++c) {
+                for (int c = c0e; c < c0e + CPW; ++c) {
                     const uint32_t src = tmem + (uint32_t)(sb * TBN + c * 32) + lane_off;
                     const uint32_t dhi = tmem + (uint32_t)(SUM_HI + c * 32) + lane_off;
                     const uint32_t dlo = tmem + (uint32_t)(SUM_LO + c * 32) + lane_off;
@@ -501,20 +505,17 @@ __global__ void __launch_bounds__(192, 1)
             tc_fence_after();
             const uint32_t acc = tmem + (uint32_t)(buf * TBN) + lane_off;
             const bool multi = nseg > 1;   // the last segment joins a running sum
-            const int z = ti.z, n0 = ti.n0, mt = ti.mt, nt = ti.nt;
+            const int n0 = ti.n0, mt = ti.mt, nt = ti.nt;
             if (!diag_mirror) {
                 const bool mirror = p.mirror && nt > mt;
-                const bool has_c = p.write_c != 0, has_t = p.T_hi != nullptr;
-                const bool has_s = p.S_hi != nullptr && (p.s_mt_lim <= 0 || mt < p.s_mt_lim);
-                const long long zs_x = p.s_col0 + z * p.s_zcol, zs_y = p.s_row0 + z * p.s_zrow;
-                const long long zt_x = p.t_col0 + z * p.t_zcol, zt_y = p.t_row0 + z * p.t_zrow;
+                const bool has_c = p.write_c != 0;
                 bool cin_ok = true;
                 if (fetch_c) {
-                    cin_ok = mbar_wait(&cin_bar[q], cin_use & 1, w);
+                    cin_ok = mbar_wait(&cin_bar[ew], cin_use & 1, w);
                     ++cin_use;
                 }
 #pragma unroll 1
-                for (int c = 0; c < NCHUNK; ++c) {
+                for (int c = c0e; c < c0e + CPW; ++c) {
                     const int j0 = n0 + c * 32;
                     uint32_t r[32];
                     if (ti.nk > 0 && ok) {
@@ -523,7 +524,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                         for (int t = 0; t < 32; ++t) r[t] = 0u;
                     }
-                    if (c == NCHUNK - 1) {   // accumulator drained: the MMA warp may reuse it
+                    if (c == c0e + CPW - 1) {   // accumulator drained: the MMA warp may reuse it
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&tempty_bar[buf]);
@@ -533,7 +534,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                     for (int t = 0; t < 32; ++t) out[t] = p.alpha * __uint_as_float(r[t]);
                     if (use_c && cin_ok) {
-                        const uint8_t* cb = cbox + c * kBoxBytes;
+                        const uint8_t* cb = cbox + (c - c0e) * kBoxBytes;
 #pragma unroll
                         for (int c4 = 0; c4 < 8; ++c4) {
                             const float4 v =
@@ -545,19 +546,6 @@ __global__ void __launch_bounds__(192, 1)
                         }
                     }
                     if (has_c) emit_block(kb, lane, out, false, p.C, p.ldc, p.c_rows, p.c_cols, zc_y + iy, zc_x + j0);
-                    if (has_s || has_t) {
-                        float hi[32], lo[32];
-#pragma unroll
-                        for (int t = 0; t < 32; ++t) split_tf32(out[t], hi[t], lo[t]);
-                        if (has_s) {
-                            emit_block(kb, lane, hi, false, p.S_hi, p.lds, p.s_rows, p.s_cols, zs_y + iy, zs_x + j0);
-                            emit_block(kb, lane, lo, false, p.S_lo, p.lds, p.s_rows, p.s_cols, zs_y + iy, zs_x + j0);
-                        }
-                        if (has_t) {
-                            emit_block(kb, lane, hi, true, p.T_hi, p.ldt, p.t_rows, p.t_cols, zt_y + j0, zt_x + iy);
-                            emit_block(kb, lane, lo, true, p.T_lo, p.ldt, p.t_rows, p.t_cols, zt_y + j0, zt_x + iy);
-                        }
-                    }
                     if (mirror) emit_block(kb, lane, out, true, p.C, p.ldc, p.c_rows, p.c_cols, zc_y + j0, zc_x + iy);
                 }
             } else {
@@ -568,7 +556,7 @@ __global__ void __launch_bounds__(192, 1)
                 const int rbase = iy;
                 const long long zr = zc_y, zcc = zc_x;
 #pragma unroll 1
-                for (int c = 0; c < NCHUNK; ++c) {
+                for (int c = c0e; c < c0e + CPW; ++c) {
                     const int j0 = n0 + c * 32;
                     uint32_t r[32];
                     if (ti.nk > 0 && ok) {
@@ -577,7 +565,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                         for (int t = 0; t < 32; ++t) r[t] = 0u;
                     }
-                    if (c == NCHUNK - 1) {
+                    if (c == c0e + CPW - 1) {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&tempty_bar[buf]);
@@ -637,11 +625,10 @@ struct Mat {
     uint64_t rows, cols, ld;  // elements
 };
 
-// Output matrices of the epilogue (ptr == nullptr: not written).  C is also the
-// matrix read when beta != 0 and the target of mirrored writes.
+// The epilogue's output matrix C (ptr == nullptr: not written), also the matrix read when
+// beta != 0 and the target of mirrored writes.
 struct EpiMats {
-    Mat c{nullptr, 0, 0, 0}, s_hi{nullptr, 0, 0, 0}, s_lo{nullptr, 0, 0, 0}, t_hi{nullptr, 0, 0, 0},
-        t_lo{nullptr, 0, 0, 0};
+    Mat c{nullptr, 0, 0, 0};
 };
 
 inline bool make_out_map(CUtensorMap* map, const Mat& m, const CUtensorMap& fallback, bool no_alloc = false) {
@@ -702,16 +689,6 @@ cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2
     p.ldc = (long long)o.c.ld;
     p.c_rows = (long long)o.c.rows;
     p.c_cols = (long long)o.c.cols;
-    p.s_rows = (long long)o.s_hi.rows;
-    p.s_cols = (long long)o.s_hi.cols;
-    p.t_rows = (long long)o.t_hi.rows;
-    p.t_cols = (long long)o.t_hi.cols;
-    p.S_hi = static_cast<float*>(const_cast<void*>(o.s_hi.ptr));
-    p.S_lo = static_cast<float*>(const_cast<void*>(o.s_lo.ptr));
-    p.lds = (long long)o.s_hi.ld;
-    p.T_hi = static_cast<float*>(const_cast<void*>(o.t_hi.ptr));
-    p.T_lo = static_cast<float*>(const_cast<void*>(o.t_lo.ptr));
-    p.ldt = (long long)o.t_hi.ld;
     if (!epilogue_fits(p)) return cudaErrorInvalidValue;
     p.tiles_m = (p.M + gq::BM - 1) / gq::BM;
     p.tiles_n = (p.N + TBN - 1) / TBN;
@@ -727,8 +704,9 @@ cudaError_t launch_gemm(const Mat& a, const Mat& a2, const Mat& b, const Mat& b2
     const unsigned grid = (unsigned)std::min<long long>(tiles, max_ctas > 0 ? max_ctas : num_sms());
     {
         TimedScope ts__(no_alloc ? nullptr : name, stream);
-        e = after_event ? launch_plain(kern, dim3(grid), dim3(192), (size_t)smem, stream, ma, ma2, mb, mb2, mc, p)
-                        : launch_pdl(kern, dim3(grid), dim3(192), (size_t)smem, stream, ma, ma2, mb, mb2, mc, p);
+        constexpr int nthr = gq::gemm_threads<TBN>();
+        e = after_event ? launch_plain(kern, dim3(grid), dim3(nthr), (size_t)smem, stream, ma, ma2, mb, mb2, mc, p)
+                        : launch_pdl(kern, dim3(grid), dim3(nthr), (size_t)smem, stream, ma, ma2, mb, mb2, mc, p);
     }
     return e != cudaSuccess ? e : cudaGetLastError();
 }
