@@ -80,18 +80,32 @@ __global__ void __launch_bounds__(256) damp_copy_kernel(const float* __restrict_
         }
         return;
     }
-    // diagonal block: A[i][j] = H[min(i,j)][max(i,j)] (the few transposed reads are strided)
-    for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-        const int r = e >> 7, c = e & 127;
-        const long long i = r0 + r, j = c0 + c;
-        float v = 0.f;
-        if (i < d && j < d) {
-            v = (r <= c) ? H[i * d + j] : H[j * d + i];
-            if (r <= c && !isfinite(v)) record_status(GPTQ_ERR_NONFINITE, i * d + j);
+    // diagonal block: A[i][j] = H[min(i,j)][max(i,j)], by 32x32 sub-tiles of the upper
+    // triangle read row by row and written both ways through shared memory
+    __shared__ float tile[32][33];
+    for (int bi = 0; bi < 4; ++bi)
+        for (int bj = bi; bj < 4; ++bj) {
+            __syncthreads();   // the previous sub-tile's readers are done
+            for (int t = threadIdx.x; t < 32 * 32; t += blockDim.x) {
+                const int rr = t >> 5, cc = t & 31;
+                const long long i = r0 + 32 * bi + rr, j = c0 + 32 * bj + cc;
+                float v = 0.f;
+                if (i < d && j < d && (bi < bj || rr <= cc)) {
+                    v = H[i * d + j];
+                    if (!isfinite(v)) record_status(GPTQ_ERR_NONFINITE, i * d + j);
+                }
+                tile[rr][cc] = v;
+            }
+            __syncthreads();
+            for (int t = threadIdx.x; t < 32 * 32; t += blockDim.x) {
+                const int rr = t >> 5, cc = t & 31;
+                const long long i = r0 + 32 * bi + rr, j = c0 + 32 * bj + cc;
+                float v = (bi < bj || rr <= cc) ? tile[rr][cc] : tile[cc][rr];
+                if (i == j) v = (i < d) ? v + l : 1.f;
+                A[i * n + j] = v;
+                if (bi < bj) A[(r0 + 32 * bj + rr) * n + c0 + 32 * bi + cc] = tile[cc][rr];
+            }
         }
-        if (i == j) v = (i < d) ? v + l : 1.f;
-        A[i * n + j] = v;
-    }
 }
 
 // The damped copy of damp_copy_kernel for the permuted Hessian: A[i][j] =
