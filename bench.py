@@ -460,6 +460,97 @@ def run_dqgemm(args) -> None:
         "step_ms_min": min(ms), "step_ms_median": statistics.median(ms)}), flush=True)
 
 
+def run_gptq2d(args) -> None:
+    """GPTQ-2D two-sided rounding (GPTQ-2D summary, method steps 1-3): a batch of 148
+    problems of 128 x 128 (one CTA per problem, one per SM), fp64, sharing U_left and
+    U_right; X ~ 3 N(0, 1).  Roofline: fp64 FMA issue (148 SMs x 64 fp64 FMA per clock x
+    1965 MHz) over the algorithmic flops (the dot product of each entry with its column of
+    U_left, i + 1 terms, and the push of its error along its row, n - j terms)."""
+    import numpy as np
+    import torch
+
+    from post_weight_quantization_14_b200 import gptq as G
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    m = n = 128
+    batch = 148
+    rng = np.random.default_rng(11)
+
+    def spd(k):
+        a = rng.standard_normal((k, k)) + 2.0 * np.eye(k)
+        return a.T @ a + 0.1 * np.eye(k)
+
+    def upper_factor_of_inverse(h):   # U with U^T U = h^-1 (plain numpy; inputs only)
+        return np.linalg.cholesky(np.linalg.inv(h)).T.copy()
+
+    UL = upper_factor_of_inverse(spd(m))
+    UR = upper_factor_of_inverse(spd(n))
+    X = rng.standard_normal((batch, m, n)) * 3.0
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    Xd, ULd, URd = t(X), t(UL), t(UR)
+    Z = torch.empty((batch, m, n), dtype=torch.int32, device=dev)
+    ws = torch.empty(G.lib().gptq_2d_workspace_bytes(m, n, batch), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        G.gptq_2d_round(Xd, ULd, URd, Z, workspace=ws)
+    G.gptq_sync_status()
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.3)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in evs:
+        flush.fill_(1)
+        a.record(stream)
+        G.gptq_2d_round(Xd, ULd, URd, Z, workspace=ws)
+        b.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    G.gptq_sync_status()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+    fma = batch * (n * m * (m + 1) / 2 + m * n * (n + 1) / 2)
+    achieved = 2.0 * fma / (ms / 1e3) / 1e12
+    peak = 148 * 64 * 2 * 1.965e9 / 1e12
+
+    # end to end: X in from pinned host memory, Z back to pinned host memory
+    X_host = torch.from_numpy(X).pin_memory()
+    Z_host = torch.empty((batch, m, n), dtype=torch.int32).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    torch.cuda.synchronize()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(stream)
+    for _ in range(e2e_steps):
+        Xd.copy_(X_host, non_blocking=True)
+        G.gptq_2d_round(Xd, ULd, URd, Z, workspace=ws)
+        Z_host.copy_(Z, non_blocking=True)
+    eb.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ea.elapsed_time(eb) / e2e_steps
+
+    cpu = None
+    if not args.no_cpu_baseline:
+        from oracle import gptq_oracle as O
+        t0 = time.perf_counter()
+        O.gptq2d_antidiagonal(X[0], UL, UR)
+        secs = time.perf_counter() - t0
+        cpu = {"value": 1.0 / secs, "unit": "problems/s", "cores": os.cpu_count(), "kind": "oracle",
+               "sample": "one of the 148 problems (the oracle's anti-diagonal route, fp64 numpy)"}
+    line = {"metric": "GPTQ-2D two-sided rounding of 148 problems of 128 x 128 (fp64)", "value": batch / (ms / 1e3),
+            "unit": "problems/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "gptq2d: 148 problems of 128x128, X ~ 3 N(0,1), shared U_left, U_right",
+                       "l2": "flushed (256 MB write) before every step, outside the step events"},
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "traffic": None, "note": "fp64 FMA issue: 148 SMs x 64 FMA/clock x 1965 MHz (derived); the "
+                                                  "kernel walks 255 anti-diagonals with a CTA barrier after each"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": batch / (e2e_ms / 1e3), "unit": "problems/s", "h2d_bytes_per_step": int(X.nbytes),
+                    "d2h_bytes_per_step": int(batch * m * n * 4)},
+            "gpu_launches": 2 * args.steps, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -467,7 +558,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="attn", choices=["attn", "stack7b", "dqgemm"])
+    ap.add_argument("--workload", default="attn", choices=["attn", "stack7b", "dqgemm", "gptq2d"])
     ap.add_argument("--shared-input", action="store_true",
                     help="stack7b: q/k/v and gate/up share one H and U per group (one input each)")
     ap.add_argument("--desc-act", type=int, default=0, choices=[0, 1, 2],
@@ -496,6 +587,8 @@ def main():
     if args.workload == "stack7b":
         run_stack(args)
         return
+    if args.workload == "gptq2d":
+        return run_gptq2d(args)
     if args.workload == "dqgemm":
         run_dqgemm(args)
         return

@@ -14,8 +14,8 @@
 //
 // One CTA (the first to start) runs the leaves in order j = T-1 .. 0.  Every other CTA
 // takes the product tasks from a global ticket counter in a fixed order (dag_step_task):
-// per step j the two tiles the next leaf needs, the rest of panel j, block column j-1, row j
-// of U, the S contributions of panel j, then the far updates.  Each task waits (bounded) for
+// per step j the copy of U_jj, the rest of panel j, block column j-1, the far updates, then
+// row j of U and the S contributions of panel j.  Each task waits (bounded) for
 // the counters of the tasks it reads from, all of which come earlier in that order; so the
 // lowest unfinished task can always run, whatever subset of CTAs is resident.  Within a CTA
 // the task fetch and TMA loads (warp 0), the MMAs (warp 1) and the epilogue (warps 2-5) are
@@ -76,15 +76,16 @@ __host__ __device__ inline DagTask dag_step_task(int T, int j, long long idx) {
         idx -= j - 1;
         if (idx < j - 1) return DagTask{DT_UPDATE, j - 2 - (int)idx, j - 1, j, 0};
         idx -= j - 1;
+        // the far updates, nearest block column first: the next leaves wait for them, so they
+        // come before this step's inverse tasks
+        for (int k = j - 2; k >= 0; --k) {
+            if (idx < k + 1) return DagTask{DT_UPDATE, (int)idx, k, j, 0};
+            idx -= k + 1;
+        }
     }
     if (idx < T - 1 - j) return DagTask{DT_FIN, j, j + 1 + (int)idx, 0, 0};
     idx -= T - 1 - j;
     if (idx < (long long)j * (T - j)) return DagTask{DT_SUPD, (int)(idx % j), j + (int)(idx / j), j, 0};
-    idx -= (long long)j * (T - j);
-    for (int k = j - 2; k >= 0; --k) {   // far updates, nearest block column first
-        if (idx < k + 1) return DagTask{DT_UPDATE, (int)idx, k, j, 0};
-        idx -= k + 1;
-    }
     return DagTask{DT_STOP, 0, 0, 0, 0};
 }
 

@@ -19,7 +19,7 @@
 
 namespace gq {
 
-constexpr int G2_THREADS = 256;
+constexpr int G2_THREADS = 1024;
 constexpr long long G2_SMEM_T_MAX = 160 * 1024;   // bytes of T kept in shared memory
 
 // ULT[i][r] = U_left[r][i]
