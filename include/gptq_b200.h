@@ -254,6 +254,28 @@ gptq_status gptq_dequant_gemm(const void* X, int64_t M, const int32_t* qweight, 
                               const int32_t* qzeros, int64_t d_out, int64_t d_in, const gptq_config* cfg, float* Y,
                               void* stream);
 
+/* ------------------------------------------------------------------ layer output error
+ * E = ||(W - W_hat) X^T||_F^2 (tutorial "阶段一": the squared error of the layer's outputs
+ * over the calibration tokens, which GPTQ minimises), and its per-row parts
+ * E_o = sum_t ((W - W_hat) X^T)[o, t]^2.
+ *   W        device fp32 [d_out, d_in] row-major: the weights before quantization (the
+ *            natural-order gptq_quantize_layer overwrites its W, so pass a copy).
+ *   W_hat    device fp32 [d_out, d_in] row-major, e.g. from gptq_dequant.
+ *   X        device [n, d_in] row-major, bf16 (raw uint16 bit patterns) or fp32.
+ *   row_loss device fp64 [d_out] or NULL; receives E_o.
+ *   loss     device fp64 [1]; receives E.
+ *   ws       device workspace of at least gptq_layer_loss_workspace_bytes(d_out, d_in, n).
+ * W - W_hat and X are split into bf16 pairs (16 significant bits; a bf16 X is exact), the
+ * product runs on the tensor cores as three bf16 products with fp32 accumulation in
+ * segments, and the squares are summed in fp64 in a fixed order (same bits every run).
+ * Relative error of E is about 1e-5 (the split and the fp32 accumulation).
+ * Requires 1 <= d_out, n <= 2^30, d_in % 8 == 0 with 8 <= d_in <= 65536, all pointers
+ * 16-byte aligned (row_loss and loss 8-byte). Nothing is allocated. */
+size_t gptq_layer_loss_workspace_bytes(int64_t d_out, int64_t d_in, int64_t n);
+gptq_status gptq_layer_loss(const float* W, const float* W_hat, const void* X, gptq_dtype xt, int64_t d_out,
+                            int64_t d_in, int64_t n, double* row_loss, double* loss, void* ws, size_t ws_bytes,
+                            void* stream);
+
 /* ------------------------------------------------------------------ two-sided rounding
  * GPTQ-2D (GPTQ-2D summary, "方法" steps 1-3 and "核心洞察"): round a real matrix X
  * (m x n) to an integer matrix Z minimising tr((X - Z)^T G_left (X - Z) G_right), given the

@@ -12,6 +12,7 @@ from .gptq import (  # noqa: F401
     QuantizedLayer,
     gptq_dequant,
     gptq_hessian_accumulate,
+    gptq_layer_loss,
     gptq_pack_int,
     gptq_prepare_hinv,
     gptq_quantize_layer,

@@ -20,6 +20,7 @@
 #include "colloop_host.cuh"
 #include "dqgemm.cuh"
 #include "gptq2d.cuh"
+#include "loss.cuh"
 
 namespace gqh {
 
@@ -622,6 +623,29 @@ gptq_status gptq_dequant_gemm(const void* X, int64_t M, const int32_t* qweight, 
         default: e = dq_gemm_run<8>(X, M, qweight, sc, qzeros, d_out, d_in, g, Y, st); break;
     }
     if (e != cudaSuccess) return cuda_fail(e, "dequant_gemm");
+    return GPTQ_OK;
+}
+
+size_t gptq_layer_loss_workspace_bytes(int64_t d_out, int64_t d_in, int64_t n) {
+    if (d_out < 1 || n < 1 || d_in < 8 || d_out > (1ll << 30) || n > (1ll << 30) || d_in > 65536) return 0;
+    return loss_ws_bytes(d_out, d_in, n);
+}
+
+gptq_status gptq_layer_loss(const float* W, const float* W_hat, const void* X, gptq_dtype xt, int64_t d_out,
+                            int64_t d_in, int64_t n, double* row_loss, double* loss, void* ws, size_t ws_bytes,
+                            void* stream) {
+    if (!W || !W_hat || !X || !loss) return fail(GPTQ_ERR_INVALID_ARG, "W, W_hat, X and loss must be non-NULL");
+    if (xt != GPTQ_BF16 && xt != GPTQ_F32) return fail(GPTQ_ERR_INVALID_ARG, "unknown X dtype %d", (int)xt);
+    if (d_out < 1 || d_out > (1ll << 30)) return fail(GPTQ_ERR_INVALID_ARG, "d_out out of range (%lld)", (long long)d_out);
+    if (n < 1 || n > (1ll << 30)) return fail(GPTQ_ERR_INVALID_ARG, "n out of range (%lld)", (long long)n);
+    if (d_in < 8 || d_in > 65536 || d_in % 8) return fail(GPTQ_ERR_INVALID_ARG, "d_in must be a multiple of 8 in [8, 65536]");
+    if (!aligned16(W) || !aligned16(W_hat) || !aligned16(X) || !aligned16(ws) ||
+        (reinterpret_cast<uintptr_t>(loss) & 7) || (reinterpret_cast<uintptr_t>(row_loss) & 7))
+        return fail(GPTQ_ERR_INVALID_ARG, "W, W_hat, X and ws must be 16-byte aligned, row_loss and loss 8-byte");
+    if (!ws || ws_bytes < loss_ws_bytes(d_out, d_in, n))
+        return fail(GPTQ_ERR_WORKSPACE, "workspace needs %zu bytes", loss_ws_bytes(d_out, d_in, n));
+    cudaError_t e = loss_run(W, W_hat, X, xt == GPTQ_BF16, d_out, d_in, n, row_loss, loss, ws, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "layer_loss");
     return GPTQ_OK;
 }
 

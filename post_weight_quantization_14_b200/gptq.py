@@ -79,6 +79,8 @@ _SIGS = {
                                              _vp, _vp, _vp, _sz, _vp]),
     "gptq_dequant_g_idx": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, ctypes.POINTER(GptqConfig), _vp, _vp]),
     "gptq_dequant_gemm": (_int, [_vp, _i64, _vp, _vp, _vp, _i64, _i64, ctypes.POINTER(GptqConfig), _vp, _vp]),
+    "gptq_layer_loss_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "gptq_layer_loss": (_int, [_vp, _vp, _vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _sz, _vp]),
     "gptq_2d_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "gptq_2d_round": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _sz, _vp]),
 }
@@ -340,6 +342,30 @@ def gptq_dequant_gemm(X: torch.Tensor, qweight, scales, qzeros, d_out: int, d_in
     _check(lib().gptq_dequant_gemm(_ptr(X), X.shape[0], _ptr(qweight), _ptr(scales), _ptr(qzeros), d_out, d_in,
                                    ctypes.byref(cfg), _ptr(Y), _stream(stream)))
     return Y
+
+
+def gptq_layer_loss(W: torch.Tensor, W_hat: torch.Tensor, X: torch.Tensor, row_loss: torch.Tensor | None = None,
+                    workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """E = ||(W - W_hat) X^T||_F^2 on the device: a float64 [1] tensor (not synchronised).
+    W, W_hat: float32 [d_out, d_in]; X: bfloat16 or float32 [n, d_in]; row_loss, when given,
+    float64 [d_out] receives each row's part."""
+    if W.dim() != 2 or X.dim() != 2 or W.shape[1] != X.shape[1]:
+        raise ValueError("W must be [d_out, d_in] and X [n, d_in]")
+    d_out, d_in = W.shape
+    if W.dtype != torch.float32 or W_hat.dtype != torch.float32 or tuple(W_hat.shape) != (d_out, d_in):
+        raise ValueError("W and W_hat must be float32 [d_out, d_in]")
+    xt = GPTQ_BF16 if X.dtype == torch.bfloat16 else GPTQ_F32 if X.dtype == torch.float32 else None
+    if xt is None:
+        raise ValueError("X must be bfloat16 or float32")
+    if row_loss is not None and (row_loss.dtype != torch.float64 or tuple(row_loss.shape) != (d_out,)):
+        raise ValueError("row_loss must be float64 [d_out]")
+    n = X.shape[0]
+    need = lib().gptq_layer_loss_workspace_bytes(d_out, d_in, n)
+    ws = workspace if workspace is not None else _workspace(need, W.device)
+    loss = torch.empty((1,), dtype=torch.float64, device=W.device)
+    _check(lib().gptq_layer_loss(_ptr(W), _ptr(W_hat), _ptr(X), xt, d_out, d_in, n, _ptr(row_loss), _ptr(loss),
+                                 _ptr(ws), ws.numel(), _stream(stream)))
+    return loss
 
 
 def gptq_2d_round(X: torch.Tensor, U_left: torch.Tensor, U_right: torch.Tensor, Z: torch.Tensor | None = None,
