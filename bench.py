@@ -208,7 +208,7 @@ def rank_probe(world: int, rank: int) -> None:
 
 # ---------------------------------------------------------------- GPU leg
 
-CHOL_KERNELS = ("chol_dag", "damp_copy", "diag_mean", "zero_lower", "perm_invert", "damp_copy_perm")
+CHOL_KERNELS = ("chol_dag", "damp_copy", "diag_mean", "perm_invert", "damp_copy_perm")
 QUANT_KERNELS = ("colloop", "trailing_update", "trailing_update_sb", "up_prep", "ut_split", "pack_zeros", "row_params",
                  "gather_cols", "unpermute_codes")
 ACT_KERNELS = ("act_sum", "act_rank", "act_perm")   # activation ordering (--desc-act 1 or 2)

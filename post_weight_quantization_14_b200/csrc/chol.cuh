@@ -51,10 +51,20 @@ __global__ void diag_mean_kernel(const float* __restrict__ H, long long d, float
 // not written.
 __global__ void __launch_bounds__(256) damp_copy_kernel(const float* __restrict__ H, long long d, long long n,
                                                         const float* __restrict__ lam, float* __restrict__ A,
-                                                        float* __restrict__ RS_hi, float* __restrict__ RS_lo) {
+                                                        float* __restrict__ RS_hi, float* __restrict__ RS_lo,
+                                                        float* __restrict__ U, int* __restrict__ ctr, int nctr) {
     const int bi = blockIdx.y, bj = blockIdx.x;
-    if (bi > bj) return;
     const long long r0 = (long long)bi * NB, c0 = (long long)bj * NB;
+    if (bi > bj) {   // the public U's strictly lower blocks are zero (d % 4 == 0)
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
+            const long long i = r0 + (e >> 5), j = c0 + (e & 31) * 4;
+            if (i < d && j < d) *reinterpret_cast<float4*>(U + i * d + j) = z;
+        }
+        return;
+    }
+    if (bi == 0 && bj == 0)   // the factorization's dependency counters start at zero
+        for (int e = threadIdx.x; e < nctr; e += blockDim.x) ctr[e] = 0;
     const float l = lam[0];
     if (bi < bj) {
         const bool last = c0 + NB == n;   // the first panel: also its tf32 split
@@ -115,9 +125,14 @@ __global__ void __launch_bounds__(256) damp_copy_kernel(const float* __restrict_
 __global__ void __launch_bounds__(256) damp_copy_perm_kernel(const float* __restrict__ H,
                                                              const int* __restrict__ perm, long long d, long long n,
                                                              const float* __restrict__ lam, float* __restrict__ A,
-                                                             float* __restrict__ RS_hi, float* __restrict__ RS_lo) {
+                                                             float* __restrict__ RS_hi, float* __restrict__ RS_lo,
+                                                             float* __restrict__ U, int* __restrict__ ctr, int nctr) {
     const long long i = blockIdx.x;
     const long long j0 = (i / NB) * NB;
+    if (i == 0)   // the factorization's dependency counters start at zero
+        for (int e = threadIdx.x; e < nctr; e += blockDim.x) ctr[e] = 0;
+    if (i < d)    // the public U's strictly lower blocks: row i left of its block
+        for (long long j = threadIdx.x; j < j0; j += blockDim.x) U[i * d + j] = 0.f;
     const long long jl = n - NB;   // the first panel (block column T-1, rows above its block): also split
     float* out = A + i * n;
     if (i >= d) {
@@ -147,19 +162,6 @@ __global__ void __launch_bounds__(256) damp_copy_perm_kernel(const float* __rest
             RS_hi[i * n + j] = h;
             RS_lo[i * n + j] = q;
         }
-    }
-}
-
-// Zero the strictly-lower 128-blocks of the d x d output U (the diagonal and upper
-// blocks are written by the factorization).
-__global__ void __launch_bounds__(256) zero_lower_blocks_kernel(float* __restrict__ U, long long d) {
-    const int bi = blockIdx.y, bj = blockIdx.x;   // one CTA per 128-block, strictly lower only
-    if (bi <= bj) return;
-    const long long r0 = (long long)bi * NB, c0 = (long long)bj * NB;
-    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
-        const long long i = r0 + (e >> 5), j = c0 + (e & 31) * 4;
-        if (i < d && j < d) *reinterpret_cast<float4*>(U + i * d + j) = z;   // d % 4 == 0
     }
 }
 
@@ -202,7 +204,9 @@ __device__ __forceinline__ void leaf_sync() { nbar_sync(5, LEAF_THREADS); }
 
 // F: factor the 32x32 diagonal block at (k0, k0); lane i holds row k0 + i.  Per pivot k the
 // dependency chain is: the pivot (one shuffle of the diagonal entry that lane k keeps current
-// from its own multipliers), 1/sqrt (rsqrt and one Newton step), the multipliers, and the
+// from its own multipliers), 1/sqrt (the hardware reciprocal square root, no refinement: its
+// few-ulp error scales the pivot's column by 1 + O(2^-22), a backward error far below the
+// fp32 rounding the factorization accumulates anyway), the multipliers, and the
 // next column's update with one more shuffle (L_{k+1,k}); the columns past it take the
 // multipliers through shared memory, one pivot behind, off that chain.
 // Writes L_kk (lower, zeros above) to P and LT, and 1/L_kk to rinv.
@@ -228,8 +232,7 @@ __device__ __forceinline__ void leaf_diag_factor(LeafSmem& S, int k0, int lane, 
         const bool pk = p > 0.f && isfinite(p);
         bad_p = (bad < 0 && !pk) ? p : bad_p;
         bad = (bad < 0 && !pk) ? k : bad;
-        float r = rsqrtf(p);
-        r = r * fmaf(-0.5f * p * r, r, 1.5f);       // one Newton step for 1/sqrt(p)
+        const float r = rsqrtf(p);   // hardware 1/sqrt (a few ulp): scales column k by 1 + O(2^-22)
         float l = (lane == k) ? p * r : a[k] * r;   // L_kk = sqrt(p); L_ik = P_ik / L_kk
         if (lane < k) l = 0.f;                      // rows above: finished, untouched
         a[k] = (lane >= k) ? l : a[k];

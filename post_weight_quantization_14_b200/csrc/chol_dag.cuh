@@ -1140,23 +1140,19 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
         GQ_TRY(cudaGetLastError());
         {
             gqh::TimedScope ts__("damp_copy_perm", st);
-            gq::damp_copy_perm_kernel<<<(unsigned)n, 256, 0, st>>>(H, perm, d, n, w.scal, w.A, w.RS_hi, w.RS_lo);
+            gq::damp_copy_perm_kernel<<<(unsigned)n, 256, 0, st>>>(H, perm, d, n, w.scal, w.A, w.RS_hi, w.RS_lo, U,
+                                                                   w.ctr, (int)gq::dag_ctr_ints((int)T));
         }
         GQ_TRY(cudaGetLastError());
     } else {
         const dim3 grid((unsigned)T, (unsigned)T);
         {
             gqh::TimedScope ts__("damp_copy", st);
-            gq::damp_copy_kernel<<<grid, 256, 0, st>>>(H, d, n, w.scal, w.A, w.RS_hi, w.RS_lo);
+            gq::damp_copy_kernel<<<grid, 256, 0, st>>>(H, d, n, w.scal, w.A, w.RS_hi, w.RS_lo, U, w.ctr,
+                                                        (int)gq::dag_ctr_ints((int)T));
         }
         GQ_TRY(cudaGetLastError());
     }
-    {
-        gqh::TimedScope ts__("zero_lower", st);   // the public U's strictly lower blocks
-        gq::zero_lower_blocks_kernel<<<dim3((unsigned)T, (unsigned)T), 256, 0, st>>>(U, d);
-    }
-    GQ_TRY(cudaGetLastError());
-    GQ_TRY(cudaMemsetAsync(w.ctr, 0, (size_t)gq::dag_ctr_ints(T) * sizeof(int), st));
     const uint64_t N = (uint64_t)n;
     gq::DagMaps m;
     if (!make_tmap_2d(&m.rs_hi, w.RS_hi, 4, N, N, N, gq::BM, 32) || !make_tmap_2d(&m.rs_lo, w.RS_lo, 4, N, N, N, gq::BM, 32) ||

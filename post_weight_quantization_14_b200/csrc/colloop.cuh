@@ -15,7 +15,8 @@
 // after the oct each lane applies the 8 errors d_c to its later slots in column order,
 // which is e_c = d_c / U_cc pushed forward with row c of U.  The normalised rows of
 // the block's 128x128 diagonal part of U are prepared once per layer and staged into
-// shared memory by one bulk (TMA) copy per CTA.
+// shared memory by four bulk (TMA) copies per CTA, one per phase, each waited for just
+// before its phase.
 // At a group's first column the scale and zero come from the current values of the
 // group's columns (min/max by an 8-lane shuffle reduction).
 // At the end of the block the kernel writes the packed codes (qweight layout), the
@@ -65,7 +66,7 @@ struct ColSmem {
     float dv[CL_ROWS][DV_LD];
     float invd[CB];
     uint8_t codes[CL_ROWS][CODE_LD];
-    uint64_t bar;
+    uint64_t bar[4];   // one per quarter of the staged rows (the 32 columns of one phase)
 };
 
 // Scale and zero of a group with grid range [lo, hi] (lo <= 0 <= hi, or -m..m).
@@ -193,20 +194,21 @@ __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p)
     const bool row_ok = row < p.d_out;
 
     if (tid == 0) {
-        mbar_init(&S.bar, 1);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mbar_init(&S.bar[i], 1);
         fence_mbar_init();
     }
     __syncthreads();
     pdl_wait();
     pdl_trigger();
-    if (tid == 0) {
-        constexpr uint32_t bytes = UP_BLOCK * 4;
-        constexpr uint32_t chunk = bytes / 4;
-        mbar_arrive_expect_tx(&S.bar, bytes);
+    if (tid == 0) {   // rows 32i .. 32i+31 (phase i's octs) complete barrier i
+        constexpr uint32_t chunk = UP_BLOCK * 4 / 4;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 4; ++i) {
+            mbar_arrive_expect_tx(&S.bar[i], chunk);
             bulk_g2s(reinterpret_cast<uint8_t*>(S.up) + i * chunk,
-                     reinterpret_cast<const uint8_t*>(p.Up) + i * chunk, chunk, &S.bar);
+                     reinterpret_cast<const uint8_t*>(p.Up) + i * chunk, chunk, &S.bar[i]);
+        }
     }
     for (int c = tid; c < CB; c += blockDim.x) S.invd[c] = (c < p.nc) ? p.inv_d[p.c0 + c] : 0.f;
 
@@ -233,28 +235,37 @@ __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p)
         qlo = -z;
         qhi = (float)MAXQ - z;
     }
-    const bool ok = mbar_wait(&S.bar, 0, -1 - (long long)blockIdx.x);
+    const bool ok = mbar_wait(&S.bar[0], 0, -1 - (long long)blockIdx.x);
     __syncthreads();
     if (!ok) return;
+    // the later quarters are waited for just before their phase (each warp decides as one,
+    // so a warp never splits across a shuffle)
+    auto staged = [&](int i) { return __all_sync(FULL, mbar_wait(&S.bar[i], 0, -1 - (long long)blockIdx.x)); };
 
     QuadState st{s, inv_s, qlo, qhi};
     run_octs<BITS, 16>(wv, 0, 4, st, p, S, lane, k, rloc, row, row_ok);
+    if (!staged(1)) return;
     run_octs<BITS, 12>(wv, 4, 8, st, p, S, lane, k, rloc, row, row_ok);
+    if (!staged(2)) return;
     run_octs<BITS, 8>(wv, 8, 12, st, p, S, lane, k, rloc, row, row_ok);
+    if (!staged(3)) return;
     run_octs<BITS, 4>(wv, 12, 16, st, p, S, lane, k, rloc, row, row_ok);
     __syncwarp();
 
-    // errors of the block (operand of the trailing update) and per-row sum of e^2
+    // errors of the block (operand of the trailing update) and per-row sum of e^2; the
+    // warp's rows are independent, so their loads, stores and reductions interleave
     const long long wrow0 = (long long)blockIdx.x * CL_ROWS + warp * RPW;
+    float acc[RPW];
+#pragma unroll
     for (int rr = 0; rr < RPW; ++rr) {
         const long long rw = wrow0 + rr;
         const int rl = warp * RPW + rr;
-        float acc = 0.f;
+        acc[rr] = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const int col = lane + 32 * q;
             const float e = S.dv[rl][col] * S.invd[col];
-            acc = fmaf(e, e, acc);
+            acc[rr] = fmaf(e, e, acc[rr]);
             if (rw < p.d_out) {
                 uint16_t h, l;
                 split_bf16(e, h, l);
@@ -262,10 +273,18 @@ __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p)
                 p.E_lo[rw * p.e_ld + col] = l;
             }
         }
+    }
 #pragma unroll
-        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
-        if (lane == 0 && rw < p.d_out && p.err_sq)
-            p.err_sq[rw] = (p.first_block ? 0.f : p.err_sq[rw]) + acc;
+    for (int o = 16; o; o >>= 1) {
+#pragma unroll
+        for (int rr = 0; rr < RPW; ++rr) acc[rr] += __shfl_xor_sync(FULL, acc[rr], o);
+    }
+    if (lane < RPW && p.err_sq) {
+        float mine = acc[0];
+#pragma unroll
+        for (int rr = 1; rr < RPW; ++rr) mine = (lane == rr) ? acc[rr] : mine;
+        const long long rw = wrow0 + lane;
+        if (rw < p.d_out) p.err_sq[rw] = (p.first_block ? 0.f : p.err_sq[rw]) + mine;
     }
 
     // packed codes: word w of this block's stream for each of the warp's 8 rows
