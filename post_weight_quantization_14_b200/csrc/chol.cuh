@@ -30,7 +30,19 @@ __global__ void diag_mean_kernel(const float* __restrict__ H, long long d, float
                                  float* __restrict__ lam_out) {
     __shared__ double part[32];
     double s = 0.0;
-    for (long long i = threadIdx.x; i < d; i += blockDim.x) s += (double)H[i * d + i];
+    // each thread adds its entries i = tid, tid + blockDim, ... in that order; eight loads in
+    // flight per step
+    for (long long i0 = threadIdx.x; i0 < d; i0 += 8LL * blockDim.x) {
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const long long i = i0 + (long long)q * blockDim.x;
+            v[q] = i < d ? H[i * d + i] : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (i0 + (long long)q * blockDim.x < d) s += (double)v[q];
+    }
     for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
     __syncthreads();
@@ -53,7 +65,19 @@ __global__ void __launch_bounds__(256) damp_copy_kernel(const float* __restrict_
                                                         const float* __restrict__ lam, float* __restrict__ A,
                                                         float* __restrict__ RS_hi, float* __restrict__ RS_lo,
                                                         float* __restrict__ U, int* __restrict__ ctr, int nctr) {
-    const int bi = blockIdx.y, bj = blockIdx.x;
+    // a 1-D grid of T*T CTAs, the T diagonal blocks first: their sub-tile passes are the
+    // longest, so they start before the copies and the zeroing rather than trail them
+    const int T = (int)(n / NB);
+    const int b = blockIdx.x;
+    int bi, bj;
+    if (b < T) {
+        bi = bj = b;
+    } else {
+        const int o = b - T;
+        bi = o / (T - 1);
+        bj = o % (T - 1);
+        if (bj >= bi) ++bj;
+    }
     const long long r0 = (long long)bi * NB, c0 = (long long)bj * NB;
     if (bi > bj) {   // the public U's strictly lower blocks are zero (d % 4 == 0)
         const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -68,54 +92,65 @@ __global__ void __launch_bounds__(256) damp_copy_kernel(const float* __restrict_
     const float l = lam[0];
     if (bi < bj) {
         const bool last = c0 + NB == n;   // the first panel: also its tf32 split
-        for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
-            const int r = e >> 5, c = (e & 31) * 4;
-            const long long i = r0 + r, j = c0 + c;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (i < d && j < d) {   // d % 4 == 0: a float4 is wholly inside or outside
-                v = *reinterpret_cast<const float4*>(H + i * d + j);
-                if (!(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w)))
-                    record_status(GPTQ_ERR_NONFINITE, i * d + j);
-            }
-            *reinterpret_cast<float4*>(A + i * n + j) = v;
+        constexpr int PER = NB * NB / 4 / 256;   // float4s per thread, all loads issued first
+        float4 v[PER];
+        long long bad = -1;
+#pragma unroll
+        for (int q = 0; q < PER; ++q) {
+            const int e = threadIdx.x + 256 * q;
+            const long long i = r0 + (e >> 5), j = c0 + (e & 31) * 4;
+            v[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < d && j < d) v[q] = *reinterpret_cast<const float4*>(H + i * d + j);   // d % 4 == 0
+        }
+#pragma unroll
+        for (int q = 0; q < PER; ++q) {
+            const int e = threadIdx.x + 256 * q;
+            const long long i = r0 + (e >> 5), j = c0 + (e & 31) * 4;
+            if (bad < 0 && !(isfinite(v[q].x) && isfinite(v[q].y) && isfinite(v[q].z) && isfinite(v[q].w)))
+                bad = i * d + j;
+            *reinterpret_cast<float4*>(A + i * n + j) = v[q];
             if (last) {
-                float4 h, q;
-                split_tf32(v.x, h.x, q.x);
-                split_tf32(v.y, h.y, q.y);
-                split_tf32(v.z, h.z, q.z);
-                split_tf32(v.w, h.w, q.w);
+                float4 h, lo;
+                split_tf32(v[q].x, h.x, lo.x);
+                split_tf32(v[q].y, h.y, lo.y);
+                split_tf32(v[q].z, h.z, lo.z);
+                split_tf32(v[q].w, h.w, lo.w);
                 *reinterpret_cast<float4*>(RS_hi + i * n + j) = h;
-                *reinterpret_cast<float4*>(RS_lo + i * n + j) = q;
+                *reinterpret_cast<float4*>(RS_lo + i * n + j) = lo;
             }
         }
+        if (bad >= 0) record_status(GPTQ_ERR_NONFINITE, bad);
         return;
     }
     // diagonal block: A[i][j] = H[min(i,j)][max(i,j)], by 32x32 sub-tiles of the upper
-    // triangle read row by row and written both ways through shared memory
+    // triangle read row by row and written both ways through shared memory (a small tile:
+    // the static shared memory of the one kernel bounds the residency of every CTA)
     __shared__ float tile[32][33];
-    for (int bi = 0; bi < 4; ++bi)
-        for (int bj = bi; bj < 4; ++bj) {
+    long long bad = -1;
+    for (int sbi = 0; sbi < 4; ++sbi)
+        for (int sbj = sbi; sbj < 4; ++sbj) {
             __syncthreads();   // the previous sub-tile's readers are done
             for (int t = threadIdx.x; t < 32 * 32; t += blockDim.x) {
                 const int rr = t >> 5, cc = t & 31;
-                const long long i = r0 + 32 * bi + rr, j = c0 + 32 * bj + cc;
+                const long long i = r0 + 32 * sbi + rr, j = c0 + 32 * sbj + cc;
                 float v = 0.f;
-                if (i < d && j < d && (bi < bj || rr <= cc)) {
+                if (i < d && j < d && (sbi < sbj || rr <= cc)) {
                     v = H[i * d + j];
-                    if (!isfinite(v)) record_status(GPTQ_ERR_NONFINITE, i * d + j);
+                    if (bad < 0 && !isfinite(v)) bad = i * d + j;
                 }
                 tile[rr][cc] = v;
             }
             __syncthreads();
             for (int t = threadIdx.x; t < 32 * 32; t += blockDim.x) {
                 const int rr = t >> 5, cc = t & 31;
-                const long long i = r0 + 32 * bi + rr, j = c0 + 32 * bj + cc;
-                float v = (bi < bj || rr <= cc) ? tile[rr][cc] : tile[cc][rr];
+                const long long i = r0 + 32 * sbi + rr, j = c0 + 32 * sbj + cc;
+                float v = (sbi < sbj || rr <= cc) ? tile[rr][cc] : tile[cc][rr];
                 if (i == j) v = (i < d) ? v + l : 1.f;
                 A[i * n + j] = v;
-                if (bi < bj) A[(r0 + 32 * bj + rr) * n + c0 + 32 * bi + cc] = tile[cc][rr];
+                if (sbi < sbj) A[(r0 + 32 * sbj + rr) * n + c0 + 32 * sbi + cc] = tile[cc][rr];
             }
         }
+    if (bad >= 0) record_status(GPTQ_ERR_NONFINITE, bad);
 }
 
 // The damped copy of damp_copy_kernel for the permuted Hessian: A[i][j] =

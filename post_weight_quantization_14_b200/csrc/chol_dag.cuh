@@ -1145,10 +1145,9 @@ inline cudaError_t hinv_run(const float* H, long long d, float damp_rel, float* 
         }
         GQ_TRY(cudaGetLastError());
     } else {
-        const dim3 grid((unsigned)T, (unsigned)T);
         {
             gqh::TimedScope ts__("damp_copy", st);
-            gq::damp_copy_kernel<<<grid, 256, 0, st>>>(H, d, n, w.scal, w.A, w.RS_hi, w.RS_lo, U, w.ctr,
+            gq::damp_copy_kernel<<<(unsigned)(T * T), 256, 0, st>>>(H, d, n, w.scal, w.A, w.RS_hi, w.RS_lo, U, w.ctr,
                                                         (int)gq::dag_ctr_ints((int)T));
         }
         GQ_TRY(cudaGetLastError());

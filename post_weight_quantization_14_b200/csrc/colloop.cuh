@@ -36,8 +36,9 @@ constexpr int RPW = 32 / LPR;            // rows per warp
 constexpr int CL_WARPS = 4;
 constexpr int CL_ROWS = CL_WARPS * RPW;  // rows per CTA
 constexpr int UP_LD = 20;                // padded slot stride of one lane's row segment (16 used)
-constexpr int UP_ROW = LPR * UP_LD;      // floats per normalised U row
-constexpr int UP_BLOCK = CB * UP_ROW;    // floats per block (81920 bytes)
+constexpr int UP_OCT = LPR * UP_LD;      // offset of a row's eight in-oct entries
+constexpr int UP_ROW = UP_OCT + 8;       // floats per normalised U row
+constexpr int UP_BLOCK = CB * UP_ROW;    // floats per block (86016 bytes)
 constexpr int CODE_LD = 132;
 constexpr int DV_LD = 129;
 constexpr float kF16MinPos = 5.9604644775390625e-08f;  // 2^-24, smallest positive fp16
@@ -156,9 +157,12 @@ __device__ __forceinline__ void run_octs(float (&wv)[SLOTS], int t0, int t1, Qua
             dd[j] = d;
             my_r = (k == j) ? r : my_r;
             my_d = (k == j) ? d : my_d;
-            const float* urow = S.up + (c8 + j) * UP_ROW;   // slot 0 of lane m at offset m * UP_LD
+            const float* urow = S.up + (c8 + j) * UP_ROW + UP_OCT;   // U[c8+j][c8+m] / U[c8+j][c8+j]
+            const float4 ua = *reinterpret_cast<const float4*>(urow);
+            const float4 ub = *reinterpret_cast<const float4*>(urow + 4);
+            const float uo[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
 #pragma unroll
-            for (int m = j + 1; m < LPR; ++m) v[m] = fmaf(-d, urow[m * UP_LD], v[m]);
+            for (int m = j + 1; m < LPR; ++m) v[m] = fmaf(-d, uo[m], v[m]);
         }
         // the errors applied to this lane's later slots, in column order
 #pragma unroll
@@ -306,7 +310,8 @@ __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p)
 
 // Normalised, lane-permuted, oct-shifted rows of each 128x128 diagonal block of U:
 // Up[b][c][k*UP_LD + i] = U[c0+c, c0+j] / U[c0+c, c0+c] with j = k + 8*(c/8 + i) for j > c
-// (0 otherwise), and inv_d[c] = 1 / U[c, c].
+// (0 otherwise), followed by the row's in-oct entries Up[b][c][UP_OCT + m] (the same value
+// for j = 8*(c/8) + m), and inv_d[c] = 1 / U[c, c].
 __global__ void up_prep_kernel(const float* __restrict__ U, long long d, float* __restrict__ Up,
                                float* __restrict__ inv_d) {
     const int b = blockIdx.y, c = blockIdx.x;
@@ -316,32 +321,57 @@ __global__ void up_prep_kernel(const float* __restrict__ U, long long d, float* 
     float* dst = Up + ((long long)b * CB + c) * UP_ROW;
     for (int e = threadIdx.x; e < UP_ROW; e += blockDim.x) {
         const int kk = e / UP_LD, i = e % UP_LD;
-        const int j = kk + LPR * ((c / LPR) + i);
+        const bool oct = e >= UP_OCT;
+        const int j = oct ? LPR * (c / LPR) + (e - UP_OCT) : kk + LPR * ((c / LPR) + i);
         float v = 0.f;
-        if (i < SLOTS && c < nc && j < nc && j > c) v = __fdiv_rn(U[(c0 + c) * d + c0 + j], ucc);
+        if ((oct || i < SLOTS) && c < nc && j < nc && j > c) v = __fdiv_rn(U[(c0 + c) * d + c0 + j], ucc);
         dst[e] = v;
     }
     if (threadIdx.x == 0 && c < nc) inv_d[c0 + c] = __frcp_rn(ucc);
 }
 
-// UT[j, i] = bf16 split of U[i, j] for the 32x32 tiles on or above the diagonal of U.
-__global__ void ut_split_kernel(const float* __restrict__ U, long long d, uint16_t* __restrict__ UT_hi,
-                                uint16_t* __restrict__ UT_lo) {
-    __shared__ float tile[32][33];
+// UT[j, i] = bf16 split of U[i, j] for the 64x64 tiles on or above the diagonal of U.
+// 256 threads per tile: four float4 loads each (all issued first) into a padded tile, then
+// 16-byte stores of eight consecutive bf16 values of a UT row per array.  d % 8 == 0.
+constexpr int UTS = 64;
+__global__ void __launch_bounds__(256) ut_split_kernel(const float* __restrict__ U, long long d,
+                                                       uint16_t* __restrict__ UT_hi, uint16_t* __restrict__ UT_lo) {
+    __shared__ float tile[UTS][UTS + 1];
     const long long bi = blockIdx.y, bj = blockIdx.x;  // tile of U
     if (bi > bj) return;
-    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
-        const long long i = bi * 32 + r, j = bj * 32 + threadIdx.x;
-        tile[r][threadIdx.x] = (i < d && j < d) ? U[i * d + j] : 0.f;
+    float4 v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int e = threadIdx.x + 256 * q, r = e >> 4, c = (e & 15) * 4;
+        const long long i = bi * UTS + r, j = bj * UTS + c;
+        v[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < d && j < d) v[q] = *reinterpret_cast<const float4*>(U + i * d + j);   // d % 4 == 0
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int e = threadIdx.x + 256 * q, r = e >> 4, c = (e & 15) * 4;
+        tile[r][c] = v[q].x;
+        tile[r][c + 1] = v[q].y;
+        tile[r][c + 2] = v[q].z;
+        tile[r][c + 3] = v[q].w;
     }
     __syncthreads();
-    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
-        const long long j = bj * 32 + r, i = bi * 32 + threadIdx.x;
-        if (i < d && j < d) {
-            uint16_t h, l;
-            split_bf16(tile[threadIdx.x][r], h, l);
-            UT_hi[j * d + i] = h;
-            UT_lo[j * d + i] = l;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {   // UT row jr of the tile, UT columns ir0 .. ir0 + 7
+        const int e = threadIdx.x + 256 * q, jr = e >> 3, ir0 = (e & 7) * 8;
+        const long long j = bj * UTS + jr, i0 = bi * UTS + ir0;
+        if (j < d && i0 < d) {   // d % 8 == 0: the eight columns are wholly inside
+            uint32_t h[4], l[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                uint16_t h0, l0, h1, l1;
+                split_bf16(tile[ir0 + 2 * p][jr], h0, l0);
+                split_bf16(tile[ir0 + 2 * p + 1][jr], h1, l1);
+                h[p] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                l[p] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+            }
+            *reinterpret_cast<uint4*>(UT_hi + j * d + i0) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4*>(UT_lo + j * d + i0) = make_uint4(l[0], l[1], l[2], l[3]);
         }
     }
 }

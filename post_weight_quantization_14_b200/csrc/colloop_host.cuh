@@ -73,10 +73,10 @@ cudaError_t quant_run_bits(float* W, const float* U, long long d_out, long long 
             gq::up_prep_kernel<<<grid, 160, 0, st>>>(U, d_in, w.Up, w.inv_d);
         }
         GQ_TRY(cudaGetLastError());
-        dim3 tb(32, 8), g2((unsigned)((d_in + 31) / 32), (unsigned)((d_in + 31) / 32));
+        const unsigned nt = (unsigned)((d_in + gq::UTS - 1) / gq::UTS);
         {
             gqh::TimedScope ts__("ut_split", st);
-            gq::ut_split_kernel<<<g2, tb, 0, st>>>(U, d_in, w.UT_hi, w.UT_lo);
+            gq::ut_split_kernel<<<dim3(nt, nt), 256, 0, st>>>(U, d_in, w.UT_hi, w.UT_lo);
         }
         GQ_TRY(cudaGetLastError());
     }
