@@ -203,8 +203,10 @@ __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p)
         fence_mbar_init();
     }
     __syncthreads();
-    pdl_wait();
-    pdl_trigger();
+    // The staged U rows and 1/U_cc come from the layer's preparation kernels, which finished
+    // before the grid this one waits for began (every grid of the sequence lets its dependent
+    // start only after its own wait), so they are read before the wait: the copies overlap
+    // the tail of the preceding trailing update.  W, which that update writes, is read after.
     if (tid == 0) {   // rows 32i .. 32i+31 (phase i's octs) complete barrier i
         constexpr uint32_t chunk = UP_BLOCK * 4 / 4;
 #pragma unroll
@@ -215,6 +217,8 @@ __global__ void __launch_bounds__(CL_WARPS * 32) colloop_kernel(const ColArgs p)
         }
     }
     for (int c = tid; c < CB; c += blockDim.x) S.invd[c] = (c < p.nc) ? p.inv_d[p.c0 + c] : 0.f;
+    pdl_wait();
+    pdl_trigger();
 
     float wv[SLOTS];
     {
