@@ -106,6 +106,7 @@ cudaError_t quant_run_bits(float* W, const float* U, long long d_out, long long 
         p.beta = 1.f;
         p.c_col0 = (int)e;
         p.write_c = 1;
+        p.b_early = 1;   // U^T's split is made before the first column loop
         EpiMats o;
         o.c = Mat{W, (uint64_t)d_out, (uint64_t)d_in, (uint64_t)d_in};
         // few 128-wide tiles: 128x32 tiles spread the work over more SMs, within one wave.

@@ -59,6 +59,8 @@ struct GemmArgs {
     int c_row0, c_col0, c_zrow, c_zcol;
     int write_c;
     int mirror;       // also write C[j, i] for tiles above the diagonal
+    int b_early;      // B was written before the grid this launch waits for began: the first
+                      // tile's first stages load B before the wait (A after it)
 };
 
 constexpr int BM = 128;
@@ -292,17 +294,35 @@ __global__ void __launch_bounds__(gemm_threads<TBN>(), 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    pdl_wait();
-    pdl_trigger();
-
+    // b_early: the producer arms the first tile's first stages with their full byte count and
+    // loads their B parts before the wait; the A parts follow it, and a stage completes only
+    // when both have landed.  Every thread still signals its dependents after its own wait.
+    int nearly = 0;
     if (warp == 0 && lane == 0) {
-        // ---------------- TMA producer: one ring of stages across all tiles of this CTA
         prefetch_tmap(&mA);
         prefetch_tmap(&mB);
         if (NOPS == 2) {
             prefetch_tmap(&mA2);
             prefetch_tmap(&mB2);
         }
+        if (p.b_early && (int)blockIdx.x < total) {
+            const TileInfo ti = tile_info<KT, TBN>(p, blockIdx.x, tiles_per_batch);
+            const int bx = p.b_col0 + ti.z * p.b_zcol, by = p.b_row0 + ti.z * p.b_zrow + ti.n0;
+            nearly = min(STAGES, ti.nk);
+            for (int kt = 0; kt < nearly; ++kt) {   // fresh stages: nothing to wait for
+                uint8_t* st = smem + kt * STAGE_BYTES;
+                mbar_arrive_expect_tx(&full_bar[kt], STAGE_BYTES);
+                const int k = ti.kbeg + kt * KT;
+                tma_load_2d(st + NOPS * A_BYTES, &mB, &full_bar[kt], bx + k, by);
+                if (NOPS == 2) tma_load_2d(st + NOPS * A_BYTES + B_BYTES, &mB2, &full_bar[kt], bx + k, by);
+            }
+        }
+    }
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp == 0 && lane == 0) {
+        // ---------------- TMA producer: one ring of stages across all tiles of this CTA
         uint32_t kiter = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
@@ -312,13 +332,18 @@ __global__ void __launch_bounds__(gemm_threads<TBN>(), 1)
             for (int kt = 0; kt < ti.nk; ++kt, ++kiter) {
                 const int s = kiter % STAGES;
                 const uint32_t it = kiter / STAGES;
+                uint8_t* st = smem + s * STAGE_BYTES;
+                const int k = ti.kbeg + kt * KT;
+                if ((int)kiter < nearly) {   // armed and its B issued before the wait
+                    tma_load_2d(st, &mA, &full_bar[s], ax + k, ay);
+                    if (NOPS == 2) tma_load_2d(st + A_BYTES, &mA2, &full_bar[s], ax + k, ay);
+                    continue;
+                }
                 if (!mbar_wait(&empty_bar[s], (it & 1) ^ 1, w)) {
                     ok = false;
                     break;
                 }
-                uint8_t* st = smem + s * STAGE_BYTES;
                 mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
-                const int k = ti.kbeg + kt * KT;
                 tma_load_2d(st, &mA, &full_bar[s], ax + k, ay);
                 if (NOPS == 2) tma_load_2d(st + A_BYTES, &mA2, &full_bar[s], ax + k, ay);
                 tma_load_2d(st + NOPS * A_BYTES, &mB, &full_bar[s], bx + k, by);
