@@ -213,8 +213,9 @@ QUANT_KERNELS = ("colloop", "trailing_update", "trailing_update_sb", "up_prep", 
                  "gather_cols", "unpermute_codes")
 ACT_KERNELS = ("act_sum", "act_rank", "act_perm")   # activation ordering (--desc-act 1 or 2)
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu --set full capture of this
-# workload, for kernels whose launches all do the same work (the kernel's ncu summary under profiles/).
-TRAFFIC_PER_LAUNCH = {"colloop": 2249472, "hessian_syrk": 16856320 + 10733568}
+# workload, for kernels whose launches all do the same work and whose code has not changed since the capture
+# (the kernel's ncu summary under profiles/); the column loop and the generic GEMM changed after theirs.
+TRAFFIC_PER_LAUNCH = {"chol_dag": 39034112 + 311716096}
 # Sum of the stage bounds for this layer: Hessian 21.0 us (bf16), factor + invert 168.1 us and
 # trailing updates 244.3 us (3xTF32 at a third of bf16 x 1.1/2.25), column loop 11.6 us (HBM).
 # The trailing updates here run as bf16x3 products (a third of bf16, 122 us at that rate); the
